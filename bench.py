@@ -1,0 +1,541 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 SSD library: prefill tokens/s (fraction of the bf16 tensor peak)
+and cached decode steps/s (fraction of HBM bandwidth).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill_130m|prefill_2p7b_long|decode_2p7b] [--no-extras]
+
+One process per GPU (torchrun for N > 1).  Every rank runs its own independent
+problem (weak scaling, no collective on the data path); rank 0 prints one JSON line
+with the whole-job value = units of all ranks / max-over-ranks device time.
+
+Workloads (synthetic, seeded; the shapes of Mamba-2 SSD layers):
+  prefill_130m       bf16 x/B/C, fp32 dt/A/D/state: batch 8, 2048 tokens, 24 heads,
+                     P 64, N 128, 1 group, chunk 256                     (headline)
+  prefill_2p7b_long  batch 4, 16384 tokens, 80 heads, P 64, N 128, chunk 256
+  decode_2p7b        batch 64, 80 heads, P 64, N 128 fp32 state seeded by a 512-token
+                     prefill; 1024 decode steps with fresh inputs, one CUDA graph
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from state_space_model_05_b200 import inputs as gen  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+WORKLOADS = {
+    "prefill_130m": dict(kind="prefill", batch=8, seqlen=2048, nheads=24, headdim=64, ngroups=1,
+                         dstate=128, chunk_len=256, dtype="bf16"),
+    "prefill_2p7b_long": dict(kind="prefill", batch=4, seqlen=16384, nheads=80, headdim=64,
+                              ngroups=1, dstate=128, chunk_len=256, dtype="bf16"),
+    "decode_2p7b": dict(kind="decode", batch=64, nheads=80, headdim=64, ngroups=1, dstate=128,
+                        prefill_len=512, prefill_chunk=64, steps=1024, dtype="f32"),
+}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ accounting
+def prefill_flops(w) -> dict:
+    """Algorithmic (causal-exact) FLOPs per call, total and per kernel."""
+    b, T, H, P, G, N, Q = (w[k] for k in ("batch", "seqlen", "nheads", "headdim", "ngroups", "dstate", "chunk_len"))
+    tokens = b * T
+    gemm1 = tokens * G * (Q + 1) * N          # C B^T, lower triangle incl. diagonal
+    gemm2 = tokens * H * (Q + 1) * P          # (masked) X
+    cstate = tokens * H * 2 * N * P           # chunk states
+    cout = tokens * H * 2 * N * P             # carried state -> output
+    return {"total": gemm1 + gemm2 + cstate + cout,
+            "chunk_output": gemm1 + gemm2 + cout, "chunk_state": cstate}
+
+
+def prefill_bytes(w) -> dict:
+    b, T, H, P, G, N, Q = (w[k] for k in ("batch", "seqlen", "nheads", "headdim", "ngroups", "dstate", "chunk_len"))
+    e = 2 if w["dtype"] == "bf16" else 4
+    c = -(-T // Q)
+    io = b * T * (2 * H * P * e + 2 * G * N * e + H * 4) + b * H * P * N * 4
+    return {"total": io,
+            "state_scan": 2 * b * H * c * P * N * 4 + b * H * P * N * 4,
+            "chunk_cumsum": b * T * H * 4 + b * H * c * Q * 4}
+
+
+def decode_bytes(w) -> int:
+    b, H, P, G, N = (w[k] for k in ("batch", "nheads", "headdim", "ngroups", "dstate"))
+    return 2 * b * H * P * N * 4 + 2 * b * H * P * 4 + 2 * b * G * N * 4 + b * H * 4
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "state_space_model_05_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on this source."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    sha = kernel_source_sha()
+    for ln in lines:
+        if ln.startswith("#") or "=" not in ln:
+            continue
+        kv = dict(tok.split("=", 1) for tok in ln.split())
+        if kv.get("kernel") == kernel and kv.get("workload") == workload and kv.get("source_sha") == sha:
+            return int(float(kv["dram_bytes_per_launch"]))
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of this GPU's clocks and throttle reasons."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.proc = None
+        self.out = None
+        if gpu_id is None:
+            return
+        try:
+            self.out = open(f"/tmp/ssd_clocks_{os.getpid()}.csv", "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        for ln in open(self.out.name).read().splitlines():
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.out.name)
+        if not rows:
+            return {"samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(value: float, world: int) -> float:
+    """Max over ranks of a host float (device time per rank)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ our arm
+def _dev(a, dtype):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device="cuda", dtype=dtype)
+
+
+def prefill_problem(w, seed):
+    shape = gen.SSDShape(w["batch"], w["seqlen"], w["nheads"], w["headdim"], w["ngroups"], w["dstate"])
+    inp = gen.prefill_inputs(shape, seed=seed)
+    if w["dtype"] == "bf16":
+        inp.x, inp.B, inp.C = gen.round_bf16(inp.x), gen.round_bf16(inp.B), gen.round_bf16(inp.C)
+    return inp
+
+
+def run_prefill(w, steps, warmup, rank, world, name, e2e=True):
+    import torch
+    import state_space_model_05_b200 as ssd
+    from state_space_model_05_b200 import binding
+    dt_ = torch.bfloat16 if w["dtype"] == "bf16" else torch.float32
+    inp = prefill_problem(w, seed=rank)
+    b, T, H, P, G, N, Q = (w[k] for k in ("batch", "seqlen", "nheads", "headdim", "ngroups", "dstate", "chunk_len"))
+    code = binding.SSD_BF16 if w["dtype"] == "bf16" else binding.SSD_F32
+    ws_bytes = ssd.ssd_prefill_workspace_bytes(b, T, H, P, G, N, Q, code)
+    per_replica = prefill_bytes(w)["total"] + ws_bytes + b * T * H * P * (2 if w["dtype"] == "bf16" else 4)
+    replicas = max(1, math.ceil(3 * L2_BYTES / per_replica))
+    reps = []
+    for _ in range(replicas):
+        reps.append(dict(x=_dev(inp.x, dt_), dt=_dev(inp.dt, torch.float32), A=_dev(inp.A, torch.float32),
+                         B=_dev(inp.B, dt_), C=_dev(inp.C, dt_), D=_dev(inp.D, torch.float32),
+                         y=torch.empty((b, T, H, P), device="cuda", dtype=dt_),
+                         st=torch.empty((b, H, P, N), device="cuda", dtype=torch.float32),
+                         ws=torch.empty(ws_bytes, device="cuda", dtype=torch.uint8)))
+
+    def step(i):
+        r = reps[i % replicas]
+        ssd.ssd_prefill(r["x"], r["dt"], r["A"], r["B"], r["C"], r["D"], Q, y=r["y"],
+                        final_state=r["st"], workspace=r["ws"])
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert ssd.ssd_device_status() == 0
+    binding.ssd_profile_reset()
+    binding.ssd_profile_enable(True)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    s0.record()
+    for i in range(steps):
+        step(i)
+    s1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    binding.ssd_profile_enable(False)
+    kernels = binding.ssd_profile_read()
+    ms = s0.elapsed_time(s1)
+    status = ssd.ssd_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after {name}")
+    ms_max = reduce_max(ms, world)
+    tokens = b * T * steps * world
+    res = {"ms_total": ms_max, "ms_per_step": ms_max / steps, "tokens_per_s": tokens / (ms_max / 1e3),
+           "kernels": kernels, "replicas": replicas, "launches": sum(v[1] for v in kernels.values())}
+
+    if e2e:
+        # end to end through the public call with host buffers: H2D inputs, prefill, D2H outputs
+        pin = lambda a, d: torch.from_numpy(np.ascontiguousarray(a)).to(d).pin_memory()
+        hx, hdt, hB, hC = pin(inp.x, dt_), pin(inp.dt, torch.float32), pin(inp.B, dt_), pin(inp.C, dt_)
+        hy = torch.empty((b, T, H, P), dtype=dt_).pin_memory()
+        hst = torch.empty((b, H, P, N), dtype=torch.float32).pin_memory()
+        r = reps[0]
+
+        def e2e_step():
+            r["x"].copy_(hx, non_blocking=True)
+            r["dt"].copy_(hdt, non_blocking=True)
+            r["B"].copy_(hB, non_blocking=True)
+            r["C"].copy_(hC, non_blocking=True)
+            ssd.ssd_prefill(r["x"], r["dt"], r["A"], r["B"], r["C"], r["D"], Q, y=r["y"],
+                            final_state=r["st"], workspace=r["ws"])
+            hy.copy_(r["y"], non_blocking=True)
+            hst.copy_(r["st"], non_blocking=True)
+
+        for _ in range(max(1, warmup)):
+            e2e_step()
+        barrier(world)
+        torch.cuda.synchronize()
+        s0.record()
+        for _ in range(steps):
+            e2e_step()
+        s1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        ems = reduce_max(s0.elapsed_time(s1), world)
+        h2d = sum(t.numel() * t.element_size() for t in (hx, hdt, hB, hC))
+        d2h = hy.numel() * hy.element_size() + hst.numel() * hst.element_size()
+        res["e2e"] = {"value": tokens / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h}
+    return res
+
+
+def run_decode(w, repeats, warmup, rank, world):
+    import torch
+    import state_space_model_05_b200 as ssd
+    from state_space_model_05_b200 import binding
+    b, H, P, G, N, S = (w[k] for k in ("batch", "nheads", "headdim", "ngroups", "dstate", "steps"))
+    shape = gen.SSDShape(b, w["prefill_len"], H, P, G, N)
+    inp = gen.prefill_inputs(shape, seed=rank)
+    f32 = torch.float32
+    _, state = ssd.ssd_prefill(_dev(inp.x, f32), _dev(inp.dt, f32), _dev(inp.A, f32), _dev(inp.B, f32),
+                               _dev(inp.C, f32), _dev(inp.D, f32), w["prefill_chunk"])
+    dec = gen.decode_inputs(gen.SSDShape(b, 1, H, P, G, N), steps=S, seed=1000 + rank)
+    X, DT, Bs, Cs = (_dev(a, f32) for a in (dec.x, dec.dt, dec.B, dec.C))
+    A, D = _dev(inp.A, f32), _dev(inp.D, f32)
+    y = torch.empty((b, H, P), device="cuda")
+    del inp
+    torch.cuda.synchronize()
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for k in range(4):                           # eager warm-up before capture
+            ssd.ssd_decode_step(state, X[k], DT[k], A, Bs[k], Cs[k], D, y_t=y)
+    torch.cuda.synchronize()
+    binding.ssd_profile_reset()
+    binding.ssd_profile_enable(True)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for k in range(S):
+                ssd.ssd_decode_step(state, X[k], DT[k], A, Bs[k], Cs[k], D, y_t=y)
+    binding.ssd_profile_enable(False)
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    s0.record()
+    for _ in range(repeats):
+        g.replay()
+    s1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    kernels = binding.ssd_profile_read()              # events of the latest replay
+    ms = reduce_max(s0.elapsed_time(s1), world)
+    status = ssd.ssd_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after decode")
+    steps_total = S * repeats
+    kms, klaunch = kernels.get("decode_step", (float("nan"), 0))
+    nbytes = decode_bytes(w)
+    res = {"steps_per_s": steps_total * world / (ms / 1e3), "ms_per_step": ms / steps_total,
+           "gbs": nbytes * steps_total / (ms / 1e3) / 1e9, "kernel_ms": kms / max(klaunch, 1),
+           "launches": steps_total, "bytes_per_step": nbytes}
+    del g
+    return res
+
+
+def roofline_prefill(w, res, peaks, src, workload):
+    flops = prefill_flops(w)
+    byts = prefill_bytes(w)
+    kernels = res["kernels"]
+    dom = max(kernels, key=lambda k: kernels[k][0])
+    ms, n = kernels[dom]
+    per_launch_ms = ms / n
+    if dom.startswith("chunk_output") or dom.startswith("chunk_state"):
+        work = flops["chunk_output" if dom.startswith("chunk_output") else "chunk_state"]
+        achieved = work / (per_launch_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s"}
+    else:
+        work = byts[dom]
+        achieved = work / (per_launch_ms / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s"}
+    roof.update({"frac": achieved / peak, "traffic": recorded_traffic(dom, workload), "kernel": dom,
+                 "kernel_ms": per_launch_ms, "peak_source": src})
+    return roof
+
+
+def ours(args, rank, world):
+    import torch
+    from state_space_model_05_b200.build import build
+    build()
+    w = WORKLOADS[args.workload]
+    peaks, src = load_peaks()
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+    except Exception:  # noqa: BLE001
+        gpu_id = str(torch.cuda.current_device())
+    clocks = ClockSampler(gpu_id)
+    line = {"metric": "", "value": None, "unit": "", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "data": "synthetic (seeded; see DESIGN.md input recipe)"}
+    if w["kind"] == "prefill":
+        res = run_prefill(w, args.steps, args.warmup, rank, world, args.workload)
+        flops = prefill_flops(w)["total"]
+        line.update({"metric": "SSD prefill tokens/s", "value": res["tokens_per_s"], "unit": "tokens/s",
+                     "ms_per_step": res["ms_per_step"], "dtype": w["dtype"]})
+        line["prefill_tflops"] = flops / (res["ms_per_step"] / 1e3) / 1e12
+        line["prefill_tensor_frac"] = line["prefill_tflops"] / peaks["bf16_tflops"]
+        line["roofline"] = roofline_prefill(w, res, peaks, src, args.workload)
+        line["e2e"] = res.get("e2e")
+        line["gpu_launches"] = res["launches"]
+        line["kernels_ms"] = {k: v[0] / v[1] for k, v in res["kernels"].items()}
+        cfg = {"workload": args.workload, **{k: w[k] for k in w if k != "kind"},
+               "l2": f"inputs rotated over {res['replicas']} resident replicas (> 3x L2) between steps"}
+    else:
+        res = run_decode(w, max(1, args.steps // 100), max(1, args.warmup // 3), rank, world)
+        line.update({"metric": "SSD decode steps/s", "value": res["steps_per_s"], "unit": "steps/s",
+                     "ms_per_step": res["ms_per_step"], "dtype": "f32"})
+        kgbs = res["bytes_per_step"] / (res["kernel_ms"] / 1e3) / 1e9
+        line["roofline"] = {"bound": "hbm", "achieved": kgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": kgbs / peaks["hbm_gbs"], "traffic": recorded_traffic("decode_step", args.workload),
+                            "kernel": "decode_step", "peak_source": src}
+        line["gpu_launches"] = res["launches"]
+        line["e2e"] = None
+        cfg = {"workload": args.workload, **{k: w[k] for k in w if k != "kind"}}
+    cfg["parallelism"] = f"independent problem per GPU x{world}"
+    line["config"] = cfg
+
+    if not args.no_extras and args.workload == "prefill_130m":
+        dw = WORKLOADS["decode_2p7b"]
+        d = run_decode(dw, 3, 1, rank, world)
+        kgbs = d["bytes_per_step"] / (d["kernel_ms"] / 1e3) / 1e9
+        line["decode_2p7b"] = {"value": d["steps_per_s"], "unit": "steps/s", "ms_per_step": d["ms_per_step"],
+                               "gbs_whole_step": d["gbs"], "roofline": {
+                                   "bound": "hbm", "achieved": kgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                   "frac": kgbs / peaks["hbm_gbs"], "kernel": "decode_step",
+                                   "traffic": recorded_traffic("decode_step", "decode_2p7b"), "peak_source": src},
+                               "config": {k: dw[k] for k in dw if k != "kind"}}
+        lw = WORKLOADS["prefill_2p7b_long"]
+        l = run_prefill(lw, 5, 2, rank, world, "prefill_2p7b_long", e2e=False)
+        fl = prefill_flops(lw)["total"]
+        line["prefill_2p7b_long"] = {"value": l["tokens_per_s"], "unit": "tokens/s", "ms_per_step": l["ms_per_step"],
+                                     "prefill_tflops": fl / (l["ms_per_step"] / 1e3) / 1e12,
+                                     "prefill_tensor_frac": fl / (l["ms_per_step"] / 1e3) / 1e12 / peaks["bf16_tflops"],
+                                     "roofline": roofline_prefill(lw, l, peaks, src, "prefill_2p7b_long"),
+                                     "kernels_ms": {k: v[0] / v[1] for k, v in l["kernels"].items()}}
+    line["clocks"] = clocks.stop()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and w["kind"] == "prefill":
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=20.0)
+    return line
+
+
+# ------------------------------------------------------------------ oracle timing
+def oracle_sample_step(w, inp, units):
+    import oracle
+    t = time.perf_counter()
+    oracle.prefill(inp.x, inp.dt, inp.A, inp.B, inp.C, inp.D, units=units)
+    return time.perf_counter() - t
+
+
+def cpu_baseline(w, budget_s=20.0):
+    import oracle
+    oracle.build()
+    inp = prefill_problem(w, seed=0)
+    H, T = w["nheads"], w["seqlen"]
+    n_all = w["batch"] * H
+    probe = list(range(min(n_all, max(1, oracle.threads()))))
+    t1 = oracle_sample_step(w, inp, probe)
+    per_unit = t1 / len(probe)
+    n = int(min(n_all, max(len(probe), budget_s / max(per_unit, 1e-9))))
+    units = list(range(n))
+    t = oracle_sample_step(w, inp, units)
+    tokens = n / H * T
+    return {"value": tokens / t, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{n} of {n_all} (batch, head) units of the {w['batch']}x{T}-token workload, "
+                      f"fp64 sequential recurrence, {t:.2f} s"}
+
+
+def reference(args, rank, world):
+    """The fp64 CPU oracle as the reference arm (rank 0 only)."""
+    import oracle
+    oracle.build()
+    w = WORKLOADS[args.workload]
+    if w["kind"] != "prefill":
+        return {"impl": "reference", "unavailable": "the oracle reference arm times the prefill workloads"}
+    inp = prefill_problem(w, seed=0)
+    H, T = w["nheads"], w["seqlen"]
+    n_all = w["batch"] * H
+    probe = list(range(min(n_all, max(1, oracle.threads()))))
+    per_unit = oracle_sample_step(w, inp, probe) / len(probe)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    n = int(min(n_all, max(len(probe), budget / max(per_unit, 1e-9))))
+    units = list(range(n))
+    for _ in range(args.warmup):
+        oracle_sample_step(w, inp, units)
+    total = sum(oracle_sample_step(w, inp, units) for _ in range(args.steps))
+    tokens = n / H * T * args.steps
+    value = tokens / total
+    sample = f"{n} of {n_all} (batch, head) units per step of the {w['batch']}x{T}-token workload"
+    return {"impl": "reference", "metric": "SSD prefill tokens/s", "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": {"workload": args.workload, **{k: w[k] for k in w if k != "kind"}},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill_130m")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        if rank != 0:
+            return 0
+        print(json.dumps(reference(args, rank, world)), flush=True)
+        return 0
+    rank, world, _ = dist_setup()
+    try:
+        line = ours(args, rank, world)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

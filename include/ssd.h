@@ -1,0 +1,148 @@
+/*
+ * ssd.h -- C ABI of the B200 (sm_100a) Mamba-2 state-space-duality (SSD) library.
+ *
+ * The operation.  "Compiler-First State Space Duality and Portable O(1)
+ * Autoregressive Caching for Inference" (gist.science summary of arXiv
+ * 2603.09555), section "2. Metodologia", describes the SSD layer of Mamba-2 as
+ * a recurrence with per-head diagonal (scalar) decay that can be evaluated in
+ * fixed-size chunks (prefill over the whole context) or one token at a time
+ * against an O(1) state cache kept on the device (decode), with the decay
+ * exponent taken in fp32.  For batch b, head h, group g = h / (nheads/ngroups):
+ *
+ *     a_t = exp(dt_t * A_h)
+ *     H_t = a_t * H_{t-1} + dt_t * B_t x_t^T          (H: dstate x headdim)
+ *     y_t = C_t^T H_t + D_h * x_t
+ *
+ * ssd_prefill evaluates it over `seqlen` tokens in chunks of `chunk_len`:
+ * per chunk the inclusive cumulative sum of dt*A (the decay exponents), the
+ * intra-chunk product (C B^T o L)(dt x) with the lower-triangular decay mask
+ * L[t][s] = exp(sum_{r=s+1..t} dt_r A_h), the chunk's end state, the state
+ * carried across chunks, and the carried state's contribution to y plus the
+ * D skip.  ssd_decode_step advances the state cache by one token in place.
+ * The result does not depend on chunk_len (up to rounding).
+ *
+ * Layouts (row-major, innermost last; all tensors contiguous):
+ *     x, y         [batch][seqlen][nheads][headdim]       dtype `dtype`
+ *     dt           [batch][seqlen][nheads]                fp32, dt > 0 (already softplus'd)
+ *     A, D         [nheads]                               fp32
+ *     B, C         [batch][seqlen][ngroups][dstate]       dtype `dtype`
+ *     state        [batch][nheads][headdim][dstate]       fp32 (dstate innermost)
+ *     decode x_t, y_t [batch][nheads][headdim]; dt_t [batch][nheads];
+ *     decode B_t, C_t [batch][ngroups][dstate]
+ *
+ * Ownership: the caller allocates every buffer, device memory throughout
+ * (including the prefill workspace); the library allocates no device memory
+ * and keeps no state between calls besides one device error word per device
+ * (and, only while kernel profiling is enabled, host-side event records).
+ *
+ * Streams and errors: every call is asynchronous on `stream` (a cudaStream_t
+ * passed as void*, NULL = legacy default stream) and never synchronises.
+ * Argument errors are detected on the host and returned before anything is
+ * launched; nothing is written in that case.  A failed launch returns
+ * SSD_ERR_CUDA.  A kernel that gives up a bounded wait records SSD_ERR_TIMEOUT
+ * in the device error word, which ssd_device_status reads and clears.
+ *
+ * Requirements: nheads % ngroups == 0; headdim and dstate multiples of 8 with
+ * headdim <= 128 and dstate <= 256 (prefill) or <= 512 (decode); chunk_len in
+ * [1, 256]; every pointer 16-byte aligned; batch in [0, 65535] and seqlen >= 0
+ * (batch 0 does nothing; seqlen 0 only copies init_state, or zeros, to
+ * final_state).  Sizes outside these ranges return SSD_ERR_UNSUPPORTED or
+ * SSD_ERR_SHAPE.  bf16 prefills with headdim 64, dstate 128 and chunk_len
+ * 128 or 256 run on the tensor cores (tcgen05); every other shape runs the
+ * same chunked algorithm on the CUDA cores in fp32.
+ */
+#ifndef SSD_H
+#define SSD_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_NULL = 1,        /* a required pointer is NULL */
+    SSD_ERR_SHAPE = 2,       /* a size is out of range or inconsistent */
+    SSD_ERR_DTYPE = 3,       /* unknown dtype */
+    SSD_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned */
+    SSD_ERR_UNSUPPORTED = 5, /* valid, but not a shape this build implements */
+    SSD_ERR_CUDA = 6,        /* a CUDA call or launch failed */
+    SSD_ERR_TIMEOUT = 7,     /* a device-side bounded wait expired */
+    SSD_ERR_WORKSPACE = 8    /* workspace missing or smaller than required */
+} ssd_status_t;
+
+/* Storage type of x, B, C and y (and of x_t, B_t, C_t, y_t for decode).
+ * dt, A, D and the state are always fp32; accumulation is always fp32. */
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype_t;
+
+/* Version of this ABI (major * 100 + minor). */
+int ssd_abi_version(void);
+
+/* Human-readable name of a status code; never NULL. */
+const char* ssd_status_string(ssd_status_t status);
+
+/*
+ * Bytes of device workspace ssd_prefill needs for these sizes (0 when the
+ * sizes are invalid).  The workspace holds the per-chunk decay exponents and
+ * the per-chunk states; its contents need no initialisation and are not
+ * meaningful after the call.
+ */
+size_t ssd_prefill_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int ngroups,
+                                   int dstate, int chunk_len, ssd_dtype_t dtype);
+
+/*
+ * Chunked prefill.  Reads x, dt, A, B, C, D (and init_state when non-NULL,
+ * the state before the first token; NULL means zeros); writes y and
+ * final_state (the state after the last token).  x, B, C and y are `dtype`;
+ * y is rounded once to `dtype` from fp32.  `workspace` must hold at least
+ * ssd_prefill_workspace_bytes(...) bytes of device memory.
+ * init_state may be the same buffer as final_state (each state element is
+ * read before it is written); otherwise no output may overlap any input.
+ */
+ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const void* B,
+                         const void* C, const float* D, const float* init_state, int batch,
+                         int seqlen, int nheads, int headdim, int ngroups, int dstate,
+                         int chunk_len, ssd_dtype_t dtype, void* y, float* final_state,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One decode step on the state cache, in place: each fp32 state row is read
+ * once, decayed by exp(dt_t * A_h), given the rank-1 update dt_t B_t x_t^T,
+ * reduced against C_t for y_t, and written back.  x_t, B_t, C_t, y_t are
+ * `dtype`.  No host synchronisation; any number of steps may be queued or
+ * captured in a CUDA graph.
+ */
+ssd_status_t ssd_decode_step(float* state, const void* x_t, const float* dt_t, const float* A,
+                             const void* B_t, const void* C_t, const float* D, int batch,
+                             int nheads, int headdim, int ngroups, int dstate, ssd_dtype_t dtype,
+                             void* y_t, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears this device's error word.
+ * Returns SSD_OK, SSD_ERR_TIMEOUT (a bounded wait expired in a kernel since
+ * the last call), or SSD_ERR_CUDA when the stream reports a CUDA error.
+ */
+ssd_status_t ssd_device_status(void* stream);
+
+/*
+ * Kernel profiling (diagnostics; off by default).  While enabled, ssd_prefill
+ * and ssd_decode_step record a CUDA event before and after each kernel they
+ * launch, on the call's stream (so the events may also be captured in a CUDA
+ * graph; they then re-record on every replay and a read reflects the latest
+ * replay).  ssd_profile_read synchronises on
+ * the recorded events and returns, per kernel name, the summed milliseconds
+ * and the number of launches since the last ssd_profile_reset.  Not thread
+ * safe; meant for benchmarks.
+ */
+void ssd_profile_enable(int on);
+void ssd_profile_reset(void);
+/* Writes up to max_kernels entries; returns the number written, or -1 on a
+ * CUDA error.  `names` receives static strings owned by the library. */
+int ssd_profile_read(int max_kernels, const char** names, double* total_ms, long long* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_H */

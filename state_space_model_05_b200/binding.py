@@ -1,0 +1,177 @@
+"""ctypes binding of the SSD C ABI (``include/ssd.h``).
+
+Argument marshalling only: tensors are passed as device pointers together with
+the current CUDA stream; every step of the computation runs in the CUDA library.
+There is no fallback -- if ``libssd.so`` is missing or a call fails, an exception
+is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libssd.so")
+
+SSD_OK = 0
+SSD_ERR_TIMEOUT = 7
+SSD_F32 = 0
+SSD_BF16 = 1
+
+STATUS_NAMES = {0: "SSD_OK", 1: "SSD_ERR_NULL", 2: "SSD_ERR_SHAPE", 3: "SSD_ERR_DTYPE",
+                4: "SSD_ERR_ALIGN", 5: "SSD_ERR_UNSUPPORTED", 6: "SSD_ERR_CUDA",
+                7: "SSD_ERR_TIMEOUT", 8: "SSD_ERR_WORKSPACE"}
+
+# exported symbols and their ctypes signatures, as declared in include/ssd.h
+_P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = {
+    "ssd_abi_version": ([], _I),
+    "ssd_status_string": ([_I], ctypes.c_char_p),
+    "ssd_prefill_workspace_bytes": ([_I, _I, _I, _I, _I, _I, _I, _I], _Z),
+    "ssd_prefill": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _Z, _P], _I),
+    "ssd_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
+    "ssd_device_status": ([_P], _I),
+    "ssd_profile_enable": ([_I], None),
+    "ssd_profile_reset": ([], None),
+    "ssd_profile_read": ([_I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),
+                          ctypes.POINTER(ctypes.c_longlong)], _I),
+}
+
+_lib = None
+
+
+class SSDError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({_status_text(status)})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if the CUDA extension has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"SSD CUDA library not built: {LIB_PATH} is missing "
+                               "(run `python -m state_space_model_05_b200.build`)")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(l, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = l
+    return _lib
+
+
+def _status_text(status: int) -> str:
+    try:
+        return lib().ssd_status_string(status).decode()
+    except Exception:  # noqa: BLE001 - only used for messages
+        return "?"
+
+
+def _check(status: int, what: str):
+    if status != SSD_OK:
+        raise SSDError(status, what)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SSD_F32
+    if t.dtype == torch.bfloat16:
+        return SSD_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}")
+
+
+def ssd_prefill_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len, dtype_code):
+    return int(lib().ssd_prefill_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate,
+                                                 chunk_len, dtype_code))
+
+
+def ssd_prefill(x, dt, A, B, C, D, chunk_len, init_state=None, y=None, final_state=None,
+                workspace=None, stream=None):
+    """Chunked SSD prefill.  Shapes as in ``include/ssd.h``; returns ``(y, final_state)``."""
+    for t, n in ((x, "x"), (B, "B"), (C, "C")):
+        _need(t, n, x.dtype)
+    for t, n in ((dt, "dt"), (A, "A"), (D, "D")):
+        _need(t, n, torch.float32)
+    code = _dtype_code(x)
+    batch, seqlen, nheads, headdim = x.shape
+    ngroups, dstate = B.shape[2], B.shape[3]
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None:
+        final_state = torch.empty((batch, nheads, headdim, dstate), device=x.device, dtype=torch.float32)
+    if init_state is not None:
+        _need(init_state, "init_state", torch.float32)
+    need = ssd_prefill_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len, code)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=x.device, dtype=torch.uint8)
+    st = lib().ssd_prefill(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state),
+                           batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len, code,
+                           _ptr(y), _ptr(final_state), _ptr(workspace), workspace.numel(),
+                           _stream(stream))
+    _check(st, "ssd_prefill")
+    return y, final_state
+
+
+def ssd_decode_step(state, x_t, dt_t, A, B_t, C_t, D, y_t=None, stream=None):
+    """One decode step; ``state`` [b][H][P][N] fp32 is updated in place.  Returns ``y_t``."""
+    _need(state, "state", torch.float32)
+    for t, n in ((x_t, "x_t"), (B_t, "B_t"), (C_t, "C_t")):
+        _need(t, n, x_t.dtype)
+    for t, n in ((dt_t, "dt_t"), (A, "A"), (D, "D")):
+        _need(t, n, torch.float32)
+    batch, nheads, headdim = x_t.shape
+    ngroups, dstate = B_t.shape[1], B_t.shape[2]
+    if y_t is None:
+        y_t = torch.empty_like(x_t)
+    st = lib().ssd_decode_step(_ptr(state), _ptr(x_t), _ptr(dt_t), _ptr(A), _ptr(B_t), _ptr(C_t),
+                               _ptr(D), batch, nheads, headdim, ngroups, dstate, _dtype_code(x_t),
+                               _ptr(y_t), _stream(stream))
+    _check(st, "ssd_decode_step")
+    return y_t
+
+
+def ssd_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error word."""
+    return int(lib().ssd_device_status(_stream(stream)))
+
+
+def ssd_profile_enable(on: bool = True):
+    lib().ssd_profile_enable(1 if on else 0)
+
+
+def ssd_profile_reset():
+    lib().ssd_profile_reset()
+
+
+def ssd_profile_read() -> dict:
+    """{kernel name: (total_ms, launches)} since the last reset (synchronises)."""
+    n = 16
+    names = (ctypes.c_char_p * n)()
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_longlong * n)()
+    k = lib().ssd_profile_read(n, names, ms, cnt)
+    if k < 0:
+        raise SSDError(6, "ssd_profile_read")
+    return {names[i].decode(): (ms[i], cnt[i]) for i in range(k)}

@@ -1,0 +1,261 @@
+// C ABI of the SSD library: argument validation, workspace sizing and dispatch.
+// Every entry point validates on the host before launching anything and only
+// enqueues work on the caller's stream.
+#include <stdint.h>
+#include <string.h>
+
+#include <vector>
+
+#include "common.cuh"
+#include "prefill_tc.h"
+
+namespace ssd {
+
+__device__ int g_error_word = 0;
+
+int* device_error_word()
+{
+    static int* cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+        cache[dev] = static_cast<int*>(p);
+    }
+    return cache[dev];
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ssd_status_t check_common(int batch, int nheads, int headdim, int ngroups, int dstate,
+                          ssd_dtype_t dtype, int max_dstate)
+{
+    if (dtype != SSD_F32 && dtype != SSD_BF16) return SSD_ERR_DTYPE;
+    if (batch < 0 || batch > 65535) return SSD_ERR_SHAPE;
+    if (nheads < 1 || nheads > 65535 || ngroups < 1 || nheads % ngroups != 0) return SSD_ERR_SHAPE;
+    if (headdim < 8 || headdim % 8 != 0 || dstate < 8 || dstate % 8 != 0) return SSD_ERR_SHAPE;
+    if (headdim > 128 || dstate > max_dstate) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+ssd_status_t prefill_dims(int batch, int seqlen, int nheads, int headdim, int ngroups, int dstate,
+                          int chunk_len, ssd_dtype_t dtype, Dims* d)
+{
+    ssd_status_t st = check_common(batch, nheads, headdim, ngroups, dstate, dtype, 256);
+    if (st != SSD_OK) return st;
+    if (seqlen < 0 || chunk_len < 1) return SSD_ERR_SHAPE;
+    if (chunk_len > 256) return SSD_ERR_UNSUPPORTED;
+    d->batch = batch;
+    d->seqlen = seqlen;
+    d->nheads = nheads;
+    d->headdim = headdim;
+    d->ngroups = ngroups;
+    d->dstate = dstate;
+    d->chunk_len = chunk_len;
+    d->nchunks = (seqlen + chunk_len - 1) / chunk_len;
+    return SSD_OK;
+}
+
+ssd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
+
+// ---- opt-in kernel profiling: an event pair around each launch -------------------
+enum Stage { kCumsum, kStateTc, kStateSimt, kScan, kOutTc, kOutSimt, kDecode, kCopy, kNumStages };
+const char* const kStageNames[kNumStages] = {"chunk_cumsum", "chunk_state_tc", "chunk_state_simt",
+                                              "state_scan", "chunk_output_tc", "chunk_output_simt",
+                                              "decode_step", "copy_state"};
+struct ProfRecord { int stage; cudaEvent_t begin, end; };
+struct Profiler {
+    bool on = false;
+    std::vector<ProfRecord> records;
+    std::vector<cudaEvent_t> pool;
+    size_t used = 0;
+    cudaEvent_t next() {
+        if (used == pool.size()) {
+            cudaEvent_t e = nullptr;
+            if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+            pool.push_back(e);
+        }
+        return pool[used++];
+    }
+};
+Profiler g_prof;
+
+// Runs `launch` between two profiling events when profiling is enabled.
+template <typename F>
+cudaError_t profiled(int stage, cudaStream_t s, F&& launch)
+{
+    if (!g_prof.on) return launch();
+    cudaEvent_t a = g_prof.next(), b = g_prof.next();
+    if (a) cudaEventRecord(a, s);
+    const cudaError_t e = launch();
+    if (b) cudaEventRecord(b, s);
+    if (a && b) g_prof.records.push_back({stage, a, b});
+    return e;
+}
+
+}  // namespace
+
+size_t prefill_workspace_layout(const Dims& d, void* base, PrefillWorkspace* ws)
+{
+    const size_t units = (size_t)d.batch * d.nheads * d.nchunks;
+    const size_t lam_bytes = align_up(units * d.chunk_len * sizeof(float));
+    const size_t st_bytes = align_up(units * d.headdim * d.dstate * sizeof(float));
+    if (ws) {
+        char* p = static_cast<char*>(base);
+        ws->lam = reinterpret_cast<float*>(p);
+        ws->states = reinterpret_cast<float*>(p + lam_bytes);
+    }
+    return lam_bytes + st_bytes;
+}
+
+}  // namespace ssd
+
+using namespace ssd;
+
+extern "C" {
+
+int ssd_abi_version(void) { return 100; }
+
+const char* ssd_status_string(ssd_status_t s)
+{
+    switch (s) {
+        case SSD_OK: return "ok";
+        case SSD_ERR_NULL: return "a required pointer is NULL";
+        case SSD_ERR_SHAPE: return "invalid or inconsistent sizes";
+        case SSD_ERR_DTYPE: return "unknown dtype";
+        case SSD_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        case SSD_ERR_UNSUPPORTED: return "shape not supported by this build";
+        case SSD_ERR_CUDA: return "CUDA error";
+        case SSD_ERR_TIMEOUT: return "device-side bounded wait expired";
+        case SSD_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+size_t ssd_prefill_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int ngroups,
+                                   int dstate, int chunk_len, ssd_dtype_t dtype)
+{
+    Dims d;
+    if (prefill_dims(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len, dtype, &d) != SSD_OK)
+        return 0;
+    return prefill_workspace_layout(d, nullptr, nullptr);
+}
+
+ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const void* B,
+                         const void* C, const float* D, const float* init_state, int batch,
+                         int seqlen, int nheads, int headdim, int ngroups, int dstate,
+                         int chunk_len, ssd_dtype_t dtype, void* y, float* final_state,
+                         void* workspace, size_t workspace_bytes, void* stream)
+{
+    Dims d;
+    ssd_status_t st = prefill_dims(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len,
+                                   dtype, &d);
+    if (st != SSD_OK) return st;
+    if (batch == 0) return SSD_OK;
+    if (!final_state) return SSD_ERR_NULL;
+    if (!aligned16(final_state) || !aligned16(init_state)) return SSD_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (seqlen == 0)
+        return from_cuda(profiled(kCopy, s, [&] { return launch_copy_state(d, init_state, final_state, s); }));
+
+    if (!x || !dt || !A || !B || !C || !D || !y) return SSD_ERR_NULL;
+    if (!aligned16(x) || !aligned16(dt) || !aligned16(A) || !aligned16(B) || !aligned16(C) ||
+        !aligned16(D) || !aligned16(y) || !aligned16(workspace))
+        return SSD_ERR_ALIGN;
+    PrefillWorkspace ws;
+    const size_t need = prefill_workspace_layout(d, workspace, &ws);
+    if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
+
+    const bool tc = dtype == SSD_BF16 && tc_prefill_supported(d);
+    cudaError_t e = profiled(kCumsum, s, [&] { return launch_chunk_cumsum(d, dt, A, ws.lam, s); });
+    if (e == cudaSuccess) {
+        e = tc ? profiled(kStateTc, s, [&] { return launch_chunk_state_tc(d, x, dt, B, ws.lam, ws.states, s); })
+               : profiled(kStateSimt, s, [&] {
+                     return launch_chunk_state_simt(d, dtype, x, dt, B, ws.lam, ws.states, s);
+                 });
+    }
+    if (e == cudaSuccess)
+        e = profiled(kScan, s, [&] {
+            return launch_state_scan(d, ws.lam, ws.states, init_state, final_state, s);
+        });
+    if (e == cudaSuccess) {
+        e = tc ? profiled(kOutTc, s, [&] {
+                     return launch_chunk_output_tc(d, x, dt, B, C, D, ws.lam, ws.states, y, s);
+                 })
+               : profiled(kOutSimt, s, [&] {
+                     return launch_chunk_output_simt(d, dtype, x, dt, B, C, D, ws.lam, ws.states, y, s);
+                 });
+    }
+    return from_cuda(e);
+}
+
+ssd_status_t ssd_decode_step(float* state, const void* x_t, const float* dt_t, const float* A,
+                             const void* B_t, const void* C_t, const float* D, int batch,
+                             int nheads, int headdim, int ngroups, int dstate, ssd_dtype_t dtype,
+                             void* y_t, void* stream)
+{
+    ssd_status_t st = check_common(batch, nheads, headdim, ngroups, dstate, dtype, 512);
+    if (st != SSD_OK) return st;
+    if (batch == 0) return SSD_OK;
+    if (!state || !x_t || !dt_t || !A || !B_t || !C_t || !D || !y_t) return SSD_ERR_NULL;
+    if (!aligned16(state) || !aligned16(x_t) || !aligned16(dt_t) || !aligned16(A) ||
+        !aligned16(B_t) || !aligned16(C_t) || !aligned16(D) || !aligned16(y_t))
+        return SSD_ERR_ALIGN;
+    Dims d{batch, 1, nheads, headdim, ngroups, dstate, 1, 1};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return from_cuda(profiled(kDecode, s, [&] {
+        return launch_decode(d, dtype, state, x_t, dt_t, A, B_t, C_t, D, y_t, s);
+    }));
+}
+
+ssd_status_t ssd_device_status(void* stream)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SSD_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(int)) != cudaSuccess) return SSD_ERR_CUDA;
+    if (word != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return SSD_ERR_CUDA;
+        return static_cast<ssd_status_t>(word);
+    }
+    return SSD_OK;
+}
+
+void ssd_profile_enable(int on) { g_prof.on = on != 0; }
+
+void ssd_profile_reset(void)
+{
+    g_prof.records.clear();
+    g_prof.used = 0;
+}
+
+int ssd_profile_read(int max_kernels, const char** names, double* total_ms, long long* launches)
+{
+    double ms[kNumStages] = {0};
+    long long n[kNumStages] = {0};
+    for (const ProfRecord& r : g_prof.records) {
+        if (cudaEventSynchronize(r.end) != cudaSuccess) return -1;
+        float t = 0.f;
+        if (cudaEventElapsedTime(&t, r.begin, r.end) != cudaSuccess) return -1;
+        ms[r.stage] += t;
+        n[r.stage] += 1;
+    }
+    int k = 0;
+    for (int i = 0; i < kNumStages && k < max_kernels; ++i) {
+        if (n[i] == 0) continue;
+        if (names) names[k] = kStageNames[i];
+        if (total_ms) total_ms[k] = ms[i];
+        if (launches) launches[k] = n[i];
+        ++k;
+    }
+    return k;
+}
+
+}  // extern "C"

@@ -1,0 +1,78 @@
+// Shared internals of the SSD library (device helpers, launch declarations).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ssd.h"
+
+namespace ssd {
+
+// Device error word (one per device, defined in api.cu): kernels that wait set it
+// when a bounded wait expires; ssd_device_status reads and clears it.  Kernels get
+// its address as an argument.
+int* device_error_word();   // host: address on the current device (nullptr on failure)
+
+__device__ __forceinline__ void record_error(int* err, int code) {
+    if (err) atomicCAS(err, 0, code);
+}
+
+// ---- element loads/stores for the two storage types -------------------------------
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float load(const float* p) { return *p; }
+    static __device__ __forceinline__ void store(float* p, float v) { *p = v; }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float load(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+    static __device__ __forceinline__ void store(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+};
+
+// Four consecutive elements as fp32 (16-byte load for fp32, 8-byte for bf16).
+template <typename T> __device__ __forceinline__ float4 load4(const T* p);
+template <> __device__ __forceinline__ float4 load4<float>(const float* p) {
+    return *reinterpret_cast<const float4*>(p);
+}
+template <> __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    float4 r;
+    r.x = __uint_as_float(u.x << 16);
+    r.y = __uint_as_float(u.x & 0xFFFF0000u);
+    r.z = __uint_as_float(u.y << 16);
+    r.w = __uint_as_float(u.y & 0xFFFF0000u);
+    return r;
+}
+
+// ---- problem description passed to every launcher ---------------------------------
+struct Dims {
+    int batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len, nchunks;
+};
+
+// Workspace layout of the chunked prefill (byte offsets from the workspace base).
+struct PrefillWorkspace {
+    float* lam;      // [batch][nheads][nchunks][chunk_len]   inclusive cumsum of dt*A
+    float* states;   // [batch][nheads][nchunks][headdim][dstate]
+};
+size_t prefill_workspace_layout(const Dims& d, void* base, PrefillWorkspace* ws);
+
+// ---- launchers (return cudaGetLastError() of their launches) -----------------------
+cudaError_t launch_decode(const Dims& d, ssd_dtype_t dtype, float* state, const void* x,
+                          const float* dt, const float* A, const void* B, const void* C,
+                          const float* D, void* y, cudaStream_t s);
+
+cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, float* lam,
+                                cudaStream_t s);
+cudaError_t launch_chunk_state_simt(const Dims& d, ssd_dtype_t dtype, const void* x,
+                                    const float* dt, const void* B, const float* lam,
+                                    float* states, cudaStream_t s);
+cudaError_t launch_state_scan(const Dims& d, const float* lam, float* states,
+                              const float* init_state, float* final_state, cudaStream_t s);
+cudaError_t launch_chunk_output_simt(const Dims& d, ssd_dtype_t dtype, const void* x,
+                                     const float* dt, const void* B, const void* C,
+                                     const float* D, const float* lam, const float* states,
+                                     void* y, cudaStream_t s);
+cudaError_t launch_copy_state(const Dims& d, const float* init_state, float* final_state,
+                              cudaStream_t s);
+
+}  // namespace ssd

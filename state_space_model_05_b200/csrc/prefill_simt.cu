@@ -1,0 +1,408 @@
+// Chunked SSD prefill on the CUDA cores (fp32 arithmetic), plus the two kernels
+// the tensor-core path shares with it: the per-chunk decay cumsum and the scan of
+// chunk states across chunks.
+//
+// "Compiler-First State Space Duality and Portable O(1) Autoregressive Caching
+// for Inference", section "2. Metodologia": the recurrence splits into chunks of
+// fixed size; inside a chunk it is a masked matrix product built from a static
+// lower-triangular mask; across chunks only an N x P state per (batch, head) is
+// carried; the decay exponents are formed in fp32.  For chunk c of head h with
+// Lam_t the inclusive cumsum of dt*A over the chunk's tokens:
+//   (1) Lam_t = sum_{r <= t, r in chunk} dt_r A_h
+//   (2) y_t  = sum_{s <= t} (C_t . B_s) exp(Lam_t - Lam_s) dt_s x_s
+//   (3) S_c  = sum_s exp(Lam_end - Lam_s) dt_s x_s B_s^T      (chunk state from zero)
+//       H_{c+1} = exp(Lam_end) H_c + S_c                      (carried state)
+//   (4) y_t += exp(Lam_t) H_c C_t + D_h x_t
+// States are stored [headdim][dstate].  Tokens past seqlen in the last chunk act
+// as dt = 0, x = 0 (an exact identity on the state).
+#include "common.cuh"
+
+namespace ssd {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+// ----------------------------------------------------------------------------------
+// (1) per (b, chunk, head-tile): Lam over the chunk, written [b][h][c][Q].
+// The chunk's dt block [Q][nheads] is contiguous in memory; it is staged through
+// shared memory so that both the read and the write are coalesced.
+// ----------------------------------------------------------------------------------
+constexpr int kCumsumHeads = 32;
+
+__global__ void __launch_bounds__(kThreads)
+chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
+                    float* __restrict__ lam, int seqlen, int nheads, int Q, int nchunks)
+{
+    extern __shared__ float sm_dt[];                   // [Q][kCumsumHeads]
+    const int c = blockIdx.x, h0 = blockIdx.y * kCumsumHeads, b = blockIdx.z;
+    const int nh = min(kCumsumHeads, nheads - h0);
+    const int t0 = c * Q;
+    for (int i = threadIdx.x; i < Q * kCumsumHeads; i += blockDim.x) {
+        const int t = i / kCumsumHeads, hh = i - t * kCumsumHeads;
+        float v = 0.f;
+        if (hh < nh && t0 + t < seqlen) v = dt[((size_t)b * seqlen + t0 + t) * nheads + h0 + hh];
+        sm_dt[i] = v;
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int hh = warp; hh < nh; hh += kThreads / 32) {
+        const float Ah = A[h0 + hh];
+        float carry = 0.f;
+        float* out = lam + (((size_t)b * nheads + h0 + hh) * nchunks + c) * Q;
+        for (int base = 0; base < Q; base += 32) {
+            const int t = base + lane;
+            float v = (t < Q) ? sm_dt[t * kCumsumHeads + hh] * Ah : 0.f;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
+            }
+            v += carry;
+            if (t < Q) out[t] = v;
+            carry = __shfl_sync(0xffffffffu, v, 31);
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------------
+// (3a) per (b, h, c): chunk state S_c[p][n] = sum_s w_s x_s[p] B_s[n],
+//      w_s = exp(Lam_end - Lam_s) dt_s.
+// Thread (ty, tx): tx owns the n-quad 4tx..4tx+3, ty owns rows ty + rpp*k.
+// ----------------------------------------------------------------------------------
+constexpr int kTokTile = 32;
+constexpr int kMaxRows = 8;
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+chunk_state_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
+                        const T* __restrict__ Bm, const float* __restrict__ lam,
+                        float* __restrict__ states, int seqlen, int nheads, int headdim,
+                        int ngroups, int dstate, int Q, int nchunks)
+{
+    extern __shared__ float sm[];
+    float* sx = sm;                                    // [kTokTile][headdim]
+    float* sb = sx + kTokTile * headdim;               // [kTokTile][dstate]
+    float* sw = sb + kTokTile * dstate;                // [kTokTile]
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int g = h / (nheads / ngroups);
+    const int t0 = c * Q;
+    const int qlen = min(Q, seqlen - t0);
+    const float* lamc = lam + (((size_t)b * nheads + h) * nchunks + c) * Q;
+    const float lam_end = lamc[Q - 1];
+
+    const int nq = dstate >> 2;
+    const int rpp = kThreads / nq;                     // rows per pass
+    const int tx = threadIdx.x % nq, ty = threadIdx.x / nq;
+    const bool active = ty < rpp;
+    float* out = states + (((size_t)b * nheads + h) * nchunks + c) * headdim * dstate;
+
+    for (int pbase = 0; pbase < headdim; pbase += rpp * kMaxRows) {
+        float4 acc[kMaxRows];
+#pragma unroll
+        for (int k = 0; k < kMaxRows; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s0 = 0; s0 < qlen; s0 += kTokTile) {
+            const int ns = min(kTokTile, qlen - s0);
+            __syncthreads();
+            for (int i = threadIdx.x; i < kTokTile * headdim; i += kThreads) {
+                const int s = i / headdim, p = i - s * headdim;
+                sx[i] = s < ns ? Elem<T>::load(x + (((size_t)b * seqlen + t0 + s0 + s) * nheads + h) * headdim + p) : 0.f;
+            }
+            for (int i = threadIdx.x; i < kTokTile * dstate; i += kThreads) {
+                const int s = i / dstate, n = i - s * dstate;
+                sb[i] = s < ns ? Elem<T>::load(Bm + (((size_t)b * seqlen + t0 + s0 + s) * ngroups + g) * dstate + n) : 0.f;
+            }
+            if (threadIdx.x < kTokTile) {
+                const int s = threadIdx.x;
+                sw[s] = s < ns ? expf(lam_end - lamc[s0 + s]) * dt[((size_t)b * seqlen + t0 + s0 + s) * nheads + h] : 0.f;
+            }
+            __syncthreads();
+            if (active) {
+                for (int s = 0; s < ns; ++s) {
+                    const float4 bv = *reinterpret_cast<const float4*>(sb + s * dstate + 4 * tx);
+                    const float ws = sw[s];
+#pragma unroll
+                    for (int k = 0; k < kMaxRows; ++k) {
+                        const int p = pbase + ty + rpp * k;
+                        if (p < headdim) {
+                            const float xv = ws * sx[s * headdim + p];
+                            acc[k].x = fmaf(xv, bv.x, acc[k].x);
+                            acc[k].y = fmaf(xv, bv.y, acc[k].y);
+                            acc[k].z = fmaf(xv, bv.z, acc[k].z);
+                            acc[k].w = fmaf(xv, bv.w, acc[k].w);
+                        }
+                    }
+                }
+            }
+        }
+        if (active) {
+#pragma unroll
+            for (int k = 0; k < kMaxRows; ++k) {
+                const int p = pbase + ty + rpp * k;
+                if (p < headdim) *reinterpret_cast<float4*>(out + (size_t)p * dstate + 4 * tx) = acc[k];
+            }
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------------
+// (3b) per (b, h): walk the chunks in order, replacing each chunk state S_c by the
+// state at the chunk's start H_c, and write the final state.  Each thread owns four
+// consecutive state elements.  In place: init_state may alias final_state.
+// ----------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads)
+state_scan_kernel(const float* __restrict__ lam, float* __restrict__ states,
+                  const float* init_state, float* final_state, int nheads, int PN, int Q,
+                  int nchunks)
+{
+    const int bh = blockIdx.y;
+    const int e = 4 * (blockIdx.x * kThreads + threadIdx.x);
+    if (e >= PN) return;
+    float4 hs = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (init_state) hs = *reinterpret_cast<const float4*>(init_state + (size_t)bh * PN + e);
+    const float* lamr = lam + (size_t)bh * nchunks * Q;
+    float* st = states + (size_t)bh * nchunks * PN + e;
+    float4 nxt = nchunks > 0 ? *reinterpret_cast<const float4*>(st) : hs;
+    for (int c = 0; c < nchunks; ++c) {
+        const float4 sc = nxt;
+        if (c + 1 < nchunks) nxt = *reinterpret_cast<const float4*>(st + (size_t)(c + 1) * PN);
+        *reinterpret_cast<float4*>(st + (size_t)c * PN) = hs;
+        const float ec = expf(lamr[(size_t)c * Q + Q - 1]);
+        hs.x = fmaf(ec, hs.x, sc.x);
+        hs.y = fmaf(ec, hs.y, sc.y);
+        hs.z = fmaf(ec, hs.z, sc.z);
+        hs.w = fmaf(ec, hs.w, sc.w);
+    }
+    *reinterpret_cast<float4*>(final_state + (size_t)bh * PN + e) = hs;
+}
+
+// ----------------------------------------------------------------------------------
+// (2)+(4) per (b, h, c): y for the chunk's tokens, in tiles of kTokTile tokens.
+//   y_t = sum_{s<=t} M[t][s] x_s + exp(Lam_t) H_c C_t + D x_t,
+//   M[t][s] = (C_t . B_s) exp(Lam_t - Lam_s) dt_s.
+// ----------------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+chunk_output_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
+                         const T* __restrict__ Bm, const T* __restrict__ Cm,
+                         const float* __restrict__ D, const float* __restrict__ lam,
+                         const float* __restrict__ states, T* __restrict__ y, int seqlen,
+                         int nheads, int headdim, int ngroups, int dstate, int Q, int nchunks)
+{
+    extern __shared__ float sm[];
+    float* sH = sm;                                    // [headdim][dstate + 1]
+    const int ldH = dstate + 1;
+    float* sC = sH + headdim * ldH;                    // [kTokTile][dstate + 1]
+    float* sB = sC + kTokTile * ldH;                   // [kTokTile][dstate + 1]
+    float* sX = sB + kTokTile * ldH;                   // [kTokTile][headdim]
+    float* sM = sX + kTokTile * headdim;               // [kTokTile][kTokTile + 1]
+    const int ldM = kTokTile + 1;
+    float* sLs = sM + kTokTile * ldM;                  // [kTokTile] Lam_s
+    float* sDs = sLs + kTokTile;                       // [kTokTile] dt_s
+
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int g = h / (nheads / ngroups);
+    const int t0 = c * Q;
+    const int qlen = min(Q, seqlen - t0);
+    const float* lamc = lam + (((size_t)b * nheads + h) * nchunks + c) * Q;
+    const float* Hc = states + (((size_t)b * nheads + h) * nchunks + c) * headdim * dstate;
+    const float Dh = D[h];
+    const size_t tok_stride_x = (size_t)nheads * headdim;
+    const size_t tok_stride_b = (size_t)ngroups * dstate;
+    const T* xbase = x + ((size_t)b * seqlen + t0) * tok_stride_x + (size_t)h * headdim;
+    T* ybase = y + ((size_t)b * seqlen + t0) * tok_stride_x + (size_t)h * headdim;
+    const T* Bbase = Bm + ((size_t)b * seqlen + t0) * tok_stride_b + (size_t)g * dstate;
+    const T* Cbase = Cm + ((size_t)b * seqlen + t0) * tok_stride_b + (size_t)g * dstate;
+
+    for (int i = threadIdx.x; i < headdim * dstate; i += kThreads) {
+        const int p = i / dstate, n = i - p * dstate;
+        sH[p * ldH + n] = Hc[i];
+    }
+
+    // output tile: kTokTile x headdim, each thread owns (t = tid / tpr, p = tid % tpr + k*tpr)
+    const int tpr = kThreads / kTokTile;               // threads per token row = 8
+    const int my_t = threadIdx.x / tpr, my_p0 = threadIdx.x % tpr;
+
+    for (int tt = 0; tt < qlen; tt += kTokTile) {
+        const int nt = min(kTokTile, qlen - tt);
+        __syncthreads();
+        for (int i = threadIdx.x; i < kTokTile * dstate; i += kThreads) {
+            const int t = i / dstate, n = i - t * dstate;
+            sC[t * ldH + n] = t < nt ? Elem<T>::load(Cbase + (size_t)(tt + t) * tok_stride_b + n) : 0.f;
+        }
+        __syncthreads();
+        // carried-state term and skip
+        float acc[16];
+        const int nper = (headdim + tpr - 1) / tpr;    // <= 16 for headdim <= 128
+        const float lt = (my_t < nt) ? lamc[tt + my_t] : 0.f;
+        const float et = expf(lt);
+        for (int k = 0; k < nper; ++k) {
+            const int p = my_p0 + k * tpr;
+            float v = 0.f;
+            if (p < headdim && my_t < nt) {
+                const float* hr = sH + p * ldH;
+                const float* cr = sC + my_t * ldH;
+                for (int n = 0; n < dstate; ++n) v = fmaf(cr[n], hr[n], v);
+                v *= et;
+            }
+            acc[k] = v;
+        }
+        // intra-chunk masked product, source tokens s <= t in tiles
+        for (int ss = 0; ss <= tt; ss += kTokTile) {
+            const int ns = min(kTokTile, qlen - ss);
+            __syncthreads();
+            for (int i = threadIdx.x; i < kTokTile * dstate; i += kThreads) {
+                const int s = i / dstate, n = i - s * dstate;
+                sB[s * ldH + n] = s < ns ? Elem<T>::load(Bbase + (size_t)(ss + s) * tok_stride_b + n) : 0.f;
+            }
+            for (int i = threadIdx.x; i < kTokTile * headdim; i += kThreads) {
+                const int s = i / headdim, p = i - s * headdim;
+                sX[i] = s < ns ? Elem<T>::load(xbase + (size_t)(ss + s) * tok_stride_x + p) : 0.f;
+            }
+            if (threadIdx.x < kTokTile) {
+                const int s = threadIdx.x;
+                sLs[s] = s < ns ? lamc[ss + s] : 0.f;
+                sDs[s] = s < ns ? dt[((size_t)b * seqlen + t0 + ss + s) * nheads + h] : 0.f;
+            }
+            __syncthreads();
+            // M tile: thread computes entries (t = i / kTokTile, s = i % kTokTile)
+            for (int i = threadIdx.x; i < kTokTile * kTokTile; i += kThreads) {
+                const int t = i / kTokTile, s = i - t * kTokTile;
+                float m = 0.f;
+                if (t < nt && s < ns && ss + s <= tt + t) {
+                    const float* cr = sC + t * ldH;
+                    const float* br = sB + s * ldH;
+                    float cb = 0.f;
+                    for (int n = 0; n < dstate; ++n) cb = fmaf(cr[n], br[n], cb);
+                    m = cb * expf(lamc[tt + t] - sLs[s]) * sDs[s];
+                }
+                sM[t * ldM + s] = m;
+            }
+            __syncthreads();
+            if (my_t < nt) {
+                for (int k = 0; k < nper; ++k) {
+                    const int p = my_p0 + k * tpr;
+                    if (p < headdim) {
+                        float v = acc[k];
+                        for (int s = 0; s < ns; ++s) v = fmaf(sM[my_t * ldM + s], sX[s * headdim + p], v);
+                        acc[k] = v;
+                    }
+                }
+            }
+        }
+        if (my_t < nt) {
+            const T* xr = xbase + (size_t)(tt + my_t) * tok_stride_x;
+            T* yr = ybase + (size_t)(tt + my_t) * tok_stride_x;
+            for (int k = 0; k < nper; ++k) {
+                const int p = my_p0 + k * tpr;
+                if (p < headdim) Elem<T>::store(yr + p, fmaf(Dh, Elem<T>::load(xr + p), acc[k]));
+            }
+        }
+    }
+}
+
+// zero-length prefill: final = init (or zeros)
+__global__ void copy_state_kernel(const float* init_state, float* final_state, size_t n)
+{
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) final_state[i] = init_state ? init_state[i] : 0.f;
+}
+
+template <typename T>
+cudaError_t chunk_state_simt_t(const Dims& d, const void* x, const float* dt, const void* B,
+                               const float* lam, float* states, cudaStream_t s)
+{
+    const size_t smem = sizeof(float) * (kTokTile * (d.headdim + d.dstate) + kTokTile);
+    auto k = chunk_state_simt_kernel<T>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(d.nchunks, d.nheads, d.batch);
+    k<<<grid, kThreads, smem, s>>>(static_cast<const T*>(x), dt, static_cast<const T*>(B), lam,
+                                   states, d.seqlen, d.nheads, d.headdim, d.ngroups, d.dstate,
+                                   d.chunk_len, d.nchunks);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t chunk_output_simt_t(const Dims& d, const void* x, const float* dt, const void* B,
+                                const void* C, const float* D, const float* lam,
+                                const float* states, void* y, cudaStream_t s)
+{
+    const int ldH = d.dstate + 1;
+    const size_t smem = sizeof(float) * ((size_t)d.headdim * ldH + 2 * kTokTile * ldH +
+                                         kTokTile * d.headdim + kTokTile * (kTokTile + 1) +
+                                         2 * kTokTile);
+    auto k = chunk_output_simt_kernel<T>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(d.nchunks, d.nheads, d.batch);
+    k<<<grid, kThreads, smem, s>>>(static_cast<const T*>(x), dt, static_cast<const T*>(B),
+                                   static_cast<const T*>(C), D, lam, states, static_cast<T*>(y),
+                                   d.seqlen, d.nheads, d.headdim, d.ngroups, d.dstate,
+                                   d.chunk_len, d.nchunks);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t simt_output_smem_bytes(int headdim, int dstate)
+{
+    const int ldH = dstate + 1;
+    return sizeof(float) * ((size_t)headdim * ldH + 2 * kTokTile * ldH + kTokTile * headdim +
+                            kTokTile * (kTokTile + 1) + 2 * kTokTile);
+}
+
+cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, float* lam,
+                                cudaStream_t s)
+{
+    if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
+    const size_t smem = sizeof(float) * d.chunk_len * kCumsumHeads;
+    cudaError_t e = cudaFuncSetAttribute(chunk_cumsum_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(d.nchunks, (d.nheads + kCumsumHeads - 1) / kCumsumHeads, d.batch);
+    chunk_cumsum_kernel<<<grid, kThreads, smem, s>>>(dt, A, lam, d.seqlen, d.nheads, d.chunk_len,
+                                                     d.nchunks);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_state_simt(const Dims& d, ssd_dtype_t dtype, const void* x,
+                                    const float* dt, const void* B, const float* lam,
+                                    float* states, cudaStream_t s)
+{
+    if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
+    if (dtype == SSD_F32) return chunk_state_simt_t<float>(d, x, dt, B, lam, states, s);
+    return chunk_state_simt_t<__nv_bfloat16>(d, x, dt, B, lam, states, s);
+}
+
+cudaError_t launch_state_scan(const Dims& d, const float* lam, float* states,
+                              const float* init_state, float* final_state, cudaStream_t s)
+{
+    if (d.batch == 0) return cudaSuccess;
+    const int PN = d.headdim * d.dstate;
+    dim3 grid((PN / 4 + kThreads - 1) / kThreads, d.batch * d.nheads);
+    state_scan_kernel<<<grid, kThreads, 0, s>>>(lam, states, init_state, final_state, d.nheads,
+                                                PN, d.chunk_len, d.nchunks);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_output_simt(const Dims& d, ssd_dtype_t dtype, const void* x,
+                                     const float* dt, const void* B, const void* C,
+                                     const float* D, const float* lam, const float* states,
+                                     void* y, cudaStream_t s)
+{
+    if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
+    if (dtype == SSD_F32) return chunk_output_simt_t<float>(d, x, dt, B, C, D, lam, states, y, s);
+    return chunk_output_simt_t<__nv_bfloat16>(d, x, dt, B, C, D, lam, states, y, s);
+}
+
+cudaError_t launch_copy_state(const Dims& d, const float* init_state, float* final_state,
+                              cudaStream_t s)
+{
+    const size_t n = (size_t)d.batch * d.nheads * d.headdim * d.dstate;
+    if (n == 0) return cudaSuccess;
+    copy_state_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(init_state, final_state, n);
+    return cudaGetLastError();
+}
+
+}  // namespace ssd

@@ -1,0 +1,121 @@
+"""C ABI checks that need no GPU: the library loads, exports every function that
+include/ssd.h declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from state_space_model_05_b200 import binding
+from state_space_model_05_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssd.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssd_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_function(lib):
+    names = declared_functions()
+    assert "ssd_prefill" in names and "ssd_decode_step" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in ssd.h but not exported"
+    assert set(names) == set(binding.SIGNATURES), "binding signatures out of sync with ssd.h"
+
+
+def test_status_strings(lib):
+    for code in range(0, 9):
+        s = lib.ssd_status_string(code)
+        assert s and s.decode() != "unknown status"
+    assert lib.ssd_status_string(99).decode() == "unknown status"
+    assert lib.ssd_abi_version() == 100
+
+
+def _ws(*a):
+    return binding.ssd_prefill_workspace_bytes(*a)
+
+
+def test_workspace_bytes(lib):
+    # lam [b][H][c][Q] + states [b][H][c][P][N], each rounded up to 256 bytes
+    b, T, H, P, G, N, Q = 2, 300, 4, 64, 1, 128, 128
+    c = 3
+    lam = b * H * c * Q * 4
+    st = b * H * c * P * N * 4
+    up = lambda v: (v + 255) // 256 * 256
+    assert _ws(b, T, H, P, G, N, Q, binding.SSD_BF16) == up(lam) + up(st)
+    assert _ws(b, 0, H, P, G, N, Q, binding.SSD_F32) == 0
+    assert _ws(b, T, H, 63, G, N, Q, binding.SSD_F32) == 0          # headdim not a multiple of 8
+    assert _ws(b, T, 3, P, 2, N, Q, binding.SSD_F32) == 0           # nheads % ngroups
+    assert _ws(b, T, H, P, G, N, 0, binding.SSD_F32) == 0
+    assert _ws(b, T, H, P, G, N, Q, 7) == 0                         # bad dtype
+
+
+FAKE = 0x10000  # 16-byte aligned dummy address; never dereferenced (calls fail validation first)
+
+
+def _prefill(lib, **kw):
+    a = dict(x=FAKE, dt=FAKE, A=FAKE, B=FAKE, C=FAKE, D=FAKE, init=None, batch=1, seqlen=16,
+             nheads=2, headdim=64, ngroups=1, dstate=128, chunk_len=16, dtype=binding.SSD_F32,
+             y=FAKE, final=FAKE, ws=FAKE, ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return lib.ssd_prefill(a["x"], a["dt"], a["A"], a["B"], a["C"], a["D"], a["init"], a["batch"],
+                           a["seqlen"], a["nheads"], a["headdim"], a["ngroups"], a["dstate"],
+                           a["chunk_len"], a["dtype"], a["y"], a["final"], a["ws"], a["ws_bytes"],
+                           a["stream"])
+
+
+def test_prefill_validation(lib):
+    E = binding
+    assert _prefill(lib, nheads=3, ngroups=2) == 2
+    assert _prefill(lib, headdim=12) == 2
+    assert _prefill(lib, dstate=0) == 2
+    assert _prefill(lib, seqlen=-1) == 2
+    assert _prefill(lib, chunk_len=0) == 2
+    assert _prefill(lib, chunk_len=512) == 5
+    assert _prefill(lib, headdim=256) == 5
+    assert _prefill(lib, dtype=5) == 3
+    assert _prefill(lib, x=None) == 1
+    assert _prefill(lib, final=None) == 1
+    assert _prefill(lib, y=FAKE + 4) == 4
+    assert _prefill(lib, init=FAKE + 8) == 4
+    assert _prefill(lib, ws_bytes=16) == 8
+    assert _prefill(lib, ws=None) == 8
+    assert _prefill(lib, batch=0) == 0          # nothing to do, nothing launched
+
+
+def _decode(lib, **kw):
+    a = dict(state=FAKE, x=FAKE, dt=FAKE, A=FAKE, B=FAKE, C=FAKE, D=FAKE, batch=2, nheads=4,
+             headdim=64, ngroups=1, dstate=128, dtype=binding.SSD_F32, y=FAKE, stream=None)
+    a.update(kw)
+    return lib.ssd_decode_step(a["state"], a["x"], a["dt"], a["A"], a["B"], a["C"], a["D"],
+                               a["batch"], a["nheads"], a["headdim"], a["ngroups"], a["dstate"],
+                               a["dtype"], a["y"], a["stream"])
+
+
+def test_decode_validation(lib):
+    assert _decode(lib, nheads=5, ngroups=2) == 2
+    assert _decode(lib, dstate=1024) == 5
+    assert _decode(lib, dstate=20) == 2
+    assert _decode(lib, state=None) == 1
+    assert _decode(lib, y=None) == 1
+    assert _decode(lib, B=FAKE + 2) == 4
+    assert _decode(lib, dtype=9) == 3
+    assert _decode(lib, batch=-1) == 2
+    assert _decode(lib, batch=0) == 0
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(binding, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        binding.lib()

@@ -1,0 +1,167 @@
+"""GPU parity of ssd_prefill against the fp64 oracle on seeded inputs.
+
+Workloads: the fp32 single SSD layer (batch 1, 256 tokens, 4 heads, P = N = 64,
+chunk 64), the Mamba-2-130M-shaped bf16 layer (batch 8, 2048 tokens, 24 heads,
+P 64, N 128, chunk 256) and the 2.7B-shaped long bf16 prefill (batch 4, 16384
+tokens, 80 heads, chunk 256; sampled (batch, head) units), plus ragged, empty,
+grouped, init-state and chunk-length cases.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import (assert_bf16_y, assert_fp32, assert_state, gpu_prefill, gpu_units,
+                    oracle_prefill, problem, to_dev)
+from state_space_model_05_b200 import inputs as gen
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _built():
+    from state_space_model_05_b200.build import build
+    build()
+    oracle.build()
+
+
+def _check_fp32(inp, Q, init=None):
+    b, T, H, P = inp.x.shape
+    y, st = gpu_prefill(inp, Q, bf16=False, init=init)
+    yo, so = oracle_prefill(inp, init=None if init is None else init.reshape(b * H, P, -1))
+    assert_fp32(y, oracle.units_to_bthp(yo, b, H), f"y Q={Q}")
+    assert_fp32(st, so.reshape(st.shape), f"state Q={Q}")
+    return y, st
+
+
+def _check_bf16(inp, Q, init=None):
+    b, T, H, P = inp.x.shape
+    y, st = gpu_prefill(inp, Q, bf16=True, init=init)
+    yo, so = oracle_prefill(inp, init=None if init is None else init.reshape(b * H, P, -1))
+    assert_bf16_y(y, oracle.units_to_bthp(yo, b, H), f"y Q={Q}")
+    assert_state(st, so.reshape(st.shape), f"state Q={Q}")
+    return y, st
+
+
+# --------------------------------------------------------------------- fp32 path
+def test_fp32_single_layer_workload():
+    """fp32 single layer: b=1, T=256, H=4, P=N=64, G=1, chunk 64, seed 0."""
+    inp = problem(gen.SSDShape(1, 256, 4, 64, 1, 64), bf16=False, seed=0)
+    _check_fp32(inp, 64)
+
+
+@pytest.mark.parametrize("T,Q", [(1, 64), (63, 64), (200, 64), (300, 128), (257, 256), (100, 1),
+                                 (100, 7), (130, 33)])
+def test_fp32_ragged_and_chunk_lengths(T, Q):
+    inp = problem(gen.SSDShape(2, T, 4, 64, 2, 64), bf16=False, seed=T + Q)
+    _check_fp32(inp, Q)
+
+
+def test_fp32_chunk_length_invariance():
+    inp = problem(gen.SSDShape(1, 320, 2, 32, 1, 128), bf16=False, seed=5)
+    ys = [gpu_prefill(inp, Q, bf16=False)[0] for Q in (16, 64, 100, 256)]
+    for y in ys[1:]:
+        assert_fp32(y, ys[0], "chunk invariance")
+    _check_fp32(inp, 64)
+
+
+def test_fp32_odd_dims_and_groups():
+    inp = problem(gen.SSDShape(3, 150, 6, 24, 3, 40), bf16=False, seed=9)
+    _check_fp32(inp, 32)
+
+
+def test_fp32_init_state_and_resume():
+    rng = np.random.default_rng(3)
+    inp = problem(gen.SSDShape(2, 272, 4, 64, 1, 64), bf16=False, seed=11)
+    init = (rng.standard_normal((2, 4, 64, 64)) * 0.1).astype(np.float32)
+    _check_fp32(inp, 64, init=init)
+    # prefill(T1) then prefill(T2, init = final of the first) == prefill(T1 + T2)
+    from state_space_model_05_b200 import ssd_prefill
+    dev = lambda a: to_dev(a)
+    y_full, s_full = ssd_prefill(dev(inp.x), dev(inp.dt), dev(inp.A), dev(inp.B), dev(inp.C), dev(inp.D), 64)
+    T1 = 100
+    y1, s1 = ssd_prefill(dev(inp.x[:, :T1]), dev(inp.dt[:, :T1]), dev(inp.A), dev(inp.B[:, :T1]),
+                         dev(inp.C[:, :T1]), dev(inp.D), 64)
+    y2, s2 = ssd_prefill(dev(inp.x[:, T1:]), dev(inp.dt[:, T1:]), dev(inp.A), dev(inp.B[:, T1:]),
+                         dev(inp.C[:, T1:]), dev(inp.D), 64, init_state=s1)
+    assert_fp32(torch.cat([y1, y2], 1).cpu().numpy(), y_full.cpu().numpy(), "split prefill y")
+    assert_fp32(s2.cpu().numpy(), s_full.cpu().numpy(), "split prefill state")
+
+
+def test_fp32_init_aliases_final():
+    rng = np.random.default_rng(4)
+    inp = problem(gen.SSDShape(1, 90, 2, 16, 1, 32), bf16=False, seed=12)
+    init = rng.standard_normal((1, 2, 16, 32)).astype(np.float32)
+    from state_space_model_05_b200 import ssd_prefill
+    st = to_dev(init)
+    y, st2 = ssd_prefill(to_dev(inp.x), to_dev(inp.dt), to_dev(inp.A), to_dev(inp.B), to_dev(inp.C),
+                         to_dev(inp.D), 32, init_state=st, final_state=st)
+    assert st2.data_ptr() == st.data_ptr()
+    yo, so = oracle_prefill(inp, init=init.reshape(2, 16, 32))
+    assert_fp32(st.cpu().numpy(), so.reshape(1, 2, 16, 32), "aliased state")
+
+
+def test_empty_sequence_copies_init():
+    from state_space_model_05_b200 import ssd_prefill
+    rng = np.random.default_rng(5)
+    init = to_dev(rng.standard_normal((2, 3, 8, 16)).astype(np.float32))
+    x = torch.empty((2, 0, 3, 8), device="cuda")
+    dt = torch.empty((2, 0, 3), device="cuda")
+    B = torch.empty((2, 0, 1, 16), device="cuda")
+    A = -torch.ones(3, device="cuda")
+    D = torch.ones(3, device="cuda")
+    y, st = ssd_prefill(x, dt, A, B, B, D, 16, init_state=init)
+    assert y.shape == (2, 0, 3, 8)
+    assert torch.equal(st, init)
+    _, st0 = ssd_prefill(x, dt, A, B, B, D, 16)
+    assert torch.count_nonzero(st0) == 0
+
+
+# --------------------------------------------------------------------- bf16 path
+def test_bf16_130m_layer_full():
+    """130M-shaped layer: b=8, T=2048, H=24, P=64, N=128, G=1, chunk 256, all outputs."""
+    inp = problem(gen.SSDShape(8, 2048, 24, 64, 1, 128), bf16=True, seed=0)
+    _check_bf16(inp, 256)
+
+
+@pytest.mark.parametrize("T,Q,G", [(1000, 256, 2), (300, 128, 1), (129, 128, 4), (1, 256, 1),
+                                   (512, 64, 1), (700, 100, 1)])
+def test_bf16_ragged_groups_chunks(T, Q, G):
+    """Tensor-core path (Q 128/256, partial last chunk, G > 1) and the SIMT path (other Q)."""
+    inp = problem(gen.SSDShape(2, T, 4, 64, G, 128), bf16=True, seed=T + Q + G)
+    _check_bf16(inp, Q)
+
+
+def test_bf16_init_state():
+    rng = np.random.default_rng(6)
+    inp = problem(gen.SSDShape(2, 600, 4, 64, 1, 128), bf16=True, seed=21)
+    init = (rng.standard_normal((2, 4, 64, 128)) * 0.05).astype(np.float32)
+    _check_bf16(inp, 256, init=init)
+
+
+def test_bf16_chunk_length_invariance():
+    inp = problem(gen.SSDShape(1, 1024, 8, 64, 1, 128), bf16=True, seed=22)
+    b, T, H, P = inp.x.shape
+    yo, so = oracle_prefill(inp)
+    for Q in (128, 256, 64):
+        y, st = gpu_prefill(inp, Q, bf16=True)
+        assert_bf16_y(y, oracle.units_to_bthp(yo, b, H), f"Q={Q}")
+        assert_state(st, so.reshape(st.shape), f"Q={Q}")
+
+
+def test_bf16_27b_long_prefill_sampled():
+    """2.7B-shaped long prefill (b=4, T=16384, H=80, P=64, N=128, chunk 256) at full size,
+    checked on sampled (batch, head) units: all tokens of y and the final state."""
+    inp = problem(gen.SSDShape(4, 16384, 80, 64, 1, 128), bf16=True, seed=0)
+    y, st = gpu_prefill(inp, 256, bf16=True)
+    rng = np.random.default_rng(0)
+    units = sorted(rng.choice(4 * 80, size=8, replace=False).tolist())
+    yo, so = oracle_prefill(inp, units=units)
+    assert_bf16_y(gpu_units(y, units, 80), yo, "y sampled")
+    assert_state(st.reshape(4 * 80, 64, 128)[units], so, "state sampled")
+    assert np.isfinite(y).all() and np.isfinite(st).all()
+
+
+def test_device_status_clean():
+    from state_space_model_05_b200 import ssd_device_status
+    assert ssd_device_status() == 0
