@@ -326,14 +326,19 @@ def run_decode(w, repeats, warmup, rank, world):
         for k in range(4):                           # eager warm-up before capture
             ssd.ssd_decode_step(state, X[k], DT[k], A, Bs[k], Cs[k], D, y_t=y)
     torch.cuda.synchronize()
-    binding.ssd_profile_reset()
-    binding.ssd_profile_enable(True)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(side):
-        with torch.cuda.graph(g, stream=side):
-            for k in range(S):
-                ssd.ssd_decode_step(state, X[k], DT[k], A, Bs[k], Cs[k], D, y_t=y)
-    binding.ssd_profile_enable(False)
+
+    def capture(profile: bool):
+        binding.ssd_profile_reset()
+        binding.ssd_profile_enable(profile)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                for k in range(S):
+                    ssd.ssd_decode_step(state, X[k], DT[k], A, Bs[k], Cs[k], D, y_t=y)
+        binding.ssd_profile_enable(False)
+        return graph
+
+    g = capture(False)                               # the timed loop: 1024 launches, no events
     for _ in range(warmup):
         g.replay()
     torch.cuda.synchronize()
@@ -346,8 +351,11 @@ def run_decode(w, repeats, warmup, rank, world):
     s1.record()
     torch.cuda.synchronize()
     barrier(world)
-    kernels = binding.ssd_profile_read()              # events of the latest replay
     ms = reduce_max(s0.elapsed_time(s1), world)
+    gp = capture(True)                               # same loop with an event pair per launch
+    gp.replay()
+    torch.cuda.synchronize()
+    kernels = binding.ssd_profile_read()
     status = ssd.ssd_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after decode")
@@ -357,7 +365,7 @@ def run_decode(w, repeats, warmup, rank, world):
     res = {"steps_per_s": steps_total * world / (ms / 1e3), "ms_per_step": ms / steps_total,
            "gbs": nbytes * steps_total / (ms / 1e3) / 1e9, "kernel_ms": kms / max(klaunch, 1),
            "launches": steps_total, "bytes_per_step": nbytes}
-    del g
+    del g, gp
     return res
 
 

@@ -93,9 +93,14 @@ cudaError_t profiled(int stage, cudaStream_t s, F&& launch)
 {
     if (!g_prof.on) return launch();
     cudaEvent_t a = g_prof.next(), b = g_prof.next();
-    if (a) cudaEventRecord(a, s);
+    // inside a stream capture an event record must be marked external to become a
+    // timed record node of the graph (otherwise it is only a dependency marker)
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(s, &cap);
+    const unsigned flags = cap == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : 0u;
+    if (a) cudaEventRecordWithFlags(a, s, flags);
     const cudaError_t e = launch();
-    if (b) cudaEventRecord(b, s);
+    if (b) cudaEventRecordWithFlags(b, s, flags);
     if (a && b) g_prof.records.push_back({stage, a, b});
     return e;
 }

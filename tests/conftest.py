@@ -21,3 +21,16 @@ def oracle_mod():
 TESTS = os.path.dirname(os.path.abspath(__file__))
 if TESTS not in sys.path:
     sys.path.insert(0, TESTS)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    path = os.environ.get("PARITY_REPORT")
+    if not path:
+        return
+    try:
+        import json
+        import parity
+        with open(path, "w") as f:
+            json.dump(parity.REPORT, f, indent=1)
+    except Exception:  # noqa: BLE001 - reporting must not change the test outcome
+        pass

@@ -21,6 +21,15 @@ from state_space_model_05_b200 import inputs as gen
 FP32_TOL = 1e-4
 BF16_TOL = 2e-2
 
+# every measured error, written to $PARITY_REPORT at the end of the session (conftest)
+REPORT = []
+
+
+def _record(kind, what, **vals):
+    import os
+    REPORT.append({"test": os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0], "check": kind,
+                   "what": what, **{k: float(v) for k, v in vals.items()}})
+
 
 def rms(o):
     return float(np.sqrt(np.mean(np.square(o)))) if o.size else 0.0
@@ -46,6 +55,7 @@ def fp32_errors(g, o):
 
 def assert_fp32(g, o, what="", tol=FP32_TOL):
     rel, nrm = fp32_errors(g, o)
+    _record("fp32", what, max_rel=rel, max_over_rms=nrm, tol=tol)
     assert rel <= tol and nrm <= tol, f"{what}: max rel {rel:.3e}, max/RMS {nrm:.3e} (tol {tol})"
     return rel, nrm
 
@@ -61,6 +71,7 @@ def bf16_y_error(g, o):
 
 def assert_bf16_y(g, o, what="", tol=BF16_TOL):
     ex, raw = bf16_y_error(g, o)
+    _record("bf16_y", what, excess_over_rms=ex, raw_over_rms=raw, tol=tol)
     assert ex <= tol, f"{what}: max excess/RMS {ex:.3e} (raw {raw:.3e}, tol {tol})"
     return ex, raw
 
@@ -69,6 +80,7 @@ def assert_state(g, o, what="", tol=BF16_TOL):
     g = np.asarray(g, dtype=np.float64)
     o = np.asarray(o, dtype=np.float64)
     e = float(np.abs(g - o).max() / rms(o))
+    _record("state", what, max_over_rms=e, tol=tol)
     assert e <= tol, f"{what}: max/RMS {e:.3e} (tol {tol})"
     return e
 
