@@ -119,6 +119,29 @@ ssd_status_t ssd_decode_step(float* state, const void* x_t, const float* dt_t, c
                              void* y_t, void* stream);
 
 /*
+ * ssd_prefill without a workspace argument, for callers that may not allocate
+ * device memory (a host framework's execution hook that must stay inside the
+ * memory it planned, or code running during a CUDA stream capture, where
+ * cudaMalloc would break the capture).  The paper has no counterpart to this
+ * entry point; it is a deployment convenience.
+ *
+ * The workspace comes from a 64 MiB buffer built into the library's device
+ * image (held by every GPU that loads the library until the process exits).
+ * Sizes whose ssd_prefill_workspace_bytes exceeds 64 MiB return
+ * SSD_ERR_WORKSPACE before anything is launched.  The first call on a device
+ * looks up the buffer's device address (with that device current); make that
+ * first call before any stream capture.  All calls share the one buffer:
+ * calls that overlap on the GPU (e.g. on two streams) race and must be
+ * serialised by the caller.  Nothing needs clearing between calls.
+ * Everything else is as for ssd_prefill.
+ */
+ssd_status_t ssd_prefill_noalloc(const void* x, const float* dt, const float* A, const void* B,
+                                 const void* C, const float* D, const float* init_state,
+                                 int batch, int seqlen, int nheads, int headdim, int ngroups,
+                                 int dstate, int chunk_len, ssd_dtype_t dtype, void* y,
+                                 float* final_state, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears this device's error word.
  * Returns SSD_OK, SSD_ERR_TIMEOUT (a bounded wait expired in a kernel since
  * the last call), or SSD_ERR_CUDA when the stream reports a CUDA error.

@@ -32,6 +32,7 @@ SIGNATURES = {
     "ssd_prefill_workspace_bytes": ([_I, _I, _I, _I, _I, _I, _I, _I], _Z),
     "ssd_prefill": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _Z, _P], _I),
     "ssd_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
+    "ssd_prefill_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P], _I),
     "ssd_device_status": ([_P], _I),
     "ssd_profile_enable": ([_I], None),
     "ssd_profile_reset": ([], None),

@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libssd.so")
 
-SOURCES = ["api.cu", "decode.cu", "prefill_simt.cu", "prefill_tc.cu"]
+SOURCES = ["api.cu", "decode.cu", "prefill_simt.cu", "prefill_tc.cu", "prefill_noalloc.cu"]
 HEADERS = ["common.cuh", "ptx.cuh", "prefill_tc.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
