@@ -62,13 +62,16 @@ def prefill_flops(w) -> dict:
 
 
 def prefill_bytes(w) -> dict:
+    """Algorithmic bytes per call: whole path, and per kernel of the tensor-core path."""
     b, T, H, P, G, N, Q = (w[k] for k in ("batch", "seqlen", "nheads", "headdim", "ngroups", "dstate", "chunk_len"))
     e = 2 if w["dtype"] == "bf16" else 4
     c = -(-T // Q)
     io = b * T * (2 * H * P * e + 2 * G * N * e + H * 4) + b * H * P * N * 4
     return {"total": io,
+            # x and B in, dt/Lam in, one bf16 start-state image per (b, h, chunk) out, final state out
+            "chunk_state_scan_tc": b * T * (H * P * e + G * N * e + 2 * H * 4) + b * H * c * P * N * 2 + b * H * P * N * 4,
             "state_scan": 2 * b * H * c * P * N * 4 + b * H * P * N * 4,
-            "chunk_cumsum": b * T * H * 4 + b * H * c * Q * 4}
+            "chunk_cumsum": b * T * H * 4 + 2 * b * H * c * Q * 4}
 
 
 def decode_bytes(w) -> int:
@@ -376,7 +379,7 @@ def roofline_prefill(w, res, peaks, src, workload):
     dom = max(kernels, key=lambda k: kernels[k][0])
     ms, n = kernels[dom]
     per_launch_ms = ms / n
-    if dom.startswith("chunk_output") or dom.startswith("chunk_state"):
+    if dom.startswith("chunk_output") or dom == "chunk_state_simt":
         work = flops["chunk_output" if dom.startswith("chunk_output") else "chunk_state"]
         achieved = work / (per_launch_ms / 1e3) / 1e12
         peak = peaks["bf16_tflops"]

@@ -67,7 +67,7 @@ ssd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_E
 
 // ---- opt-in kernel profiling: an event pair around each launch -------------------
 enum Stage { kCumsum, kStateTc, kStateSimt, kScan, kOutTc, kOutSimt, kDecode, kCopy, kNumStages };
-const char* const kStageNames[kNumStages] = {"chunk_cumsum", "chunk_state_tc", "chunk_state_simt",
+const char* const kStageNames[kNumStages] = {"chunk_cumsum", "chunk_state_scan_tc", "chunk_state_simt",
                                               "state_scan", "chunk_output_tc", "chunk_output_simt",
                                               "decode_step", "copy_state"};
 struct ProfRecord { int stage; cudaEvent_t begin, end; };
@@ -150,6 +150,8 @@ size_t ssd_prefill_workspace_bytes(int batch, int seqlen, int nheads, int headdi
     Dims d;
     if (prefill_dims(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len, dtype, &d) != SSD_OK)
         return 0;
+    if (d.nchunks == 0 || d.batch == 0) return 0;
+    if (dtype == SSD_BF16 && tc_prefill_supported(d)) return tc_workspace_layout(d, nullptr, nullptr);
     return prefill_workspace_layout(d, nullptr, nullptr);
 }
 
@@ -174,30 +176,42 @@ ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const v
     if (!aligned16(x) || !aligned16(dt) || !aligned16(A) || !aligned16(B) || !aligned16(C) ||
         !aligned16(D) || !aligned16(y) || !aligned16(workspace))
         return SSD_ERR_ALIGN;
+    const bool tc = dtype == SSD_BF16 && tc_prefill_supported(d);
+    if (tc) {
+        TcWorkspace w;
+        const size_t need = tc_workspace_layout(d, workspace, &w);
+        if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
+        const int nflags = d.batch * d.nheads + 1;
+        cudaError_t e = profiled(kCumsum, s, [&] {
+            return launch_chunk_cumsum(d, dt, A, w.lam, w.dtT, w.flags, nflags, s);
+        });
+        if (e == cudaSuccess)
+            e = profiled(kStateTc, s, [&] {
+                return launch_chunk_state_scan_tc(d, x, B, w, init_state, final_state, s);
+            });
+        if (e == cudaSuccess)
+            e = profiled(kOutTc, s, [&] { return launch_chunk_output_tc(d, x, B, C, D, w, y, s); });
+        return from_cuda(e);
+    }
+
     PrefillWorkspace ws;
     const size_t need = prefill_workspace_layout(d, workspace, &ws);
     if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
-
-    const bool tc = dtype == SSD_BF16 && tc_prefill_supported(d);
-    cudaError_t e = profiled(kCumsum, s, [&] { return launch_chunk_cumsum(d, dt, A, ws.lam, s); });
-    if (e == cudaSuccess) {
-        e = tc ? profiled(kStateTc, s, [&] { return launch_chunk_state_tc(d, x, dt, B, ws.lam, ws.states, s); })
-               : profiled(kStateSimt, s, [&] {
-                     return launch_chunk_state_simt(d, dtype, x, dt, B, ws.lam, ws.states, s);
-                 });
-    }
+    cudaError_t e = profiled(kCumsum, s, [&] {
+        return launch_chunk_cumsum(d, dt, A, ws.lam, nullptr, nullptr, 0, s);
+    });
+    if (e == cudaSuccess)
+        e = profiled(kStateSimt, s, [&] {
+            return launch_chunk_state_simt(d, dtype, x, dt, B, ws.lam, ws.states, s);
+        });
     if (e == cudaSuccess)
         e = profiled(kScan, s, [&] {
             return launch_state_scan(d, ws.lam, ws.states, init_state, final_state, s);
         });
-    if (e == cudaSuccess) {
-        e = tc ? profiled(kOutTc, s, [&] {
-                     return launch_chunk_output_tc(d, x, dt, B, C, D, ws.lam, ws.states, y, s);
-                 })
-               : profiled(kOutSimt, s, [&] {
-                     return launch_chunk_output_simt(d, dtype, x, dt, B, C, D, ws.lam, ws.states, y, s);
-                 });
-    }
+    if (e == cudaSuccess)
+        e = profiled(kOutSimt, s, [&] {
+            return launch_chunk_output_simt(d, dtype, x, dt, B, C, D, ws.lam, ws.states, y, s);
+        });
     return from_cuda(e);
 }
 

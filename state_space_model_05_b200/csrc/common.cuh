@@ -49,7 +49,7 @@ struct Dims {
     int batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len, nchunks;
 };
 
-// Workspace layout of the chunked prefill (byte offsets from the workspace base).
+// Workspace layout of the CUDA-core chunked prefill (offsets from the workspace base).
 struct PrefillWorkspace {
     float* lam;      // [batch][nheads][nchunks][chunk_len]   inclusive cumsum of dt*A
     float* states;   // [batch][nheads][nchunks][headdim][dstate]
@@ -62,7 +62,7 @@ cudaError_t launch_decode(const Dims& d, ssd_dtype_t dtype, float* state, const 
                           const float* D, void* y, cudaStream_t s);
 
 cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, float* lam,
-                                cudaStream_t s);
+                                float* dtT, int* zero, int nzero, cudaStream_t s);
 cudaError_t launch_chunk_state_simt(const Dims& d, ssd_dtype_t dtype, const void* x,
                                     const float* dt, const void* B, const float* lam,
                                     float* states, cudaStream_t s);

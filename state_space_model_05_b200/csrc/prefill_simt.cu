@@ -28,14 +28,19 @@ constexpr int kThreads = 256;
 // The chunk's dt block [Q][nheads] is contiguous in memory; it is staged through
 // shared memory so that both the read and the write are coalesced.
 // ----------------------------------------------------------------------------------
-constexpr int kCumsumHeads = 32;
+constexpr int kCumsumHeads = 8;      // one warp per head
 
+// Also writes dt transposed to [b][h][c][Q] when dtT is non-null (zero past seqlen),
+// and zeroes `nzero` words at `zero` (look-back flags of the tensor-core path).
 __global__ void __launch_bounds__(kThreads)
 chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
-                    float* __restrict__ lam, int seqlen, int nheads, int Q, int nchunks)
+                    float* __restrict__ lam, float* __restrict__ dtT, int* __restrict__ zero,
+                    int nzero, int seqlen, int nheads, int Q, int nchunks)
 {
     extern __shared__ float sm_dt[];                   // [Q][kCumsumHeads]
     const int c = blockIdx.x, h0 = blockIdx.y * kCumsumHeads, b = blockIdx.z;
+    if (zero && c == 0 && blockIdx.y == 0 && b == 0)
+        for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
     const int nh = min(kCumsumHeads, nheads - h0);
     const int t0 = c * Q;
     for (int i = threadIdx.x; i < Q * kCumsumHeads; i += blockDim.x) {
@@ -46,20 +51,25 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
     }
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int hh = warp; hh < nh; hh += kThreads / 32) {
+    if (warp < nh) {
+        const int hh = warp;
         const float Ah = A[h0 + hh];
         float carry = 0.f;
-        float* out = lam + (((size_t)b * nheads + h0 + hh) * nchunks + c) * Q;
+        const size_t row = (((size_t)b * nheads + h0 + hh) * nchunks + c) * Q;
         for (int base = 0; base < Q; base += 32) {
             const int t = base + lane;
-            float v = (t < Q) ? sm_dt[t * kCumsumHeads + hh] * Ah : 0.f;
+            const float d = (t < Q) ? sm_dt[t * kCumsumHeads + hh] : 0.f;
+            float v = d * Ah;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float u = __shfl_up_sync(0xffffffffu, v, o);
                 if (lane >= o) v += u;
             }
             v += carry;
-            if (t < Q) out[t] = v;
+            if (t < Q) {
+                lam[row + t] = v;
+                if (dtT) dtT[row + t] = d;
+            }
             carry = __shfl_sync(0xffffffffu, v, 31);
         }
     }
@@ -353,16 +363,13 @@ size_t simt_output_smem_bytes(int headdim, int dstate)
 }
 
 cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, float* lam,
-                                cudaStream_t s)
+                                float* dtT, int* zero, int nzero, cudaStream_t s)
 {
     if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
     const size_t smem = sizeof(float) * d.chunk_len * kCumsumHeads;
-    cudaError_t e = cudaFuncSetAttribute(chunk_cumsum_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     dim3 grid(d.nchunks, (d.nheads + kCumsumHeads - 1) / kCumsumHeads, d.batch);
-    chunk_cumsum_kernel<<<grid, kThreads, smem, s>>>(dt, A, lam, d.seqlen, d.nheads, d.chunk_len,
-                                                     d.nchunks);
+    chunk_cumsum_kernel<<<grid, kThreads, smem, s>>>(dt, A, lam, dtT, zero, nzero, d.seqlen,
+                                                     d.nheads, d.chunk_len, d.nchunks);
     return cudaGetLastError();
 }
 

@@ -1,26 +1,36 @@
 // Tensor-core stages of the bf16 chunked SSD prefill on sm_100a: tcgen05.mma with
 // TMEM accumulators, operands staged in shared memory by TMA (128-byte swizzle).
 //
-// "Compiler-First State Space Duality and Portable O(1) Autoregressive Caching
-// for Inference", section "2. Metodologia": the SSD layer is dominated by matrix
-// contractions (einsums) inside fixed-size chunks, masked by a static
-// lower-triangular decay mask whose exponents are taken in fp32.  On B200 those
-// contractions run on the 5th-generation tensor cores (bf16 in, fp32 accumulate):
+// "Compiler-First State Space Duality and Portable O(1) Autoregressive Caching for
+// Inference", section "2. Metodologia": the SSD layer is dominated by matrix
+// contractions inside fixed-size chunks, masked by a static lower-triangular decay
+// mask whose exponents are taken in fp32, and chunks communicate only through an
+// N x P state per (batch, head).  Two kernels follow the per-chunk decay cumsum:
 //
-//   chunk_state_tc  (per b, chunk c, head h):
-//       S_c^T = B_c^T (w o X_c)            M = dstate 128, N = headdim 64, K = chunk
-//       with w_s = exp(Lam_end - Lam_s) dt_s applied to the rows of X in shared memory;
-//       both operands are fp16 (converted in shared memory) so that the carried and
-//       final states see 2^-12 rather than 2^-9 relative rounding per term.
-//   chunk_output_tc (per b, c, h and 128-token tile t of the chunk):
-//       G  = C_t B_{s<=t}^T               M = 128 tokens, N = 128 or 256 sources, K = dstate
-//       Yo = C_t H_c^T                    M = 128, N = headdim, K = dstate
-//       P  = G o exp(Lam_t - Lam_s) o dt_s (s <= t), rounded to bf16 in shared memory
-//       Yd = P X_{s<=t}                   M = 128, N = headdim, K = 128 or 256
-//       y  = Yd + exp(Lam_t) Yo + D_h x_t  -> bf16
+// chunk_state_scan_kernel -- one CTA per (chunk c, batch b, head h):
+//     S_c^T = B_c^T (w o X_c),  w_s = exp(Lam_end - Lam_s) dt_s        (tcgen05, fp16 in)
+//     H_{c+1} = exp(Lam_end) H_c + S_c                                  (fp32, look-back)
+//   The carried state goes from chunk to chunk by decoupled look-back: CTAs take
+//   tickets in launch order (chunk-major), so a CTA only ever waits for CTAs that
+//   have already started; the state of chunk c is handed over in an fp32 two-slot
+//   ring per (b, h) that stays in L2, released with a flag.  Every CTA also writes
+//   its chunk's start state H_c once, as the bf16 operand image the output kernel
+//   loads directly, and the last chunk writes the final state.
 //
-// One thread issues all TMA loads and MMAs of a CTA; every wait on an mbarrier is
-// bounded and records SSD_ERR_TIMEOUT in the device error word on expiry.
+// chunk_output_kernel -- one CTA per (chunk c, 128-token tile i, head group, b),
+//   warp-specialised: warp 0 issues TMA loads, warp 1 issues tcgen05.mma, warps 4-11
+//   build the masked matrix P, warps 12-15 run the epilogue.  Per CTA:
+//     G = C_i B_{s < 128(i+1)}^T                (once; shared by the group's heads)
+//   and per head h of the group (double-buffered operands and accumulators):
+//     P = G o exp(Lam_t - Lam_s) o dt_s (s <= t), bf16 in shared memory
+//     Yd = P X,  Yo = C_i H_c^T                 (tcgen05)
+//     y  = Yd + exp(Lam_t) Yo + D_h x_t  -> bf16
+//   Off-diagonal 32-column blocks of P use exp(Lam_t - Lam_r) exp(Lam_r - Lam_s)
+//   with r the block's last column (both factors <= 1); only blocks that cross the
+//   diagonal take one exponential per element.
+//
+// Every wait is bounded; expiry records SSD_ERR_TIMEOUT in the device error word and
+// the CTA drains without further waiting.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -33,8 +43,9 @@ using namespace ptx;
 
 namespace {
 
-constexpr int kTcThreads = 128;
 constexpr int kBox = 16384;                    // one TMA box: 128 rows x 128 bytes
+constexpr int kHImage = 16384;                 // bf16 H_c image: 2 x 64 rows x 128 B
+constexpr int kP = 64, kN = 128;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -43,25 +54,29 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // Byte offset of 16-byte chunk q of row r in a 128B-swizzled tile.
 __device__ __forceinline__ uint32_t sw128(int r, int q) { return r * 128 + ((q ^ (r & 7)) << 4); }
 
-// ---------------------------------------------------------------- chunk state
+// ================================================================ chunk state + scan
+constexpr int kScanThreads = 128;
+
 template <int Q>
-struct StateSmem {
+struct ScanSmem {
     static constexpr int kB = 0;                   // [2 n-halves][Q rows][128 B]
-    static constexpr int kX = 2 * Q * 128;         // [Q rows][128 B]
+    static constexpr int kX = 2 * Q * 128;         // [Q rows][128 B]; later the H_c image
     static constexpr int kW = kX + Q * 128;        // float[Q]
-    static constexpr int kBar = kW + Q * 4;        // 2 x mbarrier
+    static constexpr int kBar = kW + Q * 4;        // 2 mbarriers
     static constexpr int kSlot = kBar + 16;        // TMEM address
-    static constexpr int kBytes = kSlot + 16 + 1024;
+    static constexpr int kTicket = kSlot + 4;
+    static constexpr int kBytes = kTicket + 12 + 1024;
 };
 
 template <int Q>
-__global__ void __launch_bounds__(kTcThreads, 1)
-chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-                      const float* __restrict__ dt, const float* __restrict__ lam,
-                      float* __restrict__ states, int seqlen, int nheads, int ngroups, int nchunks,
-                      int* err)
+__global__ void __launch_bounds__(kScanThreads, 2)
+chunk_state_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
+                        const float* __restrict__ lam, const float* __restrict__ dtT,
+                        const float* __restrict__ init_state, float* final_state,
+                        float* __restrict__ ring, uint8_t* __restrict__ himg, int* flags,
+                        int* ticket, int batch, int nheads, int ngroups, int nchunks, int* err)
 {
-    using L = StateSmem<Q>;
+    using L = ScanSmem<Q>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     uint8_t* sB = sm + L::kB;
@@ -69,14 +84,11 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
     float* sw = reinterpret_cast<float*>(sm + L::kW);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
     uint32_t* slot = reinterpret_cast<uint32_t*>(sm + L::kSlot);
+    int* sticket = reinterpret_cast<int*>(sm + L::kTicket);
 
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int g = h / (nheads / ngroups);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int t0 = c * Q;
-    const int qlen = min(Q, seqlen - t0);
-
     if (tid == 0) {
+        *sticket = atomicAdd(ticket, 1);
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
         fence_mbar_init();
@@ -90,48 +102,53 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *slot;
+    const int BH = batch * nheads;
+    const int k = *sticket;
+    const int c = k / BH, bh = k - c * BH;
+    const int b = bh / nheads, h = bh - b * nheads;
+    const int g = h / (nheads / ngroups);
+    const int t0 = c * Q;
 
     if (tid == 0) {
         mbar_expect_tx(&bars[0], 3 * Q * 128);
 #pragma unroll
         for (int rb = 0; rb < Q / 128; ++rb) {
-            tma_load_3d(sB + rb * kBox, &tm_b, g * 128, t0 + rb * 128, b, &bars[0]);
-            tma_load_3d(sB + Q * 128 + rb * kBox, &tm_b, g * 128 + 64, t0 + rb * 128, b, &bars[0]);
-            tma_load_3d(sX + rb * kBox, &tm_x, h * 64, t0 + rb * 128, b, &bars[0]);
+            tma_load_3d(sB + rb * kBox, &tm_b, g * kN, t0 + rb * 128, b, &bars[0]);
+            tma_load_3d(sB + Q * 128 + rb * kBox, &tm_b, g * kN + 64, t0 + rb * 128, b, &bars[0]);
+            tma_load_3d(sX + rb * kBox, &tm_x, h * kP, t0 + rb * 128, b, &bars[0]);
         }
     }
-    const float* lamc = lam + (((size_t)b * nheads + h) * nchunks + c) * Q;
-    const float lam_end = lamc[Q - 1];
-    for (int s = tid; s < Q; s += kTcThreads)
-        sw[s] = s < qlen ? expf(lam_end - lamc[s]) * dt[((size_t)b * seqlen + t0 + s) * nheads + h] : 0.f;
+    const size_t row = ((size_t)bh * nchunks + c) * Q;
+    const float lam_end = lam[row + Q - 1];
+    for (int s = tid; s < Q; s += kScanThreads) sw[s] = expf(lam_end - lam[row + s]) * dtT[row + s];
     __syncthreads();
 
     bool ok = mbar_wait(&bars[0], 0, err);
     if (ok) {
-        // Operands go to the tensor cores as fp16 (3 more mantissa bits than bf16; every
-        // bf16 input and every w x product of these workloads is far inside fp16 range).
+        // Operands go to the tensor cores as fp16 (3 more mantissa bits than bf16; the
+        // bf16 inputs and the w x products of these workloads lie far inside fp16 range):
         // X~ = w o X and B are converted in place; a row's 16-byte chunks all belong to it.
-        for (int s = tid; s < Q; s += kTcThreads) {
+        for (int s = tid; s < Q; s += kScanThreads) {
             const float w = sw[s];
-            uint4* row = reinterpret_cast<uint4*>(sX + s * 128);
+            uint4* r4 = reinterpret_cast<uint4*>(sX + s * 128);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                uint4 u = row[q];
+                uint4 u = r4[q];
                 u.x = pack_f16x2(bf16lo(u.x) * w, bf16hi(u.x) * w);
                 u.y = pack_f16x2(bf16lo(u.y) * w, bf16hi(u.y) * w);
                 u.z = pack_f16x2(bf16lo(u.z) * w, bf16hi(u.z) * w);
                 u.w = pack_f16x2(bf16lo(u.w) * w, bf16hi(u.w) * w);
-                row[q] = u;
+                r4[q] = u;
             }
         }
-        for (int i = tid; i < 2 * Q * 8; i += kTcThreads) {
-            uint4* chunk = reinterpret_cast<uint4*>(sB) + i;
-            uint4 u = *chunk;
+        for (int i = tid; i < 2 * Q * 8; i += kScanThreads) {
+            uint4* ch = reinterpret_cast<uint4*>(sB) + i;
+            uint4 u = *ch;
             u.x = pack_f16x2(bf16lo(u.x), bf16hi(u.x));
             u.y = pack_f16x2(bf16lo(u.y), bf16hi(u.y));
             u.z = pack_f16x2(bf16lo(u.z), bf16hi(u.z));
             u.w = pack_f16x2(bf16lo(u.w), bf16hi(u.w));
-            *chunk = u;
+            *ch = u;
         }
     }
     fence_proxy_async_smem();
@@ -145,26 +162,61 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
         for (int ks = 0; ks < Q / 16; ++ks) {
             const uint64_t ad = smem_desc_sw128(aB + ks * 2048, Q * 128, 1024);
             const uint64_t bd = smem_desc_sw128(aX + ks * 2048, Q * 128, 1024);
-            umma_bf16(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
+            umma_f16(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
         }
         umma_commit(&bars[1]);
     }
     if (ok) ok = mbar_wait(&bars[1], 0, err);
     ok = __syncthreads_and(ok);
     tc_fence_after();
-    if (ok) {
-        uint32_t v0[32], v1[32];
-        const uint32_t ta = tmem + ((uint32_t)(warp * 32) << 16);
-        tmem_ld32(ta, v0);
-        tmem_ld32(ta + 32, v1);
-        tmem_wait_ld();
-        const int n = warp * 32 + lane;
-        float* out = states + (((size_t)b * nheads + h) * nchunks + c) * (64 * 128) + n;
-#pragma unroll
-        for (int p = 0; p < 32; ++p) out[p * 128] = __uint_as_float(v0[p]);
-#pragma unroll
-        for (int p = 0; p < 32; ++p) out[(p + 32) * 128] = __uint_as_float(v1[p]);
+
+    // ---- look-back: the state at the start of this chunk
+    if (c > 0 && tid == 0) {
+        uint32_t it = 0;
+        while (ld_acquire_gpu(flags + bh) < c) {
+            if (++it > (1u << 24)) {
+                record_error(err, SSD_ERR_TIMEOUT);
+                break;
+            }
+        }
+        __threadfence();
     }
+    __syncthreads();
+
+    const int n = warp * 32 + lane;                 // TMEM lane = state column n
+    const float ec = expf(lam_end);
+    float* ring_bh = ring + (size_t)bh * 2 * kP * kN;
+    const float* hsrc = c == 0 ? (init_state ? init_state + (size_t)bh * kP * kN : nullptr)
+                               : ring_bh + (size_t)(c & 1) * kP * kN;
+    const bool last = c == nchunks - 1;
+    float* hdst = last ? final_state + (size_t)bh * kP * kN : ring_bh + (size_t)((c + 1) & 1) * kP * kN;
+    uint16_t* himg_s = reinterpret_cast<uint16_t*>(sX);            // X~ is no longer needed
+    const int kb = n >> 6, qn = (n & 63) >> 3, jn = n & 7;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + half * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int pp = 0; pp < 32; ++pp) {
+            const int p = half * 32 + pp;
+            const float hc = hsrc ? __ldcg(hsrc + p * kN + n) : 0.f;
+            const float sc = ok ? __uint_as_float(v[pp]) : 0.f;
+            hdst[p * kN + n] = fmaf(ec, hc, sc);
+            const __nv_bfloat16 hb = __float2bfloat16_rn(hc);
+            himg_s[(kb * 8192 + p * 128 + ((qn ^ (p & 7)) << 4) + jn * 2) >> 1] =
+                *reinterpret_cast<const uint16_t*>(&hb);
+        }
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0 && !last) st_release_gpu(flags + bh, c + 1);
+
+    // bf16 image of H_c for the output kernel
+    uint4* dst = reinterpret_cast<uint4*>(himg + ((size_t)bh * nchunks + c) * kHImage);
+    const uint4* src = reinterpret_cast<const uint4*>(sX);
+    for (int i = tid; i < kHImage / 16; i += kScanThreads) dst[i] = src[i];
+
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -173,30 +225,39 @@ chunk_state_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_con
     }
 }
 
-// ---------------------------------------------------------------- chunk output
+// ================================================================ chunk output
+constexpr int kOutThreads = 512;
+constexpr int kWarpTma = 0, kWarpMma = 1, kWarpP0 = 4, kWarpE0 = 12;
+constexpr int kPThreads = 256, kEThreads = 128;
+
 template <int Q>
 struct OutSmem {
     static constexpr int kC = 0;                        // [2 n-halves][128 rows][128 B]
-    static constexpr int kB = 2 * kBox;                 // [2 n-halves][Q rows][128 B]
-    static constexpr int kX = kB + 2 * Q * 128;         // [Q rows][128 B]
-    static constexpr int kP = kX + Q * 128;             // [Q/64 s-blocks][128 rows][128 B]
-    static constexpr int kH = kP + (Q / 64) * kBox;     // [2 n-halves][64 rows][128 B]
-    static constexpr int kLam = kH + 2 * 8192;          // float[Q]
-    static constexpr int kDt = kLam + Q * 4;            // float[Q]
-    static constexpr int kBar = kDt + Q * 4;
-    static constexpr int kSlot = kBar + 16;
-    static constexpr int kBytes = kSlot + 16 + 1024;
+    static constexpr int kB = 2 * kBox;                 // [2 n-halves][Q rows][128 B]; then P
+    static constexpr int kSlot0 = kB + 2 * Q * 128;     // per-head slots
+    static constexpr int kXo = 0;                       //   X  [Q rows][128 B]
+    static constexpr int kHo = Q * 128;                 //   H_c image (16 KB)
+    static constexpr int kLo = kHo + kHImage;           //   Lam[Q]
+    static constexpr int kDo = kLo + Q * 4;             //   dt[Q]
+    static constexpr int kVo = kDo + Q * 4;             //   column factors v[Q]
+    static constexpr int kSlotBytes = (kVo + Q * 4 + 1023) / 1024 * 1024;
+    static constexpr int kBar = kSlot0 + 2 * kSlotBytes;
+    static constexpr int kNumBars = 12;
+    static constexpr int kSlotTm = kBar + kNumBars * 8;
+    static constexpr int kAbort = kSlotTm + 4;
+    static constexpr int kBytes = kAbort + 12 + 1024;
 };
 
-constexpr uint32_t kColS = 0, kColYd = 256, kColYo = 320;
+enum { BAR_CB = 0, BAR_S = 1, BAR_XFULL = 2, BAR_XEMPTY = 4, BAR_PFULL = 6, BAR_PEMPTY = 7,
+       BAR_AFULL = 8, BAR_AEMPTY = 10 };
 
 template <int Q>
-__global__ void __launch_bounds__(kTcThreads, 1)
-chunk_output_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-                       const __grid_constant__ CUtensorMap tm_c, const float* __restrict__ dt,
-                       const float* __restrict__ D, const float* __restrict__ lam,
-                       const float* __restrict__ states, __nv_bfloat16* __restrict__ y, int seqlen,
-                       int nheads, int ngroups, int nchunks, int* err)
+__global__ void __launch_bounds__(kOutThreads, 1)
+chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
+                    const __grid_constant__ CUtensorMap tm_c, const float* __restrict__ lam,
+                    const float* __restrict__ dtT, const uint8_t* __restrict__ himg,
+                    const float* __restrict__ D, __nv_bfloat16* __restrict__ y, int seqlen,
+                    int nheads, int ngroups, int nchunks, int heads_per_cta, int* err)
 {
     using L = OutSmem<Q>;
     constexpr int NT = Q / 128;
@@ -204,172 +265,215 @@ chunk_output_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_co
     uint8_t* sm = align1024(smem_raw);
     uint8_t* sC = sm + L::kC;
     uint8_t* sB = sm + L::kB;
-    uint8_t* sX = sm + L::kX;
-    uint8_t* sP = sm + L::kP;
-    uint8_t* sH = sm + L::kH;
-    float* sLam = reinterpret_cast<float*>(sm + L::kLam);
-    float* sDt = reinterpret_cast<float*>(sm + L::kDt);
+    uint8_t* sP = sB;                                   // B is dead once G is computed
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
-    uint32_t* slot = reinterpret_cast<uint32_t*>(sm + L::kSlot);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::kSlotTm);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kAbort);
 
-    const int c = blockIdx.x / NT, it = blockIdx.x % NT, h = blockIdx.y, b = blockIdx.z;
-    const int g = h / (nheads / ngroups);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x / NT, it = blockIdx.x - c * NT;
+    const int hg = blockIdx.y, b = blockIdx.z;
+    const int h0 = hg * heads_per_cta;
+    const int g = h0 / (nheads / ngroups);
     const int R = 128 * (it + 1);                       // source tokens s in [0, R)
     const int t0 = c * Q;
     const int qlen = min(Q, seqlen - t0);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
+        mbar_init(&bars[BAR_CB], 1);
+        mbar_init(&bars[BAR_S], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars[BAR_XFULL + s], 1);
+            mbar_init(&bars[BAR_XEMPTY + s], kEThreads);
+            mbar_init(&bars[BAR_AFULL + s], 1);
+            mbar_init(&bars[BAR_AEMPTY + s], kEThreads);
+        }
+        mbar_init(&bars[BAR_PFULL], kPThreads);
+        mbar_init(&bars[BAR_PEMPTY], 1);
+        *abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
     }
-    if (warp == 0) {
-        tmem_alloc(slot, 512);
+    if (warp == kWarpMma) {
+        tmem_alloc(tslot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *slot;
+    const uint32_t tmem = *tslot;
 
-    if (tid == 0) {
-        mbar_expect_tx(&bars[0], 2 * kBox + (it + 1) * 3 * kBox);
-        tma_load_3d(sC, &tm_c, g * 128, t0 + it * 128, b, &bars[0]);
-        tma_load_3d(sC + kBox, &tm_c, g * 128 + 64, t0 + it * 128, b, &bars[0]);
-        for (int rb = 0; rb <= it; ++rb) {
-            tma_load_3d(sB + rb * kBox, &tm_b, g * 128, t0 + rb * 128, b, &bars[0]);
-            tma_load_3d(sB + Q * 128 + rb * kBox, &tm_b, g * 128 + 64, t0 + rb * 128, b, &bars[0]);
-            tma_load_3d(sX + rb * kBox, &tm_x, h * 64, t0 + rb * 128, b, &bars[0]);
-        }
-    }
-    const float* lamc = lam + (((size_t)b * nheads + h) * nchunks + c) * Q;
-    for (int s = tid; s < R; s += kTcThreads) {
-        sLam[s] = lamc[s];
-        sDt[s] = s < qlen ? dt[((size_t)b * seqlen + t0 + s) * nheads + h] : 0.f;
-    }
-    // carried state H_c [64][128] fp32 -> bf16, K-major swizzled B operand
-    const float* Hc = states + (((size_t)b * nheads + h) * nchunks + c) * (64 * 128);
-    for (int id = tid; id < 64 * 16; id += kTcThreads) {
-        const int p = id >> 4, kb = (id >> 3) & 1, q = id & 7;
-        const float4* src = reinterpret_cast<const float4*>(Hc + p * 128 + kb * 64 + q * 8);
-        const float4 f0 = src[0], f1 = src[1];
-        uint4 u;
-        u.x = pack_bf16x2(f0.x, f0.y);
-        u.y = pack_bf16x2(f0.z, f0.w);
-        u.z = pack_bf16x2(f1.x, f1.y);
-        u.w = pack_bf16x2(f1.z, f1.w);
-        *reinterpret_cast<uint4*>(sH + kb * 8192 + sw128(p, q)) = u;
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
+    auto slot_base = [&](int s) { return sm + L::kSlot0 + s * L::kSlotBytes; };
 
-    bool ok = mbar_wait(&bars[0], 0, err);
-    ok = __syncthreads_and(ok);
-    if (tid == 0 && ok) {
-        tc_fence_after();
-        const uint32_t idS = idesc_bf16_f32(128, R, false, false);
-        constexpr uint32_t idY = idesc_bf16_f32(128, 64, false, false);
-        const uint32_t aC = smem_u32(sC), aB = smem_u32(sB), aH = smem_u32(sH);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
-            const uint64_t ad = smem_desc_sw128(aC + kb * kBox + off, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(aB + kb * (Q * 128) + off, 16, 1024);
-            umma_bf16(tmem + kColS, ad, bd, idS, ks > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
-            const uint64_t ad = smem_desc_sw128(aC + kb * kBox + off, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(aH + kb * 8192 + off, 16, 1024);
-            umma_bf16(tmem + kColYo, ad, bd, idY, ks > 0 ? 1u : 0u);
-        }
-        umma_commit(&bars[1]);
-    }
-    if (ok) ok = mbar_wait(&bars[1], 0, err);
-    ok = __syncthreads_and(ok);
-    tc_fence_after();
-
-    const int r = warp * 32 + lane;                     // TMEM lane = tile row
-    const int tl = it * 128 + r;                        // token index within the chunk
-    const float lam_t = sLam[tl];
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-    if (ok) {
-        for (int cb = 0; cb < R / 32; ++cb) {
-            uint32_t v[32];
-            tmem_ld32(trow + kColS + cb * 32, v);
-            tmem_wait_ld();
-            uint32_t pk[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int s0 = cb * 32 + 2 * j;
-                const float p0 = s0 <= tl ? __uint_as_float(v[2 * j]) * expf(lam_t - sLam[s0]) * sDt[s0] : 0.f;
-                const float p1 = s0 + 1 <= tl ? __uint_as_float(v[2 * j + 1]) * expf(lam_t - sLam[s0 + 1]) * sDt[s0 + 1] : 0.f;
-                pk[j] = pack_bf16x2(p0, p1);
+    if (warp == kWarpTma) {
+        if (lane == 0) {
+            mbar_expect_tx(&bars[BAR_CB], 2 * kBox + (it + 1) * 2 * kBox);
+            tma_load_3d(sC, &tm_c, g * kN, t0 + it * 128, b, &bars[BAR_CB]);
+            tma_load_3d(sC + kBox, &tm_c, g * kN + 64, t0 + it * 128, b, &bars[BAR_CB]);
+            for (int rb = 0; rb <= it; ++rb) {
+                tma_load_3d(sB + rb * kBox, &tm_b, g * kN, t0 + rb * 128, b, &bars[BAR_CB]);
+                tma_load_3d(sB + Q * 128 + rb * kBox, &tm_b, g * kN + 64, t0 + rb * 128, b, &bars[BAR_CB]);
             }
-            uint8_t* blk = sP + (cb >> 1) * kBox;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int q = (cb & 1) * 4 + k;
-                *reinterpret_cast<uint4*>(blk + sw128(r, q)) =
-                    make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+            for (int j = 0; j < heads_per_cta; ++j) {
+                const int s = j & 1, use = j >> 1;
+                if (j >= 2 && !mbar_wait_or_abort(&bars[BAR_XEMPTY + s], (use - 1) & 1, err, abort_flag)) break;
+                const int h = h0 + j;
+                const size_t bh = (size_t)b * nheads + h;
+                uint8_t* sl = slot_base(s);
+                mbar_expect_tx(&bars[BAR_XFULL + s], (it + 1) * kBox + kHImage + 2 * R * 4);
+                for (int rb = 0; rb <= it; ++rb)
+                    tma_load_3d(sl + L::kXo + rb * kBox, &tm_x, h * kP, t0 + rb * 128, b, &bars[BAR_XFULL + s]);
+                bulk_load(sl + L::kHo, himg + (bh * nchunks + c) * kHImage, kHImage, &bars[BAR_XFULL + s]);
+                bulk_load(sl + L::kLo, lam + (bh * nchunks + c) * Q, R * 4, &bars[BAR_XFULL + s]);
+                bulk_load(sl + L::kDo, dtT + (bh * nchunks + c) * Q, R * 4, &bars[BAR_XFULL + s]);
             }
         }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && ok) {
-        tc_fence_after();
-        constexpr uint32_t idY = idesc_bf16_f32(128, 64, false, true);
-        const uint32_t aP = smem_u32(sP), aX = smem_u32(sX);
-        for (int ks = 0; ks < R / 16; ++ks) {
-            const uint64_t ad = smem_desc_sw128(aP + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(aX + ks * 2048, Q * 128, 1024);
-            umma_bf16(tmem + kColYd, ad, bd, idY, ks > 0 ? 1u : 0u);
+    } else if (warp == kWarpMma) {
+        if (lane == 0 && mbar_wait_or_abort(&bars[BAR_CB], 0, err, abort_flag)) {
+            tc_fence_after();
+            const uint32_t aC = smem_u32(sC), aB = smem_u32(sB), aP = smem_u32(sP);
+            const uint32_t idG = idesc_bf16_f32(128, R, false, false);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
+                umma_f16(tmem, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
+                         smem_desc_sw128(aB + kb * (Q * 128) + off, 16, 1024), idG, ks > 0 ? 1u : 0u);
+            }
+            umma_commit(&bars[BAR_S]);
+            constexpr uint32_t idYd = idesc_bf16_f32(128, 64, false, true);
+            constexpr uint32_t idYo = idesc_bf16_f32(128, 64, false, false);
+            for (int j = 0; j < heads_per_cta; ++j) {
+                const int s = j & 1, use = j >> 1;
+                if (!mbar_wait_or_abort(&bars[BAR_XFULL + s], use & 1, err, abort_flag)) break;
+                if (!mbar_wait_or_abort(&bars[BAR_PFULL], j & 1, err, abort_flag)) break;
+                if (j >= 2 && !mbar_wait_or_abort(&bars[BAR_AEMPTY + s], (use - 1) & 1, err, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t acc = tmem + 256 + s * 128;
+                const uint32_t aX = smem_u32(slot_base(s) + L::kXo), aH = smem_u32(slot_base(s) + L::kHo);
+                for (int ks = 0; ks < R / 16; ++ks)
+                    umma_f16(acc, smem_desc_sw128(aP + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
+                             smem_desc_sw128(aX + ks * 2048, Q * 128, 1024), idYd, ks > 0 ? 1u : 0u);
+                umma_commit(&bars[BAR_PEMPTY]);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
+                    umma_f16(acc + 64, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
+                             smem_desc_sw128(aH + kb * 8192 + off, 16, 1024), idYo, ks > 0 ? 1u : 0u);
+                }
+                umma_commit(&bars[BAR_AFULL + s]);
+            }
         }
-        umma_commit(&bars[1]);
-    }
-    if (ok) ok = mbar_wait(&bars[1], 1, err);
-    ok = __syncthreads_and(ok);
-    tc_fence_after();
-
-    if (ok) {
-        const int tg = t0 + tl;
-        const float e = expf(lam_t);
-        const float Dh = D[h];
-        const uint8_t* xrow = sX + tl * 128;
-        __nv_bfloat16* yrow = y + (((size_t)b * seqlen + tg) * nheads + h) * 64;
+    } else if (warp >= kWarpP0 && warp < kWarpE0) {
+        // ---- P = G o L o dt for this thread's row, half of the 32-column blocks
+        const int pw = warp - kWarpP0;
+        const int q = warp & 3, colhalf = pw >> 2;
+        const int r = q * 32 + lane;
+        const int tl = it * 128 + r;
+        const int ptid = tid - kWarpP0 * 32;
+        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+        bool live = mbar_wait_or_abort(&bars[BAR_S], 0, err, abort_flag);
+        tc_fence_after();
+        for (int j = 0; j < heads_per_cta; ++j) {
+            const int s = j & 1, use = j >> 1;
+            live = live && mbar_wait_or_abort(&bars[BAR_XFULL + s], use & 1, err, abort_flag);
+            // all P threads agree before touching the slot (no thread may leave the
+            // named barrier below while another still waits in it)
+            if (!named_bar_and(1, kPThreads, live)) break;
+            const float* sLam = reinterpret_cast<const float*>(slot_base(s) + L::kLo);
+            const float* sDt = reinterpret_cast<const float*>(slot_base(s) + L::kDo);
+            float* sV = reinterpret_cast<float*>(slot_base(s) + L::kVo);
+            for (int si = ptid; si < R; si += kPThreads)
+                sV[si] = expf(sLam[si | 31] - sLam[si]) * sDt[si];
+            // the previous head's GEMM must have read P before it is overwritten; this
+            // barrier also publishes sV to all P threads
+            if (j >= 1) live = mbar_wait_or_abort(&bars[BAR_PEMPTY], (j - 1) & 1, err, abort_flag);
+            if (!named_bar_and(1, kPThreads, live)) break;
+            const float lam_t = sLam[tl];
+            for (int kc = colhalf; kc < R / 32; kc += 2) {
+                const int s0 = kc * 32;
+                uint32_t v[32];
+                tmem_ld32(trow + s0, v);
+                tmem_wait_ld();
+                uint32_t pk[16];
+                if (s0 + 31 <= tl) {
+                    const float u = expf(lam_t - sLam[s0 + 31]);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            uint32_t yd[32], yo[32];
-            tmem_ld32(trow + kColYd + half * 32, yd);
-            tmem_ld32(trow + kColYo + half * 32, yo);
-            tmem_wait_ld();
-            if (tl < qlen) {
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * u * sV[s0 + 2 * e],
+                                            __uint_as_float(v[2 * e + 1]) * u * sV[s0 + 2 * e + 1]);
+                } else if (s0 > tl) {
 #pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const int q = half * 4 + qq;
-                    const uint4 xu = *reinterpret_cast<const uint4*>(xrow + ((q ^ (tl & 7)) << 4));
-                    const uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w};
-                    uint32_t o[4];
+                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                } else {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int j = qq * 8 + 2 * k;
-                        const float a0 = __uint_as_float(yd[j]) + e * __uint_as_float(yo[j]) + Dh * bf16lo(xw[k]);
-                        const float a1 = __uint_as_float(yd[j + 1]) + e * __uint_as_float(yo[j + 1]) + Dh * bf16hi(xw[k]);
-                        o[k] = pack_bf16x2(a0, a1);
+                    for (int e = 0; e < 16; ++e) {
+                        const int sa = s0 + 2 * e, sb = sa + 1;
+                        const float pa = sa <= tl ? __uint_as_float(v[2 * e]) * expf(lam_t - sLam[sa]) * sDt[sa] : 0.f;
+                        const float pb = sb <= tl ? __uint_as_float(v[2 * e + 1]) * expf(lam_t - sLam[sb]) * sDt[sb] : 0.f;
+                        pk[e] = pack_bf16x2(pa, pb);
                     }
-                    *reinterpret_cast<uint4*>(yrow + q * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                uint8_t* blk = sP + (kc >> 1) * kBox;
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4)
+                    *reinterpret_cast<uint4*>(blk + sw128(r, (kc & 1) * 4 + k4)) =
+                        make_uint4(pk[4 * k4], pk[4 * k4 + 1], pk[4 * k4 + 2], pk[4 * k4 + 3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[BAR_PFULL]);
+        }
+    } else if (warp >= kWarpE0) {
+        // ---- epilogue: y = Yd + exp(Lam_t) Yo + D x
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const int tl = it * 128 + r;
+        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+        for (int j = 0; j < heads_per_cta; ++j) {
+            const int s = j & 1, use = j >> 1;
+            if (!mbar_wait_or_abort(&bars[BAR_AFULL + s], use & 1, err, abort_flag)) break;
+            tc_fence_after();
+            const int h = h0 + j;
+            const uint8_t* sl = slot_base(s);
+            const float lam_t = reinterpret_cast<const float*>(sl + L::kLo)[tl];
+            const float e = expf(lam_t);
+            const float Dh = D[h];
+            const uint8_t* xrow = sl + L::kXo + tl * 128;
+            __nv_bfloat16* yrow = y + (((size_t)b * seqlen + t0 + tl) * nheads + h) * kP;
+            const uint32_t acc = trow + 256 + s * 128;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t yd[32], yo[32];
+                tmem_ld32(acc + half * 32, yd);
+                tmem_ld32(acc + 64 + half * 32, yo);
+                tmem_wait_ld();
+                if (tl < qlen) {
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        const int qx = half * 4 + qq;
+                        const uint4 xu = *reinterpret_cast<const uint4*>(xrow + ((qx ^ (tl & 7)) << 4));
+                        const uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w};
+                        uint32_t o[4];
+#pragma unroll
+                        for (int k2 = 0; k2 < 4; ++k2) {
+                            const int jj = qq * 8 + 2 * k2;
+                            const float a0 = fmaf(e, __uint_as_float(yo[jj]), __uint_as_float(yd[jj])) + Dh * bf16lo(xw[k2]);
+                            const float a1 = fmaf(e, __uint_as_float(yo[jj + 1]), __uint_as_float(yd[jj + 1])) + Dh * bf16hi(xw[k2]);
+                            o[k2] = pack_bf16x2(a0, a1);
+                        }
+                        *reinterpret_cast<uint4*>(yrow + qx * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
                 }
             }
+            tc_fence_before();
+            mbar_arrive(&bars[BAR_AEMPTY + s]);
+            mbar_arrive(&bars[BAR_XEMPTY + s]);
         }
     }
+
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -403,34 +507,46 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int Q>
-cudaError_t chunk_state_tc_t(const Dims& d, const CUtensorMap& mx, const CUtensorMap& mb,
-                             const float* dt, const float* lam, float* states, cudaStream_t s)
+// Heads per output CTA: the largest divisor of (heads per group) that is <= 8, so that a
+// CTA's heads share one B/C group.
+int heads_per_cta(const Dims& d)
 {
-    auto k = chunk_state_tc_kernel<Q>;
+    const int hpg = d.nheads / d.ngroups;
+    for (int k = 8; k > 1; --k)
+        if (hpg % k == 0) return k;
+    return 1;
+}
+
+template <int Q>
+cudaError_t scan_t(const Dims& d, const CUtensorMap& mx, const CUtensorMap& mb, const TcWorkspace& w,
+                   const float* init_state, float* final_state, cudaStream_t s)
+{
+    auto k = chunk_state_scan_kernel<Q>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         StateSmem<Q>::kBytes);
+                                         ScanSmem<Q>::kBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid(d.nchunks, d.nheads, d.batch);
-    k<<<grid, kTcThreads, StateSmem<Q>::kBytes, s>>>(mx, mb, dt, lam, states, d.seqlen, d.nheads,
-                                                     d.ngroups, d.nchunks, device_error_word());
+    const unsigned grid = (unsigned)((size_t)d.nchunks * d.batch * d.nheads);
+    k<<<grid, kScanThreads, ScanSmem<Q>::kBytes, s>>>(mx, mb, w.lam, w.dtT, init_state, final_state,
+                                                      w.ring, w.himg, w.flags, w.flags + d.batch * d.nheads,
+                                                      d.batch, d.nheads, d.ngroups, d.nchunks,
+                                                      device_error_word());
     return cudaGetLastError();
 }
 
 template <int Q>
-cudaError_t chunk_output_tc_t(const Dims& d, const CUtensorMap& mx, const CUtensorMap& mb,
-                              const CUtensorMap& mc, const float* dt, const float* D,
-                              const float* lam, const float* states, void* y, cudaStream_t s)
+cudaError_t output_t(const Dims& d, const CUtensorMap& mx, const CUtensorMap& mb, const CUtensorMap& mc,
+                     const TcWorkspace& w, const float* D, void* y, cudaStream_t s)
 {
-    auto k = chunk_output_tc_kernel<Q>;
+    auto k = chunk_output_kernel<Q>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          OutSmem<Q>::kBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid(d.nchunks * (Q / 128), d.nheads, d.batch);
-    k<<<grid, kTcThreads, OutSmem<Q>::kBytes, s>>>(mx, mb, mc, dt, D, lam, states,
-                                                   static_cast<__nv_bfloat16*>(y), d.seqlen,
-                                                   d.nheads, d.ngroups, d.nchunks,
-                                                   device_error_word());
+    const int hpc = heads_per_cta(d);
+    dim3 grid(d.nchunks * (Q / 128), d.nheads / hpc, d.batch);
+    k<<<grid, kOutThreads, OutSmem<Q>::kBytes, s>>>(mx, mb, mc, w.lam, w.dtT, w.himg, D,
+                                                    static_cast<__nv_bfloat16*>(y), d.seqlen,
+                                                    d.nheads, d.ngroups, d.nchunks, hpc,
+                                                    device_error_word());
     return cudaGetLastError();
 }
 
@@ -438,33 +554,52 @@ cudaError_t chunk_output_tc_t(const Dims& d, const CUtensorMap& mx, const CUtens
 
 bool tc_prefill_supported(const Dims& d)
 {
-    return d.headdim == 64 && d.dstate == 128 && (d.chunk_len == 128 || d.chunk_len == 256);
+    return d.headdim == kP && d.dstate == kN && (d.chunk_len == 128 || d.chunk_len == 256);
 }
 
-cudaError_t launch_chunk_state_tc(const Dims& d, const void* x, const float* dt, const void* B,
-                                  const float* lam, float* states, cudaStream_t s)
+size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w)
+{
+    auto up = [](size_t v) { return (v + 255) & ~size_t(255); };
+    const size_t BH = (size_t)d.batch * d.nheads;
+    const size_t lam_b = up(BH * d.nchunks * d.chunk_len * sizeof(float));
+    const size_t ring_b = up(BH * 2 * kP * kN * sizeof(float));
+    const size_t himg_b = up(BH * d.nchunks * kHImage);
+    const size_t flag_b = up((BH + 1) * sizeof(int));
+    if (w) {
+        char* p = static_cast<char*>(base);
+        w->lam = reinterpret_cast<float*>(p);
+        w->dtT = reinterpret_cast<float*>(p + lam_b);
+        w->ring = reinterpret_cast<float*>(p + 2 * lam_b);
+        w->himg = reinterpret_cast<uint8_t*>(p + 2 * lam_b + ring_b);
+        w->flags = reinterpret_cast<int*>(p + 2 * lam_b + ring_b + himg_b);
+    }
+    return 2 * lam_b + ring_b + himg_b + flag_b;
+}
+
+cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void* B,
+                                       const TcWorkspace& w, const float* init_state,
+                                       float* final_state, cudaStream_t s)
 {
     if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
     CUtensorMap mx, mb;
-    if (!make_map(&mx, x, (uint64_t)d.nheads * 64, d.seqlen, d.batch) ||
-        !make_map(&mb, B, (uint64_t)d.ngroups * 128, d.seqlen, d.batch))
+    if (!make_map(&mx, x, (uint64_t)d.nheads * kP, d.seqlen, d.batch) ||
+        !make_map(&mb, B, (uint64_t)d.ngroups * kN, d.seqlen, d.batch))
         return cudaErrorInvalidValue;
-    if (d.chunk_len == 256) return chunk_state_tc_t<256>(d, mx, mb, dt, lam, states, s);
-    return chunk_state_tc_t<128>(d, mx, mb, dt, lam, states, s);
+    if (d.chunk_len == 256) return scan_t<256>(d, mx, mb, w, init_state, final_state, s);
+    return scan_t<128>(d, mx, mb, w, init_state, final_state, s);
 }
 
-cudaError_t launch_chunk_output_tc(const Dims& d, const void* x, const float* dt, const void* B,
-                                   const void* C, const float* D, const float* lam,
-                                   const float* states, void* y, cudaStream_t s)
+cudaError_t launch_chunk_output_tc(const Dims& d, const void* x, const void* B, const void* C,
+                                   const float* D, const TcWorkspace& w, void* y, cudaStream_t s)
 {
     if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
     CUtensorMap mx, mb, mc;
-    if (!make_map(&mx, x, (uint64_t)d.nheads * 64, d.seqlen, d.batch) ||
-        !make_map(&mb, B, (uint64_t)d.ngroups * 128, d.seqlen, d.batch) ||
-        !make_map(&mc, C, (uint64_t)d.ngroups * 128, d.seqlen, d.batch))
+    if (!make_map(&mx, x, (uint64_t)d.nheads * kP, d.seqlen, d.batch) ||
+        !make_map(&mb, B, (uint64_t)d.ngroups * kN, d.seqlen, d.batch) ||
+        !make_map(&mc, C, (uint64_t)d.ngroups * kN, d.seqlen, d.batch))
         return cudaErrorInvalidValue;
-    if (d.chunk_len == 256) return chunk_output_tc_t<256>(d, mx, mb, mc, dt, D, lam, states, y, s);
-    return chunk_output_tc_t<128>(d, mx, mb, mc, dt, D, lam, states, y, s);
+    if (d.chunk_len == 256) return output_t<256>(d, mx, mb, mc, w, D, y, s);
+    return output_t<128>(d, mx, mb, mc, w, D, y, s);
 }
 
 }  // namespace ssd

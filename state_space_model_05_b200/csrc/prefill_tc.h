@@ -8,14 +8,24 @@ namespace ssd {
 // headdim 64, dstate 128, chunk_len 128 or 256, bf16 storage.
 bool tc_prefill_supported(const Dims& d);
 
-// Chunk states S_c = B_c^T (w o X_c), w_s = exp(Lam_end - Lam_s) dt_s, written
-// fp32 [b][h][c][headdim][dstate].
-cudaError_t launch_chunk_state_tc(const Dims& d, const void* x, const float* dt, const void* B,
-                                  const float* lam, float* states, cudaStream_t s);
+// Workspace of the tensor-core path.
+struct TcWorkspace {
+    float* lam;       // [b][h][c][Q] inclusive cumsum of dt*A within each chunk
+    float* dtT;       // [b][h][c][Q] dt, zero past seqlen
+    float* ring;      // [b*h][2][64][128] fp32 hand-off slots of the carried state
+    uint8_t* himg;    // [b][h][c] 16 KB bf16 image of each chunk's start state
+    int* flags;       // [b*h] chunks published so far, then one ticket counter
+};
+size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w);
+
+// Chunk states and the inter-chunk scan (decoupled look-back), writing the chunk
+// start states (bf16 images) and the final state.
+cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void* B,
+                                       const TcWorkspace& w, const float* init_state,
+                                       float* final_state, cudaStream_t s);
 
 // y = (C B^T o L o dt) X + diag(exp Lam) C H_c^T + D x, bf16 out.
-cudaError_t launch_chunk_output_tc(const Dims& d, const void* x, const float* dt, const void* B,
-                                   const void* C, const float* D, const float* lam,
-                                   const float* states, void* y, cudaStream_t s);
+cudaError_t launch_chunk_output_tc(const Dims& d, const void* x, const void* B, const void* C,
+                                   const float* D, const TcWorkspace& w, void* y, cudaStream_t s);
 
 }  // namespace ssd

@@ -46,13 +46,21 @@ def _ws(*a):
 
 
 def test_workspace_bytes(lib):
-    # lam [b][H][c][Q] + states [b][H][c][P][N], each rounded up to 256 bytes
+    up = lambda v: (v + 255) // 256 * 256
     b, T, H, P, G, N, Q = 2, 300, 4, 64, 1, 128, 128
     c = 3
+    # CUDA-core path: lam [b][H][c][Q] + states [b][H][c][P][N]
     lam = b * H * c * Q * 4
     st = b * H * c * P * N * 4
-    up = lambda v: (v + 255) // 256 * 256
-    assert _ws(b, T, H, P, G, N, Q, binding.SSD_BF16) == up(lam) + up(st)
+    assert _ws(b, T, H, P, G, N, Q, binding.SSD_F32) == up(lam) + up(st)
+    # tensor-core path (bf16, P 64, N 128, Q 128/256): lam + dt^T, fp32 hand-off ring,
+    # bf16 chunk-start-state images, look-back flags + ticket
+    ring = b * H * 2 * P * N * 4
+    himg = b * H * c * 16384
+    flags = (b * H + 1) * 4
+    assert _ws(b, T, H, P, G, N, Q, binding.SSD_BF16) == 2 * up(lam) + up(ring) + up(himg) + up(flags)
+    # bf16 with other shapes uses the CUDA-core layout
+    assert _ws(b, T, H, P, G, N, 64, binding.SSD_BF16) == up(b * H * 5 * 64 * 4) + up(b * H * 5 * P * N * 4)
     assert _ws(b, 0, H, P, G, N, Q, binding.SSD_F32) == 0
     assert _ws(b, T, H, 63, G, N, Q, binding.SSD_F32) == 0          # headdim not a multiple of 8
     assert _ws(b, T, 3, P, 2, N, Q, binding.SSD_F32) == 0           # nheads % ngroups
