@@ -55,7 +55,7 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 __device__ __forceinline__ uint32_t sw128(int r, int q) { return r * 128 + ((q ^ (r & 7)) << 4); }
 
 // ================================================================ chunk state + scan
-constexpr int kScanThreads = 128;
+constexpr int kScanThreads = 256;            // warps w and w+4 share TMEM lane quarter w
 
 template <int Q>
 struct ScanSmem {
@@ -183,7 +183,8 @@ chunk_state_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_c
     }
     __syncthreads();
 
-    const int n = warp * 32 + lane;                 // TMEM lane = state column n
+    const int n = (warp & 3) * 32 + lane;           // TMEM lane = state column n
+    const int half = warp >> 2;                     // rows p in [32 half, 32 half + 32)
     const float ec = expf(lam_end);
     float* ring_bh = ring + (size_t)bh * 2 * kP * kN;
     const float* hsrc = c == 0 ? (init_state ? init_state + (size_t)bh * kP * kN : nullptr)
@@ -192,21 +193,22 @@ chunk_state_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_c
     float* hdst = last ? final_state + (size_t)bh * kP * kN : ring_bh + (size_t)((c + 1) & 1) * kP * kN;
     uint16_t* himg_s = reinterpret_cast<uint16_t*>(sX);            // X~ is no longer needed
     const int kb = n >> 6, qn = (n & 63) >> 3, jn = n & 7;
+    uint32_t v[32];
+    tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + half * 32, v);
+    float hc[32];
+    // all loads of the carried state first (the hand-off ring is read and written by
+    // this CTA, so loads must not wait behind the stores)
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        uint32_t v[32];
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + half * 32, v);
-        tmem_wait_ld();
+    for (int pp = 0; pp < 32; ++pp) hc[pp] = hsrc ? __ldcg(hsrc + (half * 32 + pp) * kN + n) : 0.f;
+    tmem_wait_ld();
 #pragma unroll
-        for (int pp = 0; pp < 32; ++pp) {
-            const int p = half * 32 + pp;
-            const float hc = hsrc ? __ldcg(hsrc + p * kN + n) : 0.f;
-            const float sc = ok ? __uint_as_float(v[pp]) : 0.f;
-            hdst[p * kN + n] = fmaf(ec, hc, sc);
-            const __nv_bfloat16 hb = __float2bfloat16_rn(hc);
-            himg_s[(kb * 8192 + p * 128 + ((qn ^ (p & 7)) << 4) + jn * 2) >> 1] =
-                *reinterpret_cast<const uint16_t*>(&hb);
-        }
+    for (int pp = 0; pp < 32; ++pp) {
+        const int p = half * 32 + pp;
+        const float sc = ok ? __uint_as_float(v[pp]) : 0.f;
+        hdst[p * kN + n] = fmaf(ec, hc[pp], sc);
+        const __nv_bfloat16 hb = __float2bfloat16_rn(hc[pp]);
+        himg_s[(kb * 8192 + p * 128 + ((qn ^ (p & 7)) << 4) + jn * 2) >> 1] =
+            *reinterpret_cast<const uint16_t*>(&hb);
     }
     __threadfence();
     __syncthreads();
@@ -242,14 +244,17 @@ struct OutSmem {
     static constexpr int kVo = kDo + Q * 4;             //   column factors v[Q]
     static constexpr int kSlotBytes = (kVo + Q * 4 + 1023) / 1024 * 1024;
     static constexpr int kBar = kSlot0 + 2 * kSlotBytes;
-    static constexpr int kNumBars = 12;
+    static constexpr int kNumBars = 14;
     static constexpr int kSlotTm = kBar + kNumBars * 8;
     static constexpr int kAbort = kSlotTm + 4;
     static constexpr int kBytes = kAbort + 12 + 1024;
 };
 
-enum { BAR_CB = 0, BAR_S = 1, BAR_XFULL = 2, BAR_XEMPTY = 4, BAR_PFULL = 6, BAR_PEMPTY = 7,
-       BAR_AFULL = 8, BAR_AEMPTY = 10 };
+// P is produced and consumed in K-halves of 128 source columns (the halves alternate
+// between the two 32 KB halves of the P buffer), so the P warps build half 0 of head
+// j + 1 while the tensor core still multiplies half 1 of head j.
+enum { BAR_CB = 0, BAR_S = 1, BAR_XFULL = 2, BAR_XEMPTY = 4, BAR_PFULL = 6, BAR_PEMPTY = 8,
+       BAR_AFULL = 10, BAR_AEMPTY = 12 };
 
 template <int Q>
 __global__ void __launch_bounds__(kOutThreads, 1)
@@ -288,8 +293,10 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             mbar_init(&bars[BAR_AFULL + s], 1);
             mbar_init(&bars[BAR_AEMPTY + s], kEThreads);
         }
-        mbar_init(&bars[BAR_PFULL], kPThreads);
-        mbar_init(&bars[BAR_PEMPTY], 1);
+        for (int hf = 0; hf < 2; ++hf) {
+            mbar_init(&bars[BAR_PFULL + hf], kPThreads);
+            mbar_init(&bars[BAR_PEMPTY + hf], 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -342,24 +349,32 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             umma_commit(&bars[BAR_S]);
             constexpr uint32_t idYd = idesc_bf16_f32(128, 64, false, true);
             constexpr uint32_t idYo = idesc_bf16_f32(128, 64, false, false);
+            const int nhalf = R / 128;
             for (int j = 0; j < heads_per_cta; ++j) {
                 const int s = j & 1, use = j >> 1;
                 if (!mbar_wait_or_abort(&bars[BAR_XFULL + s], use & 1, err, abort_flag)) break;
-                if (!mbar_wait_or_abort(&bars[BAR_PFULL], j & 1, err, abort_flag)) break;
                 if (j >= 2 && !mbar_wait_or_abort(&bars[BAR_AEMPTY + s], (use - 1) & 1, err, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t acc = tmem + 256 + s * 128;
                 const uint32_t aX = smem_u32(slot_base(s) + L::kXo), aH = smem_u32(slot_base(s) + L::kHo);
-                for (int ks = 0; ks < R / 16; ++ks)
-                    umma_f16(acc, smem_desc_sw128(aP + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
-                             smem_desc_sw128(aX + ks * 2048, Q * 128, 1024), idYd, ks > 0 ? 1u : 0u);
-                umma_commit(&bars[BAR_PEMPTY]);
+                // Yo = C_i H_c^T needs no P: issue it first
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
                     umma_f16(acc + 64, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
                              smem_desc_sw128(aH + kb * 8192 + off, 16, 1024), idYo, ks > 0 ? 1u : 0u);
                 }
+                bool good = true;
+                for (int hf = 0; hf < nhalf && good; ++hf) {
+                    good = mbar_wait_or_abort(&bars[BAR_PFULL + hf], j & 1, err, abort_flag);
+                    if (!good) break;
+                    tc_fence_after();
+                    for (int ks = hf * 8; ks < hf * 8 + 8; ++ks)
+                        umma_f16(acc, smem_desc_sw128(aP + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
+                                 smem_desc_sw128(aX + ks * 2048, Q * 128, 1024), idYd, ks > 0 ? 1u : 0u);
+                    umma_commit(&bars[BAR_PEMPTY + hf]);
+                }
+                if (!good) break;
                 umma_commit(&bars[BAR_AFULL + s]);
             }
         }
@@ -373,55 +388,67 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
         bool live = mbar_wait_or_abort(&bars[BAR_S], 0, err, abort_flag);
         tc_fence_after();
+        const int nhalf = R / 128;
         for (int j = 0; j < heads_per_cta; ++j) {
             const int s = j & 1, use = j >> 1;
             live = live && mbar_wait_or_abort(&bars[BAR_XFULL + s], use & 1, err, abort_flag);
-            // all P threads agree before touching the slot (no thread may leave the
-            // named barrier below while another still waits in it)
+            // all P threads agree before touching the slot (no thread may leave a named
+            // barrier while another still waits in it)
             if (!named_bar_and(1, kPThreads, live)) break;
             const float* sLam = reinterpret_cast<const float*>(slot_base(s) + L::kLo);
             const float* sDt = reinterpret_cast<const float*>(slot_base(s) + L::kDo);
             float* sV = reinterpret_cast<float*>(slot_base(s) + L::kVo);
             for (int si = ptid; si < R; si += kPThreads)
                 sV[si] = expf(sLam[si | 31] - sLam[si]) * sDt[si];
-            // the previous head's GEMM must have read P before it is overwritten; this
-            // barrier also publishes sV to all P threads
-            if (j >= 1) live = mbar_wait_or_abort(&bars[BAR_PEMPTY], (j - 1) & 1, err, abort_flag);
-            if (!named_bar_and(1, kPThreads, live)) break;
             const float lam_t = sLam[tl];
-            for (int kc = colhalf; kc < R / 32; kc += 2) {
-                const int s0 = kc * 32;
-                uint32_t v[32];
-                tmem_ld32(trow + s0, v);
-                tmem_wait_ld();
-                uint32_t pk[16];
-                if (s0 + 31 <= tl) {
-                    const float u = expf(lam_t - sLam[s0 + 31]);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * u * sV[s0 + 2 * e],
-                                            __uint_as_float(v[2 * e + 1]) * u * sV[s0 + 2 * e + 1]);
-                } else if (s0 > tl) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int sa = s0 + 2 * e, sb = sa + 1;
-                        const float pa = sa <= tl ? __uint_as_float(v[2 * e]) * expf(lam_t - sLam[sa]) * sDt[sa] : 0.f;
-                        const float pb = sb <= tl ? __uint_as_float(v[2 * e + 1]) * expf(lam_t - sLam[sb]) * sDt[sb] : 0.f;
-                        pk[e] = pack_bf16x2(pa, pb);
-                    }
+            for (int hf = 0; hf < nhalf; ++hf) {
+                // the previous head's GEMM must be done with this half of P; the barrier
+                // also publishes sV to all P threads
+                if (j >= 1) live = mbar_wait_or_abort(&bars[BAR_PEMPTY + hf], (j - 1) & 1, err, abort_flag);
+                if (!named_bar_and(1, kPThreads, live)) {
+                    live = false;
+                    break;
                 }
-                uint8_t* blk = sP + (kc >> 1) * kBox;
+                const int kc0 = hf * 4 + colhalf, kc1 = kc0 + 2;
+                uint32_t v0[32], v1[32];
+                tmem_ld32(trow + kc0 * 32, v0);
+                tmem_ld32(trow + kc1 * 32, v1);
+                tmem_wait_ld();
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4)
-                    *reinterpret_cast<uint4*>(blk + sw128(r, (kc & 1) * 4 + k4)) =
-                        make_uint4(pk[4 * k4], pk[4 * k4 + 1], pk[4 * k4 + 2], pk[4 * k4 + 3]);
+                for (int w2 = 0; w2 < 2; ++w2) {
+                    const int kc = w2 ? kc1 : kc0;
+                    const uint32_t* v = w2 ? v1 : v0;
+                    const int s0 = kc * 32;
+                    uint32_t pk[16];
+                    if (s0 + 31 <= tl) {
+                        const float u = expf(lam_t - sLam[s0 + 31]);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * u * sV[s0 + 2 * e],
+                                                __uint_as_float(v[2 * e + 1]) * u * sV[s0 + 2 * e + 1]);
+                    } else if (s0 > tl) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int sa = s0 + 2 * e, sb = sa + 1;
+                            const float pa = sa <= tl ? __uint_as_float(v[2 * e]) * expf(lam_t - sLam[sa]) * sDt[sa] : 0.f;
+                            const float pb = sb <= tl ? __uint_as_float(v[2 * e + 1]) * expf(lam_t - sLam[sb]) * sDt[sb] : 0.f;
+                            pk[e] = pack_bf16x2(pa, pb);
+                        }
+                    }
+                    uint8_t* blk = sP + (kc >> 1) * kBox;
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        *reinterpret_cast<uint4*>(blk + sw128(r, (kc & 1) * 4 + k4)) =
+                            make_uint4(pk[4 * k4], pk[4 * k4 + 1], pk[4 * k4 + 2], pk[4 * k4 + 3]);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bars[BAR_PFULL + hf]);
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bars[BAR_PFULL]);
+            if (!live) break;                               // uniform: set only from the barrier
         }
     } else if (warp >= kWarpE0) {
         // ---- epilogue: y = Yd + exp(Lam_t) Yo + D x
