@@ -128,18 +128,17 @@ chunk_state_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_c
         // Operands go to the tensor cores as fp16 (3 more mantissa bits than bf16; the
         // bf16 inputs and the w x products of these workloads lie far inside fp16 range):
         // X~ = w o X and B are converted in place; a row's 16-byte chunks all belong to it.
-        for (int s = tid; s < Q; s += kScanThreads) {
-            const float w = sw[s];
-            uint4* r4 = reinterpret_cast<uint4*>(sX + s * 128);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                uint4 u = r4[q];
-                u.x = pack_f16x2(bf16lo(u.x) * w, bf16hi(u.x) * w);
-                u.y = pack_f16x2(bf16lo(u.y) * w, bf16hi(u.y) * w);
-                u.z = pack_f16x2(bf16lo(u.z) * w, bf16hi(u.z) * w);
-                u.w = pack_f16x2(bf16lo(u.w) * w, bf16hi(u.w) * w);
-                r4[q] = u;
-            }
+        // consecutive threads take consecutive 16-byte chunks (bank-conflict free);
+        // chunk i belongs to row i / 8 whatever its swizzled position
+        for (int i = tid; i < Q * 8; i += kScanThreads) {
+            const float w = sw[i >> 3];
+            uint4* ch = reinterpret_cast<uint4*>(sX) + i;
+            uint4 u = *ch;
+            u.x = pack_f16x2(bf16lo(u.x) * w, bf16hi(u.x) * w);
+            u.y = pack_f16x2(bf16lo(u.y) * w, bf16hi(u.y) * w);
+            u.z = pack_f16x2(bf16lo(u.z) * w, bf16hi(u.z) * w);
+            u.w = pack_f16x2(bf16lo(u.w) * w, bf16hi(u.w) * w);
+            *ch = u;
         }
         for (int i = tid; i < 2 * Q * 8; i += kScanThreads) {
             uint4* ch = reinterpret_cast<uint4*>(sB) + i;
@@ -210,9 +209,13 @@ chunk_state_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_c
         himg_s[(kb * 8192 + p * 128 + ((qn ^ (p & 7)) << 4) + jn * 2) >> 1] =
             *reinterpret_cast<const uint16_t*>(&hb);
     }
-    __threadfence();
+    // the CTA barrier orders every thread's hand-off stores before thread 0's fence,
+    // which makes them visible at GPU scope before the flag (cumulativity)
     __syncthreads();
-    if (tid == 0 && !last) st_release_gpu(flags + bh, c + 1);
+    if (tid == 0 && !last) {
+        __threadfence();
+        st_release_gpu(flags + bh, c + 1);
+    }
 
     // bf16 image of H_c for the output kernel
     uint4* dst = reinterpret_cast<uint4*>(himg + ((size_t)bh * nchunks + c) * kHImage);
