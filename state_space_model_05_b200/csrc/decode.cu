@@ -10,10 +10,10 @@
 // The step is bound by HBM: every state element is read once and written once
 // (8 bytes) for about five flops.  Design: one CTA of 8 warps per (b, h); each
 // warp owns consecutive state rows (one row = dstate fp32 = 512 B at N=128) and
-// issues ROWS 16-byte row loads before using any of them.  Four CTAs stay resident
-// per SM (<= 64 registers, ROWS = 4 at N <= 128): measured on B200 this keeps
-// more bytes in flight than fewer, larger batches per thread.  B_t and C_t are read once per CTA into
-// registers (lane j holds elements 4j..4j+3).  The y reduction along dstate is a
+// issues ROWS 16-byte row loads before using any of them.  At dstate <= 128 four
+// CTAs stay resident per SM (<= 64 registers, ROWS = 4): measured on B200 this
+// keeps more bytes in flight than fewer, larger batches per thread.  B_t and C_t
+// are read once per CTA into registers (lane j holds elements 4j..4j+3).  The y reduction along dstate is a
 // warp shuffle tree; the state is written back with 16-byte stores.
 #include "common.cuh"
 
@@ -33,7 +33,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 // QPL: float4 quads of a state row per lane (dstate <= 128 * QPL).
 // ROWS: rows a warp holds in flight at once.
 template <typename T, int QPL, int ROWS>
-__global__ void __launch_bounds__(kDecodeThreads, 4)
+__global__ void __launch_bounds__(kDecodeThreads, QPL == 1 ? 4 : 2)
 decode_step_kernel(float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
                    const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
                    const float* __restrict__ D, T* __restrict__ y, int nheads, int headdim,
