@@ -206,6 +206,14 @@ def reduce_sum(value: float, world: int) -> float:
     return float(t.item())
 
 
+def whole_job_rate(units_local: float, ms_local: float, world: int):
+    """Weak scaling: every rank processed its own units in ms_local of device time.
+    Returns (units of all ranks / max-over-ranks time in s, max-over-ranks ms)."""
+    ms_max = reduce_max(ms_local, world)
+    units = reduce_sum(units_local, world)
+    return units / (ms_max / 1e3), ms_max
+
+
 # ------------------------------------------------------------------ our arm
 def _dev(a, dtype):
     import torch
@@ -265,9 +273,9 @@ def run_prefill(w, steps, warmup, rank, world, name, e2e=True):
     status = ssd.ssd_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after {name}")
-    ms_max = reduce_max(ms, world)
+    rate, ms_max = whole_job_rate(b * T * steps, ms, world)
     tokens = b * T * steps * world
-    res = {"ms_total": ms_max, "ms_per_step": ms_max / steps, "tokens_per_s": tokens / (ms_max / 1e3),
+    res = {"ms_total": ms_max, "ms_per_step": ms_max / steps, "tokens_per_s": rate,
            "kernels": kernels, "replicas": replicas, "launches": sum(v[1] for v in kernels.values())}
 
     if e2e:
@@ -298,10 +306,10 @@ def run_prefill(w, steps, warmup, rank, world, name, e2e=True):
         s1.record()
         torch.cuda.synchronize()
         barrier(world)
-        ems = reduce_max(s0.elapsed_time(s1), world)
+        erate, _ = whole_job_rate(b * T * steps, s0.elapsed_time(s1), world)
         h2d = sum(t.numel() * t.element_size() for t in (hx, hdt, hB, hC))
         d2h = hy.numel() * hy.element_size() + hst.numel() * hst.element_size()
-        res["e2e"] = {"value": tokens / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        res["e2e"] = {"value": erate, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                       "d2h_bytes_per_step": d2h}
     return res
 
@@ -354,7 +362,8 @@ def run_decode(w, repeats, warmup, rank, world):
     s1.record()
     torch.cuda.synchronize()
     barrier(world)
-    ms = reduce_max(s0.elapsed_time(s1), world)
+    steps_total = S * repeats
+    rate, ms = whole_job_rate(steps_total, s0.elapsed_time(s1), world)
     gp = capture(True)                               # same loop with an event pair per launch
     gp.replay()
     torch.cuda.synchronize()
@@ -362,10 +371,9 @@ def run_decode(w, repeats, warmup, rank, world):
     status = ssd.ssd_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after decode")
-    steps_total = S * repeats
     kms, klaunch = kernels.get("decode_step", (float("nan"), 0))
     nbytes = decode_bytes(w)
-    res = {"steps_per_s": steps_total * world / (ms / 1e3), "ms_per_step": ms / steps_total,
+    res = {"steps_per_s": rate, "ms_per_step": ms / steps_total,
            "gbs": nbytes * steps_total / (ms / 1e3) / 1e9, "kernel_ms": kms / max(klaunch, 1),
            "launches": steps_total, "bytes_per_step": nbytes}
     del g, gp
