@@ -14,6 +14,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libssd.so")
+GEN_LIB = os.path.join(HERE, "libssd_inputs.so")
+GEN_SRC = os.path.join(CSRC, "gen", "gen_inputs.cu")
 
 SOURCES = ["api.cu", "decode.cu", "prefill_simt.cu", "prefill_tc.cu", "prefill_noalloc.cu"]
 HEADERS = ["common.cuh", "ptx.cuh", "prefill_tc.h"]
@@ -41,7 +43,18 @@ def stale(target: str = LIB) -> bool:
     return any(os.path.getmtime(f) > t for f in _inputs())
 
 
+def build_inputs(force: bool = False) -> str:
+    """The seeded device input generator (random draws only), a library of its own."""
+    deps = [GEN_SRC, os.path.join(INCLUDE, "ssd_inputs.h")]
+    if force or not os.path.exists(GEN_LIB) or any(os.path.getmtime(f) > os.path.getmtime(GEN_LIB) for f in deps):
+        subprocess.check_call([nvcc(), *ARCH, "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
+                               "-I", INCLUDE, "-o", GEN_LIB + ".tmp", GEN_SRC])
+        os.replace(GEN_LIB + ".tmp", GEN_LIB)
+    return GEN_LIB
+
+
 def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+    build_inputs(force)
     if not force and not stale():
         return LIB
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",

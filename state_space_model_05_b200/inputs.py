@@ -211,3 +211,93 @@ def dt_table() -> np.ndarray:
     k = np.arange(1 << DT_TABLE_BITS, dtype=np.float64)
     lo, hi = math.log(DT_MIN), math.log(DT_MAX)
     return np.exp(lo + (k + 0.5) / (1 << DT_TABLE_BITS) * (hi - lo)).astype(np.float32)
+
+
+# --------------------------------------------------------------------------------------
+# Device-side twin of the counter-based generator (libssd_inputs.so, include/ssd_inputs.h),
+# for workloads too large to draw on the host.  Same definitions as philox_normal /
+# philox_uniform_index above; the two produce bit-identical values.
+# --------------------------------------------------------------------------------------
+_gen_lib = None
+
+
+def _gen():
+    global _gen_lib
+    if _gen_lib is None:
+        import ctypes
+        import os
+        path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssd_inputs.so")
+        if not os.path.exists(path):
+            raise RuntimeError(f"input generator library not built: {path} is missing")
+        lib = ctypes.CDLL(path)
+        P, Z, U64, U32, F, I = (ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint64, ctypes.c_uint32,
+                                ctypes.c_float, ctypes.c_int)
+        lib.ssd_gen_normal.argtypes = [P, Z, U64, U32, F, U64, P]
+        lib.ssd_gen_normal.restype = I
+        lib.ssd_gen_table.argtypes = [P, Z, P, I, U64, U32, U64, P]
+        lib.ssd_gen_table.restype = I
+        _gen_lib = lib
+    return _gen_lib
+
+
+def _cuda_stream():
+    import ctypes
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def device_normal(out, seed: int, stream_id: int, scale: float = 1.0, first_index: int = 0):
+    """Fill the contiguous fp32 CUDA tensor `out` with philox_normal(stream_id, i) * scale."""
+    import ctypes
+    rc = _gen().ssd_gen_normal(ctypes.c_void_p(out.data_ptr()), out.numel(), seed, stream_id,
+                               float(np.float32(scale)), first_index, _cuda_stream())
+    if rc:
+        raise RuntimeError(f"ssd_gen_normal failed ({rc})")
+    return out
+
+
+def device_table(out, table, bits: int, seed: int, stream_id: int, first_index: int = 0):
+    """Fill `out` with table[philox_uniform_index(stream_id, i, bits)] (table on the device)."""
+    import ctypes
+    rc = _gen().ssd_gen_table(ctypes.c_void_p(out.data_ptr()), out.numel(),
+                              ctypes.c_void_p(table.data_ptr()), bits, seed, stream_id, first_index,
+                              _cuda_stream())
+    if rc:
+        raise RuntimeError(f"ssd_gen_table failed ({rc})")
+    return out
+
+
+# Stream numbering of the deep decode stack (L layers, fresh inputs every step): one
+# Philox stream per (tensor, layer, step); element indices follow the tensor's layout.
+DEEP_X, DEEP_B, DEEP_C, DEEP_DT, DEEP_STATE = 0, 1, 2, 3, 4
+DEEP_SEED = 0
+
+
+def deep_stream(tensor: int, layer: int, step: int = 0) -> int:
+    assert 0 <= tensor < 16 and 0 <= layer < 4096 and 0 <= step < 65536
+    return (tensor << 28) | (layer << 16) | step
+
+
+def deep_head_params(layer: int, nheads: int):
+    """A_h, D_h of one layer (host draws, PCG64 seeded by the layer index)."""
+    rng = np.random.Generator(np.random.PCG64(1000 + layer))
+    A, D, _ = head_params(rng, nheads)
+    return A, D
+
+
+def deep_unit_inputs(layer: int, b: int, h: int, steps: int, shape: SSDShape, seed: int = DEEP_SEED):
+    """Host regeneration of one (layer, batch, head) unit of the deep decode stack:
+    initial state [P][N], and per step x [P], dt, B [N], C [N]."""
+    P, N, H, G = shape.headdim, shape.dstate, shape.nheads, shape.ngroups
+    g = h // (H // G)
+    st = philox_normal(deep_stream(DEEP_STATE, layer), (b * H + h) * P * N + np.arange(P * N), seed)
+    xs, dts, Bs, Cs = [], [], [], []
+    inv = np.float32(1.0 / math.sqrt(N))
+    table = dt_table()
+    for k in range(steps):
+        xs.append(philox_normal(deep_stream(DEEP_X, layer, k), (b * H + h) * P + np.arange(P), seed))
+        Bs.append(philox_normal(deep_stream(DEEP_B, layer, k), (b * G + g) * N + np.arange(N), seed) * inv)
+        Cs.append(philox_normal(deep_stream(DEEP_C, layer, k), (b * G + g) * N + np.arange(N), seed) * inv)
+        dts.append(table[philox_uniform_index(deep_stream(DEEP_DT, layer, k), np.array([b * H + h]),
+                                              seed, DT_TABLE_BITS)][0])
+    return (st.reshape(P, N), np.stack(xs), np.array(dts, dtype=np.float32), np.stack(Bs), np.stack(Cs))
