@@ -142,6 +142,16 @@ ssd_status_t ssd_prefill_noalloc(const void* x, const float* dt, const float* A,
                                  float* final_state, void* stream);
 
 /*
+ * Diagnostic: runs the library's bounded device waits against conditions that never
+ * become true (an mbarrier nothing arrives on, a flag nothing sets), with short
+ * limits.  Both waits expire, so after it the device error word holds SSD_ERR_TIMEOUT
+ * (read it with ssd_device_status) and the CUDA context stays usable.  `scratch` is 3
+ * ints of device memory: [0] is the flag, [1] and [2] receive 1 if the mbarrier wait,
+ * respectively the flag wait, completed (0 when it gave up, as expected).
+ */
+ssd_status_t ssd_selftest_bounded_waits(int* scratch, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears this device's error word.
  * Returns SSD_OK, SSD_ERR_TIMEOUT (a bounded wait expired in a kernel since
  * the last call), or SSD_ERR_CUDA when the stream reports a CUDA error.

@@ -34,6 +34,7 @@ SIGNATURES = {
     "ssd_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ssd_prefill_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P], _I),
     "ssd_device_status": ([_P], _I),
+    "ssd_selftest_bounded_waits": ([_P, _P], _I),
     "ssd_profile_enable": ([_I], None),
     "ssd_profile_reset": ([], None),
     "ssd_profile_read": ([_I, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_double),

@@ -171,13 +171,7 @@ chunk_state_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_c
 
     // ---- look-back: the state at the start of this chunk
     if (c > 0 && tid == 0) {
-        uint32_t it = 0;
-        while (ld_acquire_gpu(flags + bh) < c) {
-            if (++it > (1u << 24)) {
-                record_error(err, SSD_ERR_TIMEOUT);
-                break;
-            }
-        }
+        wait_flag_geq(flags + bh, c, err);
         __threadfence();
     }
     __syncthreads();

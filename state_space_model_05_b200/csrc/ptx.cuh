@@ -92,6 +92,16 @@ __device__ __forceinline__ void st_release_gpu(int* p, int v) {
     asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Bounded spin until *flag >= value (acquire).  On expiry records SSD_ERR_TIMEOUT and
+// returns false.
+__device__ __forceinline__ bool wait_flag_geq(const int* flag, int value, int* err,
+                                              uint32_t max_iters = (1u << 24)) {
+    for (uint32_t it = 0; it < max_iters; ++it)
+        if (ld_acquire_gpu(flag) >= value) return true;
+    record_error(err, SSD_ERR_TIMEOUT);
+    return false;
+}
+
 // ---------------------------------------------------------------- proxies / TMA
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -127,3 +127,7 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         binding.lib()
+
+
+def test_selftest_rejects_null_scratch(lib):
+    assert lib.ssd_selftest_bounded_waits(None, None) == 1
