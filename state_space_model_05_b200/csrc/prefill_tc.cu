@@ -225,33 +225,51 @@ chunk_state_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_c
 }
 
 // ================================================================ chunk output
+// One CTA per (chunk c, 128-token tile i, head group, batch b); warp 0 issues TMA and
+// bulk loads, warp 1 issues tcgen05.mma, warps 4-11 build the masked operands, warps
+// 12-15 run the epilogue.  With t the tile's tokens (chunk-relative, 128 i .. 128 i + 127):
+//
+//   G_d = C_t B_{diag}^T   (diagonal 128 x 128 block; fp32 in TMEM, shared by the heads)
+//   G_o = C_t B_{s<128}^T  (i = 1 only: off-diagonal block; bf16 in shared memory, shared)
+//   per head h (operands, P buffers and accumulators double-buffered across heads):
+//     P   = G_d o exp(Lam_t - Lam_s) o dt_s  (s <= t, diagonal block; bf16)
+//     Yd  = P X_diag
+//     Z   = G_o (v o dt o X_{s<128}),  v_s = exp(Lam_127 - Lam_s)               (i = 1)
+//     Yo  = C_t H_c^T
+//     y_t = Yd + u_t (Z + kappa Yo) + D_h x_t,   u_t = exp(Lam_t - Lam_r), kappa = exp(Lam_r)
+//   with r = 127 for i = 1 (so exp(Lam_t - Lam_s) = u_t v_s on the off-diagonal block and
+//   exp(Lam_t) = u_t kappa; every factor <= 1) and Lam_r = 0, Z = 0 for i = 0.
+// The off-diagonal block's mask thus costs a per-row and a per-column scale instead of
+// a masked matrix per head; only the diagonal block is built elementwise, and there
+// the off-diagonal 32-column sub-blocks use exp(Lam_t - Lam_q) exp(Lam_q - Lam_s) with q
+// the sub-block's last column.
 constexpr int kOutThreads = 512;
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpP0 = 4, kWarpE0 = 12;
 constexpr int kPThreads = 256, kEThreads = 128;
+constexpr uint32_t kColGd = 384, kColGo = 256;           // TMEM columns of G_d and G_o
+constexpr uint32_t kAccCols = 192;                       // per slot: Yd +0, Z +64, Yo +128
 
 template <int Q>
 struct OutSmem {
     static constexpr int kC = 0;                        // [2 n-halves][128 rows][128 B]
-    static constexpr int kB = 2 * kBox;                 // [2 n-halves][Q rows][128 B]; then P
-    static constexpr int kSlot0 = kB + 2 * Q * 128;     // per-head slots
+    static constexpr int kB = 2 * kBox;                 // [2][Q rows][128 B]; then 2 P buffers
+    static constexpr int kGo = kB + 2 * Q * 128;        // G_o bf16 [2 k-blocks][128][128 B]
+    static constexpr int kH = kGo + 2 * kBox;           // H_c image (single buffer)
+    static constexpr int kSlot0 = kH + kHImage;         // per-head slots
     static constexpr int kXo = 0;                       //   X  [Q rows][128 B]
-    static constexpr int kHo = Q * 128;                 //   H_c image (16 KB)
-    static constexpr int kLo = kHo + kHImage;           //   Lam[Q]
+    static constexpr int kLo = Q * 128;                 //   Lam[Q]
     static constexpr int kDo = kLo + Q * 4;             //   dt[Q]
     static constexpr int kVo = kDo + Q * 4;             //   column factors v[Q]
     static constexpr int kSlotBytes = (kVo + Q * 4 + 1023) / 1024 * 1024;
     static constexpr int kBar = kSlot0 + 2 * kSlotBytes;
-    static constexpr int kNumBars = 14;
+    static constexpr int kNumBars = 20;
     static constexpr int kSlotTm = kBar + kNumBars * 8;
     static constexpr int kAbort = kSlotTm + 4;
     static constexpr int kBytes = kAbort + 12 + 1024;
 };
 
-// P is produced and consumed in K-halves of 128 source columns (the halves alternate
-// between the two 32 KB halves of the P buffer), so the P warps build half 0 of head
-// j + 1 while the tensor core still multiplies half 1 of head j.
-enum { BAR_CB = 0, BAR_S = 1, BAR_XFULL = 2, BAR_XEMPTY = 4, BAR_PFULL = 6, BAR_PEMPTY = 8,
-       BAR_AFULL = 10, BAR_AEMPTY = 12 };
+enum { BAR_CB = 0, BAR_S = 1, BAR_GO = 2, BAR_HFULL = 3, BAR_HEMPTY = 4, BAR_XFULL = 5,
+       BAR_XEMPTY = 7, BAR_PFULL = 9, BAR_PEMPTY = 11, BAR_AFULL = 13, BAR_AEMPTY = 15 };
 
 template <int Q>
 __global__ void __launch_bounds__(kOutThreads, 1)
@@ -267,7 +285,8 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     uint8_t* sm = align1024(smem_raw);
     uint8_t* sC = sm + L::kC;
     uint8_t* sB = sm + L::kB;
-    uint8_t* sP = sB;                                   // B is dead once G is computed
+    uint8_t* sGo = sm + L::kGo;
+    uint8_t* sH = sm + L::kH;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::kSlotTm);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kAbort);
@@ -277,6 +296,7 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     const int h0 = hg * heads_per_cta;
     const int g = h0 / (nheads / ngroups);
     const int R = 128 * (it + 1);                       // source tokens s in [0, R)
+    const int d0 = 128 * it;                            // first column of the diagonal block
     const int t0 = c * Q;
     const int qlen = min(Q, seqlen - t0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -284,15 +304,16 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     if (tid == 0) {
         mbar_init(&bars[BAR_CB], 1);
         mbar_init(&bars[BAR_S], 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars[BAR_XFULL + s], 1);
-            mbar_init(&bars[BAR_XEMPTY + s], kEThreads);
-            mbar_init(&bars[BAR_AFULL + s], 1);
-            mbar_init(&bars[BAR_AEMPTY + s], kEThreads);
-        }
-        for (int hf = 0; hf < 2; ++hf) {
-            mbar_init(&bars[BAR_PFULL + hf], kPThreads);
-            mbar_init(&bars[BAR_PEMPTY + hf], 1);
+        mbar_init(&bars[BAR_GO], kPThreads);
+        mbar_init(&bars[BAR_HFULL], 1);
+        mbar_init(&bars[BAR_HEMPTY], 1);
+        for (int s2 = 0; s2 < 2; ++s2) {
+            mbar_init(&bars[BAR_XFULL + s2], 1);
+            mbar_init(&bars[BAR_XEMPTY + s2], kEThreads);
+            mbar_init(&bars[BAR_PFULL + s2], kPThreads);
+            mbar_init(&bars[BAR_PEMPTY + s2], 1);
+            mbar_init(&bars[BAR_AFULL + s2], 1);
+            mbar_init(&bars[BAR_AEMPTY + s2], kEThreads);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -307,7 +328,8 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     tc_fence_after();
     const uint32_t tmem = *tslot;
 
-    auto slot_base = [&](int s) { return sm + L::kSlot0 + s * L::kSlotBytes; };
+    auto slot_base = [&](int s2) { return sm + L::kSlot0 + s2 * L::kSlotBytes; };
+    auto pbuf = [&](int b2) { return sB + b2 * (2 * kBox); };
 
     if (warp == kWarpTma) {
         if (lane == 0) {
@@ -319,157 +341,209 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 tma_load_3d(sB + Q * 128 + rb * kBox, &tm_b, g * kN + 64, t0 + rb * 128, b, &bars[BAR_CB]);
             }
             for (int j = 0; j < heads_per_cta; ++j) {
-                const int s = j & 1, use = j >> 1;
-                if (j >= 2 && !mbar_wait_or_abort(&bars[BAR_XEMPTY + s], (use - 1) & 1, err, abort_flag)) break;
+                const int s2 = j & 1, use = j >> 1;
                 const int h = h0 + j;
                 const size_t bh = (size_t)b * nheads + h;
-                uint8_t* sl = slot_base(s);
-                mbar_expect_tx(&bars[BAR_XFULL + s], (it + 1) * kBox + kHImage + 2 * R * 4);
+                if (j >= 2 && !mbar_wait_or_abort(&bars[BAR_XEMPTY + s2], (use - 1) & 1, err, abort_flag)) break;
+                uint8_t* sl = slot_base(s2);
+                mbar_expect_tx(&bars[BAR_XFULL + s2], (it + 1) * kBox + 2 * R * 4);
                 for (int rb = 0; rb <= it; ++rb)
-                    tma_load_3d(sl + L::kXo + rb * kBox, &tm_x, h * kP, t0 + rb * 128, b, &bars[BAR_XFULL + s]);
-                bulk_load(sl + L::kHo, himg + (bh * nchunks + c) * kHImage, kHImage, &bars[BAR_XFULL + s]);
-                bulk_load(sl + L::kLo, lam + (bh * nchunks + c) * Q, R * 4, &bars[BAR_XFULL + s]);
-                bulk_load(sl + L::kDo, dtT + (bh * nchunks + c) * Q, R * 4, &bars[BAR_XFULL + s]);
+                    tma_load_3d(sl + L::kXo + rb * kBox, &tm_x, h * kP, t0 + rb * 128, b, &bars[BAR_XFULL + s2]);
+                bulk_load(sl + L::kLo, lam + (bh * nchunks + c) * Q, R * 4, &bars[BAR_XFULL + s2]);
+                bulk_load(sl + L::kDo, dtT + (bh * nchunks + c) * Q, R * 4, &bars[BAR_XFULL + s2]);
+                if (j >= 1 && !mbar_wait_or_abort(&bars[BAR_HEMPTY], (j - 1) & 1, err, abort_flag)) break;
+                mbar_expect_tx(&bars[BAR_HFULL], kHImage);
+                bulk_load(sH, himg + (bh * nchunks + c) * kHImage, kHImage, &bars[BAR_HFULL]);
             }
         }
     } else if (warp == kWarpMma) {
         if (lane == 0 && mbar_wait_or_abort(&bars[BAR_CB], 0, err, abort_flag)) {
             tc_fence_after();
-            const uint32_t aC = smem_u32(sC), aB = smem_u32(sB), aP = smem_u32(sP);
+            const uint32_t aC = smem_u32(sC), aB = smem_u32(sB), aGo = smem_u32(sGo), aH = smem_u32(sH);
+            // G = C_t B_{s<R}^T into columns [512 - R, 512): G_o (i = 1) then G_d
             const uint32_t idG = idesc_bf16_f32(128, R, false, false);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
-                umma_f16(tmem, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
+                umma_f16(tmem + 512 - R, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
                          smem_desc_sw128(aB + kb * (Q * 128) + off, 16, 1024), idG, ks > 0 ? 1u : 0u);
             }
             umma_commit(&bars[BAR_S]);
-            constexpr uint32_t idYd = idesc_bf16_f32(128, 64, false, true);
-            constexpr uint32_t idYo = idesc_bf16_f32(128, 64, false, false);
-            const int nhalf = R / 128;
-            for (int j = 0; j < heads_per_cta; ++j) {
-                const int s = j & 1, use = j >> 1;
-                if (!mbar_wait_or_abort(&bars[BAR_XFULL + s], use & 1, err, abort_flag)) break;
-                if (j >= 2 && !mbar_wait_or_abort(&bars[BAR_AEMPTY + s], (use - 1) & 1, err, abort_flag)) break;
+            constexpr uint32_t idK = idesc_bf16_f32(128, 64, false, false);
+            constexpr uint32_t idMN = idesc_bf16_f32(128, 64, false, true);
+            // G_o lives in shared memory (and its TMEM columns become accumulator space)
+            bool good = it == 0 || mbar_wait_or_abort(&bars[BAR_GO], 0, err, abort_flag);
+            for (int j = 0; j < heads_per_cta && good; ++j) {
+                const int s2 = j & 1, use = j >> 1;
+                good = mbar_wait_or_abort(&bars[BAR_XFULL + s2], use & 1, err, abort_flag) &&
+                       mbar_wait_or_abort(&bars[BAR_HFULL], j & 1, err, abort_flag) &&
+                       (j < 2 || mbar_wait_or_abort(&bars[BAR_AEMPTY + s2], (use - 1) & 1, err, abort_flag));
+                if (!good) break;
                 tc_fence_after();
-                const uint32_t acc = tmem + 256 + s * 128;
-                const uint32_t aX = smem_u32(slot_base(s) + L::kXo), aH = smem_u32(slot_base(s) + L::kHo);
-                // Yo = C_i H_c^T needs no P: issue it first
+                const uint32_t acc = tmem + s2 * kAccCols;
+                const uint32_t aX = smem_u32(slot_base(s2) + L::kXo);
+                // Yo = C_t H_c^T (needs no P)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
-                    umma_f16(acc + 64, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
-                             smem_desc_sw128(aH + kb * 8192 + off, 16, 1024), idYo, ks > 0 ? 1u : 0u);
+                    umma_f16(acc + 128, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
+                             smem_desc_sw128(aH + kb * 8192 + off, 16, 1024), idK, ks > 0 ? 1u : 0u);
                 }
-                bool good = true;
-                for (int hf = 0; hf < nhalf && good; ++hf) {
-                    good = mbar_wait_or_abort(&bars[BAR_PFULL + hf], j & 1, err, abort_flag);
-                    if (!good) break;
-                    tc_fence_after();
-                    for (int ks = hf * 8; ks < hf * 8 + 8; ++ks)
-                        umma_f16(acc, smem_desc_sw128(aP + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
-                                 smem_desc_sw128(aX + ks * 2048, Q * 128, 1024), idYd, ks > 0 ? 1u : 0u);
-                    umma_commit(&bars[BAR_PEMPTY + hf]);
-                }
+                umma_commit(&bars[BAR_HEMPTY]);
+                good = mbar_wait_or_abort(&bars[BAR_PFULL + s2], use & 1, err, abort_flag);
                 if (!good) break;
-                umma_commit(&bars[BAR_AFULL + s]);
+                tc_fence_after();
+                if (it == 1) {
+                    // Z = G_o (v o dt o X_{s<128})
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        umma_f16(acc + 64, smem_desc_sw128(aGo + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
+                                 smem_desc_sw128(aX + ks * 2048, Q * 128, 1024), idMN, ks > 0 ? 1u : 0u);
+                }
+                // Yd = P X_diag
+                const uint32_t aP = smem_u32(pbuf(s2));
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_f16(acc, smem_desc_sw128(aP + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
+                             smem_desc_sw128(aX + d0 * 128 + ks * 2048, Q * 128, 1024), idMN, ks > 0 ? 1u : 0u);
+                umma_commit(&bars[BAR_PEMPTY + s2]);
+                umma_commit(&bars[BAR_AFULL + s2]);
             }
         }
     } else if (warp >= kWarpP0 && warp < kWarpE0) {
-        // ---- P = G o L o dt for this thread's row, half of the 32-column blocks
         const int pw = warp - kWarpP0;
         const int q = warp & 3, colhalf = pw >> 2;
-        const int r = q * 32 + lane;
-        const int tl = it * 128 + r;
+        const int r = q * 32 + lane;                    // tile row
+        const int tl = d0 + r;                          // chunk-relative token
         const int ptid = tid - kWarpP0 * 32;
         const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
         bool live = mbar_wait_or_abort(&bars[BAR_S], 0, err, abort_flag);
         tc_fence_after();
-        const int nhalf = R / 128;
-        for (int j = 0; j < heads_per_cta; ++j) {
-            const int s = j & 1, use = j >> 1;
-            live = live && mbar_wait_or_abort(&bars[BAR_XFULL + s], use & 1, err, abort_flag);
-            // all P threads agree before touching the slot (no thread may leave a named
-            // barrier while another still waits in it)
-            if (!named_bar_and(1, kPThreads, live)) break;
-            const float* sLam = reinterpret_cast<const float*>(slot_base(s) + L::kLo);
-            const float* sDt = reinterpret_cast<const float*>(slot_base(s) + L::kDo);
-            float* sV = reinterpret_cast<float*>(slot_base(s) + L::kVo);
-            for (int si = ptid; si < R; si += kPThreads)
-                sV[si] = expf(sLam[si | 31] - sLam[si]) * sDt[si];
-            const float lam_t = sLam[tl];
-            for (int hf = 0; hf < nhalf; ++hf) {
-                // the previous head's GEMM must be done with this half of P; the barrier
-                // also publishes sV to all P threads
-                if (j >= 1) live = mbar_wait_or_abort(&bars[BAR_PEMPTY + hf], (j - 1) & 1, err, abort_flag);
-                if (!named_bar_and(1, kPThreads, live)) {
-                    live = false;
-                    break;
-                }
-                const int kc0 = hf * 4 + colhalf, kc1 = kc0 + 2;
+        if (it == 1) {
+            // G_o -> bf16, K-major swizzled, once for all heads
+            if (live) {
                 uint32_t v0[32], v1[32];
-                tmem_ld32(trow + kc0 * 32, v0);
-                tmem_ld32(trow + kc1 * 32, v1);
+                tmem_ld32(trow + kColGo + colhalf * 64, v0);
+                tmem_ld32(trow + kColGo + colhalf * 64 + 32, v1);
                 tmem_wait_ld();
 #pragma unroll
                 for (int w2 = 0; w2 < 2; ++w2) {
-                    const int kc = w2 ? kc1 : kc0;
                     const uint32_t* v = w2 ? v1 : v0;
-                    const int s0 = kc * 32;
-                    uint32_t pk[16];
-                    if (s0 + 31 <= tl) {
-                        const float u = expf(lam_t - sLam[s0 + 31]);
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * u * sV[s0 + 2 * e],
-                                                __uint_as_float(v[2 * e + 1]) * u * sV[s0 + 2 * e + 1]);
-                    } else if (s0 > tl) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int sa = s0 + 2 * e, sb = sa + 1;
-                            const float pa = sa <= tl ? __uint_as_float(v[2 * e]) * expf(lam_t - sLam[sa]) * sDt[sa] : 0.f;
-                            const float pb = sb <= tl ? __uint_as_float(v[2 * e + 1]) * expf(lam_t - sLam[sb]) * sDt[sb] : 0.f;
-                            pk[e] = pack_bf16x2(pa, pb);
-                        }
-                    }
-                    uint8_t* blk = sP + (kc >> 1) * kBox;
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4)
-                        *reinterpret_cast<uint4*>(blk + sw128(r, (kc & 1) * 4 + k4)) =
-                            make_uint4(pk[4 * k4], pk[4 * k4 + 1], pk[4 * k4 + 2], pk[4 * k4 + 3]);
+                        *reinterpret_cast<uint4*>(sGo + colhalf * kBox + sw128(r, w2 * 4 + k4)) = make_uint4(
+                            pack_bf16x2(__uint_as_float(v[8 * k4]), __uint_as_float(v[8 * k4 + 1])),
+                            pack_bf16x2(__uint_as_float(v[8 * k4 + 2]), __uint_as_float(v[8 * k4 + 3])),
+                            pack_bf16x2(__uint_as_float(v[8 * k4 + 4]), __uint_as_float(v[8 * k4 + 5])),
+                            pack_bf16x2(__uint_as_float(v[8 * k4 + 6]), __uint_as_float(v[8 * k4 + 7])));
                 }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive(&bars[BAR_PFULL + hf]);
             }
-            if (!live) break;                               // uniform: set only from the barrier
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[BAR_GO]);
+        }
+        for (int j = 0; j < heads_per_cta; ++j) {
+            const int s2 = j & 1, use = j >> 1;
+            live = live && mbar_wait_or_abort(&bars[BAR_XFULL + s2], use & 1, err, abort_flag);
+            // all P threads agree before touching the slot (no thread may leave a named
+            // barrier while another still waits in it)
+            if (!named_bar_and(1, kPThreads, live)) break;
+            uint8_t* sl = slot_base(s2);
+            const float* sLam = reinterpret_cast<const float*>(sl + L::kLo);
+            const float* sDt = reinterpret_cast<const float*>(sl + L::kDo);
+            float* sV = reinterpret_cast<float*>(sl + L::kVo);
+            // column factors: diagonal block (reference = last column of each 32-block);
+            // i = 1 also the off-diagonal weights exp(Lam_127 - Lam_s) dt_s
+            for (int si = ptid; si < 128; si += kPThreads)
+                sV[d0 + si] = expf(sLam[(d0 + si) | 31] - sLam[d0 + si]) * sDt[d0 + si];
+            if (it == 1)
+                for (int si = ptid; si < 128; si += kPThreads)
+                    sV[si] = expf(sLam[127] - sLam[si]) * sDt[si];
+            if (!named_bar_and(1, kPThreads, live)) break;
+            if (it == 1) {
+                // X~ = v o dt o X on rows 0..127, in place (bf16); consecutive threads take
+                // consecutive 16-byte chunks; chunk i belongs to row i / 8
+                for (int i = ptid; i < 128 * 8; i += kPThreads) {
+                    const float w = sV[i >> 3];
+                    uint4* ch = reinterpret_cast<uint4*>(sl + L::kXo) + i;
+                    uint4 u = *ch;
+                    u.x = pack_bf16x2(bf16lo(u.x) * w, bf16hi(u.x) * w);
+                    u.y = pack_bf16x2(bf16lo(u.y) * w, bf16hi(u.y) * w);
+                    u.z = pack_bf16x2(bf16lo(u.z) * w, bf16hi(u.z) * w);
+                    u.w = pack_bf16x2(bf16lo(u.w) * w, bf16hi(u.w) * w);
+                    *ch = u;
+                }
+            }
+            // the GEMMs of head j - 2 must be done with this P buffer
+            if (j >= 2) live = mbar_wait_or_abort(&bars[BAR_PEMPTY + s2], (use - 1) & 1, err, abort_flag);
+            if (!named_bar_and(1, kPThreads, live)) break;
+            const float lam_t = sLam[tl];
+            uint8_t* P = pbuf(s2);
+            const int kc0 = colhalf, kc1 = colhalf + 2;
+            uint32_t v0[32], v1[32];
+            tmem_ld32(trow + kColGd + kc0 * 32, v0);
+            tmem_ld32(trow + kColGd + kc1 * 32, v1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int w2 = 0; w2 < 2; ++w2) {
+                const int kc = w2 ? kc1 : kc0;
+                const uint32_t* v = w2 ? v1 : v0;
+                const int s0 = d0 + kc * 32;
+                uint32_t pk[16];
+                if (s0 + 31 <= tl) {
+                    const float u = expf(lam_t - sLam[s0 + 31]);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * u * sV[s0 + 2 * e],
+                                            __uint_as_float(v[2 * e + 1]) * u * sV[s0 + 2 * e + 1]);
+                } else if (s0 > tl) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int sa = s0 + 2 * e, sb = sa + 1;
+                        const float pa = sa <= tl ? __uint_as_float(v[2 * e]) * expf(lam_t - sLam[sa]) * sDt[sa] : 0.f;
+                        const float pb = sb <= tl ? __uint_as_float(v[2 * e + 1]) * expf(lam_t - sLam[sb]) * sDt[sb] : 0.f;
+                        pk[e] = pack_bf16x2(pa, pb);
+                    }
+                }
+                uint8_t* blk = P + (kc >> 1) * kBox;
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4)
+                    *reinterpret_cast<uint4*>(blk + sw128(r, (kc & 1) * 4 + k4)) =
+                        make_uint4(pk[4 * k4], pk[4 * k4 + 1], pk[4 * k4 + 2], pk[4 * k4 + 3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[BAR_PFULL + s2]);
         }
     } else if (warp >= kWarpE0) {
-        // ---- epilogue: y = Yd + exp(Lam_t) Yo + D x
+        // ---- epilogue: y = Yd + u_t (Z + kappa Yo) + D x
         const int q = warp & 3;
         const int r = q * 32 + lane;
-        const int tl = it * 128 + r;
+        const int tl = d0 + r;
         const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
         for (int j = 0; j < heads_per_cta; ++j) {
-            const int s = j & 1, use = j >> 1;
-            if (!mbar_wait_or_abort(&bars[BAR_AFULL + s], use & 1, err, abort_flag)) break;
+            const int s2 = j & 1, use = j >> 1;
+            if (!mbar_wait_or_abort(&bars[BAR_AFULL + s2], use & 1, err, abort_flag)) break;
             tc_fence_after();
             const int h = h0 + j;
-            const uint8_t* sl = slot_base(s);
-            const float lam_t = reinterpret_cast<const float*>(sl + L::kLo)[tl];
-            const float e = expf(lam_t);
+            const uint8_t* sl = slot_base(s2);
+            const float* sLam = reinterpret_cast<const float*>(sl + L::kLo);
+            const float lam_r = it == 1 ? sLam[127] : 0.f;
+            const float u = expf(sLam[tl] - lam_r);
+            const float kappa = expf(lam_r);
             const float Dh = D[h];
             const uint8_t* xrow = sl + L::kXo + tl * 128;
             __nv_bfloat16* yrow = y + (((size_t)b * seqlen + t0 + tl) * nheads + h) * kP;
-            const uint32_t acc = trow + 256 + s * 128;
+            const uint32_t acc = trow + s2 * kAccCols;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                uint32_t yd[32], yo[32];
+                uint32_t yd[32], yz[32], yo[32];
                 tmem_ld32(acc + half * 32, yd);
-                tmem_ld32(acc + 64 + half * 32, yo);
+                tmem_ld32(acc + 64 + half * 32, yz);
+                tmem_ld32(acc + 128 + half * 32, yo);
                 tmem_wait_ld();
                 if (tl < qlen) {
 #pragma unroll
@@ -481,8 +555,10 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
 #pragma unroll
                         for (int k2 = 0; k2 < 4; ++k2) {
                             const int jj = qq * 8 + 2 * k2;
-                            const float a0 = fmaf(e, __uint_as_float(yo[jj]), __uint_as_float(yd[jj])) + Dh * bf16lo(xw[k2]);
-                            const float a1 = fmaf(e, __uint_as_float(yo[jj + 1]), __uint_as_float(yd[jj + 1])) + Dh * bf16hi(xw[k2]);
+                            const float z0 = it == 1 ? __uint_as_float(yz[jj]) : 0.f;
+                            const float z1 = it == 1 ? __uint_as_float(yz[jj + 1]) : 0.f;
+                            const float a0 = fmaf(u, fmaf(kappa, __uint_as_float(yo[jj]), z0), __uint_as_float(yd[jj])) + Dh * bf16lo(xw[k2]);
+                            const float a1 = fmaf(u, fmaf(kappa, __uint_as_float(yo[jj + 1]), z1), __uint_as_float(yd[jj + 1])) + Dh * bf16hi(xw[k2]);
                             o[k2] = pack_bf16x2(a0, a1);
                         }
                         *reinterpret_cast<uint4*>(yrow + qx * 8) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -490,8 +566,8 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 }
             }
             tc_fence_before();
-            mbar_arrive(&bars[BAR_AEMPTY + s]);
-            mbar_arrive(&bars[BAR_XEMPTY + s]);
+            mbar_arrive(&bars[BAR_AEMPTY + s2]);
+            mbar_arrive(&bars[BAR_XEMPTY + s2]);
         }
     }
 
