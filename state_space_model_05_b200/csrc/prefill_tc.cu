@@ -240,9 +240,11 @@ chunk_state_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_c
 //   with r = 127 for i = 1 (so exp(Lam_t - Lam_s) = u_t v_s on the off-diagonal block and
 //   exp(Lam_t) = u_t kappa; every factor <= 1) and Lam_r = 0, Z = 0 for i = 0.
 // The off-diagonal block's mask thus costs a per-row and a per-column scale instead of
-// a masked matrix per head; only the diagonal block is built elementwise, and there
-// the off-diagonal 32-column sub-blocks use exp(Lam_t - Lam_q) exp(Lam_q - Lam_s) with q
-// the sub-block's last column.
+// a masked matrix per head; only the diagonal block is built elementwise.  There,
+// 32-column sub-blocks below the diagonal use exp(Lam_t - Lam_q) exp(Lam_q - Lam_s) with q
+// the sub-block's last column (both <= 1); sub-blocks on the diagonal use the first
+// column as reference when their own decay is below 40 (both factors within e^+-40) and
+// fall back to one exponential per element otherwise.
 constexpr int kOutThreads = 512;
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpP0 = 4, kWarpE0 = 12;
 constexpr int kPThreads = 256, kEThreads = 128;
@@ -259,8 +261,9 @@ struct OutSmem {
     static constexpr int kXo = 0;                       //   X  [Q rows][128 B]
     static constexpr int kLo = Q * 128;                 //   Lam[Q]
     static constexpr int kDo = kLo + Q * 4;             //   dt[Q]
-    static constexpr int kVo = kDo + Q * 4;             //   column factors v[Q]
-    static constexpr int kSlotBytes = (kVo + Q * 4 + 1023) / 1024 * 1024;
+    static constexpr int kVo = kDo + Q * 4;             //   column factors, block-end reference
+    static constexpr int kWo = kVo + Q * 4;             //   column factors, block-start reference
+    static constexpr int kSlotBytes = (kWo + Q * 4 + 1023) / 1024 * 1024;
     static constexpr int kBar = kSlot0 + 2 * kSlotBytes;
     static constexpr int kNumBars = 20;
     static constexpr int kSlotTm = kBar + kNumBars * 8;
@@ -452,10 +455,16 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             const float* sLam = reinterpret_cast<const float*>(sl + L::kLo);
             const float* sDt = reinterpret_cast<const float*>(sl + L::kDo);
             float* sV = reinterpret_cast<float*>(sl + L::kVo);
-            // column factors: diagonal block (reference = last column of each 32-block);
-            // i = 1 also the off-diagonal weights exp(Lam_127 - Lam_s) dt_s
-            for (int si = ptid; si < 128; si += kPThreads)
-                sV[d0 + si] = expf(sLam[(d0 + si) | 31] - sLam[d0 + si]) * sDt[d0 + si];
+            float* sW = reinterpret_cast<float*>(sl + L::kWo);
+            // column factors of the diagonal block, per 32-column sub-block: reference its
+            // last column (factor <= 1) and its first column (factor >= 1, used only where
+            // the sub-block's own decay is small); i = 1 also the off-diagonal weights
+            // exp(Lam_127 - Lam_s) dt_s
+            for (int si = ptid; si < 128; si += kPThreads) {
+                const int sg = d0 + si;
+                sV[sg] = expf(sLam[sg | 31] - sLam[sg]) * sDt[sg];
+                sW[sg] = expf(sLam[sg & ~31] - sLam[sg]) * sDt[sg];
+            }
             if (it == 1)
                 for (int si = ptid; si < 128; si += kPThreads)
                     sV[si] = expf(sLam[127] - sLam[si]) * sDt[si];
@@ -499,7 +508,20 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 } else if (s0 > tl) {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                } else if (sLam[s0] - sLam[s0 + 31] < 40.f) {
+                    // sub-block on the diagonal with modest internal decay:
+                    // exp(Lam_t - Lam_s) = exp(Lam_t - Lam_s0) exp(Lam_s0 - Lam_s), both
+                    // factors within e^+-40 (fully normal fp32)
+                    const float u = expf(lam_t - sLam[s0]);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int sa = s0 + 2 * e;
+                        const float pa = __uint_as_float(v[2 * e]) * u * sW[sa];
+                        const float pb = __uint_as_float(v[2 * e + 1]) * u * sW[sa + 1];
+                        pk[e] = pack_bf16x2(sa <= tl ? pa : 0.f, sa + 1 <= tl ? pb : 0.f);
+                    }
                 } else {
+                    // strong decay inside the sub-block: one exponential per element
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const int sa = s0 + 2 * e, sb = sa + 1;
