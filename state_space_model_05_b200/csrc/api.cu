@@ -183,11 +183,11 @@ ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const v
         if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
         const int nflags = d.batch * d.nheads + 1;
         cudaError_t e = profiled(kCumsum, s, [&] {
-            return launch_chunk_cumsum(d, dt, A, w.lam, w.dtT, w.flags, nflags, s);
+            return launch_chunk_cumsum(d, dt, A, w.lam, w.dtT, w.flags, nflags, B, w.b16, s);
         });
         if (e == cudaSuccess)
             e = profiled(kStateTc, s, [&] {
-                return launch_chunk_state_scan_tc(d, x, B, w, init_state, final_state, s);
+                return launch_chunk_state_scan_tc(d, x, w.b16, w, init_state, final_state, s);
             });
         if (e == cudaSuccess)
             e = profiled(kOutTc, s, [&] { return launch_chunk_output_tc(d, x, B, C, D, w, y, s); });
@@ -198,7 +198,7 @@ ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const v
     const size_t need = prefill_workspace_layout(d, workspace, &ws);
     if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
     cudaError_t e = profiled(kCumsum, s, [&] {
-        return launch_chunk_cumsum(d, dt, A, ws.lam, nullptr, nullptr, 0, s);
+        return launch_chunk_cumsum(d, dt, A, ws.lam, nullptr, nullptr, 0, nullptr, nullptr, s);
     });
     if (e == cudaSuccess)
         e = profiled(kStateSimt, s, [&] {

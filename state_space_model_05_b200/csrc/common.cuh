@@ -62,7 +62,8 @@ cudaError_t launch_decode(const Dims& d, ssd_dtype_t dtype, float* state, const 
                           const float* D, void* y, cudaStream_t s);
 
 cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, float* lam,
-                                float* dtT, int* zero, int nzero, cudaStream_t s);
+                                float* dtT, int* zero, int nzero, const void* b_bf16, void* b_f16,
+                                cudaStream_t s);
 cudaError_t launch_chunk_state_simt(const Dims& d, ssd_dtype_t dtype, const void* x,
                                     const float* dt, const void* B, const float* lam,
                                     float* states, cudaStream_t s);

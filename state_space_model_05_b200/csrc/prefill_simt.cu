@@ -30,17 +30,39 @@ constexpr int kThreads = 256;
 // ----------------------------------------------------------------------------------
 constexpr int kCumsumHeads = 8;      // one warp per head
 
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
+    const float lo = __uint_as_float(u << 16), hi = __uint_as_float(u & 0xFFFF0000u);
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 // Also writes dt transposed to [b][h][c][Q] when dtT is non-null (zero past seqlen),
 // and zeroes `nzero` words at `zero` (look-back flags of the tensor-core path).
 __global__ void __launch_bounds__(kThreads)
 chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
                     float* __restrict__ lam, float* __restrict__ dtT, int* __restrict__ zero,
-                    int nzero, int seqlen, int nheads, int Q, int nchunks)
+                    int nzero, const uint4* __restrict__ b_bf16, uint4* __restrict__ b_f16,
+                    int b_row_chunks, int seqlen, int nheads, int Q, int nchunks)
 {
     extern __shared__ float sm_dt[];                   // [Q][kCumsumHeads]
     const int c = blockIdx.x, h0 = blockIdx.y * kCumsumHeads, b = blockIdx.z;
     if (zero && c == 0 && blockIdx.y == 0 && b == 0)
         for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
+    if (b_f16 && blockIdx.y == 0) {
+        // fp16 copy of this chunk's rows of B (bf16 -> fp16 is exact for these values'
+        // range), the operand format of the tensor-core chunk-state GEMM
+        const int rows = min(Q, seqlen - c * Q);
+        const size_t first = ((size_t)b * seqlen + (size_t)c * Q) * b_row_chunks;
+        for (int i = threadIdx.x; i < rows * b_row_chunks; i += blockDim.x) {
+            uint4 u = b_bf16[first + i];
+            u.x = bf16x2_to_f16x2(u.x);
+            u.y = bf16x2_to_f16x2(u.y);
+            u.z = bf16x2_to_f16x2(u.z);
+            u.w = bf16x2_to_f16x2(u.w);
+            b_f16[first + i] = u;
+        }
+    }
     const int nh = min(kCumsumHeads, nheads - h0);
     const int t0 = c * Q;
     for (int i = threadIdx.x; i < Q * kCumsumHeads; i += blockDim.x) {
@@ -363,13 +385,15 @@ size_t simt_output_smem_bytes(int headdim, int dstate)
 }
 
 cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, float* lam,
-                                float* dtT, int* zero, int nzero, cudaStream_t s)
+                                float* dtT, int* zero, int nzero, const void* b_bf16, void* b_f16,
+                                cudaStream_t s)
 {
     if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
     const size_t smem = sizeof(float) * d.chunk_len * kCumsumHeads;
     dim3 grid(d.nchunks, (d.nheads + kCumsumHeads - 1) / kCumsumHeads, d.batch);
-    chunk_cumsum_kernel<<<grid, kThreads, smem, s>>>(dt, A, lam, dtT, zero, nzero, d.seqlen,
-                                                     d.nheads, d.chunk_len, d.nchunks);
+    chunk_cumsum_kernel<<<grid, kThreads, smem, s>>>(
+        dt, A, lam, dtT, zero, nzero, static_cast<const uint4*>(b_bf16), static_cast<uint4*>(b_f16),
+        d.ngroups * d.dstate / 8, d.seqlen, d.nheads, d.chunk_len, d.nchunks);
     return cudaGetLastError();
 }
 

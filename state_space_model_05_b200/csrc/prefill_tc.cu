@@ -127,7 +127,7 @@ chunk_state_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_c
     if (ok) {
         // Operands go to the tensor cores as fp16 (3 more mantissa bits than bf16; the
         // bf16 inputs and the w x products of these workloads lie far inside fp16 range):
-        // X~ = w o X and B are converted in place; a row's 16-byte chunks all belong to it.
+        // B arrives as the fp16 copy the cumsum kernel wrote; X~ = w o X is converted here.
         // consecutive threads take consecutive 16-byte chunks (bank-conflict free);
         // chunk i belongs to row i / 8 whatever its swizzled position
         for (int i = tid; i < Q * 8; i += kScanThreads) {
@@ -138,15 +138,6 @@ chunk_state_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_c
             u.y = pack_f16x2(bf16lo(u.y) * w, bf16hi(u.y) * w);
             u.z = pack_f16x2(bf16lo(u.z) * w, bf16hi(u.z) * w);
             u.w = pack_f16x2(bf16lo(u.w) * w, bf16hi(u.w) * w);
-            *ch = u;
-        }
-        for (int i = tid; i < 2 * Q * 8; i += kScanThreads) {
-            uint4* ch = reinterpret_cast<uint4*>(sB) + i;
-            uint4 u = *ch;
-            u.x = pack_f16x2(bf16lo(u.x), bf16hi(u.x));
-            u.y = pack_f16x2(bf16lo(u.y), bf16hi(u.y));
-            u.z = pack_f16x2(bf16lo(u.z), bf16hi(u.z));
-            u.w = pack_f16x2(bf16lo(u.w), bf16hi(u.w));
             *ch = u;
         }
     }
@@ -165,11 +156,8 @@ chunk_state_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_c
         }
         umma_commit(&bars[1]);
     }
-    if (ok) ok = mbar_wait(&bars[1], 0, err);
-    ok = __syncthreads_and(ok);
-    tc_fence_after();
-
-    // ---- look-back: the state at the start of this chunk
+    // ---- look-back while the tensor core computes S_c: the state at the start of this
+    // chunk (the predecessor's flag, then its hand-off slot)
     if (c > 0 && tid == 0) {
         wait_flag_geq(flags + bh, c, err);
         __threadfence();
@@ -186,13 +174,16 @@ chunk_state_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_c
     float* hdst = last ? final_state + (size_t)bh * kP * kN : ring_bh + (size_t)((c + 1) & 1) * kP * kN;
     uint16_t* himg_s = reinterpret_cast<uint16_t*>(sX);            // X~ is no longer needed
     const int kb = n >> 6, qn = (n & 63) >> 3, jn = n & 7;
-    uint32_t v[32];
-    tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + half * 32, v);
     float hc[32];
     // all loads of the carried state first (the hand-off ring is read and written by
     // this CTA, so loads must not wait behind the stores)
 #pragma unroll
     for (int pp = 0; pp < 32; ++pp) hc[pp] = hsrc ? __ldcg(hsrc + (half * 32 + pp) * kN + n) : 0.f;
+    if (ok) ok = mbar_wait(&bars[1], 0, err);
+    ok = __syncthreads_and(ok);
+    tc_fence_after();
+    uint32_t v[32];
+    tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + half * 32, v);
     tmem_wait_ld();
 #pragma unroll
     for (int pp = 0; pp < 32; ++pp) {
@@ -277,7 +268,8 @@ enum { BAR_CB = 0, BAR_S = 1, BAR_GO = 2, BAR_HFULL = 3, BAR_HEMPTY = 4, BAR_XFU
 template <int Q>
 __global__ void __launch_bounds__(kOutThreads, 1)
 chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-                    const __grid_constant__ CUtensorMap tm_c, const float* __restrict__ lam,
+                    const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
+                    const float* __restrict__ lam,
                     const float* __restrict__ dtT, const uint8_t* __restrict__ himg,
                     const float* __restrict__ D, __nv_bfloat16* __restrict__ y, int seqlen,
                     int nheads, int ngroups, int nchunks, int heads_per_cta, int* err)
@@ -312,7 +304,7 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         mbar_init(&bars[BAR_HEMPTY], 1);
         for (int s2 = 0; s2 < 2; ++s2) {
             mbar_init(&bars[BAR_XFULL + s2], 1);
-            mbar_init(&bars[BAR_XEMPTY + s2], kEThreads);
+            mbar_init(&bars[BAR_XEMPTY + s2], 1);
             mbar_init(&bars[BAR_PFULL + s2], kPThreads);
             mbar_init(&bars[BAR_PEMPTY + s2], 1);
             mbar_init(&bars[BAR_AFULL + s2], 1);
@@ -541,24 +533,25 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             mbar_arrive(&bars[BAR_PFULL + s2]);
         }
     } else if (warp >= kWarpE0) {
-        // ---- epilogue: y = Yd + u_t (Z + kappa Yo) + D x
+        // ---- epilogue: y = Yd + u_t (Z + kappa Yo) + D x, written in place over the
+        // tile's x rows (each thread its own row), then one TMA store of the tile
         const int q = warp & 3;
         const int r = q * 32 + lane;
         const int tl = d0 + r;
+        const int etid = tid - kWarpE0 * 32;
         const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
         for (int j = 0; j < heads_per_cta; ++j) {
             const int s2 = j & 1, use = j >> 1;
             if (!mbar_wait_or_abort(&bars[BAR_AFULL + s2], use & 1, err, abort_flag)) break;
             tc_fence_after();
             const int h = h0 + j;
-            const uint8_t* sl = slot_base(s2);
+            uint8_t* sl = slot_base(s2);
             const float* sLam = reinterpret_cast<const float*>(sl + L::kLo);
             const float lam_r = it == 1 ? sLam[127] : 0.f;
             const float u = expf(sLam[tl] - lam_r);
             const float kappa = expf(lam_r);
             const float Dh = D[h];
-            const uint8_t* xrow = sl + L::kXo + tl * 128;
-            __nv_bfloat16* yrow = y + (((size_t)b * seqlen + t0 + tl) * nheads + h) * kP;
+            uint8_t* xrow = sl + L::kXo + tl * 128;
             const uint32_t acc = trow + s2 * kAccCols;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -567,30 +560,37 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 tmem_ld32(acc + 64 + half * 32, yz);
                 tmem_ld32(acc + 128 + half * 32, yo);
                 tmem_wait_ld();
-                if (tl < qlen) {
 #pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) {
-                        const int qx = half * 4 + qq;
-                        const uint4 xu = *reinterpret_cast<const uint4*>(xrow + ((qx ^ (tl & 7)) << 4));
-                        const uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w};
-                        uint32_t o[4];
+                for (int qq = 0; qq < 4; ++qq) {
+                    const int qx = half * 4 + qq;
+                    uint4* xp = reinterpret_cast<uint4*>(xrow + ((qx ^ (tl & 7)) << 4));
+                    const uint4 xu = *xp;
+                    const uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w};
+                    uint32_t o[4];
 #pragma unroll
-                        for (int k2 = 0; k2 < 4; ++k2) {
-                            const int jj = qq * 8 + 2 * k2;
-                            const float z0 = it == 1 ? __uint_as_float(yz[jj]) : 0.f;
-                            const float z1 = it == 1 ? __uint_as_float(yz[jj + 1]) : 0.f;
-                            const float a0 = fmaf(u, fmaf(kappa, __uint_as_float(yo[jj]), z0), __uint_as_float(yd[jj])) + Dh * bf16lo(xw[k2]);
-                            const float a1 = fmaf(u, fmaf(kappa, __uint_as_float(yo[jj + 1]), z1), __uint_as_float(yd[jj + 1])) + Dh * bf16hi(xw[k2]);
-                            o[k2] = pack_bf16x2(a0, a1);
-                        }
-                        *reinterpret_cast<uint4*>(yrow + qx * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+                    for (int k2 = 0; k2 < 4; ++k2) {
+                        const int jj = qq * 8 + 2 * k2;
+                        const float z0 = it == 1 ? __uint_as_float(yz[jj]) : 0.f;
+                        const float z1 = it == 1 ? __uint_as_float(yz[jj + 1]) : 0.f;
+                        const float a0 = fmaf(u, fmaf(kappa, __uint_as_float(yo[jj]), z0), __uint_as_float(yd[jj])) + Dh * bf16lo(xw[k2]);
+                        const float a1 = fmaf(u, fmaf(kappa, __uint_as_float(yo[jj + 1]), z1), __uint_as_float(yd[jj + 1])) + Dh * bf16hi(xw[k2]);
+                        o[k2] = pack_bf16x2(a0, a1);
                     }
+                    *xp = make_uint4(o[0], o[1], o[2], o[3]);
                 }
             }
             tc_fence_before();
             mbar_arrive(&bars[BAR_AEMPTY + s2]);
-            mbar_arrive(&bars[BAR_XEMPTY + s2]);
+            fence_proxy_async_smem();                       // y rows -> visible to the TMA unit
+            named_bar_sync(2, kEThreads);
+            if (etid == 0) {
+                tma_store_3d(&tm_y, h * kP, t0 + d0, b, sl + L::kXo + d0 * 128);
+                bulk_commit_group();
+                bulk_wait_group_read0();                    // the slot may be refilled now
+                mbar_arrive(&bars[BAR_XEMPTY + s2]);
+            }
         }
+        if (etid == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     }
 
     tc_fence_before();
@@ -615,8 +615,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
-// bf16 tensor [outer][rows][inner] read in boxes of 64 (inner) x 128 (rows), 128B swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer)
+// 16-bit tensor [outer][rows][inner] read in boxes of 64 (inner) x 128 (rows), 128B swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
+              CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
 {
     auto fn = encode_fn();
     if (!fn) return false;
@@ -624,7 +625,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
     cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
     cuuint32_t box[3] = {64, 128, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+    return fn(m, type, 3, const_cast<void*>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -657,7 +658,7 @@ cudaError_t scan_t(const Dims& d, const CUtensorMap& mx, const CUtensorMap& mb, 
 
 template <int Q>
 cudaError_t output_t(const Dims& d, const CUtensorMap& mx, const CUtensorMap& mb, const CUtensorMap& mc,
-                     const TcWorkspace& w, const float* D, void* y, cudaStream_t s)
+                     const CUtensorMap& my, const TcWorkspace& w, const float* D, void* y, cudaStream_t s)
 {
     auto k = chunk_output_kernel<Q>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -665,7 +666,7 @@ cudaError_t output_t(const Dims& d, const CUtensorMap& mx, const CUtensorMap& mb
     if (e != cudaSuccess) return e;
     const int hpc = heads_per_cta(d);
     dim3 grid(d.nchunks * (Q / 128), d.nheads / hpc, d.batch);
-    k<<<grid, kOutThreads, OutSmem<Q>::kBytes, s>>>(mx, mb, mc, w.lam, w.dtT, w.himg, D,
+    k<<<grid, kOutThreads, OutSmem<Q>::kBytes, s>>>(mx, mb, mc, my, w.lam, w.dtT, w.himg, D,
                                                     static_cast<__nv_bfloat16*>(y), d.seqlen,
                                                     d.nheads, d.ngroups, d.nchunks, hpc,
                                                     device_error_word());
@@ -687,6 +688,7 @@ size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w)
     const size_t ring_b = up(BH * 2 * kP * kN * sizeof(float));
     const size_t himg_b = up(BH * d.nchunks * kHImage);
     const size_t flag_b = up((BH + 1) * sizeof(int));
+    const size_t b16_b = up((size_t)d.batch * d.seqlen * d.ngroups * kN * 2);
     if (w) {
         char* p = static_cast<char*>(base);
         w->lam = reinterpret_cast<float*>(p);
@@ -694,18 +696,19 @@ size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w)
         w->ring = reinterpret_cast<float*>(p + 2 * lam_b);
         w->himg = reinterpret_cast<uint8_t*>(p + 2 * lam_b + ring_b);
         w->flags = reinterpret_cast<int*>(p + 2 * lam_b + ring_b + himg_b);
+        w->b16 = p + 2 * lam_b + ring_b + himg_b + flag_b;
     }
-    return 2 * lam_b + ring_b + himg_b + flag_b;
+    return 2 * lam_b + ring_b + himg_b + flag_b + b16_b;
 }
 
-cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void* B,
+cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void* B_f16,
                                        const TcWorkspace& w, const float* init_state,
                                        float* final_state, cudaStream_t s)
 {
     if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
     CUtensorMap mx, mb;
     if (!make_map(&mx, x, (uint64_t)d.nheads * kP, d.seqlen, d.batch) ||
-        !make_map(&mb, B, (uint64_t)d.ngroups * kN, d.seqlen, d.batch))
+        !make_map(&mb, B_f16, (uint64_t)d.ngroups * kN, d.seqlen, d.batch, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
         return cudaErrorInvalidValue;
     if (d.chunk_len == 256) return scan_t<256>(d, mx, mb, w, init_state, final_state, s);
     return scan_t<128>(d, mx, mb, w, init_state, final_state, s);
@@ -715,13 +718,14 @@ cudaError_t launch_chunk_output_tc(const Dims& d, const void* x, const void* B, 
                                    const float* D, const TcWorkspace& w, void* y, cudaStream_t s)
 {
     if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
-    CUtensorMap mx, mb, mc;
+    CUtensorMap mx, mb, mc, my;
     if (!make_map(&mx, x, (uint64_t)d.nheads * kP, d.seqlen, d.batch) ||
         !make_map(&mb, B, (uint64_t)d.ngroups * kN, d.seqlen, d.batch) ||
-        !make_map(&mc, C, (uint64_t)d.ngroups * kN, d.seqlen, d.batch))
+        !make_map(&mc, C, (uint64_t)d.ngroups * kN, d.seqlen, d.batch) ||
+        !make_map(&my, y, (uint64_t)d.nheads * kP, d.seqlen, d.batch))
         return cudaErrorInvalidValue;
-    if (d.chunk_len == 256) return output_t<256>(d, mx, mb, mc, w, D, y, s);
-    return output_t<128>(d, mx, mb, mc, w, D, y, s);
+    if (d.chunk_len == 256) return output_t<256>(d, mx, mb, mc, my, w, D, y, s);
+    return output_t<128>(d, mx, mb, mc, my, w, D, y, s);
 }
 
 }  // namespace ssd
