@@ -56,13 +56,18 @@ struct PrefillWorkspace {
 };
 size_t prefill_workspace_layout(const Dims& d, void* base, PrefillWorkspace* ws);
 
+constexpr int kMaxChunk = 256;               // largest chunk length Q
+
 // ---- launchers (return cudaGetLastError() of their launches) -----------------------
 cudaError_t launch_decode(const Dims& d, ssd_dtype_t dtype, float* state, const void* x,
                           const float* dt, const float* A, const void* B, const void* C,
                           const float* D, void* y, cudaStream_t s);
 
+// Lambda (within-chunk cumulative sum of dt A) for every (b, h, chunk) row; optionally
+// dt transposed to the same layout, the chunk-state weights exp(Lambda_end - Lambda) dt,
+// and an fp16 copy of a bf16 B.  Null outputs are skipped.
 cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, float* lam,
-                                float* dtT, int* zero, int nzero, const void* b_bf16, void* b_f16,
+                                float* dtT, float* wts, const void* b_bf16, void* b_f16,
                                 cudaStream_t s);
 cudaError_t launch_chunk_state_simt(const Dims& d, ssd_dtype_t dtype, const void* x,
                                     const float* dt, const void* B, const float* lam,

@@ -41,20 +41,21 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
 // and zeroes `nzero` words at `zero` (look-back flags of the tensor-core path).
 __global__ void __launch_bounds__(kThreads)
 chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
-                    float* __restrict__ lam, float* __restrict__ dtT, int* __restrict__ zero,
-                    int nzero, const uint4* __restrict__ b_bf16, uint4* __restrict__ b_f16,
+                    float* __restrict__ lam, float* __restrict__ dtT, float* __restrict__ wts,
+                    const uint4* __restrict__ b_bf16, uint4* __restrict__ b_f16,
                     int b_row_chunks, int seqlen, int nheads, int Q, int nchunks)
 {
     extern __shared__ float sm_dt[];                   // [Q][kCumsumHeads]
     const int c = blockIdx.x, h0 = blockIdx.y * kCumsumHeads, b = blockIdx.z;
-    if (zero && c == 0 && blockIdx.y == 0 && b == 0)
-        for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
-    if (b_f16 && blockIdx.y == 0) {
+    if (b_f16) {
         // fp16 copy of this chunk's rows of B (bf16 -> fp16 is exact for these values'
-        // range), the operand format of the tensor-core chunk-state GEMM
+        // range), the operand format of the tensor-core chunk-state GEMM; the head blocks
+        // of a chunk split its rows between them
         const int rows = min(Q, seqlen - c * Q);
-        const size_t first = ((size_t)b * seqlen + (size_t)c * Q) * b_row_chunks;
-        for (int i = threadIdx.x; i < rows * b_row_chunks; i += blockDim.x) {
+        const int r0 = (int)(((long long)rows * blockIdx.y) / gridDim.y);
+        const int r1 = (int)(((long long)rows * (blockIdx.y + 1)) / gridDim.y);
+        const size_t first = ((size_t)b * seqlen + (size_t)c * Q + r0) * b_row_chunks;
+        for (int i = threadIdx.x; i < (r1 - r0) * b_row_chunks; i += blockDim.x) {
             uint4 u = b_bf16[first + i];
             u.x = bf16x2_to_f16x2(u.x);
             u.y = bf16x2_to_f16x2(u.y);
@@ -78,8 +79,11 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
         const float Ah = A[h0 + hh];
         float carry = 0.f;
         const size_t row = (((size_t)b * nheads + h0 + hh) * nchunks + c) * Q;
-        for (int base = 0; base < Q; base += 32) {
-            const int t = base + lane;
+        float lv[kMaxChunk / 32], dv[kMaxChunk / 32];
+#pragma unroll
+        for (int j = 0; j < kMaxChunk / 32; ++j) {
+            const int t = j * 32 + lane;
+            if (j * 32 >= Q) break;
             const float d = (t < Q) ? sm_dt[t * kCumsumHeads + hh] : 0.f;
             float v = d * Ah;
 #pragma unroll
@@ -92,7 +96,18 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
                 lam[row + t] = v;
                 if (dtT) dtT[row + t] = d;
             }
+            lv[j] = v;
+            dv[j] = d;
             carry = __shfl_sync(0xffffffffu, v, 31);
+        }
+        if (wts) {
+            // chunk-state weights w_s = exp(Lambda_end - Lambda_s) dt_s (carry = Lambda_end)
+#pragma unroll
+            for (int j = 0; j < kMaxChunk / 32; ++j) {
+                const int t = j * 32 + lane;
+                if (j * 32 >= Q) break;
+                if (t < Q) wts[row + t] = expf(carry - lv[j]) * dv[j];
+            }
         }
     }
 }
@@ -385,14 +400,14 @@ size_t simt_output_smem_bytes(int headdim, int dstate)
 }
 
 cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, float* lam,
-                                float* dtT, int* zero, int nzero, const void* b_bf16, void* b_f16,
+                                float* dtT, float* wts, const void* b_bf16, void* b_f16,
                                 cudaStream_t s)
 {
     if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
     const size_t smem = sizeof(float) * d.chunk_len * kCumsumHeads;
     dim3 grid(d.nchunks, (d.nheads + kCumsumHeads - 1) / kCumsumHeads, d.batch);
     chunk_cumsum_kernel<<<grid, kThreads, smem, s>>>(
-        dt, A, lam, dtT, zero, nzero, static_cast<const uint4*>(b_bf16), static_cast<uint4*>(b_f16),
+        dt, A, lam, dtT, wts, static_cast<const uint4*>(b_bf16), static_cast<uint4*>(b_f16),
         d.ngroups * d.dstate / 8, d.seqlen, d.nheads, d.chunk_len, d.nchunks);
     return cudaGetLastError();
 }

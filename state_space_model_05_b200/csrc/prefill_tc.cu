@@ -54,166 +54,230 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // Byte offset of 16-byte chunk q of row r in a 128B-swizzled tile.
 __device__ __forceinline__ uint32_t sw128(int r, int q) { return r * 128 + ((q ^ (r & 7)) << 4); }
 
-// ================================================================ chunk state + scan
-constexpr int kScanThreads = 256;            // warps w and w+4 share TMEM lane quarter w
+// ================================================================ chunk states: persistent walk
+// One resident CTA per (batch b, group g, range of 1-3 heads) walks the chunks of its
+// heads in order, so the carried state never leaves the CTA (registers) and no chunk
+// waits for another CTA.  The heads' chunk states form one tcgen05 chain with the heads
+// stacked along N (N = 64 x heads); B_c is staged once per chunk for all of them.
+// Operands stream through a 4-deep ring of 64-row quarter-chunk stages (fp16 B quarter,
+// one X quarter per head, the heads' weights w_s); two TMEM accumulators alternate
+// between chunks.  Warp-specialised: one warp issues the loads, one the MMAs, and eight
+// worker warps (which hold the carried state) form X~ = w o X and update the state;
+// the update of chunk c - 1 runs a stage into chunk c, once its accumulator is complete.
+constexpr int kWalkWorkers = 8;                               // warps w, w + 4: TMEM lane quarter w
+constexpr int kWalkThreads = (kWalkWorkers + 2) * 32;         // + load warp + MMA warp
+constexpr int kWalkHeads = 3;                                 // heads per CTA (at most)
+constexpr int kWalkStages = 4;
+constexpr int kQBox = 8192;                                   // one 64-row x 128-byte box
 
-template <int Q>
-struct ScanSmem {
-    static constexpr int kB = 0;                   // [2 n-halves][Q rows][128 B]
-    static constexpr int kX = 2 * Q * 128;         // [Q rows][128 B]; later the H_c image
-    static constexpr int kW = kX + Q * 128;        // float[Q]
-    static constexpr int kBar = kW + Q * 4;        // 2 mbarriers
-    static constexpr int kSlot = kBar + 16;        // TMEM address
-    static constexpr int kTicket = kSlot + 4;
-    static constexpr int kBytes = kTicket + 12 + 1024;
+struct WalkSmem {
+    static constexpr int kStageX = 2 * kQBox;                         // after the B quarter
+    static constexpr int kStageW = kStageX + kWalkHeads * kQBox;      // float[heads][64]
+    static constexpr int kStageBytes = kStageW + 1024;                // 41 KB
+    static constexpr int kBar = kWalkStages * kStageBytes;            // full, conv, empty, acc
+    static constexpr int kSlot = kBar + (3 * kWalkStages + 2) * 8;
+    static constexpr int kBytes = kSlot + 16 + 1024;
+};
+static_assert(WalkSmem::kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
+static_assert(WalkSmem::kBytes <= 227 * 1024, "walk shared memory");
+
+struct WalkMaps {
+    CUtensorMap x1, x2;          // x as (P, T, H, b), boxes of 1 / 2 heads x 64 rows
+    CUtensorMap b;               // fp16 B as (64, T, 2G, b), box: both halves x 64 rows
+    CUtensorMap w;               // weights as (nchunks Q, b H) fp32, box 64 x 3 heads
 };
 
 template <int Q>
-__global__ void __launch_bounds__(kScanThreads, 2)
-chunk_state_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-                        const float* __restrict__ lam, const float* __restrict__ dtT,
+__global__ void __launch_bounds__(kWalkThreads, 1)
+chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __restrict__ lam,
                         const float* __restrict__ init_state, float* final_state,
-                        float* __restrict__ ring, uint8_t* __restrict__ himg, int* flags,
-                        int* ticket, int batch, int nheads, int ngroups, int nchunks, int* err)
+                        uint8_t* __restrict__ himg, int nheads, int ngroups, int nchunks,
+                        int ctas_per_group, int* err)
 {
-    using L = ScanSmem<Q>;
+    using L = WalkSmem;
+    constexpr int NQ = Q / 64;                          // stages per chunk
+    constexpr int S = kWalkStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
-    uint8_t* sB = sm + L::kB;
-    uint8_t* sX = sm + L::kX;
-    float* sw = reinterpret_cast<float*>(sm + L::kW);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::kBar);
+    uint64_t* conv = full + S;
+    uint64_t* empty = conv + S;
+    uint64_t* accb = empty + S;
     uint32_t* slot = reinterpret_cast<uint32_t*>(sm + L::kSlot);
-    int* sticket = reinterpret_cast<int*>(sm + L::kTicket);
 
+    // this CTA's heads: a contiguous range of one (b, g)
+    const int hpg = nheads / ngroups;
+    const int unit = blockIdx.x / ctas_per_group, part = blockIdx.x - unit * ctas_per_group;
+    const int b = unit / ngroups, g = unit - b * ngroups;
+    const int hlo = g * hpg + (part * hpg) / ctas_per_group;
+    const int nh = g * hpg + ((part + 1) * hpg) / ctas_per_group - hlo;     // 1..3
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int total = nchunks * NQ;
+    auto stage = [&](int st) { return sm + st * L::kStageBytes; };
+
     if (tid == 0) {
-        *sticket = atomicAdd(ticket, 1);
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
+        for (int i = 0; i < S; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&conv[i], kWalkWorkers);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(&accb[0], 1);
+        mbar_init(&accb[1], 1);
         fence_mbar_init();
-        fence_proxy_async_smem();
     }
-    if (warp == 0) {
-        tmem_alloc(slot, 64);
+    if (warp == kWalkWorkers + 1) {
+        tmem_alloc(slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *slot;
-    const int BH = batch * nheads;
-    const int k = *sticket;
-    const int c = k / BH, bh = k - c * BH;
-    const int b = bh / nheads, h = bh - b * nheads;
-    const int g = h / (nheads / ngroups);
-    const int t0 = c * Q;
 
-    if (tid == 0) {
-        mbar_expect_tx(&bars[0], 3 * Q * 128);
+    if (warp == kWalkWorkers) {
+        // ---------------------------------------------------------------- loads
+        if (lane == 0) {
+            int issued = 0;
+            for (int k = 0; k < total; ++k) {
+                const int st = k % S;
+                if (k >= S && !mbar_wait(&empty[st], ((k / S) + 1) & 1, err)) break;
+                const int c = k / NQ, row = c * Q + (k - c * NQ) * 64;
+                uint8_t* sg = stage(st);
+                mbar_expect_tx(&full[st], (2 + nh) * kQBox + kWalkHeads * 256);
+                tma_load_4d(sg, &maps.b, 0, row, 2 * g, b, &full[st]);
+                int hh = 0;
+                if (nh >= 2) {
+                    tma_load_4d(sg + L::kStageX + hh * kQBox, &maps.x2, 0, row, hlo + hh, b, &full[st]);
+                    hh += 2;
+                }
+                if (nh - hh >= 1)
+                    tma_load_4d(sg + L::kStageX + hh * kQBox, &maps.x1, 0, row, hlo + hh, b, &full[st]);
+                tma_load_2d(sg + L::kStageW, &maps.w, row, b * nheads + hlo, &full[st]);
+                issued = k + 1;
+            }
+            // the CTA does not exit with loads in flight
+            for (int k = max(0, issued - S); k < issued; ++k) mbar_wait(&full[k % S], (k / S) & 1, err);
+        }
+    } else if (warp == kWalkWorkers + 1) {
+        // ---------------------------------------------------------------- MMAs
+        if (lane == 0) {
+            const uint32_t idesc = idesc_f16_f32(128, 64 * nh, true, true);
+            int done = 0;
+            for (int k = 0; k < total; ++k) {
+                const int st = k % S, c = k / NQ, qq = k - c * NQ;
+                if (!mbar_wait(&conv[st], (k / S) & 1, err)) break;
+                tc_fence_after();
+                const uint32_t aB = smem_u32(stage(st)), aX = aB + L::kStageX;
+                // S_c[n][64 hh + p] += sum_s B_s[n] X~_s[hh][p] over this stage's 64 rows
 #pragma unroll
-        for (int rb = 0; rb < Q / 128; ++rb) {
-            tma_load_3d(sB + rb * kBox, &tm_b, g * kN, t0 + rb * 128, b, &bars[0]);
-            tma_load_3d(sB + Q * 128 + rb * kBox, &tm_b, g * kN + 64, t0 + rb * 128, b, &bars[0]);
-            tma_load_3d(sX + rb * kBox, &tm_x, h * kP, t0 + rb * 128, b, &bars[0]);
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_f16(tmem + (c & 1) * 256, smem_desc_sw128(aB + ks * 2048, kQBox, 1024),
+                             smem_desc_sw128(aX + ks * 2048, kQBox, 1024), idesc,
+                             (qq > 0 || ks > 0) ? 1u : 0u);
+                umma_commit(&empty[st]);
+                if (qq == NQ - 1) umma_commit(&accb[c & 1]);
+                done = k + 1;
+            }
+            // the CTA does not release TMEM with MMAs in flight
+            if (done > 0) mbar_wait(&empty[(done - 1) % S], ((done - 1) / S) & 1, err);
+        }
+    } else {
+        // ---------------------------------------------------------------- workers
+        // carried state: thread owns column n and rows p = 32 half + pp, for each head
+        const int n = (warp & 3) * 32 + lane;
+        const int half = warp >> 2;
+        const int kb = n >> 6, qn = (n & 63) >> 3, jn = n & 7;
+        float Hs[kWalkHeads][32];
+#pragma unroll
+        for (int hh = 0; hh < kWalkHeads; ++hh) {
+#pragma unroll
+            for (int pp = 0; pp < 32; ++pp) {
+                const int p = half * 32 + pp;
+                Hs[hh][pp] = (hh < nh && init_state)
+                                 ? init_state[((size_t)(b * nheads + hlo + hh) * kP + p) * kN + n] : 0.f;
+            }
+        }
+        bool ok = true;
+
+        // state update for chunk cc: write the bf16 image of H_cc, then H <- exp(Lam_end) H + S_cc
+        auto update = [&](int cc) {
+            float e[kWalkHeads];
+#pragma unroll
+            for (int hh = 0; hh < kWalkHeads; ++hh)
+                e[hh] = hh < nh ? lam[((size_t)(b * nheads + hlo + hh) * nchunks + cc) * Q + Q - 1] : 0.f;
+            if (ok) ok = mbar_wait(&accb[cc & 1], (cc >> 1) & 1, err);
+            tc_fence_after();
+            const uint32_t acc = tmem + (cc & 1) * 256 + ((uint32_t)((warp & 3) * 32) << 16) + half * 32;
+#pragma unroll
+            for (int hh = 0; hh < kWalkHeads; ++hh) {
+                if (hh < nh) {                           // uniform across the CTA
+                    const float eh = expf(e[hh]);
+                    uint16_t* img = reinterpret_cast<uint16_t*>(
+                        himg + ((size_t)(b * nheads + hlo + hh) * nchunks + cc) * kHImage);
+#pragma unroll
+                    for (int q16 = 0; q16 < 2; ++q16) {
+                        uint32_t v[16];
+                        tmem_ld16(acc + hh * 64 + q16 * 16, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int pp = q16 * 16 + j, p = half * 32 + pp;
+                            const __nv_bfloat16 hbv = __float2bfloat16_rn(Hs[hh][pp]);
+                            img[(kb * 8192 + p * 128 + ((qn ^ (p & 7)) << 4) + jn * 2) >> 1] =
+                                *reinterpret_cast<const uint16_t*>(&hbv);
+                            Hs[hh][pp] = fmaf(eh, Hs[hh][pp], ok ? __uint_as_float(v[j]) : 0.f);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+        };
+
+        for (int k = 0; k < total; ++k) {
+            const int st = k % S, c = k / NQ, qq = k - c * NQ;
+            if (ok) ok = mbar_wait(&full[st], (k / S) & 1, err);
+            if (ok) {
+                // X~ = w o X -> fp16 in place; consecutive threads take consecutive
+                // 16-byte chunks; chunk i: head i / 512, row (i / 8) % 64
+                uint8_t* sx = stage(st) + L::kStageX;
+                const float* sw = reinterpret_cast<const float*>(stage(st) + L::kStageW);
+                for (int i = tid; i < nh * 512; i += kWalkWorkers * 32) {
+                    const float w = sw[(i >> 9) * 64 + ((i >> 3) & 63)];
+                    uint4* ch = reinterpret_cast<uint4*>(sx) + i;
+                    uint4 u = *ch;
+                    u.x = pack_f16x2(bf16lo(u.x) * w, bf16hi(u.x) * w);
+                    u.y = pack_f16x2(bf16lo(u.y) * w, bf16hi(u.y) * w);
+                    u.z = pack_f16x2(bf16lo(u.z) * w, bf16hi(u.z) * w);
+                    u.w = pack_f16x2(bf16lo(u.w) * w, bf16hi(u.w) * w);
+                    *ch = u;
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&conv[st]);
+            if (qq == 1 && c > 0) update(c - 1);
+        }
+        if (nchunks > 0) update(nchunks - 1);
+#pragma unroll
+        for (int hh = 0; hh < kWalkHeads; ++hh) {
+            if (hh < nh) {
+#pragma unroll
+                for (int pp = 0; pp < 32; ++pp) {
+                    const int p = half * 32 + pp;
+                    final_state[((size_t)(b * nheads + hlo + hh) * kP + p) * kN + n] = Hs[hh][pp];
+                }
+            }
         }
     }
-    const size_t row = ((size_t)bh * nchunks + c) * Q;
-    const float lam_end = lam[row + Q - 1];
-    for (int s = tid; s < Q; s += kScanThreads) sw[s] = expf(lam_end - lam[row + s]) * dtT[row + s];
-    __syncthreads();
-
-    bool ok = mbar_wait(&bars[0], 0, err);
-    if (ok) {
-        // Operands go to the tensor cores as fp16 (3 more mantissa bits than bf16; the
-        // bf16 inputs and the w x products of these workloads lie far inside fp16 range):
-        // B arrives as the fp16 copy the cumsum kernel wrote; X~ = w o X is converted here.
-        // consecutive threads take consecutive 16-byte chunks (bank-conflict free);
-        // chunk i belongs to row i / 8 whatever its swizzled position
-        for (int i = tid; i < Q * 8; i += kScanThreads) {
-            const float w = sw[i >> 3];
-            uint4* ch = reinterpret_cast<uint4*>(sX) + i;
-            uint4 u = *ch;
-            u.x = pack_f16x2(bf16lo(u.x) * w, bf16hi(u.x) * w);
-            u.y = pack_f16x2(bf16lo(u.y) * w, bf16hi(u.y) * w);
-            u.z = pack_f16x2(bf16lo(u.z) * w, bf16hi(u.z) * w);
-            u.w = pack_f16x2(bf16lo(u.w) * w, bf16hi(u.w) * w);
-            *ch = u;
-        }
-    }
-    fence_proxy_async_smem();
-    ok = __syncthreads_and(ok);
-
-    if (tid == 0 && ok) {
-        tc_fence_after();
-        constexpr uint32_t idesc = idesc_f16_f32(128, 64, true, true);
-        const uint32_t aB = smem_u32(sB), aX = smem_u32(sX);
-#pragma unroll
-        for (int ks = 0; ks < Q / 16; ++ks) {
-            const uint64_t ad = smem_desc_sw128(aB + ks * 2048, Q * 128, 1024);
-            const uint64_t bd = smem_desc_sw128(aX + ks * 2048, Q * 128, 1024);
-            umma_f16(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
-        }
-        umma_commit(&bars[1]);
-    }
-    // ---- look-back while the tensor core computes S_c: the state at the start of this
-    // chunk (the predecessor's flag, then its hand-off slot)
-    if (c > 0 && tid == 0) {
-        wait_flag_geq(flags + bh, c, err);
-        __threadfence();
-    }
-    __syncthreads();
-
-    const int n = (warp & 3) * 32 + lane;           // TMEM lane = state column n
-    const int half = warp >> 2;                     // rows p in [32 half, 32 half + 32)
-    const float ec = expf(lam_end);
-    float* ring_bh = ring + (size_t)bh * 2 * kP * kN;
-    const float* hsrc = c == 0 ? (init_state ? init_state + (size_t)bh * kP * kN : nullptr)
-                               : ring_bh + (size_t)(c & 1) * kP * kN;
-    const bool last = c == nchunks - 1;
-    float* hdst = last ? final_state + (size_t)bh * kP * kN : ring_bh + (size_t)((c + 1) & 1) * kP * kN;
-    uint16_t* himg_s = reinterpret_cast<uint16_t*>(sX);            // X~ is no longer needed
-    const int kb = n >> 6, qn = (n & 63) >> 3, jn = n & 7;
-    float hc[32];
-    // all loads of the carried state first (the hand-off ring is read and written by
-    // this CTA, so loads must not wait behind the stores)
-#pragma unroll
-    for (int pp = 0; pp < 32; ++pp) hc[pp] = hsrc ? __ldcg(hsrc + (half * 32 + pp) * kN + n) : 0.f;
-    if (ok) ok = mbar_wait(&bars[1], 0, err);
-    ok = __syncthreads_and(ok);
-    tc_fence_after();
-    uint32_t v[32];
-    tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + half * 32, v);
-    tmem_wait_ld();
-#pragma unroll
-    for (int pp = 0; pp < 32; ++pp) {
-        const int p = half * 32 + pp;
-        const float sc = ok ? __uint_as_float(v[pp]) : 0.f;
-        hdst[p * kN + n] = fmaf(ec, hc[pp], sc);
-        const __nv_bfloat16 hb = __float2bfloat16_rn(hc[pp]);
-        himg_s[(kb * 8192 + p * 128 + ((qn ^ (p & 7)) << 4) + jn * 2) >> 1] =
-            *reinterpret_cast<const uint16_t*>(&hb);
-    }
-    // the CTA barrier orders every thread's hand-off stores before thread 0's fence,
-    // which makes them visible at GPU scope before the flag (cumulativity)
-    __syncthreads();
-    if (tid == 0 && !last) {
-        __threadfence();
-        st_release_gpu(flags + bh, c + 1);
-    }
-
-    // bf16 image of H_c for the output kernel
-    uint4* dst = reinterpret_cast<uint4*>(himg + ((size_t)bh * nchunks + c) * kHImage);
-    const uint4* src = reinterpret_cast<const uint4*>(sX);
-    for (int i = tid; i < kHImage / 16; i += kScanThreads) dst[i] = src[i];
-
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == kWalkWorkers + 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 64);
+        tmem_dealloc(tmem, 512);
     }
 }
+
+
 
 // ================================================================ chunk output
 // One CTA per (chunk c, 128-token tile i, head group, batch b); warp 0 issues TMA and
@@ -615,18 +679,38 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
-// 16-bit tensor [outer][rows][inner] read in boxes of 64 (inner) x 128 (rows), 128B swizzle.
+// 16-bit tensor [outer][rows][inner] read in boxes of 64 (inner) x box_rows, 128B swizzle.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
-              CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
+              CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, uint32_t box_rows = 128)
 {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {inner, rows, outer};
     cuuint64_t strides[2] = {inner * 2, inner * rows * 2};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, type, 3, const_cast<void*>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tiled map of `rank` dimensions (dim 0 contiguous; strides in bytes for dims 1..rank-1),
+// 128-byte swizzle or none; out-of-range elements read as zero.
+bool encode_map(CUtensorMap* m, CUtensorMapDataType type, int rank, const void* base,
+                const uint64_t* dims, const uint64_t* strides, const uint32_t* box, bool swizzle)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gd[5], gs[4];
+    cuuint32_t bx[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        gd[i] = dims[i];
+        bx[i] = box[i];
+        es[i] = 1;
+        if (i) gs[i - 1] = strides[i - 1];
+    }
+    return fn(m, type, rank, const_cast<void*>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -640,19 +724,40 @@ int heads_per_cta(const Dims& d)
     return 1;
 }
 
-template <int Q>
-cudaError_t scan_t(const Dims& d, const CUtensorMap& mx, const CUtensorMap& mb, const TcWorkspace& w,
-                   const float* init_state, float* final_state, cudaStream_t s)
+int sm_count()
 {
-    auto k = chunk_state_scan_kernel<Q>;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cache[dev] && cudaDeviceGetAttribute(&cache[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        cache[dev] = 148;
+    return cache[dev];
+}
+
+// CTAs per (b, g) of the walk: enough that each holds at most 3 heads, and as many as
+// fill the SMs otherwise (never more than there are heads).
+int walk_ctas_per_group(const Dims& d)
+{
+    const int hpg = d.nheads / d.ngroups;
+    const int units = d.batch * d.ngroups;
+    int cpg = (hpg + kWalkHeads - 1) / kWalkHeads;
+    cpg = max(cpg, sm_count() / units);
+    return min(cpg, hpg);
+}
+
+template <int Q>
+cudaError_t walk_t(const Dims& d, const WalkMaps& maps, const TcWorkspace& w, const float* init_state,
+                   float* final_state, cudaStream_t s)
+{
+    auto k = chunk_state_walk_kernel<Q>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         ScanSmem<Q>::kBytes);
+                                         WalkSmem::kBytes);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)((size_t)d.nchunks * d.batch * d.nheads);
-    k<<<grid, kScanThreads, ScanSmem<Q>::kBytes, s>>>(mx, mb, w.lam, w.dtT, init_state, final_state,
-                                                      w.ring, w.himg, w.flags, w.flags + d.batch * d.nheads,
-                                                      d.batch, d.nheads, d.ngroups, d.nchunks,
-                                                      device_error_word());
+    const int cpg = walk_ctas_per_group(d);
+    const unsigned grid = (unsigned)(d.batch * d.ngroups * cpg);
+    k<<<grid, kWalkThreads, WalkSmem::kBytes, s>>>(maps, w.lam, init_state, final_state, w.himg,
+                                                    d.nheads, d.ngroups, d.nchunks, cpg,
+                                                    device_error_word());
     return cudaGetLastError();
 }
 
@@ -685,20 +790,17 @@ size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w)
     auto up = [](size_t v) { return (v + 255) & ~size_t(255); };
     const size_t BH = (size_t)d.batch * d.nheads;
     const size_t lam_b = up(BH * d.nchunks * d.chunk_len * sizeof(float));
-    const size_t ring_b = up(BH * 2 * kP * kN * sizeof(float));
     const size_t himg_b = up(BH * d.nchunks * kHImage);
-    const size_t flag_b = up((BH + 1) * sizeof(int));
     const size_t b16_b = up((size_t)d.batch * d.seqlen * d.ngroups * kN * 2);
     if (w) {
         char* p = static_cast<char*>(base);
         w->lam = reinterpret_cast<float*>(p);
         w->dtT = reinterpret_cast<float*>(p + lam_b);
-        w->ring = reinterpret_cast<float*>(p + 2 * lam_b);
-        w->himg = reinterpret_cast<uint8_t*>(p + 2 * lam_b + ring_b);
-        w->flags = reinterpret_cast<int*>(p + 2 * lam_b + ring_b + himg_b);
-        w->b16 = p + 2 * lam_b + ring_b + himg_b + flag_b;
+        w->wts = reinterpret_cast<float*>(p + 2 * lam_b);
+        w->himg = reinterpret_cast<uint8_t*>(p + 3 * lam_b);
+        w->b16 = p + 3 * lam_b + himg_b;
     }
-    return 2 * lam_b + ring_b + himg_b + flag_b + b16_b;
+    return 3 * lam_b + himg_b + b16_b;
 }
 
 cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void* B_f16,
@@ -706,12 +808,27 @@ cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void*
                                        float* final_state, cudaStream_t s)
 {
     if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
-    CUtensorMap mx, mb;
-    if (!make_map(&mx, x, (uint64_t)d.nheads * kP, d.seqlen, d.batch) ||
-        !make_map(&mb, B_f16, (uint64_t)d.ngroups * kN, d.seqlen, d.batch, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+    const uint64_t T = d.seqlen, H = d.nheads, G = d.ngroups, Bt = d.batch;
+    WalkMaps m;
+    // x [b][T][H][P] bf16 seen as (p, t, h, b): one box = 64 rows of 1 or 2 heads
+    const uint64_t xdim[4] = {kP, T, H, Bt};
+    const uint64_t xstr[3] = {H * kP * 2, kP * 2, T * H * kP * 2};
+    const uint32_t xbox1[4] = {64, 64, 1, 1}, xbox2[4] = {64, 64, 2, 1};
+    // fp16 B [b][T][G][N] seen as (n mod 64, t, 2 g + n / 64, b)
+    const uint64_t bdim[4] = {64, T, 2 * G, Bt};
+    const uint64_t bstr[3] = {G * kN * 2, 128, T * G * kN * 2};
+    const uint32_t bbox[4] = {64, 64, 2, 1};
+    // weights [b h][c Q] fp32
+    const uint64_t wdim[2] = {(uint64_t)d.nchunks * d.chunk_len, Bt * H};
+    const uint64_t wstr[1] = {(uint64_t)d.nchunks * d.chunk_len * 4};
+    const uint32_t wbox[2] = {64, kWalkHeads};
+    if (!encode_map(&m.x1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, x, xdim, xstr, xbox1, true) ||
+        !encode_map(&m.x2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, x, xdim, xstr, xbox2, true) ||
+        !encode_map(&m.b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, B_f16, bdim, bstr, bbox, true) ||
+        !encode_map(&m.w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, w.wts, wdim, wstr, wbox, false))
         return cudaErrorInvalidValue;
-    if (d.chunk_len == 256) return scan_t<256>(d, mx, mb, w, init_state, final_state, s);
-    return scan_t<128>(d, mx, mb, w, init_state, final_state, s);
+    if (d.chunk_len == 256) return walk_t<256>(d, m, w, init_state, final_state, s);
+    return walk_t<128>(d, m, w, init_state, final_state, s);
 }
 
 cudaError_t launch_chunk_output_tc(const Dims& d, const void* x, const void* B, const void* C,

@@ -12,15 +12,15 @@ bool tc_prefill_supported(const Dims& d);
 struct TcWorkspace {
     float* lam;       // [b][h][c][Q] inclusive cumsum of dt*A within each chunk
     float* dtT;       // [b][h][c][Q] dt, zero past seqlen
-    float* ring;      // [b*h][2][64][128] fp32 hand-off slots of the carried state
+    float* wts;       // [b][h][c][Q] chunk-state weights exp(Lam_end - Lam) dt
     uint8_t* himg;    // [b][h][c] 16 KB bf16 image of each chunk's start state
-    int* flags;       // [b*h] chunks published so far, then one ticket counter
     void* b16;        // [b][T][G][N] fp16 copy of B (operand of the chunk-state GEMM)
 };
 size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w);
 
-// Chunk states and the inter-chunk scan (decoupled look-back), writing the chunk
-// start states (bf16 images) and the final state.  B_f16 is the fp16 copy of B.
+// Chunk states and the inter-chunk recurrence (persistent walk over each head's chunks),
+// writing the chunk start states (bf16 images) and the final state.  B_f16 is the fp16
+// copy of B.
 cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void* B_f16,
                                        const TcWorkspace& w, const float* init_state,
                                        float* final_state, cudaStream_t s);

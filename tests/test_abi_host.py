@@ -53,13 +53,11 @@ def test_workspace_bytes(lib):
     lam = b * H * c * Q * 4
     st = b * H * c * P * N * 4
     assert _ws(b, T, H, P, G, N, Q, binding.SSD_F32) == up(lam) + up(st)
-    # tensor-core path (bf16, P 64, N 128, Q 128/256): lam + dt^T, fp32 hand-off ring,
-    # bf16 chunk-start-state images, look-back flags + ticket, fp16 copy of B
-    ring = b * H * 2 * P * N * 4
+    # tensor-core path (bf16, P 64, N 128, Q 128/256): lam, dt^T and the chunk-state
+    # weights (same layout), bf16 chunk-start-state images, fp16 copy of B
     himg = b * H * c * 16384
-    flags = (b * H + 1) * 4
     b16 = b * T * G * N * 2          # fp16 copy of B for the chunk-state GEMM
-    assert _ws(b, T, H, P, G, N, Q, binding.SSD_BF16) == 2 * up(lam) + up(ring) + up(himg) + up(flags) + up(b16)
+    assert _ws(b, T, H, P, G, N, Q, binding.SSD_BF16) == 3 * up(lam) + up(himg) + up(b16)
     # bf16 with other shapes uses the CUDA-core layout
     assert _ws(b, T, H, P, G, N, 64, binding.SSD_BF16) == up(b * H * 5 * 64 * 4) + up(b * H * 5 * P * N * 4)
     assert _ws(b, 0, H, P, G, N, Q, binding.SSD_F32) == 0
