@@ -74,7 +74,8 @@ struct WalkSmem {
     static constexpr int kStageX = 2 * kQBox;                         // after the B quarter
     static constexpr int kStageW = kStageX + kWalkHeads * kQBox;      // float[heads][64]
     static constexpr int kStageBytes = kStageW + 1024;                // 41 KB
-    static constexpr int kBar = kWalkStages * kStageBytes;            // full, conv, empty, acc
+    static constexpr int kImg = kWalkStages * kStageBytes;            // 2 x 16 KB state images
+    static constexpr int kBar = kImg + 2 * kHImage;                   // full, conv, empty, acc
     static constexpr int kSlot = kBar + (3 * kWalkStages + 2) * 8;
     static constexpr int kBytes = kSlot + 16 + 1024;
 };
@@ -186,7 +187,6 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
         // carried state: thread owns column n and rows p = 32 half + pp, for each head
         const int n = (warp & 3) * 32 + lane;
         const int half = warp >> 2;
-        const int kb = n >> 6, qn = (n & 63) >> 3, jn = n & 7;
         float Hs[kWalkHeads][32];
 #pragma unroll
         for (int hh = 0; hh < kWalkHeads; ++hh) {
@@ -199,9 +199,14 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
         }
         bool ok = true;
 
-        // state update for chunk cc: write the bf16 image of H_cc, then H <- exp(Lam_end) H + S_cc
+        // state update for chunk cc: write the bf16 image of H_cc, then H <- exp(Lam_end) H + S_cc.
+        // The image is the MN-major (p contiguous) 128-byte-swizzled operand tile: row n holds
+        // p = 0..63, its 16-byte chunk j (p = 8j..8j+7) stored at chunk j ^ (n mod 8).  It is
+        // assembled in shared memory (two buffers, alternating per head) and written to
+        // global memory with one bulk copy by thread 0.
+        int img_count = 0;                               // images written so far (buffer parity)
         auto update = [&](int cc) {
-            float e[kWalkHeads];
+            float e[kWalkHeads];                         // Lam_end per head
 #pragma unroll
             for (int hh = 0; hh < kWalkHeads; ++hh)
                 e[hh] = hh < nh ? lam[((size_t)(b * nheads + hlo + hh) * nchunks + cc) * Q + Q - 1] : 0.f;
@@ -211,22 +216,34 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
 #pragma unroll
             for (int hh = 0; hh < kWalkHeads; ++hh) {
                 if (hh < nh) {                           // uniform across the CTA
+                    uint8_t* simg = sm + L::kImg + (img_count & 1) * kHImage;
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const float* h8 = &Hs[hh][8 * jj];
+                        const uint4 v = make_uint4(pack_bf16x2(h8[0], h8[1]), pack_bf16x2(h8[2], h8[3]),
+                                                   pack_bf16x2(h8[4], h8[5]), pack_bf16x2(h8[6], h8[7]));
+                        *reinterpret_cast<uint4*>(simg + n * 128 + (((4 * half + jj) ^ (n & 7)) << 4)) = v;
+                    }
+                    fence_proxy_async_smem();
+                    // the store of the previous image (other buffer) has read its source
+                    // before anyone passes this barrier and overwrites that buffer
+                    if (tid == 0) bulk_wait_group_read0();
+                    named_bar_sync(1, kWalkWorkers * 32);
+                    if (tid == 0) {
+                        bulk_store(himg + ((size_t)(b * nheads + hlo + hh) * nchunks + cc) * kHImage, simg,
+                                   kHImage);
+                        bulk_commit_group();
+                    }
+                    ++img_count;
                     const float eh = expf(e[hh]);
-                    uint16_t* img = reinterpret_cast<uint16_t*>(
-                        himg + ((size_t)(b * nheads + hlo + hh) * nchunks + cc) * kHImage);
 #pragma unroll
                     for (int q16 = 0; q16 < 2; ++q16) {
                         uint32_t v[16];
                         tmem_ld16(acc + hh * 64 + q16 * 16, v);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int pp = q16 * 16 + j, p = half * 32 + pp;
-                            const __nv_bfloat16 hbv = __float2bfloat16_rn(Hs[hh][pp]);
-                            img[(kb * 8192 + p * 128 + ((qn ^ (p & 7)) << 4) + jn * 2) >> 1] =
-                                *reinterpret_cast<const uint16_t*>(&hbv);
-                            Hs[hh][pp] = fmaf(eh, Hs[hh][pp], ok ? __uint_as_float(v[j]) : 0.f);
-                        }
+                        for (int j = 0; j < 16; ++j)
+                            Hs[hh][q16 * 16 + j] = fmaf(eh, Hs[hh][q16 * 16 + j], ok ? __uint_as_float(v[j]) : 0.f);
                     }
                 }
             }
@@ -239,17 +256,35 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
             if (ok) {
                 // X~ = w o X -> fp16 in place; consecutive threads take consecutive
                 // 16-byte chunks; chunk i: head i / 512, row (i / 8) % 64
-                uint8_t* sx = stage(st) + L::kStageX;
+                uint4* sx = reinterpret_cast<uint4*>(stage(st) + L::kStageX);
                 const float* sw = reinterpret_cast<const float*>(stage(st) + L::kStageW);
-                for (int i = tid; i < nh * 512; i += kWalkWorkers * 32) {
-                    const float w = sw[(i >> 9) * 64 + ((i >> 3) & 63)];
-                    uint4* ch = reinterpret_cast<uint4*>(sx) + i;
-                    uint4 u = *ch;
-                    u.x = pack_f16x2(bf16lo(u.x) * w, bf16hi(u.x) * w);
-                    u.y = pack_f16x2(bf16lo(u.y) * w, bf16hi(u.y) * w);
-                    u.z = pack_f16x2(bf16lo(u.z) * w, bf16hi(u.z) * w);
-                    u.w = pack_f16x2(bf16lo(u.w) * w, bf16hi(u.w) * w);
-                    *ch = u;
+                constexpr int kPer = kWalkHeads * 512 / (kWalkWorkers * 32);   // chunks per thread
+                constexpr int kBatch = 3;                                       // loads in flight
+                static_assert(kPer % kBatch == 0, "conversion batches");
+#pragma unroll
+                for (int j0 = 0; j0 < kPer; j0 += kBatch) {
+                    uint4 u[kBatch];
+                    float w[kBatch];
+#pragma unroll
+                    for (int j = 0; j < kBatch; ++j) {
+                        const int i = tid + (j0 + j) * kWalkWorkers * 32;
+                        if (i < nh * 512) {
+                            u[j] = sx[i];
+                            w[j] = sw[(i >> 9) * 64 + ((i >> 3) & 63)];
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < kBatch; ++j) {
+                        const int i = tid + (j0 + j) * kWalkWorkers * 32;
+                        if (i < nh * 512) {
+                            uint4 v = u[j];
+                            v.x = pack_f16x2(bf16lo(v.x) * w[j], bf16hi(v.x) * w[j]);
+                            v.y = pack_f16x2(bf16lo(v.y) * w[j], bf16hi(v.y) * w[j]);
+                            v.z = pack_f16x2(bf16lo(v.z) * w[j], bf16hi(v.z) * w[j]);
+                            v.w = pack_f16x2(bf16lo(v.w) * w[j], bf16hi(v.w) * w[j]);
+                            sx[i] = v;
+                        }
+                    }
                 }
             }
             fence_proxy_async_smem();
@@ -258,6 +293,7 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
             if (qq == 1 && c > 0) update(c - 1);
         }
         if (nchunks > 0) update(nchunks - 1);
+        if (tid == 0) bulk_wait_group0();
 #pragma unroll
         for (int hh = 0; hh < kWalkHeads; ++hh) {
             if (hh < nh) {
@@ -428,7 +464,6 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                          smem_desc_sw128(aB + kb * (Q * 128) + off, 16, 1024), idG, ks > 0 ? 1u : 0u);
             }
             umma_commit(&bars[BAR_S]);
-            constexpr uint32_t idK = idesc_bf16_f32(128, 64, false, false);
             constexpr uint32_t idMN = idesc_bf16_f32(128, 64, false, true);
             // G_o lives in shared memory (and its TMEM columns become accumulator space)
             bool good = it == 0 || mbar_wait_or_abort(&bars[BAR_GO], 0, err, abort_flag);
@@ -446,7 +481,7 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
                     umma_f16(acc + 128, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
-                             smem_desc_sw128(aH + kb * 8192 + off, 16, 1024), idK, ks > 0 ? 1u : 0u);
+                             smem_desc_sw128(aH + ks * 2048, 8192, 1024), idMN, ks > 0 ? 1u : 0u);
                 }
                 umma_commit(&bars[BAR_HEMPTY]);
                 good = mbar_wait_or_abort(&bars[BAR_PFULL + s2], use & 1, err, abort_flag);
