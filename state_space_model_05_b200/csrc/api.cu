@@ -151,7 +151,8 @@ size_t ssd_prefill_workspace_bytes(int batch, int seqlen, int nheads, int headdi
     if (prefill_dims(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len, dtype, &d) != SSD_OK)
         return 0;
     if (d.nchunks == 0 || d.batch == 0) return 0;
-    if (dtype == SSD_BF16 && tc_prefill_supported(d)) return tc_workspace_layout(d, nullptr, nullptr);
+    if (dtype == SSD_BF16 && tc_prefill_supported(d))
+        return tc_workspace_layout(tc_block_dims(d), nullptr, nullptr);
     return prefill_workspace_layout(d, nullptr, nullptr);
 }
 
@@ -178,18 +179,19 @@ ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const v
         return SSD_ERR_ALIGN;
     const bool tc = dtype == SSD_BF16 && tc_prefill_supported(d);
     if (tc) {
+        const Dims t = tc_block_dims(d);
         TcWorkspace w;
-        const size_t need = tc_workspace_layout(d, workspace, &w);
+        const size_t need = tc_workspace_layout(t, workspace, &w);
         if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
         cudaError_t e = profiled(kCumsum, s, [&] {
-            return launch_chunk_cumsum(d, dt, A, w.lam, w.dtT, w.wts, B, w.b16, s);
+            return launch_chunk_cumsum(t, dt, A, w.lam, w.dtT, w.wts, B, w.b16, s);
         });
         if (e == cudaSuccess)
             e = profiled(kStateTc, s, [&] {
-                return launch_chunk_state_scan_tc(d, x, w.b16, w, init_state, final_state, s);
+                return launch_chunk_state_scan_tc(t, x, w.b16, w, init_state, final_state, s);
             });
         if (e == cudaSuccess)
-            e = profiled(kOutTc, s, [&] { return launch_chunk_output_tc(d, x, B, C, D, w, y, s); });
+            e = profiled(kOutTc, s, [&] { return launch_chunk_output_tc(t, x, B, C, D, w, y, s); });
         return from_cuda(e);
     }
 

@@ -315,104 +315,93 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
 
 
 
-// ================================================================ chunk output
-// One CTA per (chunk c, 128-token tile i, head group, batch b); warp 0 issues TMA and
-// bulk loads, warp 1 issues tcgen05.mma, warps 4-11 build the masked operands, warps
-// 12-15 run the epilogue.  With t the tile's tokens (chunk-relative, 128 i .. 128 i + 127):
+// ================================================================ block output
+// One CTA per (128-token block k, head group, batch b); warp 0 issues TMA and bulk loads,
+// warp 1 issues tcgen05.mma, warps 4-11 build the masked diagonal operand, warps 12-15
+// run the epilogue.  With t, s the block's tokens and Lam the decay cumsum from the
+// block start:
 //
-//   G_d = C_t B_{diag}^T   (diagonal 128 x 128 block; fp32 in TMEM, shared by the heads)
-//   G_o = C_t B_{s<128}^T  (i = 1 only: off-diagonal block; bf16 in shared memory, shared)
-//   per head h (operands, P buffers and accumulators double-buffered across heads):
-//     P   = G_d o exp(Lam_t - Lam_s) o dt_s  (s <= t, diagonal block; bf16)
-//     Yd  = P X_diag
-//     Z   = G_o (v o dt o X_{s<128}),  v_s = exp(Lam_127 - Lam_s)               (i = 1)
-//     Yo  = C_t H_c^T
-//     y_t = Yd + u_t (Z + kappa Yo) + D_h x_t,   u_t = exp(Lam_t - Lam_r), kappa = exp(Lam_r)
-//   with r = 127 for i = 1 (so exp(Lam_t - Lam_s) = u_t v_s on the off-diagonal block and
-//   exp(Lam_t) = u_t kappa; every factor <= 1) and Lam_r = 0, Z = 0 for i = 0.
-// The off-diagonal block's mask thus costs a per-row and a per-column scale instead of
-// a masked matrix per head; only the diagonal block is built elementwise.  There,
-// 32-column sub-blocks below the diagonal use exp(Lam_t - Lam_q) exp(Lam_q - Lam_s) with q
-// the sub-block's last column (both <= 1); sub-blocks on the diagonal use the first
-// column as reference when their own decay is below 40 (both factors within e^+-40) and
-// fall back to one exponential per element otherwise.
+//   G   = C_t B_s^T                           (once per CTA; fp32 in TMEM, shared by the heads)
+//   per head h (operand slots three deep, P buffers and accumulators double/triple-buffered):
+//     P   = G o exp(Lam_t - Lam_s) o dt_s     (s <= t; bf16)
+//     Yd  = P X_s,   Yo = C_t H_k^T           (tcgen05; H_k = state at the block start)
+//     y_t = Yd + exp(Lam_t) Yo + D_h x_t      -> bf16, written over x_t and TMA-stored
+//
+// A chunk longer than 128 tokens is handled as consecutive 128-token blocks: its strictly
+// lower off-diagonal blocks enter through the state at each block start (the exact rank-N
+// factorisation of those blocks), which the chunk-state walk provides every 128 tokens.
+// Below-diagonal 32-column sub-blocks of P use exp(Lam_t - Lam_q) exp(Lam_q - Lam_s) with q
+// the sub-block's last column (both <= 1); sub-blocks on the diagonal use the first column
+// as reference when their own decay is below 40 (both factors within e^+-40) and fall
+// back to one exponential per element otherwise.
+constexpr int kBlk = 128;                                // tokens per output block
 constexpr int kOutThreads = 512;
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpP0 = 4, kWarpE0 = 12;
 constexpr int kPThreads = 256, kEThreads = 128;
-constexpr uint32_t kColGd = 384, kColGo = 256;           // TMEM columns of G_d and G_o
-constexpr uint32_t kAccCols = 192;                       // per slot: Yd +0, Z +64, Yo +128
+constexpr int kOutSlots = 3;
+constexpr uint32_t kColG = 384;                          // TMEM columns of G
+constexpr uint32_t kAccCols = 128;                       // per slot: Yd +0, Yo +64
 
-template <int Q>
 struct OutSmem {
-    static constexpr int kC = 0;                        // [2 n-halves][128 rows][128 B]
-    static constexpr int kB = 2 * kBox;                 // [2][Q rows][128 B]; then 2 P buffers
-    static constexpr int kGo = kB + 2 * Q * 128;        // G_o bf16 [2 k-blocks][128][128 B]
-    static constexpr int kH = kGo + 2 * kBox;           // H_c image (single buffer)
-    static constexpr int kSlot0 = kH + kHImage;         // per-head slots
-    static constexpr int kXo = 0;                       //   X  [Q rows][128 B]
-    static constexpr int kLo = Q * 128;                 //   Lam[Q]
-    static constexpr int kDo = kLo + Q * 4;             //   dt[Q]
-    static constexpr int kVo = kDo + Q * 4;             //   column factors, block-end reference
-    static constexpr int kWo = kVo + Q * 4;             //   column factors, block-start reference
-    static constexpr int kSlotBytes = (kWo + Q * 4 + 1023) / 1024 * 1024;
-    static constexpr int kBar = kSlot0 + 2 * kSlotBytes;
-    static constexpr int kNumBars = 20;
+    static constexpr int kC = 0;                         // C_t [2 n-halves][128 rows][128 B]
+    static constexpr int kP0 = 2 * kBox;                 // B_s (operand of G), then P buffer 0
+    static constexpr int kP1 = kP0 + 2 * kBox;           // P buffer 1
+    static constexpr int kSlot0 = kP1 + 2 * kBox;        // per-head operand slots
+    static constexpr int kXo = 0;                        //   x (then y) [128 rows][128 B]
+    static constexpr int kHo = kBox;                     //   H_k image (MN-major, 16 KB)
+    static constexpr int kLo = kHo + kHImage;            //   Lam[128]
+    static constexpr int kDo = kLo + 512;                //   dt[128]
+    static constexpr int kVo = kDo + 512;                //   column factors, sub-block-end reference
+    static constexpr int kWo = kVo + 512;                //   column factors, sub-block-start reference
+    static constexpr int kSlotBytes = (kWo + 512 + 1023) / 1024 * 1024;
+    static constexpr int kBar = kSlot0 + kOutSlots * kSlotBytes;
+    static constexpr int kNumBars = 18;
     static constexpr int kSlotTm = kBar + kNumBars * 8;
     static constexpr int kAbort = kSlotTm + 4;
     static constexpr int kBytes = kAbort + 12 + 1024;
 };
+static_assert(OutSmem::kSlotBytes % 1024 == 0, "slots keep 1024-byte alignment");
+static_assert(OutSmem::kBytes <= 227 * 1024, "output shared memory");
 
-enum { BAR_CB = 0, BAR_S = 1, BAR_GO = 2, BAR_HFULL = 3, BAR_HEMPTY = 4, BAR_XFULL = 5,
-       BAR_XEMPTY = 7, BAR_PFULL = 9, BAR_PEMPTY = 11, BAR_AFULL = 13, BAR_AEMPTY = 15 };
+enum { BAR_CB = 0, BAR_S = 1, BAR_XFULL = 2, BAR_XEMPTY = 5, BAR_AFULL = 8, BAR_AEMPTY = 11,
+       BAR_PFULL = 14, BAR_PEMPTY = 16 };
 
-template <int Q>
 __global__ void __launch_bounds__(kOutThreads, 1)
-chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
+block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
-                    const float* __restrict__ lam,
-                    const float* __restrict__ dtT, const uint8_t* __restrict__ himg,
-                    const float* __restrict__ D, __nv_bfloat16* __restrict__ y, int seqlen,
-                    int nheads, int ngroups, int nchunks, int heads_per_cta, int* err)
+                    const float* __restrict__ lam, const float* __restrict__ dtT,
+                    const uint8_t* __restrict__ himg, const float* __restrict__ D, int nheads,
+                    int ngroups, int nblocks, int heads_per_cta, int* err)
 {
-    using L = OutSmem<Q>;
-    constexpr int NT = Q / 128;
+    using L = OutSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     uint8_t* sC = sm + L::kC;
-    uint8_t* sB = sm + L::kB;
-    uint8_t* sGo = sm + L::kGo;
-    uint8_t* sH = sm + L::kH;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::kSlotTm);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kAbort);
 
-    const int c = blockIdx.x / NT, it = blockIdx.x - c * NT;
-    const int hg = blockIdx.y, b = blockIdx.z;
+    const int k = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
     const int h0 = hg * heads_per_cta;
     const int g = h0 / (nheads / ngroups);
-    const int R = 128 * (it + 1);                       // source tokens s in [0, R)
-    const int d0 = 128 * it;                            // first column of the diagonal block
-    const int t0 = c * Q;
-    const int qlen = min(Q, seqlen - t0);
+    const int t0 = k * kBlk;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
         mbar_init(&bars[BAR_CB], 1);
         mbar_init(&bars[BAR_S], 1);
-        mbar_init(&bars[BAR_GO], kPThreads);
-        mbar_init(&bars[BAR_HFULL], 1);
-        mbar_init(&bars[BAR_HEMPTY], 1);
-        for (int s2 = 0; s2 < 2; ++s2) {
-            mbar_init(&bars[BAR_XFULL + s2], 1);
-            mbar_init(&bars[BAR_XEMPTY + s2], 1);
-            mbar_init(&bars[BAR_PFULL + s2], kPThreads);
-            mbar_init(&bars[BAR_PEMPTY + s2], 1);
-            mbar_init(&bars[BAR_AFULL + s2], 1);
-            mbar_init(&bars[BAR_AEMPTY + s2], kEThreads);
+        for (int s = 0; s < kOutSlots; ++s) {
+            mbar_init(&bars[BAR_XFULL + s], 1);
+            mbar_init(&bars[BAR_XEMPTY + s], 1);
+            mbar_init(&bars[BAR_AFULL + s], 1);
+            mbar_init(&bars[BAR_AEMPTY + s], kEThreads);
+        }
+        for (int p = 0; p < 2; ++p) {
+            mbar_init(&bars[BAR_PFULL + p], kPThreads);
+            mbar_init(&bars[BAR_PEMPTY + p], 1);
         }
         *abort_flag = 0;
         fence_mbar_init();
-        fence_proxy_async_smem();
     }
     if (warp == kWarpMma) {
         tmem_alloc(tslot, 512);
@@ -423,180 +412,127 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     tc_fence_after();
     const uint32_t tmem = *tslot;
 
-    auto slot_base = [&](int s2) { return sm + L::kSlot0 + s2 * L::kSlotBytes; };
-    auto pbuf = [&](int b2) { return sB + b2 * (2 * kBox); };
+    auto slot = [&](int s) { return sm + L::kSlot0 + s * L::kSlotBytes; };
+    auto pbuf = [&](int p) { return sm + (p ? L::kP1 : L::kP0); };
 
     if (warp == kWarpTma) {
         if (lane == 0) {
-            mbar_expect_tx(&bars[BAR_CB], 2 * kBox + (it + 1) * 2 * kBox);
-            tma_load_3d(sC, &tm_c, g * kN, t0 + it * 128, b, &bars[BAR_CB]);
-            tma_load_3d(sC + kBox, &tm_c, g * kN + 64, t0 + it * 128, b, &bars[BAR_CB]);
-            for (int rb = 0; rb <= it; ++rb) {
-                tma_load_3d(sB + rb * kBox, &tm_b, g * kN, t0 + rb * 128, b, &bars[BAR_CB]);
-                tma_load_3d(sB + Q * 128 + rb * kBox, &tm_b, g * kN + 64, t0 + rb * 128, b, &bars[BAR_CB]);
-            }
+            mbar_expect_tx(&bars[BAR_CB], 4 * kBox);
+            tma_load_3d(sC, &tm_c, g * kN, t0, b, &bars[BAR_CB]);
+            tma_load_3d(sC + kBox, &tm_c, g * kN + 64, t0, b, &bars[BAR_CB]);
+            tma_load_3d(pbuf(0), &tm_b, g * kN, t0, b, &bars[BAR_CB]);
+            tma_load_3d(pbuf(0) + kBox, &tm_b, g * kN + 64, t0, b, &bars[BAR_CB]);
             for (int j = 0; j < heads_per_cta; ++j) {
-                const int s2 = j & 1, use = j >> 1;
-                const int h = h0 + j;
-                const size_t bh = (size_t)b * nheads + h;
-                if (j >= 2 && !mbar_wait_or_abort(&bars[BAR_XEMPTY + s2], (use - 1) & 1, err, abort_flag)) break;
-                uint8_t* sl = slot_base(s2);
-                mbar_expect_tx(&bars[BAR_XFULL + s2], (it + 1) * kBox + 2 * R * 4);
-                for (int rb = 0; rb <= it; ++rb)
-                    tma_load_3d(sl + L::kXo + rb * kBox, &tm_x, h * kP, t0 + rb * 128, b, &bars[BAR_XFULL + s2]);
-                bulk_load(sl + L::kLo, lam + (bh * nchunks + c) * Q, R * 4, &bars[BAR_XFULL + s2]);
-                bulk_load(sl + L::kDo, dtT + (bh * nchunks + c) * Q, R * 4, &bars[BAR_XFULL + s2]);
-                if (j >= 1 && !mbar_wait_or_abort(&bars[BAR_HEMPTY], (j - 1) & 1, err, abort_flag)) break;
-                mbar_expect_tx(&bars[BAR_HFULL], kHImage);
-                bulk_load(sH, himg + (bh * nchunks + c) * kHImage, kHImage, &bars[BAR_HFULL]);
+                const int s = j % kOutSlots, use = j / kOutSlots;
+                const size_t bh = (size_t)b * nheads + h0 + j;
+                if (j >= kOutSlots &&
+                    !mbar_wait_or_abort(&bars[BAR_XEMPTY + s], (use - 1) & 1, err, abort_flag))
+                    break;
+                uint8_t* sl = slot(s);
+                mbar_expect_tx(&bars[BAR_XFULL + s], kBox + kHImage + 2 * 512);
+                tma_load_3d(sl + L::kXo, &tm_x, (h0 + j) * kP, t0, b, &bars[BAR_XFULL + s]);
+                bulk_load(sl + L::kHo, himg + (bh * nblocks + k) * kHImage, kHImage, &bars[BAR_XFULL + s]);
+                bulk_load(sl + L::kLo, lam + (bh * nblocks + k) * kBlk, 512, &bars[BAR_XFULL + s]);
+                bulk_load(sl + L::kDo, dtT + (bh * nblocks + k) * kBlk, 512, &bars[BAR_XFULL + s]);
             }
         }
     } else if (warp == kWarpMma) {
         if (lane == 0 && mbar_wait_or_abort(&bars[BAR_CB], 0, err, abort_flag)) {
             tc_fence_after();
-            const uint32_t aC = smem_u32(sC), aB = smem_u32(sB), aGo = smem_u32(sGo), aH = smem_u32(sH);
-            // G = C_t B_{s<R}^T into columns [512 - R, 512): G_o (i = 1) then G_d
-            const uint32_t idG = idesc_bf16_f32(128, R, false, false);
+            const uint32_t aC = smem_u32(sC), aB = smem_u32(pbuf(0));
+            // G = C_t B_s^T (K = N = 128 state columns) into columns [384, 512)
+            const uint32_t idG = idesc_bf16_f32(128, 128, false, false);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
-                umma_f16(tmem + 512 - R, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
-                         smem_desc_sw128(aB + kb * (Q * 128) + off, 16, 1024), idG, ks > 0 ? 1u : 0u);
+                umma_f16(tmem + kColG, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
+                         smem_desc_sw128(aB + kb * kBox + off, 16, 1024), idG, ks > 0 ? 1u : 0u);
             }
             umma_commit(&bars[BAR_S]);
             constexpr uint32_t idMN = idesc_bf16_f32(128, 64, false, true);
-            // G_o lives in shared memory (and its TMEM columns become accumulator space)
-            bool good = it == 0 || mbar_wait_or_abort(&bars[BAR_GO], 0, err, abort_flag);
+            // Yo of head j is issued as soon as its slot is loaded; Yd of head j once P_j is built
+            auto issue_yd = [&](int j) -> bool {
+                const int s = j % kOutSlots, p = j & 1;
+                if (!mbar_wait_or_abort(&bars[BAR_PFULL + p], (j >> 1) & 1, err, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t aP = smem_u32(pbuf(p)), aX = smem_u32(slot(s) + L::kXo);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_f16(tmem + s * kAccCols, smem_desc_sw128(aP + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
+                             smem_desc_sw128(aX + ks * 2048, kBox, 1024), idMN, ks > 0 ? 1u : 0u);
+                umma_commit(&bars[BAR_PEMPTY + p]);
+                umma_commit(&bars[BAR_AFULL + s]);
+                return true;
+            };
+            bool good = true;
             for (int j = 0; j < heads_per_cta && good; ++j) {
-                const int s2 = j & 1, use = j >> 1;
-                good = mbar_wait_or_abort(&bars[BAR_XFULL + s2], use & 1, err, abort_flag) &&
-                       mbar_wait_or_abort(&bars[BAR_HFULL], j & 1, err, abort_flag) &&
-                       (j < 2 || mbar_wait_or_abort(&bars[BAR_AEMPTY + s2], (use - 1) & 1, err, abort_flag));
+                const int s = j % kOutSlots, use = j / kOutSlots;
+                good = mbar_wait_or_abort(&bars[BAR_XFULL + s], use & 1, err, abort_flag) &&
+                       (j < kOutSlots ||
+                        mbar_wait_or_abort(&bars[BAR_AEMPTY + s], (use - 1) & 1, err, abort_flag));
                 if (!good) break;
                 tc_fence_after();
-                const uint32_t acc = tmem + s2 * kAccCols;
-                const uint32_t aX = smem_u32(slot_base(s2) + L::kXo);
-                // Yo = C_t H_c^T (needs no P)
+                const uint32_t aH = smem_u32(slot(s) + L::kHo);
+                // Yo = C_t H_k^T: A = C (K-major over n), B = H image (MN-major, p contiguous)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
-                    umma_f16(acc + 128, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
+                    umma_f16(tmem + s * kAccCols + 64, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
                              smem_desc_sw128(aH + ks * 2048, 8192, 1024), idMN, ks > 0 ? 1u : 0u);
                 }
-                umma_commit(&bars[BAR_HEMPTY]);
-                good = mbar_wait_or_abort(&bars[BAR_PFULL + s2], use & 1, err, abort_flag);
-                if (!good) break;
-                tc_fence_after();
-                if (it == 1) {
-                    // Z = G_o (v o dt o X_{s<128})
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        umma_f16(acc + 64, smem_desc_sw128(aGo + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
-                                 smem_desc_sw128(aX + ks * 2048, Q * 128, 1024), idMN, ks > 0 ? 1u : 0u);
-                }
-                // Yd = P X_diag
-                const uint32_t aP = smem_u32(pbuf(s2));
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    umma_f16(acc, smem_desc_sw128(aP + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
-                             smem_desc_sw128(aX + d0 * 128 + ks * 2048, Q * 128, 1024), idMN, ks > 0 ? 1u : 0u);
-                umma_commit(&bars[BAR_PEMPTY + s2]);
-                umma_commit(&bars[BAR_AFULL + s2]);
+                if (j >= 1) good = issue_yd(j - 1);
             }
+            if (good && heads_per_cta > 0) issue_yd(heads_per_cta - 1);
         }
     } else if (warp >= kWarpP0 && warp < kWarpE0) {
         const int pw = warp - kWarpP0;
         const int q = warp & 3, colhalf = pw >> 2;
-        const int r = q * 32 + lane;                    // tile row
-        const int tl = d0 + r;                          // chunk-relative token
+        const int r = q * 32 + lane;                    // block row t
         const int ptid = tid - kWarpP0 * 32;
         const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
         bool live = mbar_wait_or_abort(&bars[BAR_S], 0, err, abort_flag);
         tc_fence_after();
-        if (it == 1) {
-            // G_o -> bf16, K-major swizzled, once for all heads
-            if (live) {
-                uint32_t v0[32], v1[32];
-                tmem_ld32(trow + kColGo + colhalf * 64, v0);
-                tmem_ld32(trow + kColGo + colhalf * 64 + 32, v1);
-                tmem_wait_ld();
-#pragma unroll
-                for (int w2 = 0; w2 < 2; ++w2) {
-                    const uint32_t* v = w2 ? v1 : v0;
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4)
-                        *reinterpret_cast<uint4*>(sGo + colhalf * kBox + sw128(r, w2 * 4 + k4)) = make_uint4(
-                            pack_bf16x2(__uint_as_float(v[8 * k4]), __uint_as_float(v[8 * k4 + 1])),
-                            pack_bf16x2(__uint_as_float(v[8 * k4 + 2]), __uint_as_float(v[8 * k4 + 3])),
-                            pack_bf16x2(__uint_as_float(v[8 * k4 + 4]), __uint_as_float(v[8 * k4 + 5])),
-                            pack_bf16x2(__uint_as_float(v[8 * k4 + 6]), __uint_as_float(v[8 * k4 + 7])));
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bars[BAR_GO]);
-        }
         for (int j = 0; j < heads_per_cta; ++j) {
-            const int s2 = j & 1, use = j >> 1;
-            live = live && mbar_wait_or_abort(&bars[BAR_XFULL + s2], use & 1, err, abort_flag);
+            const int s = j % kOutSlots, p = j & 1;
+            live = live && mbar_wait_or_abort(&bars[BAR_XFULL + s], (j / kOutSlots) & 1, err, abort_flag);
             // all P threads agree before touching the slot (no thread may leave a named
             // barrier while another still waits in it)
             if (!named_bar_and(1, kPThreads, live)) break;
-            uint8_t* sl = slot_base(s2);
+            uint8_t* sl = slot(s);
             const float* sLam = reinterpret_cast<const float*>(sl + L::kLo);
             const float* sDt = reinterpret_cast<const float*>(sl + L::kDo);
             float* sV = reinterpret_cast<float*>(sl + L::kVo);
             float* sW = reinterpret_cast<float*>(sl + L::kWo);
-            // column factors of the diagonal block, per 32-column sub-block: reference its
-            // last column (factor <= 1) and its first column (factor >= 1, used only where
-            // the sub-block's own decay is small); i = 1 also the off-diagonal weights
-            // exp(Lam_127 - Lam_s) dt_s
-            for (int si = ptid; si < 128; si += kPThreads) {
-                const int sg = d0 + si;
-                sV[sg] = expf(sLam[sg | 31] - sLam[sg]) * sDt[sg];
-                sW[sg] = expf(sLam[sg & ~31] - sLam[sg]) * sDt[sg];
+            // column factors per 32-column sub-block: reference its last column (factor <= 1)
+            // and its first column (factor >= 1, used only where the sub-block's own decay
+            // is small)
+            if (ptid < kBlk) {
+                sV[ptid] = expf(sLam[ptid | 31] - sLam[ptid]) * sDt[ptid];
+                sW[ptid] = expf(sLam[ptid & ~31] - sLam[ptid]) * sDt[ptid];
             }
-            if (it == 1)
-                for (int si = ptid; si < 128; si += kPThreads)
-                    sV[si] = expf(sLam[127] - sLam[si]) * sDt[si];
+            // the GEMM of head j - 2 must be done with this P buffer
+            if (j >= 2) live = mbar_wait_or_abort(&bars[BAR_PEMPTY + p], ((j >> 1) - 1) & 1, err, abort_flag);
             if (!named_bar_and(1, kPThreads, live)) break;
-            if (it == 1) {
-                // X~ = v o dt o X on rows 0..127, in place (bf16); consecutive threads take
-                // consecutive 16-byte chunks; chunk i belongs to row i / 8
-                for (int i = ptid; i < 128 * 8; i += kPThreads) {
-                    const float w = sV[i >> 3];
-                    uint4* ch = reinterpret_cast<uint4*>(sl + L::kXo) + i;
-                    uint4 u = *ch;
-                    u.x = pack_bf16x2(bf16lo(u.x) * w, bf16hi(u.x) * w);
-                    u.y = pack_bf16x2(bf16lo(u.y) * w, bf16hi(u.y) * w);
-                    u.z = pack_bf16x2(bf16lo(u.z) * w, bf16hi(u.z) * w);
-                    u.w = pack_bf16x2(bf16lo(u.w) * w, bf16hi(u.w) * w);
-                    *ch = u;
-                }
-            }
-            // the GEMMs of head j - 2 must be done with this P buffer
-            if (j >= 2) live = mbar_wait_or_abort(&bars[BAR_PEMPTY + s2], (use - 1) & 1, err, abort_flag);
-            if (!named_bar_and(1, kPThreads, live)) break;
-            const float lam_t = sLam[tl];
-            uint8_t* P = pbuf(s2);
+            const float lam_t = sLam[r];
+            uint8_t* P = pbuf(p);
             const int kc0 = colhalf, kc1 = colhalf + 2;
             uint32_t v0[32], v1[32];
-            tmem_ld32(trow + kColGd + kc0 * 32, v0);
-            tmem_ld32(trow + kColGd + kc1 * 32, v1);
+            tmem_ld32(trow + kColG + kc0 * 32, v0);
+            tmem_ld32(trow + kColG + kc1 * 32, v1);
             tmem_wait_ld();
 #pragma unroll
             for (int w2 = 0; w2 < 2; ++w2) {
                 const int kc = w2 ? kc1 : kc0;
                 const uint32_t* v = w2 ? v1 : v0;
-                const int s0 = d0 + kc * 32;
+                const int s0 = kc * 32;
                 uint32_t pk[16];
-                if (s0 + 31 <= tl) {
+                if (s0 + 31 <= r) {
                     const float u = expf(lam_t - sLam[s0 + 31]);
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
                         pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * u * sV[s0 + 2 * e],
                                             __uint_as_float(v[2 * e + 1]) * u * sV[s0 + 2 * e + 1]);
-                } else if (s0 > tl) {
+                } else if (s0 > r) {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) pk[e] = 0u;
                 } else if (sLam[s0] - sLam[s0 + 31] < 40.f) {
@@ -609,15 +545,15 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                         const int sa = s0 + 2 * e;
                         const float pa = __uint_as_float(v[2 * e]) * u * sW[sa];
                         const float pb = __uint_as_float(v[2 * e + 1]) * u * sW[sa + 1];
-                        pk[e] = pack_bf16x2(sa <= tl ? pa : 0.f, sa + 1 <= tl ? pb : 0.f);
+                        pk[e] = pack_bf16x2(sa <= r ? pa : 0.f, sa + 1 <= r ? pb : 0.f);
                     }
                 } else {
                     // strong decay inside the sub-block: one exponential per element
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const int sa = s0 + 2 * e, sb = sa + 1;
-                        const float pa = sa <= tl ? __uint_as_float(v[2 * e]) * expf(lam_t - sLam[sa]) * sDt[sa] : 0.f;
-                        const float pb = sb <= tl ? __uint_as_float(v[2 * e + 1]) * expf(lam_t - sLam[sb]) * sDt[sb] : 0.f;
+                        const float pa = sa <= r ? __uint_as_float(v[2 * e]) * expf(lam_t - sLam[sa]) * sDt[sa] : 0.f;
+                        const float pb = sb <= r ? __uint_as_float(v[2 * e + 1]) * expf(lam_t - sLam[sb]) * sDt[sb] : 0.f;
                         pk[e] = pack_bf16x2(pa, pb);
                     }
                 }
@@ -629,67 +565,60 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bars[BAR_PFULL + s2]);
+            mbar_arrive(&bars[BAR_PFULL + p]);
         }
     } else if (warp >= kWarpE0) {
-        // ---- epilogue: y = Yd + u_t (Z + kappa Yo) + D x, written in place over the
-        // tile's x rows (each thread its own row), then one TMA store of the tile
+        // ---- epilogue: y = Yd + exp(Lam_t) Yo + D x, written in place over the block's
+        // x rows (each thread its own row), then one TMA store of the block
         const int q = warp & 3;
         const int r = q * 32 + lane;
-        const int tl = d0 + r;
         const int etid = tid - kWarpE0 * 32;
         const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
         for (int j = 0; j < heads_per_cta; ++j) {
-            const int s2 = j & 1, use = j >> 1;
-            if (!mbar_wait_or_abort(&bars[BAR_AFULL + s2], use & 1, err, abort_flag)) break;
+            const int s = j % kOutSlots;
+            if (!mbar_wait_or_abort(&bars[BAR_AFULL + s], (j / kOutSlots) & 1, err, abort_flag)) break;
             tc_fence_after();
             const int h = h0 + j;
-            uint8_t* sl = slot_base(s2);
-            const float* sLam = reinterpret_cast<const float*>(sl + L::kLo);
-            const float lam_r = it == 1 ? sLam[127] : 0.f;
-            const float u = expf(sLam[tl] - lam_r);
-            const float kappa = expf(lam_r);
+            uint8_t* sl = slot(s);
+            const float u = expf(reinterpret_cast<const float*>(sl + L::kLo)[r]);
             const float Dh = D[h];
-            uint8_t* xrow = sl + L::kXo + tl * 128;
-            const uint32_t acc = trow + s2 * kAccCols;
+            uint8_t* xrow = sl + L::kXo + r * 128;
+            const uint32_t acc = trow + s * kAccCols;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                uint32_t yd[32], yz[32], yo[32];
+                uint32_t yd[32], yo[32];
                 tmem_ld32(acc + half * 32, yd);
-                tmem_ld32(acc + 64 + half * 32, yz);
-                tmem_ld32(acc + 128 + half * 32, yo);
+                tmem_ld32(acc + 64 + half * 32, yo);
                 tmem_wait_ld();
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
                     const int qx = half * 4 + qq;
-                    uint4* xp = reinterpret_cast<uint4*>(xrow + ((qx ^ (tl & 7)) << 4));
+                    uint4* xp = reinterpret_cast<uint4*>(xrow + ((qx ^ (r & 7)) << 4));
                     const uint4 xu = *xp;
                     const uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w};
                     uint32_t o[4];
 #pragma unroll
                     for (int k2 = 0; k2 < 4; ++k2) {
                         const int jj = qq * 8 + 2 * k2;
-                        const float z0 = it == 1 ? __uint_as_float(yz[jj]) : 0.f;
-                        const float z1 = it == 1 ? __uint_as_float(yz[jj + 1]) : 0.f;
-                        const float a0 = fmaf(u, fmaf(kappa, __uint_as_float(yo[jj]), z0), __uint_as_float(yd[jj])) + Dh * bf16lo(xw[k2]);
-                        const float a1 = fmaf(u, fmaf(kappa, __uint_as_float(yo[jj + 1]), z1), __uint_as_float(yd[jj + 1])) + Dh * bf16hi(xw[k2]);
+                        const float a0 = fmaf(u, __uint_as_float(yo[jj]), __uint_as_float(yd[jj])) + Dh * bf16lo(xw[k2]);
+                        const float a1 = fmaf(u, __uint_as_float(yo[jj + 1]), __uint_as_float(yd[jj + 1])) + Dh * bf16hi(xw[k2]);
                         o[k2] = pack_bf16x2(a0, a1);
                     }
                     *xp = make_uint4(o[0], o[1], o[2], o[3]);
                 }
             }
             tc_fence_before();
-            mbar_arrive(&bars[BAR_AEMPTY + s2]);
+            mbar_arrive(&bars[BAR_AEMPTY + s]);
             fence_proxy_async_smem();                       // y rows -> visible to the TMA unit
             named_bar_sync(2, kEThreads);
             if (etid == 0) {
-                tma_store_3d(&tm_y, h * kP, t0 + d0, b, sl + L::kXo + d0 * 128);
+                tma_store_3d(&tm_y, h * kP, t0, b, sl + L::kXo);
                 bulk_commit_group();
                 bulk_wait_group_read0();                    // the slot may be refilled now
-                mbar_arrive(&bars[BAR_XEMPTY + s2]);
+                mbar_arrive(&bars[BAR_XEMPTY + s]);
             }
         }
-        if (etid == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        if (etid == 0) bulk_wait_group0();
     }
 
     tc_fence_before();
@@ -699,6 +628,7 @@ chunk_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         tmem_dealloc(tmem, 512);
     }
 }
+
 
 // ---------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
@@ -796,20 +726,17 @@ cudaError_t walk_t(const Dims& d, const WalkMaps& maps, const TcWorkspace& w, co
     return cudaGetLastError();
 }
 
-template <int Q>
-cudaError_t output_t(const Dims& d, const CUtensorMap& mx, const CUtensorMap& mb, const CUtensorMap& mc,
-                     const CUtensorMap& my, const TcWorkspace& w, const float* D, void* y, cudaStream_t s)
+cudaError_t output_launch(const Dims& d, const CUtensorMap& mx, const CUtensorMap& mb,
+                          const CUtensorMap& mc, const CUtensorMap& my, const TcWorkspace& w,
+                          const float* D, cudaStream_t s)
 {
-    auto k = chunk_output_kernel<Q>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         OutSmem<Q>::kBytes);
+    auto k = block_output_kernel;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, OutSmem::kBytes);
     if (e != cudaSuccess) return e;
     const int hpc = heads_per_cta(d);
-    dim3 grid(d.nchunks * (Q / 128), d.nheads / hpc, d.batch);
-    k<<<grid, kOutThreads, OutSmem<Q>::kBytes, s>>>(mx, mb, mc, my, w.lam, w.dtT, w.himg, D,
-                                                    static_cast<__nv_bfloat16*>(y), d.seqlen,
-                                                    d.nheads, d.ngroups, d.nchunks, hpc,
-                                                    device_error_word());
+    dim3 grid(d.nchunks, d.nheads / hpc, d.batch);
+    k<<<grid, kOutThreads, OutSmem::kBytes, s>>>(mx, mb, mc, my, w.lam, w.dtT, w.himg, D, d.nheads,
+                                                d.ngroups, d.nchunks, hpc, device_error_word());
     return cudaGetLastError();
 }
 
@@ -818,6 +745,14 @@ cudaError_t output_t(const Dims& d, const CUtensorMap& mx, const CUtensorMap& mb
 bool tc_prefill_supported(const Dims& d)
 {
     return d.headdim == kP && d.dstate == kN && (d.chunk_len == 128 || d.chunk_len == 256);
+}
+
+Dims tc_block_dims(const Dims& d)
+{
+    Dims t = d;
+    t.chunk_len = kBlk;
+    t.nchunks = (d.seqlen + kBlk - 1) / kBlk;
+    return t;
 }
 
 size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w)
@@ -862,8 +797,8 @@ cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void*
         !encode_map(&m.b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, B_f16, bdim, bstr, bbox, true) ||
         !encode_map(&m.w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, w.wts, wdim, wstr, wbox, false))
         return cudaErrorInvalidValue;
-    if (d.chunk_len == 256) return walk_t<256>(d, m, w, init_state, final_state, s);
-    return walk_t<128>(d, m, w, init_state, final_state, s);
+    if (d.chunk_len != kBlk) return cudaErrorInvalidValue;
+    return walk_t<kBlk>(d, m, w, init_state, final_state, s);
 }
 
 cudaError_t launch_chunk_output_tc(const Dims& d, const void* x, const void* B, const void* C,
@@ -871,13 +806,13 @@ cudaError_t launch_chunk_output_tc(const Dims& d, const void* x, const void* B, 
 {
     if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
     CUtensorMap mx, mb, mc, my;
+    if (d.chunk_len != kBlk) return cudaErrorInvalidValue;
     if (!make_map(&mx, x, (uint64_t)d.nheads * kP, d.seqlen, d.batch) ||
         !make_map(&mb, B, (uint64_t)d.ngroups * kN, d.seqlen, d.batch) ||
         !make_map(&mc, C, (uint64_t)d.ngroups * kN, d.seqlen, d.batch) ||
         !make_map(&my, y, (uint64_t)d.nheads * kP, d.seqlen, d.batch))
         return cudaErrorInvalidValue;
-    if (d.chunk_len == 256) return output_t<256>(d, mx, mb, mc, my, w, D, y, s);
-    return output_t<128>(d, mx, mb, mc, my, w, D, y, s);
+    return output_launch(d, mx, mb, mc, my, w, D, s);
 }
 
 }  // namespace ssd

@@ -8,7 +8,12 @@ namespace ssd {
 // headdim 64, dstate 128, chunk_len 128 or 256, bf16 storage.
 bool tc_prefill_supported(const Dims& d);
 
-// Workspace of the tensor-core path.
+// The tensor-core stages work in 128-token blocks: the problem with chunk_len = 128 and
+// nchunks = ceil(seqlen / 128).  A 256-token chunk is two such blocks, its off-diagonal
+// 128 x 128 block entering through the state at its midpoint (an exact factorisation).
+Dims tc_block_dims(const Dims& d);
+
+// Workspace of the tensor-core path (sized and indexed by the 128-token block dims).
 struct TcWorkspace {
     float* lam;       // [b][h][c][Q] inclusive cumsum of dt*A within each chunk
     float* dtT;       // [b][h][c][Q] dt, zero past seqlen
@@ -25,7 +30,7 @@ cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void*
                                        const TcWorkspace& w, const float* init_state,
                                        float* final_state, cudaStream_t s);
 
-// y = (C B^T o L o dt) X + diag(exp Lam) C H_c^T + D x, bf16 out.
+// Per 128-token block: y = (C B^T o L o dt) X + diag(exp Lam) C H_k^T + D x, bf16 out.
 cudaError_t launch_chunk_output_tc(const Dims& d, const void* x, const void* B, const void* C,
                                    const float* D, const TcWorkspace& w, void* y, cudaStream_t s);
 
