@@ -450,39 +450,55 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             }
             umma_commit(&bars[BAR_S]);
             constexpr uint32_t idMN = idesc_bf16_f32(128, 64, false, true);
-            // Yo of head j is issued as soon as its slot is loaded; Yd of head j once P_j is built
-            auto issue_yd = [&](int j) -> bool {
-                const int s = j % kOutSlots, p = j & 1;
-                if (!mbar_wait_or_abort(&bars[BAR_PFULL + p], (j >> 1) & 1, err, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t aP = smem_u32(pbuf(p)), aX = smem_u32(slot(s) + L::kXo);
+            // Yo of a head is issued as soon as its slot is loaded (and its accumulator free),
+            // Yd as soon as its P is built; the two streams are polled, not ordered
+            int jo = 0, jd = 0;
+            uint32_t idle = 0;
+            while (jd < heads_per_cta) {
+                bool progressed = false;
+                if (jo < heads_per_cta) {
+                    const int s = jo % kOutSlots, use = jo / kOutSlots;
+                    if (mbar_try_wait(&bars[BAR_XFULL + s], use & 1) &&
+                        (jo < kOutSlots || mbar_try_wait(&bars[BAR_AEMPTY + s], (use - 1) & 1))) {
+                        tc_fence_after();
+                        const uint32_t aH = smem_u32(slot(s) + L::kHo);
+                        // Yo = C_t H_k^T: A = C (K-major over n), B = H image (MN-major, p contiguous)
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    umma_f16(tmem + s * kAccCols, smem_desc_sw128(aP + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
-                             smem_desc_sw128(aX + ks * 2048, kBox, 1024), idMN, ks > 0 ? 1u : 0u);
-                umma_commit(&bars[BAR_PEMPTY + p]);
-                umma_commit(&bars[BAR_AFULL + s]);
-                return true;
-            };
-            bool good = true;
-            for (int j = 0; j < heads_per_cta && good; ++j) {
-                const int s = j % kOutSlots, use = j / kOutSlots;
-                good = mbar_wait_or_abort(&bars[BAR_XFULL + s], use & 1, err, abort_flag) &&
-                       (j < kOutSlots ||
-                        mbar_wait_or_abort(&bars[BAR_AEMPTY + s], (use - 1) & 1, err, abort_flag));
-                if (!good) break;
-                tc_fence_after();
-                const uint32_t aH = smem_u32(slot(s) + L::kHo);
-                // Yo = C_t H_k^T: A = C (K-major over n), B = H image (MN-major, p contiguous)
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
-                    umma_f16(tmem + s * kAccCols + 64, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
-                             smem_desc_sw128(aH + ks * 2048, 8192, 1024), idMN, ks > 0 ? 1u : 0u);
+                        for (int ks = 0; ks < 8; ++ks) {
+                            const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
+                            umma_f16(tmem + s * kAccCols + 64, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
+                                     smem_desc_sw128(aH + ks * 2048, 8192, 1024), idMN, ks > 0 ? 1u : 0u);
+                        }
+                        ++jo;
+                        progressed = true;
+                    }
                 }
-                if (j >= 1) good = issue_yd(j - 1);
+                if (jd < jo) {
+                    const int s = jd % kOutSlots, p = jd & 1;
+                    if (mbar_try_wait(&bars[BAR_PFULL + p], (jd >> 1) & 1)) {
+                        tc_fence_after();
+                        const uint32_t aP = smem_u32(pbuf(p)), aX = smem_u32(slot(s) + L::kXo);
+                        // Yd = P X: A = P (K-major over s), B = X (MN-major, p contiguous)
+#pragma unroll
+                        for (int ks = 0; ks < 8; ++ks)
+                            umma_f16(tmem + s * kAccCols, smem_desc_sw128(aP + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
+                                     smem_desc_sw128(aX + ks * 2048, kBox, 1024), idMN, ks > 0 ? 1u : 0u);
+                        umma_commit(&bars[BAR_PEMPTY + p]);
+                        umma_commit(&bars[BAR_AFULL + s]);
+                        ++jd;
+                        progressed = true;
+                    }
+                }
+                if (progressed) {
+                    idle = 0;
+                } else if (++idle >= (1u << 22) || ((idle & 1023u) == 0 && *abort_flag)) {
+                    if (idle >= (1u << 22)) {
+                        record_error(err, SSD_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                    }
+                    break;
+                }
             }
-            if (good && heads_per_cta > 0) issue_yd(heads_per_cta - 1);
         }
     } else if (warp >= kWarpP0 && warp < kWarpE0) {
         const int pw = warp - kWarpP0;
@@ -679,14 +695,28 @@ bool encode_map(CUtensorMap* m, CUtensorMapDataType type, int rank, const void* 
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Heads per output CTA: the largest divisor of (heads per group) that is <= 8, so that a
-// CTA's heads share one B/C group.
+int sm_count();
+
+// Heads per output CTA: a divisor of the heads per group (so a CTA's heads share one B/C
+// group), chosen to minimise waves x (heads + 3): each CTA pays about three heads' worth
+// of pipeline fill and drain, and G = C B^T is computed once per CTA.
 int heads_per_cta(const Dims& d)
 {
     const int hpg = d.nheads / d.ngroups;
-    for (int k = 8; k > 1; --k)
-        if (hpg % k == 0) return k;
-    return 1;
+    const long long units = (long long)d.nchunks * d.batch * d.ngroups;     // (block, b, g)
+    const int sms = sm_count();
+    int best = 1;
+    long long best_cost = -1;
+    for (int k = 1; k <= hpg && k <= 64; ++k) {
+        if (hpg % k) continue;
+        const long long ctas = units * (hpg / k);
+        const long long cost = (ctas + sms - 1) / sms * (k + 3);
+        if (best_cost < 0 || cost < best_cost || (cost == best_cost && k > best)) {
+            best = k;
+            best_cost = cost;
+        }
+    }
+    return best;
 }
 
 int sm_count()
