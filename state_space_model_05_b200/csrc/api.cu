@@ -184,7 +184,7 @@ ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const v
         const size_t need = tc_workspace_layout(t, workspace, &w);
         if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
         cudaError_t e = profiled(kCumsum, s, [&] {
-            return launch_chunk_cumsum(t, dt, A, w.lam, w.dtT, w.wts, B, w.b16, s);
+            return launch_chunk_cumsum(t, dt, A, w.fac, true, w.wts, B, w.b16, s);
         });
         if (e == cudaSuccess)
             e = profiled(kStateTc, s, [&] {
@@ -199,7 +199,7 @@ ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const v
     const size_t need = prefill_workspace_layout(d, workspace, &ws);
     if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
     cudaError_t e = profiled(kCumsum, s, [&] {
-        return launch_chunk_cumsum(d, dt, A, ws.lam, nullptr, nullptr, nullptr, nullptr, s);
+        return launch_chunk_cumsum(d, dt, A, ws.lam, false, nullptr, nullptr, nullptr, s);
     });
     if (e == cudaSuccess)
         e = profiled(kStateSimt, s, [&] {

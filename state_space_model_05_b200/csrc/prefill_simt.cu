@@ -37,11 +37,13 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
     return r;
 }
 
-// Also writes dt transposed to [b][h][c][Q] when dtT is non-null (zero past seqlen),
-// and zeroes `nzero` words at `zero` (look-back flags of the tensor-core path).
+// Per (b, h, chunk) row of `fac` (stride fac_stride floats): Lam[Q]; with `extras` also
+// dt[Q] (zero past seqlen) and the column factors of each 32-token sub-block,
+// exp(Lam_last - Lam_s) dt_s and exp(Lam_first - Lam_s) dt_s.  With `wts`, the chunk-state
+// weights exp(Lam_end - Lam_s) dt_s ([b][h][c][Q]); with `b_f16`, an fp16 copy of B.
 __global__ void __launch_bounds__(kThreads)
 chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
-                    float* __restrict__ lam, float* __restrict__ dtT, float* __restrict__ wts,
+                    float* __restrict__ fac, int fac_stride, bool extras, float* __restrict__ wts,
                     const uint4* __restrict__ b_bf16, uint4* __restrict__ b_f16,
                     int b_row_chunks, int seqlen, int nheads, int Q, int nchunks)
 {
@@ -78,7 +80,8 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
         const int hh = warp;
         const float Ah = A[h0 + hh];
         float carry = 0.f;
-        const size_t row = (((size_t)b * nheads + h0 + hh) * nchunks + c) * Q;
+        const size_t unit = ((size_t)b * nheads + h0 + hh) * nchunks + c;
+        float* f = fac + unit * fac_stride;
         float lv[kMaxChunk / 32], dv[kMaxChunk / 32];
 #pragma unroll
         for (int j = 0; j < kMaxChunk / 32; ++j) {
@@ -92,10 +95,17 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
                 if (lane >= o) v += u;
             }
             v += carry;
-            if (t < Q) {
-                lam[row + t] = v;
-                if (dtT) dtT[row + t] = d;
+            if (extras) {
+                // column factors per 32-token sub-block (one warp pass = one sub-block):
+                // exp(Lam_last - Lam_s) dt_s and exp(Lam_first - Lam_s) dt_s
+                const float vlast = __shfl_sync(0xffffffffu, v, 31), vfirst = __shfl_sync(0xffffffffu, v, 0);
+                if (t < Q) {
+                    f[Q + t] = d;
+                    f[2 * Q + t] = expf(vlast - v) * d;
+                    f[3 * Q + t] = expf(vfirst - v) * d;
+                }
             }
+            if (t < Q) f[t] = v;
             lv[j] = v;
             dv[j] = d;
             carry = __shfl_sync(0xffffffffu, v, 31);
@@ -106,7 +116,7 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
             for (int j = 0; j < kMaxChunk / 32; ++j) {
                 const int t = j * 32 + lane;
                 if (j * 32 >= Q) break;
-                if (t < Q) wts[row + t] = expf(carry - lv[j]) * dv[j];
+                if (t < Q) wts[unit * Q + t] = expf(carry - lv[j]) * dv[j];
             }
         }
     }
@@ -399,15 +409,16 @@ size_t simt_output_smem_bytes(int headdim, int dstate)
                             kTokTile * (kTokTile + 1) + 2 * kTokTile);
 }
 
-cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, float* lam,
-                                float* dtT, float* wts, const void* b_bf16, void* b_f16,
+cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, float* fac,
+                                bool extras, float* wts, const void* b_bf16, void* b_f16,
                                 cudaStream_t s)
 {
     if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
     const size_t smem = sizeof(float) * d.chunk_len * kCumsumHeads;
     dim3 grid(d.nchunks, (d.nheads + kCumsumHeads - 1) / kCumsumHeads, d.batch);
     chunk_cumsum_kernel<<<grid, kThreads, smem, s>>>(
-        dt, A, lam, dtT, wts, static_cast<const uint4*>(b_bf16), static_cast<uint4*>(b_f16),
+        dt, A, fac, extras ? 4 * d.chunk_len : d.chunk_len, extras, wts,
+        static_cast<const uint4*>(b_bf16), static_cast<uint4*>(b_f16),
         d.ngroups * d.dstate / 8, d.seqlen, d.nheads, d.chunk_len, d.nchunks);
     return cudaGetLastError();
 }

@@ -90,7 +90,7 @@ struct WalkMaps {
 
 template <int Q>
 __global__ void __launch_bounds__(kWalkThreads, 1)
-chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __restrict__ lam,
+chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __restrict__ fac,
                         const float* __restrict__ init_state, float* final_state,
                         uint8_t* __restrict__ himg, int nheads, int ngroups, int nchunks,
                         int ctas_per_group, int* err)
@@ -209,7 +209,7 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
             float e[kWalkHeads];                         // Lam_end per head
 #pragma unroll
             for (int hh = 0; hh < kWalkHeads; ++hh)
-                e[hh] = hh < nh ? lam[((size_t)(b * nheads + hlo + hh) * nchunks + cc) * Q + Q - 1] : 0.f;
+                e[hh] = hh < nh ? fac[((size_t)(b * nheads + hlo + hh) * nchunks + cc) * 4 * Q + Q - 1] : 0.f;
             if (ok) ok = mbar_wait(&accb[cc & 1], (cc >> 1) & 1, err);
             tc_fence_after();
             const uint32_t acc = tmem + (cc & 1) * 256 + ((uint32_t)((warp & 3) * 32) << 16) + half * 32;
@@ -338,24 +338,26 @@ constexpr int kBlk = 128;                                // tokens per output bl
 constexpr int kOutThreads = 512;
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpP0 = 4, kWarpE0 = 12;
 constexpr int kPThreads = 256, kEThreads = 128;
-constexpr int kOutSlots = 3;
+constexpr int kXSlots = 4;                               // x / y operand slots
+constexpr int kHSlots = 3;                               // state image slots (freed after Yo)
+constexpr int kAccSlots = 3;                             // TMEM accumulator pairs
 constexpr uint32_t kColG = 384;                          // TMEM columns of G
-constexpr uint32_t kAccCols = 128;                       // per slot: Yd +0, Yo +64
+constexpr uint32_t kAccCols = 128;                       // per accumulator: Yd +0, Yo +64
 
 struct OutSmem {
     static constexpr int kC = 0;                         // C_t [2 n-halves][128 rows][128 B]
     static constexpr int kP0 = 2 * kBox;                 // B_s (operand of G), then P buffer 0
     static constexpr int kP1 = kP0 + 2 * kBox;           // P buffer 1
-    static constexpr int kSlot0 = kP1 + 2 * kBox;        // per-head operand slots
+    static constexpr int kH0 = kP1 + 2 * kBox;           // state image slots (MN-major, 16 KB each)
+    static constexpr int kSlot0 = kH0 + kHSlots * kHImage;  // x slots
     static constexpr int kXo = 0;                        //   x (then y) [128 rows][128 B]
-    static constexpr int kHo = kBox;                     //   H_k image (MN-major, 16 KB)
-    static constexpr int kLo = kHo + kHImage;            //   Lam[128]
+    static constexpr int kLo = kBox;                     //   Lam[128]
     static constexpr int kDo = kLo + 512;                //   dt[128]
     static constexpr int kVo = kDo + 512;                //   column factors, sub-block-end reference
     static constexpr int kWo = kVo + 512;                //   column factors, sub-block-start reference
     static constexpr int kSlotBytes = (kWo + 512 + 1023) / 1024 * 1024;
-    static constexpr int kBar = kSlot0 + kOutSlots * kSlotBytes;
-    static constexpr int kNumBars = 18;
+    static constexpr int kBar = kSlot0 + kXSlots * kSlotBytes;
+    static constexpr int kNumBars = 2 + 2 * kXSlots + 2 * kAccSlots + kHSlots + 4;
     static constexpr int kSlotTm = kBar + kNumBars * 8;
     static constexpr int kAbort = kSlotTm + 4;
     static constexpr int kBytes = kAbort + 12 + 1024;
@@ -363,13 +365,14 @@ struct OutSmem {
 static_assert(OutSmem::kSlotBytes % 1024 == 0, "slots keep 1024-byte alignment");
 static_assert(OutSmem::kBytes <= 227 * 1024, "output shared memory");
 
-enum { BAR_CB = 0, BAR_S = 1, BAR_XFULL = 2, BAR_XEMPTY = 5, BAR_AFULL = 8, BAR_AEMPTY = 11,
-       BAR_PFULL = 14, BAR_PEMPTY = 16 };
+enum { BAR_CB = 0, BAR_S = 1, BAR_XFULL = 2, BAR_XEMPTY = BAR_XFULL + kXSlots,
+       BAR_AFULL = BAR_XEMPTY + kXSlots, BAR_AEMPTY = BAR_AFULL + kAccSlots,
+       BAR_HEMPTY = BAR_AEMPTY + kAccSlots, BAR_PFULL = BAR_HEMPTY + kHSlots, BAR_PEMPTY = BAR_PFULL + 2 };
 
 __global__ void __launch_bounds__(kOutThreads, 1)
 block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
-                    const float* __restrict__ lam, const float* __restrict__ dtT,
+                    const float* __restrict__ fac,
                     const uint8_t* __restrict__ himg, const float* __restrict__ D, int nheads,
                     int ngroups, int nblocks, int heads_per_cta, int* err)
 {
@@ -390,12 +393,15 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     if (tid == 0) {
         mbar_init(&bars[BAR_CB], 1);
         mbar_init(&bars[BAR_S], 1);
-        for (int s = 0; s < kOutSlots; ++s) {
+        for (int s = 0; s < kXSlots; ++s) {
             mbar_init(&bars[BAR_XFULL + s], 1);
             mbar_init(&bars[BAR_XEMPTY + s], 1);
+        }
+        for (int s = 0; s < kAccSlots; ++s) {
             mbar_init(&bars[BAR_AFULL + s], 1);
             mbar_init(&bars[BAR_AEMPTY + s], kEThreads);
         }
+        for (int s = 0; s < kHSlots; ++s) mbar_init(&bars[BAR_HEMPTY + s], 1);
         for (int p = 0; p < 2; ++p) {
             mbar_init(&bars[BAR_PFULL + p], kPThreads);
             mbar_init(&bars[BAR_PEMPTY + p], 1);
@@ -413,6 +419,7 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     const uint32_t tmem = *tslot;
 
     auto slot = [&](int s) { return sm + L::kSlot0 + s * L::kSlotBytes; };
+    auto hslot = [&](int s) { return sm + L::kH0 + s * kHImage; };
     auto pbuf = [&](int p) { return sm + (p ? L::kP1 : L::kP0); };
 
     if (warp == kWarpTma) {
@@ -423,17 +430,19 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             tma_load_3d(pbuf(0), &tm_b, g * kN, t0, b, &bars[BAR_CB]);
             tma_load_3d(pbuf(0) + kBox, &tm_b, g * kN + 64, t0, b, &bars[BAR_CB]);
             for (int j = 0; j < heads_per_cta; ++j) {
-                const int s = j % kOutSlots, use = j / kOutSlots;
+                const int s = j % kXSlots, hs = j % kHSlots;
                 const size_t bh = (size_t)b * nheads + h0 + j;
-                if (j >= kOutSlots &&
-                    !mbar_wait_or_abort(&bars[BAR_XEMPTY + s], (use - 1) & 1, err, abort_flag))
+                if (j >= kXSlots &&
+                    !mbar_wait_or_abort(&bars[BAR_XEMPTY + s], (j / kXSlots - 1) & 1, err, abort_flag))
+                    break;
+                if (j >= kHSlots &&
+                    !mbar_wait_or_abort(&bars[BAR_HEMPTY + hs], (j / kHSlots - 1) & 1, err, abort_flag))
                     break;
                 uint8_t* sl = slot(s);
-                mbar_expect_tx(&bars[BAR_XFULL + s], kBox + kHImage + 2 * 512);
+                mbar_expect_tx(&bars[BAR_XFULL + s], kBox + kHImage + 4 * 512);
                 tma_load_3d(sl + L::kXo, &tm_x, (h0 + j) * kP, t0, b, &bars[BAR_XFULL + s]);
-                bulk_load(sl + L::kHo, himg + (bh * nblocks + k) * kHImage, kHImage, &bars[BAR_XFULL + s]);
-                bulk_load(sl + L::kLo, lam + (bh * nblocks + k) * kBlk, 512, &bars[BAR_XFULL + s]);
-                bulk_load(sl + L::kDo, dtT + (bh * nblocks + k) * kBlk, 512, &bars[BAR_XFULL + s]);
+                bulk_load(hslot(hs), himg + (bh * nblocks + k) * kHImage, kHImage, &bars[BAR_XFULL + s]);
+                bulk_load(sl + L::kLo, fac + (bh * nblocks + k) * 4 * kBlk, 4 * 512, &bars[BAR_XFULL + s]);
             }
         }
     } else if (warp == kWarpMma) {
@@ -457,34 +466,35 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             while (jd < heads_per_cta) {
                 bool progressed = false;
                 if (jo < heads_per_cta) {
-                    const int s = jo % kOutSlots, use = jo / kOutSlots;
-                    if (mbar_try_wait(&bars[BAR_XFULL + s], use & 1) &&
-                        (jo < kOutSlots || mbar_try_wait(&bars[BAR_AEMPTY + s], (use - 1) & 1))) {
+                    const int s = jo % kXSlots, a = jo % kAccSlots;
+                    if (mbar_try_wait(&bars[BAR_XFULL + s], (jo / kXSlots) & 1) &&
+                        (jo < kAccSlots || mbar_try_wait(&bars[BAR_AEMPTY + a], (jo / kAccSlots - 1) & 1))) {
                         tc_fence_after();
-                        const uint32_t aH = smem_u32(slot(s) + L::kHo);
+                        const uint32_t aH = smem_u32(hslot(jo % kHSlots));
                         // Yo = C_t H_k^T: A = C (K-major over n), B = H image (MN-major, p contiguous)
 #pragma unroll
                         for (int ks = 0; ks < 8; ++ks) {
                             const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
-                            umma_f16(tmem + s * kAccCols + 64, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
+                            umma_f16(tmem + a * kAccCols + 64, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
                                      smem_desc_sw128(aH + ks * 2048, 8192, 1024), idMN, ks > 0 ? 1u : 0u);
                         }
+                        umma_commit(&bars[BAR_HEMPTY + jo % kHSlots]);
                         ++jo;
                         progressed = true;
                     }
                 }
                 if (jd < jo) {
-                    const int s = jd % kOutSlots, p = jd & 1;
+                    const int s = jd % kXSlots, a = jd % kAccSlots, p = jd & 1;
                     if (mbar_try_wait(&bars[BAR_PFULL + p], (jd >> 1) & 1)) {
                         tc_fence_after();
                         const uint32_t aP = smem_u32(pbuf(p)), aX = smem_u32(slot(s) + L::kXo);
                         // Yd = P X: A = P (K-major over s), B = X (MN-major, p contiguous)
 #pragma unroll
                         for (int ks = 0; ks < 8; ++ks)
-                            umma_f16(tmem + s * kAccCols, smem_desc_sw128(aP + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
+                            umma_f16(tmem + a * kAccCols, smem_desc_sw128(aP + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
                                      smem_desc_sw128(aX + ks * 2048, kBox, 1024), idMN, ks > 0 ? 1u : 0u);
                         umma_commit(&bars[BAR_PEMPTY + p]);
-                        umma_commit(&bars[BAR_AFULL + s]);
+                        umma_commit(&bars[BAR_AFULL + a]);
                         ++jd;
                         progressed = true;
                     }
@@ -504,38 +514,34 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         const int pw = warp - kWarpP0;
         const int q = warp & 3, colhalf = pw >> 2;
         const int r = q * 32 + lane;                    // block row t
-        const int ptid = tid - kWarpP0 * 32;
         const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
         bool live = mbar_wait_or_abort(&bars[BAR_S], 0, err, abort_flag);
         tc_fence_after();
-        for (int j = 0; j < heads_per_cta; ++j) {
-            const int s = j % kOutSlots, p = j & 1;
-            live = live && mbar_wait_or_abort(&bars[BAR_XFULL + s], (j / kOutSlots) & 1, err, abort_flag);
-            // all P threads agree before touching the slot (no thread may leave a named
-            // barrier while another still waits in it)
-            if (!named_bar_and(1, kPThreads, live)) break;
+        // this thread's G entries (row r, sub-blocks kc0 and kc1), the same for every head
+        const int kc0 = colhalf, kc1 = colhalf + 2;
+        uint32_t v0[32], v1[32];
+        tmem_ld32(trow + kColG + kc0 * 32, v0);
+        tmem_ld32(trow + kColG + kc1 * 32, v1);
+        tmem_wait_ld();
+        // Every thread waits on the barriers itself (bounded), so the loop needs no
+        // named barrier; a thread that gives up leaves PFULL incomplete and the MMA
+        // thread's bounded wait reports it.
+        for (int j = 0; j < heads_per_cta && live; ++j) {
+            const int s = j % kXSlots, p = j & 1;
+            live = mbar_wait_or_abort(&bars[BAR_XFULL + s], (j / kXSlots) & 1, err, abort_flag) &&
+                   // the GEMM of head j - 2 must be done with this P buffer
+                   (j < 2 || mbar_wait_or_abort(&bars[BAR_PEMPTY + p], ((j >> 1) - 1) & 1, err, abort_flag));
+            if (!live) break;
             uint8_t* sl = slot(s);
+            // Lam, dt and the column factors of each 32-column sub-block: sV references the
+            // sub-block's last column (factor <= 1), sW its first (used only where the
+            // sub-block's own decay is small)
             const float* sLam = reinterpret_cast<const float*>(sl + L::kLo);
             const float* sDt = reinterpret_cast<const float*>(sl + L::kDo);
-            float* sV = reinterpret_cast<float*>(sl + L::kVo);
-            float* sW = reinterpret_cast<float*>(sl + L::kWo);
-            // column factors per 32-column sub-block: reference its last column (factor <= 1)
-            // and its first column (factor >= 1, used only where the sub-block's own decay
-            // is small)
-            if (ptid < kBlk) {
-                sV[ptid] = expf(sLam[ptid | 31] - sLam[ptid]) * sDt[ptid];
-                sW[ptid] = expf(sLam[ptid & ~31] - sLam[ptid]) * sDt[ptid];
-            }
-            // the GEMM of head j - 2 must be done with this P buffer
-            if (j >= 2) live = mbar_wait_or_abort(&bars[BAR_PEMPTY + p], ((j >> 1) - 1) & 1, err, abort_flag);
-            if (!named_bar_and(1, kPThreads, live)) break;
+            const float* sV = reinterpret_cast<const float*>(sl + L::kVo);
+            const float* sW = reinterpret_cast<const float*>(sl + L::kWo);
             const float lam_t = sLam[r];
             uint8_t* P = pbuf(p);
-            const int kc0 = colhalf, kc1 = colhalf + 2;
-            uint32_t v0[32], v1[32];
-            tmem_ld32(trow + kColG + kc0 * 32, v0);
-            tmem_ld32(trow + kColG + kc1 * 32, v1);
-            tmem_wait_ld();
 #pragma unroll
             for (int w2 = 0; w2 < 2; ++w2) {
                 const int kc = w2 ? kc1 : kc0;
@@ -591,15 +597,15 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         const int etid = tid - kWarpE0 * 32;
         const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
         for (int j = 0; j < heads_per_cta; ++j) {
-            const int s = j % kOutSlots;
-            if (!mbar_wait_or_abort(&bars[BAR_AFULL + s], (j / kOutSlots) & 1, err, abort_flag)) break;
+            const int s = j % kXSlots, a = j % kAccSlots;
+            if (!mbar_wait_or_abort(&bars[BAR_AFULL + a], (j / kAccSlots) & 1, err, abort_flag)) break;
             tc_fence_after();
             const int h = h0 + j;
             uint8_t* sl = slot(s);
             const float u = expf(reinterpret_cast<const float*>(sl + L::kLo)[r]);
             const float Dh = D[h];
             uint8_t* xrow = sl + L::kXo + r * 128;
-            const uint32_t acc = trow + s * kAccCols;
+            const uint32_t acc = trow + a * kAccCols;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t yd[32], yo[32];
@@ -624,14 +630,17 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 }
             }
             tc_fence_before();
-            mbar_arrive(&bars[BAR_AEMPTY + s]);
+            mbar_arrive(&bars[BAR_AEMPTY + a]);
             fence_proxy_async_smem();                       // y rows -> visible to the TMA unit
             named_bar_sync(2, kEThreads);
             if (etid == 0) {
                 tma_store_3d(&tm_y, h * kP, t0, b, sl + L::kXo);
                 bulk_commit_group();
-                bulk_wait_group_read0();                    // the slot may be refilled now
-                mbar_arrive(&bars[BAR_XEMPTY + s]);
+                // the store of the previous head has read its slot: that slot may be refilled
+                if (j >= 1) {
+                    bulk_wait_group_read1();
+                    mbar_arrive(&bars[BAR_XEMPTY + (j - 1) % kXSlots]);
+                }
             }
         }
         if (etid == 0) bulk_wait_group0();
@@ -750,7 +759,7 @@ cudaError_t walk_t(const Dims& d, const WalkMaps& maps, const TcWorkspace& w, co
     if (e != cudaSuccess) return e;
     const int cpg = walk_ctas_per_group(d);
     const unsigned grid = (unsigned)(d.batch * d.ngroups * cpg);
-    k<<<grid, kWalkThreads, WalkSmem::kBytes, s>>>(maps, w.lam, init_state, final_state, w.himg,
+    k<<<grid, kWalkThreads, WalkSmem::kBytes, s>>>(maps, w.fac, init_state, final_state, w.himg,
                                                     d.nheads, d.ngroups, d.nchunks, cpg,
                                                     device_error_word());
     return cudaGetLastError();
@@ -765,7 +774,7 @@ cudaError_t output_launch(const Dims& d, const CUtensorMap& mx, const CUtensorMa
     if (e != cudaSuccess) return e;
     const int hpc = heads_per_cta(d);
     dim3 grid(d.nchunks, d.nheads / hpc, d.batch);
-    k<<<grid, kOutThreads, OutSmem::kBytes, s>>>(mx, mb, mc, my, w.lam, w.dtT, w.himg, D, d.nheads,
+    k<<<grid, kOutThreads, OutSmem::kBytes, s>>>(mx, mb, mc, my, w.fac, w.himg, D, d.nheads,
                                                 d.ngroups, d.nchunks, hpc, device_error_word());
     return cudaGetLastError();
 }
@@ -794,13 +803,12 @@ size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w)
     const size_t b16_b = up((size_t)d.batch * d.seqlen * d.ngroups * kN * 2);
     if (w) {
         char* p = static_cast<char*>(base);
-        w->lam = reinterpret_cast<float*>(p);
-        w->dtT = reinterpret_cast<float*>(p + lam_b);
-        w->wts = reinterpret_cast<float*>(p + 2 * lam_b);
-        w->himg = reinterpret_cast<uint8_t*>(p + 3 * lam_b);
-        w->b16 = p + 3 * lam_b + himg_b;
+        w->fac = reinterpret_cast<float*>(p);
+        w->wts = reinterpret_cast<float*>(p + 4 * lam_b);
+        w->himg = reinterpret_cast<uint8_t*>(p + 5 * lam_b);
+        w->b16 = p + 5 * lam_b + himg_b;
     }
-    return 3 * lam_b + himg_b + b16_b;
+    return 5 * lam_b + himg_b + b16_b;
 }
 
 cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void* B_f16,

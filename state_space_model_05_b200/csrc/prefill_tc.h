@@ -15,8 +15,9 @@ Dims tc_block_dims(const Dims& d);
 
 // Workspace of the tensor-core path (sized and indexed by the 128-token block dims).
 struct TcWorkspace {
-    float* lam;       // [b][h][c][Q] inclusive cumsum of dt*A within each chunk
-    float* dtT;       // [b][h][c][Q] dt, zero past seqlen
+    float* fac;       // [b][h][c][4][Q] Lam (inclusive cumsum of dt A within each block),
+                      //   dt (zero past seqlen), and the two column factors of each
+                      //   32-token sub-block: exp(Lam_last - Lam_s) dt_s, exp(Lam_first - Lam_s) dt_s
     float* wts;       // [b][h][c][Q] chunk-state weights exp(Lam_end - Lam) dt
     uint8_t* himg;    // [b][h][c] 16 KB bf16 image of each chunk's start state
     void* b16;        // [b][T][G][N] fp16 copy of B (operand of the chunk-state GEMM)

@@ -53,11 +53,15 @@ def test_workspace_bytes(lib):
     lam = b * H * c * Q * 4
     st = b * H * c * P * N * 4
     assert _ws(b, T, H, P, G, N, Q, binding.SSD_F32) == up(lam) + up(st)
-    # tensor-core path (bf16, P 64, N 128, Q 128/256): lam, dt^T and the chunk-state
-    # weights (same layout), bf16 chunk-start-state images, fp16 copy of B
-    himg = b * H * c * 16384
-    b16 = b * T * G * N * 2          # fp16 copy of B for the chunk-state GEMM
-    assert _ws(b, T, H, P, G, N, Q, binding.SSD_BF16) == 3 * up(lam) + up(himg) + up(b16)
+    # tensor-core path (bf16, P 64, N 128, Q 128/256), sized by 128-token blocks: per block
+    # Lam, dt and two column-factor rows, the chunk-state weights, bf16 block-start-state
+    # images, fp16 copy of B
+    def tc_bytes(T):
+        nb = -(-T // 128)
+        lam128 = b * H * nb * 128 * 4
+        return 5 * up(lam128) + up(b * H * nb * 16384) + up(b * T * G * N * 2)
+    assert _ws(b, T, H, P, G, N, Q, binding.SSD_BF16) == tc_bytes(T)
+    assert _ws(b, T, H, P, G, N, 256, binding.SSD_BF16) == tc_bytes(T)
     # bf16 with other shapes uses the CUDA-core layout
     assert _ws(b, T, H, P, G, N, 64, binding.SSD_BF16) == up(b * H * 5 * 64 * 4) + up(b * H * 5 * P * N * 4)
     assert _ws(b, 0, H, P, G, N, Q, binding.SSD_F32) == 0
