@@ -51,9 +51,18 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # ------------------------------------------------------------------ accounting
-def prefill_flops(w) -> dict:
-    """Algorithmic (causal-exact) FLOPs per call, total and per kernel."""
-    b, T, H, P, G, N, Q = (w[k] for k in ("batch", "seqlen", "nheads", "headdim", "ngroups", "dstate", "chunk_len"))
+TC_BLOCK = 128          # token block of the tensor-core path (a 256 chunk = two blocks)
+
+
+def tc_path(w) -> bool:
+    return w["dtype"] == "bf16" and w["headdim"] == 64 and w["dstate"] == 128 and w["chunk_len"] in (128, 256)
+
+
+def prefill_flops(w, q=None) -> dict:
+    """Algorithmic (causal-exact) FLOPs per call for chunk length q (default: the configured
+    chunk), total and per kernel."""
+    b, T, H, P, G, N = (w[k] for k in ("batch", "seqlen", "nheads", "headdim", "ngroups", "dstate"))
+    Q = q or w["chunk_len"]
     tokens = b * T
     gemm1 = tokens * G * (Q + 1) * N          # C B^T, lower triangle incl. diagonal
     gemm2 = tokens * H * (Q + 1) * P          # (masked) X
@@ -64,16 +73,25 @@ def prefill_flops(w) -> dict:
 
 
 def prefill_bytes(w) -> dict:
-    """Algorithmic bytes per call: whole path, and per kernel of the tensor-core path."""
+    """Algorithmic bytes per call: the whole path (x, dt, B, C read once, y and the final
+    state written once), and per kernel of the tensor-core path, counting each kernel's
+    own inputs and outputs once (the per-block state images and decay factors included)."""
     b, T, H, P, G, N, Q = (w[k] for k in ("batch", "seqlen", "nheads", "headdim", "ngroups", "dstate", "chunk_len"))
     e = 2 if w["dtype"] == "bf16" else 4
     c = -(-T // Q)
     io = b * T * (2 * H * P * e + 2 * G * N * e + H * 4) + b * H * P * N * 4
+    nb = -(-T // TC_BLOCK)
+    rows = b * H * nb * TC_BLOCK                 # (b, h, block, token) rows of the factor arrays
+    image = b * H * nb * P * N * 2               # bf16 state at every block start
     return {"total": io,
-            # x and B in, dt/Lam in, one bf16 start-state image per (b, h, chunk) out, final state out
-            "chunk_state_scan_tc": b * T * (H * P * e + G * N * e + 2 * H * 4) + b * H * c * P * N * 2 + b * H * P * N * 4,
-            "state_scan": 2 * b * H * c * P * N * 4 + b * H * P * N * 4,
-            "chunk_cumsum": b * T * H * 4 + 2 * b * H * c * Q * 4}
+            # dt in, fp16 copy of B (read bf16, write fp16), Lam/dt/two column-factor rows and
+            # the chunk-state weights out
+            "chunk_cumsum": b * T * H * 4 + 2 * b * T * G * N * 2 + 5 * rows * 4,
+            # x, fp16 B and the weights in; block-start images and the final state out
+            "chunk_state_scan_tc": b * T * (H * P * e + G * N * 2) + rows * 4 + image + b * H * P * N * 4,
+            # x, B, C, block factors and block-start images in; y out
+            "chunk_output_tc": b * T * (2 * H * P * e + 2 * G * N * e) + 4 * rows * 4 + image,
+            "state_scan": 2 * b * H * c * P * N * 4 + b * H * P * N * 4}
 
 
 def decode_bytes(w) -> int:
@@ -92,11 +110,15 @@ def load_peaks():
 
 
 def kernel_source_sha() -> str:
+    """Hash of every kernel source file (csrc and its subfolders), path and contents."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "state_space_model_05_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+    files = []
+    for dirpath, _, names in os.walk(csrc):
+        files += [os.path.join(dirpath, n) for n in names if n.endswith((".cu", ".cuh", ".h"))]
+    for path in sorted(files):
+        with open(path, "rb") as f:
+            h.update(os.path.relpath(path, csrc).encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -456,24 +478,28 @@ def run_deep_decode(w, steps, warmup, rank, world):
 
 
 def roofline_prefill(w, res, peaks, src, workload):
-    flops = prefill_flops(w)
+    """Roofline of the dominant kernel.  The tensor-core path's kernels sit far below the
+    ridge point (the output kernel does ~60 FLOP per byte it must move), so they are
+    measured against HBM bandwidth; the CUDA-core chunk-state kernel against the tensor
+    peak (the work it stands in for)."""
     byts = prefill_bytes(w)
     kernels = res["kernels"]
     dom = max(kernels, key=lambda k: kernels[k][0])
     ms, n = kernels[dom]
     per_launch_ms = ms / n
-    if dom.startswith("chunk_output") or dom == "chunk_state_simt":
-        work = flops["chunk_output" if dom.startswith("chunk_output") else "chunk_state"]
-        achieved = work / (per_launch_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s"}
-    else:
+    if dom in byts:
         work = byts[dom]
         achieved = work / (per_launch_ms / 1e3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s"}
+    else:
+        work = prefill_flops(w)["chunk_output" if dom.startswith("chunk_output") else "chunk_state"]
+        achieved = work / (per_launch_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s"}
     roof.update({"frac": achieved / peak, "traffic": recorded_traffic(dom, workload), "kernel": dom,
-                 "kernel_ms": per_launch_ms, "peak_source": src})
+                 "kernel_ms": per_launch_ms, "algorithmic_bytes": work if roof["bound"] == "hbm" else None,
+                 "peak_source": src})
     return roof
 
 
@@ -497,8 +523,14 @@ def ours(args, rank, world):
         flops = prefill_flops(w)["total"]
         line.update({"metric": "SSD prefill tokens/s", "value": res["tokens_per_s"], "unit": "tokens/s",
                      "ms_per_step": res["ms_per_step"], "dtype": w["dtype"]})
-        line["prefill_tflops"] = flops / (res["ms_per_step"] / 1e3) / 1e12
+        sec = res["ms_per_step"] / 1e3
+        # tensor-peak fraction of the whole call: FLOPs of the chunked algorithm at the
+        # configured chunk, and (tensor-core path) at the 128-token blocks it executes
+        line["prefill_tflops"] = flops / sec / 1e12
         line["prefill_tensor_frac"] = line["prefill_tflops"] / peaks["bf16_tflops"]
+        if tc_path(w):
+            line["prefill_tflops_executed"] = prefill_flops(w, TC_BLOCK)["total"] / sec / 1e12
+        line["prefill_hbm_gbs"] = prefill_bytes(w)["total"] / sec / 1e9
         line["roofline"] = roofline_prefill(w, res, peaks, src, args.workload)
         line["e2e"] = res.get("e2e")
         line["gpu_launches"] = res["launches"]
@@ -553,9 +585,12 @@ def ours(args, rank, world):
         lw = WORKLOADS["prefill_2p7b_long"]
         l = run_prefill(lw, 5, 2, rank, world, "prefill_2p7b_long", e2e=False)
         fl = prefill_flops(lw)["total"]
+        lsec = l["ms_per_step"] / 1e3
         line["prefill_2p7b_long"] = {"value": l["tokens_per_s"], "unit": "tokens/s", "ms_per_step": l["ms_per_step"],
-                                     "prefill_tflops": fl / (l["ms_per_step"] / 1e3) / 1e12,
-                                     "prefill_tensor_frac": fl / (l["ms_per_step"] / 1e3) / 1e12 / peaks["bf16_tflops"],
+                                     "prefill_tflops": fl / lsec / 1e12,
+                                     "prefill_tensor_frac": fl / lsec / 1e12 / peaks["bf16_tflops"],
+                                     "prefill_tflops_executed": prefill_flops(lw, TC_BLOCK)["total"] / lsec / 1e12,
+                                     "prefill_hbm_gbs": prefill_bytes(lw)["total"] / lsec / 1e9,
                                      "roofline": roofline_prefill(lw, l, peaks, src, "prefill_2p7b_long"),
                                      "kernels_ms": {k: v[0] / v[1] for k, v in l["kernels"].items()}}
     line["clocks"] = clocks.stop()

@@ -1,0 +1,61 @@
+"""Host-side pieces of bench.py that need no GPU: workload accounting, the kernel-source
+hash that keys recorded ncu traffic, and the shape of the roofline record."""
+import os
+
+import bench
+
+
+def test_kernel_source_sha_covers_subfolders(tmp_path, monkeypatch):
+    sha = bench.kernel_source_sha()
+    assert len(sha) == 16 and sha == bench.kernel_source_sha()
+    # a file in a subfolder of csrc changes the hash (the device generator lives in one)
+    root = tmp_path / "repo"
+    (root / "state_space_model_05_b200" / "csrc" / "gen").mkdir(parents=True)
+    (root / "state_space_model_05_b200" / "csrc" / "a.cu").write_text("x")
+    (root / "state_space_model_05_b200" / "csrc" / "gen" / "b.cu").write_text("y")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    h1 = bench.kernel_source_sha()
+    (root / "state_space_model_05_b200" / "csrc" / "gen" / "b.cu").write_text("z")
+    assert bench.kernel_source_sha() != h1
+
+
+def test_recorded_traffic_requires_matching_source(tmp_path, monkeypatch):
+    root = tmp_path / "repo"
+    (root / "state_space_model_05_b200" / "csrc").mkdir(parents=True)
+    (root / "state_space_model_05_b200" / "csrc" / "k.cu").write_text("k")
+    (root / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    sha = bench.kernel_source_sha()
+    (root / "profiles" / "ncu_traffic.txt").write_text(
+        f"kernel=kx workload=wy source_sha={sha} dram_bytes_per_launch=1234\n"
+        f"kernel=kx workload=wz source_sha=0000000000000000 dram_bytes_per_launch=99\n")
+    assert bench.recorded_traffic("kx", "wy") == 1234
+    assert bench.recorded_traffic("kx", "wz") is None
+    assert bench.recorded_traffic("other", "wy") is None
+
+
+def test_prefill_accounting():
+    w = bench.WORKLOADS["prefill_2p7b_long"]
+    b, T, H, P, N = 4, 16384, 80, 64, 128
+    byts = bench.prefill_bytes(w)
+    # whole path: x, y bf16; B, C bf16; dt fp32; final state fp32
+    assert byts["total"] == b * T * (2 * H * P * 2 + 2 * N * 2 + H * 4) + b * H * P * N * 4
+    # the output kernel moves at least x, y and one bf16 state per 128-token block
+    assert byts["chunk_output_tc"] > b * T * 2 * H * P * 2 + b * H * (T // 128) * P * N * 2
+    f256, f128 = bench.prefill_flops(w)["total"], bench.prefill_flops(w, 128)["total"]
+    assert f256 == b * T * ((256 + 1) * N + H * ((256 + 1) * P + 4 * N * P))
+    assert f128 < f256
+    assert bench.tc_path(w) and not bench.tc_path(dict(w, dtype="f32"))
+
+
+def test_roofline_prefill_record():
+    w = bench.WORKLOADS["prefill_130m"]
+    res = {"kernels": {"chunk_cumsum": (1.0, 100), "chunk_state_scan_tc": (4.0, 100),
+                       "chunk_output_tc": (5.0, 100)}}
+    peaks = {"hbm_gbs": 6545.3, "bf16_tflops": 1651.2}
+    r = bench.roofline_prefill(w, res, peaks, "measured", "prefill_130m")
+    assert r["kernel"] == "chunk_output_tc" and r["bound"] == "hbm" and r["unit"] == "GB/s"
+    expect = bench.prefill_bytes(w)["chunk_output_tc"] / (0.05e-3) / 1e9
+    assert abs(r["achieved"] - expect) < 1e-6 * expect
+    assert abs(r["frac"] - r["achieved"] / 6545.3) < 1e-12
+    assert set(r) >= {"bound", "achieved", "peak", "unit", "frac", "traffic"}
