@@ -66,8 +66,9 @@ cudaError_t launch_decode(const Dims& d, ssd_dtype_t dtype, float* state, const 
 // Lambda (within-chunk cumulative sum of dt A) for every (b, h, chunk) row of `fac`:
 // [b][h][c][Q], or with `extras` [b][h][c][4][Q] holding Lambda, dt and the two column
 // factors per 32-token sub-block (exp(Lam_last - Lam_s) dt_s, exp(Lam_first - Lam_s) dt_s;
-// Q a multiple of 32).  Optionally the chunk-state weights exp(Lam_end - Lam_s) dt_s
-// ([b][h][c][Q]) and an fp16 copy of a bf16 B.  Null outputs are skipped.
+// Q a multiple of 32).  Optionally the chunk-state weights exp(Lam_end - Lam_s) dt_s followed
+// by exp(Lam_end) and three zeros ([b][h][c][Q + 4]), and an fp16 copy of a bf16 B.  Null
+// outputs are skipped.
 cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, float* fac,
                                 bool extras, float* wts, const void* b_bf16, void* b_f16,
                                 cudaStream_t s);

@@ -111,13 +111,16 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
             carry = __shfl_sync(0xffffffffu, v, 31);
         }
         if (wts) {
-            // chunk-state weights w_s = exp(Lambda_end - Lambda_s) dt_s (carry = Lambda_end)
+            // chunk-state weights w_s = exp(Lambda_end - Lambda_s) dt_s (carry = Lambda_end),
+            // then the chunk's decay exp(Lambda_end) and zero padding: Q + 4 floats per row
+            float* wr = wts + unit * (Q + 4);
 #pragma unroll
             for (int j = 0; j < kMaxChunk / 32; ++j) {
                 const int t = j * 32 + lane;
                 if (j * 32 >= Q) break;
-                if (t < Q) wts[unit * Q + t] = expf(carry - lv[j]) * dv[j];
+                if (t < Q) wr[t] = expf(carry - lv[j]) * dv[j];
             }
+            if (lane < 4) wr[Q + lane] = lane == 0 ? expf(carry) : 0.f;
         }
     }
 }

@@ -59,23 +59,27 @@ __device__ __forceinline__ uint32_t sw128(int r, int q) { return r * 128 + ((q ^
 // heads in order, so the carried state never leaves the CTA (registers) and no chunk
 // waits for another CTA.  The heads' chunk states form one tcgen05 chain with the heads
 // stacked along N (N = 64 x heads); B_c is staged once per chunk for all of them.
-// Operands stream through a 4-deep ring of 64-row quarter-chunk stages (fp16 B quarter,
-// one X quarter per head, the heads' weights w_s); two TMEM accumulators alternate
-// between chunks.  Warp-specialised: one warp issues the loads, one the MMAs, and eight
-// worker warps (which hold the carried state) form X~ = w o X and update the state;
-// the update of chunk c - 1 runs a stage into chunk c, once its accumulator is complete.
+// Operands stream through a 4-deep ring of 64-row stages (fp16 B rows, one X box per
+// head, the heads' weights w_s and, with a chunk's last stage, its decay exp(Lam_end));
+// two TMEM accumulators alternate between chunks.  Warp-specialised: one warp issues the
+// loads, one the MMAs, and eight worker warps (which hold the carried state) form
+// X~ = w o X and update the state; the update of chunk c - 1 runs a stage into chunk c,
+// once its accumulator is complete.  Each worker warp writes its own 2 KB piece of every
+// bf16 start-state image (the image's 64-byte-swizzled layout makes that piece
+// contiguous) and stores it with one bulk copy, so the update needs no CTA-wide barrier.
 constexpr int kWalkWorkers = 8;                               // warps w, w + 4: TMEM lane quarter w
 constexpr int kWalkThreads = (kWalkWorkers + 2) * 32;         // + load warp + MMA warp
 constexpr int kWalkHeads = 3;                                 // heads per CTA (at most)
 constexpr int kWalkStages = 4;
 constexpr int kQBox = 8192;                                   // one 64-row x 128-byte box
+constexpr int kWRow = 68;                                     // weights per head in a stage (+ decay)
 
 struct WalkSmem {
-    static constexpr int kStageX = 2 * kQBox;                         // after the B quarter
-    static constexpr int kStageW = kStageX + kWalkHeads * kQBox;      // float[heads][64]
+    static constexpr int kStageX = 2 * kQBox;                         // after the B rows
+    static constexpr int kStageW = kStageX + kWalkHeads * kQBox;      // float[heads][68]
     static constexpr int kStageBytes = kStageW + 1024;                // 41 KB
-    static constexpr int kImg = kWalkStages * kStageBytes;            // 2 x 16 KB state images
-    static constexpr int kBar = kImg + 2 * kHImage;                   // full, conv, empty, acc
+    static constexpr int kImg = kWalkStages * kStageBytes;            // state images, one per head
+    static constexpr int kBar = kImg + kWalkHeads * kHImage;          // full, conv, empty, acc
     static constexpr int kSlot = kBar + (3 * kWalkStages + 2) * 8;
     static constexpr int kBytes = kSlot + 16 + 1024;
 };
@@ -85,7 +89,7 @@ static_assert(WalkSmem::kBytes <= 227 * 1024, "walk shared memory");
 struct WalkMaps {
     CUtensorMap x1, x2;          // x as (P, T, H, b), boxes of 1 / 2 heads x 64 rows
     CUtensorMap b;               // fp16 B as (64, T, 2G, b), box: both halves x 64 rows
-    CUtensorMap w;               // weights as (nchunks Q, b H) fp32, box 64 x 3 heads
+    CUtensorMap w;               // weights as (nchunks (Q + 4), b H) fp32, box 68 x 3 heads
 };
 
 template <int Q>
@@ -142,9 +146,9 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
             for (int k = 0; k < total; ++k) {
                 const int st = k % S;
                 if (k >= S && !mbar_wait(&empty[st], ((k / S) + 1) & 1, err)) break;
-                const int c = k / NQ, row = c * Q + (k - c * NQ) * 64;
+                const int c = k / NQ, qq = k - c * NQ, row = c * Q + qq * 64;
                 uint8_t* sg = stage(st);
-                mbar_expect_tx(&full[st], (2 + nh) * kQBox + kWalkHeads * 256);
+                mbar_expect_tx(&full[st], (2 + nh) * kQBox + kWalkHeads * kWRow * 4);
                 tma_load_4d(sg, &maps.b, 0, row, 2 * g, b, &full[st]);
                 int hh = 0;
                 if (nh >= 2) {
@@ -153,7 +157,7 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
                 }
                 if (nh - hh >= 1)
                     tma_load_4d(sg + L::kStageX + hh * kQBox, &maps.x1, 0, row, hlo + hh, b, &full[st]);
-                tma_load_2d(sg + L::kStageW, &maps.w, row, b * nheads + hlo, &full[st]);
+                tma_load_2d(sg + L::kStageW, &maps.w, c * (Q + 4) + qq * 64, b * nheads + hlo, &full[st]);
                 issued = k + 1;
             }
             // the CTA does not exit with loads in flight
@@ -199,65 +203,72 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
         }
         bool ok = true;
 
-        // state update for chunk cc: write the bf16 image of H_cc, then H <- exp(Lam_end) H + S_cc.
-        // The image is the MN-major (p contiguous) 128-byte-swizzled operand tile: row n holds
-        // p = 0..63, its 16-byte chunk j (p = 8j..8j+7) stored at chunk j ^ (n mod 8).  It is
-        // assembled in shared memory (two buffers, alternating per head) and written to
-        // global memory with one bulk copy by thread 0.
-        int img_count = 0;                               // images written so far (buffer parity)
-        auto update = [&](int cc) {
-            float e[kWalkHeads];                         // Lam_end per head
+        // bf16 image of the carried state as the start state of chunk cc.  The image is the
+        // MN-major operand tile with 64-byte swizzle: two p-halves of [128 n][32 p], row n of
+        // a half holding p in four 16-byte chunks, chunk j stored at j ^ ((n / 2) mod 4).
+        // This warp's piece (rows 32 (warp mod 4) .. + 31 of half warp / 4) is contiguous.
+        const uint32_t piece = half * 8192 + (warp & 3) * 2048;
+        auto write_images = [&](int cc) {
+            if (lane == 0) bulk_wait_group_read0();      // this warp's previous stores have read
+            __syncwarp();
 #pragma unroll
-            for (int hh = 0; hh < kWalkHeads; ++hh)
-                e[hh] = hh < nh ? fac[((size_t)(b * nheads + hlo + hh) * nchunks + cc) * 4 * Q + Q - 1] : 0.f;
+            for (int hh = 0; hh < kWalkHeads; ++hh) {
+                if (hh < nh) {
+                    uint8_t* row = sm + L::kImg + hh * kHImage + piece + lane * 64;
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const float* h8 = &Hs[hh][8 * jj];
+                        *reinterpret_cast<uint4*>(row + ((jj ^ ((n >> 1) & 3)) << 4)) =
+                            make_uint4(pack_bf16x2(h8[0], h8[1]), pack_bf16x2(h8[2], h8[3]),
+                                       pack_bf16x2(h8[4], h8[5]), pack_bf16x2(h8[6], h8[7]));
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                for (int hh = 0; hh < nh; ++hh)
+                    bulk_store(himg + ((size_t)(b * nheads + hlo + hh) * nchunks + cc) * kHImage + piece,
+                               sm + L::kImg + hh * kHImage + piece, 2048);
+                bulk_commit_group();
+            }
+        };
+        // H <- exp(Lam_end) H + S_cc: the start state of chunk cc + 1
+        auto update = [&](int cc, const float (&e)[kWalkHeads]) {
             if (ok) ok = mbar_wait(&accb[cc & 1], (cc >> 1) & 1, err);
             tc_fence_after();
             const uint32_t acc = tmem + (cc & 1) * 256 + ((uint32_t)((warp & 3) * 32) << 16) + half * 32;
 #pragma unroll
             for (int hh = 0; hh < kWalkHeads; ++hh) {
                 if (hh < nh) {                           // uniform across the CTA
-                    uint8_t* simg = sm + L::kImg + (img_count & 1) * kHImage;
+                    uint32_t v[32];
+                    tmem_ld16(acc + hh * 64, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+                    tmem_ld16(acc + hh * 64 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const float* h8 = &Hs[hh][8 * jj];
-                        const uint4 v = make_uint4(pack_bf16x2(h8[0], h8[1]), pack_bf16x2(h8[2], h8[3]),
-                                                   pack_bf16x2(h8[4], h8[5]), pack_bf16x2(h8[6], h8[7]));
-                        *reinterpret_cast<uint4*>(simg + n * 128 + (((4 * half + jj) ^ (n & 7)) << 4)) = v;
-                    }
-                    fence_proxy_async_smem();
-                    // the store of the previous image (other buffer) has read its source
-                    // before anyone passes this barrier and overwrites that buffer
-                    if (tid == 0) bulk_wait_group_read0();
-                    named_bar_sync(1, kWalkWorkers * 32);
-                    if (tid == 0) {
-                        bulk_store(himg + ((size_t)(b * nheads + hlo + hh) * nchunks + cc) * kHImage, simg,
-                                   kHImage);
-                        bulk_commit_group();
-                    }
-                    ++img_count;
-                    const float eh = expf(e[hh]);
-#pragma unroll
-                    for (int q16 = 0; q16 < 2; ++q16) {
-                        uint32_t v[16];
-                        tmem_ld16(acc + hh * 64 + q16 * 16, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            Hs[hh][q16 * 16 + j] = fmaf(eh, Hs[hh][q16 * 16 + j], ok ? __uint_as_float(v[j]) : 0.f);
-                    }
+                    for (int j = 0; j < 32; ++j)
+                        Hs[hh][j] = fmaf(e[hh], Hs[hh][j], ok ? __uint_as_float(v[j]) : 0.f);
                 }
             }
             tc_fence_before();
+            if (cc + 1 < nchunks) write_images(cc + 1);
         };
 
+        write_images(0);
+        float e_prev[kWalkHeads] = {0.f, 0.f, 0.f};     // decay of the chunk before the current one
         for (int k = 0; k < total; ++k) {
             const int st = k % S, c = k / NQ, qq = k - c * NQ;
             if (ok) ok = mbar_wait(&full[st], (k / S) & 1, err);
+            float e_cur[kWalkHeads] = {0.f, 0.f, 0.f};
             if (ok) {
                 // X~ = w o X -> fp16 in place; consecutive threads take consecutive
                 // 16-byte chunks; chunk i: head i / 512, row (i / 8) % 64
                 uint4* sx = reinterpret_cast<uint4*>(stage(st) + L::kStageX);
                 const float* sw = reinterpret_cast<const float*>(stage(st) + L::kStageW);
+                if (qq == NQ - 1) {
+#pragma unroll
+                    for (int hh = 0; hh < kWalkHeads; ++hh) e_cur[hh] = sw[hh * kWRow + 64];
+                }
                 constexpr int kPer = kWalkHeads * 512 / (kWalkWorkers * 32);   // chunks per thread
                 constexpr int kBatch = 3;                                       // loads in flight
                 static_assert(kPer % kBatch == 0, "conversion batches");
@@ -270,7 +281,7 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
                         const int i = tid + (j0 + j) * kWalkWorkers * 32;
                         if (i < nh * 512) {
                             u[j] = sx[i];
-                            w[j] = sw[(i >> 9) * 64 + ((i >> 3) & 63)];
+                            w[j] = sw[(i >> 9) * kWRow + ((i >> 3) & 63)];
                         }
                     }
 #pragma unroll
@@ -290,10 +301,16 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&conv[st]);
-            if (qq == 1 && c > 0) update(c - 1);
+            if (qq == NQ - 1) {
+                // the previous chunk's accumulator is complete by now (its MMAs were issued a
+                // chunk ago); its decay was read with that chunk's last stage
+                if (c > 0) update(c - 1, e_prev);
+#pragma unroll
+                for (int hh = 0; hh < kWalkHeads; ++hh) e_prev[hh] = e_cur[hh];
+            }
         }
-        if (nchunks > 0) update(nchunks - 1);
-        if (tid == 0) bulk_wait_group0();
+        if (nchunks > 0) update(nchunks - 1, e_prev);
+        if (lane == 0) bulk_wait_group0();
 #pragma unroll
         for (int hh = 0; hh < kWalkHeads; ++hh) {
             if (hh < nh) {
@@ -471,12 +488,13 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                         (jo < kAccSlots || mbar_try_wait(&bars[BAR_AEMPTY + a], (jo / kAccSlots - 1) & 1))) {
                         tc_fence_after();
                         const uint32_t aH = smem_u32(hslot(jo % kHSlots));
-                        // Yo = C_t H_k^T: A = C (K-major over n), B = H image (MN-major, p contiguous)
+                        // Yo = C_t H_k^T: A = C (K-major over n), B = H image (MN-major, 64-byte
+                        // swizzle: p-halves 8 KB apart, 8-row groups of n 512 B apart)
 #pragma unroll
                         for (int ks = 0; ks < 8; ++ks) {
                             const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
                             umma_f16(tmem + a * kAccCols + 64, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
-                                     smem_desc_sw128(aH + ks * 2048, 8192, 1024), idMN, ks > 0 ? 1u : 0u);
+                                     smem_desc_sw64(aH + ks * 1024, 8192, 512), idMN, ks > 0 ? 1u : 0u);
                         }
                         umma_commit(&bars[BAR_HEMPTY + jo % kHSlots]);
                         ++jo;
@@ -798,17 +816,18 @@ size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w)
 {
     auto up = [](size_t v) { return (v + 255) & ~size_t(255); };
     const size_t BH = (size_t)d.batch * d.nheads;
-    const size_t lam_b = up(BH * d.nchunks * d.chunk_len * sizeof(float));
+    const size_t fac_b = up(BH * d.nchunks * 4 * d.chunk_len * sizeof(float));
+    const size_t wts_b = up(BH * d.nchunks * (d.chunk_len + 4) * sizeof(float));
     const size_t himg_b = up(BH * d.nchunks * kHImage);
     const size_t b16_b = up((size_t)d.batch * d.seqlen * d.ngroups * kN * 2);
     if (w) {
         char* p = static_cast<char*>(base);
         w->fac = reinterpret_cast<float*>(p);
-        w->wts = reinterpret_cast<float*>(p + 4 * lam_b);
-        w->himg = reinterpret_cast<uint8_t*>(p + 5 * lam_b);
-        w->b16 = p + 5 * lam_b + himg_b;
+        w->wts = reinterpret_cast<float*>(p + fac_b);
+        w->himg = reinterpret_cast<uint8_t*>(p + fac_b + wts_b);
+        w->b16 = p + fac_b + wts_b + himg_b;
     }
-    return 5 * lam_b + himg_b + b16_b;
+    return fac_b + wts_b + himg_b + b16_b;
 }
 
 cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void* B_f16,
@@ -826,10 +845,11 @@ cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void*
     const uint64_t bdim[4] = {64, T, 2 * G, Bt};
     const uint64_t bstr[3] = {G * kN * 2, 128, T * G * kN * 2};
     const uint32_t bbox[4] = {64, 64, 2, 1};
-    // weights [b h][c Q] fp32
-    const uint64_t wdim[2] = {(uint64_t)d.nchunks * d.chunk_len, Bt * H};
-    const uint64_t wstr[1] = {(uint64_t)d.nchunks * d.chunk_len * 4};
-    const uint32_t wbox[2] = {64, kWalkHeads};
+    // weights [b h][c][Q + 4] fp32: a box is 68 floats of 3 heads (a stage's 64 weights,
+    // and for the block's last stage the block decay after them)
+    const uint64_t wdim[2] = {(uint64_t)d.nchunks * (d.chunk_len + 4), Bt * H};
+    const uint64_t wstr[1] = {(uint64_t)d.nchunks * (d.chunk_len + 4) * 4};
+    const uint32_t wbox[2] = {kWRow, kWalkHeads};
     if (!encode_map(&m.x1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, x, xdim, xstr, xbox1, true) ||
         !encode_map(&m.x2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, x, xdim, xstr, xbox2, true) ||
         !encode_map(&m.b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, B_f16, bdim, bstr, bbox, true) ||

@@ -18,8 +18,10 @@ struct TcWorkspace {
     float* fac;       // [b][h][c][4][Q] Lam (inclusive cumsum of dt A within each block),
                       //   dt (zero past seqlen), and the two column factors of each
                       //   32-token sub-block: exp(Lam_last - Lam_s) dt_s, exp(Lam_first - Lam_s) dt_s
-    float* wts;       // [b][h][c][Q] chunk-state weights exp(Lam_end - Lam) dt
-    uint8_t* himg;    // [b][h][c] 16 KB bf16 image of each chunk's start state
+    float* wts;       // [b][h][c][Q + 4] chunk-state weights exp(Lam_end - Lam) dt, then
+                      //   exp(Lam_end) and three zeros
+    uint8_t* himg;    // [b][h][c] 16 KB bf16 image of each block's start state (MN-major,
+                      //   64-byte swizzle: two 8 KB p-halves of [128 n][32 p])
     void* b16;        // [b][T][G][N] fp16 copy of B (operand of the chunk-state GEMM)
 };
 size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w);

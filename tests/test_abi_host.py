@@ -54,12 +54,13 @@ def test_workspace_bytes(lib):
     st = b * H * c * P * N * 4
     assert _ws(b, T, H, P, G, N, Q, binding.SSD_F32) == up(lam) + up(st)
     # tensor-core path (bf16, P 64, N 128, Q 128/256), sized by 128-token blocks: per block
-    # Lam, dt and two column-factor rows, the chunk-state weights, bf16 block-start-state
-    # images, fp16 copy of B
+    # Lam, dt and two column-factor rows, the chunk-state weights and block decay, bf16
+    # block-start-state images, fp16 copy of B
     def tc_bytes(T):
         nb = -(-T // 128)
-        lam128 = b * H * nb * 128 * 4
-        return 5 * up(lam128) + up(b * H * nb * 16384) + up(b * T * G * N * 2)
+        fac = b * H * nb * 4 * 128 * 4           # Lam, dt, two column-factor rows
+        wts = b * H * nb * (128 + 4) * 4          # chunk-state weights + block decay
+        return up(fac) + up(wts) + up(b * H * nb * 16384) + up(b * T * G * N * 2)
     assert _ws(b, T, H, P, G, N, Q, binding.SSD_BF16) == tc_bytes(T)
     assert _ws(b, T, H, P, G, N, 256, binding.SSD_BF16) == tc_bytes(T)
     # bf16 with other shapes uses the CUDA-core layout
