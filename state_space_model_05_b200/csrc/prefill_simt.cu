@@ -48,6 +48,8 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
                     int b_row_chunks, int seqlen, int nheads, int Q, int nchunks)
 {
     extern __shared__ float sm_dt[];                   // [Q][kCumsumHeads]
+    // the next kernel of the stream (launched as a programmatic dependent) may stage its setup
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int c = blockIdx.x, h0 = blockIdx.y * kCumsumHeads, b = blockIdx.z;
     if (b_f16) {
         // fp16 copy of this chunk's rows of B (bf16 -> fp16 is exact for these values'

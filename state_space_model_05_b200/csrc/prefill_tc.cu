@@ -138,10 +138,12 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *slot;
+    griddep_launch_dependents();
 
     if (warp == kWalkWorkers) {
         // ---------------------------------------------------------------- loads
         if (lane == 0) {
+            griddep_wait();                              // fp16 B and the weights come from the cumsum kernel
             int issued = 0;
             for (int k = 0; k < total; ++k) {
                 const int st = k % S;
@@ -446,6 +448,7 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             tma_load_3d(sC + kBox, &tm_c, g * kN + 64, t0, b, &bars[BAR_CB]);
             tma_load_3d(pbuf(0), &tm_b, g * kN, t0, b, &bars[BAR_CB]);
             tma_load_3d(pbuf(0) + kBox, &tm_b, g * kN + 64, t0, b, &bars[BAR_CB]);
+            griddep_wait();                              // block factors and state images come from earlier kernels
             for (int j = 0; j < heads_per_cta; ++j) {
                 const int s = j % kXSlots, hs = j % kHSlots;
                 const size_t bh = (size_t)b * nheads + h0 + j;
@@ -746,6 +749,25 @@ int heads_per_cta(const Dims& d)
     return best;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start while the previous
+// kernel of the stream finishes, and waits (griddepcontrol.wait) before reading its output.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 int sm_count()
 {
     static int cache[64] = {0};
@@ -777,10 +799,9 @@ cudaError_t walk_t(const Dims& d, const WalkMaps& maps, const TcWorkspace& w, co
     if (e != cudaSuccess) return e;
     const int cpg = walk_ctas_per_group(d);
     const unsigned grid = (unsigned)(d.batch * d.ngroups * cpg);
-    k<<<grid, kWalkThreads, WalkSmem::kBytes, s>>>(maps, w.fac, init_state, final_state, w.himg,
-                                                    d.nheads, d.ngroups, d.nchunks, cpg,
-                                                    device_error_word());
-    return cudaGetLastError();
+    return launch_dependent(k, dim3(grid), dim3(kWalkThreads), WalkSmem::kBytes, s, maps, w.fac,
+                            init_state, final_state, w.himg, d.nheads, d.ngroups, d.nchunks, cpg,
+                            device_error_word());
 }
 
 cudaError_t output_launch(const Dims& d, const CUtensorMap& mx, const CUtensorMap& mb,
@@ -792,9 +813,8 @@ cudaError_t output_launch(const Dims& d, const CUtensorMap& mx, const CUtensorMa
     if (e != cudaSuccess) return e;
     const int hpc = heads_per_cta(d);
     dim3 grid(d.nchunks, d.nheads / hpc, d.batch);
-    k<<<grid, kOutThreads, OutSmem::kBytes, s>>>(mx, mb, mc, my, w.fac, w.himg, D, d.nheads,
-                                                d.ngroups, d.nchunks, hpc, device_error_word());
-    return cudaGetLastError();
+    return launch_dependent(k, grid, dim3(kOutThreads), OutSmem::kBytes, s, mx, mb, mc, my, w.fac,
+                            w.himg, D, d.nheads, d.ngroups, d.nchunks, hpc, device_error_word());
 }
 
 }  // namespace
