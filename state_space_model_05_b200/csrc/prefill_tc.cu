@@ -657,11 +657,8 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             if (etid == 0) {
                 tma_store_3d(&tm_y, h * kP, t0, b, sl + L::kXo);
                 bulk_commit_group();
-                // the store of the previous head has read its slot: that slot may be refilled
-                if (j >= 1) {
-                    bulk_wait_group_read1();
-                    mbar_arrive(&bars[BAR_XEMPTY + (j - 1) % kXSlots]);
-                }
+                bulk_wait_group_read0();                    // the slot may be refilled now
+                mbar_arrive(&bars[BAR_XEMPTY + s]);
             }
         }
         if (etid == 0) bulk_wait_group0();
