@@ -51,9 +51,6 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Byte offset of 16-byte chunk q of row r in a 128B-swizzled tile.
-__device__ __forceinline__ uint32_t sw128(int r, int q) { return r * 128 + ((q ^ (r & 7)) << 4); }
-
 // ================================================================ chunk states: persistent walk
 // One resident CTA per (batch b, group g, range of 1-3 heads) walks the chunks of its
 // heads in order, so the carried state never leaves the CTA (registers) and no chunk
@@ -357,17 +354,16 @@ constexpr int kBlk = 128;                                // tokens per output bl
 constexpr int kOutThreads = 512;
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpP0 = 4, kWarpE0 = 12;
 constexpr int kPThreads = 256, kEThreads = 128;
-constexpr int kXSlots = 4;                               // x / y operand slots
+constexpr int kXSlots = 6;                               // x / y operand slots
 constexpr int kHSlots = 3;                               // state image slots (freed after Yo)
 constexpr int kAccSlots = 3;                             // TMEM accumulator pairs
-constexpr uint32_t kColG = 384;                          // TMEM columns of G
+constexpr uint32_t kColG = 384;                          // TMEM columns of G, later of the two P buffers
 constexpr uint32_t kAccCols = 128;                       // per accumulator: Yd +0, Yo +64
 
 struct OutSmem {
     static constexpr int kC = 0;                         // C_t [2 n-halves][128 rows][128 B]
-    static constexpr int kP0 = 2 * kBox;                 // B_s (operand of G), then P buffer 0
-    static constexpr int kP1 = kP0 + 2 * kBox;           // P buffer 1
-    static constexpr int kH0 = kP1 + 2 * kBox;           // state image slots (MN-major, 16 KB each)
+    static constexpr int kB = 2 * kBox;                  // B_s (operand of G)
+    static constexpr int kH0 = kB + 2 * kBox;            // state image slots (MN-major, 16 KB each)
     static constexpr int kSlot0 = kH0 + kHSlots * kHImage;  // x slots
     static constexpr int kXo = 0;                        //   x (then y) [128 rows][128 B]
     static constexpr int kLo = kBox;                     //   Lam[128]
@@ -439,15 +435,16 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
 
     auto slot = [&](int s) { return sm + L::kSlot0 + s * L::kSlotBytes; };
     auto hslot = [&](int s) { return sm + L::kH0 + s * kHImage; };
-    auto pbuf = [&](int p) { return sm + (p ? L::kP1 : L::kP0); };
+    // P buffer p: 64 TMEM columns (128 bf16 per row), over G's columns once G is in registers
+    auto pcol = [&](int p) { return kColG + (uint32_t)p * 64; };
 
     if (warp == kWarpTma) {
         if (lane == 0) {
             mbar_expect_tx(&bars[BAR_CB], 4 * kBox);
             tma_load_3d(sC, &tm_c, g * kN, t0, b, &bars[BAR_CB]);
             tma_load_3d(sC + kBox, &tm_c, g * kN + 64, t0, b, &bars[BAR_CB]);
-            tma_load_3d(pbuf(0), &tm_b, g * kN, t0, b, &bars[BAR_CB]);
-            tma_load_3d(pbuf(0) + kBox, &tm_b, g * kN + 64, t0, b, &bars[BAR_CB]);
+            tma_load_3d(sm + L::kB, &tm_b, g * kN, t0, b, &bars[BAR_CB]);
+            tma_load_3d(sm + L::kB + kBox, &tm_b, g * kN + 64, t0, b, &bars[BAR_CB]);
             griddep_wait();                              // block factors and state images come from earlier kernels
             for (int j = 0; j < heads_per_cta; ++j) {
                 const int s = j % kXSlots, hs = j % kHSlots;
@@ -468,7 +465,7 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     } else if (warp == kWarpMma) {
         if (lane == 0 && mbar_wait_or_abort(&bars[BAR_CB], 0, err, abort_flag)) {
             tc_fence_after();
-            const uint32_t aC = smem_u32(sC), aB = smem_u32(pbuf(0));
+            const uint32_t aC = smem_u32(sC), aB = smem_u32(sm + L::kB);
             // G = C_t B_s^T (K = N = 128 state columns) into columns [384, 512)
             const uint32_t idG = idesc_bf16_f32(128, 128, false, false);
 #pragma unroll
@@ -508,12 +505,12 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     const int s = jd % kXSlots, a = jd % kAccSlots, p = jd & 1;
                     if (mbar_try_wait(&bars[BAR_PFULL + p], (jd >> 1) & 1)) {
                         tc_fence_after();
-                        const uint32_t aP = smem_u32(pbuf(p)), aX = smem_u32(slot(s) + L::kXo);
-                        // Yd = P X: A = P (K-major over s), B = X (MN-major, p contiguous)
+                        const uint32_t aX = smem_u32(slot(s) + L::kXo);
+                        // Yd = P X: A = P in TMEM (eight columns per 16 tokens), B = X (MN-major)
 #pragma unroll
                         for (int ks = 0; ks < 8; ++ks)
-                            umma_f16(tmem + a * kAccCols, smem_desc_sw128(aP + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
-                                     smem_desc_sw128(aX + ks * 2048, kBox, 1024), idMN, ks > 0 ? 1u : 0u);
+                            umma_f16_ts(tmem + a * kAccCols, tmem + pcol(p) + ks * 8,
+                                        smem_desc_sw128(aX + ks * 2048, kBox, 1024), idMN, ks > 0 ? 1u : 0u);
                         umma_commit(&bars[BAR_PEMPTY + p]);
                         umma_commit(&bars[BAR_AFULL + a]);
                         ++jd;
@@ -538,12 +535,16 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
         const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
         bool live = mbar_wait_or_abort(&bars[BAR_S], 0, err, abort_flag);
         tc_fence_after();
-        // this thread's G entries (row r, sub-blocks kc0 and kc1), the same for every head
+        // this thread's G entries (row r, sub-blocks kc0 and kc1), the same for every head;
+        // once every P thread holds its entries, G's columns become the P buffers
         const int kc0 = colhalf, kc1 = colhalf + 2;
         uint32_t v0[32], v1[32];
         tmem_ld32(trow + kColG + kc0 * 32, v0);
         tmem_ld32(trow + kColG + kc1 * 32, v1);
         tmem_wait_ld();
+        tc_fence_before();
+        live = named_bar_and(1, kPThreads, live);
+        tc_fence_after();
         // Every thread waits on the barriers itself (bounded), so the loop needs no
         // named barrier; a thread that gives up leaves PFULL incomplete and the MMA
         // thread's bounded wait reports it.
@@ -562,7 +563,6 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             const float* sV = reinterpret_cast<const float*>(sl + L::kVo);
             const float* sW = reinterpret_cast<const float*>(sl + L::kWo);
             const float lam_t = sLam[r];
-            uint8_t* P = pbuf(p);
 #pragma unroll
             for (int w2 = 0; w2 < 2; ++w2) {
                 const int kc = w2 ? kc1 : kc0;
@@ -600,13 +600,9 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                         pk[e] = pack_bf16x2(pa, pb);
                     }
                 }
-                uint8_t* blk = P + (kc >> 1) * kBox;
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4)
-                    *reinterpret_cast<uint4*>(blk + sw128(r, (kc & 1) * 4 + k4)) =
-                        make_uint4(pk[4 * k4], pk[4 * k4 + 1], pk[4 * k4 + 2], pk[4 * k4 + 3]);
+                tmem_st16(trow + pcol(p) + kc * 16, pk);  // tokens 32 kc .. 32 kc + 31 of row r
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars[BAR_PFULL + p]);
         }
