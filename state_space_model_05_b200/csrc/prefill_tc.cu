@@ -66,22 +66,28 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // contiguous) and stores it with one bulk copy, so the update needs no CTA-wide barrier.
 constexpr int kWalkWorkers = 8;                               // warps w, w + 4: TMEM lane quarter w
 constexpr int kWalkThreads = (kWalkWorkers + 2) * 32;         // + load warp + MMA warp
-constexpr int kWalkHeads = 3;                                 // heads per CTA (at most)
-constexpr int kWalkStages = 4;
 constexpr int kQBox = 8192;                                   // one 64-row x 128-byte box
 constexpr int kWRow = 68;                                     // weights per head in a stage (+ decay)
 
-struct WalkSmem {
-    static constexpr int kStageX = 2 * kQBox;                         // after the B rows
-    static constexpr int kStageW = kStageX + kWalkHeads * kQBox;      // float[heads][68]
-    static constexpr int kStageBytes = kStageW + 1024;                // 41 KB
-    static constexpr int kImg = kWalkStages * kStageBytes;            // state images, one per head
-    static constexpr int kBar = kImg + kWalkHeads * kHImage;          // full, conv, empty, acc
-    static constexpr int kSlot = kBar + (3 * kWalkStages + 2) * 8;
+// Two shapes of the walk: up to three heads per CTA, one CTA per SM (many chains per SM);
+// or one head per CTA with two CTAs per SM, so that two latency-bound chains interleave
+// (when all chains fit in two CTAs per SM).
+template <int NH>
+struct WalkCfg {
+    static constexpr int kStages = NH == 1 ? 3 : 4;
+    static constexpr int kCtasPerSm = NH == 1 ? 2 : 1;
+    static constexpr uint32_t kTmemCols = NH == 1 ? 128 : 512;     // two accumulators of 64 NH columns
+    static constexpr uint32_t kAccStride = NH == 1 ? 64 : 256;
+    static constexpr int kStageX = 2 * kQBox;                       // after the B rows
+    static constexpr int kStageW = kStageX + NH * kQBox;            // float[heads][68]
+    static constexpr int kStageBytes = kStageW + 1024;
+    static constexpr int kImg = kStages * kStageBytes;              // state images, one per head
+    static constexpr int kBar = kImg + NH * kHImage;                // full, conv, empty, acc
+    static constexpr int kSlot = kBar + (3 * kStages + 2) * 8;
     static constexpr int kBytes = kSlot + 16 + 1024;
+    static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
+    static_assert(kBytes * kCtasPerSm <= 227 * 1024, "walk shared memory");
 };
-static_assert(WalkSmem::kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
-static_assert(WalkSmem::kBytes <= 227 * 1024, "walk shared memory");
 
 struct WalkMaps {
     CUtensorMap x1, x2;          // x as (P, T, H, b), boxes of 1 / 2 heads x 64 rows
@@ -89,16 +95,16 @@ struct WalkMaps {
     CUtensorMap w;               // weights as (nchunks (Q + 4), b H) fp32, box 68 x 3 heads
 };
 
-template <int Q>
-__global__ void __launch_bounds__(kWalkThreads, 1)
+template <int Q, int NH>
+__global__ void __launch_bounds__(kWalkThreads, WalkCfg<NH>::kCtasPerSm)
 chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __restrict__ fac,
                         const float* __restrict__ init_state, float* final_state,
                         uint8_t* __restrict__ himg, int nheads, int ngroups, int nchunks,
                         int ctas_per_group, int* err)
 {
-    using L = WalkSmem;
+    using L = WalkCfg<NH>;
     constexpr int NQ = Q / 64;                          // stages per chunk
-    constexpr int S = kWalkStages;
+    constexpr int S = L::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::kBar);
@@ -128,7 +134,7 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
         fence_mbar_init();
     }
     if (warp == kWalkWorkers + 1) {
-        tmem_alloc(slot, 512);
+        tmem_alloc(slot, L::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -147,10 +153,10 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
                 if (k >= S && !mbar_wait(&empty[st], ((k / S) + 1) & 1, err)) break;
                 const int c = k / NQ, qq = k - c * NQ, row = c * Q + qq * 64;
                 uint8_t* sg = stage(st);
-                mbar_expect_tx(&full[st], (2 + nh) * kQBox + kWalkHeads * kWRow * 4);
+                mbar_expect_tx(&full[st], (2 + nh) * kQBox + NH * kWRow * 4);
                 tma_load_4d(sg, &maps.b, 0, row, 2 * g, b, &full[st]);
                 int hh = 0;
-                if (nh >= 2) {
+                if (NH > 1 && nh >= 2) {
                     tma_load_4d(sg + L::kStageX + hh * kQBox, &maps.x2, 0, row, hlo + hh, b, &full[st]);
                     hh += 2;
                 }
@@ -175,7 +181,7 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
                 // S_c[n][64 hh + p] += sum_s B_s[n] X~_s[hh][p] over this stage's 64 rows
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    umma_f16(tmem + (c & 1) * 256, smem_desc_sw128(aB + ks * 2048, kQBox, 1024),
+                    umma_f16(tmem + (c & 1) * L::kAccStride, smem_desc_sw128(aB + ks * 2048, kQBox, 1024),
                              smem_desc_sw128(aX + ks * 2048, kQBox, 1024), idesc,
                              (qq > 0 || ks > 0) ? 1u : 0u);
                 umma_commit(&empty[st]);
@@ -190,9 +196,9 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
         // carried state: thread owns column n and rows p = 32 half + pp, for each head
         const int n = (warp & 3) * 32 + lane;
         const int half = warp >> 2;
-        float Hs[kWalkHeads][32];
+        float Hs[NH][32];
 #pragma unroll
-        for (int hh = 0; hh < kWalkHeads; ++hh) {
+        for (int hh = 0; hh < NH; ++hh) {
 #pragma unroll
             for (int pp = 0; pp < 32; ++pp) {
                 const int p = half * 32 + pp;
@@ -211,7 +217,7 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
             if (lane == 0) bulk_wait_group_read0();      // this warp's previous stores have read
             __syncwarp();
 #pragma unroll
-            for (int hh = 0; hh < kWalkHeads; ++hh) {
+            for (int hh = 0; hh < NH; ++hh) {
                 if (hh < nh) {
                     uint8_t* row = sm + L::kImg + hh * kHImage + piece + lane * 64;
 #pragma unroll
@@ -233,12 +239,12 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
             }
         };
         // H <- exp(Lam_end) H + S_cc: the start state of chunk cc + 1
-        auto update = [&](int cc, const float (&e)[kWalkHeads]) {
+        auto update = [&](int cc, const float (&e)[NH]) {
             if (ok) ok = mbar_wait(&accb[cc & 1], (cc >> 1) & 1, err);
             tc_fence_after();
-            const uint32_t acc = tmem + (cc & 1) * 256 + ((uint32_t)((warp & 3) * 32) << 16) + half * 32;
+            const uint32_t acc = tmem + (cc & 1) * L::kAccStride + ((uint32_t)((warp & 3) * 32) << 16) + half * 32;
 #pragma unroll
-            for (int hh = 0; hh < kWalkHeads; ++hh) {
+            for (int hh = 0; hh < NH; ++hh) {
                 if (hh < nh) {                           // uniform across the CTA
                     uint32_t v[32];
                     tmem_ld16(acc + hh * 64, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
@@ -254,11 +260,15 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
         };
 
         write_images(0);
-        float e_prev[kWalkHeads] = {0.f, 0.f, 0.f};     // decay of the chunk before the current one
+        float e_prev[NH];                                // decay of the chunk before the current one
+#pragma unroll
+        for (int hh = 0; hh < NH; ++hh) e_prev[hh] = 0.f;
         for (int k = 0; k < total; ++k) {
             const int st = k % S, c = k / NQ, qq = k - c * NQ;
             if (ok) ok = mbar_wait(&full[st], (k / S) & 1, err);
-            float e_cur[kWalkHeads] = {0.f, 0.f, 0.f};
+            float e_cur[NH];
+#pragma unroll
+            for (int hh = 0; hh < NH; ++hh) e_cur[hh] = 0.f;
             if (ok) {
                 // X~ = w o X -> fp16 in place; consecutive threads take consecutive
                 // 16-byte chunks; chunk i: head i / 512, row (i / 8) % 64
@@ -266,10 +276,10 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
                 const float* sw = reinterpret_cast<const float*>(stage(st) + L::kStageW);
                 if (qq == NQ - 1) {
 #pragma unroll
-                    for (int hh = 0; hh < kWalkHeads; ++hh) e_cur[hh] = sw[hh * kWRow + 64];
+                    for (int hh = 0; hh < NH; ++hh) e_cur[hh] = sw[hh * kWRow + 64];
                 }
-                constexpr int kPer = kWalkHeads * 512 / (kWalkWorkers * 32);   // chunks per thread
-                constexpr int kBatch = 3;                                       // loads in flight
+                constexpr int kPer = NH * 512 / (kWalkWorkers * 32);   // chunks per thread
+                constexpr int kBatch = kPer % 3 == 0 ? 3 : kPer;                // loads in flight
                 static_assert(kPer % kBatch == 0, "conversion batches");
 #pragma unroll
                 for (int j0 = 0; j0 < kPer; j0 += kBatch) {
@@ -305,13 +315,13 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
                 // chunk ago); its decay was read with that chunk's last stage
                 if (c > 0) update(c - 1, e_prev);
 #pragma unroll
-                for (int hh = 0; hh < kWalkHeads; ++hh) e_prev[hh] = e_cur[hh];
+                for (int hh = 0; hh < NH; ++hh) e_prev[hh] = e_cur[hh];
             }
         }
         if (nchunks > 0) update(nchunks - 1, e_prev);
         if (lane == 0) bulk_wait_group0();
 #pragma unroll
-        for (int hh = 0; hh < kWalkHeads; ++hh) {
+        for (int hh = 0; hh < NH; ++hh) {
             if (hh < nh) {
 #pragma unroll
                 for (int pp = 0; pp < 32; ++pp) {
@@ -325,7 +335,7 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
     __syncthreads();
     if (warp == kWalkWorkers + 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, L::kTmemCols);
     }
 }
 
@@ -771,28 +781,35 @@ int sm_count()
     return cache[dev];
 }
 
-// CTAs per (b, g) of the walk: enough that each holds at most 3 heads, and as many as
+// Walk shape: one head per CTA (two CTAs per SM) when every (b, h) chain fits in the
+// SMs that way, else up to three heads per CTA.
+int walk_heads(const Dims& d)
+{
+    return (long long)d.batch * d.nheads <= (long long)WalkCfg<1>::kCtasPerSm * sm_count() ? 1 : 3;
+}
+
+// CTAs per (b, g) of the walk: enough that each holds at most nh heads, and as many as
 // fill the SMs otherwise (never more than there are heads).
-int walk_ctas_per_group(const Dims& d)
+int walk_ctas_per_group(const Dims& d, int nh)
 {
     const int hpg = d.nheads / d.ngroups;
     const int units = d.batch * d.ngroups;
-    int cpg = (hpg + kWalkHeads - 1) / kWalkHeads;
+    int cpg = (hpg + nh - 1) / nh;
     cpg = max(cpg, sm_count() / units);
     return min(cpg, hpg);
 }
 
-template <int Q>
+template <int Q, int NH>
 cudaError_t walk_t(const Dims& d, const WalkMaps& maps, const TcWorkspace& w, const float* init_state,
                    float* final_state, cudaStream_t s)
 {
-    auto k = chunk_state_walk_kernel<Q>;
+    auto k = chunk_state_walk_kernel<Q, NH>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         WalkSmem::kBytes);
+                                         WalkCfg<NH>::kBytes);
     if (e != cudaSuccess) return e;
-    const int cpg = walk_ctas_per_group(d);
+    const int cpg = walk_ctas_per_group(d, NH);
     const unsigned grid = (unsigned)(d.batch * d.ngroups * cpg);
-    return launch_dependent(k, dim3(grid), dim3(kWalkThreads), WalkSmem::kBytes, s, maps, w.fac,
+    return launch_dependent(k, dim3(grid), dim3(kWalkThreads), WalkCfg<NH>::kBytes, s, maps, w.fac,
                             init_state, final_state, w.himg, d.nheads, d.ngroups, d.nchunks, cpg,
                             device_error_word());
 }
@@ -858,18 +875,20 @@ cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void*
     const uint64_t bdim[4] = {64, T, 2 * G, Bt};
     const uint64_t bstr[3] = {G * kN * 2, 128, T * G * kN * 2};
     const uint32_t bbox[4] = {64, 64, 2, 1};
-    // weights [b h][c][Q + 4] fp32: a box is 68 floats of 3 heads (a stage's 64 weights,
-    // and for the block's last stage the block decay after them)
+    // weights [b h][c][Q + 4] fp32: a box is 68 floats of the CTA's heads (a stage's 64
+    // weights, and for the block's last stage the block decay after them)
+    const int nh = walk_heads(d);
     const uint64_t wdim[2] = {(uint64_t)d.nchunks * (d.chunk_len + 4), Bt * H};
     const uint64_t wstr[1] = {(uint64_t)d.nchunks * (d.chunk_len + 4) * 4};
-    const uint32_t wbox[2] = {kWRow, kWalkHeads};
+    const uint32_t wbox[2] = {kWRow, (uint32_t)nh};
     if (!encode_map(&m.x1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, x, xdim, xstr, xbox1, true) ||
         !encode_map(&m.x2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, x, xdim, xstr, xbox2, true) ||
         !encode_map(&m.b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, B_f16, bdim, bstr, bbox, true) ||
         !encode_map(&m.w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, w.wts, wdim, wstr, wbox, false))
         return cudaErrorInvalidValue;
     if (d.chunk_len != kBlk) return cudaErrorInvalidValue;
-    return walk_t<kBlk>(d, m, w, init_state, final_state, s);
+    if (nh == 1) return walk_t<kBlk, 1>(d, m, w, init_state, final_state, s);
+    return walk_t<kBlk, 3>(d, m, w, init_state, final_state, s);
 }
 
 cudaError_t launch_chunk_output_tc(const Dims& d, const void* x, const void* B, const void* C,

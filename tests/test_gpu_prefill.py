@@ -149,6 +149,17 @@ def test_bf16_chunk_length_invariance():
         assert_state(st, so.reshape(st.shape), f"Q={Q}")
 
 
+@pytest.mark.parametrize("G,with_init", [(1, False), (2, True)])
+def test_bf16_many_chains_full(G, with_init):
+    """More (batch, head) chains than two per SM (here 320): the chunk-state walk packs up to
+    three heads per CTA.  Every token and the final state are checked."""
+    inp = problem(gen.SSDShape(4, 384, 80, 64, G, 128), bf16=True, seed=30 + G)
+    init = None
+    if with_init:
+        init = (np.random.default_rng(7).standard_normal((4, 80, 64, 128)) * 0.05).astype(np.float32)
+    _check_bf16(inp, 256, init=init)
+
+
 def test_bf16_27b_long_prefill_sampled():
     """2.7B-shaped long prefill (b=4, T=16384, H=80, P=64, N=128, chunk 256) at full size,
     checked on sampled (batch, head) units: all tokens of y and the final state."""
