@@ -51,6 +51,15 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
     // the next kernel of the stream (launched as a programmatic dependent) may stage its setup
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int c = blockIdx.x, h0 = blockIdx.y * kCumsumHeads, b = blockIdx.z;
+    const int nh = min(kCumsumHeads, nheads - h0);
+    const int t0 = c * Q;
+    // dt rows first, so that their loads and those of the B copy below are in flight together
+    for (int i = threadIdx.x; i < Q * kCumsumHeads; i += blockDim.x) {
+        const int t = i / kCumsumHeads, hh = i - t * kCumsumHeads;
+        float v = 0.f;
+        if (hh < nh && t0 + t < seqlen) v = dt[((size_t)b * seqlen + t0 + t) * nheads + h0 + hh];
+        sm_dt[i] = v;
+    }
     if (b_f16) {
         // fp16 copy of this chunk's rows of B (bf16 -> fp16 is exact for these values'
         // range), the operand format of the tensor-core chunk-state GEMM; the head blocks
@@ -59,22 +68,27 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
         const int r0 = (int)(((long long)rows * blockIdx.y) / gridDim.y);
         const int r1 = (int)(((long long)rows * (blockIdx.y + 1)) / gridDim.y);
         const size_t first = ((size_t)b * seqlen + (size_t)c * Q + r0) * b_row_chunks;
-        for (int i = threadIdx.x; i < (r1 - r0) * b_row_chunks; i += blockDim.x) {
-            uint4 u = b_bf16[first + i];
-            u.x = bf16x2_to_f16x2(u.x);
-            u.y = bf16x2_to_f16x2(u.y);
-            u.z = bf16x2_to_f16x2(u.z);
-            u.w = bf16x2_to_f16x2(u.w);
-            b_f16[first + i] = u;
+        const int n = (r1 - r0) * b_row_chunks;
+        constexpr int kUnroll = 4;
+        for (int i0 = threadIdx.x; i0 < n; i0 += kUnroll * blockDim.x) {
+            uint4 u[kUnroll];
+#pragma unroll
+            for (int j = 0; j < kUnroll; ++j) {
+                const int i = i0 + j * blockDim.x;
+                if (i < n) u[j] = b_bf16[first + i];
+            }
+#pragma unroll
+            for (int j = 0; j < kUnroll; ++j) {
+                const int i = i0 + j * blockDim.x;
+                if (i < n) {
+                    u[j].x = bf16x2_to_f16x2(u[j].x);
+                    u[j].y = bf16x2_to_f16x2(u[j].y);
+                    u[j].z = bf16x2_to_f16x2(u[j].z);
+                    u[j].w = bf16x2_to_f16x2(u[j].w);
+                    b_f16[first + i] = u[j];
+                }
+            }
         }
-    }
-    const int nh = min(kCumsumHeads, nheads - h0);
-    const int t0 = c * Q;
-    for (int i = threadIdx.x; i < Q * kCumsumHeads; i += blockDim.x) {
-        const int t = i / kCumsumHeads, hh = i - t * kCumsumHeads;
-        float v = 0.f;
-        if (hh < nh && t0 + t < seqlen) v = dt[((size_t)b * seqlen + t0 + t) * nheads + h0 + hh];
-        sm_dt[i] = v;
     }
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
