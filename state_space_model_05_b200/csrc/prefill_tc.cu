@@ -1,36 +1,35 @@
 // Tensor-core stages of the bf16 chunked SSD prefill on sm_100a: tcgen05.mma with
-// TMEM accumulators, operands staged in shared memory by TMA (128-byte swizzle).
+// TMEM accumulators, operands staged in shared memory by TMA.
 //
 // "Compiler-First State Space Duality and Portable O(1) Autoregressive Caching for
 // Inference", section "2. Metodologia": the SSD layer is dominated by matrix
 // contractions inside fixed-size chunks, masked by a static lower-triangular decay
 // mask whose exponents are taken in fp32, and chunks communicate only through an
-// N x P state per (batch, head).  Two kernels follow the per-chunk decay cumsum:
+// N x P state per (batch, head).  These stages work in 128-token blocks: a 256-token
+// chunk is two blocks, and the off-diagonal 128 x 128 block of its decay mask enters
+// through the state at the chunk's midpoint, which is that block's exact rank-N
+// factorisation.  After the per-block decay cumsum (prefill_simt.cu) come two kernels:
 //
-// chunk_state_scan_kernel -- one CTA per (chunk c, batch b, head h):
-//     S_c^T = B_c^T (w o X_c),  w_s = exp(Lam_end - Lam_s) dt_s        (tcgen05, fp16 in)
-//     H_{c+1} = exp(Lam_end) H_c + S_c                                  (fp32, look-back)
-//   The carried state goes from chunk to chunk by decoupled look-back: CTAs take
-//   tickets in launch order (chunk-major), so a CTA only ever waits for CTAs that
-//   have already started; the state of chunk c is handed over in an fp32 two-slot
-//   ring per (b, h) that stays in L2, released with a flag.  Every CTA also writes
-//   its chunk's start state H_c once, as the bf16 operand image the output kernel
-//   loads directly, and the last chunk writes the final state.
+// chunk_state_walk_kernel -- persistent: one CTA per (batch b, group g, 1-3 heads) walks
+//   the blocks of its heads in order, the carried state held in the worker threads'
+//   registers (no cross-CTA hand-off):
+//     S_k = B_k^T (w o X_k),  w_s = exp(Lam_end - Lam_s) dt_s         (tcgen05, fp16 in)
+//     H_{k+1} = exp(Lam_end) H_k + S_k                                 (fp32)
+//   and writes every block's start state H_k once, as the bf16 operand image the output
+//   kernel loads, plus the final state.
 //
-// chunk_output_kernel -- one CTA per (chunk c, 128-token tile i, head group, b),
-//   warp-specialised: warp 0 issues TMA loads, warp 1 issues tcgen05.mma, warps 4-11
-//   build the masked matrix P, warps 12-15 run the epilogue.  Per CTA:
-//     G = C_i B_{s < 128(i+1)}^T                (once; shared by the group's heads)
-//   and per head h of the group (double-buffered operands and accumulators):
-//     P = G o exp(Lam_t - Lam_s) o dt_s (s <= t), bf16 in shared memory
-//     Yd = P X,  Yo = C_i H_c^T                 (tcgen05)
+// block_output_kernel -- one CTA per (block k, range of heads of one group, b),
+//   warp-specialised: warp 0 issues TMA and bulk loads, warp 1 issues tcgen05.mma, warps
+//   4-11 build the masked matrix P in TMEM, warps 12-15 run the epilogue:
+//     G  = C_k B_k^T                            (once per CTA; shared by its heads)
+//     P  = G o exp(Lam_t - Lam_s) o dt_s (s <= t), bf16 in TMEM (the MMA's A operand)
+//     Yd = P X,  Yo = C_k H_k^T                 (tcgen05)
 //     y  = Yd + exp(Lam_t) Yo + D_h x_t  -> bf16
-//   Off-diagonal 32-column blocks of P use exp(Lam_t - Lam_r) exp(Lam_r - Lam_s)
-//   with r the block's last column (both factors <= 1); only blocks that cross the
-//   diagonal take one exponential per element.
 //
-// Every wait is bounded; expiry records SSD_ERR_TIMEOUT in the device error word and
-// the CTA drains without further waiting.
+// Both kernels are launched as programmatic dependents: their setup (barriers, TMEM, and
+// for the output kernel the C/B loads and G) overlaps the previous kernel's tail.  Every
+// wait is bounded; expiry records SSD_ERR_TIMEOUT in the device error word and the CTA
+// drains without further waiting.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
