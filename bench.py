@@ -417,9 +417,10 @@ class DeepStack:
     i.i.d. N(0,1) on the device, and fresh per-layer inputs drawn on the device every step
     (counter-based generator; the host can regenerate any element)."""
 
-    def __init__(self, w):
+    def __init__(self, w, one_launch=True):
         import torch
         self.w = w
+        self.one_launch = one_launch
         L, b, H, P, G, N = (w[k] for k in ("layers", "batch", "nheads", "headdim", "ngroups", "dstate"))
         f32 = torch.float32
         self.states = torch.empty((L, b, H, P, N), device="cuda", dtype=f32)
@@ -435,6 +436,10 @@ class DeepStack:
         self.y = torch.empty((L, b, H, P), device="cuda", dtype=f32)
         self.table = _dev(gen.dt_table(), f32)
         self.inv = float(np.float32(1.0 / math.sqrt(N)))
+        from state_space_model_05_b200 import binding
+        self.layers = binding.decode_layer_table(
+            [{"state": self.states[l], "x_t": self.x[l], "dt_t": self.dt[l], "A": self.A[l], "B_t": self.B[l],
+              "C_t": self.C[l], "D": self.D[l], "y_t": self.y[l]} for l in range(L)])
 
     def draw(self, step):
         for l in range(self.w["layers"]):
@@ -445,17 +450,24 @@ class DeepStack:
                              gen.deep_stream(gen.DEEP_DT, l, step))
 
     def step(self):
+        """One token for every layer: one launch for the whole stack, or one per layer."""
         import state_space_model_05_b200 as ssd
-        for l in range(self.w["layers"]):
+        w = self.w
+        if self.one_launch:
+            ssd.ssd_decode_step_layers(self.layers, w["batch"], w["nheads"], w["headdim"], w["ngroups"],
+                                       w["dstate"], self.x.dtype)
+            return
+        for l in range(w["layers"]):
             ssd.ssd_decode_step(self.states[l], self.x[l], self.dt[l], self.A[l], self.B[l], self.C[l],
                                 self.D[l], y_t=self.y[l])
 
 
-def run_deep_decode(w, steps, warmup, rank, world):
-    """Per step: draw the step's inputs (untimed), then time the L decode launches."""
+def run_deep_decode(w, steps, warmup, rank, world, one_launch=True):
+    """Per step: draw the step's inputs (untimed), then time the decode of all L layers
+    (one launch for the stack, or one launch per layer)."""
     import torch
     import state_space_model_05_b200 as ssd
-    stack = DeepStack(w)
+    stack = DeepStack(w, one_launch=one_launch)
     steps = min(steps, w["steps"])
     for k in range(warmup):                         # warm-up steps use their own streams
         stack.draw(w["steps"] + k)
@@ -479,7 +491,8 @@ def run_deep_decode(w, steps, warmup, rank, world):
     L, b, H, P, G, N = (w[k] for k in ("layers", "batch", "nheads", "headdim", "ngroups", "dstate"))
     per_layer = decode_bytes({"batch": b, "nheads": H, "headdim": P, "ngroups": G, "dstate": N})
     res = {"steps_per_s": rate, "ms_per_step": ms / steps, "bytes_per_step": L * per_layer,
-           "gbs": L * per_layer * steps / (ms / 1e3) / 1e9, "launches": steps * L, "steps": steps}
+           "gbs": L * per_layer * steps / (ms / 1e3) / 1e9, "launches": steps * (1 if one_launch else L),
+           "steps": steps}
     del stack
     torch.cuda.empty_cache()
     return res
@@ -550,8 +563,8 @@ def ours(args, rank, world):
         line.update({"metric": "SSD decode steps/s (64-layer stack)", "value": res["steps_per_s"],
                      "unit": "steps/s", "ms_per_step": res["ms_per_step"], "dtype": "f32"})
         line["roofline"] = {"bound": "hbm", "achieved": res["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                            "frac": res["gbs"] / peaks["hbm_gbs"], "traffic": None, "kernel": "decode_step",
-                            "peak_source": src}
+                            "frac": res["gbs"] / peaks["hbm_gbs"], "traffic": None,
+                            "kernel": "decode_layers (all layers, one launch per step)", "peak_source": src}
         line["gpu_launches"] = res["launches"]
         line["e2e"] = None
         cfg = {"workload": args.workload, **{k: w[k] for k in w if k != "kind"}}
@@ -583,12 +596,15 @@ def ours(args, rank, world):
                                    "traffic": recorded_traffic("decode_step", "decode_2p7b"), "peak_source": src},
                                "config": {k: dw[k] for k in dw if k != "kind"}}
         ddw = WORKLOADS["deep_decode_2p7b"]
-        dd = run_deep_decode(ddw, 64, 3, rank, world)
+        dd = run_deep_decode(ddw, 64, 3, rank, world, one_launch=True)
+        dp = run_deep_decode(ddw, 64, 3, rank, world, one_launch=False)
         line["deep_decode_2p7b"] = {"value": dd["steps_per_s"], "unit": "steps/s", "ms_per_step": dd["ms_per_step"],
-                                    "steps_timed": dd["steps"], "roofline": {
+                                    "steps_timed": dd["steps"], "launches_per_step": 1, "roofline": {
                                         "bound": "hbm", "achieved": dd["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                        "frac": dd["gbs"] / peaks["hbm_gbs"], "kernel": "decode_step x 64 layers",
+                                        "frac": dd["gbs"] / peaks["hbm_gbs"], "kernel": "decode_layers (64 layers, one launch)",
                                         "peak_source": src},
+                                    "per_layer_launches": {"value": dp["steps_per_s"], "ms_per_step": dp["ms_per_step"],
+                                                           "gbs": dp["gbs"], "launches_per_step": ddw["layers"]},
                                     "config": {k: ddw[k] for k in ddw if k != "kind"}}
         lw = WORKLOADS["prefill_2p7b_long"]
         l = run_prefill(lw, 5, 2, rank, world, "prefill_2p7b_long", e2e=False)

@@ -119,6 +119,37 @@ ssd_status_t ssd_decode_step(float* state, const void* x_t, const float* dt_t, c
                              void* y_t, void* stream);
 
 /*
+ * One layer's tensors for ssd_decode_step_layers: the arguments of ssd_decode_step for
+ * that layer (device pointers, layouts as there; every pointer 16-byte aligned).
+ */
+typedef struct {
+    float* state;          /* [batch][nheads][headdim][dstate] fp32, in/out */
+    const void* x_t;       /* [batch][nheads][headdim] dtype */
+    const float* dt_t;     /* [batch][nheads] */
+    const float* A;        /* [nheads] */
+    const void* B_t;       /* [batch][ngroups][dstate] dtype */
+    const void* C_t;       /* [batch][ngroups][dstate] dtype */
+    const float* D;        /* [nheads] */
+    void* y_t;             /* [batch][nheads][headdim] dtype */
+} ssd_decode_layer_t;
+
+/*
+ * One decode step of every layer of a stack, in one launch: for each of the n_layers
+ * entries of `layers` (a DEVICE array of ssd_decode_layer_t, read by the kernel), exactly
+ * what ssd_decode_step does for that layer.  All layers share the sizes and dtype.  The
+ * pages run the cache update inside one compiled on-device loop ("Compiler-First State
+ * Space Duality ...", section "2. Metodologia"); this is that idea across layers: one
+ * launch per token for the whole stack.  The sizes are checked on the host
+ * (SSD_ERR_SHAPE/DTYPE, SSD_ERR_NULL for a NULL table); the entries are checked on the
+ * device: an entry with a NULL or misaligned pointer is skipped and records
+ * SSD_ERR_NULL / SSD_ERR_ALIGN in the device error word (ssd_device_status).  The layers'
+ * state buffers must not overlap one another or any input.
+ */
+ssd_status_t ssd_decode_step_layers(const ssd_decode_layer_t* layers, int n_layers, int batch,
+                                    int nheads, int headdim, int ngroups, int dstate,
+                                    ssd_dtype_t dtype, void* stream);
+
+/*
  * ssd_prefill without a workspace argument, for callers that may not allocate
  * device memory (a host framework's execution hook that must stay inside the
  * memory it planned, or code running during a CUDA stream capture, where

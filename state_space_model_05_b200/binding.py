@@ -16,6 +16,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libssd.so")
 
 SSD_OK = 0
+SSD_ERR_NULL = 1
+SSD_ERR_ALIGN = 4
 SSD_ERR_TIMEOUT = 7
 SSD_F32 = 0
 SSD_BF16 = 1
@@ -32,6 +34,7 @@ SIGNATURES = {
     "ssd_prefill_workspace_bytes": ([_I, _I, _I, _I, _I, _I, _I, _I], _Z),
     "ssd_prefill": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _Z, _P], _I),
     "ssd_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
+    "ssd_decode_step_layers": ([_P, _I, _I, _I, _I, _I, _I, _I, _P], _I),
     "ssd_prefill_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P], _I),
     "ssd_device_status": ([_P], _I),
     "ssd_selftest_bounded_waits": ([_P, _P], _I),
@@ -152,6 +155,28 @@ def ssd_decode_step(state, x_t, dt_t, A, B_t, C_t, D, y_t=None, stream=None):
                                _ptr(y_t), _stream(stream))
     _check(st, "ssd_decode_step")
     return y_t
+
+
+# field order of ssd_decode_layer_t
+LAYER_FIELDS = ("state", "x_t", "dt_t", "A", "B_t", "C_t", "D", "y_t")
+
+
+def decode_layer_table(layers, device=None):
+    """Device array of ssd_decode_layer_t (int64 [n_layers][8]) from a list of dicts of
+    tensors keyed by LAYER_FIELDS (their data pointers, in field order)."""
+    rows = [[int(layer[f].data_ptr()) for f in LAYER_FIELDS] for layer in layers]
+    dev = device or layers[0]["state"].device
+    return torch.tensor(rows, dtype=torch.int64, device=dev).reshape(len(rows), len(LAYER_FIELDS))
+
+
+def ssd_decode_step_layers(table, batch, nheads, headdim, ngroups, dstate, dtype, stream=None):
+    """One decode step of every layer in ``table`` (from decode_layer_table), one launch."""
+    if not table.is_cuda or table.dtype != torch.int64 or table.dim() != 2 or table.shape[1] != len(LAYER_FIELDS):
+        raise ValueError("table must be a CUDA int64 [n_layers][8] tensor")
+    code = SSD_BF16 if dtype in (torch.bfloat16, SSD_BF16) else SSD_F32
+    st = lib().ssd_decode_step_layers(_ptr(table), table.shape[0], batch, nheads, headdim, ngroups,
+                                      dstate, code, _stream(stream))
+    _check(st, "ssd_decode_step_layers")
 
 
 def ssd_device_status(stream=None) -> int:

@@ -66,10 +66,10 @@ ssd_status_t prefill_dims(int batch, int seqlen, int nheads, int headdim, int ng
 ssd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
 
 // ---- opt-in kernel profiling: an event pair around each launch -------------------
-enum Stage { kCumsum, kStateTc, kStateSimt, kScan, kOutTc, kOutSimt, kDecode, kCopy, kNumStages };
+enum Stage { kCumsum, kStateTc, kStateSimt, kScan, kOutTc, kOutSimt, kDecode, kCopy, kDecodeLayers, kNumStages };
 const char* const kStageNames[kNumStages] = {"chunk_cumsum", "chunk_state_scan_tc", "chunk_state_simt",
                                               "state_scan", "chunk_output_tc", "chunk_output_simt",
-                                              "decode_step", "copy_state"};
+                                              "decode_step", "copy_state", "decode_step_layers"};
 struct ProfRecord { int stage; cudaEvent_t begin, end; };
 struct Profiler {
     bool on = false;
@@ -126,7 +126,7 @@ using namespace ssd;
 
 extern "C" {
 
-int ssd_abi_version(void) { return 100; }
+int ssd_abi_version(void) { return 101; }
 
 const char* ssd_status_string(ssd_status_t s)
 {
@@ -214,6 +214,23 @@ ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const v
             return launch_chunk_output_simt(d, dtype, x, dt, B, C, D, ws.lam, ws.states, y, s);
         });
     return from_cuda(e);
+}
+
+ssd_status_t ssd_decode_step_layers(const ssd_decode_layer_t* layers, int n_layers, int batch,
+                                    int nheads, int headdim, int ngroups, int dstate,
+                                    ssd_dtype_t dtype, void* stream)
+{
+    ssd_status_t st = check_common(batch, nheads, headdim, ngroups, dstate, dtype, 512);
+    if (st != SSD_OK) return st;
+    if (n_layers < 0 || n_layers > 65535) return SSD_ERR_SHAPE;
+    if (batch == 0 || n_layers == 0) return SSD_OK;
+    if (!layers) return SSD_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(layers) % alignof(ssd_decode_layer_t)) return SSD_ERR_ALIGN;
+    Dims d{batch, 1, nheads, headdim, ngroups, dstate, 1, 1};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return from_cuda(profiled(kDecodeLayers, s, [&] {
+        return launch_decode_layers(d, dtype, layers, n_layers, s);
+    }));
 }
 
 ssd_status_t ssd_decode_step(float* state, const void* x_t, const float* dt_t, const float* A,

@@ -59,6 +59,10 @@ size_t prefill_workspace_layout(const Dims& d, void* base, PrefillWorkspace* ws)
 constexpr int kMaxChunk = 256;               // largest chunk length Q
 
 // ---- launchers (return cudaGetLastError() of their launches) -----------------------
+// Every layer of a stack, one launch (layers: device array of n_layers entries).
+cudaError_t launch_decode_layers(const Dims& d, ssd_dtype_t dtype, const ssd_decode_layer_t* layers,
+                                 int n_layers, cudaStream_t s);
+
 cudaError_t launch_decode(const Dims& d, ssd_dtype_t dtype, float* state, const void* x,
                           const float* dt, const float* A, const void* B, const void* C,
                           const float* D, void* y, cudaStream_t s);

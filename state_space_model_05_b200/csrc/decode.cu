@@ -30,16 +30,16 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// One (b, h) unit of the step, by one CTA.
 // QPL: float4 quads of a state row per lane (dstate <= 128 * QPL).
 // ROWS: rows a warp holds in flight at once.
 template <typename T, int QPL, int ROWS>
-__global__ void __launch_bounds__(kDecodeThreads, QPL == 1 ? 4 : 2)
-decode_step_kernel(float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
-                   const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
-                   const float* __restrict__ D, T* __restrict__ y, int nheads, int headdim,
-                   int ngroups, int dstate)
+__device__ __forceinline__ void decode_unit(float* __restrict__ state, const T* __restrict__ x,
+                                            const float* __restrict__ dt, const float* __restrict__ A,
+                                            const T* __restrict__ Bm, const T* __restrict__ Cm,
+                                            const float* __restrict__ D, T* __restrict__ y, int unit,
+                                            int nheads, int headdim, int ngroups, int dstate)
 {
-    const int unit = blockIdx.x;                       // b * nheads + h
     const int b = unit / nheads;
     const int h = unit - b * nheads;
     const int g = h / (nheads / ngroups);
@@ -115,6 +115,41 @@ decode_step_kernel(float* __restrict__ state, const T* __restrict__ x, const flo
 }
 
 template <typename T, int QPL, int ROWS>
+__global__ void __launch_bounds__(kDecodeThreads, QPL == 1 ? 4 : 2)
+decode_step_kernel(float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
+                   const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
+                   const float* __restrict__ D, T* __restrict__ y, int nheads, int headdim,
+                   int ngroups, int dstate)
+{
+    decode_unit<T, QPL, ROWS>(state, x, dt, A, Bm, Cm, D, y, blockIdx.x, nheads, headdim, ngroups, dstate);
+}
+
+// Every layer of a stack in one launch: blockIdx.y is the layer, whose tensors come from
+// the table.  A layer entry with a null or misaligned pointer is skipped and recorded.
+template <typename T, int QPL, int ROWS>
+__global__ void __launch_bounds__(kDecodeThreads, QPL == 1 ? 4 : 2)
+decode_layers_kernel(const ssd_decode_layer_t* __restrict__ layers, int nheads, int headdim,
+                     int ngroups, int dstate, int* err)
+{
+    const ssd_decode_layer_t L = layers[blockIdx.y];
+    const uintptr_t any = reinterpret_cast<uintptr_t>(L.state) | reinterpret_cast<uintptr_t>(L.x_t) |
+                          reinterpret_cast<uintptr_t>(L.dt_t) | reinterpret_cast<uintptr_t>(L.A) |
+                          reinterpret_cast<uintptr_t>(L.B_t) | reinterpret_cast<uintptr_t>(L.C_t) |
+                          reinterpret_cast<uintptr_t>(L.D) | reinterpret_cast<uintptr_t>(L.y_t);
+    if (!L.state || !L.x_t || !L.dt_t || !L.A || !L.B_t || !L.C_t || !L.D || !L.y_t) {
+        if (threadIdx.x == 0) record_error(err, SSD_ERR_NULL);
+        return;
+    }
+    if (any & 15u) {
+        if (threadIdx.x == 0) record_error(err, SSD_ERR_ALIGN);
+        return;
+    }
+    decode_unit<T, QPL, ROWS>(L.state, static_cast<const T*>(L.x_t), L.dt_t, L.A,
+                              static_cast<const T*>(L.B_t), static_cast<const T*>(L.C_t), L.D,
+                              static_cast<T*>(L.y_t), blockIdx.x, nheads, headdim, ngroups, dstate);
+}
+
+template <typename T, int QPL, int ROWS>
 cudaError_t launch_decode_t(const Dims& d, float* state, const void* x, const float* dt,
                             const float* A, const void* B, const void* C, const float* D, void* y,
                             cudaStream_t s)
@@ -124,6 +159,24 @@ cudaError_t launch_decode_t(const Dims& d, float* state, const void* x, const fl
         state, static_cast<const T*>(x), dt, A, static_cast<const T*>(B), static_cast<const T*>(C),
         D, static_cast<T*>(y), d.nheads, d.headdim, d.ngroups, d.dstate);
     return cudaGetLastError();
+}
+
+template <typename T, int QPL, int ROWS>
+cudaError_t launch_layers_t(const Dims& d, const ssd_decode_layer_t* layers, int n_layers, cudaStream_t s)
+{
+    const dim3 grid((unsigned)(d.batch * d.nheads), (unsigned)n_layers);
+    decode_layers_kernel<T, QPL, ROWS><<<grid, kDecodeThreads, 0, s>>>(layers, d.nheads, d.headdim, d.ngroups,
+                                                                      d.dstate, device_error_word());
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_layers_dtype(const Dims& d, const ssd_decode_layer_t* layers, int n_layers, cudaStream_t s)
+{
+    if (d.dstate <= 128) return launch_layers_t<T, 1, 4>(d, layers, n_layers, s);
+    if (d.dstate <= 256) return launch_layers_t<T, 2, 4>(d, layers, n_layers, s);
+    if (d.dstate <= 512) return launch_layers_t<T, 4, 2>(d, layers, n_layers, s);
+    return cudaErrorInvalidValue;   // rejected earlier by argument validation
 }
 
 template <typename T>
@@ -138,6 +191,14 @@ cudaError_t launch_decode_dtype(const Dims& d, float* state, const void* x, cons
 }
 
 }  // namespace
+
+cudaError_t launch_decode_layers(const Dims& d, ssd_dtype_t dtype, const ssd_decode_layer_t* layers,
+                                 int n_layers, cudaStream_t s)
+{
+    if (d.batch == 0 || n_layers == 0) return cudaSuccess;
+    if (dtype == SSD_F32) return launch_layers_dtype<float>(d, layers, n_layers, s);
+    return launch_layers_dtype<__nv_bfloat16>(d, layers, n_layers, s);
+}
 
 cudaError_t launch_decode(const Dims& d, ssd_dtype_t dtype, float* state, const void* x,
                           const float* dt, const float* A, const void* B, const void* C,

@@ -38,7 +38,7 @@ def test_status_strings(lib):
         s = lib.ssd_status_string(code)
         assert s and s.decode() != "unknown status"
     assert lib.ssd_status_string(99).decode() == "unknown status"
-    assert lib.ssd_abi_version() == 100
+    assert lib.ssd_abi_version() == 101
 
 
 def _ws(*a):
@@ -124,6 +124,19 @@ def test_decode_validation(lib):
     assert _decode(lib, dtype=9) == 3
     assert _decode(lib, batch=-1) == 2
     assert _decode(lib, batch=0) == 0
+
+
+def test_decode_layers_validation(lib):
+    """Sizes are checked on the host before any launch; the table is read only by the kernel."""
+    f = lib.ssd_decode_step_layers
+    assert f(FAKE, 4, 2, 6, 64, 4, 128, binding.SSD_F32, None) == 2      # nheads % ngroups
+    assert f(FAKE, 4, 2, 8, 64, 4, 1024, binding.SSD_F32, None) == 5     # dstate > 512
+    assert f(FAKE, 4, 2, 8, 64, 4, 128, 7, None) == 3                    # dtype
+    assert f(FAKE, -1, 2, 8, 64, 4, 128, binding.SSD_F32, None) == 2     # n_layers
+    assert f(None, 4, 2, 8, 64, 4, 128, binding.SSD_F32, None) == 1      # NULL table
+    assert f(FAKE + 4, 4, 2, 8, 64, 4, 128, binding.SSD_F32, None) == 4  # misaligned table
+    assert f(None, 0, 2, 8, 64, 4, 128, binding.SSD_F32, None) == 0      # nothing to do
+    assert f(None, 4, 0, 8, 64, 4, 128, binding.SSD_F32, None) == 0
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

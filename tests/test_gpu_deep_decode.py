@@ -76,3 +76,49 @@ def test_deep_decode_stack_256_steps_sampled():
         assert_fp32(st_gpu[u], state[0], f"unit {(l, bb, h)} final state")
     del stack
     torch.cuda.empty_cache()
+
+
+def _small_stack(one_launch, layers=4, batch=8):
+    import bench
+    w = dict(bench.WORKLOADS["deep_decode_2p7b"], layers=layers, batch=batch)
+    return bench.DeepStack(w, one_launch=one_launch)
+
+
+def test_one_launch_stack_equals_per_layer_launches():
+    """The stack in one launch does exactly the per-layer steps: bitwise equal states and y."""
+    a, b = _small_stack(True), _small_stack(False)
+    for k in range(5):
+        a.draw(k)
+        b.draw(k)
+        a.step()
+        b.step()
+        torch.cuda.synchronize()
+        assert torch.equal(a.y, b.y), f"y step {k}"
+    assert torch.equal(a.states, b.states)
+    from state_space_model_05_b200 import ssd_device_status
+    assert ssd_device_status() == 0
+
+
+def test_one_launch_stack_skips_and_reports_bad_entries():
+    """An entry with a misaligned or NULL pointer is skipped and recorded in the device error
+    word (checked on the device before any access); the other layers are stepped."""
+    from state_space_model_05_b200 import binding, ssd_device_status
+    a, b = _small_stack(True), _small_stack(False)
+    a.draw(0)
+    b.draw(0)
+    before = a.states.clone()
+    table = a.layers.clone()
+    table[1, 0] += 4                       # layer 1: state pointer off by 4 bytes
+    table[2, 7] = 0                        # layer 2: NULL y pointer
+    w = a.w
+    binding.ssd_decode_step_layers(table, w["batch"], w["nheads"], w["headdim"], w["ngroups"],
+                                   w["dstate"], torch.float32)
+    status = ssd_device_status()
+    assert status in (binding.SSD_ERR_ALIGN, binding.SSD_ERR_NULL)
+    assert ssd_device_status() == 0        # reading clears it
+    b.step()
+    torch.cuda.synchronize()
+    for l in (0, 3):
+        assert torch.equal(a.states[l], b.states[l]), f"layer {l} stepped"
+    for l in (1, 2):
+        assert torch.equal(a.states[l], before[l]), f"layer {l} untouched"
