@@ -44,6 +44,10 @@ WORKLOADS = {
                               ngroups=1, dstate=128, chunk_len=256, dtype="bf16"),
     "decode_2p7b": dict(kind="decode", batch=64, nheads=80, headdim=64, ngroups=1, dstate=128,
                         prefill_len=512, prefill_chunk=64, steps=1024, dtype="f32"),
+    # Gated DeltaNet decode: the page's model shape (16 query/key heads, 32 value heads,
+    # dk = dv = 128) at batch 1 (2 MB of state, L2-resident) and at batch 64 (128 MB, HBM)
+    "gdn_decode_b1": dict(kind="gdn", batch=1, heads_qk=16, heads_v=32, dk=128, dv=128, steps=1024),
+    "gdn_decode_b64": dict(kind="gdn", batch=64, heads_qk=16, heads_v=32, dk=128, dv=128, steps=256),
     "deep_decode_2p7b": dict(kind="deep_decode", layers=64, batch=256, nheads=80, headdim=64, ngroups=1,
                              dstate=128, steps=256, dtype="f32"),
 }
@@ -346,6 +350,57 @@ def run_prefill(w, steps, warmup, rank, world, name, e2e=True):
     return res
 
 
+def gdn_bytes(w) -> int:
+    """Algorithmic bytes of one GDN decode step: the state read and written once, q, k, v,
+    gate, beta read, the output written (fp32)."""
+    b, hqk, hv, dk, dv = (w[k] for k in ("batch", "heads_qk", "heads_v", "dk", "dv"))
+    return 2 * b * hv * dk * dv * 4 + 2 * b * hqk * dk * 4 + 2 * b * hv * dv * 4 + 2 * b * hv * 4
+
+
+def run_gdn(w, repeats, warmup, rank, world):
+    """GDN decode steps with per-step inputs pre-generated on the device, one CUDA graph
+    of ``steps`` launches, timed with CUDA events over graph replays."""
+    import torch
+    import state_space_model_05_b200 as ssd
+    shape = gen.GDNShape(w["batch"], w["heads_qk"], w["heads_v"], w["dk"], w["dv"])
+    S = w["steps"]
+    inp = gen.gdn_inputs(shape, S, seed=20 + rank)
+    f32 = torch.float32
+    Q, K, V, G, Bt = (_dev(a, f32) for a in (inp.q, inp.k, inp.v, inp.gate, inp.beta))
+    state = _dev(inp.state, f32)
+    out = torch.empty((shape.batch, shape.heads_v, shape.dv), device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for t in range(4):
+            ssd.ssd_gdn_decode_step(state, Q[t], K[t], V[t], G[t], Bt[t], out=out)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            for t in range(S):
+                ssd.ssd_gdn_decode_step(state, Q[t], K[t], V[t], G[t], Bt[t], out=out)
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    s0.record()
+    for _ in range(repeats):
+        graph.replay()
+    s1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    if ssd.ssd_device_status() != 0:
+        raise RuntimeError("device status after GDN decode")
+    steps_total = S * repeats
+    rate, ms = whole_job_rate(steps_total, s0.elapsed_time(s1), world)
+    nbytes = gdn_bytes(w)
+    return {"steps_per_s": rate, "us_per_step": ms / steps_total * 1e3, "bytes_per_step": nbytes,
+            "gbs": nbytes * steps_total / (ms / 1e3) / 1e9, "launches": steps_total}
+
+
 def run_decode(w, repeats, warmup, rank, world):
     import torch
     import state_space_model_05_b200 as ssd
@@ -558,6 +613,16 @@ def ours(args, rank, world):
         line["kernels_ms"] = {k: v[0] / v[1] for k, v in res["kernels"].items()}
         cfg = {"workload": args.workload, **{k: w[k] for k in w if k != "kind"},
                "l2": f"inputs rotated over {res['replicas']} resident replicas (> 3x L2) between steps"}
+    elif w["kind"] == "gdn":
+        res = run_gdn(w, max(1, args.steps // 100), max(1, args.warmup // 3), rank, world)
+        line.update({"metric": "GDN decode steps/s", "value": res["steps_per_s"], "unit": "steps/s",
+                     "ms_per_step": res["us_per_step"] / 1e3, "dtype": "f32"})
+        line["roofline"] = {"bound": "hbm", "achieved": res["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": res["gbs"] / peaks["hbm_gbs"], "traffic": None,
+                            "kernel": "gdn_decode_step", "peak_source": src}
+        line["gpu_launches"] = res["launches"]
+        line["e2e"] = None
+        cfg = {"workload": args.workload, **{k: w[k] for k in w if k != "kind"}}
     elif w["kind"] == "deep_decode":
         res = run_deep_decode(w, args.steps, 3, rank, world)
         line.update({"metric": "SSD decode steps/s (64-layer stack)", "value": res["steps_per_s"],
@@ -606,6 +671,15 @@ def ours(args, rank, world):
                                     "per_layer_launches": {"value": dp["steps_per_s"], "ms_per_step": dp["ms_per_step"],
                                                            "gbs": dp["gbs"], "launches_per_step": ddw["layers"]},
                                     "config": {k: ddw[k] for k in ddw if k != "kind"}}
+        for name in ("gdn_decode_b1", "gdn_decode_b64"):
+            gw = WORKLOADS[name]
+            r = run_gdn(gw, 3, 1, rank, world)
+            line[name] = {"value": r["steps_per_s"], "unit": "steps/s", "us_per_step": r["us_per_step"],
+                          "roofline": {"bound": "hbm", "achieved": r["gbs"], "peak": peaks["hbm_gbs"],
+                                       "unit": "GB/s", "frac": r["gbs"] / peaks["hbm_gbs"],
+                                       "kernel": "gdn_decode_step", "peak_source": src,
+                                       "note": "state L2-resident" if gw["batch"] == 1 else "state in HBM"},
+                          "config": {k: gw[k] for k in gw if k != "kind"}}
         lw = WORKLOADS["prefill_2p7b_long"]
         l = run_prefill(lw, 5, 2, rank, world, "prefill_2p7b_long", e2e=False)
         fl = prefill_flops(lw)["total"]

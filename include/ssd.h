@@ -150,6 +150,27 @@ ssd_status_t ssd_decode_step_layers(const ssd_decode_layer_t* layers, int n_laye
                                     ssd_dtype_t dtype, void* stream);
 
 /*
+ * Gated DeltaNet decode step (a second recurrent workload, on its own state cache):
+ * "Persistent-State Dataflow Accelerator for Memory-Bound Linear Attention Decode on
+ * FPGA", section 2.B.  Per (b, value head h), with query/key head hk = h / (heads_v /
+ * heads_qk) (section 2.C: value heads grouped on shared query/key heads):
+ *     dv = beta (v - gate S^T k);   S <- gate S + k dv^T;   out = S^T q  (updated S)
+ * computed as one read pass and one write pass over S (out = gate S_old^T q + (q.k) dv).
+ * The page leaves dv undefined; the gated delta rule above is the reading used.
+ *   state  [batch][heads_v][dk][dv] fp32, in/out (dv innermost)
+ *   q, k   [batch][heads_qk][dk] dtype;  v, out [batch][heads_v][dv] dtype
+ *   gate, beta [batch][heads_v] fp32 (gate in (0, 1], beta in [0, 1] for a contracting
+ *   update; any finite values are computed as given)
+ * Requirements: heads_v % heads_qk == 0; dk a multiple of 8 up to 128; dv a multiple of
+ * 4 up to 128 (else SSD_ERR_SHAPE / SSD_ERR_UNSUPPORTED); 16-byte aligned pointers.
+ * Asynchronous on `stream`; the state buffer must not overlap any input or `out`.
+ */
+ssd_status_t ssd_gdn_decode_step(float* state, const void* q, const void* k, const void* v,
+                                 const float* gate, const float* beta, int batch, int heads_qk,
+                                 int heads_v, int dk, int dv, ssd_dtype_t dtype, void* out,
+                                 void* stream);
+
+/*
  * ssd_prefill without a workspace argument, for callers that may not allocate
  * device memory (a host framework's execution hook that must stay inside the
  * memory it planned, or code running during a CUDA stream capture, where

@@ -35,6 +35,7 @@ SIGNATURES = {
     "ssd_prefill": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _Z, _P], _I),
     "ssd_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ssd_decode_step_layers": ([_P, _I, _I, _I, _I, _I, _I, _I, _P], _I),
+    "ssd_gdn_decode_step": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ssd_prefill_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P], _I),
     "ssd_device_status": ([_P], _I),
     "ssd_selftest_bounded_waits": ([_P, _P], _I),
@@ -177,6 +178,25 @@ def ssd_decode_step_layers(table, batch, nheads, headdim, ngroups, dstate, dtype
     st = lib().ssd_decode_step_layers(_ptr(table), table.shape[0], batch, nheads, headdim, ngroups,
                                       dstate, code, _stream(stream))
     _check(st, "ssd_decode_step_layers")
+
+
+def ssd_gdn_decode_step(state, q, k, v, gate, beta, out=None, stream=None):
+    """One Gated DeltaNet decode step; ``state`` [b][hv][dk][dv] fp32 is updated in place.
+    q, k [b][hqk][dk]; v [b][hv][dv] (fp32 or bf16, all alike); gate, beta [b][hv] fp32.
+    Returns ``out`` [b][hv][dv]."""
+    _need(state, "state", torch.float32)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, q.dtype)
+    for t, n in ((gate, "gate"), (beta, "beta")):
+        _need(t, n, torch.float32)
+    batch, hqk, dk = q.shape
+    hv, dv = v.shape[1], v.shape[2]
+    if out is None:
+        out = torch.empty_like(v)
+    st = lib().ssd_gdn_decode_step(_ptr(state), _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(beta), batch,
+                                   hqk, hv, dk, dv, _dtype_code(q), _ptr(out), _stream(stream))
+    _check(st, "ssd_gdn_decode_step")
+    return out
 
 
 def ssd_device_status(stream=None) -> int:

@@ -66,10 +66,12 @@ ssd_status_t prefill_dims(int batch, int seqlen, int nheads, int headdim, int ng
 ssd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
 
 // ---- opt-in kernel profiling: an event pair around each launch -------------------
-enum Stage { kCumsum, kStateTc, kStateSimt, kScan, kOutTc, kOutSimt, kDecode, kCopy, kDecodeLayers, kNumStages };
+enum Stage { kCumsum, kStateTc, kStateSimt, kScan, kOutTc, kOutSimt, kDecode, kCopy, kDecodeLayers, kGdn,
+             kNumStages };
 const char* const kStageNames[kNumStages] = {"chunk_cumsum", "chunk_state_scan_tc", "chunk_state_simt",
                                               "state_scan", "chunk_output_tc", "chunk_output_simt",
-                                              "decode_step", "copy_state", "decode_step_layers"};
+                                              "decode_step", "copy_state", "decode_step_layers",
+                                              "gdn_decode_step"};
 struct ProfRecord { int stage; cudaEvent_t begin, end; };
 struct Profiler {
     bool on = false;
@@ -214,6 +216,28 @@ ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const v
             return launch_chunk_output_simt(d, dtype, x, dt, B, C, D, ws.lam, ws.states, y, s);
         });
     return from_cuda(e);
+}
+
+ssd_status_t ssd_gdn_decode_step(float* state, const void* q, const void* k, const void* v,
+                                 const float* gate, const float* beta, int batch, int heads_qk,
+                                 int heads_v, int dk, int dv, ssd_dtype_t dtype, void* out,
+                                 void* stream)
+{
+    if (dtype != SSD_F32 && dtype != SSD_BF16) return SSD_ERR_DTYPE;
+    if (batch < 0 || heads_qk <= 0 || heads_v <= 0 || heads_v % heads_qk != 0 || dk <= 0 || dv <= 0 ||
+        dk % 8 != 0 || dv % 4 != 0)
+        return SSD_ERR_SHAPE;
+    if (!gdn_sizes_supported(dk, dv)) return SSD_ERR_UNSUPPORTED;
+    if ((long long)batch * heads_v > 0x7fffffffLL) return SSD_ERR_SHAPE;
+    if (batch == 0) return SSD_OK;
+    if (!state || !q || !k || !v || !gate || !beta || !out) return SSD_ERR_NULL;
+    if (!aligned16(state) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate) ||
+        !aligned16(beta) || !aligned16(out))
+        return SSD_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return from_cuda(profiled(kGdn, s, [&] {
+        return launch_gdn_decode(dtype, state, q, k, v, gate, beta, out, batch, heads_qk, heads_v, dk, dv, s);
+    }));
 }
 
 ssd_status_t ssd_decode_step_layers(const ssd_decode_layer_t* layers, int n_layers, int batch,

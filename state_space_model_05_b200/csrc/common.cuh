@@ -59,6 +59,12 @@ size_t prefill_workspace_layout(const Dims& d, void* base, PrefillWorkspace* ws)
 constexpr int kMaxChunk = 256;               // largest chunk length Q
 
 // ---- launchers (return cudaGetLastError() of their launches) -----------------------
+// Gated DeltaNet decode step (gdn_decode.cu).
+bool gdn_sizes_supported(int dk, int dv);
+cudaError_t launch_gdn_decode(ssd_dtype_t dtype, float* state, const void* q, const void* k,
+                              const void* v, const float* gate, const float* beta, void* out,
+                              int batch, int hqk, int hv, int dk, int dv, cudaStream_t s);
+
 // Every layer of a stack, one launch (layers: device array of n_layers entries).
 cudaError_t launch_decode_layers(const Dims& d, ssd_dtype_t dtype, const ssd_decode_layer_t* layers,
                                  int n_layers, cudaStream_t s);

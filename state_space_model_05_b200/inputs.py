@@ -116,6 +116,41 @@ def state_inputs(batch: int, nheads: int, headdim: int, dstate: int, seed: int =
     return rng.standard_normal((batch, nheads, headdim, dstate), dtype=np.float32)
 
 
+@dataclass
+class GDNShape:
+    batch: int
+    heads_qk: int
+    heads_v: int
+    dk: int
+    dv: int
+
+
+@dataclass
+class GDNInputs:
+    q: np.ndarray       # [steps][b][hqk][dk] fp32, unit rows
+    k: np.ndarray       # [steps][b][hqk][dk] fp32, unit rows
+    v: np.ndarray       # [steps][b][hv][dv] fp32
+    gate: np.ndarray    # [steps][b][hv] fp32 in [0.85, 1)
+    beta: np.ndarray    # [steps][b][hv] fp32 in (0, 1)
+    state: np.ndarray   # [b][hv][dk][dv] fp32, the state before the first step
+
+
+def gdn_inputs(shape: GDNShape, steps: int, seed: int = 3) -> GDNInputs:
+    """Seeded Gated DeltaNet decode inputs (draw order q, k, v, gate, beta, state):
+    q, k unit vectors (normalised N(0, 1) rows), v ~ N(0, 1), gate ~ U(0.85, 1),
+    beta = sigmoid(N(0, 1)), initial state ~ N(0, 0.1^2)."""
+    rng = np.random.default_rng(seed)
+    b, hqk, hv, dk, dv = shape.batch, shape.heads_qk, shape.heads_v, shape.dk, shape.dv
+    unit = lambda a: (a / np.linalg.norm(a, axis=-1, keepdims=True)).astype(np.float32)
+    q = unit(rng.standard_normal((steps, b, hqk, dk)))
+    k = unit(rng.standard_normal((steps, b, hqk, dk)))
+    v = rng.standard_normal((steps, b, hv, dv)).astype(np.float32)
+    gate = rng.uniform(0.85, 1.0, (steps, b, hv)).astype(np.float32)
+    beta = (1.0 / (1.0 + np.exp(-rng.standard_normal((steps, b, hv))))).astype(np.float32)
+    state = (0.1 * rng.standard_normal((b, hv, dk, dv))).astype(np.float32)
+    return GDNInputs(q, k, v, gate, beta, state)
+
+
 def round_bf16(a: np.ndarray) -> np.ndarray:
     """Round fp32 values to the nearest bf16 (ties to even); returned as fp32.
 

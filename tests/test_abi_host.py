@@ -139,6 +139,24 @@ def test_decode_layers_validation(lib):
     assert f(None, 4, 0, 8, 64, 4, 128, binding.SSD_F32, None) == 0
 
 
+def test_gdn_validation(lib):
+    f = lib.ssd_gdn_decode_step
+    F = FAKE
+    args = lambda **kw: [kw.get("state", F), F, F, F, F, F, kw.get("batch", 2), kw.get("hqk", 16),
+                         kw.get("hv", 32), kw.get("dk", 128), kw.get("dv", 128), kw.get("dtype", binding.SSD_F32),
+                         kw.get("out", F), None]
+    assert f(*args(hv=24, hqk=16)) == 2        # value heads not a multiple of query/key heads
+    assert f(*args(dk=12)) == 2                # dk not a multiple of 8
+    assert f(*args(dv=6)) == 2                 # dv not a multiple of 4
+    assert f(*args(dk=256)) == 5               # beyond the supported state
+    assert f(*args(dv=256)) == 5
+    assert f(*args(dtype=4)) == 3
+    assert f(*args(state=None)) == 1
+    assert f(*args(out=F + 8)) == 4
+    assert f(*args(batch=-1)) == 2
+    assert f(*args(batch=0, state=None)) == 0  # nothing to do
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(binding, "_lib", None)
