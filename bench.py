@@ -256,7 +256,7 @@ def prefill_problem(w, seed):
     return inp
 
 
-def run_prefill(w, steps, warmup, rank, world, name, e2e=True):
+def run_prefill(w, steps, warmup, rank, world, name, e2e=True, dt_softplus=False):
     import torch
     import state_space_model_05_b200 as ssd
     from state_space_model_05_b200 import binding
@@ -269,7 +269,8 @@ def run_prefill(w, steps, warmup, rank, world, name, e2e=True):
     replicas = max(1, math.ceil(3 * L2_BYTES / per_replica))
     reps = []
     for _ in range(replicas):
-        reps.append(dict(x=_dev(inp.x, dt_), dt=_dev(inp.dt, torch.float32), A=_dev(inp.A, torch.float32),
+        reps.append(dict(x=_dev(inp.x, dt_), dt=_dev(inp.dt_raw if dt_softplus else inp.dt, torch.float32),
+                         dt_bias=_dev(inp.dt_bias, torch.float32), A=_dev(inp.A, torch.float32),
                          B=_dev(inp.B, dt_), C=_dev(inp.C, dt_), D=_dev(inp.D, torch.float32),
                          y=torch.empty((b, T, H, P), device="cuda", dtype=dt_),
                          st=torch.empty((b, H, P, N), device="cuda", dtype=torch.float32),
@@ -278,7 +279,8 @@ def run_prefill(w, steps, warmup, rank, world, name, e2e=True):
     def step(i):
         r = reps[i % replicas]
         ssd.ssd_prefill(r["x"], r["dt"], r["A"], r["B"], r["C"], r["D"], Q, y=r["y"],
-                        final_state=r["st"], workspace=r["ws"])
+                        final_state=r["st"], workspace=r["ws"], dt_softplus=dt_softplus,
+                        dt_bias=r["dt_bias"] if dt_softplus else None)
 
     for i in range(warmup):
         step(i)
@@ -671,6 +673,11 @@ def ours(args, rank, world):
                                     "per_layer_launches": {"value": dp["steps_per_s"], "ms_per_step": dp["ms_per_step"],
                                                            "gbs": dp["gbs"], "launches_per_step": ddw["layers"]},
                                     "config": {k: ddw[k] for k in ddw if k != "kind"}}
+        # the same headline prefill with dt = softplus(dt_raw + dt_bias) formed in the kernels
+        r = run_prefill(w, 100, 5, rank, world, "prefill_130m_dtraw", e2e=False, dt_softplus=True)
+        line["prefill_130m_dt_softplus"] = {"value": r["tokens_per_s"], "unit": "tokens/s",
+                                            "ms_per_step": r["ms_per_step"],
+                                            "kernels_ms": {k: v[0] / v[1] for k, v in r["kernels"].items()}}
         for name in ("gdn_decode_b1", "gdn_decode_b64"):
             gw = WORKLOADS[name]
             r = run_gdn(gw, 3, 1, rank, world)

@@ -119,6 +119,28 @@ ssd_status_t ssd_decode_step(float* state, const void* x_t, const float* dt_t, c
                              void* y_t, void* stream);
 
 /*
+ * ssd_prefill / ssd_decode_step with the dt pre-processing folded into the kernels: the dt
+ * the recurrence uses is softplus(dt_raw + dt_bias[h]) (softplus(z) = log(1 + exp(z)); z
+ * itself above 40), formed in double precision and rounded to fp32 once, so a caller
+ * passes the projection's raw dt.
+ * dt_raw has dt's layout; dt_bias is [nheads] fp32 (16-byte aligned) or NULL for no bias.
+ * The pages feed the SSD a positive dt and say nothing of how it is produced; this is the
+ * softplus parameterisation of dt the synthetic workloads use (dt = softplus(z + b_h)).
+ * Everything else, including the workspace size, is as for the plain call.
+ */
+ssd_status_t ssd_prefill_dtraw(const void* x, const float* dt_raw, const float* dt_bias,
+                               const float* A, const void* B, const void* C, const float* D,
+                               const float* init_state, int batch, int seqlen, int nheads,
+                               int headdim, int ngroups, int dstate, int chunk_len,
+                               ssd_dtype_t dtype, void* y, float* final_state, void* workspace,
+                               size_t workspace_bytes, void* stream);
+ssd_status_t ssd_decode_step_dtraw(float* state, const void* x_t, const float* dt_raw_t,
+                                   const float* dt_bias, const float* A, const void* B_t,
+                                   const void* C_t, const float* D, int batch, int nheads,
+                                   int headdim, int ngroups, int dstate, ssd_dtype_t dtype,
+                                   void* y_t, void* stream);
+
+/*
  * One layer's tensors for ssd_decode_step_layers: the arguments of ssd_decode_step for
  * that layer (device pointers, layouts as there; every pointer 16-byte aligned).
  */

@@ -60,6 +60,15 @@ def _ptr(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
+def softplus_dt(dt_raw, dt_bias=None):
+    """dt = softplus(dt_raw + dt_bias[h]) in fp64, softplus(z) = log(1 + exp(z)), in the
+    overflow-free form max(z, 0) + log1p(exp(-|z|)).  dt_raw [..][H], dt_bias [H] or None."""
+    z = np.asarray(dt_raw, dtype=np.float64)
+    if dt_bias is not None:
+        z = z + np.asarray(dt_bias, dtype=np.float64)
+    return np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z)))
+
+
 def threads(nthreads: int = 0) -> int:
     return _load().ssd_oracle_threads(int(nthreads))
 

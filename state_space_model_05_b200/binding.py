@@ -36,6 +36,8 @@ SIGNATURES = {
     "ssd_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ssd_decode_step_layers": ([_P, _I, _I, _I, _I, _I, _I, _I, _P], _I),
     "ssd_gdn_decode_step": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
+    "ssd_prefill_dtraw": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _Z, _P], _I),
+    "ssd_decode_step_dtraw": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ssd_prefill_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P], _I),
     "ssd_device_status": ([_P], _I),
     "ssd_selftest_bounded_waits": ([_P, _P], _I),
@@ -114,8 +116,9 @@ def ssd_prefill_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate,
 
 
 def ssd_prefill(x, dt, A, B, C, D, chunk_len, init_state=None, y=None, final_state=None,
-                workspace=None, stream=None):
-    """Chunked SSD prefill.  Shapes as in ``include/ssd.h``; returns ``(y, final_state)``."""
+                workspace=None, stream=None, dt_softplus=False, dt_bias=None):
+    """Chunked SSD prefill.  Shapes as in ``include/ssd.h``; returns ``(y, final_state)``.
+    With ``dt_softplus`` the kernels use softplus(dt + dt_bias) (ssd_prefill_dtraw)."""
     for t, n in ((x, "x"), (B, "B"), (C, "C")):
         _need(t, n, x.dtype)
     for t, n in ((dt, "dt"), (A, "A"), (D, "D")):
@@ -132,6 +135,15 @@ def ssd_prefill(x, dt, A, B, C, D, chunk_len, init_state=None, y=None, final_sta
     need = ssd_prefill_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len, code)
     if workspace is None:
         workspace = torch.empty(max(need, 1), device=x.device, dtype=torch.uint8)
+    if dt_softplus:
+        if dt_bias is not None:
+            _need(dt_bias, "dt_bias", torch.float32)
+        st = lib().ssd_prefill_dtraw(_ptr(x), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                     _ptr(init_state), batch, seqlen, nheads, headdim, ngroups, dstate,
+                                     chunk_len, code, _ptr(y), _ptr(final_state), _ptr(workspace),
+                                     workspace.numel(), _stream(stream))
+        _check(st, "ssd_prefill_dtraw")
+        return y, final_state
     st = lib().ssd_prefill(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state),
                            batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len, code,
                            _ptr(y), _ptr(final_state), _ptr(workspace), workspace.numel(),
@@ -140,8 +152,10 @@ def ssd_prefill(x, dt, A, B, C, D, chunk_len, init_state=None, y=None, final_sta
     return y, final_state
 
 
-def ssd_decode_step(state, x_t, dt_t, A, B_t, C_t, D, y_t=None, stream=None):
-    """One decode step; ``state`` [b][H][P][N] fp32 is updated in place.  Returns ``y_t``."""
+def ssd_decode_step(state, x_t, dt_t, A, B_t, C_t, D, y_t=None, stream=None, dt_softplus=False,
+                    dt_bias=None):
+    """One decode step; ``state`` [b][H][P][N] fp32 is updated in place.  Returns ``y_t``.
+    With ``dt_softplus`` the kernel uses softplus(dt_t + dt_bias) (ssd_decode_step_dtraw)."""
     _need(state, "state", torch.float32)
     for t, n in ((x_t, "x_t"), (B_t, "B_t"), (C_t, "C_t")):
         _need(t, n, x_t.dtype)
@@ -151,6 +165,14 @@ def ssd_decode_step(state, x_t, dt_t, A, B_t, C_t, D, y_t=None, stream=None):
     ngroups, dstate = B_t.shape[1], B_t.shape[2]
     if y_t is None:
         y_t = torch.empty_like(x_t)
+    if dt_softplus:
+        if dt_bias is not None:
+            _need(dt_bias, "dt_bias", torch.float32)
+        st = lib().ssd_decode_step_dtraw(_ptr(state), _ptr(x_t), _ptr(dt_t), _ptr(dt_bias), _ptr(A), _ptr(B_t),
+                                         _ptr(C_t), _ptr(D), batch, nheads, headdim, ngroups, dstate,
+                                         _dtype_code(x_t), _ptr(y_t), _stream(stream))
+        _check(st, "ssd_decode_step_dtraw")
+        return y_t
     st = lib().ssd_decode_step(_ptr(state), _ptr(x_t), _ptr(dt_t), _ptr(A), _ptr(B_t), _ptr(C_t),
                                _ptr(D), batch, nheads, headdim, ngroups, dstate, _dtype_code(x_t),
                                _ptr(y_t), _stream(stream))

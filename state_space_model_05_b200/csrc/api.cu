@@ -158,16 +158,22 @@ size_t ssd_prefill_workspace_bytes(int batch, int seqlen, int nheads, int headdi
     return prefill_workspace_layout(d, nullptr, nullptr);
 }
 
-ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const void* B,
-                         const void* C, const float* D, const float* init_state, int batch,
-                         int seqlen, int nheads, int headdim, int ngroups, int dstate,
-                         int chunk_len, ssd_dtype_t dtype, void* y, float* final_state,
-                         void* workspace, size_t workspace_bytes, void* stream)
+namespace {
+
+// ssd_prefill and ssd_prefill_dtraw: dt_softplus selects dt = softplus(dt_in + dt_bias[h]).
+ssd_status_t prefill_impl(const void* x, const float* dt, const float* dt_bias, int dt_softplus,
+                          const float* A, const void* B, const void* C, const float* D,
+                          const float* init_state, int batch, int seqlen, int nheads, int headdim,
+                          int ngroups, int dstate, int chunk_len, ssd_dtype_t dtype, void* y,
+                          float* final_state, void* workspace, size_t workspace_bytes, void* stream)
 {
     Dims d;
     ssd_status_t st = prefill_dims(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len,
                                    dtype, &d);
     if (st != SSD_OK) return st;
+    if (dt_softplus && dt_bias && !aligned16(dt_bias)) return SSD_ERR_ALIGN;
+    d.dt_bias = dt_bias;
+    d.dt_softplus = dt_softplus;
     if (batch == 0) return SSD_OK;
     if (!final_state) return SSD_ERR_NULL;
     if (!aligned16(final_state) || !aligned16(init_state)) return SSD_ERR_ALIGN;
@@ -218,6 +224,31 @@ ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const v
     return from_cuda(e);
 }
 
+}  // namespace
+
+ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const void* B,
+                         const void* C, const float* D, const float* init_state, int batch,
+                         int seqlen, int nheads, int headdim, int ngroups, int dstate,
+                         int chunk_len, ssd_dtype_t dtype, void* y, float* final_state,
+                         void* workspace, size_t workspace_bytes, void* stream)
+{
+    return prefill_impl(x, dt, nullptr, 0, A, B, C, D, init_state, batch, seqlen, nheads, headdim,
+                        ngroups, dstate, chunk_len, dtype, y, final_state, workspace, workspace_bytes,
+                        stream);
+}
+
+ssd_status_t ssd_prefill_dtraw(const void* x, const float* dt_raw, const float* dt_bias,
+                               const float* A, const void* B, const void* C, const float* D,
+                               const float* init_state, int batch, int seqlen, int nheads,
+                               int headdim, int ngroups, int dstate, int chunk_len,
+                               ssd_dtype_t dtype, void* y, float* final_state, void* workspace,
+                               size_t workspace_bytes, void* stream)
+{
+    return prefill_impl(x, dt_raw, dt_bias, 1, A, B, C, D, init_state, batch, seqlen, nheads, headdim,
+                        ngroups, dstate, chunk_len, dtype, y, final_state, workspace, workspace_bytes,
+                        stream);
+}
+
 ssd_status_t ssd_gdn_decode_step(float* state, const void* q, const void* k, const void* v,
                                  const float* gate, const float* beta, int batch, int heads_qk,
                                  int heads_v, int dk, int dv, ssd_dtype_t dtype, void* out,
@@ -257,23 +288,49 @@ ssd_status_t ssd_decode_step_layers(const ssd_decode_layer_t* layers, int n_laye
     }));
 }
 
-ssd_status_t ssd_decode_step(float* state, const void* x_t, const float* dt_t, const float* A,
-                             const void* B_t, const void* C_t, const float* D, int batch,
-                             int nheads, int headdim, int ngroups, int dstate, ssd_dtype_t dtype,
-                             void* y_t, void* stream)
+namespace {
+
+ssd_status_t decode_impl(float* state, const void* x_t, const float* dt_t, const float* dt_bias,
+                         int dt_softplus, const float* A, const void* B_t, const void* C_t,
+                         const float* D, int batch, int nheads, int headdim, int ngroups, int dstate,
+                         ssd_dtype_t dtype, void* y_t, void* stream)
 {
     ssd_status_t st = check_common(batch, nheads, headdim, ngroups, dstate, dtype, 512);
     if (st != SSD_OK) return st;
     if (batch == 0) return SSD_OK;
     if (!state || !x_t || !dt_t || !A || !B_t || !C_t || !D || !y_t) return SSD_ERR_NULL;
     if (!aligned16(state) || !aligned16(x_t) || !aligned16(dt_t) || !aligned16(A) ||
-        !aligned16(B_t) || !aligned16(C_t) || !aligned16(D) || !aligned16(y_t))
+        !aligned16(B_t) || !aligned16(C_t) || !aligned16(D) || !aligned16(y_t) ||
+        (dt_softplus && dt_bias && !aligned16(dt_bias)))
         return SSD_ERR_ALIGN;
     Dims d{batch, 1, nheads, headdim, ngroups, dstate, 1, 1};
+    d.dt_bias = dt_bias;
+    d.dt_softplus = dt_softplus;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return from_cuda(profiled(kDecode, s, [&] {
         return launch_decode(d, dtype, state, x_t, dt_t, A, B_t, C_t, D, y_t, s);
     }));
+}
+
+}  // namespace
+
+ssd_status_t ssd_decode_step(float* state, const void* x_t, const float* dt_t, const float* A,
+                             const void* B_t, const void* C_t, const float* D, int batch,
+                             int nheads, int headdim, int ngroups, int dstate, ssd_dtype_t dtype,
+                             void* y_t, void* stream)
+{
+    return decode_impl(state, x_t, dt_t, nullptr, 0, A, B_t, C_t, D, batch, nheads, headdim, ngroups,
+                       dstate, dtype, y_t, stream);
+}
+
+ssd_status_t ssd_decode_step_dtraw(float* state, const void* x_t, const float* dt_raw_t,
+                                   const float* dt_bias, const float* A, const void* B_t,
+                                   const void* C_t, const float* D, int batch, int nheads,
+                                   int headdim, int ngroups, int dstate, ssd_dtype_t dtype,
+                                   void* y_t, void* stream)
+{
+    return decode_impl(state, x_t, dt_raw_t, dt_bias, 1, A, B_t, C_t, D, batch, nheads, headdim, ngroups,
+                       dstate, dtype, y_t, stream);
 }
 
 ssd_status_t ssd_device_status(void* stream)

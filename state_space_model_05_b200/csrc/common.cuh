@@ -47,7 +47,21 @@ template <> __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bf
 // ---- problem description passed to every launcher ---------------------------------
 struct Dims {
     int batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len, nchunks;
+    // dt as the kernels use it: dt_in itself, or with dt_softplus softplus(dt_in + dt_bias[h])
+    // (dt_bias may be null: no bias)
+    const float* dt_bias = nullptr;
+    int dt_softplus = 0;
 };
+
+// The dt a kernel uses for head h from the dt input value `in`.  With dt_softplus the sum
+// in + dt_bias[h] and softplus(z) = log(1 + exp(z)) (z itself above 40) are formed in
+// double precision and rounded to fp32 once: for small dt, softplus(z) ~ exp(z) turns an
+// fp32 rounding of z into a relative error of dt that the decay exponents then accumulate.
+__device__ __forceinline__ float dt_value(float in, const float* dt_bias, int dt_softplus, int h) {
+    if (!dt_softplus) return in;
+    const double z = (double)in + (dt_bias ? (double)dt_bias[h] : 0.0);
+    return (float)(z > 40.0 ? z : log1p(exp(z)));
+}
 
 // Workspace layout of the CUDA-core chunked prefill (offsets from the workspace base).
 struct PrefillWorkspace {

@@ -38,7 +38,8 @@ __device__ __forceinline__ void decode_unit(float* __restrict__ state, const T* 
                                             const float* __restrict__ dt, const float* __restrict__ A,
                                             const T* __restrict__ Bm, const T* __restrict__ Cm,
                                             const float* __restrict__ D, T* __restrict__ y, int unit,
-                                            int nheads, int headdim, int ngroups, int dstate)
+                                            int nheads, int headdim, int ngroups, int dstate,
+                                            const float* __restrict__ dt_bias = nullptr, int dt_softplus = 0)
 {
     const int b = unit / nheads;
     const int h = unit - b * nheads;
@@ -47,7 +48,7 @@ __device__ __forceinline__ void decode_unit(float* __restrict__ state, const T* 
     const int warp = threadIdx.x >> 5;
     const int nq = dstate >> 2;                        // quads per row
 
-    const float dtv = dt[unit];
+    const float dtv = dt_value(dt[unit], dt_bias, dt_softplus, h);
     const float a = expf(dtv * A[h]);                  // fp32 decay exponent
     const float Dh = D[h];
 
@@ -119,9 +120,10 @@ __global__ void __launch_bounds__(kDecodeThreads, QPL == 1 ? 4 : 2)
 decode_step_kernel(float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
                    const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
                    const float* __restrict__ D, T* __restrict__ y, int nheads, int headdim,
-                   int ngroups, int dstate)
+                   int ngroups, int dstate, const float* __restrict__ dt_bias, int dt_softplus)
 {
-    decode_unit<T, QPL, ROWS>(state, x, dt, A, Bm, Cm, D, y, blockIdx.x, nheads, headdim, ngroups, dstate);
+    decode_unit<T, QPL, ROWS>(state, x, dt, A, Bm, Cm, D, y, blockIdx.x, nheads, headdim, ngroups, dstate,
+                              dt_bias, dt_softplus);
 }
 
 // Every layer of a stack in one launch: blockIdx.y is the layer, whose tensors come from
@@ -157,7 +159,7 @@ cudaError_t launch_decode_t(const Dims& d, float* state, const void* x, const fl
     const unsigned grid = (unsigned)(d.batch * d.nheads);
     decode_step_kernel<T, QPL, ROWS><<<grid, kDecodeThreads, 0, s>>>(
         state, static_cast<const T*>(x), dt, A, static_cast<const T*>(B), static_cast<const T*>(C),
-        D, static_cast<T*>(y), d.nheads, d.headdim, d.ngroups, d.dstate);
+        D, static_cast<T*>(y), d.nheads, d.headdim, d.ngroups, d.dstate, d.dt_bias, d.dt_softplus);
     return cudaGetLastError();
 }
 

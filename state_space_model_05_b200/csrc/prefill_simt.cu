@@ -45,7 +45,8 @@ __global__ void __launch_bounds__(kThreads)
 chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
                     float* __restrict__ fac, int fac_stride, bool extras, float* __restrict__ wts,
                     const uint4* __restrict__ b_bf16, uint4* __restrict__ b_f16,
-                    int b_row_chunks, int seqlen, int nheads, int Q, int nchunks)
+                    int b_row_chunks, int seqlen, int nheads, int Q, int nchunks,
+                    const float* __restrict__ dt_bias, int dt_softplus)
 {
     extern __shared__ float sm_dt[];                   // [Q][kCumsumHeads]
     // the next kernel of the stream (launched as a programmatic dependent) may stage its setup
@@ -57,7 +58,8 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
     for (int i = threadIdx.x; i < Q * kCumsumHeads; i += blockDim.x) {
         const int t = i / kCumsumHeads, hh = i - t * kCumsumHeads;
         float v = 0.f;
-        if (hh < nh && t0 + t < seqlen) v = dt[((size_t)b * seqlen + t0 + t) * nheads + h0 + hh];
+        if (hh < nh && t0 + t < seqlen)
+            v = dt_value(dt[((size_t)b * seqlen + t0 + t) * nheads + h0 + hh], dt_bias, dt_softplus, h0 + hh);
         sm_dt[i] = v;
     }
     if (b_f16) {
@@ -154,7 +156,8 @@ __global__ void __launch_bounds__(kThreads)
 chunk_state_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
                         const T* __restrict__ Bm, const float* __restrict__ lam,
                         float* __restrict__ states, int seqlen, int nheads, int headdim,
-                        int ngroups, int dstate, int Q, int nchunks)
+                        int ngroups, int dstate, int Q, int nchunks, const float* __restrict__ dt_bias,
+                        int dt_softplus)
 {
     extern __shared__ float sm[];
     float* sx = sm;                                    // [kTokTile][headdim]
@@ -190,7 +193,9 @@ chunk_state_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
             }
             if (threadIdx.x < kTokTile) {
                 const int s = threadIdx.x;
-                sw[s] = s < ns ? expf(lam_end - lamc[s0 + s]) * dt[((size_t)b * seqlen + t0 + s0 + s) * nheads + h] : 0.f;
+                sw[s] = s < ns ? expf(lam_end - lamc[s0 + s]) *
+                                     dt_value(dt[((size_t)b * seqlen + t0 + s0 + s) * nheads + h], dt_bias, dt_softplus, h)
+                               : 0.f;
             }
             __syncthreads();
             if (active) {
@@ -263,7 +268,8 @@ chunk_output_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
                          const T* __restrict__ Bm, const T* __restrict__ Cm,
                          const float* __restrict__ D, const float* __restrict__ lam,
                          const float* __restrict__ states, T* __restrict__ y, int seqlen,
-                         int nheads, int headdim, int ngroups, int dstate, int Q, int nchunks)
+                         int nheads, int headdim, int ngroups, int dstate, int Q, int nchunks,
+                         const float* __restrict__ dt_bias, int dt_softplus)
 {
     extern __shared__ float sm[];
     float* sH = sm;                                    // [headdim][dstate + 1]
@@ -338,7 +344,8 @@ chunk_output_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
             if (threadIdx.x < kTokTile) {
                 const int s = threadIdx.x;
                 sLs[s] = s < ns ? lamc[ss + s] : 0.f;
-                sDs[s] = s < ns ? dt[((size_t)b * seqlen + t0 + ss + s) * nheads + h] : 0.f;
+                sDs[s] = s < ns ? dt_value(dt[((size_t)b * seqlen + t0 + ss + s) * nheads + h], dt_bias, dt_softplus, h)
+                                : 0.f;
             }
             __syncthreads();
             // M tile: thread computes entries (t = i / kTokTile, s = i % kTokTile)
@@ -395,7 +402,7 @@ cudaError_t chunk_state_simt_t(const Dims& d, const void* x, const float* dt, co
     dim3 grid(d.nchunks, d.nheads, d.batch);
     k<<<grid, kThreads, smem, s>>>(static_cast<const T*>(x), dt, static_cast<const T*>(B), lam,
                                    states, d.seqlen, d.nheads, d.headdim, d.ngroups, d.dstate,
-                                   d.chunk_len, d.nchunks);
+                                   d.chunk_len, d.nchunks, d.dt_bias, d.dt_softplus);
     return cudaGetLastError();
 }
 
@@ -415,7 +422,7 @@ cudaError_t chunk_output_simt_t(const Dims& d, const void* x, const float* dt, c
     k<<<grid, kThreads, smem, s>>>(static_cast<const T*>(x), dt, static_cast<const T*>(B),
                                    static_cast<const T*>(C), D, lam, states, static_cast<T*>(y),
                                    d.seqlen, d.nheads, d.headdim, d.ngroups, d.dstate,
-                                   d.chunk_len, d.nchunks);
+                                   d.chunk_len, d.nchunks, d.dt_bias, d.dt_softplus);
     return cudaGetLastError();
 }
 
@@ -438,7 +445,7 @@ cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, 
     chunk_cumsum_kernel<<<grid, kThreads, smem, s>>>(
         dt, A, fac, extras ? 4 * d.chunk_len : d.chunk_len, extras, wts,
         static_cast<const uint4*>(b_bf16), static_cast<uint4*>(b_f16),
-        d.ngroups * d.dstate / 8, d.seqlen, d.nheads, d.chunk_len, d.nchunks);
+        d.ngroups * d.dstate / 8, d.seqlen, d.nheads, d.chunk_len, d.nchunks, d.dt_bias, d.dt_softplus);
     return cudaGetLastError();
 }
 

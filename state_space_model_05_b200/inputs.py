@@ -64,6 +64,8 @@ class PrefillInputs:
     B: np.ndarray    # [batch][seqlen][ngroups][dstate]
     C: np.ndarray    # [batch][seqlen][ngroups][dstate]
     D: np.ndarray    # [nheads]
+    dt_raw: np.ndarray = None   # [batch][seqlen][nheads] fp32: 0.5 z, so dt = softplus(dt_raw + dt_bias)
+    dt_bias: np.ndarray = None  # [nheads] fp32: b_h
 
 
 @dataclass
@@ -94,7 +96,8 @@ def prefill_inputs(shape: SSDShape, seed: int = 0) -> PrefillInputs:
     inv = np.float32(1.0 / math.sqrt(s.dstate))
     B = rng.standard_normal((s.batch, s.seqlen, s.ngroups, s.dstate), dtype=np.float32) * inv
     C = rng.standard_normal((s.batch, s.seqlen, s.ngroups, s.dstate), dtype=np.float32) * inv
-    return PrefillInputs(x=x, dt=dt, A=A, B=B, C=C, D=D)
+    return PrefillInputs(x=x, dt=dt, A=A, B=B, C=C, D=D, dt_raw=(0.5 * z).astype(np.float32),
+                         dt_bias=bias.astype(np.float32))
 
 
 def decode_inputs(shape: SSDShape, steps: int, seed: int = 1) -> DecodeInputs:

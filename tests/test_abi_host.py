@@ -139,6 +139,21 @@ def test_decode_layers_validation(lib):
     assert f(None, 4, 0, 8, 64, 4, 128, binding.SSD_F32, None) == 0
 
 
+def test_dtraw_validation(lib):
+    """The raw-dt variants validate like the plain calls, and reject a misaligned bias
+    (every call here fails validation before any launch)."""
+    F = FAKE
+    f = lib.ssd_decode_step_dtraw
+    assert f(F, F, F, F + 4, F, F, F, F, 2, 8, 64, 4, 128, binding.SSD_F32, F, None) == 4
+    assert f(F, F, F, None, F, F, F, F, 2, 6, 64, 4, 128, binding.SSD_F32, F, None) == 2
+    p = lib.ssd_prefill_dtraw
+    args = [F, F, F + 4, F, F, F, F, None, 2, 300, 4, 64, 1, 128, 128, binding.SSD_BF16, F, F, F, 1 << 30, None]
+    assert p(*args) == 4                                   # misaligned bias
+    args[2] = F
+    args[9] = -1
+    assert p(*args) == 2                                   # bad seqlen
+
+
 def test_gdn_validation(lib):
     f = lib.ssd_gdn_decode_step
     F = FAKE

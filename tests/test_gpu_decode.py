@@ -152,3 +152,27 @@ def test_27b_cached_decode_1024_steps_sampled():
         yo = oracle.decode_step(so, dec.x[k], dec.dt[k], inp.A, dec.B[k], dec.C[k], inp.D, units=units)
         assert_fp32(ys_h[k], yo, f"y step {k}")
     assert_fp32(state.reshape(b * H, P, N)[uidx].cpu().numpy(), so, "state after 1024 steps")
+
+
+def test_dt_softplus_folded_into_decode():
+    """ssd_decode_step_dtraw: dt_t = softplus(dt_raw_t + dt_bias) formed in the kernel; the
+    oracle steps on the fp64 softplus of the same raw values."""
+    from state_space_model_05_b200 import ssd_decode_step
+    b, H, P, G, N = 3, 8, 64, 2, 128
+    s = gen.SSDShape(b, 1, H, P, G, N)
+    rng = np.random.default_rng(77)
+    st0 = rng.standard_normal((b, H, P, N)).astype(np.float32)
+    inp = problem(s, bf16=False, seed=78)
+    dec = gen.decode_inputs(s, steps=4, seed=79)
+    raw = (0.5 * rng.standard_normal((4, b, H))).astype(np.float32)
+    bias = inp.dt_bias
+    state = to_dev(st0)
+    so = st0.reshape(b * H, P, N).astype(np.float64)
+    for k in range(4):
+        x, _, B, C = _decode_dev(dec, k)
+        y = ssd_decode_step(state, x, to_dev(raw[k]), to_dev(inp.A), B, C, to_dev(inp.D), dt_softplus=True,
+                            dt_bias=to_dev(bias))
+        dt64 = oracle.softplus_dt(raw[k], bias)
+        yo = oracle.decode_step(so, dec.x[k], dt64, inp.A, dec.B[k], dec.C[k], inp.D)
+        assert_fp32(y.cpu().numpy().reshape(b * H, P), yo, f"dtraw y step {k}")
+    assert_fp32(state.cpu().numpy().reshape(b * H, P, N), so, "dtraw state")

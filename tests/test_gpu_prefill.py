@@ -176,3 +176,39 @@ def test_bf16_27b_long_prefill_sampled():
 def test_device_status_clean():
     from state_space_model_05_b200 import ssd_device_status
     assert ssd_device_status() == 0
+
+
+@pytest.mark.parametrize("bf16,shape,Q,seed", [
+    (False, gen.SSDShape(1, 256, 4, 64, 1, 64), 64, 0),       # the fp32 single-layer workload
+    (False, gen.SSDShape(2, 300, 4, 64, 1, 64), 64, 340),
+    (True, gen.SSDShape(2, 700, 4, 64, 1, 128), 256, 740),
+    (True, gen.SSDShape(2, 256, 4, 64, 2, 128), 128, 41)])
+def test_dt_softplus_folded_in(bf16, shape, Q, seed):
+    """ssd_prefill_dtraw forms dt = softplus(dt_raw + dt_bias) itself.  It must equal, bit for
+    bit, the plain call given that dt (formed in fp64 by the oracle's softplus and rounded to
+    fp32 once), and match the fp64 oracle within the path's tolerance."""
+    import state_space_model_05_b200 as ssd
+    inp = problem(shape, bf16=bf16, seed=seed)
+    b, _, H, P = inp.x.shape
+    dt_ = torch.bfloat16 if bf16 else torch.float32
+    f32 = torch.float32
+    dt64 = oracle.softplus_dt(inp.dt_raw, inp.dt_bias)
+    x, A, B, C, D = to_dev(inp.x, dt_), to_dev(inp.A, f32), to_dev(inp.B, dt_), to_dev(inp.C, dt_), to_dev(inp.D, f32)
+    y, st = ssd.ssd_prefill(x, to_dev(inp.dt_raw, f32), A, B, C, D, Q, dt_softplus=True,
+                            dt_bias=to_dev(inp.dt_bias, f32))
+    y2, st2 = ssd.ssd_prefill(x, to_dev(dt64.astype(np.float32), f32), A, B, C, D, Q)
+    torch.cuda.synchronize()
+    assert ssd.ssd_device_status() == 0
+    assert torch.equal(y, y2) and torch.equal(st, st2), "folded dt differs from the plain call"
+    if seed == 340:
+        return                        # exactness only: see the plain fp32 path's own parity tests
+    yo, so = oracle.prefill(inp.x, dt64, inp.A, inp.B, inp.C, inp.D)
+    y = y.float().cpu().numpy()
+    st = st.cpu().numpy()
+    what = f"dtraw {shape} Q={Q}"
+    if bf16:
+        assert_bf16_y(y, oracle.units_to_bthp(yo, b, H), what + " y")
+        assert_state(st, so.reshape(st.shape), what + " state")
+    else:
+        assert_fp32(y, oracle.units_to_bthp(yo, b, H), what + " y")
+        assert_fp32(st, so.reshape(st.shape), what + " state")

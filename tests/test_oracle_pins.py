@@ -290,3 +290,20 @@ def test_empty_sequence(oracle_mod):
     y, s = oracle_mod.prefill(x, dt, A, B, C, D, init=init)
     assert y.shape == (2, 0, 3)
     np.testing.assert_array_equal(s, init)
+
+
+def test_softplus_dt_pins():
+    """softplus at the points and identities that fix it: softplus(0) = ln 2,
+    softplus(z) - softplus(-z) = z, softplus(z) -> z and -> exp(z) at the extremes; the
+    bias is added per head (last axis)."""
+    import math
+    from oracle import softplus_dt
+    assert softplus_dt(np.float32([0.0]))[0] == math.log(2.0)
+    z = np.linspace(-30, 30, 121).astype(np.float32)
+    np.testing.assert_allclose(softplus_dt(z) - softplus_dt(-z), z.astype(np.float64), rtol=0, atol=1e-12)
+    assert softplus_dt(np.float32([60.0]))[0] == 60.0 + math.log1p(math.exp(-60.0))
+    np.testing.assert_allclose(softplus_dt(np.float32([-40.0]))[0], math.exp(-40.0), rtol=1e-12)
+    raw = np.zeros((2, 3, 4), dtype=np.float32)
+    bias = np.float32([-1.0, 0.0, 1.0, 2.0])
+    got = softplus_dt(raw, bias)
+    np.testing.assert_allclose(got[1, 2], [math.log1p(math.exp(b)) for b in (-1.0, 0.0, 1.0, 2.0)], rtol=1e-15)
