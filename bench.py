@@ -352,6 +352,59 @@ def run_prefill(w, steps, warmup, rank, world, name, e2e=True, dt_softplus=False
     return res
 
 
+def varlen_lengths(total, seed=0, lo=64, hi=960):
+    """Seeded sequence lengths, uniform in [lo, hi), cut to sum to ``total``."""
+    rng = np.random.default_rng(seed)
+    out = []
+    while sum(out) < total:
+        out.append(int(rng.integers(lo, hi)))
+    out[-1] -= sum(out) - total
+    return out
+
+
+def run_prefill_varlen(w, steps, warmup, rank, world):
+    """The prefill workload's tokens as one packed batch of mixed-length sequences."""
+    import torch
+    import state_space_model_05_b200 as ssd
+    b, T, H, P, G, N, Q = (w[k] for k in ("batch", "seqlen", "nheads", "headdim", "ngroups", "dstate", "chunk_len"))
+    total = b * T
+    lengths = varlen_lengths(total, seed=rank)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32, device="cuda")
+    inp = prefill_problem(dict(w, batch=1, seqlen=total), seed=rank)
+    bf, f32 = torch.bfloat16, torch.float32
+    per = total * (2 * H * P * 2 + 2 * G * N * 2 + H * 4) + 2 * len(lengths) * H * P * N * 4
+    replicas = max(1, math.ceil(3 * L2_BYTES / per))
+    reps = [dict(x=_dev(inp.x[0], bf), dt=_dev(inp.dt[0], f32), A=_dev(inp.A, f32), B=_dev(inp.B[0], bf),
+                 C=_dev(inp.C[0], bf), D=_dev(inp.D, f32)) for _ in range(replicas)]
+    for r in reps:
+        r["y"], r["st"] = ssd.ssd_prefill_varlen(r["x"], r["dt"], r["A"], r["B"], r["C"], r["D"], cu, Q)
+    nbytes = int(ssd.binding.lib().ssd_prefill_varlen_workspace_bytes(len(lengths), total, H, P, G, N, Q, 1))
+    wsp = torch.empty(nbytes, device="cuda", dtype=torch.uint8)
+
+    def step(i):
+        r = reps[i % replicas]
+        ssd.ssd_prefill_varlen(r["x"], r["dt"], r["A"], r["B"], r["C"], r["D"], cu, Q, y=r["y"],
+                               final_states=r["st"], workspace=wsp)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    s0.record()
+    for i in range(steps):
+        step(i)
+    s1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    if ssd.ssd_device_status() != 0:
+        raise RuntimeError("device status after varlen prefill")
+    rate, ms = whole_job_rate(total * steps, s0.elapsed_time(s1), world)
+    return {"tokens_per_s": rate, "ms_per_step": ms / steps, "nseq": len(lengths),
+            "lengths": f"{len(lengths)} sequences, {min(lengths)}..{max(lengths)} tokens (seeded)"}
+
+
 def gdn_bytes(w) -> int:
     """Algorithmic bytes of one GDN decode step: the state read and written once, q, k, v,
     gate, beta read, the output written (fp32)."""
@@ -678,6 +731,10 @@ def ours(args, rank, world):
         line["prefill_130m_dt_softplus"] = {"value": r["tokens_per_s"], "unit": "tokens/s",
                                             "ms_per_step": r["ms_per_step"],
                                             "kernels_ms": {k: v[0] / v[1] for k, v in r["kernels"].items()}}
+        # the same tokens as one packed batch of mixed-length sequences (state reset per sequence)
+        vr = run_prefill_varlen(w, 100, 5, rank, world)
+        line["prefill_130m_varlen"] = {"value": vr["tokens_per_s"], "unit": "tokens/s",
+                                       "ms_per_step": vr["ms_per_step"], "sequences": vr["lengths"]}
         for name in ("gdn_decode_b1", "gdn_decode_b64"):
             gw = WORKLOADS[name]
             r = run_gdn(gw, 3, 1, rank, world)

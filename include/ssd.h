@@ -141,6 +141,31 @@ ssd_status_t ssd_decode_step_dtraw(float* state, const void* x_t, const float* d
                                    void* y_t, void* stream);
 
 /*
+ * Packed variable-length prefill: nseq sequences laid end to end along one token axis, the
+ * state reset at every sequence start.  Sequence i is tokens cu_seqlens[i] ..
+ * cu_seqlens[i + 1] - 1 of x, dt, B, C and y, which have the layouts of ssd_prefill with
+ * batch 1 and seqlen = total_tokens; it starts from init_states[i] (NULL: zeros) and ends in
+ * final_states[i] ([nseq][nheads][headdim][dstate] fp32).  Equivalent to one ssd_prefill per
+ * sequence, in one call; the pages' cache carries one state per sequence ("Compiler-First
+ * State Space Duality ...", section "2. Metodologia"), and this is prefill of many cached
+ * sequences at once.
+ *   cu_seqlens: DEVICE array of nseq + 1 int32 offsets, read by the kernels: cu_seqlens[0]
+ *   = 0, non-decreasing, cu_seqlens[nseq] = total_tokens (else SSD_ERR_SHAPE is recorded
+ *   in the device error word and nothing is computed).  Empty sequences are allowed.
+ * Supported on the tensor-core path only: bf16, headdim 64, dstate 128, chunk_len 128 or
+ * 256 (else SSD_ERR_UNSUPPORTED).  `workspace` must hold
+ * ssd_prefill_varlen_workspace_bytes(...) bytes (0 when total_tokens is 0).
+ */
+size_t ssd_prefill_varlen_workspace_bytes(int nseq, int total_tokens, int nheads, int headdim,
+                                          int ngroups, int dstate, int chunk_len, ssd_dtype_t dtype);
+ssd_status_t ssd_prefill_varlen(const void* x, const float* dt, const float* A, const void* B,
+                                const void* C, const float* D, const float* init_states,
+                                const int* cu_seqlens, int nseq, int total_tokens, int nheads,
+                                int headdim, int ngroups, int dstate, int chunk_len, ssd_dtype_t dtype,
+                                void* y, float* final_states, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/*
  * One layer's tensors for ssd_decode_step_layers: the arguments of ssd_decode_step for
  * that layer (device pointers, layouts as there; every pointer 16-byte aligned).
  */

@@ -10,8 +10,8 @@ missing.
 """
 from .binding import (SSDError, decode_layer_table, ssd_decode_step,  # noqa: F401
                       ssd_decode_step_layers, ssd_device_status, ssd_gdn_decode_step, ssd_prefill,
-                      ssd_prefill_workspace_bytes)
+                      ssd_prefill_varlen, ssd_prefill_workspace_bytes)
 
 __all__ = ["SSDError", "ssd_prefill", "ssd_decode_step", "ssd_decode_step_layers",
-           "decode_layer_table", "ssd_gdn_decode_step", "ssd_prefill_workspace_bytes",
+           "decode_layer_table", "ssd_gdn_decode_step", "ssd_prefill_varlen", "ssd_prefill_workspace_bytes",
            "ssd_device_status"]

@@ -36,6 +36,8 @@ SIGNATURES = {
     "ssd_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ssd_decode_step_layers": ([_P, _I, _I, _I, _I, _I, _I, _I, _P], _I),
     "ssd_gdn_decode_step": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
+    "ssd_prefill_varlen_workspace_bytes": ([_I, _I, _I, _I, _I, _I, _I, _I], _Z),
+    "ssd_prefill_varlen": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _Z, _P], _I),
     "ssd_prefill_dtraw": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _Z, _P], _I),
     "ssd_decode_step_dtraw": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ssd_prefill_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P], _I),
@@ -150,6 +152,38 @@ def ssd_prefill(x, dt, A, B, C, D, chunk_len, init_state=None, y=None, final_sta
                            _stream(stream))
     _check(st, "ssd_prefill")
     return y, final_state
+
+
+def ssd_prefill_varlen(x, dt, A, B, C, D, cu_seqlens, chunk_len, init_states=None, y=None,
+                       final_states=None, workspace=None, stream=None):
+    """Packed variable-length prefill.  x [T][H][P], dt [T][H], B/C [T][G][N] (the batch-1
+    layouts without the batch axis), cu_seqlens a CUDA int32 tensor of nseq + 1 offsets.
+    Returns ``(y, final_states)``, final_states [nseq][H][P][N]."""
+    for t, n in ((x, "x"), (B, "B"), (C, "C")):
+        _need(t, n, x.dtype)
+    for t, n in ((dt, "dt"), (A, "A"), (D, "D")):
+        _need(t, n, torch.float32)
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    code = _dtype_code(x)
+    total, nheads, headdim = x.shape
+    ngroups, dstate = B.shape[1], B.shape[2]
+    nseq = cu_seqlens.numel() - 1
+    if y is None:
+        y = torch.empty_like(x)
+    if final_states is None:
+        final_states = torch.empty((nseq, nheads, headdim, dstate), device=x.device, dtype=torch.float32)
+    if init_states is not None:
+        _need(init_states, "init_states", torch.float32)
+    need = int(lib().ssd_prefill_varlen_workspace_bytes(nseq, total, nheads, headdim, ngroups, dstate,
+                                                        chunk_len, code))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=x.device, dtype=torch.uint8)
+    st = lib().ssd_prefill_varlen(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_states),
+                                  _ptr(cu_seqlens), nseq, total, nheads, headdim, ngroups, dstate, chunk_len,
+                                  code, _ptr(y), _ptr(final_states), _ptr(workspace), workspace.numel(),
+                                  _stream(stream))
+    _check(st, "ssd_prefill_varlen")
+    return y, final_states
 
 
 def ssd_decode_step(state, x_t, dt_t, A, B_t, C_t, D, y_t=None, stream=None, dt_softplus=False,

@@ -226,6 +226,75 @@ ssd_status_t prefill_impl(const void* x, const float* dt, const float* dt_bias, 
 
 }  // namespace
 
+namespace {
+
+ssd_status_t varlen_dims(int nseq, int total_tokens, int nheads, int headdim, int ngroups, int dstate,
+                         int chunk_len, ssd_dtype_t dtype, Dims* t)
+{
+    ssd_status_t st = check_common(1, nheads, headdim, ngroups, dstate, dtype, 256);
+    if (st != SSD_OK) return st;
+    if (nseq < 1 || nseq > (1 << 20) || total_tokens < 0 || chunk_len < 1) return SSD_ERR_SHAPE;
+    Dims d{1, total_tokens, nheads, headdim, ngroups, dstate, chunk_len, 1};
+    if (dtype != SSD_BF16 || !tc_prefill_supported(d)) return SSD_ERR_UNSUPPORTED;
+    *t = tc_varlen_dims(nseq, total_tokens, nheads, headdim, ngroups, dstate);
+    return SSD_OK;
+}
+
+}  // namespace
+
+size_t ssd_prefill_varlen_workspace_bytes(int nseq, int total_tokens, int nheads, int headdim,
+                                          int ngroups, int dstate, int chunk_len, ssd_dtype_t dtype)
+{
+    Dims t;
+    if (varlen_dims(nseq, total_tokens, nheads, headdim, ngroups, dstate, chunk_len, dtype, &t) != SSD_OK)
+        return 0;
+    if (total_tokens == 0) return 0;
+    return tc_varlen_workspace_layout(t, nullptr, nullptr, nullptr, nullptr);
+}
+
+ssd_status_t ssd_prefill_varlen(const void* x, const float* dt, const float* A, const void* B,
+                                const void* C, const float* D, const float* init_states,
+                                const int* cu_seqlens, int nseq, int total_tokens, int nheads,
+                                int headdim, int ngroups, int dstate, int chunk_len, ssd_dtype_t dtype,
+                                void* y, float* final_states, void* workspace, size_t workspace_bytes,
+                                void* stream)
+{
+    Dims t;
+    ssd_status_t st = varlen_dims(nseq, total_tokens, nheads, headdim, ngroups, dstate, chunk_len, dtype, &t);
+    if (st != SSD_OK) return st;
+    if (!final_states || !cu_seqlens) return SSD_ERR_NULL;
+    if (!aligned16(final_states) || !aligned16(init_states) || reinterpret_cast<uintptr_t>(cu_seqlens) % 4)
+        return SSD_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (total_tokens == 0) {
+        Dims c{nseq, 0, nheads, headdim, ngroups, dstate, chunk_len, 0};
+        return from_cuda(profiled(kCopy, s, [&] { return launch_copy_state(c, init_states, final_states, s); }));
+    }
+    if (!x || !dt || !A || !B || !C || !D || !y) return SSD_ERR_NULL;
+    if (!aligned16(x) || !aligned16(dt) || !aligned16(A) || !aligned16(B) || !aligned16(C) ||
+        !aligned16(D) || !aligned16(y) || !aligned16(workspace))
+        return SSD_ERR_ALIGN;
+    TcWorkspace w;
+    int* first = nullptr;
+    int* seqof = nullptr;
+    const size_t need = tc_varlen_workspace_layout(t, workspace, &w, &first, &seqof);
+    if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
+    t.cu_seqlens = cu_seqlens;
+    t.vl_first = first;
+    t.vl_seq = seqof;
+    cudaError_t e = profiled(kCumsum, s, [&] {
+        cudaError_t r = launch_varlen_table(t, s);
+        return r != cudaSuccess ? r : launch_chunk_cumsum(t, dt, A, w.fac, true, w.wts, B, w.b16, s);
+    });
+    if (e == cudaSuccess)
+        e = profiled(kStateTc, s, [&] {
+            return launch_chunk_state_scan_tc(t, x, w.b16, w, init_states, final_states, s);
+        });
+    if (e == cudaSuccess)
+        e = profiled(kOutTc, s, [&] { return launch_chunk_output_tc(t, x, B, C, D, w, y, s); });
+    return from_cuda(e);
+}
+
 ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const void* B,
                          const void* C, const float* D, const float* init_state, int batch,
                          int seqlen, int nheads, int headdim, int ngroups, int dstate,

@@ -51,7 +51,24 @@ struct Dims {
     // (dt_bias may be null: no bias)
     const float* dt_bias = nullptr;
     int dt_softplus = 0;
+    // Packed variable-length mode (tensor-core path): batch 1, nseq sequences end to end
+    // along seqlen; nchunks is then an upper bound on the blocks of all sequences.
+    int nseq = 0;                   // 0: batched mode
+    const int* cu_seqlens = nullptr;  // device [nseq + 1] token offsets
+    const int* vl_first = nullptr;    // device [nseq + 1] first block of each sequence, then the total
+    const int* vl_seq = nullptr;      // device [nchunks] sequence of each block, -1 past the total
 };
+
+// Rows of block kb in packed variable-length mode: false if kb holds no tokens.
+__device__ __forceinline__ bool varlen_block(const int* cu, const int* first, const int* seqof, int kb,
+                                             int Q, int* seq, int* t0, int* len) {
+    const int s = seqof[kb];
+    if (s < 0) return false;
+    *seq = s;
+    *t0 = cu[s] + (kb - first[s]) * Q;
+    *len = min(Q, cu[s + 1] - *t0);
+    return true;
+}
 
 // The dt a kernel uses for head h from the dt input value `in`.  With dt_softplus the sum
 // in + dt_bias[h] and softplus(z) = log(1 + exp(z)) (z itself above 40) are formed in

@@ -46,19 +46,27 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
                     float* __restrict__ fac, int fac_stride, bool extras, float* __restrict__ wts,
                     const uint4* __restrict__ b_bf16, uint4* __restrict__ b_f16,
                     int b_row_chunks, int seqlen, int nheads, int Q, int nchunks,
-                    const float* __restrict__ dt_bias, int dt_softplus)
+                    const float* __restrict__ dt_bias, int dt_softplus, const int* __restrict__ vl_cu,
+                    const int* __restrict__ vl_first, const int* __restrict__ vl_seq)
 {
     extern __shared__ float sm_dt[];                   // [Q][kCumsumHeads]
     // the next kernel of the stream (launched as a programmatic dependent) may stage its setup
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int c = blockIdx.x, h0 = blockIdx.y * kCumsumHeads, b = blockIdx.z;
     const int nh = min(kCumsumHeads, nheads - h0);
-    const int t0 = c * Q;
+    // rows t0 .. t0 + valid - 1 of batch b are this chunk's tokens; in packed variable-length
+    // mode (batch 1) chunk c is a block of one sequence, and rows past its end (the next
+    // sequence's) count as padding: dt = 0
+    int t0 = c * Q, valid = min(Q, seqlen - c * Q);
+    if (vl_seq) {
+        int sq;
+        if (!varlen_block(vl_cu, vl_first, vl_seq, c, Q, &sq, &t0, &valid)) return;
+    }
     // dt rows first, so that their loads and those of the B copy below are in flight together
     for (int i = threadIdx.x; i < Q * kCumsumHeads; i += blockDim.x) {
         const int t = i / kCumsumHeads, hh = i - t * kCumsumHeads;
         float v = 0.f;
-        if (hh < nh && t0 + t < seqlen)
+        if (hh < nh && t < valid)
             v = dt_value(dt[((size_t)b * seqlen + t0 + t) * nheads + h0 + hh], dt_bias, dt_softplus, h0 + hh);
         sm_dt[i] = v;
     }
@@ -66,10 +74,10 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
         // fp16 copy of this chunk's rows of B (bf16 -> fp16 is exact for these values'
         // range), the operand format of the tensor-core chunk-state GEMM; the head blocks
         // of a chunk split its rows between them
-        const int rows = min(Q, seqlen - c * Q);
+        const int rows = valid;
         const int r0 = (int)(((long long)rows * blockIdx.y) / gridDim.y);
         const int r1 = (int)(((long long)rows * (blockIdx.y + 1)) / gridDim.y);
-        const size_t first = ((size_t)b * seqlen + (size_t)c * Q + r0) * b_row_chunks;
+        const size_t first = ((size_t)b * seqlen + (size_t)t0 + r0) * b_row_chunks;
         const int n = (r1 - r0) * b_row_chunks;
         constexpr int kUnroll = 4;
         for (int i0 = threadIdx.x; i0 < n; i0 += kUnroll * blockDim.x) {
@@ -445,7 +453,8 @@ cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, 
     chunk_cumsum_kernel<<<grid, kThreads, smem, s>>>(
         dt, A, fac, extras ? 4 * d.chunk_len : d.chunk_len, extras, wts,
         static_cast<const uint4*>(b_bf16), static_cast<uint4*>(b_f16),
-        d.ngroups * d.dstate / 8, d.seqlen, d.nheads, d.chunk_len, d.nchunks, d.dt_bias, d.dt_softplus);
+        d.ngroups * d.dstate / 8, d.seqlen, d.nheads, d.chunk_len, d.nchunks, d.dt_bias, d.dt_softplus,
+        d.cu_seqlens, d.vl_first, d.vl_seq);
     return cudaGetLastError();
 }
 

@@ -44,10 +44,62 @@ namespace {
 
 constexpr int kBox = 16384;                    // one TMA box: 128 rows x 128 bytes
 constexpr int kHImage = 16384;                 // bf16 H_c image: 2 x 64 rows x 128 B
+constexpr int kBlk = 128;                       // tokens per block of the tensor-core path
 constexpr int kP = 64, kN = 128;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// ================================================================ packed variable-length table
+// From cu_seqlens (nseq + 1 token offsets): the first 128-token block of every sequence
+// (the exclusive prefix sum of ceil(len / 128)), then the total, and the sequence of every
+// block (-1 past the total).  Offsets that do not start at 0, decrease, or do not end at
+// total_tokens record SSD_ERR_SHAPE and leave every block empty (no kernel then does work).
+constexpr int kTableThreads = 1024;
+
+__global__ void __launch_bounds__(kTableThreads)
+varlen_table_kernel(const int* __restrict__ cu, int nseq, int total_tokens, int max_blocks,
+                    int* __restrict__ first, int* __restrict__ seqof, int* err)
+{
+    __shared__ int part[kTableThreads];
+    __shared__ int bad;
+    const int tid = threadIdx.x;
+    if (tid == 0) bad = (cu[0] != 0 || cu[nseq] != total_tokens) ? 1 : 0;
+    __syncthreads();
+    const int per = (nseq + kTableThreads - 1) / kTableThreads;
+    const int s0 = min(nseq, tid * per), s1 = min(nseq, s0 + per);
+    int sum = 0, neg = 0;
+    for (int s = s0; s < s1; ++s) {
+        const int len = cu[s + 1] - cu[s];
+        neg |= len < 0;
+        sum += (max(len, 0) + kBlk - 1) / kBlk;
+    }
+    if (neg) atomicOr(&bad, 1);
+    part[tid] = sum;
+    __syncthreads();
+    for (int o = 1; o < kTableThreads; o <<= 1) {      // inclusive scan of the partial counts
+        const int v = tid >= o ? part[tid - o] : 0;
+        __syncthreads();
+        part[tid] += v;
+        __syncthreads();
+    }
+    const int total = part[kTableThreads - 1];
+    if (bad || total > max_blocks) {
+        if (tid == 0) record_error(err, SSD_ERR_SHAPE);
+        for (int i = tid; i < max_blocks; i += kTableThreads) seqof[i] = -1;
+        for (int i = tid; i <= nseq; i += kTableThreads) first[i] = 0;
+        return;
+    }
+    int base = tid ? part[tid - 1] : 0;
+    for (int s = s0; s < s1; ++s) {
+        first[s] = base;
+        const int nb = (cu[s + 1] - cu[s] + kBlk - 1) / kBlk;
+        for (int k = 0; k < nb; ++k) seqof[base + k] = s;
+        base += nb;
+    }
+    if (tid == 0) first[nseq] = total;
+    for (int i = total + tid; i < max_blocks; i += kTableThreads) seqof[i] = -1;
 }
 
 // ================================================================ chunk states: persistent walk
@@ -99,7 +151,8 @@ __global__ void __launch_bounds__(kWalkThreads, WalkCfg<NH>::kCtasPerSm)
 chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __restrict__ fac,
                         const float* __restrict__ init_state, float* final_state,
                         uint8_t* __restrict__ himg, int nheads, int ngroups, int nchunks,
-                        int ctas_per_group, int* err)
+                        int ctas_per_group, int* err, const int* __restrict__ vl_cu,
+                        const int* __restrict__ vl_first)
 {
     using L = WalkCfg<NH>;
     constexpr int NQ = Q / 64;                          // stages per chunk
@@ -119,7 +172,19 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
     const int hlo = g * hpg + (part * hpg) / ctas_per_group;
     const int nh = g * hpg + ((part + 1) * hpg) / ctas_per_group - hlo;     // 1..3
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int total = nchunks * NQ;
+    // the chain's blocks: batched, chunks 0 .. nchunks - 1 of batch b; packed variable-length
+    // (b is then the sequence), the sequence's blocks blk0 .. blk0 + nblk - 1, whose rows
+    // start at row0 of the single batch
+    int row0 = 0, blk0 = 0, nblk = nchunks, bt = b;
+    if (vl_first) {
+        griddep_wait();                                  // the block table comes from an earlier kernel
+        row0 = vl_cu[b];
+        blk0 = vl_first[b];
+        nblk = vl_first[b + 1] - blk0;
+        bt = 0;
+    }
+    const int sb = vl_first ? 0 : b;                     // batch index of the per-block arrays
+    const int total = nblk * NQ;
     auto stage = [&](int st) { return sm + st * L::kStageBytes; };
 
     if (tid == 0) {
@@ -150,18 +215,18 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
             for (int k = 0; k < total; ++k) {
                 const int st = k % S;
                 if (k >= S && !mbar_wait(&empty[st], ((k / S) + 1) & 1, err)) break;
-                const int c = k / NQ, qq = k - c * NQ, row = c * Q + qq * 64;
+                const int c = k / NQ, qq = k - c * NQ, row = row0 + c * Q + qq * 64;
                 uint8_t* sg = stage(st);
                 mbar_expect_tx(&full[st], (2 + nh) * kQBox + NH * kWRow * 4);
-                tma_load_4d(sg, &maps.b, 0, row, 2 * g, b, &full[st]);
+                tma_load_4d(sg, &maps.b, 0, row, 2 * g, bt, &full[st]);
                 int hh = 0;
                 if (NH > 1 && nh >= 2) {
-                    tma_load_4d(sg + L::kStageX + hh * kQBox, &maps.x2, 0, row, hlo + hh, b, &full[st]);
+                    tma_load_4d(sg + L::kStageX + hh * kQBox, &maps.x2, 0, row, hlo + hh, bt, &full[st]);
                     hh += 2;
                 }
                 if (nh - hh >= 1)
-                    tma_load_4d(sg + L::kStageX + hh * kQBox, &maps.x1, 0, row, hlo + hh, b, &full[st]);
-                tma_load_2d(sg + L::kStageW, &maps.w, c * (Q + 4) + qq * 64, b * nheads + hlo, &full[st]);
+                    tma_load_4d(sg + L::kStageX + hh * kQBox, &maps.x1, 0, row, hlo + hh, bt, &full[st]);
+                tma_load_2d(sg + L::kStageW, &maps.w, (blk0 + c) * (Q + 4) + qq * 64, sb * nheads + hlo, &full[st]);
                 issued = k + 1;
             }
             // the CTA does not exit with loads in flight
@@ -232,7 +297,7 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
             __syncwarp();
             if (lane == 0) {
                 for (int hh = 0; hh < nh; ++hh)
-                    bulk_store(himg + ((size_t)(b * nheads + hlo + hh) * nchunks + cc) * kHImage + piece,
+                    bulk_store(himg + ((size_t)(sb * nheads + hlo + hh) * nchunks + blk0 + cc) * kHImage + piece,
                                sm + L::kImg + hh * kHImage + piece, 2048);
                 bulk_commit_group();
             }
@@ -255,10 +320,10 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
                 }
             }
             tc_fence_before();
-            if (cc + 1 < nchunks) write_images(cc + 1);
+            if (cc + 1 < nblk) write_images(cc + 1);
         };
 
-        write_images(0);
+        if (nblk > 0) write_images(0);
         float e_prev[NH];                                // decay of the chunk before the current one
 #pragma unroll
         for (int hh = 0; hh < NH; ++hh) e_prev[hh] = 0.f;
@@ -317,7 +382,7 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
                 for (int hh = 0; hh < NH; ++hh) e_prev[hh] = e_cur[hh];
             }
         }
-        if (nchunks > 0) update(nchunks - 1, e_prev);
+        if (nblk > 0) update(nblk - 1, e_prev);
         if (lane == 0) bulk_wait_group0();
 #pragma unroll
         for (int hh = 0; hh < NH; ++hh) {
@@ -359,7 +424,6 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
 // the sub-block's last column (both <= 1); sub-blocks on the diagonal use the first column
 // as reference when their own decay is below 40 (both factors within e^+-40) and fall
 // back to one exponential per element otherwise.
-constexpr int kBlk = 128;                                // tokens per output block
 constexpr int kOutThreads = 512;
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpP0 = 4, kWarpE0 = 12;
 constexpr int kPThreads = 256, kEThreads = 128;
@@ -398,7 +462,9 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
                     const float* __restrict__ fac,
                     const uint8_t* __restrict__ himg, const float* __restrict__ D, int nheads,
-                    int ngroups, int nblocks, int heads_per_cta, int* err)
+                    int ngroups, int nblocks, int heads_per_cta, int* err, __nv_bfloat16* __restrict__ y,
+                    const int* __restrict__ vl_cu, const int* __restrict__ vl_first,
+                    const int* __restrict__ vl_seq)
 {
     using L = OutSmem;
     extern __shared__ uint8_t smem_raw[];
@@ -408,10 +474,18 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::kSlotTm);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kAbort);
 
-    const int k = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
+    // block k: rows t0 .. t0 + 127 of batch b; in packed variable-length mode (batch 1) block k
+    // of the table, rows t0 .. t0 + len - 1 of its sequence (the rest belong to the next one:
+    // their dt is 0, and their y rows are not stored)
+    const int k = blockIdx.x, hg = blockIdx.y;
+    int b = blockIdx.z, t0 = k * kBlk, len = kBlk;
+    if (vl_seq) {
+        int sq;
+        if (!varlen_block(vl_cu, vl_first, vl_seq, k, kBlk, &sq, &t0, &len)) return;
+        b = 0;
+    }
     const int h0 = hg * heads_per_cta;
     const int g = h0 / (nheads / ngroups);
-    const int t0 = k * kBlk;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
@@ -652,7 +726,11 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                         const float a1 = fmaf(u, __uint_as_float(yo[jj + 1]), __uint_as_float(yd[jj + 1])) + Dh * bf16hi(xw[k2]);
                         o[k2] = pack_bf16x2(a0, a1);
                     }
-                    *xp = make_uint4(o[0], o[1], o[2], o[3]);
+                    if (len == kBlk)
+                        *xp = make_uint4(o[0], o[1], o[2], o[3]);
+                    else if (r < len)                       // partial block: the row goes out directly
+                        *reinterpret_cast<uint4*>(y + ((size_t)(t0 + r) * nheads + h) * kP + qx * 8) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
                 }
             }
             tc_fence_before();
@@ -660,9 +738,11 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             fence_proxy_async_smem();                       // y rows -> visible to the TMA unit
             named_bar_sync(2, kEThreads);
             if (etid == 0) {
-                tma_store_3d(&tm_y, h * kP, t0, b, sl + L::kXo);
-                bulk_commit_group();
-                bulk_wait_group_read0();                    // the slot may be refilled now
+                if (len == kBlk) {
+                    tma_store_3d(&tm_y, h * kP, t0, b, sl + L::kXo);
+                    bulk_commit_group();
+                    bulk_wait_group_read0();                // the slot may be refilled now
+                }
                 mbar_arrive(&bars[BAR_XEMPTY + s]);
             }
         }
@@ -782,9 +862,12 @@ int sm_count()
 
 // Walk shape: one head per CTA (two CTAs per SM) when every (b, h) chain fits in the
 // SMs that way, else up to three heads per CTA.
+// (b, h) chains of the walk: batch x heads, or sequences x heads in packed variable-length mode
+long long walk_chains(const Dims& d) { return (long long)(d.nseq ? d.nseq : d.batch) * d.nheads; }
+
 int walk_heads(const Dims& d)
 {
-    return (long long)d.batch * d.nheads <= (long long)WalkCfg<1>::kCtasPerSm * sm_count() ? 1 : 3;
+    return walk_chains(d) <= (long long)WalkCfg<1>::kCtasPerSm * sm_count() ? 1 : 3;
 }
 
 // CTAs per (b, g) of the walk: enough that each holds at most nh heads, and as many as
@@ -792,7 +875,7 @@ int walk_heads(const Dims& d)
 int walk_ctas_per_group(const Dims& d, int nh)
 {
     const int hpg = d.nheads / d.ngroups;
-    const int units = d.batch * d.ngroups;
+    const int units = (d.nseq ? d.nseq : d.batch) * d.ngroups;
     int cpg = (hpg + nh - 1) / nh;
     cpg = max(cpg, sm_count() / units);
     return min(cpg, hpg);
@@ -807,15 +890,15 @@ cudaError_t walk_t(const Dims& d, const WalkMaps& maps, const TcWorkspace& w, co
                                          WalkCfg<NH>::kBytes);
     if (e != cudaSuccess) return e;
     const int cpg = walk_ctas_per_group(d, NH);
-    const unsigned grid = (unsigned)(d.batch * d.ngroups * cpg);
+    const unsigned grid = (unsigned)((d.nseq ? d.nseq : d.batch) * d.ngroups * cpg);
     return launch_dependent(k, dim3(grid), dim3(kWalkThreads), WalkCfg<NH>::kBytes, s, maps, w.fac,
                             init_state, final_state, w.himg, d.nheads, d.ngroups, d.nchunks, cpg,
-                            device_error_word());
+                            device_error_word(), d.cu_seqlens, d.vl_first);
 }
 
 cudaError_t output_launch(const Dims& d, const CUtensorMap& mx, const CUtensorMap& mb,
                           const CUtensorMap& mc, const CUtensorMap& my, const TcWorkspace& w,
-                          const float* D, cudaStream_t s)
+                          const float* D, void* y, cudaStream_t s)
 {
     auto k = block_output_kernel;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, OutSmem::kBytes);
@@ -823,7 +906,8 @@ cudaError_t output_launch(const Dims& d, const CUtensorMap& mx, const CUtensorMa
     const int hpc = heads_per_cta(d);
     dim3 grid(d.nchunks, d.nheads / hpc, d.batch);
     return launch_dependent(k, grid, dim3(kOutThreads), OutSmem::kBytes, s, mx, mb, mc, my, w.fac,
-                            w.himg, D, d.nheads, d.ngroups, d.nchunks, hpc, device_error_word());
+                            w.himg, D, d.nheads, d.ngroups, d.nchunks, hpc, device_error_word(),
+                            static_cast<__nv_bfloat16*>(y), d.cu_seqlens, d.vl_first, d.vl_seq);
 }
 
 }  // namespace
@@ -857,6 +941,32 @@ size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w)
         w->b16 = p + fac_b + wts_b + himg_b;
     }
     return fac_b + wts_b + himg_b + b16_b;
+}
+
+Dims tc_varlen_dims(int nseq, int total_tokens, int nheads, int headdim, int ngroups, int dstate)
+{
+    Dims t{1, total_tokens, nheads, headdim, ngroups, dstate, kBlk, total_tokens / kBlk + nseq};
+    t.nseq = nseq;
+    return t;
+}
+
+size_t tc_varlen_workspace_layout(const Dims& t, void* base, TcWorkspace* w, int** first, int** seqof)
+{
+    auto up = [](size_t v) { return (v + 255) & ~size_t(255); };
+    const size_t main = tc_workspace_layout(t, base, w);
+    const size_t first_b = up((size_t)(t.nseq + 1) * sizeof(int));
+    const size_t seq_b = up((size_t)t.nchunks * sizeof(int));
+    if (first) *first = reinterpret_cast<int*>(static_cast<char*>(base) + main);
+    if (seqof) *seqof = reinterpret_cast<int*>(static_cast<char*>(base) + main + first_b);
+    return main + first_b + seq_b;
+}
+
+cudaError_t launch_varlen_table(const Dims& t, cudaStream_t s)
+{
+    varlen_table_kernel<<<1, kTableThreads, 0, s>>>(t.cu_seqlens, t.nseq, t.seqlen, t.nchunks,
+                                                    const_cast<int*>(t.vl_first), const_cast<int*>(t.vl_seq),
+                                                    device_error_word());
+    return cudaGetLastError();
 }
 
 cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void* B_f16,
@@ -901,7 +1011,7 @@ cudaError_t launch_chunk_output_tc(const Dims& d, const void* x, const void* B, 
         !make_map(&mc, C, (uint64_t)d.ngroups * kN, d.seqlen, d.batch) ||
         !make_map(&my, y, (uint64_t)d.nheads * kP, d.seqlen, d.batch))
         return cudaErrorInvalidValue;
-    return output_launch(d, mx, mb, mc, my, w, D, s);
+    return output_launch(d, mx, mb, mc, my, w, D, y, s);
 }
 
 }  // namespace ssd

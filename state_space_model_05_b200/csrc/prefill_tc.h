@@ -26,6 +26,12 @@ struct TcWorkspace {
 };
 size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w);
 
+// Packed variable-length prefill: the block dims (batch 1, an upper bound of blocks), the
+// workspace (the tensor-core workspace, then the block table), and the table kernel.
+Dims tc_varlen_dims(int nseq, int total_tokens, int nheads, int headdim, int ngroups, int dstate);
+size_t tc_varlen_workspace_layout(const Dims& t, void* base, TcWorkspace* w, int** first, int** seqof);
+cudaError_t launch_varlen_table(const Dims& t, cudaStream_t s);
+
 // Chunk states and the inter-chunk recurrence (persistent walk over each head's chunks),
 // writing the chunk start states (bf16 images) and the final state.  B_f16 is the fp16
 // copy of B.

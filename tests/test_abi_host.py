@@ -154,6 +154,29 @@ def test_dtraw_validation(lib):
     assert p(*args) == 2                                   # bad seqlen
 
 
+def test_varlen_validation(lib):
+    F = FAKE
+    ws = lib.ssd_prefill_varlen_workspace_bytes
+    up = lambda v: (v + 255) // 256 * 256
+    nseq, T, H = 3, 1000, 4
+    nb = T // 128 + nseq                             # block bound: floor(T / 128) + nseq
+    main = (up(H * nb * 4 * 128 * 4) + up(H * nb * 132 * 4) + up(H * nb * 16384) + up(T * 128 * 2))
+    assert ws(nseq, T, H, 64, 1, 128, 256, binding.SSD_BF16) == main + up((nseq + 1) * 4) + up(nb * 4)
+    assert ws(nseq, 0, H, 64, 1, 128, 256, binding.SSD_BF16) == 0
+    assert ws(nseq, T, H, 64, 1, 128, 256, binding.SSD_F32) == 0          # tensor-core path only
+    f = lib.ssd_prefill_varlen
+    args = lambda **kw: [F, F, F, F, F, F, None, kw.get("cu", F), kw.get("nseq", 3), kw.get("T", 1000), 4,
+                         kw.get("P", 64), 1, 128, kw.get("Q", 256), kw.get("dtype", binding.SSD_BF16), F, F, F,
+                         1 << 30, None]
+    assert f(*args(dtype=binding.SSD_F32)) == 5
+    assert f(*args(P=32)) == 5
+    assert f(*args(Q=64)) == 5
+    assert f(*args(nseq=0)) == 2
+    assert f(*args(T=-1)) == 2
+    assert f(*args(cu=None)) == 1
+    assert f(*args(cu=F + 2)) == 4
+
+
 def test_gdn_validation(lib):
     f = lib.ssd_gdn_decode_step
     F = FAKE
