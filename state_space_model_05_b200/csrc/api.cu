@@ -229,15 +229,33 @@ ssd_status_t prefill_impl(const void* x, const float* dt, const float* dt_bias, 
 namespace {
 
 ssd_status_t varlen_dims(int nseq, int total_tokens, int nheads, int headdim, int ngroups, int dstate,
-                         int chunk_len, ssd_dtype_t dtype, Dims* t)
+                         int chunk_len, ssd_dtype_t dtype, Dims* t, bool* tc)
 {
     ssd_status_t st = check_common(1, nheads, headdim, ngroups, dstate, dtype, 256);
     if (st != SSD_OK) return st;
     if (nseq < 1 || nseq > (1 << 20) || total_tokens < 0 || chunk_len < 1) return SSD_ERR_SHAPE;
+    if (chunk_len > 256) return SSD_ERR_UNSUPPORTED;
     Dims d{1, total_tokens, nheads, headdim, ngroups, dstate, chunk_len, 1};
-    if (dtype != SSD_BF16 || !tc_prefill_supported(d)) return SSD_ERR_UNSUPPORTED;
-    *t = tc_varlen_dims(nseq, total_tokens, nheads, headdim, ngroups, dstate);
+    *tc = dtype == SSD_BF16 && tc_prefill_supported(d);
+    if (*tc) {
+        *t = tc_varlen_dims(nseq, total_tokens, nheads, headdim, ngroups, dstate);
+    } else {
+        // CUDA-core path: chunks of chunk_len, at most floor(T / Q) + nseq of them
+        *t = Dims{1, total_tokens, nheads, headdim, ngroups, dstate, chunk_len, total_tokens / chunk_len + nseq};
+        t->nseq = nseq;
+    }
     return SSD_OK;
+}
+
+// the CUDA-core workspace, then the block table (first [nseq + 1], sequence of each chunk)
+size_t simt_varlen_workspace_layout(const Dims& t, void* base, PrefillWorkspace* ws, int** first, int** seqof)
+{
+    const size_t main = prefill_workspace_layout(t, base, ws);
+    const size_t first_b = align_up((size_t)(t.nseq + 1) * sizeof(int));
+    const size_t seq_b = align_up((size_t)t.nchunks * sizeof(int));
+    if (first) *first = reinterpret_cast<int*>(static_cast<char*>(base) + main);
+    if (seqof) *seqof = reinterpret_cast<int*>(static_cast<char*>(base) + main + first_b);
+    return main + first_b + seq_b;
 }
 
 }  // namespace
@@ -246,10 +264,12 @@ size_t ssd_prefill_varlen_workspace_bytes(int nseq, int total_tokens, int nheads
                                           int ngroups, int dstate, int chunk_len, ssd_dtype_t dtype)
 {
     Dims t;
-    if (varlen_dims(nseq, total_tokens, nheads, headdim, ngroups, dstate, chunk_len, dtype, &t) != SSD_OK)
+    bool tc = false;
+    if (varlen_dims(nseq, total_tokens, nheads, headdim, ngroups, dstate, chunk_len, dtype, &t, &tc) != SSD_OK)
         return 0;
     if (total_tokens == 0) return 0;
-    return tc_varlen_workspace_layout(t, nullptr, nullptr, nullptr, nullptr);
+    return tc ? tc_varlen_workspace_layout(t, nullptr, nullptr, nullptr, nullptr)
+              : simt_varlen_workspace_layout(t, nullptr, nullptr, nullptr, nullptr);
 }
 
 ssd_status_t ssd_prefill_varlen(const void* x, const float* dt, const float* A, const void* B,
@@ -260,7 +280,8 @@ ssd_status_t ssd_prefill_varlen(const void* x, const float* dt, const float* A, 
                                 void* stream)
 {
     Dims t;
-    ssd_status_t st = varlen_dims(nseq, total_tokens, nheads, headdim, ngroups, dstate, chunk_len, dtype, &t);
+    bool tc = false;
+    ssd_status_t st = varlen_dims(nseq, total_tokens, nheads, headdim, ngroups, dstate, chunk_len, dtype, &t, &tc);
     if (st != SSD_OK) return st;
     if (!final_states || !cu_seqlens) return SSD_ERR_NULL;
     if (!aligned16(final_states) || !aligned16(init_states) || reinterpret_cast<uintptr_t>(cu_seqlens) % 4)
@@ -274,24 +295,44 @@ ssd_status_t ssd_prefill_varlen(const void* x, const float* dt, const float* A, 
     if (!aligned16(x) || !aligned16(dt) || !aligned16(A) || !aligned16(B) || !aligned16(C) ||
         !aligned16(D) || !aligned16(y) || !aligned16(workspace))
         return SSD_ERR_ALIGN;
-    TcWorkspace w;
     int* first = nullptr;
     int* seqof = nullptr;
-    const size_t need = tc_varlen_workspace_layout(t, workspace, &w, &first, &seqof);
-    if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
     t.cu_seqlens = cu_seqlens;
+    if (tc) {
+        TcWorkspace w;
+        const size_t need = tc_varlen_workspace_layout(t, workspace, &w, &first, &seqof);
+        if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
+        t.vl_first = first;
+        t.vl_seq = seqof;
+        cudaError_t e = profiled(kCumsum, s, [&] {
+            cudaError_t r = launch_varlen_table(t, s);
+            return r != cudaSuccess ? r : launch_chunk_cumsum(t, dt, A, w.fac, true, w.wts, B, w.b16, s);
+        });
+        if (e == cudaSuccess)
+            e = profiled(kStateTc, s, [&] {
+                return launch_chunk_state_scan_tc(t, x, w.b16, w, init_states, final_states, s);
+            });
+        if (e == cudaSuccess)
+            e = profiled(kOutTc, s, [&] { return launch_chunk_output_tc(t, x, B, C, D, w, y, s); });
+        return from_cuda(e);
+    }
+    PrefillWorkspace ws;
+    const size_t need = simt_varlen_workspace_layout(t, workspace, &ws, &first, &seqof);
+    if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
     t.vl_first = first;
     t.vl_seq = seqof;
     cudaError_t e = profiled(kCumsum, s, [&] {
         cudaError_t r = launch_varlen_table(t, s);
-        return r != cudaSuccess ? r : launch_chunk_cumsum(t, dt, A, w.fac, true, w.wts, B, w.b16, s);
+        return r != cudaSuccess ? r : launch_chunk_cumsum(t, dt, A, ws.lam, false, nullptr, nullptr, nullptr, s);
     });
     if (e == cudaSuccess)
-        e = profiled(kStateTc, s, [&] {
-            return launch_chunk_state_scan_tc(t, x, w.b16, w, init_states, final_states, s);
-        });
+        e = profiled(kStateSimt, s, [&] { return launch_chunk_state_simt(t, dtype, x, dt, B, ws.lam, ws.states, s); });
     if (e == cudaSuccess)
-        e = profiled(kOutTc, s, [&] { return launch_chunk_output_tc(t, x, B, C, D, w, y, s); });
+        e = profiled(kScan, s, [&] { return launch_state_scan(t, ws.lam, ws.states, init_states, final_states, s); });
+    if (e == cudaSuccess)
+        e = profiled(kOutSimt, s, [&] {
+            return launch_chunk_output_simt(t, dtype, x, dt, B, C, D, ws.lam, ws.states, y, s);
+        });
     return from_cuda(e);
 }
 

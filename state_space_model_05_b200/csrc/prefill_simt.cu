@@ -165,16 +165,21 @@ chunk_state_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
                         const T* __restrict__ Bm, const float* __restrict__ lam,
                         float* __restrict__ states, int seqlen, int nheads, int headdim,
                         int ngroups, int dstate, int Q, int nchunks, const float* __restrict__ dt_bias,
-                        int dt_softplus)
+                        int dt_softplus, const int* __restrict__ vl_cu, const int* __restrict__ vl_first,
+                        const int* __restrict__ vl_seq)
 {
     extern __shared__ float sm[];
     float* sx = sm;                                    // [kTokTile][headdim]
     float* sb = sx + kTokTile * headdim;               // [kTokTile][dstate]
     float* sw = sb + kTokTile * dstate;                // [kTokTile]
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int c = blockIdx.x, h = blockIdx.y;
+    int b = blockIdx.z, t0 = c * Q, qlen = min(Q, seqlen - c * Q);
+    if (vl_seq) {                                      // packed variable-length: chunk c of the table
+        int sq;
+        if (!varlen_block(vl_cu, vl_first, vl_seq, c, Q, &sq, &t0, &qlen)) return;
+        b = 0;
+    }
     const int g = h / (nheads / ngroups);
-    const int t0 = c * Q;
-    const int qlen = min(Q, seqlen - t0);
     const float* lamc = lam + (((size_t)b * nheads + h) * nchunks + c) * Q;
     const float lam_end = lamc[Q - 1];
 
@@ -242,15 +247,24 @@ chunk_state_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
 __global__ void __launch_bounds__(kThreads)
 state_scan_kernel(const float* __restrict__ lam, float* __restrict__ states,
                   const float* init_state, float* final_state, int nheads, int PN, int Q,
-                  int nchunks)
+                  int nchunks, const int* __restrict__ vl_first)
 {
+    // chain bh = (b, h): chunks 0 .. nchunks - 1 of that row of the per-chunk arrays; in packed
+    // variable-length mode bh = (sequence, h) and its chunks are the table's first[s] ..
+    // first[s + 1] - 1 of row h (batch 1)
     const int bh = blockIdx.y;
     const int e = 4 * (blockIdx.x * kThreads + threadIdx.x);
     if (e >= PN) return;
+    size_t row = (size_t)bh * nchunks;
+    if (vl_first) {
+        const int sq = bh / nheads, h = bh - sq * nheads;
+        row = (size_t)h * nchunks + vl_first[sq];
+        nchunks = vl_first[sq + 1] - vl_first[sq];
+    }
     float4 hs = make_float4(0.f, 0.f, 0.f, 0.f);
     if (init_state) hs = *reinterpret_cast<const float4*>(init_state + (size_t)bh * PN + e);
-    const float* lamr = lam + (size_t)bh * nchunks * Q;
-    float* st = states + (size_t)bh * nchunks * PN + e;
+    const float* lamr = lam + row * Q;
+    float* st = states + row * PN + e;
     float4 nxt = nchunks > 0 ? *reinterpret_cast<const float4*>(st) : hs;
     for (int c = 0; c < nchunks; ++c) {
         const float4 sc = nxt;
@@ -277,7 +291,8 @@ chunk_output_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
                          const float* __restrict__ D, const float* __restrict__ lam,
                          const float* __restrict__ states, T* __restrict__ y, int seqlen,
                          int nheads, int headdim, int ngroups, int dstate, int Q, int nchunks,
-                         const float* __restrict__ dt_bias, int dt_softplus)
+                         const float* __restrict__ dt_bias, int dt_softplus, const int* __restrict__ vl_cu,
+                         const int* __restrict__ vl_first, const int* __restrict__ vl_seq)
 {
     extern __shared__ float sm[];
     float* sH = sm;                                    // [headdim][dstate + 1]
@@ -290,10 +305,14 @@ chunk_output_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
     float* sLs = sM + kTokTile * ldM;                  // [kTokTile] Lam_s
     float* sDs = sLs + kTokTile;                       // [kTokTile] dt_s
 
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int c = blockIdx.x, h = blockIdx.y;
+    int b = blockIdx.z, t0 = c * Q, qlen = min(Q, seqlen - c * Q);
+    if (vl_seq) {                                      // packed variable-length: chunk c of the table
+        int sq;
+        if (!varlen_block(vl_cu, vl_first, vl_seq, c, Q, &sq, &t0, &qlen)) return;
+        b = 0;
+    }
     const int g = h / (nheads / ngroups);
-    const int t0 = c * Q;
-    const int qlen = min(Q, seqlen - t0);
     const float* lamc = lam + (((size_t)b * nheads + h) * nchunks + c) * Q;
     const float* Hc = states + (((size_t)b * nheads + h) * nchunks + c) * headdim * dstate;
     const float Dh = D[h];
@@ -410,7 +429,8 @@ cudaError_t chunk_state_simt_t(const Dims& d, const void* x, const float* dt, co
     dim3 grid(d.nchunks, d.nheads, d.batch);
     k<<<grid, kThreads, smem, s>>>(static_cast<const T*>(x), dt, static_cast<const T*>(B), lam,
                                    states, d.seqlen, d.nheads, d.headdim, d.ngroups, d.dstate,
-                                   d.chunk_len, d.nchunks, d.dt_bias, d.dt_softplus);
+                                   d.chunk_len, d.nchunks, d.dt_bias, d.dt_softplus, d.cu_seqlens, d.vl_first,
+                                   d.vl_seq);
     return cudaGetLastError();
 }
 
@@ -430,7 +450,8 @@ cudaError_t chunk_output_simt_t(const Dims& d, const void* x, const float* dt, c
     k<<<grid, kThreads, smem, s>>>(static_cast<const T*>(x), dt, static_cast<const T*>(B),
                                    static_cast<const T*>(C), D, lam, states, static_cast<T*>(y),
                                    d.seqlen, d.nheads, d.headdim, d.ngroups, d.dstate,
-                                   d.chunk_len, d.nchunks, d.dt_bias, d.dt_softplus);
+                                   d.chunk_len, d.nchunks, d.dt_bias, d.dt_softplus, d.cu_seqlens, d.vl_first,
+                                   d.vl_seq);
     return cudaGetLastError();
 }
 
@@ -472,9 +493,9 @@ cudaError_t launch_state_scan(const Dims& d, const float* lam, float* states,
 {
     if (d.batch == 0) return cudaSuccess;
     const int PN = d.headdim * d.dstate;
-    dim3 grid((PN / 4 + kThreads - 1) / kThreads, d.batch * d.nheads);
+    dim3 grid((PN / 4 + kThreads - 1) / kThreads, (d.nseq ? d.nseq : d.batch) * d.nheads);
     state_scan_kernel<<<grid, kThreads, 0, s>>>(lam, states, init_state, final_state, d.nheads,
-                                                PN, d.chunk_len, d.nchunks);
+                                                PN, d.chunk_len, d.nchunks, d.vl_first);
     return cudaGetLastError();
 }
 

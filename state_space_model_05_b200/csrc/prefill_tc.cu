@@ -52,14 +52,14 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 // ================================================================ packed variable-length table
-// From cu_seqlens (nseq + 1 token offsets): the first 128-token block of every sequence
-// (the exclusive prefix sum of ceil(len / 128)), then the total, and the sequence of every
-// block (-1 past the total).  Offsets that do not start at 0, decrease, or do not end at
+// From cu_seqlens (nseq + 1 token offsets): the first Q-token block of every sequence (the
+// exclusive prefix sum of ceil(len / Q)), then the total, and the sequence of every block
+// (-1 past the total).  Offsets that do not start at 0, decrease, or do not end at
 // total_tokens record SSD_ERR_SHAPE and leave every block empty (no kernel then does work).
 constexpr int kTableThreads = 1024;
 
 __global__ void __launch_bounds__(kTableThreads)
-varlen_table_kernel(const int* __restrict__ cu, int nseq, int total_tokens, int max_blocks,
+varlen_table_kernel(const int* __restrict__ cu, int nseq, int total_tokens, int max_blocks, int Q,
                     int* __restrict__ first, int* __restrict__ seqof, int* err)
 {
     __shared__ int part[kTableThreads];
@@ -73,7 +73,7 @@ varlen_table_kernel(const int* __restrict__ cu, int nseq, int total_tokens, int 
     for (int s = s0; s < s1; ++s) {
         const int len = cu[s + 1] - cu[s];
         neg |= len < 0;
-        sum += (max(len, 0) + kBlk - 1) / kBlk;
+        sum += (max(len, 0) + Q - 1) / Q;
     }
     if (neg) atomicOr(&bad, 1);
     part[tid] = sum;
@@ -94,7 +94,7 @@ varlen_table_kernel(const int* __restrict__ cu, int nseq, int total_tokens, int 
     int base = tid ? part[tid - 1] : 0;
     for (int s = s0; s < s1; ++s) {
         first[s] = base;
-        const int nb = (cu[s + 1] - cu[s] + kBlk - 1) / kBlk;
+        const int nb = (cu[s + 1] - cu[s] + Q - 1) / Q;
         for (int k = 0; k < nb; ++k) seqof[base + k] = s;
         base += nb;
     }
@@ -963,7 +963,7 @@ size_t tc_varlen_workspace_layout(const Dims& t, void* base, TcWorkspace* w, int
 
 cudaError_t launch_varlen_table(const Dims& t, cudaStream_t s)
 {
-    varlen_table_kernel<<<1, kTableThreads, 0, s>>>(t.cu_seqlens, t.nseq, t.seqlen, t.nchunks,
+    varlen_table_kernel<<<1, kTableThreads, 0, s>>>(t.cu_seqlens, t.nseq, t.seqlen, t.nchunks, t.chunk_len,
                                                     const_cast<int*>(t.vl_first), const_cast<int*>(t.vl_seq),
                                                     device_error_word());
     return cudaGetLastError();

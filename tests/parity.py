@@ -1,7 +1,7 @@
 """Tolerance checks shared by the GPU parity tests.
 
 fp32 path (max relative error 1e-4):
-  (a) max |g - o| / |o| over elements with |o| >= 1e-2 * RMS(o)  <= 1e-4
+  (a) max |g - o| / |o| over elements with |o| >= 1e-1 * RMS(o)  <= 1e-4
   (b) max |g - o| / RMS(o) over all elements                      <= 1e-4
 bf16-input path (2e-2 normalised to the output RMS):
   y (stored as bf16): max over elements of (|g - o| - h) / RMS(o) <= 2e-2, where h is
@@ -48,7 +48,10 @@ def fp32_errors(g, o):
     if o.size == 0 or r == 0:
         return 0.0, 0.0
     d = np.abs(g - o)
-    big = np.abs(o) >= 1e-2 * r
+    # relative error is taken where it is meaningful: elements at least 1e-1 RMS.  An fp32
+    # sum over T tokens carries ~sqrt(T) 2^-24 RMS of absolute noise (1e-6 RMS at T = 300),
+    # which is already 1e-4 relative at 1e-2 RMS; smaller elements are bounded by max/RMS.
+    big = np.abs(o) >= 1e-1 * r
     rel = float((d[big] / np.abs(o[big])).max()) if big.any() else 0.0
     return rel, float(d.max() / r)
 

@@ -155,22 +155,28 @@ def test_dtraw_validation(lib):
 
 
 def test_varlen_validation(lib):
+    """Workspace sizes of both paths; every call below fails validation before any launch
+    (a zero workspace where the sizes themselves are valid)."""
     F = FAKE
     ws = lib.ssd_prefill_varlen_workspace_bytes
     up = lambda v: (v + 255) // 256 * 256
     nseq, T, H = 3, 1000, 4
-    nb = T // 128 + nseq                             # block bound: floor(T / 128) + nseq
+    nb = T // 128 + nseq                             # tensor-core block bound: floor(T / 128) + nseq
     main = (up(H * nb * 4 * 128 * 4) + up(H * nb * 132 * 4) + up(H * nb * 16384) + up(T * 128 * 2))
     assert ws(nseq, T, H, 64, 1, 128, 256, binding.SSD_BF16) == main + up((nseq + 1) * 4) + up(nb * 4)
     assert ws(nseq, 0, H, 64, 1, 128, 256, binding.SSD_BF16) == 0
-    assert ws(nseq, T, H, 64, 1, 128, 256, binding.SSD_F32) == 0          # tensor-core path only
+    nc = T // 64 + nseq                              # CUDA-core chunks of 64: lam + per-chunk fp32 states
+    simt = up(H * nc * 64 * 4) + up(H * nc * 64 * 128 * 4)
+    assert ws(nseq, T, H, 64, 1, 128, 64, binding.SSD_F32) == simt + up((nseq + 1) * 4) + up(nc * 4)
     f = lib.ssd_prefill_varlen
     args = lambda **kw: [F, F, F, F, F, F, None, kw.get("cu", F), kw.get("nseq", 3), kw.get("T", 1000), 4,
                          kw.get("P", 64), 1, 128, kw.get("Q", 256), kw.get("dtype", binding.SSD_BF16), F, F, F,
-                         1 << 30, None]
-    assert f(*args(dtype=binding.SSD_F32)) == 5
-    assert f(*args(P=32)) == 5
-    assert f(*args(Q=64)) == 5
+                         kw.get("wsb", 0), None]
+    assert f(*args()) == 8                           # workspace too small (checked before any launch)
+    assert f(*args(dtype=binding.SSD_F32)) == 8      # CUDA-core path, same check
+    assert f(*args(Q=512)) == 5
+    assert f(*args(P=12)) == 2
+    assert f(*args(dtype=7)) == 3
     assert f(*args(nseq=0)) == 2
     assert f(*args(T=-1)) == 2
     assert f(*args(cu=None)) == 1

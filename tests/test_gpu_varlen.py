@@ -111,3 +111,54 @@ def test_bad_offsets_are_reported_not_read():
     torch.cuda.synchronize()
     assert ssd.ssd_device_status() == 2               # SSD_ERR_SHAPE
     assert torch.count_nonzero(y) == 0
+
+
+@pytest.mark.parametrize("bf16,Q,N", [(False, 64, 64), (False, 100, 128), (True, 64, 128)])
+def test_cuda_core_path_mixed_lengths(bf16, Q, N):
+    """The CUDA-core path (fp32, or chunk lengths the tensor-core path does not take)."""
+    import state_space_model_05_b200 as ssd
+    from parity import assert_fp32
+    lengths = [150, 0, 1, 63, 64, 65, 300, 7]
+    T = sum(lengths)
+    inp = gen.prefill_inputs(gen.SSDShape(1, T, 4, 64, 2, N), seed=Q + N)
+    if bf16:
+        inp.x, inp.B, inp.C = gen.round_bf16(inp.x), gen.round_bf16(inp.B), gen.round_bf16(inp.C)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    dt_ = torch.bfloat16 if bf16 else torch.float32
+    f32 = torch.float32
+    rng = np.random.default_rng(3)
+    init = (0.1 * rng.standard_normal((len(lengths), 4, 64, N))).astype(np.float32)
+    y, st = ssd.ssd_prefill_varlen(to_dev(inp.x[0], dt_), to_dev(inp.dt[0], f32), to_dev(inp.A, f32),
+                                   to_dev(inp.B[0], dt_), to_dev(inp.C[0], dt_), to_dev(inp.D, f32),
+                                   torch.from_numpy(cu).cuda(), Q, init_states=to_dev(init, f32))
+    torch.cuda.synchronize()
+    assert ssd.ssd_device_status() == 0
+    y, st = y.float().cpu().numpy(), st.cpu().numpy()
+    for i, n in enumerate(lengths):
+        a, b = cu[i], cu[i + 1]
+        if n == 0:
+            assert np.array_equal(st[i], init[i])
+            continue
+        yo, so = oracle.prefill(inp.x[:, a:b], inp.dt[:, a:b], inp.A, inp.B[:, a:b], inp.C[:, a:b], inp.D,
+                                init=init[i].astype(np.float64))
+        what = f"varlen CUDA-core Q={Q} seq {i} (len {n})"
+        if bf16:
+            assert_bf16_y(y[a:b], oracle.units_to_bthp(yo, 1, 4)[0], what + " y")
+            assert_state(st[i], so.reshape(st[i].shape), what + " state")
+        else:
+            assert_fp32(y[a:b], oracle.units_to_bthp(yo, 1, 4)[0], what + " y")
+            assert_fp32(st[i], so.reshape(st[i].shape), what + " state")
+
+
+def test_cuda_core_equal_lengths_equal_batched_call_bitwise():
+    import state_space_model_05_b200 as ssd
+    inp = gen.prefill_inputs(gen.SSDShape(3, 200, 4, 32, 1, 64), seed=12)
+    f32 = torch.float32
+    x, dt, B, C = (to_dev(a, f32) for a in (inp.x, inp.dt, inp.B, inp.C))
+    A, D = to_dev(inp.A, f32), to_dev(inp.D, f32)
+    y1, s1 = ssd.ssd_prefill(x, dt, A, B, C, D, 64)
+    cu = torch.tensor([0, 200, 400, 600], dtype=torch.int32, device="cuda")
+    y2, s2 = ssd.ssd_prefill_varlen(x.reshape(600, 4, 32), dt.reshape(600, 4), A, B.reshape(600, 1, 64),
+                                    C.reshape(600, 1, 64), D, cu, 64)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.reshape(600, 4, 32), y2) and torch.equal(s1, s2)
