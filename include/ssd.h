@@ -152,8 +152,8 @@ ssd_status_t ssd_decode_step_dtraw(float* state, const void* x_t, const float* d
  *   cu_seqlens: DEVICE array of nseq + 1 int32 offsets, read by the kernels: cu_seqlens[0]
  *   = 0, non-decreasing, cu_seqlens[nseq] = total_tokens (else SSD_ERR_SHAPE is recorded
  *   in the device error word and nothing is computed).  Empty sequences are allowed.
- * Supported on the tensor-core path only: bf16, headdim 64, dstate 128, chunk_len 128 or
- * 256 (else SSD_ERR_UNSUPPORTED).  `workspace` must hold
+ * Sizes and dtypes as for ssd_prefill (the tensor-core path for bf16, headdim 64, dstate
+ * 128, chunk_len 128 or 256; the CUDA-core path otherwise).  `workspace` must hold
  * ssd_prefill_varlen_workspace_bytes(...) bytes (0 when total_tokens is 0).
  */
 size_t ssd_prefill_varlen_workspace_bytes(int nseq, int total_tokens, int nheads, int headdim,
