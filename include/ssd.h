@@ -107,6 +107,27 @@ ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const v
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Which tensor-core kernels a batched bf16 prefill (headdim 64, dstate 128, chunk_len 128
+ * or 256) runs, process-wide:
+ *   SSD_PREFILL_TWO_PASS: a chunk-state walk writes each block's start state to the
+ *     workspace, then a block-output kernel reads it back (one CTA per block and group
+ *     of heads);
+ *   SSD_PREFILL_FUSED: one kernel walks the 128-token blocks of each (batch, 1-3 heads) in
+ *     order with the states in tensor memory and writes y and the final state, after a
+ *     kernel forming G = C B^T per block (x read once, no state through HBM);
+ *   SSD_PREFILL_AUTO (the default): the two-pass kernels, the faster of the two on every
+ *     workload measured so far.
+ * Both compute the same chunked algorithm with bf16 operands and fp32 accumulation; the
+ * results agree to rounding.  Packed variable-length prefills always take the two-pass
+ * kernels, other shapes the CUDA-core path.  The workspace size covers either.  Returns
+ * SSD_ERR_SHAPE for an unknown value.  Not synchronised with calls in flight on other
+ * host threads.
+ */
+typedef enum { SSD_PREFILL_AUTO = 0, SSD_PREFILL_FUSED = 1, SSD_PREFILL_TWO_PASS = 2 } ssd_prefill_path_t;
+ssd_status_t ssd_set_prefill_path(ssd_prefill_path_t path);
+ssd_prefill_path_t ssd_get_prefill_path(void);
+
+/*
  * One decode step on the state cache, in place: each fp32 state row is read
  * once, decayed by exp(dt_t * A_h), given the rank-1 update dt_t B_t x_t^T,
  * reduced against C_t for y_t, and written back.  x_t, B_t, C_t, y_t are

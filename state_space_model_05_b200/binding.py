@@ -42,6 +42,8 @@ SIGNATURES = {
     "ssd_decode_step_dtraw": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ssd_prefill_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P], _I),
     "ssd_device_status": ([_P], _I),
+    "ssd_set_prefill_path": ([_I], _I),
+    "ssd_get_prefill_path": ([], _I),
     "ssd_selftest_bounded_waits": ([_P, _P], _I),
     "ssd_profile_enable": ([_I], None),
     "ssd_profile_reset": ([], None),
@@ -115,6 +117,22 @@ def _need(t: torch.Tensor, name: str, dtype=None):
 def ssd_prefill_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len, dtype_code):
     return int(lib().ssd_prefill_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate,
                                                  chunk_len, dtype_code))
+
+
+PREFILL_PATHS = {"auto": 0, "fused": 1, "two_pass": 2}
+
+
+def ssd_set_prefill_path(path: str) -> str:
+    """Select the tensor-core prefill kernels ("auto", "fused" or "two_pass"; see
+    ``include/ssd.h``); returns the previous setting."""
+    prev = ssd_get_prefill_path()
+    _check(lib().ssd_set_prefill_path(PREFILL_PATHS[path]), "ssd_set_prefill_path")
+    return prev
+
+
+def ssd_get_prefill_path() -> str:
+    code = int(lib().ssd_get_prefill_path())
+    return next(k for k, v in PREFILL_PATHS.items() if v == code)
 
 
 def ssd_prefill(x, dt, A, B, C, D, chunk_len, init_state=None, y=None, final_state=None,

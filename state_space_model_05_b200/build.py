@@ -17,8 +17,8 @@ LIB = os.path.join(HERE, "libssd.so")
 GEN_LIB = os.path.join(HERE, "libssd_inputs.so")
 GEN_SRC = os.path.join(CSRC, "gen", "gen_inputs.cu")
 
-SOURCES = ["api.cu", "decode.cu", "gdn_decode.cu", "prefill_simt.cu", "prefill_tc.cu", "prefill_noalloc.cu",
-           "selftest.cu"]
+SOURCES = ["api.cu", "decode.cu", "gdn_decode.cu", "prefill_simt.cu", "prefill_tc.cu", "prefill_fused.cu",
+           "prefill_noalloc.cu", "selftest.cu"]
 HEADERS = ["common.cuh", "ptx.cuh", "prefill_tc.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

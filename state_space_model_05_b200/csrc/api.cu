@@ -4,6 +4,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
 #include <vector>
 
 #include "common.cuh"
@@ -67,11 +68,14 @@ ssd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_E
 
 // ---- opt-in kernel profiling: an event pair around each launch -------------------
 enum Stage { kCumsum, kStateTc, kStateSimt, kScan, kOutTc, kOutSimt, kDecode, kCopy, kDecodeLayers, kGdn,
-             kNumStages };
+             kGram, kChain, kNumStages };
 const char* const kStageNames[kNumStages] = {"chunk_cumsum", "chunk_state_scan_tc", "chunk_state_simt",
                                               "state_scan", "chunk_output_tc", "chunk_output_simt",
                                               "decode_step", "copy_state", "decode_step_layers",
-                                              "gdn_decode_step"};
+                                              "gdn_decode_step", "block_gram_tc", "chain_prefill_tc"};
+
+// which tensor-core prefill batched calls take (ssd_set_prefill_path)
+std::atomic<int> g_prefill_path{SSD_PREFILL_AUTO};
 struct ProfRecord { int stage; cudaEvent_t begin, end; };
 struct Profiler {
     bool on = false;
@@ -191,6 +195,18 @@ ssd_status_t prefill_impl(const void* x, const float* dt, const float* dt_bias, 
         TcWorkspace w;
         const size_t need = tc_workspace_layout(t, workspace, &w);
         if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
+        if (g_prefill_path.load() == SSD_PREFILL_FUSED) {
+            // fused: decay factors, G = C B^T per block, then the chain kernel
+            cudaError_t e = profiled(kCumsum, s, [&] {
+                return launch_chunk_cumsum(t, dt, A, w.fac, true, nullptr, B, w.b16, s);
+            });
+            if (e == cudaSuccess) e = profiled(kGram, s, [&] { return launch_block_gram(t, B, C, w, s); });
+            if (e == cudaSuccess)
+                e = profiled(kChain, s, [&] {
+                    return launch_chain_prefill(t, x, C, D, w, init_state, final_state, y, s);
+                });
+            return from_cuda(e);
+        }
         cudaError_t e = profiled(kCumsum, s, [&] {
             return launch_chunk_cumsum(t, dt, A, w.fac, true, w.wts, B, w.b16, s);
         });
@@ -346,6 +362,16 @@ ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const v
                         ngroups, dstate, chunk_len, dtype, y, final_state, workspace, workspace_bytes,
                         stream);
 }
+
+ssd_status_t ssd_set_prefill_path(ssd_prefill_path_t path)
+{
+    if (path != SSD_PREFILL_AUTO && path != SSD_PREFILL_FUSED && path != SSD_PREFILL_TWO_PASS)
+        return SSD_ERR_SHAPE;
+    g_prefill_path.store(path);
+    return SSD_OK;
+}
+
+ssd_prefill_path_t ssd_get_prefill_path(void) { return static_cast<ssd_prefill_path_t>(g_prefill_path.load()); }
 
 ssd_status_t ssd_prefill_dtraw(const void* x, const float* dt_raw, const float* dt_bias,
                                const float* A, const void* B, const void* C, const float* D,

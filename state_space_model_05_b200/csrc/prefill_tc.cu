@@ -30,6 +30,8 @@
 // for the output kernel the C/B loads and G) overlaps the previous kernel's tail.  Every
 // wait is bounded; expiry records SSD_ERR_TIMEOUT in the device error word and the CTA
 // drains without further waiting.
+#include <algorithm>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -567,8 +569,8 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 bool progressed = false;
                 if (jo < heads_per_cta) {
                     const int s = jo % kXSlots, a = jo % kAccSlots;
-                    if (mbar_try_wait(&bars[BAR_XFULL + s], (jo / kXSlots) & 1) &&
-                        (jo < kAccSlots || mbar_try_wait(&bars[BAR_AEMPTY + a], (jo / kAccSlots - 1) & 1))) {
+                    if (mbar_test_wait(&bars[BAR_XFULL + s], (jo / kXSlots) & 1) &&
+                        (jo < kAccSlots || mbar_test_wait(&bars[BAR_AEMPTY + a], (jo / kAccSlots - 1) & 1))) {
                         tc_fence_after();
                         const uint32_t aH = smem_u32(hslot(jo % kHSlots));
                         // Yo = C_t H_k^T: A = C (K-major over n), B = H image (MN-major, 64-byte
@@ -586,7 +588,7 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 }
                 if (jd < jo) {
                     const int s = jd % kXSlots, a = jd % kAccSlots, p = jd & 1;
-                    if (mbar_try_wait(&bars[BAR_PFULL + p], (jd >> 1) & 1)) {
+                    if (mbar_test_wait(&bars[BAR_PFULL + p], (jd >> 1) & 1)) {
                         tc_fence_after();
                         const uint32_t aX = smem_u32(slot(s) + L::kXo);
                         // Yd = P X: A = P in TMEM (eight columns per 16 tokens), B = X (MN-major)
@@ -602,8 +604,8 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 }
                 if (progressed) {
                     idle = 0;
-                } else if (++idle >= (1u << 22) || ((idle & 1023u) == 0 && *abort_flag)) {
-                    if (idle >= (1u << 22)) {
+                } else if (++idle >= (1u << 24) || ((idle & 1023u) == 0 && *abort_flag)) {
+                    if (idle >= (1u << 24)) {
                         record_error(err, SSD_ERR_TIMEOUT);
                         *abort_flag = 1;
                     }
@@ -831,25 +833,6 @@ int heads_per_cta(const Dims& d)
     return best;
 }
 
-// Launch with programmatic stream serialisation: the kernel may start while the previous
-// kernel of the stream finishes, and waits (griddepcontrol.wait) before reading its output.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                             Args... args)
-{
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
-}
-
 int sm_count()
 {
     static int cache[64] = {0};
@@ -912,6 +895,14 @@ cudaError_t output_launch(const Dims& d, const CUtensorMap& mx, const CUtensorMa
 
 }  // namespace
 
+bool tc_make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
+                 CUtensorMapDataType type, uint32_t box_rows)
+{
+    return make_map(m, base, inner, rows, outer, type, box_rows);
+}
+
+int tc_sm_count() { return sm_count(); }
+
 bool tc_prefill_supported(const Dims& d)
 {
     return d.headdim == kP && d.dstate == kN && (d.chunk_len == 128 || d.chunk_len == 256);
@@ -933,14 +924,17 @@ size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w)
     const size_t wts_b = up(BH * d.nchunks * (d.chunk_len + 4) * sizeof(float));
     const size_t himg_b = up(BH * d.nchunks * kHImage);
     const size_t b16_b = up((size_t)d.batch * d.seqlen * d.ngroups * kN * 2);
+    const size_t gram_b = up((size_t)d.batch * d.ngroups * d.nchunks * kBlk * kBlk * 2);
+    const size_t mid_b = std::max(wts_b + himg_b, gram_b);
     if (w) {
         char* p = static_cast<char*>(base);
         w->fac = reinterpret_cast<float*>(p);
         w->wts = reinterpret_cast<float*>(p + fac_b);
         w->himg = reinterpret_cast<uint8_t*>(p + fac_b + wts_b);
-        w->b16 = p + fac_b + wts_b + himg_b;
+        w->gram = reinterpret_cast<uint4*>(p + fac_b);
+        w->b16 = p + fac_b + mid_b;
     }
-    return fac_b + wts_b + himg_b + b16_b;
+    return fac_b + mid_b + b16_b;
 }
 
 Dims tc_varlen_dims(int nseq, int total_tokens, int nheads, int headdim, int ngroups, int dstate)

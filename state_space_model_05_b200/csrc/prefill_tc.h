@@ -1,6 +1,8 @@
 // Tensor-core (tcgen05 / TMEM / TMA) stages of the bf16 chunked prefill.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace ssd {
@@ -23,7 +25,11 @@ struct TcWorkspace {
     uint8_t* himg;    // [b][h][c] 16 KB bf16 image of each block's start state (MN-major,
                       //   64-byte swizzle: two 8 KB p-halves of [128 n][32 p])
     void* b16;        // [b][T][G][N] fp16 copy of B (operand of the chunk-state GEMM)
+    uint4* gram;      // fused path, over wts / himg: [b][g][c] bf16 G = C B^T of each block,
+                      //   four planes of 32 columns ([plane][row t][32 bf16])
 };
+// Sized for either path: fac, then wts + himg (two-pass) or gram (fused), whichever is
+// larger, then b16 (both).
 size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w);
 
 // Packed variable-length prefill: the block dims (batch 1, an upper bound of blocks), the
@@ -42,5 +48,41 @@ cudaError_t launch_chunk_state_scan_tc(const Dims& d, const void* x, const void*
 // Per 128-token block: y = (C B^T o L o dt) X + diag(exp Lam) C H_k^T + D x, bf16 out.
 cudaError_t launch_chunk_output_tc(const Dims& d, const void* x, const void* B, const void* C,
                                    const float* D, const TcWorkspace& w, void* y, cudaStream_t s);
+
+// Fused path (batched, not packed variable-length), launched after the cumsum kernel:
+// G = C B^T of every block (bf16, w.gram); then one kernel that walks each (b, 1-3 heads)
+// chain of blocks with the states in TMEM and writes y and the final state.  Both are
+// programmatic dependents; the G kernel completes only after the cumsum kernel has.
+cudaError_t launch_block_gram(const Dims& d, const void* B, const void* C, const TcWorkspace& w,
+                              cudaStream_t s);
+// The chain kernel reads the fp16 copy of B (w.b16) that the cumsum kernel writes.
+cudaError_t launch_chain_prefill(const Dims& d, const void* x, const void* C, const float* D,
+                                 const TcWorkspace& w, const float* init_state, float* final_state,
+                                 void* y, cudaStream_t s);
+
+// helpers shared by the tensor-core launchers
+// 16-bit tensor [outer][rows][inner] read in boxes of 64 (inner) x box_rows, 128-byte swizzle.
+bool tc_make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
+                 CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, uint32_t box_rows = 128);
+int tc_sm_count();
+
+// Launch with programmatic stream serialisation: the kernel may start while the previous
+// kernel of the stream finishes, and waits (griddepcontrol.wait) before reading its output.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 }  // namespace ssd

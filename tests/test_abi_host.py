@@ -54,13 +54,16 @@ def test_workspace_bytes(lib):
     st = b * H * c * P * N * 4
     assert _ws(b, T, H, P, G, N, Q, binding.SSD_F32) == up(lam) + up(st)
     # tensor-core path (bf16, P 64, N 128, Q 128/256), sized by 128-token blocks: per block
-    # Lam, dt and two column-factor rows, the chunk-state weights and block decay, bf16
-    # block-start-state images, fp16 copy of B
+    # Lam, dt and two column-factor rows; then either the two-pass kernels' chunk-state
+    # weights and block decay and bf16 block-start-state images, or the fused kernels' bf16
+    # G = C B^T per (b, g, block), whichever is larger; then the fp16 copy of B (both)
     def tc_bytes(T):
         nb = -(-T // 128)
         fac = b * H * nb * 4 * 128 * 4           # Lam, dt, two column-factor rows
         wts = b * H * nb * (128 + 4) * 4          # chunk-state weights + block decay
-        return up(fac) + up(wts) + up(b * H * nb * 16384) + up(b * T * G * N * 2)
+        two_pass = up(wts) + up(b * H * nb * 16384)
+        gram = up(b * G * nb * 128 * 128 * 2)
+        return up(fac) + max(two_pass, gram) + up(b * T * G * N * 2)
     assert _ws(b, T, H, P, G, N, Q, binding.SSD_BF16) == tc_bytes(T)
     assert _ws(b, T, H, P, G, N, 256, binding.SSD_BF16) == tc_bytes(T)
     # bf16 with other shapes uses the CUDA-core layout
@@ -210,3 +213,19 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
 
 def test_selftest_rejects_null_scratch(lib):
     assert lib.ssd_selftest_bounded_waits(None, None) == 1
+
+
+def test_prefill_path_setting(lib):
+    """The tensor-core path selector: known values round-trip, others are refused."""
+    prev = lib.ssd_get_prefill_path()
+    try:
+        for v in (1, 2, 0):
+            assert lib.ssd_set_prefill_path(v) == 0
+            assert lib.ssd_get_prefill_path() == v
+        assert lib.ssd_set_prefill_path(3) == 2
+        assert lib.ssd_set_prefill_path(-1) == 2
+        assert lib.ssd_get_prefill_path() == 0
+        assert binding.ssd_set_prefill_path("two_pass") == "auto"
+        assert binding.ssd_get_prefill_path() == "two_pass"
+    finally:
+        lib.ssd_set_prefill_path(prev)

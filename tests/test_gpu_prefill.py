@@ -4,7 +4,8 @@ Workloads: the fp32 single SSD layer (batch 1, 256 tokens, 4 heads, P = N = 64,
 chunk 64), the Mamba-2-130M-shaped bf16 layer (batch 8, 2048 tokens, 24 heads,
 P 64, N 128, chunk 256) and the 2.7B-shaped long bf16 prefill (batch 4, 16384
 tokens, 80 heads, chunk 256; sampled (batch, head) units), plus ragged, empty,
-grouped, init-state and chunk-length cases.
+grouped, init-state and chunk-length cases.  The bf16 tensor-core cases run on both
+tensor-core paths: the fused chain kernel and the two-pass (walk + block output) kernels.
 """
 import numpy as np
 import pytest
@@ -23,6 +24,15 @@ def _built():
     from state_space_model_05_b200.build import build
     build()
     oracle.build()
+
+
+@pytest.fixture(params=["fused", "two_pass"])
+def tc_path(request):
+    """Runs the test once per tensor-core prefill path (process-wide setting, restored)."""
+    import state_space_model_05_b200 as ssd
+    prev = ssd.ssd_set_prefill_path(request.param)
+    yield request.param
+    ssd.ssd_set_prefill_path(prev)
 
 
 def _check_fp32(inp, Q, init=None):
@@ -118,7 +128,7 @@ def test_empty_sequence_copies_init():
 
 
 # --------------------------------------------------------------------- bf16 path
-def test_bf16_130m_layer_full():
+def test_bf16_130m_layer_full(tc_path):
     """130M-shaped layer: b=8, T=2048, H=24, P=64, N=128, G=1, chunk 256, all outputs."""
     inp = problem(gen.SSDShape(8, 2048, 24, 64, 1, 128), bf16=True, seed=0)
     _check_bf16(inp, 256)
@@ -126,20 +136,20 @@ def test_bf16_130m_layer_full():
 
 @pytest.mark.parametrize("T,Q,G", [(1000, 256, 2), (300, 128, 1), (129, 128, 4), (1, 256, 1),
                                    (512, 64, 1), (700, 100, 1)])
-def test_bf16_ragged_groups_chunks(T, Q, G):
+def test_bf16_ragged_groups_chunks(T, Q, G, tc_path):
     """Tensor-core path (Q 128/256, partial last chunk, G > 1) and the SIMT path (other Q)."""
     inp = problem(gen.SSDShape(2, T, 4, 64, G, 128), bf16=True, seed=T + Q + G)
     _check_bf16(inp, Q)
 
 
-def test_bf16_init_state():
+def test_bf16_init_state(tc_path):
     rng = np.random.default_rng(6)
     inp = problem(gen.SSDShape(2, 600, 4, 64, 1, 128), bf16=True, seed=21)
     init = (rng.standard_normal((2, 4, 64, 128)) * 0.05).astype(np.float32)
     _check_bf16(inp, 256, init=init)
 
 
-def test_bf16_chunk_length_invariance():
+def test_bf16_chunk_length_invariance(tc_path):
     inp = problem(gen.SSDShape(1, 1024, 8, 64, 1, 128), bf16=True, seed=22)
     b, T, H, P = inp.x.shape
     yo, so = oracle_prefill(inp)
@@ -150,7 +160,7 @@ def test_bf16_chunk_length_invariance():
 
 
 @pytest.mark.parametrize("G,with_init", [(1, False), (2, True)])
-def test_bf16_many_chains_full(G, with_init):
+def test_bf16_many_chains_full(G, with_init, tc_path):
     """More (batch, head) chains than two per SM (here 320): the chunk-state walk packs up to
     three heads per CTA.  Every token and the final state are checked."""
     inp = problem(gen.SSDShape(4, 384, 80, 64, G, 128), bf16=True, seed=30 + G)
@@ -160,7 +170,7 @@ def test_bf16_many_chains_full(G, with_init):
     _check_bf16(inp, 256, init=init)
 
 
-def test_bf16_27b_long_prefill_sampled():
+def test_bf16_27b_long_prefill_sampled(tc_path):
     """2.7B-shaped long prefill (b=4, T=16384, H=80, P=64, N=128, chunk 256) at full size,
     checked on sampled (batch, head) units: all tokens of y and the final state."""
     inp = problem(gen.SSDShape(4, 16384, 80, 64, 1, 128), bf16=True, seed=0)
@@ -173,6 +183,41 @@ def test_bf16_27b_long_prefill_sampled():
     assert np.isfinite(y).all() and np.isfinite(st).all()
 
 
+def test_bf16_init_aliases_final(tc_path):
+    """init_state may be the final_state buffer: each state element is read before it is
+    written."""
+    from state_space_model_05_b200 import ssd_prefill
+    rng = np.random.default_rng(12)
+    inp = problem(gen.SSDShape(2, 300, 4, 64, 1, 128), bf16=True, seed=44)
+    init = (rng.standard_normal((2, 4, 64, 128)) * 0.05).astype(np.float32)
+    bf = torch.bfloat16
+    st = to_dev(init)
+    ssd_prefill(to_dev(inp.x, bf), to_dev(inp.dt), to_dev(inp.A), to_dev(inp.B, bf), to_dev(inp.C, bf),
+                to_dev(inp.D), 256, init_state=st, final_state=st)
+    torch.cuda.synchronize()
+    yo, so = oracle_prefill(inp, init=init.reshape(8, 64, 128))
+    assert_state(st.cpu().numpy(), so.reshape(2, 4, 64, 128), "aliased state")
+
+
+def test_paths_agree_closely():
+    """The fused and two-pass kernels compute the same algorithm in bf16/fp32: their outputs
+    differ only by rounding (well inside the oracle tolerance)."""
+    import state_space_model_05_b200 as ssd
+    inp = problem(gen.SSDShape(2, 1000, 8, 64, 2, 128), bf16=True, seed=45)
+    out = {}
+    for path in ("fused", "two_pass"):
+        prev = ssd.ssd_set_prefill_path(path)
+        try:
+            out[path] = gpu_prefill(inp, 256, bf16=True)
+        finally:
+            ssd.ssd_set_prefill_path(prev)
+    (yf, sf), (yt, stt) = out["fused"], out["two_pass"]
+    ry = float(np.sqrt(np.mean(yt.astype(np.float64) ** 2)))
+    rs = float(np.sqrt(np.mean(stt.astype(np.float64) ** 2)))
+    assert float(np.abs(yf - yt).max()) / ry < 2e-2
+    assert float(np.abs(sf - stt).max()) / rs < 1e-2
+
+
 def test_device_status_clean():
     from state_space_model_05_b200 import ssd_device_status
     assert ssd_device_status() == 0
@@ -183,7 +228,7 @@ def test_device_status_clean():
     (False, gen.SSDShape(2, 300, 4, 64, 1, 64), 64, 340),
     (True, gen.SSDShape(2, 700, 4, 64, 1, 128), 256, 740),
     (True, gen.SSDShape(2, 256, 4, 64, 2, 128), 128, 41)])
-def test_dt_softplus_folded_in(bf16, shape, Q, seed):
+def test_dt_softplus_folded_in(bf16, shape, Q, seed, tc_path):
     """ssd_prefill_dtraw forms dt = softplus(dt_raw + dt_bias) itself.  It must equal, bit for
     bit, the plain call given that dt (formed in fp64 by the oracle's softplus and rounded to
     fp32 once), and match the fp64 oracle within the path's tolerance."""
