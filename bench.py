@@ -731,6 +731,17 @@ def ours(args, rank, world):
         line["prefill_130m_dt_softplus"] = {"value": r["tokens_per_s"], "unit": "tokens/s",
                                             "ms_per_step": r["ms_per_step"],
                                             "kernels_ms": {k: v[0] / v[1] for k, v in r["kernels"].items()}}
+        # the same headline prefill on the fused tensor-core path (opt-in; the default two-pass
+        # kernels are faster on this workload)
+        from state_space_model_05_b200 import binding as _binding
+        prev_path = _binding.ssd_set_prefill_path("fused")
+        try:
+            r = run_prefill(w, 100, 5, rank, world, "prefill_130m_fused", e2e=False)
+        finally:
+            _binding.ssd_set_prefill_path(prev_path)
+        line["prefill_130m_fused_path"] = {"value": r["tokens_per_s"], "unit": "tokens/s",
+                                           "ms_per_step": r["ms_per_step"],
+                                           "kernels_ms": {k: v[0] / v[1] for k, v in r["kernels"].items()}}
         # the same tokens as one packed batch of mixed-length sequences (state reset per sequence)
         vr = run_prefill_varlen(w, 100, 5, rank, world)
         line["prefill_130m_varlen"] = {"value": vr["tokens_per_s"], "unit": "tokens/s",
