@@ -29,6 +29,7 @@ constexpr int kThreads = 256;
 // shared memory so that both the read and the write are coalesced.
 // ----------------------------------------------------------------------------------
 constexpr int kCumsumHeads = 8;      // one warp per head
+static_assert(kMaxChunk * kCumsumHeads % kThreads == 0, "dt rows per thread");
 
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
     const float lo = __uint_as_float(u << 16), hi = __uint_as_float(u & 0xFFFF0000u);
@@ -62,13 +63,17 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
         int sq;
         if (!varlen_block(vl_cu, vl_first, vl_seq, c, Q, &sq, &t0, &valid)) return;
     }
-    // dt rows first, so that their loads and those of the B copy below are in flight together
-    for (int i = threadIdx.x; i < Q * kCumsumHeads; i += blockDim.x) {
+    // every dt load of this thread is issued before any is used, and the B copy's loads below
+    // go out while they are in flight; the values land in shared memory after the copy
+    constexpr int kDtPer = kMaxChunk * kCumsumHeads / kThreads;
+    float raw[kDtPer];
+    bool use[kDtPer];
+#pragma unroll
+    for (int m = 0; m < kDtPer; ++m) {
+        const int i = threadIdx.x + m * kThreads;
         const int t = i / kCumsumHeads, hh = i - t * kCumsumHeads;
-        float v = 0.f;
-        if (hh < nh && t < valid)
-            v = dt_value(dt[((size_t)b * seqlen + t0 + t) * nheads + h0 + hh], dt_bias, dt_softplus, h0 + hh);
-        sm_dt[i] = v;
+        use[m] = i < Q * kCumsumHeads && hh < nh && t < valid;
+        raw[m] = use[m] ? dt[((size_t)b * seqlen + t0 + t) * nheads + h0 + hh] : 0.f;
     }
     if (b_f16) {
         // fp16 copy of this chunk's rows of B (bf16 -> fp16 is exact for these values'
@@ -99,6 +104,12 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
                 }
             }
         }
+    }
+#pragma unroll
+    for (int m = 0; m < kDtPer; ++m) {
+        const int i = threadIdx.x + m * kThreads;
+        if (i < Q * kCumsumHeads)
+            sm_dt[i] = use[m] ? dt_value(raw[m], dt_bias, dt_softplus, h0 + (i % kCumsumHeads)) : 0.f;
     }
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
