@@ -654,13 +654,15 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                 const uint32_t* v = w2 ? v1 : v0;
                 const int s0 = kc * 32;
                 uint32_t pk[16];
-                if (s0 + 31 <= r) {
+                // the branch is taken by the warp's 32 rows (q * 32 ..) alike: a diagonal
+                // sub-block is one path for the whole warp, not two in series
+                if (kc < q) {
                     const float u = expf(lam_t - sLam[s0 + 31]);
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
                         pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * u * sV[s0 + 2 * e],
                                             __uint_as_float(v[2 * e + 1]) * u * sV[s0 + 2 * e + 1]);
-                } else if (s0 > r) {
+                } else if (kc > q) {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) pk[e] = 0u;
                 } else if (sLam[s0] - sLam[s0 + 31] < 40.f) {
