@@ -245,11 +245,11 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
                 tc_fence_after();
                 const uint32_t aB = smem_u32(stage(st)), aX = aB + L::kStageX;
                 // S_c[n][64 hh + p] += sum_s B_s[n] X~_s[hh][p] over this stage's 64 rows
+                const uint64_t dB = smem_desc_sw128(aB, kQBox, 1024), dX = smem_desc_sw128(aX, kQBox, 1024);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    umma_f16(tmem + (c & 1) * L::kAccStride, smem_desc_sw128(aB + ks * 2048, kQBox, 1024),
-                             smem_desc_sw128(aX + ks * 2048, kQBox, 1024), idesc,
-                             (qq > 0 || ks > 0) ? 1u : 0u);
+                    umma_f16(tmem + (c & 1) * L::kAccStride, desc_advance(dB, ks * 2048), desc_advance(dX, ks * 2048),
+                             idesc, (qq > 0 || ks > 0) ? 1u : 0u);
                 umma_commit(&empty[st]);
                 if (qq == NQ - 1) umma_commit(&accb[c & 1]);
                 done = k + 1;
@@ -561,6 +561,7 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
             }
             umma_commit(&bars[BAR_S]);
             constexpr uint32_t idMN = idesc_bf16_f32(128, 64, false, true);
+            const uint64_t dC = smem_desc_sw128(aC, 16, 1024);
             // Yo of a head is issued as soon as its slot is loaded (and its accumulator free),
             // Yd as soon as its P is built; the two streams are polled, not ordered
             int jo = 0, jd = 0;
@@ -575,11 +576,12 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                         const uint32_t aH = smem_u32(hslot(jo % kHSlots));
                         // Yo = C_t H_k^T: A = C (K-major over n), B = H image (MN-major, 64-byte
                         // swizzle: p-halves 8 KB apart, 8-row groups of n 512 B apart)
+                        const uint64_t dH = smem_desc_sw64(aH, 8192, 512);
 #pragma unroll
                         for (int ks = 0; ks < 8; ++ks) {
                             const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
-                            umma_f16(tmem + a * kAccCols + 64, smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
-                                     smem_desc_sw64(aH + ks * 1024, 8192, 512), idMN, ks > 0 ? 1u : 0u);
+                            umma_f16(tmem + a * kAccCols + 64, desc_advance(dC, kb * kBox + off),
+                                     desc_advance(dH, ks * 1024), idMN, ks > 0 ? 1u : 0u);
                         }
                         umma_commit(&bars[BAR_HEMPTY + jo % kHSlots]);
                         ++jo;
@@ -590,12 +592,12 @@ block_output_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_const
                     const int s = jd % kXSlots, a = jd % kAccSlots, p = jd & 1;
                     if (mbar_test_wait(&bars[BAR_PFULL + p], (jd >> 1) & 1)) {
                         tc_fence_after();
-                        const uint32_t aX = smem_u32(slot(s) + L::kXo);
+                        const uint64_t dX = smem_desc_sw128(smem_u32(slot(s) + L::kXo), kBox, 1024);
                         // Yd = P X: A = P in TMEM (eight columns per 16 tokens), B = X (MN-major)
 #pragma unroll
                         for (int ks = 0; ks < 8; ++ks)
-                            umma_f16_ts(tmem + a * kAccCols, tmem + pcol(p) + ks * 8,
-                                        smem_desc_sw128(aX + ks * 2048, kBox, 1024), idMN, ks > 0 ? 1u : 0u);
+                            umma_f16_ts(tmem + a * kAccCols, tmem + pcol(p) + ks * 8, desc_advance(dX, ks * 2048),
+                                        idMN, ks > 0 ? 1u : 0u);
                         umma_commit(&bars[BAR_PEMPTY + p]);
                         umma_commit(&bars[BAR_AFULL + a]);
                         ++jd;

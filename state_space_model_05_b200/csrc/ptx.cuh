@@ -316,6 +316,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t lbo,
     return d;
 }
 
+// A descriptor for the tile `bytes` further on in shared memory (same strides and swizzle):
+// the start-address field holds addr / 16 in 14 bits, and shared addresses stay below 2^18,
+// so the sum never carries out of the field.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) {
+    return desc + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor: kind::f16 with bf16 A and B, fp32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
     return (1u << 4)                        // D format: f32
