@@ -95,7 +95,12 @@ def prefill_bytes(w) -> dict:
             "chunk_state_scan_tc": b * T * (H * P * e + G * N * 2) + rows * 4 + image + b * H * P * N * 4,
             # x, B, C, block factors and block-start images in; y out
             "chunk_output_tc": b * T * (2 * H * P * e + 2 * G * N * e) + 4 * rows * 4 + image,
-            "state_scan": 2 * b * H * c * P * N * 4 + b * H * P * N * 4}
+            "state_scan": 2 * b * H * c * P * N * 4 + b * H * P * N * 4,
+            # fused path: B, C in; bf16 G = C B^T of every (b, g, block) out
+            "block_gram_tc": 2 * b * T * G * N * e + b * G * nb * TC_BLOCK * TC_BLOCK * 2,
+            # fused path: x, fp16 B, C, G and the block factors in; y and the final state out
+            "chain_prefill_tc": b * T * (2 * H * P * e + 2 * G * N * 2) + b * G * nb * TC_BLOCK * TC_BLOCK * 2
+                                + 4 * rows * 4 + b * H * P * N * 4}
 
 
 def decode_bytes(w) -> int:
@@ -640,6 +645,8 @@ def ours(args, rank, world):
     build()
     w = WORKLOADS[args.workload]
     peaks, src = load_peaks()
+    from state_space_model_05_b200 import binding as _binding
+    _binding.ssd_set_prefill_path(args.prefill_path)
     gpu_id = None
     try:
         gpu_id = "GPU-" + str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
@@ -700,6 +707,8 @@ def ours(args, rank, world):
         line["e2e"] = None
         cfg = {"workload": args.workload, **{k: w[k] for k in w if k != "kind"}}
     cfg["parallelism"] = f"independent problem per GPU x{world}"
+    if args.prefill_path != "auto":
+        cfg["prefill_path"] = args.prefill_path
     line["config"] = cfg
 
     if not args.no_extras and args.workload == "prefill_130m":
@@ -838,6 +847,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill_130m")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-path", choices=["auto", "fused", "two_pass"], default="auto",
+                    help="tensor-core prefill kernels (ssd_set_prefill_path)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
