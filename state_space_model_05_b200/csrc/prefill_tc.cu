@@ -112,13 +112,16 @@ varlen_table_kernel(const int* __restrict__ cu, int nseq, int total_tokens, int 
 // Operands stream through a 4-deep ring of 64-row stages (fp16 B rows, one X box per
 // head, the heads' weights w_s and, with a chunk's last stage, its decay exp(Lam_end));
 // two TMEM accumulators alternate between chunks.  Warp-specialised: one warp issues the
-// loads, one the MMAs, and eight worker warps (which hold the carried state) form
-// X~ = w o X and update the state; the update of chunk c - 1 runs a stage into chunk c,
-// once its accumulator is complete.  Each worker warp writes its own 2 KB piece of every
-// bf16 start-state image (the image's 64-byte-swizzled layout makes that piece
-// contiguous) and stores it with one bulk copy, so the update needs no CTA-wide barrier.
-constexpr int kWalkWorkers = 8;                               // warps w, w + 4: TMEM lane quarter w
-constexpr int kWalkThreads = (kWalkWorkers + 2) * 32;         // + load warp + MMA warp
+// loads, one the MMAs, four warps form X~ = w o X, and eight state warps (which hold the
+// carried state) update it as soon as a chunk's accumulator is complete and hand the
+// accumulator back, so that the update overlaps the conversion of the next stages.  Each
+// state warp writes its own 2 KB piece of every bf16 start-state image (the image's
+// 64-byte-swizzled layout makes that piece contiguous) and stores it with one bulk copy,
+// so the update needs no CTA-wide barrier.  The block decay comes from the weights rows
+// in global memory, read a block ahead.
+constexpr int kWalkWorkers = 8;                               // state warps w, w + 4: TMEM lane quarter w
+constexpr int kWalkConv = 4;                                  // warps forming X~ = w o X
+constexpr int kWalkThreads = (kWalkWorkers + 2 + kWalkConv) * 32;   // + load warp + MMA warp
 constexpr int kQBox = 8192;                                   // one 64-row x 128-byte box
 constexpr int kWRow = 68;                                     // weights per head in a stage (+ decay)
 
@@ -135,8 +138,8 @@ struct WalkCfg {
     static constexpr int kStageW = kStageX + NH * kQBox;            // float[heads][68]
     static constexpr int kStageBytes = kStageW + 1024;
     static constexpr int kImg = kStages * kStageBytes;              // state images, one per head
-    static constexpr int kBar = kImg + NH * kHImage;                // full, conv, empty, acc
-    static constexpr int kSlot = kBar + (3 * kStages + 2) * 8;
+    static constexpr int kBar = kImg + NH * kHImage;                // full, conv, empty, acc, acc free
+    static constexpr int kSlot = kBar + (3 * kStages + 4) * 8;
     static constexpr int kBytes = kSlot + 16 + 1024;
     static_assert(kStageBytes % 1024 == 0, "stages keep 1024-byte alignment");
     static_assert(kBytes * kCtasPerSm <= 227 * 1024, "walk shared memory");
@@ -150,7 +153,7 @@ struct WalkMaps {
 
 template <int Q, int NH>
 __global__ void __launch_bounds__(kWalkThreads, WalkCfg<NH>::kCtasPerSm)
-chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __restrict__ fac,
+chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __restrict__ wts,
                         const float* __restrict__ init_state, float* final_state,
                         uint8_t* __restrict__ himg, int nheads, int ngroups, int nchunks,
                         int ctas_per_group, int* err, const int* __restrict__ vl_cu,
@@ -165,6 +168,7 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
     uint64_t* conv = full + S;
     uint64_t* empty = conv + S;
     uint64_t* accb = empty + S;
+    uint64_t* accfree = accb + 2;
     uint32_t* slot = reinterpret_cast<uint32_t*>(sm + L::kSlot);
 
     // this CTA's heads: a contiguous range of one (b, g)
@@ -192,11 +196,13 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
     if (tid == 0) {
         for (int i = 0; i < S; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&conv[i], kWalkWorkers);
+            mbar_init(&conv[i], kWalkConv);
             mbar_init(&empty[i], 1);
         }
-        mbar_init(&accb[0], 1);
-        mbar_init(&accb[1], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&accb[i], 1);
+            mbar_init(&accfree[i], kWalkWorkers);
+        }
         fence_mbar_init();
     }
     if (warp == kWalkWorkers + 1) {
@@ -242,6 +248,8 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
             for (int k = 0; k < total; ++k) {
                 const int st = k % S, c = k / NQ, qq = k - c * NQ;
                 if (!mbar_wait(&conv[st], (k / S) & 1, err)) break;
+                // the state warps have read this accumulator's previous block (c - 2)
+                if (qq == 0 && c >= 2 && !mbar_wait(&accfree[c & 1], ((c >> 1) - 1) & 1, err)) break;
                 tc_fence_after();
                 const uint32_t aB = smem_u32(stage(st)), aX = aB + L::kStageX;
                 // S_c[n][64 hh + p] += sum_s B_s[n] X~_s[hh][p] over this stage's 64 rows
@@ -257,9 +265,53 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
             // the CTA does not release TMEM with MMAs in flight
             if (done > 0) mbar_wait(&empty[(done - 1) % S], ((done - 1) / S) & 1, err);
         }
+    } else if (warp >= kWalkWorkers + 2) {
+        // ---------------------------------------------------------------- X~ = w o X (fp16)
+        // consecutive threads take consecutive 16-byte chunks; chunk i: head i / 512, row
+        // (i / 8) % 64
+        const int ctid = tid - (kWalkWorkers + 2) * 32;
+        for (int k = 0; k < total; ++k) {
+            const int st = k % S;
+            if (!mbar_wait(&full[st], (k / S) & 1, err)) break;
+            uint4* sx = reinterpret_cast<uint4*>(stage(st) + L::kStageX);
+            const float* sw = reinterpret_cast<const float*>(stage(st) + L::kStageW);
+            constexpr int kPer = NH * 512 / (kWalkConv * 32);                 // chunks per thread
+            constexpr int kBatch = kPer % 3 == 0 ? 3 : kPer;                  // loads in flight
+            static_assert(kPer % kBatch == 0, "conversion batches");
+#pragma unroll
+            for (int j0 = 0; j0 < kPer; j0 += kBatch) {
+                uint4 u[kBatch];
+                float w[kBatch];
+#pragma unroll
+                for (int j = 0; j < kBatch; ++j) {
+                    const int i = ctid + (j0 + j) * kWalkConv * 32;
+                    if (i < nh * 512) {
+                        u[j] = sx[i];
+                        w[j] = sw[(i >> 9) * kWRow + ((i >> 3) & 63)];
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < kBatch; ++j) {
+                    const int i = ctid + (j0 + j) * kWalkConv * 32;
+                    if (i < nh * 512) {
+                        uint4 v = u[j];
+                        v.x = pack_f16x2(bf16lo(v.x) * w[j], bf16hi(v.x) * w[j]);
+                        v.y = pack_f16x2(bf16lo(v.y) * w[j], bf16hi(v.y) * w[j]);
+                        v.z = pack_f16x2(bf16lo(v.z) * w[j], bf16hi(v.z) * w[j]);
+                        v.w = pack_f16x2(bf16lo(v.w) * w[j], bf16hi(v.w) * w[j]);
+                        sx[i] = v;
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&conv[st]);
+        }
     } else {
-        // ---------------------------------------------------------------- workers
-        // carried state: thread owns column n and rows p = 32 half + pp, for each head
+        // ---------------------------------------------------------------- state warps
+        // carried state: thread owns column n and rows p = 32 half + pp, for each head; the
+        // update of block c runs as soon as its accumulator is complete, while the converter
+        // warps already form the next stages
         const int n = (warp & 3) * 32 + lane;
         const int half = warp >> 2;
         float Hs[NH][32];
@@ -273,6 +325,13 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
             }
         }
         bool ok = true;
+        // block decay exp(Lam_end) of each head, read from the weights rows a block ahead
+        const size_t wrow = (size_t)nchunks * (Q + 4);
+        const float* wlast = wts + (size_t)(sb * nheads + hlo) * wrow + Q;
+        auto load_e = [&](int c, float (&e)[NH]) {
+#pragma unroll
+            for (int hh = 0; hh < NH; ++hh) e[hh] = hh < nh ? wlast[hh * wrow + (size_t)(blk0 + c) * (Q + 4)] : 0.f;
+        };
 
         // bf16 image of the carried state as the start state of chunk cc.  The image is the
         // MN-major operand tile with 64-byte swizzle: two p-halves of [128 n][32 p], row n of
@@ -304,87 +363,41 @@ chunk_state_walk_kernel(const __grid_constant__ WalkMaps maps, const float* __re
                 bulk_commit_group();
             }
         };
-        // H <- exp(Lam_end) H + S_cc: the start state of chunk cc + 1
-        auto update = [&](int cc, const float (&e)[NH]) {
-            if (ok) ok = mbar_wait(&accb[cc & 1], (cc >> 1) & 1, err);
+
+        if (nblk > 0) write_images(0);
+        float e_next[NH];
+        griddep_wait();                                  // the weights rows come from the cumsum kernel
+        if (nblk > 0) load_e(0, e_next);
+        for (int c = 0; c < nblk && ok; ++c) {
+            float e[NH];
+#pragma unroll
+            for (int hh = 0; hh < NH; ++hh) e[hh] = e_next[hh];
+            if (c + 1 < nblk) load_e(c + 1, e_next);
+            // H <- exp(Lam_end) H + S_c: the start state of block c + 1
+            ok = mbar_wait(&accb[c & 1], (c >> 1) & 1, err);
+            if (!ok) break;
             tc_fence_after();
-            const uint32_t acc = tmem + (cc & 1) * L::kAccStride + ((uint32_t)((warp & 3) * 32) << 16) + half * 32;
+            const uint32_t acc = tmem + (c & 1) * L::kAccStride + ((uint32_t)((warp & 3) * 32) << 16) + half * 32;
 #pragma unroll
             for (int hh = 0; hh < NH; ++hh) {
                 if (hh < nh) {                           // uniform across the CTA
-                    uint32_t v[32];
-                    tmem_ld16(acc + hh * 64, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-                    tmem_ld16(acc + hh * 64 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-                    tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        Hs[hh][j] = fmaf(e[hh], Hs[hh][j], ok ? __uint_as_float(v[j]) : 0.f);
+                    for (int q16 = 0; q16 < 2; ++q16) {
+                        uint32_t v[16];
+                        tmem_ld16(acc + hh * 64 + 16 * q16, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            Hs[hh][16 * q16 + j] = fmaf(e[hh], Hs[hh][16 * q16 + j], __uint_as_float(v[j]));
+                    }
                 }
             }
+            // the accumulator may take block c + 2
             tc_fence_before();
-            if (cc + 1 < nblk) write_images(cc + 1);
-        };
-
-        if (nblk > 0) write_images(0);
-        float e_prev[NH];                                // decay of the chunk before the current one
-#pragma unroll
-        for (int hh = 0; hh < NH; ++hh) e_prev[hh] = 0.f;
-        for (int k = 0; k < total; ++k) {
-            const int st = k % S, c = k / NQ, qq = k - c * NQ;
-            if (ok) ok = mbar_wait(&full[st], (k / S) & 1, err);
-            float e_cur[NH];
-#pragma unroll
-            for (int hh = 0; hh < NH; ++hh) e_cur[hh] = 0.f;
-            if (ok) {
-                // X~ = w o X -> fp16 in place; consecutive threads take consecutive
-                // 16-byte chunks; chunk i: head i / 512, row (i / 8) % 64
-                uint4* sx = reinterpret_cast<uint4*>(stage(st) + L::kStageX);
-                const float* sw = reinterpret_cast<const float*>(stage(st) + L::kStageW);
-                if (qq == NQ - 1) {
-#pragma unroll
-                    for (int hh = 0; hh < NH; ++hh) e_cur[hh] = sw[hh * kWRow + 64];
-                }
-                constexpr int kPer = NH * 512 / (kWalkWorkers * 32);   // chunks per thread
-                constexpr int kBatch = kPer % 3 == 0 ? 3 : kPer;                // loads in flight
-                static_assert(kPer % kBatch == 0, "conversion batches");
-#pragma unroll
-                for (int j0 = 0; j0 < kPer; j0 += kBatch) {
-                    uint4 u[kBatch];
-                    float w[kBatch];
-#pragma unroll
-                    for (int j = 0; j < kBatch; ++j) {
-                        const int i = tid + (j0 + j) * kWalkWorkers * 32;
-                        if (i < nh * 512) {
-                            u[j] = sx[i];
-                            w[j] = sw[(i >> 9) * kWRow + ((i >> 3) & 63)];
-                        }
-                    }
-#pragma unroll
-                    for (int j = 0; j < kBatch; ++j) {
-                        const int i = tid + (j0 + j) * kWalkWorkers * 32;
-                        if (i < nh * 512) {
-                            uint4 v = u[j];
-                            v.x = pack_f16x2(bf16lo(v.x) * w[j], bf16hi(v.x) * w[j]);
-                            v.y = pack_f16x2(bf16lo(v.y) * w[j], bf16hi(v.y) * w[j]);
-                            v.z = pack_f16x2(bf16lo(v.z) * w[j], bf16hi(v.z) * w[j]);
-                            v.w = pack_f16x2(bf16lo(v.w) * w[j], bf16hi(v.w) * w[j]);
-                            sx[i] = v;
-                        }
-                    }
-                }
-            }
-            fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&conv[st]);
-            if (qq == NQ - 1) {
-                // the previous chunk's accumulator is complete by now (its MMAs were issued a
-                // chunk ago); its decay was read with that chunk's last stage
-                if (c > 0) update(c - 1, e_prev);
-#pragma unroll
-                for (int hh = 0; hh < NH; ++hh) e_prev[hh] = e_cur[hh];
-            }
+            if (lane == 0) mbar_arrive(&accfree[c & 1]);
+            if (c + 1 < nblk) write_images(c + 1);
         }
-        if (nblk > 0) update(nblk - 1, e_prev);
         if (lane == 0) bulk_wait_group0();
 #pragma unroll
         for (int hh = 0; hh < NH; ++hh) {
@@ -878,7 +891,8 @@ cudaError_t walk_t(const Dims& d, const WalkMaps& maps, const TcWorkspace& w, co
     if (e != cudaSuccess) return e;
     const int cpg = walk_ctas_per_group(d, NH);
     const unsigned grid = (unsigned)((d.nseq ? d.nseq : d.batch) * d.ngroups * cpg);
-    return launch_dependent(k, dim3(grid), dim3(kWalkThreads), WalkCfg<NH>::kBytes, s, maps, w.fac,
+    return launch_dependent(k, dim3(grid), dim3(kWalkThreads), WalkCfg<NH>::kBytes, s, maps,
+                            static_cast<const float*>(w.wts),
                             init_state, final_state, w.himg, d.nheads, d.ngroups, d.nchunks, cpg,
                             device_error_word(), d.cu_seqlens, d.vl_first);
 }
