@@ -27,8 +27,8 @@
 //   warps 2-3   X~ = w o X (fp16) into a two-deep ring
 //   warps 4-11  P from G_k (read from global memory a block ahead) and the decay factors
 //   warps 12-15 the epilogue y = Yd + exp(Lam_t) Yo + D x, each warp TMA-storing its 32 rows
-//   warps 16-19 the states: per block, C_k from shared memory into TMEM; per item, the bf16
-//               image of H for Yo, then H <- exp(Lam_end) H in TMEM, onto which S accumulates
+//   warps 16-19 the states: per item, the bf16 image of H for Yo, then H <- exp(Lam_end) H in
+//               TMEM, onto which S accumulates
 // Every wait is bounded; expiry records SSD_ERR_TIMEOUT in the device error word and the
 // CTA drains without further waiting.
 #include <cuda.h>
@@ -156,7 +156,7 @@ constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpConv = 2, kWarpP0 = 4, kWarpE0 =
 constexpr int kConvThreads = 64, kPThreads = 256;
 
 // TMEM columns: the heads' states, the two P buffers (bf16 pairs), Yo, Yd, C_k (bf16 pairs)
-constexpr uint32_t kColH = 0, kColP = 192, kColYo = 320, kColYd = 384, kColC = 448;
+constexpr uint32_t kColH = 0, kColP = 192, kColYo = 320, kColYd = 448;   // Yo: two buffers
 
 struct ChainSmem {
     static constexpr int kXSlots = 4;
@@ -181,12 +181,12 @@ static_assert(ChainSmem::kSlotBytes % 1024 == 0, "slots keep 1024-byte alignment
 static_assert(ChainSmem::kBytes <= 227 * 1024, "chain shared memory");
 
 enum {
-    CB_CSTAGED = 0, CB_CSTEMPTY, CB_CREADY,
+    CB_CSTAGED = 0, CB_CFREE,
     CB_BFULL, CB_BEMPTY = CB_BFULL + 2,
     CB_XFULL = CB_BEMPTY + 2, CB_XEMPTY = CB_XFULL + ChainSmem::kXSlots,
     CB_CONV = CB_XEMPTY + ChainSmem::kXSlots, CB_XTEMPTY = CB_CONV + 2,
     CB_UPD = CB_XTEMPTY + 2, CB_SDONE,
-    CB_YOFULL = CB_SDONE + kMaxHeads, CB_YOEMPTY, CB_YDFULL, CB_YDPRIMED,
+    CB_YOFULL = CB_SDONE + kMaxHeads, CB_YOEMPTY = CB_YOFULL + 2, CB_YDFULL = CB_YOEMPTY + 2, CB_YDPRIMED,
     CB_PFULL, CB_PEMPTY = CB_PFULL + 2, CB_COUNT = CB_PEMPTY + 2
 };
 static_assert(CB_COUNT <= ChainSmem::kNumBars, "chain barriers");
@@ -291,8 +291,7 @@ chain_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
 
     if (tid == 0) {
         mbar_init(&bars[CB_CSTAGED], 1);
-        mbar_init(&bars[CB_CSTEMPTY], 4);
-        mbar_init(&bars[CB_CREADY], 4);
+        mbar_init(&bars[CB_CFREE], 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars[CB_BFULL + i], 1);
             mbar_init(&bars[CB_BEMPTY + i], 1);
@@ -307,8 +306,10 @@ chain_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
         }
         mbar_init(&bars[CB_UPD], 4);
         for (int i = 0; i < kMaxHeads; ++i) mbar_init(&bars[CB_SDONE + i], 1);
-        mbar_init(&bars[CB_YOFULL], 1);
-        mbar_init(&bars[CB_YOEMPTY], 4);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars[CB_YOFULL + i], 1);
+            mbar_init(&bars[CB_YOEMPTY + i], 4);
+        }
         mbar_init(&bars[CB_YDFULL], 1);
         mbar_init(&bars[CB_YDPRIMED], 4);
         *abort_flag = 0;
@@ -355,7 +356,8 @@ chain_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             griddep_wait();                              // the fp16 copy of B comes from an earlier kernel
             int kc = 0, kb = 0;
             for (int k = 0; k < nblk; ++k) {
-                if (k >= 1 && !mbar_wait_or_abort(&bars[CB_CSTEMPTY], (k - 1) & 1, err, abort_flag)) break;
+                // every Yo of block k - 1 has read the staged C
+                if (k >= 1 && !mbar_wait_or_abort(&bars[CB_CFREE], (k - 1) & 1, err, abort_flag)) break;
                 mbar_expect_tx(&bars[CB_CSTAGED], 2 * kBox);
                 tma_load_3d(sm + L::kCst, &tm_c, g * kN, k * kBlk, b, &bars[CB_CSTAGED]);
                 tma_load_3d(sm + L::kCst + kBox, &tm_c, g * kN + 64, k * kBlk, b, &bars[CB_CSTAGED]);
@@ -376,7 +378,7 @@ chain_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             // ------------------------------------------------ MMA issue, two polled streams
             constexpr uint32_t idO = idesc_bf16_f32(128, 64, false, true);   // A in TMEM, B MN-major
             constexpr uint32_t idS = idesc_f16_f32(128, 64, true, true);     // A = B_k^T, B = X~: fp16, MN-major
-            const uint32_t aImg = smem_u32(sm + L::kImg);
+            const uint32_t aImg = smem_u32(sm + L::kImg), aC = smem_u32(sm + L::kCst);
             int ia = 0, ib = 0;
             uint32_t idle = 0;
             while (ib < total) {
@@ -386,15 +388,19 @@ chain_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                     const int k = ia / nh, j = ia - k * nh;
                     if (mbar_test_wait(&bars[CB_UPD], ia & 1) &&
                         mbar_test_wait(&bars[CB_CONV + (ia & 1)], (ia >> 1) & 1) &&
-                        (ia == 0 || mbar_test_wait(&bars[CB_YOEMPTY], (ia - 1) & 1)) &&
-                        (j != 0 || (mbar_test_wait(&bars[CB_CREADY], k & 1) &&
+                        (ia < 2 || mbar_test_wait(&bars[CB_YOEMPTY + (ia & 1)], ((ia >> 1) - 1) & 1)) &&
+                        (j != 0 || (mbar_test_wait(&bars[CB_CSTAGED], k & 1) &&
                                     mbar_test_wait(&bars[CB_BFULL + (k & 1)], (k >> 1) & 1)))) {
                         tc_fence_after();
+                        // Yo into buffer ia mod 2: A = C_k (shared memory, K-major over n)
 #pragma unroll 1
-                        for (int ks = 0; ks < 8; ++ks)
-                            umma_f16_ts(tmem + kColYo, tmem + kColC + ks * 8,
-                                        smem_desc_sw64(aImg + ks * 1024, 8192, 512), idO, ks > 0 ? 1u : 0u);
-                        umma_commit(&bars[CB_YOFULL]);
+                        for (int ks = 0; ks < 8; ++ks) {
+                            const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
+                            umma_f16(tmem + kColYo + 64 * (ia & 1), smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
+                                     smem_desc_sw64(aImg + ks * 1024, 8192, 512), idO, ks > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&bars[CB_YOFULL + (ia & 1)]);
+                        if (j == nh - 1) umma_commit(&bars[CB_CFREE]);
                         const uint32_t aB = smem_u32(sm + L::kB0 + (k & 1) * 2 * kBox);
                         const uint32_t aXt = smem_u32(sm + L::kXt0 + (ia & 1) * kBox);
 #pragma unroll 1
@@ -537,7 +543,7 @@ chain_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             const int k = i / nh, j = i - k * nh;
             // exp(Lam_t) Yo + D x into the Yd accumulator, onto which the MMA then adds P X
             // (no partial result waits in registers); frees Yo
-            if (!wait_warp(CB_YOFULL, i & 1)) break;
+            if (!wait_warp(CB_YOFULL + (i & 1), (i >> 1) & 1)) break;
             tc_fence_after();
             uint8_t* sl = slot(i);
             const float u = expf(reinterpret_cast<const float*>(sl + L::kLo)[r]);
@@ -546,7 +552,7 @@ chain_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
                 uint32_t v[32];
-                tmem_ld32(tl + kColYo + 32 * half, v);
+                tmem_ld32(tl + kColYo + 64 * (i & 1) + 32 * half, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
@@ -567,7 +573,7 @@ chain_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&bars[CB_YOEMPTY]);
+                mbar_arrive(&bars[CB_YOEMPTY + (i & 1)]);
                 mbar_arrive(&bars[CB_YDPRIMED]);
             }
             // y = the finished accumulator -> bf16, written over the item's x rows
@@ -624,37 +630,8 @@ chain_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
         bool live = true;
         for (int i = 0; i < total && live; ++i) {
             const int k = i / nh, j = i - k * nh;
-            // the image buffer and, at a block start, TMEM C are free once Yo of item i - 1 is done
-            if (i > 0 && !wait_warp(CB_YOFULL, (i - 1) & 1)) { live = false; break; }
-            if (j == 0) {
-                // C_k from the staging tile (row n: two 128-byte halves, 16-byte chunks swizzled
-                // by n mod 8) into TMEM as bf16 pairs (column c holds C[n][2c], C[n][2c + 1]), the
-                // A operand of Yo
-                if (!wait_warp(CB_CSTAGED, k & 1)) { live = false; break; }
-                const uint8_t* row = sm + L::kCst + n * 128;
-#pragma unroll 1
-                for (int m = 0; m < 4; ++m) {
-                    const uint8_t* hb = row + (m >> 1) * kBox;
-                    uint32_t v[16];
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        const int qn = (m & 1) * 4 + cc;
-                        const uint4 u = *reinterpret_cast<const uint4*>(hb + ((qn ^ (n & 7)) << 4));
-                        v[4 * cc] = u.x;
-                        v[4 * cc + 1] = u.y;
-                        v[4 * cc + 2] = u.z;
-                        v[4 * cc + 3] = u.w;
-                    }
-                    tmem_st16(tl + kColC + 16 * m, v);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&bars[CB_CSTEMPTY]);
-                    mbar_arrive(&bars[CB_CREADY]);
-                }
-            }
+            // the image buffer is free once Yo of item i - 1 is done
+            if (i > 0 && !wait_warp(CB_YOFULL + ((i - 1) & 1), ((i - 1) >> 1) & 1)) { live = false; break; }
             // the bf16 image of H_k (operand of Yo), then H <- exp(Lam_end) H, onto which S
             // accumulates.  Image row n holds p in two 64-byte halves, 16-byte chunk jj of a
             // half stored at jj ^ ((n / 2) mod 4) (the 64-byte swizzle of the MN-major operand).
