@@ -655,7 +655,7 @@ def ours(args, rank, world):
     clocks = ClockSampler(gpu_id)
     line = {"metric": "", "value": None, "unit": "", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "data": "synthetic (seeded; see DESIGN.md input recipe)"}
+            "vs_baseline": None, "data": "synthetic (seeded generators, state_space_model_05_b200/inputs.py)"}
     if w["kind"] == "prefill":
         res = run_prefill(w, args.steps, args.warmup, rank, world, args.workload)
         flops = prefill_flops(w)["total"]
