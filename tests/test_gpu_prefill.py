@@ -257,3 +257,38 @@ def test_dt_softplus_folded_in(bf16, shape, Q, seed, tc_path):
     else:
         assert_fp32(y, oracle.units_to_bthp(yo, b, H), what + " y")
         assert_fp32(st, so.reshape(st.shape), what + " state")
+
+
+def _strong_decay(inp, seed, scale=1.0):
+    """Heads spanning the decay range: A = -16 with dt in [0.5, 1] scale (at scale 1 the state
+    forgets within a few tokens and a 32-token sub-block of P spans e^-250 and more), A = -0.5
+    with dt = 1e-3 (almost no decay), and bursts of dt = 2 scale among dt = 0.01 on A = -16."""
+    rng = np.random.default_rng(seed)
+    b, T, H, P = inp.x.shape
+    A = np.array([-16.0, -0.5, -16.0, -4.0][:H] + [-1.0] * max(0, H - 4), dtype=np.float32)
+    dt = np.empty((b, T, H), dtype=np.float32)
+    dt[..., 0] = rng.uniform(0.5, 1.0, (b, T)) * scale
+    dt[..., 1] = 1e-3
+    dt[..., 2] = np.where(rng.random((b, T)) < 0.1, 2.0 * scale, 0.01)
+    if H > 3:
+        dt[..., 3:] = rng.uniform(0.05, 0.3, (b, T, H - 3))
+    inp.A, inp.dt = A, dt
+    return inp
+
+
+def test_bf16_strong_decay(tc_path):
+    """Decay far past the e^40 guard inside 32-token sub-blocks (the per-element path of P),
+    block decays that underflow to zero, and w o x underflowing in fp16."""
+    inp = _strong_decay(problem(gen.SSDShape(2, 700, 4, 64, 1, 128), bf16=True, seed=46), 47)
+    init = (np.random.default_rng(48).standard_normal((2, 4, 64, 128)) * 0.05).astype(np.float32)
+    _check_bf16(inp, 256, init=init)
+
+
+def test_fp32_strong_decay():
+    """The same heads with dt capped at the workloads' largest value, 0.1 (decay up to 1.6
+    per token on A = -16).  With dt 20 times larger the within-chunk decay sums reach about
+    -2000, where an fp32 ulp (1.2e-4) becomes the relative error of exp(Lam_t - Lam_s): the fp32
+    path then measures 1.4e-4 relative on large elements (the bf16 paths, above, stay within
+    their bound at that size)."""
+    inp = _strong_decay(problem(gen.SSDShape(2, 300, 4, 64, 1, 64), bf16=False, seed=49), 50, scale=0.1)
+    _check_fp32(inp, 64)
