@@ -79,6 +79,28 @@ def test_fp32_decode_shapes(b, H, P, G, N):
     assert_fp32(state.cpu().numpy().reshape(b * H, P, N), so, "state")
 
 
+def test_fp32_decode_strong_decay():
+    """Per-step decays from exp(-32) (the state almost fully replaced) to exp(-1.6e-5) (barely
+    touched), next to each other in one call."""
+    from state_space_model_05_b200 import ssd_decode_step
+    b, H, P, N = 2, 4, 64, 128
+    s = gen.SSDShape(b, 1, H, P, 1, N)
+    rng = np.random.default_rng(77)
+    st0 = rng.standard_normal((b, H, P, N)).astype(np.float32)
+    inp = problem(s, bf16=False, seed=78)
+    A = np.array([-16.0, -16.0, -0.5, -4.0], dtype=np.float32)
+    dec = gen.decode_inputs(s, steps=4, seed=79)
+    dec.dt[:] = np.array([2.0, 0.1, 3e-5, 0.05], dtype=np.float32)
+    state = to_dev(st0)
+    so = st0.reshape(b * H, P, N).astype(np.float64)
+    for k in range(4):
+        x, dt, B, C = _decode_dev(dec, k)
+        y = ssd_decode_step(state, x, dt, to_dev(A), B, C, to_dev(inp.D))
+        yo = oracle.decode_step(so, dec.x[k], dec.dt[k], A, dec.B[k], dec.C[k], inp.D)
+        assert_fp32(y.cpu().numpy().reshape(b * H, P), yo, f"y step {k}")
+    assert_fp32(state.cpu().numpy().reshape(b * H, P, N), so, "state")
+
+
 def test_bf16_decode_io():
     from state_space_model_05_b200 import ssd_decode_step
     s = gen.SSDShape(4, 1, 8, 64, 1, 128)
