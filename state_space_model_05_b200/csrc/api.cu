@@ -116,7 +116,7 @@ cudaError_t profiled(int stage, cudaStream_t s, F&& launch)
 size_t prefill_workspace_layout(const Dims& d, void* base, PrefillWorkspace* ws)
 {
     const size_t units = (size_t)d.batch * d.nheads * d.nchunks;
-    const size_t lam_bytes = align_up(units * d.chunk_len * sizeof(float));
+    const size_t lam_bytes = align_up(units * 2 * d.chunk_len * sizeof(float));   // hi and lo parts
     const size_t st_bytes = align_up(units * d.headdim * d.dstate * sizeof(float));
     if (ws) {
         char* p = static_cast<char*>(base);

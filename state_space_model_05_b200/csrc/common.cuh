@@ -82,7 +82,8 @@ __device__ __forceinline__ float dt_value(float in, const float* dt_bias, int dt
 
 // Workspace layout of the CUDA-core chunked prefill (offsets from the workspace base).
 struct PrefillWorkspace {
-    float* lam;      // [batch][nheads][nchunks][chunk_len]   inclusive cumsum of dt*A
+    float* lam;      // [batch][nheads][nchunks][2][chunk_len] inclusive cumsum of dt*A, summed
+                     //   in double and kept as two floats (hi = fl(Lam), lo = fl(Lam - hi))
     float* states;   // [batch][nheads][nchunks][headdim][dstate]
 };
 size_t prefill_workspace_layout(const Dims& d, void* base, PrefillWorkspace* ws);
@@ -105,7 +106,8 @@ cudaError_t launch_decode(const Dims& d, ssd_dtype_t dtype, float* state, const 
                           const float* D, void* y, cudaStream_t s);
 
 // Lambda (within-chunk cumulative sum of dt A) for every (b, h, chunk) row of `fac`:
-// [b][h][c][Q], or with `extras` [b][h][c][4][Q] holding Lambda, dt and the two column
+// [b][h][c][2][Q] (Lambda summed in double, as hi and lo floats), or with `extras`
+// [b][h][c][4][Q] holding Lambda (fp32), dt and the two column
 // factors per 32-token sub-block (exp(Lam_last - Lam_s) dt_s, exp(Lam_first - Lam_s) dt_s;
 // Q a multiple of 32).  Optionally the chunk-state weights exp(Lam_end - Lam_s) dt_s followed
 // by exp(Lam_end) and three zeros ([b][h][c][Q + 4]), and an fp16 copy of a bf16 B.  Null

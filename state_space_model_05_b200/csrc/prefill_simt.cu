@@ -113,6 +113,32 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
     }
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (!extras && warp < nh) {
+        // CUDA-core path: Lambda summed in double and stored as two floats, hi = fl(Lambda) and
+        // lo = fl(Lambda - hi), so that exp(Lam_t - Lam_s) stays exact to fp32 even where
+        // |Lambda| is in the thousands (strong decay): [Q] hi, then [Q] lo
+        const int hh = warp;
+        const double Ah = A[h0 + hh];
+        double carry = 0.0;
+        float* f = fac + (((size_t)b * nheads + h0 + hh) * nchunks + c) * fac_stride;
+        for (int j = 0; j * 32 < Q; ++j) {
+            const int t = j * 32 + lane;
+            double v = (t < Q) ? (double)sm_dt[t * kCumsumHeads + hh] * Ah : 0.0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const double u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
+            }
+            v += carry;
+            if (t < Q) {
+                const float hi = (float)v;
+                f[t] = hi;
+                f[Q + t] = (float)(v - (double)hi);
+            }
+            carry = __shfl_sync(0xffffffffu, v, 31);
+        }
+        return;
+    }
     if (warp < nh) {
         const int hh = warp;
         const float Ah = A[h0 + hh];
@@ -191,8 +217,9 @@ chunk_state_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
         b = 0;
     }
     const int g = h / (nheads / ngroups);
-    const float* lamc = lam + (((size_t)b * nheads + h) * nchunks + c) * Q;
-    const float lam_end = lamc[Q - 1];
+    const float* lamc = lam + (((size_t)b * nheads + h) * nchunks + c) * 2 * Q;   // hi, then lo
+    const float* lamlo = lamc + Q;
+    const float lam_end = lamc[Q - 1], lam_end_lo = lamlo[Q - 1];
 
     const int nq = dstate >> 2;
     const int rpp = kThreads / nq;                     // rows per pass
@@ -217,7 +244,7 @@ chunk_state_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
             }
             if (threadIdx.x < kTokTile) {
                 const int s = threadIdx.x;
-                sw[s] = s < ns ? expf(lam_end - lamc[s0 + s]) *
+                sw[s] = s < ns ? expf((lam_end - lamc[s0 + s]) + (lam_end_lo - lamlo[s0 + s])) *
                                      dt_value(dt[((size_t)b * seqlen + t0 + s0 + s) * nheads + h], dt_bias, dt_softplus, h)
                                : 0.f;
             }
@@ -274,14 +301,14 @@ state_scan_kernel(const float* __restrict__ lam, float* __restrict__ states,
     }
     float4 hs = make_float4(0.f, 0.f, 0.f, 0.f);
     if (init_state) hs = *reinterpret_cast<const float4*>(init_state + (size_t)bh * PN + e);
-    const float* lamr = lam + row * Q;
+    const float* lamr = lam + row * 2 * Q;             // per chunk: [Q] hi, then [Q] lo
     float* st = states + row * PN + e;
     float4 nxt = nchunks > 0 ? *reinterpret_cast<const float4*>(st) : hs;
     for (int c = 0; c < nchunks; ++c) {
         const float4 sc = nxt;
         if (c + 1 < nchunks) nxt = *reinterpret_cast<const float4*>(st + (size_t)(c + 1) * PN);
         *reinterpret_cast<float4*>(st + (size_t)c * PN) = hs;
-        const float ec = expf(lamr[(size_t)c * Q + Q - 1]);
+        const float ec = expf(lamr[(size_t)c * 2 * Q + Q - 1]) * expf(lamr[(size_t)c * 2 * Q + 2 * Q - 1]);
         hs.x = fmaf(ec, hs.x, sc.x);
         hs.y = fmaf(ec, hs.y, sc.y);
         hs.z = fmaf(ec, hs.z, sc.z);
@@ -315,6 +342,7 @@ chunk_output_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
     const int ldM = kTokTile + 1;
     float* sLs = sM + kTokTile * ldM;                  // [kTokTile] Lam_s
     float* sDs = sLs + kTokTile;                       // [kTokTile] dt_s
+    float* sLl = sDs + kTokTile;                       // [kTokTile] low part of Lam_s
 
     const int c = blockIdx.x, h = blockIdx.y;
     int b = blockIdx.z, t0 = c * Q, qlen = min(Q, seqlen - c * Q);
@@ -324,7 +352,8 @@ chunk_output_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
         b = 0;
     }
     const int g = h / (nheads / ngroups);
-    const float* lamc = lam + (((size_t)b * nheads + h) * nchunks + c) * Q;
+    const float* lamc = lam + (((size_t)b * nheads + h) * nchunks + c) * 2 * Q;   // hi, then lo
+    const float* lamlo = lamc + Q;
     const float* Hc = states + (((size_t)b * nheads + h) * nchunks + c) * headdim * dstate;
     const float Dh = D[h];
     const size_t tok_stride_x = (size_t)nheads * headdim;
@@ -355,7 +384,7 @@ chunk_output_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
         float acc[16];
         const int nper = (headdim + tpr - 1) / tpr;    // <= 16 for headdim <= 128
         const float lt = (my_t < nt) ? lamc[tt + my_t] : 0.f;
-        const float et = expf(lt);
+        const float et = (my_t < nt) ? expf(lt) * expf(lamlo[tt + my_t]) : expf(lt);
         for (int k = 0; k < nper; ++k) {
             const int p = my_p0 + k * tpr;
             float v = 0.f;
@@ -382,6 +411,7 @@ chunk_output_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
             if (threadIdx.x < kTokTile) {
                 const int s = threadIdx.x;
                 sLs[s] = s < ns ? lamc[ss + s] : 0.f;
+                sLl[s] = s < ns ? lamlo[ss + s] : 0.f;
                 sDs[s] = s < ns ? dt_value(dt[((size_t)b * seqlen + t0 + ss + s) * nheads + h], dt_bias, dt_softplus, h)
                                 : 0.f;
             }
@@ -395,7 +425,7 @@ chunk_output_simt_kernel(const T* __restrict__ x, const float* __restrict__ dt,
                     const float* br = sB + s * ldH;
                     float cb = 0.f;
                     for (int n = 0; n < dstate; ++n) cb = fmaf(cr[n], br[n], cb);
-                    m = cb * expf(lamc[tt + t] - sLs[s]) * sDs[s];
+                    m = cb * expf((lamc[tt + t] - sLs[s]) + (lamlo[tt + t] - sLl[s])) * sDs[s];
                 }
                 sM[t * ldM + s] = m;
             }
@@ -453,7 +483,7 @@ cudaError_t chunk_output_simt_t(const Dims& d, const void* x, const float* dt, c
     const int ldH = d.dstate + 1;
     const size_t smem = sizeof(float) * ((size_t)d.headdim * ldH + 2 * kTokTile * ldH +
                                          kTokTile * d.headdim + kTokTile * (kTokTile + 1) +
-                                         2 * kTokTile);
+                                         3 * kTokTile);
     auto k = chunk_output_simt_kernel<T>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -483,7 +513,7 @@ cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, 
     const size_t smem = sizeof(float) * d.chunk_len * kCumsumHeads;
     dim3 grid(d.nchunks, (d.nheads + kCumsumHeads - 1) / kCumsumHeads, d.batch);
     chunk_cumsum_kernel<<<grid, kThreads, smem, s>>>(
-        dt, A, fac, extras ? 4 * d.chunk_len : d.chunk_len, extras, wts,
+        dt, A, fac, extras ? 4 * d.chunk_len : 2 * d.chunk_len, extras, wts,
         static_cast<const uint4*>(b_bf16), static_cast<uint4*>(b_f16),
         d.ngroups * d.dstate / 8, d.seqlen, d.nheads, d.chunk_len, d.nchunks, d.dt_bias, d.dt_softplus,
         d.cu_seqlens, d.vl_first, d.vl_seq);

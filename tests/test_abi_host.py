@@ -49,8 +49,8 @@ def test_workspace_bytes(lib):
     up = lambda v: (v + 255) // 256 * 256
     b, T, H, P, G, N, Q = 2, 300, 4, 64, 1, 128, 128
     c = 3
-    # CUDA-core path: lam [b][H][c][Q] + states [b][H][c][P][N]
-    lam = b * H * c * Q * 4
+    # CUDA-core path: lam [b][H][c][2][Q] (hi and lo parts) + states [b][H][c][P][N]
+    lam = b * H * c * 2 * Q * 4
     st = b * H * c * P * N * 4
     assert _ws(b, T, H, P, G, N, Q, binding.SSD_F32) == up(lam) + up(st)
     # tensor-core path (bf16, P 64, N 128, Q 128/256), sized by 128-token blocks: per block
@@ -67,7 +67,7 @@ def test_workspace_bytes(lib):
     assert _ws(b, T, H, P, G, N, Q, binding.SSD_BF16) == tc_bytes(T)
     assert _ws(b, T, H, P, G, N, 256, binding.SSD_BF16) == tc_bytes(T)
     # bf16 with other shapes uses the CUDA-core layout
-    assert _ws(b, T, H, P, G, N, 64, binding.SSD_BF16) == up(b * H * 5 * 64 * 4) + up(b * H * 5 * P * N * 4)
+    assert _ws(b, T, H, P, G, N, 64, binding.SSD_BF16) == up(b * H * 5 * 2 * 64 * 4) + up(b * H * 5 * P * N * 4)
     assert _ws(b, 0, H, P, G, N, Q, binding.SSD_F32) == 0
     assert _ws(b, T, H, 63, G, N, Q, binding.SSD_F32) == 0          # headdim not a multiple of 8
     assert _ws(b, T, 3, P, 2, N, Q, binding.SSD_F32) == 0           # nheads % ngroups
@@ -169,7 +169,7 @@ def test_varlen_validation(lib):
     assert ws(nseq, T, H, 64, 1, 128, 256, binding.SSD_BF16) == main + up((nseq + 1) * 4) + up(nb * 4)
     assert ws(nseq, 0, H, 64, 1, 128, 256, binding.SSD_BF16) == 0
     nc = T // 64 + nseq                              # CUDA-core chunks of 64: lam + per-chunk fp32 states
-    simt = up(H * nc * 64 * 4) + up(H * nc * 64 * 128 * 4)
+    simt = up(H * nc * 2 * 64 * 4) + up(H * nc * 64 * 128 * 4)
     assert ws(nseq, T, H, 64, 1, 128, 64, binding.SSD_F32) == simt + up((nseq + 1) * 4) + up(nc * 4)
     f = lib.ssd_prefill_varlen
     args = lambda **kw: [F, F, F, F, F, F, None, kw.get("cu", F), kw.get("nseq", 3), kw.get("T", 1000), 4,

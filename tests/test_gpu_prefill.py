@@ -284,11 +284,10 @@ def test_bf16_strong_decay(tc_path):
     _check_bf16(inp, 256, init=init)
 
 
-def test_fp32_strong_decay():
-    """The same heads with dt capped at the workloads' largest value, 0.1 (decay up to 1.6
-    per token on A = -16).  With dt 20 times larger the within-chunk decay sums reach about
-    -2000, where an fp32 ulp (1.2e-4) becomes the relative error of exp(Lam_t - Lam_s): the fp32
-    path then measures 1.4e-4 relative on large elements (the bf16 paths, above, stay within
-    their bound at that size)."""
-    inp = _strong_decay(problem(gen.SSDShape(2, 300, 4, 64, 1, 64), bf16=False, seed=49), 50, scale=0.1)
+@pytest.mark.parametrize("scale", [1.0, 0.1])
+def test_fp32_strong_decay(scale):
+    """The same heads on the fp32 path, at full strength (within-chunk decay sums near -2000,
+    where a single fp32 ulp is 1.2e-4: the path keeps them as double-float hi/lo pairs) and
+    with dt capped at the workloads' largest value, 0.1."""
+    inp = _strong_decay(problem(gen.SSDShape(2, 300, 4, 64, 1, 64), bf16=False, seed=49), 50, scale=scale)
     _check_fp32(inp, 64)
