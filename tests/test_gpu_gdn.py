@@ -61,6 +61,33 @@ def test_shapes_16_steps(shape):
     assert_fp32(st, ref, f"gdn state {shape}")
 
 
+def test_degenerate_gates():
+    """Per value head, the rule's limiting cases side by side: g = 0 (the old state is wiped and
+    replaced by beta k v^T), g = 1 with beta = 0 (the state passes unchanged and o = S^T q), and
+    beta = 1 (the full delta rule: S^T k becomes v after the step)."""
+    import state_space_model_05_b200 as ssd
+    shape = gen.GDNShape(2, 2, 4, 64, 64)
+    inp = gen.gdn_inputs(shape, 3, seed=21)
+    inp.gate[:] = np.array([0.0, 1.0, 0.9, 0.5], dtype=np.float32)
+    inp.beta[:] = np.array([0.7, 0.0, 1.0, 1.0], dtype=np.float32)
+    state = _dev(inp.state)
+    ref = inp.state.astype(np.float64)
+    for t in range(3):
+        o = ssd.ssd_gdn_decode_step(state, _dev(inp.q[t]), _dev(inp.k[t]), _dev(inp.v[t]), _dev(inp.gate[t]),
+                                    _dev(inp.beta[t]))
+        want = gdn.decode_step(ref, inp.q[t], inp.k[t], inp.v[t], inp.gate[t], inp.beta[t])
+        assert_fp32(o.cpu().numpy(), want, f"gdn degenerate out step {t}")
+    torch.cuda.synchronize()
+    assert ssd.ssd_device_status() == 0
+    assert_fp32(state.cpu().numpy(), ref, "gdn degenerate state")
+    # beta = 1 heads: after the last step S^T k equals v (unit-norm k)
+    st = state.cpu().numpy().astype(np.float64)
+    for bb in range(2):
+        for h in (2, 3):
+            kk = inp.k[2][bb, h // 2].astype(np.float64)
+            np.testing.assert_allclose(st[bb, h].T @ kk, inp.v[2][bb, h], rtol=1e-4, atol=1e-4)
+
+
 def test_bf16_inputs():
     o, w, st, ref = _run(gen.GDNShape(2, 16, 32, 128, 128), 32, bf16=True, seed=9)
     assert_bf16_y(o, w, "gdn out bf16")
