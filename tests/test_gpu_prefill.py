@@ -291,3 +291,14 @@ def test_fp32_strong_decay(scale):
     with dt capped at the workloads' largest value, 0.1."""
     inp = _strong_decay(problem(gen.SSDShape(2, 300, 4, 64, 1, 64), bf16=False, seed=49), 50, scale=scale)
     _check_fp32(inp, 64)
+
+
+@pytest.mark.parametrize("bf16,Q", [(False, 256), (False, 100), (True, 256)])
+def test_max_dims(bf16, Q):
+    """headdim 128 and dstate 256, the largest prefill sizes the ABI takes (the CUDA-core path,
+    whose output kernel then holds a 128 x 257 state tile in shared memory), ragged length."""
+    inp = problem(gen.SSDShape(2, 300, 2, 128, 1, 256), bf16=bf16, seed=51 + Q)
+    if bf16:
+        _check_bf16(inp, Q)
+    else:
+        _check_fp32(inp, Q)
