@@ -20,6 +20,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -118,16 +119,25 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and with runs of whitespace collapsed: what the compiler
+    sees, so that editing a comment does not discard a recorded measurement."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_sha() -> str:
-    """Hash of every kernel source file (csrc and its subfolders), path and contents."""
+    """Hash of every kernel source file (csrc and its subfolders): path and code, comments
+    and layout excluded."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "state_space_model_05_b200", "csrc")
     files = []
     for dirpath, _, names in os.walk(csrc):
         files += [os.path.join(dirpath, n) for n in names if n.endswith((".cu", ".cuh", ".h"))]
     for path in sorted(files):
-        with open(path, "rb") as f:
-            h.update(os.path.relpath(path, csrc).encode() + f.read())
+        with open(path, encoding="utf-8", errors="replace") as f:
+            h.update((os.path.relpath(path, csrc) + "\0" + _code_only(f.read())).encode())
     return h.hexdigest()[:16]
 
 

@@ -11,7 +11,7 @@
 // factorisation.  After the per-block decay cumsum (prefill_simt.cu) come two kernels:
 //
 // chunk_state_walk_kernel -- persistent: one CTA per (batch b, group g, 1-3 heads) walks
-//   the blocks of its heads in order, the carried state held in the worker threads'
+//   the blocks of its heads in order, the carried state held in the state warps'
 //   registers (no cross-CTA hand-off):
 //     S_k = B_k^T (w o X_k),  w_s = exp(Lam_end - Lam_s) dt_s         (tcgen05, fp16 in)
 //     H_{k+1} = exp(Lam_end) H_k + S_k                                 (fp32)
@@ -109,9 +109,9 @@ varlen_table_kernel(const int* __restrict__ cu, int nseq, int total_tokens, int 
 // heads in order, so the carried state never leaves the CTA (registers) and no chunk
 // waits for another CTA.  The heads' chunk states form one tcgen05 chain with the heads
 // stacked along N (N = 64 x heads); B_c is staged once per chunk for all of them.
-// Operands stream through a 4-deep ring of 64-row stages (fp16 B rows, one X box per
-// head, the heads' weights w_s and, with a chunk's last stage, its decay exp(Lam_end));
-// two TMEM accumulators alternate between chunks.  Warp-specialised: one warp issues the
+// Operands stream through a ring of 64-row stages, three deep with one head per CTA and
+// four with up to three (fp16 B rows, one X box per head, the heads' weights w_s); two
+// TMEM accumulators alternate between chunks.  Warp-specialised: one warp issues the
 // loads, one the MMAs, four warps form X~ = w o X, and eight state warps (which hold the
 // carried state) update it as soon as a chunk's accumulator is complete and hand the
 // accumulator back, so that the update overlaps the conversion of the next stages.  Each

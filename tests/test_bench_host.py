@@ -19,6 +19,19 @@ def test_kernel_source_sha_covers_subfolders(tmp_path, monkeypatch):
     assert bench.kernel_source_sha() != h1
 
 
+def test_kernel_source_sha_ignores_comments_not_code(tmp_path, monkeypatch):
+    root = tmp_path / "repo"
+    (root / "state_space_model_05_b200" / "csrc").mkdir(parents=True)
+    src = root / "state_space_model_05_b200" / "csrc" / "k.cu"
+    src.write_text("// old note\nint f() { return 1; }  /* block */\n")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    h1 = bench.kernel_source_sha()
+    src.write_text("// a rewritten note\nint f()   {\n  return 1; }\n")
+    assert bench.kernel_source_sha() == h1
+    src.write_text("int f() { return 2; }\n")
+    assert bench.kernel_source_sha() != h1
+
+
 def test_recorded_traffic_requires_matching_source(tmp_path, monkeypatch):
     root = tmp_path / "repo"
     (root / "state_space_model_05_b200" / "csrc").mkdir(parents=True)
