@@ -6,7 +6,8 @@
 // for Inference", section "2. Metodologia": the recurrence splits into chunks of
 // fixed size; inside a chunk it is a masked matrix product built from a static
 // lower-triangular mask; across chunks only an N x P state per (batch, head) is
-// carried; the decay exponents are formed in fp32.  For chunk c of head h with
+// carried; the decay exponents are formed in fp32 (here from a double-precision cumsum
+// kept as two floats, so that differences stay exact).  For chunk c of head h with
 // Lam_t the inclusive cumsum of dt*A over the chunk's tokens:
 //   (1) Lam_t = sum_{r <= t, r in chunk} dt_r A_h
 //   (2) y_t  = sum_{s <= t} (C_t . B_s) exp(Lam_t - Lam_s) dt_s x_s
@@ -24,7 +25,8 @@ namespace {
 constexpr int kThreads = 256;
 
 // ----------------------------------------------------------------------------------
-// (1) per (b, chunk, head-tile): Lam over the chunk, written [b][h][c][Q].
+// (1) per (b, chunk, head-tile): Lam over the chunk, written [b][h][c][2][Q] (hi, lo) for the
+// CUDA-core path, or as the tensor-core path's decay factors.
 // The chunk's dt block [Q][nheads] is contiguous in memory; it is staged through
 // shared memory so that both the read and the write are coalesced.
 // ----------------------------------------------------------------------------------
@@ -38,7 +40,8 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
     return r;
 }
 
-// Per (b, h, chunk) row of `fac` (stride fac_stride floats): Lam[Q]; with `extras` also
+// Per (b, h, chunk) row of `fac` (stride fac_stride floats): without `extras`, Lam summed in
+// double as hi[Q] and lo[Q] floats; with `extras`, Lam[Q] in fp32 and also
 // dt[Q] (zero past seqlen) and the column factors of each 32-token sub-block,
 // exp(Lam_last - Lam_s) dt_s and exp(Lam_first - Lam_s) dt_s.  With `wts`, the chunk-state
 // weights exp(Lam_end - Lam_s) dt_s ([b][h][c][Q]); with `b_f16`, an fp16 copy of B.
