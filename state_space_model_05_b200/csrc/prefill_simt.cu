@@ -28,9 +28,11 @@ constexpr int kThreads = 256;
 // (1) per (b, chunk, head-tile): Lam over the chunk, written [b][h][c][2][Q] (hi, lo) for the
 // CUDA-core path, or as the tensor-core path's decay factors.
 // The chunk's dt block [Q][nheads] is contiguous in memory; it is staged through
-// shared memory so that both the read and the write are coalesced.
+// shared memory, transposed to [head][Q + 4], so that the global read is coalesced and
+// both shared-memory sides are free of bank conflicts.
 // ----------------------------------------------------------------------------------
 constexpr int kCumsumHeads = 8;      // one warp per head
+constexpr int kFacQ = 128;           // block length of the tensor-core path (decay factors)
 static_assert(kMaxChunk * kCumsumHeads % kThreads == 0, "dt rows per thread");
 
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
@@ -40,12 +42,21 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
     return r;
 }
 
+// exp(ref - Lambda_s) dt_s for four consecutive tokens
+__device__ __forceinline__ float4 decay_times_dt(float ref, float4 lam, float4 dt)
+{
+    return make_float4(expf(ref - lam.x) * dt.x, expf(ref - lam.y) * dt.y, expf(ref - lam.z) * dt.z,
+                       expf(ref - lam.w) * dt.w);
+}
+
 // Per (b, h, chunk) row of `fac` (stride fac_stride floats): without `extras`, Lam summed in
-// double as hi[Q] and lo[Q] floats; with `extras`, Lam[Q] in fp32 and also
+// double as hi[Q] and lo[Q] floats; with `extras` (Q = kFacQ), Lam[Q] in fp32 and also
 // dt[Q] (zero past seqlen) and the column factors of each 32-token sub-block,
 // exp(Lam_last - Lam_s) dt_s and exp(Lam_first - Lam_s) dt_s.  With `wts`, the chunk-state
-// weights exp(Lam_end - Lam_s) dt_s ([b][h][c][Q]); with `b_f16`, an fp16 copy of B.
-__global__ void __launch_bounds__(kThreads)
+// weights exp(Lam_end - Lam_s) dt_s, exp(Lam_end) and three zeros ([b][h][c][Q + 4]); with
+// `b_f16`, an fp16 copy of B.  Six CTAs fit on an SM (at most 42 registers a thread): on long
+// prefills the grid is several waves of short CTAs, each a chain of memory round trips.
+__global__ void __launch_bounds__(kThreads, 6)
 chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
                     float* __restrict__ fac, int fac_stride, bool extras, float* __restrict__ wts,
                     const uint4* __restrict__ b_bf16, uint4* __restrict__ b_f16,
@@ -53,7 +64,7 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
                     const float* __restrict__ dt_bias, int dt_softplus, const int* __restrict__ vl_cu,
                     const int* __restrict__ vl_first, const int* __restrict__ vl_seq)
 {
-    extern __shared__ float sm_dt[];                   // [Q][kCumsumHeads]
+    extern __shared__ float sm_dt[];                   // [kCumsumHeads][Q + 4]
     // the next kernel of the stream (launched as a programmatic dependent) may stage its setup
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int c = blockIdx.x, h0 = blockIdx.y * kCumsumHeads, b = blockIdx.z;
@@ -108,11 +119,13 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
             }
         }
     }
+    const int ldt = Q + 4;
 #pragma unroll
     for (int m = 0; m < kDtPer; ++m) {
         const int i = threadIdx.x + m * kThreads;
+        const int t = i / kCumsumHeads, hh = i - t * kCumsumHeads;
         if (i < Q * kCumsumHeads)
-            sm_dt[i] = use[m] ? dt_value(raw[m], dt_bias, dt_softplus, h0 + (i % kCumsumHeads)) : 0.f;
+            sm_dt[hh * ldt + t] = use[m] ? dt_value(raw[m], dt_bias, dt_softplus, h0 + hh) : 0.f;
     }
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -126,7 +139,7 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
         float* f = fac + (((size_t)b * nheads + h0 + hh) * nchunks + c) * fac_stride;
         for (int j = 0; j * 32 < Q; ++j) {
             const int t = j * 32 + lane;
-            double v = (t < Q) ? (double)sm_dt[t * kCumsumHeads + hh] * Ah : 0.0;
+            double v = (t < Q) ? (double)sm_dt[hh * ldt + t] * Ah : 0.0;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const double u = __shfl_up_sync(0xffffffffu, v, o);
@@ -143,50 +156,38 @@ chunk_cumsum_kernel(const float* __restrict__ dt, const float* __restrict__ A,
         return;
     }
     if (warp < nh) {
+        // tensor-core path (Q = kFacQ): lane l owns tokens 4l .. 4l + 3, so one warp scan covers
+        // the block and each factor row goes out as one 16-byte store per lane
         const int hh = warp;
         const float Ah = A[h0 + hh];
-        float carry = 0.f;
-        const size_t unit = ((size_t)b * nheads + h0 + hh) * nchunks + c;
-        float* f = fac + unit * fac_stride;
-        float lv[kMaxChunk / 32], dv[kMaxChunk / 32];
+        const float4 d = *reinterpret_cast<const float4*>(sm_dt + hh * ldt + 4 * lane);
+        const float v0 = d.x * Ah, v1 = v0 + d.y * Ah, v2 = v1 + d.z * Ah, v3 = v2 + d.w * Ah;
+        float tot = v3;                                  // inclusive scan of the lanes' sums
 #pragma unroll
-        for (int j = 0; j < kMaxChunk / 32; ++j) {
-            const int t = j * 32 + lane;
-            if (j * 32 >= Q) break;
-            const float d = (t < Q) ? sm_dt[t * kCumsumHeads + hh] : 0.f;
-            float v = d * Ah;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float u = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += u;
-            }
-            v += carry;
-            if (extras) {
-                // column factors per 32-token sub-block (one warp pass = one sub-block):
-                // exp(Lam_last - Lam_s) dt_s and exp(Lam_first - Lam_s) dt_s
-                const float vlast = __shfl_sync(0xffffffffu, v, 31), vfirst = __shfl_sync(0xffffffffu, v, 0);
-                if (t < Q) {
-                    f[Q + t] = d;
-                    f[2 * Q + t] = expf(vlast - v) * d;
-                    f[3 * Q + t] = expf(vfirst - v) * d;
-                }
-            }
-            if (t < Q) f[t] = v;
-            lv[j] = v;
-            dv[j] = d;
-            carry = __shfl_sync(0xffffffffu, v, 31);
+        for (int o = 1; o < 32; o <<= 1) {
+            const float u = __shfl_up_sync(0xffffffffu, tot, o);
+            if (lane >= o) tot += u;
         }
+        float pre = __shfl_up_sync(0xffffffffu, tot, 1);
+        if (lane == 0) pre = 0.f;
+        const float4 v = make_float4(pre + v0, pre + v1, pre + v2, pre + v3);
+        // Lambda at the block's last token, and at the last and first token of this lane's
+        // 32-token sub-block (lanes 8j .. 8j + 7 hold sub-block j)
+        const float lam_end = __shfl_sync(0xffffffffu, v.w, 31);
+        const float lam_last = __shfl_sync(0xffffffffu, v.w, lane | 7);
+        const float lam_first = __shfl_sync(0xffffffffu, v.x, lane & ~7);
+        const size_t unit = ((size_t)b * nheads + h0 + hh) * nchunks + c;
+        float4* f = reinterpret_cast<float4*>(fac + unit * fac_stride) + lane;
+        f[0] = v;
+        f[kFacQ / 4] = d;
+        f[kFacQ / 2] = decay_times_dt(lam_last, v, d);
+        f[3 * kFacQ / 4] = decay_times_dt(lam_first, v, d);
         if (wts) {
-            // chunk-state weights w_s = exp(Lambda_end - Lambda_s) dt_s (carry = Lambda_end),
-            // then the chunk's decay exp(Lambda_end) and zero padding: Q + 4 floats per row
-            float* wr = wts + unit * (Q + 4);
-#pragma unroll
-            for (int j = 0; j < kMaxChunk / 32; ++j) {
-                const int t = j * 32 + lane;
-                if (j * 32 >= Q) break;
-                if (t < Q) wr[t] = expf(carry - lv[j]) * dv[j];
-            }
-            if (lane < 4) wr[Q + lane] = lane == 0 ? expf(carry) : 0.f;
+            // chunk-state weights w_s = exp(Lambda_end - Lambda_s) dt_s, then the block's decay
+            // exp(Lambda_end) and zero padding: Q + 4 floats per row
+            float4* wr = reinterpret_cast<float4*>(wts + unit * (kFacQ + 4));
+            wr[lane] = decay_times_dt(lam_end, v, d);
+            if (lane == 0) wr[kFacQ / 4] = make_float4(expf(lam_end), 0.f, 0.f, 0.f);
         }
     }
 }
@@ -513,7 +514,8 @@ cudaError_t launch_chunk_cumsum(const Dims& d, const float* dt, const float* A, 
                                 cudaStream_t s)
 {
     if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
-    const size_t smem = sizeof(float) * d.chunk_len * kCumsumHeads;
+    if (extras && d.chunk_len != kFacQ) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(float) * (d.chunk_len + 4) * kCumsumHeads;
     dim3 grid(d.nchunks, (d.nheads + kCumsumHeads - 1) / kCumsumHeads, d.batch);
     chunk_cumsum_kernel<<<grid, kThreads, smem, s>>>(
         dt, A, fac, extras ? 4 * d.chunk_len : 2 * d.chunk_len, extras, wts,
