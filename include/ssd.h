@@ -66,7 +66,7 @@ typedef enum {
     SSD_ERR_SHAPE = 2,       /* a size is out of range or inconsistent */
     SSD_ERR_DTYPE = 3,       /* unknown dtype */
     SSD_ERR_ALIGN = 4,       /* a pointer is not 16-byte aligned */
-    SSD_ERR_UNSUPPORTED = 5, /* valid, but not a shape this build implements */
+    SSD_ERR_UNSUPPORTED = 5, /* valid, but not a shape this library implements */
     SSD_ERR_CUDA = 6,        /* a CUDA call or launch failed */
     SSD_ERR_TIMEOUT = 7,     /* a device-side bounded wait expired */
     SSD_ERR_WORKSPACE = 8    /* workspace missing or smaller than required */
