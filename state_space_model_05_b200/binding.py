@@ -114,6 +114,32 @@ def _need(t: torch.Tensor, name: str, dtype=None):
         raise TypeError(f"{name} must be {dtype}")
 
 
+def _rank(t: torch.Tensor, name: str, layout: str):
+    """Raise unless ``t`` has one axis per name in ``layout`` (e.g. "[batch][seqlen][nheads]")."""
+    if t.dim() != layout.count("["):
+        raise ValueError(f"{name} must be {layout}, got shape {tuple(t.shape)}")
+
+
+def _check_args(ref: torch.Tensor, specs):
+    """Validate the tensors of one call before anything reaches the library, which sees only
+    pointers and so cannot tell a short buffer from a right one.  ``specs`` holds
+    (tensor or None, name, expected shape, dtype or None); every tensor given must have that
+    shape, live on ``ref``'s device, be a contiguous CUDA tensor and (if stated) have that
+    dtype.  ``ref`` must be on the current device, whose stream the library launches on."""
+    for t, name, shape, _ in specs:
+        if t is not None and tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    for t, name, _, dtype in specs:
+        if t is None:
+            continue
+        _need(t, name, dtype)
+        if t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device}, expected {ref.device}")
+    if ref.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensors are on {ref.device} but the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
+
+
 def ssd_prefill_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len, dtype_code):
     return int(lib().ssd_prefill_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate,
                                                  chunk_len, dtype_code))
@@ -139,25 +165,27 @@ def ssd_prefill(x, dt, A, B, C, D, chunk_len, init_state=None, y=None, final_sta
                 workspace=None, stream=None, dt_softplus=False, dt_bias=None):
     """Chunked SSD prefill.  Shapes as in ``include/ssd.h``; returns ``(y, final_state)``.
     With ``dt_softplus`` the kernels use softplus(dt + dt_bias) (ssd_prefill_dtraw)."""
-    for t, n in ((x, "x"), (B, "B"), (C, "C")):
-        _need(t, n, x.dtype)
-    for t, n in ((dt, "dt"), (A, "A"), (D, "D")):
-        _need(t, n, torch.float32)
-    code = _dtype_code(x)
+    _rank(x, "x", "[batch][seqlen][nheads][headdim]")
+    _rank(B, "B", "[batch][seqlen][ngroups][dstate]")
     batch, seqlen, nheads, headdim = x.shape
     ngroups, dstate = B.shape[2], B.shape[3]
+    f32, state_shape = torch.float32, (batch, nheads, headdim, dstate)
+    _check_args(x, ((x, "x", x.shape, x.dtype), (dt, "dt", (batch, seqlen, nheads), f32),
+                    (A, "A", (nheads,), f32), (B, "B", B.shape, x.dtype),
+                    (C, "C", B.shape, x.dtype), (D, "D", (nheads,), f32),
+                    (init_state, "init_state", state_shape, f32), (y, "y", x.shape, x.dtype),
+                    (final_state, "final_state", state_shape, f32),
+                    (dt_bias if dt_softplus else None, "dt_bias", (nheads,), f32),
+                    (workspace, "workspace", workspace.shape if workspace is not None else (), None)))
+    code = _dtype_code(x)
     if y is None:
         y = torch.empty_like(x)
     if final_state is None:
-        final_state = torch.empty((batch, nheads, headdim, dstate), device=x.device, dtype=torch.float32)
-    if init_state is not None:
-        _need(init_state, "init_state", torch.float32)
+        final_state = torch.empty(state_shape, device=x.device, dtype=f32)
     need = ssd_prefill_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_len, code)
     if workspace is None:
         workspace = torch.empty(max(need, 1), device=x.device, dtype=torch.uint8)
     if dt_softplus:
-        if dt_bias is not None:
-            _need(dt_bias, "dt_bias", torch.float32)
         st = lib().ssd_prefill_dtraw(_ptr(x), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
                                      _ptr(init_state), batch, seqlen, nheads, headdim, ngroups, dstate,
                                      chunk_len, code, _ptr(y), _ptr(final_state), _ptr(workspace),
@@ -177,21 +205,24 @@ def ssd_prefill_varlen(x, dt, A, B, C, D, cu_seqlens, chunk_len, init_states=Non
     """Packed variable-length prefill.  x [T][H][P], dt [T][H], B/C [T][G][N] (the batch-1
     layouts without the batch axis), cu_seqlens a CUDA int32 tensor of nseq + 1 offsets.
     Returns ``(y, final_states)``, final_states [nseq][H][P][N]."""
-    for t, n in ((x, "x"), (B, "B"), (C, "C")):
-        _need(t, n, x.dtype)
-    for t, n in ((dt, "dt"), (A, "A"), (D, "D")):
-        _need(t, n, torch.float32)
-    _need(cu_seqlens, "cu_seqlens", torch.int32)
-    code = _dtype_code(x)
+    _rank(x, "x", "[tokens][nheads][headdim]")
+    _rank(B, "B", "[tokens][ngroups][dstate]")
+    _rank(cu_seqlens, "cu_seqlens", "[nseq + 1]")
     total, nheads, headdim = x.shape
     ngroups, dstate = B.shape[1], B.shape[2]
     nseq = cu_seqlens.numel() - 1
+    f32, state_shape = torch.float32, (nseq, nheads, headdim, dstate)
+    _check_args(x, ((x, "x", x.shape, x.dtype), (dt, "dt", (total, nheads), f32), (A, "A", (nheads,), f32),
+                    (B, "B", B.shape, x.dtype), (C, "C", B.shape, x.dtype), (D, "D", (nheads,), f32),
+                    (cu_seqlens, "cu_seqlens", cu_seqlens.shape, torch.int32),
+                    (init_states, "init_states", state_shape, f32), (y, "y", x.shape, x.dtype),
+                    (final_states, "final_states", state_shape, f32),
+                    (workspace, "workspace", workspace.shape if workspace is not None else (), None)))
+    code = _dtype_code(x)
     if y is None:
         y = torch.empty_like(x)
     if final_states is None:
-        final_states = torch.empty((nseq, nheads, headdim, dstate), device=x.device, dtype=torch.float32)
-    if init_states is not None:
-        _need(init_states, "init_states", torch.float32)
+        final_states = torch.empty(state_shape, device=x.device, dtype=f32)
     need = int(lib().ssd_prefill_varlen_workspace_bytes(nseq, total, nheads, headdim, ngroups, dstate,
                                                         chunk_len, code))
     if workspace is None:
@@ -208,18 +239,19 @@ def ssd_decode_step(state, x_t, dt_t, A, B_t, C_t, D, y_t=None, stream=None, dt_
                     dt_bias=None):
     """One decode step; ``state`` [b][H][P][N] fp32 is updated in place.  Returns ``y_t``.
     With ``dt_softplus`` the kernel uses softplus(dt_t + dt_bias) (ssd_decode_step_dtraw)."""
-    _need(state, "state", torch.float32)
-    for t, n in ((x_t, "x_t"), (B_t, "B_t"), (C_t, "C_t")):
-        _need(t, n, x_t.dtype)
-    for t, n in ((dt_t, "dt_t"), (A, "A"), (D, "D")):
-        _need(t, n, torch.float32)
+    _rank(x_t, "x_t", "[batch][nheads][headdim]")
+    _rank(B_t, "B_t", "[batch][ngroups][dstate]")
     batch, nheads, headdim = x_t.shape
     ngroups, dstate = B_t.shape[1], B_t.shape[2]
+    f32 = torch.float32
+    _check_args(x_t, ((state, "state", (batch, nheads, headdim, dstate), f32), (x_t, "x_t", x_t.shape, x_t.dtype),
+                      (dt_t, "dt_t", (batch, nheads), f32), (A, "A", (nheads,), f32),
+                      (B_t, "B_t", B_t.shape, x_t.dtype), (C_t, "C_t", B_t.shape, x_t.dtype),
+                      (D, "D", (nheads,), f32), (y_t, "y_t", x_t.shape, x_t.dtype),
+                      (dt_bias if dt_softplus else None, "dt_bias", (nheads,), f32)))
     if y_t is None:
         y_t = torch.empty_like(x_t)
     if dt_softplus:
-        if dt_bias is not None:
-            _need(dt_bias, "dt_bias", torch.float32)
         st = lib().ssd_decode_step_dtraw(_ptr(state), _ptr(x_t), _ptr(dt_t), _ptr(dt_bias), _ptr(A), _ptr(B_t),
                                          _ptr(C_t), _ptr(D), batch, nheads, headdim, ngroups, dstate,
                                          _dtype_code(x_t), _ptr(y_t), _stream(stream))
@@ -258,13 +290,15 @@ def ssd_gdn_decode_step(state, q, k, v, gate, beta, out=None, stream=None):
     """One Gated DeltaNet decode step; ``state`` [b][hv][dk][dv] fp32 is updated in place.
     q, k [b][hqk][dk]; v [b][hv][dv] (fp32 or bf16, all alike); gate, beta [b][hv] fp32.
     Returns ``out`` [b][hv][dv]."""
-    _need(state, "state", torch.float32)
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, n, q.dtype)
-    for t, n in ((gate, "gate"), (beta, "beta")):
-        _need(t, n, torch.float32)
+    _rank(q, "q", "[batch][heads_qk][dk]")
+    _rank(v, "v", "[batch][heads_v][dv]")
     batch, hqk, dk = q.shape
     hv, dv = v.shape[1], v.shape[2]
+    f32 = torch.float32
+    _check_args(q, ((state, "state", (batch, hv, dk, dv), f32), (q, "q", q.shape, q.dtype),
+                    (k, "k", q.shape, q.dtype), (v, "v", (batch, hv, dv), q.dtype),
+                    (gate, "gate", (batch, hv), f32), (beta, "beta", (batch, hv), f32),
+                    (out, "out", (batch, hv, dv), q.dtype)))
     if out is None:
         out = torch.empty_like(v)
     st = lib().ssd_gdn_decode_step(_ptr(state), _ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(beta), batch,
