@@ -201,16 +201,26 @@ def test_bf16_init_aliases_final(tc_path):
 
 def test_paths_agree_closely():
     """The fused and two-pass kernels compute the same algorithm in bf16/fp32: their outputs
-    differ only by rounding (well inside the oracle tolerance)."""
+    differ only by rounding (well inside the oracle tolerance).  Each setting runs its own
+    kernels and no others."""
     import state_space_model_05_b200 as ssd
+    from state_space_model_05_b200 import binding
     inp = problem(gen.SSDShape(2, 1000, 8, 64, 2, 128), bf16=True, seed=45)
-    out = {}
+    out, ran = {}, {}
     for path in ("fused", "two_pass"):
         prev = ssd.ssd_set_prefill_path(path)
+        binding.ssd_profile_reset()
+        binding.ssd_profile_enable(True)
         try:
             out[path] = gpu_prefill(inp, 256, bf16=True)
         finally:
+            binding.ssd_profile_enable(False)
             ssd.ssd_set_prefill_path(prev)
+        ran[path] = set(binding.ssd_profile_read())
+        binding.ssd_profile_reset()
+    # the setting really selects the kernels (the library's launch records name them)
+    assert ran["fused"] == {"chunk_cumsum", "block_gram_tc", "chain_prefill_tc"}, ran["fused"]
+    assert ran["two_pass"] == {"chunk_cumsum", "chunk_state_scan_tc", "chunk_output_tc"}, ran["two_pass"]
     (yf, sf), (yt, stt) = out["fused"], out["two_pass"]
     ry = float(np.sqrt(np.mean(yt.astype(np.float64) ** 2)))
     rs = float(np.sqrt(np.mean(stt.astype(np.float64) ** 2)))
