@@ -3,7 +3,8 @@
 The mistakes are planted in a temporary copy of the oracle's C source, compiled
 on the CPU; the committed oracle is untouched.  Every mutant must fail at least
 one of the pins below (hand-worked case, separately written chunked form,
-prefill/decode resume, group mapping).
+prefill/decode resume, group mapping).  Ten mutants change the recurrence wherever
+it is written; six more change the decode step alone, with the prefill correct.
 """
 import json
 import math
@@ -35,12 +36,29 @@ MUTANTS = {
     "init_ignored": (r"if \(init\)", "if (0)"),
     "decay_squared": (r"Hp\[n\] = a \* Hp\[n\]", "Hp[n] = a * a * Hp[n]"),
 }
+# the same kinds of mistake planted in the decode step alone (the prefill left correct): the
+# resume pin, prefill(T0) followed by decode steps against prefill(T), must catch each
+DECODE_MUTANTS = {
+    "decode_no_decay": MUTANTS["no_decay"],
+    "decode_exp_sign": MUTANTS["exp_sign"],
+    "decode_y_before_update": MUTANTS["y_before_update"],
+    "decode_no_skip": MUTANTS["no_skip"],
+    "decode_group_modulo": MUTANTS["group_modulo"],
+    "decode_B_ignores_batch": (r"B_t \+ \(\(size_t\)b \* ngroups \+ g\) \* dstate", "B_t + (size_t)g * dstate"),
+}
+DECODE_ENTRY = "int ssd_oracle_decode_step("
 
 
 def _build_mutant(tmp_path, name):
-    pat, rep = MUTANTS[name]
     src = open(SRC).read()
-    mutated, n = re.subn(pat, rep, src)
+    if name in DECODE_MUTANTS:
+        pat, rep = DECODE_MUTANTS[name]
+        cut = src.index(DECODE_ENTRY)
+        tail, n = re.subn(pat, rep, src[cut:])
+        mutated = src[:cut] + tail
+    else:
+        pat, rep = MUTANTS[name]
+        mutated, n = re.subn(pat, rep, src)
     assert n >= 1, f"mutation {name} did not apply"
     c = tmp_path / f"{name}.c"
     so = tmp_path / f"lib_{name}.so"
@@ -97,7 +115,7 @@ def test_unmutated_copy_passes(tmp_path):
     assert _pins_pass(oracle.bind(str(so)))
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
+@pytest.mark.parametrize("name", sorted(MUTANTS) + sorted(DECODE_MUTANTS))
 def test_mutant_is_caught(tmp_path, name):
     lib = _build_mutant(tmp_path, name)
     assert not _pins_pass(lib), f"planted mistake '{name}' passed every pin"
