@@ -1,5 +1,6 @@
 """Host-side pieces of bench.py that need no GPU: workload accounting, the kernel-source
-hash that keys recorded ncu traffic, and the shape of the roofline record."""
+hash that keys recorded ncu traffic, the shape of the roofline record, and the reference
+arm (the oracle timed on the host)."""
 import os
 
 import bench
@@ -72,3 +73,40 @@ def test_roofline_prefill_record():
     assert abs(r["achieved"] - expect) < 1e-6 * expect
     assert abs(r["frac"] - r["achieved"] / 6545.3) < 1e-12
     assert set(r) >= {"bound", "achieved", "peak", "unit", "frac", "traffic"}
+
+
+def test_reference_arm_line(monkeypatch, capsys):
+    """`bench.py --impl reference`: the oracle timed on the host, one JSON line with the
+    contract's keys, on rank 0 only."""
+    import json
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    # the oracle's per-step sample is sized from this budget: keep the test to seconds
+    monkeypatch.setattr(bench, "oracle_sample_step", _fast_sample(bench.oracle_sample_step))
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["metric"] == "SSD prefill tokens/s"
+    assert line["value"] > 0 and line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["steps"] == 1 and line["warmup"] == 3 and line["config"]["workload"] == "prefill_130m"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_do_nothing(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setattr(bench, "oracle_sample_step", lambda *a: (_ for _ in ()).throw(AssertionError("ran")))
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"]) == 0
+    assert capsys.readouterr().out == ""
+
+
+def _fast_sample(step):
+    """The real oracle step on at most two (batch, head) units."""
+    def run(w, inp, units):
+        return step(w, inp, list(units)[:2])
+    return run
