@@ -21,7 +21,13 @@
 // device address; its device address is looked up once per device with
 // cudaGetSymbolAddress (with that device current) on the first call made while that
 // device is current.  That first call should therefore happen before any stream
-// capture that includes this entry point.
+// capture that includes this entry point.  The lookup is serialised by a mutex, so two
+// host threads making their first call at once both get the one address.  The cached
+// address belongs to the device's primary context (the one the CUDA runtime uses): a
+// caller that resets the device (cudaDeviceReset) must not call this entry point again
+// in the same process, since the cached address would then be stale.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace {
@@ -35,9 +41,11 @@ constexpr int kMaxDevices = 64;
 // Device address of g_noalloc_scratch on the current device (nullptr on failure).
 void* scratch_on_current_device()
 {
+    static std::mutex lock;
     static void* addr[kMaxDevices] = {nullptr};
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> hold(lock);
     if (!addr[dev]) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
