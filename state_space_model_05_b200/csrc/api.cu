@@ -195,7 +195,7 @@ ssd_status_t prefill_impl(const void* x, const float* dt, const float* dt_bias, 
         TcWorkspace w;
         const size_t need = tc_workspace_layout(t, workspace, &w);
         if (!workspace || workspace_bytes < need) return SSD_ERR_WORKSPACE;
-        if (g_prefill_path.load() == SSD_PREFILL_FUSED) {
+        if (g_prefill_path.load() == SSD_PREFILL_FUSED && fused_prefill_supported(t)) {
             // fused: decay factors, G = C B^T per block, then the chain kernel
             cudaError_t e = profiled(kCumsum, s, [&] {
                 return launch_chunk_cumsum(t, dt, A, w.fac, true, nullptr, B, w.b16, s);

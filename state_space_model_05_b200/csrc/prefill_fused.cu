@@ -1,6 +1,5 @@
-// Fused tensor-core prefill on sm_100a: one CTA walks the 128-token blocks of one to three
-// heads of one (batch, group) in order, keeps their states in tensor memory and writes y,
-// so that x is read once and no intermediate state goes through HBM.
+// Fused tensor-core prefill on sm_100a: x is read once, y written once, and no state goes
+// through HBM except where one CTA hands a chain over to the next.
 //
 // "Compiler-First State Space Duality and Portable O(1) Autoregressive Caching for
 // Inference", section "2. Metodologia": inside a chunk the SSD layer is a masked matrix
@@ -18,19 +17,35 @@
 // these values' range; w o X rounded to fp16): 3 more mantissa bits than bf16, which the
 // state, summed over every block, needs.  G, P, X and the state image are bf16.
 //
-// chain_prefill_kernel, per CTA (b, g, heads hlo .. hlo + nh - 1), items i = k nh + j:
-//   warp 0      TMA: C_k (staging), fp16 B_k (two-deep ring), x and the decay factors of each
-//               item (four-deep ring of slots)
-//   warp 1      tcgen05.mma, polling two streams: Yo_i = C H^T with C in TMEM and the state
-//               image in shared memory, and S_i = B^T X~ accumulated onto the head's state in
-//               TMEM; then Yd_i = P X with P in TMEM
-//   warps 2-3   X~ = w o X (fp16) into a two-deep ring
-//   warps 4-11  P from G_k (read from global memory a block ahead) and the decay factors
-//   warps 12-15 the epilogue y = Yd + exp(Lam_t) Yo + D x, each warp TMA-storing its 32 rows
-//   warps 16-19 the states: per item, the bf16 image of H for Yo, then H <- exp(Lam_end) H in
-//               TMEM, onto which S accumulates
+// pair_chain_kernel works on head pairs: a unit is (b, g, heads h0, h0 + 1), and a step is
+// one 128-token block of one unit.  The two heads share C_k, B_k and G_k, and their state
+// and output GEMMs are one MMA each with the heads side by side along N (N = 128):
+//   S      = B_k^T [X~_0 | X~_1]   onto the pair's states in TMEM (lane n, column 64 j + p)
+//   Yo     = C_k [H_0 | H_1]       (the states' bf16 image in shared memory)
+//   Yd_j   = P_j X_j               (P_j in TMEM, one per head)
+// The steps of all units, unit-major, are cut into one contiguous range per CTA, so every
+// CTA does the same number of blocks however the units divide among the SMs.  A range
+// starts and ends inside a unit at most once each; the CTA runs the piece at its end first
+// (a unit's first blocks), then its whole units, then the piece at its start (a unit's last
+// blocks), whose start state the previous CTA has by then handed over through a global
+// slot.  With at least one unit of blocks per CTA that hand-off is ready before it is
+// needed; it is a bounded wait either way.
+//
+// Roles (448 threads, at most four warps per scheduler, so 128 registers a thread):
+//   warp 0      TMA: x and the decay factors of each step (two slots), C_k, fp16 B_k in
+//               64-token stages (three deep)
+//   warp 1      tcgen05.mma, polling three streams: S, Yo, Yd_j
+//   warps 2-5   X~ = w o X (fp16) for the state GEMM, then the epilogue of the previous
+//               step: y = Yd + exp(Lam_t) Yo + D x, written straight to global memory
+//   warps 6-13  per step, first the state of one head for the warp's 32 TMEM lanes (the
+//               bf16 image of H, the operand of Yo, then H <- exp(Lam_end) H, onto which S
+//               accumulates; start and end states at piece boundaries), then two of the
+//               four 32-column sub-blocks of P_j for its 32 rows, from G_k (read from
+//               global memory a step ahead) and the factors
 // Every wait is bounded; expiry records SSD_ERR_TIMEOUT in the device error word and the
 // CTA drains without further waiting.
+#include <algorithm>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -57,7 +72,8 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // One CTA per (block k, group g, batch b): G_k = C_k B_k^T (K = N = 128) on the tensor
 // cores, rounded to bf16 and stored as four planes of 32 columns, plane kc holding row t's
 // columns 32 kc .. 32 kc + 31 as 64 contiguous bytes at t * 64 -- the order in which the
-// chain kernel's P threads read them.
+// chain kernel's P threads read them.  CTA (0, 0, 0) also clears the chain kernel's
+// hand-off flags.
 constexpr int kGramThreads = 128;
 
 struct GramSmem {
@@ -70,7 +86,8 @@ struct GramSmem {
 
 __global__ void __launch_bounds__(kGramThreads)
 block_gram_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_c,
-                  uint4* __restrict__ gram, int ngroups, int nblocks, int* err)
+                  uint4* __restrict__ gram, int ngroups, int nblocks, int* __restrict__ flags, int nflags,
+                  int* err)
 {
     using L = GramSmem;
     extern __shared__ uint8_t smem_raw[];
@@ -81,6 +98,8 @@ block_gram_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
 
     const int k = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (flags && k == 0 && g == 0 && b == 0)
+        for (int i = tid; i < nflags; i += kGramThreads) flags[i] = 0;
     if (tid == 0) {
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
@@ -149,47 +168,115 @@ block_gram_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constan
     }
 }
 
+// ================================================================ the steps of a CTA
+// Steps i = u nb + k (unit u, block k) of all units, unit-major; CTA c owns [a, e) with
+// a = c W / S, e = (c + 1) W / S.  It runs them as up to three intervals: the piece of unit
+// e / nb at its end (that unit's first blocks), the whole units, and the piece of unit a / nb
+// at its start (that unit's last blocks).  A range inside one unit is one interval.
+struct StepSeq {
+    long long lo[3], hi[3];
+    long long a, e;
+    int nb;
+    __device__ void init(int c, int S, long long units, int nblk) {
+        nb = nblk;
+        const long long W = units * nblk;
+        a = (long long)c * W / S;
+        e = (long long)(c + 1) * W / S;
+        const long long ua = a / nb, ue = e / nb;
+        const long long ka = a - ua * nb;
+        for (int r = 0; r < 3; ++r) lo[r] = hi[r] = 0;
+        if (e <= (ua + 1) * nb) {
+            lo[0] = a;
+            hi[0] = e;
+        } else {
+            lo[0] = ue * nb;
+            hi[0] = e;
+            lo[1] = ka ? (ua + 1) * nb : a;
+            hi[1] = ue * nb;
+            lo[2] = ka ? a : 0;
+            hi[2] = ka ? (ua + 1) * nb : 0;
+        }
+    }
+};
+
+struct StepIter {
+    const StepSeq* q;
+    int r;
+    long long i;
+    __device__ void start(const StepSeq& s) {
+        q = &s;
+        r = 0;
+        i = s.lo[0];
+        skip();
+    }
+    __device__ void skip() {
+        while (r < 3 && i >= q->hi[r]) {
+            ++r;
+            if (r < 3) i = q->lo[r];
+        }
+    }
+    __device__ bool valid() const { return r < 3; }
+    __device__ void next() {
+        ++i;
+        skip();
+    }
+    __device__ int unit() const { return (int)(i / q->nb); }
+    __device__ int block() const { return (int)(i % q->nb); }
+    __device__ bool first() const { return i == q->lo[r] || i % q->nb == 0; }
+    __device__ bool last() const { return i == q->hi[r] - 1 || i % q->nb == q->nb - 1; }
+};
+
+// unit u -> batch, group and the pair's first head (units are (b, g, pair), b-major)
+struct UnitMap {
+    int ngroups, hpg;
+    __device__ void map(int u, int* b, int* g, int* h0) const {
+        const int pairs = hpg >> 1;
+        const int bg = u / pairs, pr = u - bg * pairs;
+        *b = bg / ngroups;
+        *g = bg - *b * ngroups;
+        *h0 = *g * hpg + 2 * pr;
+    }
+};
+
 // ================================================================ chain kernel
-constexpr int kChainThreads = 640;
-constexpr int kMaxHeads = 3;                    // heads per CTA (their states share TMEM)
-constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpConv = 2, kWarpP0 = 4, kWarpE0 = 12, kWarpG0 = 16;
-constexpr int kConvThreads = 64, kPThreads = 256;
+constexpr int kPairThreads = 448;
+constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpE0 = 2, kWarpP0 = 6;
+constexpr int kPThreads = 256;
+constexpr int kHandoffArrivals = 8;             // one per P/state warp
 
-// TMEM columns: the heads' states, the two P buffers (bf16 pairs), Yo, Yd, C_k (bf16 pairs)
-constexpr uint32_t kColH = 0, kColP = 192, kColYo = 320, kColYd = 448;   // Yo: two buffers
+// TMEM columns: the pair's states (lane n), Yd of each head, Yo of the pair (lane t), the
+// two P buffers (bf16 pairs, lane t)
+constexpr uint32_t kColH = 0, kColYd = 128, kColYo = 256, kColP = 384;
 
-struct ChainSmem {
-    static constexpr int kXSlots = 4;
-    static constexpr int kCst = 0;                       // C_k staging [2 n-halves][128 rows][128 B]
-    static constexpr int kB0 = kCst + 2 * kBox;          // B_k ring: 2 x [2 n-halves][128 rows][128 B]
-    static constexpr int kXt0 = kB0 + 4 * kBox;          // X~ ring: 2 x [128 rows][128 B]
-    static constexpr int kImg = kXt0 + 2 * kBox;         // bf16 state image (MN-major, 64-byte swizzle)
-    static constexpr int kSlot0 = kImg + kHImage;        // item slots:
-    static constexpr int kXo = 0;                        //   x (then y) [128 rows][128 B]
-    static constexpr int kLo = kBox;                     //   Lam[128]
-    static constexpr int kDo = kLo + 512;                //   dt[128]
-    static constexpr int kVo = kDo + 512;                //   column factors, sub-block-end reference
-    static constexpr int kWo = kVo + 512;                //   column factors, sub-block-start reference
-    static constexpr int kSlotBytes = kBox + 2048;
-    static constexpr int kBar = kSlot0 + kXSlots * kSlotBytes;
-    static constexpr int kNumBars = 32;
+struct PairSmem {
+    static constexpr int kC = 0;                          // C_k [2 n-halves][128 t][128 B] bf16
+    static constexpr int kBStages = 3;
+    static constexpr int kBStage = 2 * 8192;              // fp16 B: [2 n-halves][64 t][128 B]
+    static constexpr int kB0 = kC + 2 * kBox;
+    static constexpr int kXSlots = 2;
+    static constexpr int kFacBytes = 4 * 512;             // per head: Lam, dt, and two column-factor rows
+    static constexpr int kXFac = 2 * kBox;                // in a slot: x of head 0, of head 1, then factors
+    static constexpr int kXSlot = 2 * kBox + 2 * kFacBytes;
+    static constexpr int kX0 = kB0 + kBStages * kBStage;
+    static constexpr int kXt = kX0 + kXSlots * kXSlot;    // X~ [2 heads][128 t][128 B] fp16
+    static constexpr int kImg = kXt + 2 * kBox;           // state images [2 heads][2 p-halves][128 n][64 B]
+    static constexpr int kBar = kImg + 2 * kHImage;
+    static constexpr int kNumBars = 24;
     static constexpr int kTslot = kBar + kNumBars * 8;
     static constexpr int kAbort = kTslot + 4;
     static constexpr int kBytes = kAbort + 12 + 1024;
 };
-static_assert(ChainSmem::kSlotBytes % 1024 == 0, "slots keep 1024-byte alignment");
-static_assert(ChainSmem::kBytes <= 227 * 1024, "chain shared memory");
+static_assert(PairSmem::kXSlot % 1024 == 0 && PairSmem::kBStage % 1024 == 0, "1024-byte alignment");
+static_assert(PairSmem::kBytes <= 227 * 1024, "chain shared memory");
 
 enum {
-    CB_CSTAGED = 0, CB_CFREE,
-    CB_BFULL, CB_BEMPTY = CB_BFULL + 2,
-    CB_XFULL = CB_BEMPTY + 2, CB_XEMPTY = CB_XFULL + ChainSmem::kXSlots,
-    CB_CONV = CB_XEMPTY + ChainSmem::kXSlots, CB_XTEMPTY = CB_CONV + 2,
-    CB_UPD = CB_XTEMPTY + 2, CB_SDONE,
-    CB_YOFULL = CB_SDONE + kMaxHeads, CB_YOEMPTY = CB_YOFULL + 2, CB_YDFULL = CB_YOEMPTY + 2, CB_YDPRIMED,
-    CB_PFULL, CB_PEMPTY = CB_PFULL + 2, CB_COUNT = CB_PEMPTY + 2
+    PB_XF = 0, PB_XE = PB_XF + PairSmem::kXSlots,
+    PB_BF = PB_XE + PairSmem::kXSlots, PB_BE = PB_BF + PairSmem::kBStages,
+    PB_CF = PB_BE + PairSmem::kBStages, PB_CE,
+    PB_UPD, PB_CONV, PB_SD, PB_YO,
+    PB_PF, PB_YD = PB_PF + 2, PB_EPI = PB_YD + 2, PB_COUNT = PB_EPI + 2
 };
-static_assert(CB_COUNT <= ChainSmem::kNumBars, "chain barriers");
+static_assert(PB_COUNT <= PairSmem::kNumBars, "chain barriers");
 
 // x * w for the eight bf16 values of one 16-byte chunk, rounded to fp16
 __device__ __forceinline__ uint4 scale_to_f16x8(uint4 u, float w) {
@@ -225,6 +312,19 @@ __device__ __noinline__ bool chain_wait(uint64_t* bar, uint32_t parity, int* err
     return mbar_wait_or_abort(bar, parity, err, abort_flag);
 }
 
+// Bounded spin until *flag >= value (acquire), giving up early once the CTA has aborted.
+__device__ __noinline__ bool wait_handoff(const int* flag, int value, int* err, volatile int* abort_flag)
+{
+    for (uint32_t it = 0; it < (1u << 24); ++it) {
+        if (ld_acquire_gpu(flag) >= value) return true;
+        if ((it & 255u) == 255u && *abort_flag) return false;
+        __nanosleep(64);
+    }
+    record_error(err, SSD_ERR_TIMEOUT);
+    *abort_flag = 1;
+    return false;
+}
+
 // One 32-column sub-block of row r of P = G o exp(Lam_t - Lam_s) o dt_s (s <= t), from 16
 // bf16 pairs of G, stored to TMEM at taddr (warp-collective; the sub-block is below, on or
 // above the diagonal for the warp's 32 rows alike).  Below-diagonal sub-blocks use
@@ -232,14 +332,13 @@ __device__ __noinline__ bool chain_wait(uint64_t* bar, uint32_t parity, int* err
 // diagonal use the first column as reference when their own decay is below 40 (both factors
 // within e^+-40) and one exponential per element otherwise.
 __device__ __forceinline__ void p_store_subblock(uint32_t taddr, uint4 g0, uint4 g1, uint4 g2, uint4 g3, int s0,
-                                              int r, const float* sLam, const float* sDt, const float* sV,
-                                              const float* sW)
+                                                 int r, const float* sLam, const float* sDt, const float* sV,
+                                                 const float* sW)
 {
     const uint32_t gw[16] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w,
                              g2.x, g2.y, g2.z, g2.w, g3.x, g3.y, g3.z, g3.w};
     const float lam_t = sLam[r];
     uint32_t pk[16];
-    // the branch is the same for the whole warp (rows r0 .. r0 + 31): tcgen05.st is warp-collective
     const int r0 = r & ~31;
     if (s0 + 32 <= r0) {
         const float u = expf(lam_t - sLam[s0 + 31]);
@@ -265,53 +364,71 @@ __device__ __forceinline__ void p_store_subblock(uint32_t taddr, uint4 g0, uint4
     tmem_st16(taddr, pk);
 }
 
-__global__ void __launch_bounds__(kChainThreads, 1)
-chain_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b16,
-                     const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
-                     const float* __restrict__ fac, const uint4* __restrict__ gram,
-                     const float* __restrict__ D, const float* __restrict__ init_state,
-                     float* __restrict__ final_state, int seqlen, int nheads, int ngroups, int nblk,
-                     int ctas_per_group, int* err)
+// Four 16-byte chunks per lane: lane i of each group of four lanes starts with four chunks
+// of its own row and ends with chunk i of the group's four rows (that of row m at d[m]).
+__device__ __forceinline__ void transpose_quad(uint4 (&d)[4], int lane)
 {
-    using L = ChainSmem;
+#pragma unroll
+    for (int s = 2; s >= 1; s >>= 1) {
+        const bool hi = (lane & s) != 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (c & s) continue;
+            const uint4 keep = hi ? d[c | s] : d[c];
+            const uint4 send = hi ? d[c] : d[c | s];
+            uint4 got;
+            got.x = __shfl_xor_sync(0xffffffffu, send.x, s);
+            got.y = __shfl_xor_sync(0xffffffffu, send.y, s);
+            got.z = __shfl_xor_sync(0xffffffffu, send.z, s);
+            got.w = __shfl_xor_sync(0xffffffffu, send.w, s);
+            d[c] = hi ? got : keep;
+            d[c | s] = hi ? keep : got;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kPairThreads, 1)
+pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b16,
+                  const __grid_constant__ CUtensorMap tm_c, const float* __restrict__ fac,
+                  const uint4* __restrict__ gram, const float* __restrict__ D,
+                  const float* __restrict__ init_state, float* __restrict__ final_state,
+                  __nv_bfloat16* __restrict__ y, float* __restrict__ handoff, int* __restrict__ handoff_flag,
+                  int seqlen, int nheads, int ngroups, int nblk, int units, int* err)
+{
+    using L = PairSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = align1024(smem_raw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::kTslot);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kAbort);
-
-    // this CTA's heads: hlo .. hlo + nh - 1 of group g of batch b
-    const int hpg = nheads / ngroups;
-    const int unit = blockIdx.x / ctas_per_group, part = blockIdx.x - unit * ctas_per_group;
-    const int b = unit / ngroups, g = unit - b * ngroups;
-    const int hlo = g * hpg + (part * hpg) / ctas_per_group;
-    const int nh = g * hpg + ((part + 1) * hpg) / ctas_per_group - hlo;     // 1 .. kMaxHeads
-    const int total = nblk * nh;                       // items (k, j), i = k nh + j
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int cta = blockIdx.x, nctas = gridDim.x;
+
+    StepSeq seq;
+    seq.init(cta, nctas, units, nblk);
+    const UnitMap um{ngroups, nheads / ngroups};
+    const long long total = seq.e - seq.a;                // steps of this CTA
 
     if (tid == 0) {
-        mbar_init(&bars[CB_CSTAGED], 1);
-        mbar_init(&bars[CB_CFREE], 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars[CB_BFULL + i], 1);
-            mbar_init(&bars[CB_BEMPTY + i], 1);
-            mbar_init(&bars[CB_CONV + i], 2);
-            mbar_init(&bars[CB_XTEMPTY + i], 1);
-            mbar_init(&bars[CB_PFULL + i], kPThreads);
-            mbar_init(&bars[CB_PEMPTY + i], 1);
-        }
         for (int i = 0; i < L::kXSlots; ++i) {
-            mbar_init(&bars[CB_XFULL + i], 1);
-            mbar_init(&bars[CB_XEMPTY + i], 4);
+            mbar_init(&bars[PB_XF + i], 1);
+            mbar_init(&bars[PB_XE + i], 1 + 4);           // the last Yd MMA, the 4 epilogue warps
         }
-        mbar_init(&bars[CB_UPD], 4);
-        for (int i = 0; i < kMaxHeads; ++i) mbar_init(&bars[CB_SDONE + i], 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars[CB_YOFULL + i], 1);
-            mbar_init(&bars[CB_YOEMPTY + i], 4);
+        for (int i = 0; i < L::kBStages; ++i) {
+            mbar_init(&bars[PB_BF + i], 1);
+            mbar_init(&bars[PB_BE + i], 1);
         }
-        mbar_init(&bars[CB_YDFULL], 1);
-        mbar_init(&bars[CB_YDPRIMED], 4);
+        mbar_init(&bars[PB_CF], 1);
+        mbar_init(&bars[PB_CE], 1);
+        mbar_init(&bars[PB_UPD], 8);
+        mbar_init(&bars[PB_CONV], 4);
+        mbar_init(&bars[PB_SD], 1);
+        mbar_init(&bars[PB_YO], 1);
+        for (int j = 0; j < 2; ++j) {
+            mbar_init(&bars[PB_PF + j], kPThreads);
+            mbar_init(&bars[PB_YD + j], 1);
+            mbar_init(&bars[PB_EPI + j], 4);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -324,8 +441,8 @@ chain_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tslot;
 
-    auto slot = [&](int i) { return sm + L::kSlot0 + (i & (L::kXSlots - 1)) * L::kSlotBytes; };
-    // bounded wait, the same answer for the whole warp (tcgen05.ld / st are warp-collective)
+    auto xslot = [&](long long s) { return sm + L::kX0 + (int)(s & 1) * L::kXSlot; };
+    auto facp = [&](long long s, int j) { return reinterpret_cast<const float*>(xslot(s) + L::kXFac + j * L::kFacBytes); };
     auto wait_warp = [&](int bar, uint32_t parity) {
         const bool ok = chain_wait(&bars[bar], parity, err, abort_flag);
         return __all_sync(0xffffffffu, ok);
@@ -333,100 +450,137 @@ chain_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
 
     if (warp == kWarpLoad) {
         if (lane == 0) {
-            // ------------------------------------------------ x and decay factors, one slot per item
-            griddep_wait();                              // the decay factors come from an earlier kernel
-            int issued = 0;
-            for (int i = 0; i < total; ++i) {
-                const int k = i / nh, h = hlo + (i - k * nh);
-                if (i >= L::kXSlots &&
-                    !mbar_wait_or_abort(&bars[CB_XEMPTY + (i & 3)], ((i >> 2) - 1) & 1, err, abort_flag))
-                    break;
-                uint8_t* sl = slot(i);
-                mbar_expect_tx(&bars[CB_XFULL + (i & 3)], kBox + 4 * 512);
-                tma_load_3d(sl + L::kXo, &tm_x, h * kP, k * kBlk, b, &bars[CB_XFULL + (i & 3)]);
-                bulk_load(sl + L::kLo, fac + ((size_t)(b * nheads + h) * nblk + k) * 4 * kBlk, 4 * 512,
-                          &bars[CB_XFULL + (i & 3)]);
-                issued = i + 1;
-            }
-            // the CTA does not exit with loads in flight
-            for (int i = max(0, issued - L::kXSlots); i < issued; ++i)
-                mbar_wait(&bars[CB_XFULL + (i & 3)], (i >> 2) & 1, err);
-        } else if (lane == 1) {
-            // ------------------------------------------------ C_k (staging) and B_k (two-deep ring)
-            griddep_wait();                              // the fp16 copy of B comes from an earlier kernel
-            int kc = 0, kb = 0;
-            for (int k = 0; k < nblk; ++k) {
-                // every Yo of block k - 1 has read the staged C
-                if (k >= 1 && !mbar_wait_or_abort(&bars[CB_CFREE], (k - 1) & 1, err, abort_flag)) break;
-                mbar_expect_tx(&bars[CB_CSTAGED], 2 * kBox);
-                tma_load_3d(sm + L::kCst, &tm_c, g * kN, k * kBlk, b, &bars[CB_CSTAGED]);
-                tma_load_3d(sm + L::kCst + kBox, &tm_c, g * kN + 64, k * kBlk, b, &bars[CB_CSTAGED]);
-                kc = k + 1;
-                if (k >= 2 && !mbar_wait_or_abort(&bars[CB_BEMPTY + (k & 1)], ((k >> 1) - 1) & 1, err, abort_flag))
-                    break;
-                uint8_t* sb = sm + L::kB0 + (k & 1) * 2 * kBox;
-                mbar_expect_tx(&bars[CB_BFULL + (k & 1)], 2 * kBox);
-                tma_load_3d(sb, &tm_b16, g * kN, k * kBlk, b, &bars[CB_BFULL + (k & 1)]);
-                tma_load_3d(sb + kBox, &tm_b16, g * kN + 64, k * kBlk, b, &bars[CB_BFULL + (k & 1)]);
-                kb = k + 1;
-            }
-            if (kc > 0) mbar_wait(&bars[CB_CSTAGED], (kc - 1) & 1, err);
-            for (int k = max(0, kb - 2); k < kb; ++k) mbar_wait(&bars[CB_BFULL + (k & 1)], (k >> 1) & 1, err);
-        }
-    } else if (warp == kWarpMma) {
-        if (lane == 0) {
-            // ------------------------------------------------ MMA issue, two polled streams
-            constexpr uint32_t idO = idesc_bf16_f32(128, 64, false, true);   // A in TMEM, B MN-major
-            constexpr uint32_t idS = idesc_f16_f32(128, 64, true, true);     // A = B_k^T, B = X~: fp16, MN-major
-            const uint32_t aImg = smem_u32(sm + L::kImg), aC = smem_u32(sm + L::kCst);
-            int ia = 0, ib = 0;
+            // ------------------------------------------------ loads, three polled streams
+            griddep_wait();                              // factors and fp16 B come from earlier kernels
+            StepIter ix, ib, ic;
+            ix.start(seq);
+            ib.start(seq);
+            ic.start(seq);
+            long long nx = 0, nbh = 0, nc = 0;           // steps of x, 64-token halves of B, steps of C
             uint32_t idle = 0;
-            while (ib < total) {
+            while (ix.valid() || ib.valid() || ic.valid()) {
                 bool progressed = false;
-                if (ia < total) {
-                    // Yo_i = C_k H^T and S_i = B_k^T X~_i (onto the head's state)
-                    const int k = ia / nh, j = ia - k * nh;
-                    if (mbar_test_wait(&bars[CB_UPD], ia & 1) &&
-                        mbar_test_wait(&bars[CB_CONV + (ia & 1)], (ia >> 1) & 1) &&
-                        (ia < 2 || mbar_test_wait(&bars[CB_YOEMPTY + (ia & 1)], ((ia >> 1) - 1) & 1)) &&
-                        (j != 0 || (mbar_test_wait(&bars[CB_CSTAGED], k & 1) &&
-                                    mbar_test_wait(&bars[CB_BFULL + (k & 1)], (k >> 1) & 1)))) {
-                        tc_fence_after();
-                        // Yo into buffer ia mod 2: A = C_k (shared memory, K-major over n)
-#pragma unroll 1
-                        for (int ks = 0; ks < 8; ++ks) {
-                            const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
-                            umma_f16(tmem + kColYo + 64 * (ia & 1), smem_desc_sw128(aC + kb * kBox + off, 16, 1024),
-                                     smem_desc_sw64(aImg + ks * 1024, 8192, 512), idO, ks > 0 ? 1u : 0u);
-                        }
-                        umma_commit(&bars[CB_YOFULL + (ia & 1)]);
-                        if (j == nh - 1) umma_commit(&bars[CB_CFREE]);
-                        const uint32_t aB = smem_u32(sm + L::kB0 + (k & 1) * 2 * kBox);
-                        const uint32_t aXt = smem_u32(sm + L::kXt0 + (ia & 1) * kBox);
-#pragma unroll 1
-                        for (int ks = 0; ks < 8; ++ks)
-                            umma_f16(tmem + kColH + 64 * j, smem_desc_sw128(aB + ks * 2048, kBox, 1024),
-                                     smem_desc_sw128(aXt + ks * 2048, kBox, 1024), idS, 1u);
-                        umma_commit(&bars[CB_SDONE + j]);
-                        umma_commit(&bars[CB_XTEMPTY + (ia & 1)]);
-                        if (j == nh - 1) umma_commit(&bars[CB_BEMPTY + (k & 1)]);
-                        ++ia;
+                if (ix.valid() && (nx < L::kXSlots ||
+                                   mbar_test_wait(&bars[PB_XE + (nx & 1)], ((nx >> 1) - 1) & 1))) {
+                    int b, g, h0;
+                    um.map(ix.unit(), &b, &g, &h0);
+                    const int k = ix.block();
+                    uint8_t* sl = xslot(nx);
+                    uint64_t* fb = &bars[PB_XF + (nx & 1)];
+                    mbar_expect_tx(fb, 2 * kBox + 2 * L::kFacBytes);
+                    for (int j = 0; j < 2; ++j) {
+                        tma_load_3d(sl + j * kBox, &tm_x, (h0 + j) * kP, k * kBlk, b, fb);
+                        bulk_load(sl + L::kXFac + j * L::kFacBytes,
+                                  fac + ((size_t)(b * nheads + h0 + j) * nblk + k) * 4 * kBlk, L::kFacBytes, fb);
+                    }
+                    ++nx;
+                    ix.next();
+                    progressed = true;
+                }
+                if (ib.valid()) {
+                    const int st = (int)(nbh % L::kBStages);
+                    if (nbh < L::kBStages || mbar_test_wait(&bars[PB_BE + st], ((nbh / L::kBStages) - 1) & 1)) {
+                        int b, g, h0;
+                        um.map(ib.unit(), &b, &g, &h0);
+                        const int half = (int)(nbh & 1);
+                        mbar_expect_tx(&bars[PB_BF + st], L::kBStage);
+                        tma_load_4d(sm + L::kB0 + st * L::kBStage, &tm_b16, 0, ib.block() * kBlk + half * 64, 2 * g, b,
+                                    &bars[PB_BF + st]);
+                        ++nbh;
+                        if (half) ib.next();
                         progressed = true;
                     }
                 }
-                if (ib < ia) {
-                    // y_i = (exp(Lam_t) Yo_i + D x_i) + P_i X_i, onto the epilogue's first half
-                    if (mbar_test_wait(&bars[CB_PFULL + (ib & 1)], (ib >> 1) & 1) &&
-                        mbar_test_wait(&bars[CB_YDPRIMED], ib & 1)) {
+                if (ic.valid() && (nc == 0 || mbar_test_wait(&bars[PB_CE], (nc - 1) & 1))) {
+                    int b, g, h0;
+                    um.map(ic.unit(), &b, &g, &h0);
+                    mbar_expect_tx(&bars[PB_CF], 2 * kBox);
+                    tma_load_3d(sm + L::kC, &tm_c, g * kN, ic.block() * kBlk, b, &bars[PB_CF]);
+                    tma_load_3d(sm + L::kC + kBox, &tm_c, g * kN + 64, ic.block() * kBlk, b, &bars[PB_CF]);
+                    ++nc;
+                    ic.next();
+                    progressed = true;
+                }
+                if (progressed) {
+                    idle = 0;
+                } else if (++idle >= (1u << 24) || ((idle & 1023u) == 0 && *abort_flag)) {
+                    if (idle >= (1u << 24)) {
+                        record_error(err, SSD_ERR_TIMEOUT);
+                        *abort_flag = 1;
+                    }
+                    break;
+                }
+            }
+            // the CTA does not exit with loads in flight
+            for (long long s = nx > L::kXSlots ? nx - L::kXSlots : 0; s < nx; ++s)
+                mbar_wait(&bars[PB_XF + (s & 1)], (s >> 1) & 1, err);
+            for (long long h = nbh > L::kBStages ? nbh - L::kBStages : 0; h < nbh; ++h)
+                mbar_wait(&bars[PB_BF + h % L::kBStages], (h / L::kBStages) & 1, err);
+            if (nc > 0) mbar_wait(&bars[PB_CF], (nc - 1) & 1, err);
+        }
+    } else if (warp == kWarpMma) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issue, three polled streams
+            constexpr uint32_t idS = idesc_f16_f32(128, 128, true, true);     // B_k^T x X~ (fp16, MN-major)
+            constexpr uint32_t idO = idesc_bf16_f32(128, 128, false, true);   // C_k x images
+            constexpr uint32_t idD = idesc_bf16_f32(128, 64, false, true);    // P (TMEM) x X
+            const uint32_t aC = smem_u32(sm + L::kC), aXt = smem_u32(sm + L::kXt), aImg = smem_u32(sm + L::kImg);
+            long long ns = 0, no = 0, nd = 0;            // steps of S and Yo issued; heads of Yd issued
+            uint32_t idle = 0;
+            while (ns < total || no < total || nd < 2 * total) {
+                bool progressed = false;
+                if (ns < total) {
+                    const int st0 = (int)((2 * ns) % L::kBStages), st1 = (int)((2 * ns + 1) % L::kBStages);
+                    if (mbar_test_wait(&bars[PB_UPD], ns & 1) && mbar_test_wait(&bars[PB_CONV], ns & 1) &&
+                        mbar_test_wait(&bars[PB_BF + st0], ((2 * ns) / L::kBStages) & 1) &&
+                        mbar_test_wait(&bars[PB_BF + st1], ((2 * ns + 1) / L::kBStages) & 1)) {
                         tc_fence_after();
-                        const uint32_t aX = smem_u32(slot(ib) + L::kXo);
+                        // S[n][64 j + p] += sum_t B_t[n] X~_t[j][p]: A = fp16 B (MN-major, n-halves
+                        // 8 KB apart), B = X~ (MN-major, heads 16 KB apart)
+#pragma unroll 1
+                        for (int ks = 0; ks < 8; ++ks) {
+                            const int st = ks < 4 ? st0 : st1;
+                            umma_f16(tmem + kColH,
+                                     smem_desc_sw128(smem_u32(sm + L::kB0 + st * L::kBStage) + (ks & 3) * 2048, 8192, 1024),
+                                     smem_desc_sw128(aXt + ks * 2048, kBox, 1024), idS, 1u);
+                            if (ks == 3) umma_commit(&bars[PB_BE + st0]);
+                        }
+                        umma_commit(&bars[PB_BE + st1]);
+                        umma_commit(&bars[PB_SD]);
+                        ++ns;
+                        progressed = true;
+                    }
+                }
+                if (no < ns && mbar_test_wait(&bars[PB_CF], no & 1) &&
+                    (no == 0 || (mbar_test_wait(&bars[PB_EPI], (no - 1) & 1) &&
+                                 mbar_test_wait(&bars[PB_EPI + 1], (no - 1) & 1)))) {
+                    tc_fence_after();
+                    // Yo[t][64 j + p] = sum_n C_t[n] H_j[n][p]: A = C (K-major), B = the images
+                    // (MN-major, 64-byte swizzle, the four 32-column blocks 8 KB apart)
+#pragma unroll 1
+                    for (int ks = 0; ks < 8; ++ks)
+                        umma_f16(tmem + kColYo, smem_desc_sw128(aC + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
+                                 smem_desc_sw64(aImg + ks * 1024, 8192, 512), idO, ks > 0 ? 1u : 0u);
+                    umma_commit(&bars[PB_CE]);
+                    umma_commit(&bars[PB_YO]);
+                    ++no;
+                    progressed = true;
+                }
+                if (nd < 2 * total) {
+                    const long long sd = nd >> 1;
+                    const int j = (int)(nd & 1);
+                    if (mbar_test_wait(&bars[PB_PF + j], sd & 1) &&
+                        mbar_test_wait(&bars[PB_XF + (sd & 1)], (sd >> 1) & 1) &&
+                        (sd == 0 || mbar_test_wait(&bars[PB_EPI + j], (sd - 1) & 1))) {
+                        tc_fence_after();
+                        const uint32_t aX = smem_u32(xslot(sd) + j * kBox);
 #pragma unroll 1
                         for (int ks = 0; ks < 8; ++ks)
-                            umma_f16_ts(tmem + kColYd, tmem + kColP + 64 * (ib & 1) + ks * 8,
-                                        smem_desc_sw128(aX + ks * 2048, kBox, 1024), idO, 1u);
-                        umma_commit(&bars[CB_PEMPTY + (ib & 1)]);
-                        umma_commit(&bars[CB_YDFULL]);
-                        ++ib;
+                            umma_f16_ts(tmem + kColYd + 64 * j, tmem + kColP + 64 * j + ks * 8,
+                                        smem_desc_sw128(aX + ks * 2048, kBox, 1024), idD, ks > 0 ? 1u : 0u);
+                        umma_commit(&bars[PB_YD + j]);
+                        if (j == 1) umma_commit(&bars[PB_XE + (sd & 1)]);
+                        ++nd;
                         progressed = true;
                     }
                 }
@@ -440,245 +594,265 @@ chain_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
                     break;
                 }
             }
-            // the CTA does not release TMEM with MMAs in flight
-            if (ib > 0) mbar_wait(&bars[CB_YDFULL], (ib - 1) & 1, err);
-            if (ia > ib) mbar_wait(&bars[CB_XTEMPTY + ((ia - 1) & 1)], ((ia - 1) >> 1) & 1, err);
+            // the CTA does not release TMEM with MMAs in flight: every commit covers all earlier MMAs
+            if (nd > 0) mbar_wait(&bars[PB_YD + ((nd - 1) & 1)], ((nd - 1) >> 1) & 1, err);
+            if (no > 0) mbar_wait(&bars[PB_YO], (no - 1) & 1, err);
+            if (ns > 0) mbar_wait(&bars[PB_SD], (ns - 1) & 1, err);
         }
     } else if (warp < kWarpP0) {
-        // ---------------------------------------------------- X~ = w o X (fp16), w_s = exp(Lam_end - Lam_s) dt_s
-        const int cid = tid - kWarpConv * 32;
-        for (int i = 0; i < total; ++i) {
-            if (!wait_warp(CB_XFULL + (i & 3), (i >> 2) & 1)) break;
-            if (i >= 2 && !wait_warp(CB_XTEMPTY + (i & 1), ((i >> 1) - 1) & 1)) break;
-            const uint8_t* sl = slot(i);
-            const float* sLam = reinterpret_cast<const float*>(sl + L::kLo);
-            const float* sDt = reinterpret_cast<const float*>(sl + L::kDo);
-            const float lend = sLam[kBlk - 1];
-            uint8_t* xt = sm + L::kXt0 + (i & 1) * kBox;
+        // ---------------------------------------------------- X~ = w o X, then the previous step's epilogue
+        const int q = warp & 3;
+        const int t = q * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+        StepIter it;
+        it.start(seq);
+        long long s = 0;
+        int pb = 0, pk = 0, ph0 = 0;                     // the previous step: batch, block, first head
+        float pD0 = 0.f, pD1 = 0.f;
+
+        // y = Yd + exp(Lam_t) Yo + D x of step ps, row t, heads j = 0, 1, stored to global memory
+        auto epilogue = [&](long long ps) -> bool {
+            if (!wait_warp(PB_YO, ps & 1)) return false;
+            const uint8_t* sl = xslot(ps);
+            for (int j = 0; j < 2; ++j) {
+                if (!wait_warp(PB_YD + j, ps & 1)) return false;
+                tc_fence_after();
+                const float u = expf(facp(ps, j)[t]);
+                const float Dh = j ? pD1 : pD0;
+                const uint8_t* xrow = sl + j * kBox + t * 128;
+                __nv_bfloat16* yhead = y + ((size_t)pb * seqlen * nheads + ph0 + j) * kP;
+                const int rbase = pk * kBlk + q * 32 + (lane & ~3);     // the quad's first row
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    uint4 ch[4];
 #pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                const int row = cid + rr * kConvThreads;
-                const float w = expf(lend - sLam[row]) * sDt[row];
-                const uint4* src = reinterpret_cast<const uint4*>(sl + L::kXo + row * 128);
-                uint4* dst = reinterpret_cast<uint4*>(xt + row * 128);
-                uint4 u[8];
+                    for (int qq = 0; qq < 2; ++qq) {
+                        const int col = 32 * half + 16 * qq;
+                        uint32_t yd[16], yo[16];
+                        tmem_ld16(tl + kColYd + 64 * j + col, yd);
+                        tmem_ld16(tl + kColYo + 64 * j + col, yo);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int hq = 0; hq < 2; ++hq) {
+                            const int cx = 4 * half + 2 * qq + hq;          // 16-byte chunk of the row
+                            const uint4 xu = *reinterpret_cast<const uint4*>(xrow + ((cx ^ (t & 7)) << 4));
+                            const uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w};
+                            uint32_t o[4];
+#pragma unroll
+                            for (int k2 = 0; k2 < 4; ++k2) {
+                                const int e = hq * 8 + 2 * k2;
+                                const float a0 = fmaf(u, __uint_as_float(yo[e]), __uint_as_float(yd[e])) + Dh * bf16lo(xw[k2]);
+                                const float a1 = fmaf(u, __uint_as_float(yo[e + 1]), __uint_as_float(yd[e + 1])) + Dh * bf16hi(xw[k2]);
+                                o[k2] = pack_bf16x2(a0, a1);
+                            }
+                            ch[2 * qq + hq] = make_uint4(o[0], o[1], o[2], o[3]);
+                        }
+                    }
+                    if (half == 1) {
+                        // Yd and Yo of head j have been read
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bars[PB_EPI + j]);
+                    }
+                    // four lanes write one row's 64 bytes of this half per store
+                    transpose_quad(ch, lane);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const int tr = rbase + m;
+                        if (tr < seqlen)
+                            *reinterpret_cast<uint4*>(yhead + (size_t)tr * nheads * kP + 32 * half + (lane & 3) * 8) = ch[m];
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[PB_XE + (ps & 1)]);
+            return true;
+        };
+
+        bool live = true;
+        for (; it.valid() && live; it.next(), ++s) {
+            int b, g, h0;
+            um.map(it.unit(), &b, &g, &h0);
+            const int k = it.block();
+            // X~_s (the state GEMM's operand): waits for the slot and for S of the previous step
+            live = wait_warp(PB_XF + (s & 1), (s >> 1) & 1) && (s == 0 || wait_warp(PB_SD, (s - 1) & 1));
+            if (!live) break;
+            const uint8_t* sl = xslot(s);
+#pragma unroll 1
+            for (int j = 0; j < 2; ++j) {
+                const float* sLam = facp(s, j);
+                const float w = expf(sLam[kBlk - 1] - sLam[t]) * sLam[kBlk + t];
+                const uint4* src = reinterpret_cast<const uint4*>(sl + j * kBox + t * 128);
+                uint4* dst = reinterpret_cast<uint4*>(sm + L::kXt + j * kBox + t * 128);
+                uint4 u8[8];
                 // element-wise, so the chunks may be taken in any order: rotating by the row
                 // keeps the eight threads of a shared-memory phase on distinct banks
 #pragma unroll
-                for (int c = 0; c < 8; ++c) u[c] = src[(c + row) & 7];
+                for (int c = 0; c < 8; ++c) u8[c] = src[(c + t) & 7];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) dst[(c + row) & 7] = scale_to_f16x8(u[c], w);
+                for (int c = 0; c < 8; ++c) dst[(c + t) & 7] = scale_to_f16x8(u8[c], w);
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[CB_CONV + (i & 1)]);
+            if (lane == 0) mbar_arrive(&bars[PB_CONV]);
+            const float d0 = D[h0], d1 = D[h0 + 1];
+            if (s > 0) live = epilogue(s - 1);
+            pb = b;
+            pk = k;
+            ph0 = h0;
+            pD0 = d0;
+            pD1 = d1;
         }
-    } else if (warp < kWarpE0) {
-        // ---------------------------------------------------- P = G_k o exp(Lam_t - Lam_s) o dt_s, s <= t
-        // Thread (row r, column half): G_k's 32-column sub-blocks kc0 = half and kc1 = half + 2
-        // of row r, as bf16 pairs, read from global memory a block ahead into the other of
-        // two register sets.
+        if (live && s > 0) epilogue(s - 1);
+    } else {
+        // ---------------------------------------------------- state of head c, then P_j
+        // Warp (quarter q, c): TMEM lanes 32 q .. 32 q + 31.  The state part treats the lane as
+        // state row n and owns head c's 64 columns; the P part treats it as row r of P_j and
+        // builds G_k's 32-column sub-blocks kc0 = c and kc1 = c + 2, from bf16 pairs of G read
+        // from global memory a step ahead.
         const int pw = warp - kWarpP0;
-        const int q = warp & 3, colhalf = pw >> 2;
-        const int r = q * 32 + lane;
-        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-        const int kc0 = colhalf, kc1 = colhalf + 2;
-        const uint4* gbase = gram + (size_t)(b * ngroups + g) * nblk * (kGramBytes / 16);
-        auto load_g = [&](int k, uint4 (&gv)[8]) {
-            const uint4* gk = gbase + (size_t)k * (kGramBytes / 16);
+        const int q = warp & 3, c = pw >> 2;
+        const int r = q * 32 + lane;                     // = n for the state part
+        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+        const int kc0 = c, kc1 = c + 2;
+        auto load_g = [&](const StepIter& at, uint4 (&gv)[8]) {
+            int b, g, h0;
+            um.map(at.unit(), &b, &g, &h0);
+            const uint4* gk = gram + ((size_t)(b * ngroups + g) * nblk + at.block()) * (kGramBytes / 16);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                gv[c] = gk[(kc0 * kBlk + r) * 4 + c];
-                gv[4 + c] = gk[(kc1 * kBlk + r) * 4 + c];
+            for (int i = 0; i < 4; ++i) {
+                gv[i] = gk[(kc0 * kBlk + r) * 4 + i];
+                gv[4 + i] = gk[(kc1 * kBlk + r) * 4 + i];
             }
         };
-        griddep_wait();                                  // G comes from the kernel before this one
-        uint4 ga[8], gb[8];
-        if (nblk > 0) load_g(0, ga);
-        if (nblk > 1) load_g(1, gb);
+        griddep_wait();                                  // G and the hand-off flags come from earlier kernels
+        StepIter it;
+        it.start(seq);
+        // G of the current step; the next step's G is loaded once this step's P is built, and
+        // lands while the next step's state update runs
+        uint4 gv[8];
+        if (it.valid()) load_g(it, gv);
+        const uint32_t hc = tl + kColH + 64 * c;         // this warp's head's state columns
+        const int sw = (r >> 1) & 3;
+        long long s = 0;
         bool live = true;
-        for (int k = 0; k < nblk && live; ++k) {
-            const bool odd = k & 1;
-            for (int j = 0; j < nh; ++j) {
-                const int i = k * nh + j, p = i & 1;
-                live = wait_warp(CB_XFULL + (i & 3), (i >> 2) & 1) &&
-                       (i < 2 || wait_warp(CB_PEMPTY + p, ((i >> 1) - 1) & 1));
+        for (; it.valid() && live; it.next(), ++s) {
+            int b, g, h0;
+            um.map(it.unit(), &b, &g, &h0);
+            const int k = it.block();
+            // ---- state
+            if (it.first()) {
+                // start state: the initial state (or zeros) at block 0, else the previous CTA's hand-off
+                const float* src = nullptr;
+                if (k == 0) {
+                    if (init_state) src = init_state + (size_t)(b * nheads + h0 + c) * kP * kN;
+                } else {
+                    live = __all_sync(0xffffffffu, lane != 0 ||
+                                                   wait_handoff(&handoff_flag[cta], kHandoffArrivals, err, abort_flag));
+                    if (!live) break;
+                    (void)ld_acquire_gpu(&handoff_flag[cta]);     // every lane reads after an acquire
+                    src = handoff + ((size_t)cta * 2 + c) * kP * kN;
+                }
+#pragma unroll 1
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t v[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        v[e] = src ? __float_as_uint(__ldcg(src + (size_t)(16 * cc + e) * kN + r)) : 0u;
+                    tmem_st16(hc + 16 * cc, v);
+                }
+                tmem_wait_st();
+            } else {
+                live = wait_warp(PB_SD, (s - 1) & 1);
                 if (!live) break;
-                const uint8_t* sl = slot(i);
-                const float* sLam = reinterpret_cast<const float*>(sl + L::kLo);
-                const float* sDt = reinterpret_cast<const float*>(sl + L::kDo);
-                const float* sV = reinterpret_cast<const float*>(sl + L::kVo);
-                const float* sW = reinterpret_cast<const float*>(sl + L::kWo);
-                const uint32_t pc = trow + kColP + 64 * p;       // tokens 32 kc .. 32 kc + 31 at pc + 16 kc
-                // one copy of the sub-block code (the kernel's roles run different code at once,
-                // and its instruction footprint is what limits it)
+            }
+            // the image buffer is free once Yo of the previous step is done; the factors of this step
+            live = (s == 0 || wait_warp(PB_YO, (s - 1) & 1)) && wait_warp(PB_XF + (s & 1), (s >> 1) & 1);
+            if (!live) break;
+            tc_fence_after();
+            {
+                // the bf16 image of H_k (operand of Yo), then H <- exp(Lam_end) H, onto which S
+                // accumulates.  Image row n holds p in two 64-byte halves, 16-byte chunk jj of a
+                // half stored at jj ^ ((n / 2) mod 4) (the 64-byte swizzle of the MN-major operand).
+                const float e = expf(facp(s, c)[kBlk - 1]);
+                uint8_t* img = sm + L::kImg + c * kHImage + r * 64;
+#pragma unroll 1
+                for (int q16 = 0; q16 < 4; ++q16) {       // columns 16 q16 .. 16 q16 + 15
+                    uint32_t v[16];
+                    tmem_ld16(hc + 16 * q16, v);
+                    tmem_wait_ld();
+                    uint8_t* half_row = img + (q16 >> 1) * 8192;
+#pragma unroll
+                    for (int j2 = 0; j2 < 2; ++j2) {
+                        const int jj = (q16 & 1) * 2 + j2;
+                        const uint32_t* h8 = &v[8 * j2];
+                        *reinterpret_cast<uint4*>(half_row + ((jj ^ sw) << 4)) = make_uint4(
+                            pack_bf16x2(__uint_as_float(h8[0]), __uint_as_float(h8[1])),
+                            pack_bf16x2(__uint_as_float(h8[2]), __uint_as_float(h8[3])),
+                            pack_bf16x2(__uint_as_float(h8[4]), __uint_as_float(h8[5])),
+                            pack_bf16x2(__uint_as_float(h8[6]), __uint_as_float(h8[7])));
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(e * __uint_as_float(v[i]));
+                    tmem_st16(hc + 16 * q16, v);
+                }
+                tmem_wait_st();
+                fence_proxy_async_smem();                // image -> visible to the tensor cores
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[PB_UPD]);
+            }
+            if (it.last()) {
+                // end state, once S of this step has accumulated: the final state at the unit's
+                // last block, else a hand-off to the next CTA.  The next piece's first step then
+                // loads its start state over H without waiting for S again.
+                live = wait_warp(PB_SD, s & 1);
+                if (!live) break;
+                tc_fence_after();
+                const bool final_block = k == nblk - 1;
+                float* dst = final_block ? final_state + (size_t)(b * nheads + h0 + c) * kP * kN
+                                         : handoff + ((size_t)(cta + 1) * 2 + c) * kP * kN;
+#pragma unroll 1
+                for (int q16 = 0; q16 < 4; ++q16) {
+                    uint32_t v[16];
+                    tmem_ld16(hc + 16 * q16, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) dst[(size_t)(16 * q16 + e) * kN + r] = __uint_as_float(v[e]);
+                }
+                if (!final_block) {
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) atomicAdd(&handoff_flag[cta + 1], 1);
+                }
+                tc_fence_before();
+            }
+            // ---- P_j = G_k o exp(Lam_t - Lam_s) o dt_s, s <= t
+            for (int j = 0; j < 2; ++j) {
+                live = s == 0 || wait_warp(PB_YD + j, (s - 1) & 1);
+                if (!live) break;
+                const float* sLam = facp(s, j);
+                const float* sDt = sLam + kBlk;
+                const float* sV = sLam + 2 * kBlk;
+                const float* sW = sLam + 3 * kBlk;
+                const uint32_t pc = tl + kColP + 64 * j;         // tokens 32 kc .. 32 kc + 31 at pc + 16 kc
 #pragma unroll 1
                 for (int w2 = 0; w2 < 2; ++w2) {
-                    const int kc = w2 ? kc1 : kc0, o = 4 * w2;
-                    p_store_subblock(pc + kc * 16, odd ? gb[o] : ga[o], odd ? gb[o + 1] : ga[o + 1],
-                                     odd ? gb[o + 2] : ga[o + 2], odd ? gb[o + 3] : ga[o + 3], kc * 32, r,
-                                     sLam, sDt, sV, sW);
+                    const int kc = w2 ? kc1 : kc0;
+                    // constant register indices (a computed index would put the set in local memory)
+                    const uint4 g0 = w2 ? gv[4] : gv[0], g1 = w2 ? gv[5] : gv[1];
+                    const uint4 g2 = w2 ? gv[6] : gv[2], g3 = w2 ? gv[7] : gv[3];
+                    p_store_subblock(pc + kc * 16, g0, g1, g2, g3, kc * 32, r, sLam, sDt, sV, sW);
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&bars[CB_PFULL + p]);
+                mbar_arrive(&bars[PB_PF + j]);
             }
-            // block k + 2 into the register set block k used
-            if (live && k + 2 < nblk) {
-                if (odd) load_g(k + 2, gb);
-                else load_g(k + 2, ga);
-            }
-        }
-    } else if (warp < kWarpG0) {
-        // ---------------------------------------------------- epilogue (thread r: token t = r)
-        const int q = warp & 3;
-        const int r = q * 32 + lane;
-        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
-        // D of the CTA's heads, read once (a global load per item would sit on the item chain)
-        float Dv[kMaxHeads];
-#pragma unroll
-        for (int j = 0; j < kMaxHeads; ++j) Dv[j] = j < nh ? D[hlo + j] : 0.f;
-
-        for (int i = 0; i < total; ++i) {
-            const int k = i / nh, j = i - k * nh;
-            // exp(Lam_t) Yo + D x into the Yd accumulator, onto which the MMA then adds P X
-            // (no partial result waits in registers); frees Yo
-            if (!wait_warp(CB_YOFULL + (i & 1), (i >> 1) & 1)) break;
-            tc_fence_after();
-            uint8_t* sl = slot(i);
-            const float u = expf(reinterpret_cast<const float*>(sl + L::kLo)[r]);
-            const float Dh = j == 0 ? Dv[0] : (j == 1 ? Dv[1] : Dv[2]);
-            uint8_t* xrow = sl + L::kXo + r * 128;
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                uint32_t v[32];
-                tmem_ld32(tl + kColYo + 64 * (i & 1) + 32 * half, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const int qx = half * 4 + qq;
-                    const uint4 xu = *reinterpret_cast<const uint4*>(xrow + ((qx ^ (r & 7)) << 4));
-                    const uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w};
-#pragma unroll
-                    for (int k2 = 0; k2 < 4; ++k2) {
-                        const int jj = qq * 8 + 2 * k2;
-                        v[jj] = __float_as_uint(fmaf(u, __uint_as_float(v[jj]), Dh * bf16lo(xw[k2])));
-                        v[jj + 1] = __float_as_uint(fmaf(u, __uint_as_float(v[jj + 1]), Dh * bf16hi(xw[k2])));
-                    }
-                }
-                tmem_st16(tl + kColYd + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-                tmem_st16(tl + kColYd + 32 * half + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bars[CB_YOEMPTY + (i & 1)]);
-                mbar_arrive(&bars[CB_YDPRIMED]);
-            }
-            // y = the finished accumulator -> bf16, written over the item's x rows
-            if (!wait_warp(CB_YDFULL, i & 1)) break;
-            tc_fence_after();
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                uint32_t v[32];
-                tmem_ld32(tl + kColYd + 32 * half, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const int qx = half * 4 + qq;
-                    uint32_t o[4];
-#pragma unroll
-                    for (int k2 = 0; k2 < 4; ++k2)
-                        o[k2] = pack_bf16x2(__uint_as_float(v[qq * 8 + 2 * k2]), __uint_as_float(v[qq * 8 + 2 * k2 + 1]));
-                    *reinterpret_cast<uint4*>(xrow + ((qx ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                }
-            }
-            tc_fence_before();
-            // this warp's 32 rows of y (rows past seqlen are not written)
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                if (k * kBlk + 32 * q < seqlen)
-                    tma_store_3d(&tm_y, (hlo + j) * kP, k * kBlk + 32 * q, b, sl + L::kXo + q * 32 * 128);
-                bulk_commit_group();
-                bulk_wait_group_read1();                 // the previous item's rows have been read
-                if (i > 0) mbar_arrive(&bars[CB_XEMPTY + ((i - 1) & 3)]);
-            }
-        }
-        if (lane == 0) bulk_wait_group0();
-    } else {
-        // ---------------------------------------------------- states (thread n: state row n)
-        const int q = warp & 3;
-        const int n = q * 32 + lane;
-        const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
-
-        // initial states: H_j[n][p] in TMEM lane n, column 64 j + p
-        for (int j = 0; j < nh; ++j) {
-            const float* is = init_state ? init_state + (size_t)(b * nheads + hlo + j) * kP * kN : nullptr;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t v[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] = is ? __float_as_uint(is[(size_t)(16 * c + e) * kN + n]) : 0u;
-                tmem_st16(tl + kColH + 64 * j + 16 * c, v);
-            }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-
-        bool live = true;
-        for (int i = 0; i < total && live; ++i) {
-            const int k = i / nh, j = i - k * nh;
-            // the image buffer is free once Yo of item i - 1 is done
-            if (i > 0 && !wait_warp(CB_YOFULL + ((i - 1) & 1), ((i - 1) >> 1) & 1)) { live = false; break; }
-            // the bf16 image of H_k (operand of Yo), then H <- exp(Lam_end) H, onto which S
-            // accumulates.  Image row n holds p in two 64-byte halves, 16-byte chunk jj of a
-            // half stored at jj ^ ((n / 2) mod 4) (the 64-byte swizzle of the MN-major operand).
-            if (!wait_warp(CB_XFULL + (i & 3), (i >> 2) & 1)) { live = false; break; }
-            if (k > 0 && !wait_warp(CB_SDONE + j, (k - 1) & 1)) { live = false; break; }
-            tc_fence_after();
-            const float e = expf(reinterpret_cast<const float*>(slot(i) + L::kLo)[kBlk - 1]);
-            const uint32_t hc = tl + kColH + 64 * j;
-            uint8_t* img = sm + L::kImg + n * 64;
-            const int sw = (n >> 1) & 3;
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                uint32_t v[32];
-                tmem_ld32(hc + 32 * half, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const uint32_t* h8 = &v[8 * jj];
-                    *reinterpret_cast<uint4*>(img + half * 8192 + ((jj ^ sw) << 4)) = make_uint4(
-                        pack_bf16x2(__uint_as_float(h8[0]), __uint_as_float(h8[1])),
-                        pack_bf16x2(__uint_as_float(h8[2]), __uint_as_float(h8[3])),
-                        pack_bf16x2(__uint_as_float(h8[4]), __uint_as_float(h8[5])),
-                        pack_bf16x2(__uint_as_float(h8[6]), __uint_as_float(h8[7])));
-                }
-#pragma unroll
-                for (int c = 0; c < 32; ++c) v[c] = __float_as_uint(e * __uint_as_float(v[c]));
-                tmem_st16(hc + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-                tmem_st16(hc + 32 * half + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-            }
-            tmem_wait_st();
-            fence_proxy_async_smem();                    // image -> visible to the tensor cores
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[CB_UPD]);
-        }
-        // final states, once each head's last S has accumulated
-        for (int j = 0; j < nh && live; ++j) {
-            if (!wait_warp(CB_SDONE + j, (nblk - 1) & 1)) break;
-            tc_fence_after();
-            float* fs = final_state + (size_t)(b * nheads + hlo + j) * kP * kN;
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                uint32_t v[32];
-                tmem_ld32(tl + kColH + 64 * j + 32 * half, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 32; ++c) fs[(size_t)(32 * half + c) * kN + n] = __uint_as_float(v[c]);
+            // the next step's G
+            if (live) {
+                StepIter nx = it;
+                nx.next();
+                if (nx.valid()) load_g(nx, gv);
             }
         }
     }
@@ -690,18 +864,23 @@ chain_prefill_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_cons
     }
 }
 
-// CTAs per (b, g): at most three heads each, and as many as fill the SMs otherwise (never
-// more than there are heads)
-int chain_ctas_per_group(const Dims& d)
+int pair_ctas(const Dims& d)
 {
-    const int hpg = d.nheads / d.ngroups;
-    const int units = d.batch * d.ngroups;
-    int cpg = (hpg + kMaxHeads - 1) / kMaxHeads;
-    cpg = max(cpg, tc_sm_count() / max(units, 1));
-    return min(cpg, hpg);
+    const long long units = fused_units(d);
+    return (int)std::min<long long>(std::min<long long>(units, tc_sm_count()), kFusedMaxCtas);
 }
 
 }  // namespace
+
+bool fused_prefill_supported(const Dims& d)
+{
+    return d.nseq == 0 && (d.nheads / d.ngroups) % 2 == 0;
+}
+
+long long fused_units(const Dims& d)
+{
+    return (long long)d.batch * d.ngroups * ((d.nheads / d.ngroups) / 2);
+}
 
 cudaError_t launch_block_gram(const Dims& d, const void* B, const void* C, const TcWorkspace& w,
                               cudaStream_t s)
@@ -715,8 +894,10 @@ cudaError_t launch_block_gram(const Dims& d, const void* B, const void* C, const
     cudaError_t e = cudaFuncSetAttribute(block_gram_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          GramSmem::kBytes);
     if (e != cudaSuccess) return e;
+    const int nflags = fused_prefill_supported(d) ? pair_ctas(d) + 1 : 0;
     return launch_dependent(block_gram_kernel, dim3(d.nchunks, d.ngroups, d.batch), dim3(kGramThreads),
-                            GramSmem::kBytes, s, mb, mc, w.gram, d.ngroups, d.nchunks, device_error_word());
+                            GramSmem::kBytes, s, mb, mc, w.gram, d.ngroups, d.nchunks,
+                            nflags ? w.handoff_flag : nullptr, nflags, device_error_word());
 }
 
 cudaError_t launch_chain_prefill(const Dims& d, const void* x, const void* C, const float* D,
@@ -724,22 +905,25 @@ cudaError_t launch_chain_prefill(const Dims& d, const void* x, const void* C, co
                                  void* y, cudaStream_t s)
 {
     if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
-    if (d.chunk_len != kBlk || d.nseq != 0) return cudaErrorInvalidValue;
-    CUtensorMap mx, mb, mc, my;
+    if (d.chunk_len != kBlk || !fused_prefill_supported(d)) return cudaErrorInvalidValue;
+    CUtensorMap mx, mb, mc;
+    // fp16 B [b][T][G][N] seen as (n mod 64, t, 2 g + n / 64, b): a box is both n-halves of 64 rows
+    const uint64_t T = d.seqlen, G = d.ngroups, Bt = d.batch;
+    const uint64_t bdim[4] = {64, T, 2 * G, Bt};
+    const uint64_t bstr[3] = {G * kN * 2, 128, T * G * kN * 2};
+    const uint32_t bbox[4] = {64, 64, 2, 1};
     if (!tc_make_map(&mx, x, (uint64_t)d.nheads * kP, d.seqlen, d.batch) ||
-        !tc_make_map(&mb, w.b16, (uint64_t)d.ngroups * kN, d.seqlen, d.batch, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-        !tc_make_map(&mc, C, (uint64_t)d.ngroups * kN, d.seqlen, d.batch) ||
-        !tc_make_map(&my, y, (uint64_t)d.nheads * kP, d.seqlen, d.batch, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32))
+        !tc_encode_map(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, w.b16, bdim, bstr, bbox, true) ||
+        !tc_make_map(&mc, C, (uint64_t)d.ngroups * kN, d.seqlen, d.batch))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(chain_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         ChainSmem::kBytes);
+    cudaError_t e = cudaFuncSetAttribute(pair_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         PairSmem::kBytes);
     if (e != cudaSuccess) return e;
-    const int cpg = chain_ctas_per_group(d);
-    const unsigned grid = (unsigned)(d.batch * d.ngroups * cpg);
-    return launch_dependent(chain_prefill_kernel, dim3(grid), dim3(kChainThreads), ChainSmem::kBytes, s, mx,
-                            mb, mc, my, static_cast<const float*>(w.fac), static_cast<const uint4*>(w.gram), D,
-                            init_state, final_state, d.seqlen, d.nheads, d.ngroups, d.nchunks, cpg,
-                            device_error_word());
+    const int ctas = pair_ctas(d);
+    return launch_dependent(pair_chain_kernel, dim3(ctas), dim3(kPairThreads), PairSmem::kBytes, s, mx, mb, mc,
+                            static_cast<const float*>(w.fac), static_cast<const uint4*>(w.gram), D, init_state,
+                            final_state, static_cast<__nv_bfloat16*>(y), w.handoff, w.handoff_flag, d.seqlen,
+                            d.nheads, d.ngroups, d.nchunks, (int)fused_units(d), device_error_word());
 }
 
 }  // namespace ssd

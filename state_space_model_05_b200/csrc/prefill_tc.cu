@@ -921,6 +921,12 @@ bool tc_make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows
 
 int tc_sm_count() { return sm_count(); }
 
+bool tc_encode_map(CUtensorMap* m, CUtensorMapDataType type, int rank, const void* base,
+                   const uint64_t* dims, const uint64_t* strides, const uint32_t* box, bool swizzle)
+{
+    return encode_map(m, type, rank, base, dims, strides, box, swizzle);
+}
+
 bool tc_prefill_supported(const Dims& d)
 {
     return d.headdim == kP && d.dstate == kN && (d.chunk_len == 128 || d.chunk_len == 256);
@@ -943,13 +949,19 @@ size_t tc_workspace_layout(const Dims& d, void* base, TcWorkspace* w)
     const size_t himg_b = up(BH * d.nchunks * kHImage);
     const size_t b16_b = up((size_t)d.batch * d.seqlen * d.ngroups * kN * 2);
     const size_t gram_b = up((size_t)d.batch * d.ngroups * d.nchunks * kBlk * kBlk * 2);
-    const size_t mid_b = std::max(wts_b + himg_b, gram_b);
+    // fused path: a hand-off state (two heads) and flag per CTA boundary that can split a pair
+    const size_t slots = d.nseq ? 0 : (size_t)std::min<long long>(fused_units(d), kFusedMaxCtas) + 1;
+    const size_t hand_b = up(slots * 2 * kP * kN * sizeof(float));
+    const size_t flag_b = up(slots * sizeof(int));
+    const size_t mid_b = std::max(wts_b + himg_b, gram_b + hand_b + flag_b);
     if (w) {
         char* p = static_cast<char*>(base);
         w->fac = reinterpret_cast<float*>(p);
         w->wts = reinterpret_cast<float*>(p + fac_b);
         w->himg = reinterpret_cast<uint8_t*>(p + fac_b + wts_b);
         w->gram = reinterpret_cast<uint4*>(p + fac_b);
+        w->handoff = reinterpret_cast<float*>(p + fac_b + gram_b);
+        w->handoff_flag = reinterpret_cast<int*>(p + fac_b + gram_b + hand_b);
         w->b16 = p + fac_b + mid_b;
     }
     return fac_b + mid_b + b16_b;

@@ -27,6 +27,9 @@ struct TcWorkspace {
     void* b16;        // [b][T][G][N] fp16 copy of B (operand of the chunk-state GEMM)
     uint4* gram;      // fused path, over wts / himg: [b][g][c] bf16 G = C B^T of each block,
                       //   four planes of 32 columns ([plane][row t][32 bf16])
+    float* handoff;   // fused path, after gram: [slot][2 heads][P][N] fp32 states handed from one
+                      //   CTA to the next where a head pair's blocks are split between them
+    int* handoff_flag;  // fused path: [slot] arrival counts of those hand-offs
 };
 // Sized for either path: fac, then wts + himg (two-pass) or gram (fused), whichever is
 // larger, then b16 (both).
@@ -50,9 +53,10 @@ cudaError_t launch_chunk_output_tc(const Dims& d, const void* x, const void* B, 
                                    const float* D, const TcWorkspace& w, void* y, cudaStream_t s);
 
 // Fused path (batched, not packed variable-length), launched after the cumsum kernel:
-// G = C B^T of every block (bf16, w.gram); then one kernel that walks each (b, 1-3 heads)
-// chain of blocks with the states in TMEM and writes y and the final state.  Both are
-// programmatic dependents; the G kernel completes only after the cumsum kernel has.
+// G = C B^T of every block (bf16, w.gram; the same launch clears the hand-off flags); then
+// one kernel whose CTAs walk the blocks of head pairs with the pairs' states in TMEM and
+// write y and the final state.  Both are programmatic dependents; the G kernel completes
+// only after the cumsum kernel has.
 cudaError_t launch_block_gram(const Dims& d, const void* B, const void* C, const TcWorkspace& w,
                               cudaStream_t s);
 // The chain kernel reads the fp16 copy of B (w.b16) that the cumsum kernel writes.
@@ -60,10 +64,20 @@ cudaError_t launch_chain_prefill(const Dims& d, const void* x, const void* C, co
                                  const TcWorkspace& w, const float* init_state, float* final_state,
                                  void* y, cudaStream_t s);
 
+// Fused path: the head pairs' chains and the hand-off slots they may need (one per CTA
+// boundary, at most kFusedMaxCtas + 1).
+constexpr int kFusedMaxCtas = 256;
+bool fused_prefill_supported(const Dims& d);
+long long fused_units(const Dims& d);
+
 // helpers shared by the tensor-core launchers
 // 16-bit tensor [outer][rows][inner] read in boxes of 64 (inner) x box_rows, 128-byte swizzle.
 bool tc_make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
                  CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, uint32_t box_rows = 128);
+// Tiled map of `rank` dimensions (dim 0 contiguous, strides in bytes for dims 1..rank-1),
+// 128-byte swizzle or none.
+bool tc_encode_map(CUtensorMap* m, CUtensorMapDataType type, int rank, const void* base,
+                   const uint64_t* dims, const uint64_t* strides, const uint32_t* box, bool swizzle);
 int tc_sm_count();
 
 // Launch with programmatic stream serialisation: the kernel may start while the previous

@@ -56,14 +56,16 @@ def test_workspace_bytes(lib):
     # tensor-core path (bf16, P 64, N 128, Q 128/256), sized by 128-token blocks: per block
     # Lam, dt and two column-factor rows; then either the two-pass kernels' chunk-state
     # weights and block decay and bf16 block-start-state images, or the fused kernels' bf16
-    # G = C B^T per (b, g, block), whichever is larger; then the fp16 copy of B (both)
+    # G = C B^T per (b, g, block) with a two-head fp32 hand-off state and a flag per CTA
+    # boundary (head pairs, at most 256 CTAs), whichever is larger; then the fp16 copy of B
     def tc_bytes(T):
         nb = -(-T // 128)
         fac = b * H * nb * 4 * 128 * 4           # Lam, dt, two column-factor rows
         wts = b * H * nb * (128 + 4) * 4          # chunk-state weights + block decay
         two_pass = up(wts) + up(b * H * nb * 16384)
-        gram = up(b * G * nb * 128 * 128 * 2)
-        return up(fac) + max(two_pass, gram) + up(b * T * G * N * 2)
+        slots = min(b * G * (H // G // 2), 256) + 1
+        fused = up(b * G * nb * 128 * 128 * 2) + up(slots * 2 * P * N * 4) + up(slots * 4)
+        return up(fac) + max(two_pass, fused) + up(b * T * G * N * 2)
     assert _ws(b, T, H, P, G, N, Q, binding.SSD_BF16) == tc_bytes(T)
     assert _ws(b, T, H, P, G, N, 256, binding.SSD_BF16) == tc_bytes(T)
     # bf16 with other shapes uses the CUDA-core layout
