@@ -22,7 +22,7 @@
 // and output GEMMs are one MMA each with the heads side by side along N (N = 128):
 //   S      = B_k^T [X~_0 | X~_1]   onto the pair's states in TMEM (lane n, column 64 j + p)
 //   Yo     = C_k [H_0 | H_1]       (the states' bf16 image in shared memory)
-//   Yd_j   = P_j X_j               (P_j in TMEM, one per head)
+//   Yd_j   = D x_j + P_j X_j       (P_j in TMEM, one per head; D x stored first)
 // The steps of all units, unit-major, are cut into one contiguous range per CTA, so every
 // CTA does the same number of blocks however the units divide among the SMs.  A range
 // starts and ends inside a unit at most once each; the CTA runs the piece at its end first
@@ -31,12 +31,13 @@
 // slot.  With at least one unit of blocks per CTA that hand-off is ready before it is
 // needed; it is a bounded wait either way.
 //
-// Roles (448 threads, at most four warps per scheduler, so 128 registers a thread):
-//   warp 0      TMA: x and the decay factors of each step (two slots), C_k, fp16 B_k in
-//               64-token stages (three deep)
-//   warp 1      tcgen05.mma, polling three streams: S, Yo, Yd_j
-//   warps 2-5   X~ = w o X (fp16) for the state GEMM, then the epilogue of the previous
-//               step: y = Yd + exp(Lam_t) Yo + D x, written straight to global memory
+// Roles (512 threads, four warps per scheduler, so 128 registers a thread):
+//   warp 0      TMA, polling three streams: x and the decay factors of each step (two slots,
+//               fetched into L2 four steps ahead); fp16 B_k in 64-token stages (three deep); C_k
+//   warps 1, 14, 15  tcgen05.mma issue, one stream each: S, Yo, Yd_j
+//   warps 2-5   X~ = w o X (fp16) for the state GEMM; the epilogue of the previous step,
+//               y = Yd + exp(Lam_t) Yo, written straight to global memory; then D x of this
+//               step into the Yd accumulators, onto which the Yd MMA adds P X
 //   warps 6-13  per step, first the state of one head for the warp's 32 TMEM lanes (the
 //               bf16 image of H, the operand of Yo, then H <- exp(Lam_end) H, onto which S
 //               accumulates; start and end states at piece boundaries), then two of the
@@ -199,33 +200,6 @@ struct StepSeq {
     }
 };
 
-struct StepIter {
-    const StepSeq* q;
-    int r;
-    long long i;
-    __device__ void start(const StepSeq& s) {
-        q = &s;
-        r = 0;
-        i = s.lo[0];
-        skip();
-    }
-    __device__ void skip() {
-        while (r < 3 && i >= q->hi[r]) {
-            ++r;
-            if (r < 3) i = q->lo[r];
-        }
-    }
-    __device__ bool valid() const { return r < 3; }
-    __device__ void next() {
-        ++i;
-        skip();
-    }
-    __device__ int unit() const { return (int)(i / q->nb); }
-    __device__ int block() const { return (int)(i % q->nb); }
-    __device__ bool first() const { return i == q->lo[r] || i % q->nb == 0; }
-    __device__ bool last() const { return i == q->hi[r] - 1 || i % q->nb == q->nb - 1; }
-};
-
 // unit u -> batch, group and the pair's first head (units are (b, g, pair), b-major)
 struct UnitMap {
     int ngroups, hpg;
@@ -238,11 +212,60 @@ struct UnitMap {
     }
 };
 
+// Walks a CTA's steps in order.  The unit, block, batch, group and first head of the current
+// step are kept incrementally: the divisions that locate a step run only where an interval
+// starts or the unit changes, not on every step.
+struct StepIter {
+    const StepSeq* q;
+    const UnitMap* um;
+    int r;
+    long long i;
+    int u, k, b, g, h0;
+    __device__ void start(const StepSeq& s, const UnitMap& m) {
+        q = &s;
+        um = &m;
+        r = 0;
+        i = s.lo[0];
+        skip();
+    }
+    __device__ void locate() {
+        u = (int)(i / q->nb);
+        k = (int)(i - (long long)u * q->nb);
+        um->map(u, &b, &g, &h0);
+    }
+    __device__ void skip() {
+        while (r < 3 && i >= q->hi[r]) {
+            ++r;
+            if (r < 3) i = q->lo[r];
+        }
+        if (r < 3) locate();
+    }
+    __device__ bool valid() const { return r < 3; }
+    __device__ void next() {
+        ++i;
+        if (i >= q->hi[r]) {
+            skip();
+            return;
+        }
+        if (++k == q->nb) {
+            k = 0;
+            ++u;
+            um->map(u, &b, &g, &h0);
+        }
+    }
+    __device__ int unit() const { return u; }
+    __device__ int block() const { return k; }
+    __device__ bool first() const { return i == q->lo[r] || k == 0; }
+    __device__ bool last() const { return i == q->hi[r] - 1 || k == q->nb - 1; }
+};
+
 // ================================================================ chain kernel
-constexpr int kPairThreads = 448;
-constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpE0 = 2, kWarpP0 = 6;
+constexpr int kPairThreads = 512;
+constexpr int kWarpLoad = 0, kWarpMma = 1, kWarpE0 = 2, kWarpP0 = 6, kWarpMmaO = 14, kWarpMmaD = 15;
+constexpr int kWarpMmaS = kWarpMma;
 constexpr int kPThreads = 256;
 constexpr int kHandoffArrivals = 8;             // one per P/state warp
+constexpr int kPrefetchSteps = 4;               // steps of x fetched into L2 ahead of their loads
 
 // TMEM columns: the pair's states (lane n), Yd of each head, Yo of the pair (lane t), the
 // two P buffers (bf16 pairs, lane t)
@@ -274,7 +297,7 @@ enum {
     PB_BF = PB_XE + PairSmem::kXSlots, PB_BE = PB_BF + PairSmem::kBStages,
     PB_CF = PB_BE + PairSmem::kBStages, PB_CE,
     PB_UPD, PB_CONV, PB_SD, PB_YO,
-    PB_PF, PB_YD = PB_PF + 2, PB_EPI = PB_YD + 2, PB_COUNT = PB_EPI + 2
+    PB_PF, PB_YD = PB_PF + 2, PB_EPI = PB_YD + 2, PB_DXR = PB_EPI + 2, PB_COUNT = PB_DXR + 2
 };
 static_assert(PB_COUNT <= PairSmem::kNumBars, "chain barriers");
 
@@ -307,9 +330,22 @@ __device__ __noinline__ void p_subblock_strong_decay(uint32_t taddr, uint4 g0, u
 }
 
 // Bounded wait (as mbar_wait_or_abort), one out-of-line copy for all the kernel's call sites.
+// Between polls the thread sleeps (64 ns, doubling to 512 ns): a dozen roles wait at any
+// moment, and a spinning waiter takes issue slots from the warps that do the work.  Gives
+// up after about 2^22 polls (seconds), or soon after another thread has recorded a timeout.
 __device__ __noinline__ bool chain_wait(uint64_t* bar, uint32_t parity, int* err, volatile int* abort_flag)
 {
-    return mbar_wait_or_abort(bar, parity, err, abort_flag);
+    if (mbar_try_wait(bar, parity)) return true;
+    uint32_t ns = 64;
+    for (uint32_t i = 0; i < (1u << 22); ++i) {
+        __nanosleep(ns);
+        if (mbar_try_wait(bar, parity)) return true;
+        if (ns < 512) ns <<= 1;
+        if ((i & 255u) == 255u && *abort_flag) return false;
+    }
+    record_error(err, SSD_ERR_TIMEOUT);
+    *abort_flag = 1;
+    return false;
 }
 
 // Bounded spin until *flag >= value (acquire), giving up early once the CTA has aborted.
@@ -342,20 +378,27 @@ __device__ __forceinline__ void p_store_subblock(uint32_t taddr, uint4 g0, uint4
     const int r0 = r & ~31;
     if (s0 + 32 <= r0) {
         const float u = expf(lam_t - sLam[s0 + 31]);
+        const float4* v4 = reinterpret_cast<const float4*>(sV + s0);
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(bf16lo(gw[e]) * u * sV[s0 + 2 * e], bf16hi(gw[e]) * u * sV[s0 + 2 * e + 1]);
+        for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 f = v4[e4];
+            pk[2 * e4] = pack_bf16x2(bf16lo(gw[2 * e4]) * u * f.x, bf16hi(gw[2 * e4]) * u * f.y);
+            pk[2 * e4 + 1] = pack_bf16x2(bf16lo(gw[2 * e4 + 1]) * u * f.z, bf16hi(gw[2 * e4 + 1]) * u * f.w);
+        }
     } else if (s0 >= r0 + 32) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) pk[e] = 0u;
     } else if (sLam[s0] - sLam[s0 + 31] < 40.f) {
         const float u = expf(lam_t - sLam[s0]);
+        const float4* w4 = reinterpret_cast<const float4*>(sW + s0);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const int sa = s0 + 2 * e;
-            const float pa = bf16lo(gw[e]) * u * sW[sa];
-            const float pb = bf16hi(gw[e]) * u * sW[sa + 1];
-            pk[e] = pack_bf16x2(sa <= r ? pa : 0.f, sa + 1 <= r ? pb : 0.f);
+        for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 f = w4[e4];
+            const int sa = s0 + 4 * e4;
+            pk[2 * e4] = pack_bf16x2(sa <= r ? bf16lo(gw[2 * e4]) * u * f.x : 0.f,
+                                     sa + 1 <= r ? bf16hi(gw[2 * e4]) * u * f.y : 0.f);
+            pk[2 * e4 + 1] = pack_bf16x2(sa + 2 <= r ? bf16lo(gw[2 * e4 + 1]) * u * f.z : 0.f,
+                                         sa + 3 <= r ? bf16hi(gw[2 * e4 + 1]) * u * f.w : 0.f);
         }
     } else {
         p_subblock_strong_decay(taddr, g0, g1, g2, g3, s0, r, sLam, sDt);
@@ -407,12 +450,12 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
     StepSeq seq;
     seq.init(cta, nctas, units, nblk);
     const UnitMap um{ngroups, nheads / ngroups};
-    const long long total = seq.e - seq.a;                // steps of this CTA
+    const int total = (int)(seq.e - seq.a);               // steps of this CTA
 
     if (tid == 0) {
         for (int i = 0; i < L::kXSlots; ++i) {
             mbar_init(&bars[PB_XF + i], 1);
-            mbar_init(&bars[PB_XE + i], 1 + 4);           // the last Yd MMA, the 4 epilogue warps
+            mbar_init(&bars[PB_XE + i], 1 + 4);           // the last Yd MMA, the 4 X~ / epilogue warps
         }
         for (int i = 0; i < L::kBStages; ++i) {
             mbar_init(&bars[PB_BF + i], 1);
@@ -428,6 +471,7 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
             mbar_init(&bars[PB_PF + j], kPThreads);
             mbar_init(&bars[PB_YD + j], 1);
             mbar_init(&bars[PB_EPI + j], 4);
+            mbar_init(&bars[PB_DXR + j], 4);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -441,8 +485,8 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
     tc_fence_after();
     const uint32_t tmem = *tslot;
 
-    auto xslot = [&](long long s) { return sm + L::kX0 + (int)(s & 1) * L::kXSlot; };
-    auto facp = [&](long long s, int j) { return reinterpret_cast<const float*>(xslot(s) + L::kXFac + j * L::kFacBytes); };
+    auto xslot = [&](int s) { return sm + L::kX0 + (s & 1) * L::kXSlot; };
+    auto facp = [&](int s, int j) { return reinterpret_cast<const float*>(xslot(s) + L::kXFac + j * L::kFacBytes); };
     auto wait_warp = [&](int bar, uint32_t parity) {
         const bool ok = chain_wait(&bars[bar], parity, err, abort_flag);
         return __all_sync(0xffffffffu, ok);
@@ -452,18 +496,29 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
         if (lane == 0) {
             // ------------------------------------------------ loads, three polled streams
             griddep_wait();                              // factors and fp16 B come from earlier kernels
-            StepIter ix, ib, ic;
-            ix.start(seq);
-            ib.start(seq);
-            ic.start(seq);
-            long long nx = 0, nbh = 0, nc = 0;           // steps of x, 64-token halves of B, steps of C
+            StepIter ix, ib, ic, ip;
+            ix.start(seq, um);
+            ib.start(seq, um);
+            ic.start(seq, um);
+            // x and the decay factors of the steps ahead are fetched into L2 first, so that a
+            // slot's own load (issued once the slot is free) finds them there
+            ip.start(seq, um);
+            auto prefetch = [&](const StepIter& at) {
+                const int b = at.b, g = at.g, h0 = at.h0;
+                const int k = at.block();
+                for (int j = 0; j < 2; ++j) {
+                    tma_prefetch_3d(&tm_x, (h0 + j) * kP, k * kBlk, b);
+                    bulk_prefetch_l2(fac + ((size_t)(b * nheads + h0 + j) * nblk + k) * 4 * kBlk, L::kFacBytes);
+                }
+            };
+            for (int i = 0; i < kPrefetchSteps && ip.valid(); ++i, ip.next()) prefetch(ip);
+            int nx = 0, nbh = 0, nc = 0;           // steps of x, 64-token halves of B, steps of C
             uint32_t idle = 0;
             while (ix.valid() || ib.valid() || ic.valid()) {
                 bool progressed = false;
                 if (ix.valid() && (nx < L::kXSlots ||
                                    mbar_test_wait(&bars[PB_XE + (nx & 1)], ((nx >> 1) - 1) & 1))) {
-                    int b, g, h0;
-                    um.map(ix.unit(), &b, &g, &h0);
+                    const int b = ix.b, g = ix.g, h0 = ix.h0;
                     const int k = ix.block();
                     uint8_t* sl = xslot(nx);
                     uint64_t* fb = &bars[PB_XF + (nx & 1)];
@@ -475,13 +530,16 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                     }
                     ++nx;
                     ix.next();
+                    if (ip.valid()) {
+                        prefetch(ip);
+                        ip.next();
+                    }
                     progressed = true;
                 }
                 if (ib.valid()) {
                     const int st = (int)(nbh % L::kBStages);
                     if (nbh < L::kBStages || mbar_test_wait(&bars[PB_BE + st], ((nbh / L::kBStages) - 1) & 1)) {
-                        int b, g, h0;
-                        um.map(ib.unit(), &b, &g, &h0);
+                        const int b = ib.b, g = ib.g, h0 = ib.h0;
                         const int half = (int)(nbh & 1);
                         mbar_expect_tx(&bars[PB_BF + st], L::kBStage);
                         tma_load_4d(sm + L::kB0 + st * L::kBStage, &tm_b16, 0, ib.block() * kBlk + half * 64, 2 * g, b,
@@ -492,8 +550,7 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                     }
                 }
                 if (ic.valid() && (nc == 0 || mbar_test_wait(&bars[PB_CE], (nc - 1) & 1))) {
-                    int b, g, h0;
-                    um.map(ic.unit(), &b, &g, &h0);
+                    const int b = ic.b, g = ic.g, h0 = ic.h0;
                     mbar_expect_tx(&bars[PB_CF], 2 * kBox);
                     tma_load_3d(sm + L::kC, &tm_c, g * kN, ic.block() * kBlk, b, &bars[PB_CF]);
                     tma_load_3d(sm + L::kC + kBox, &tm_c, g * kN + 64, ic.block() * kBlk, b, &bars[PB_CF]);
@@ -503,7 +560,7 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                 }
                 if (progressed) {
                     idle = 0;
-                } else if (++idle >= (1u << 24) || ((idle & 1023u) == 0 && *abort_flag)) {
+                } else if (__nanosleep(128), ++idle >= (1u << 24) || ((idle & 1023u) == 0 && *abort_flag)) {
                     if (idle >= (1u << 24)) {
                         record_error(err, SSD_ERR_TIMEOUT);
                         *abort_flag = 1;
@@ -512,147 +569,135 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                 }
             }
             // the CTA does not exit with loads in flight
-            for (long long s = nx > L::kXSlots ? nx - L::kXSlots : 0; s < nx; ++s)
-                mbar_wait(&bars[PB_XF + (s & 1)], (s >> 1) & 1, err);
-            for (long long h = nbh > L::kBStages ? nbh - L::kBStages : 0; h < nbh; ++h)
+            for (int t = nx > L::kXSlots ? nx - L::kXSlots : 0; t < nx; ++t)
+                mbar_wait(&bars[PB_XF + (t & 1)], (t >> 1) & 1, err);
+            for (int h = nbh > L::kBStages ? nbh - L::kBStages : 0; h < nbh; ++h)
                 mbar_wait(&bars[PB_BF + h % L::kBStages], (h / L::kBStages) & 1, err);
             if (nc > 0) mbar_wait(&bars[PB_CF], (nc - 1) & 1, err);
         }
-    } else if (warp == kWarpMma) {
+    } else if (warp == kWarpMmaS) {
         if (lane == 0) {
-            // ------------------------------------------------ MMA issue, three polled streams
-            constexpr uint32_t idS = idesc_f16_f32(128, 128, true, true);     // B_k^T x X~ (fp16, MN-major)
-            constexpr uint32_t idO = idesc_bf16_f32(128, 128, false, true);   // C_k x images
-            constexpr uint32_t idD = idesc_bf16_f32(128, 64, false, true);    // P (TMEM) x X
-            const uint32_t aC = smem_u32(sm + L::kC), aXt = smem_u32(sm + L::kXt), aImg = smem_u32(sm + L::kImg);
-            long long ns = 0, no = 0, nd = 0;            // steps of S and Yo issued; heads of Yd issued
-            uint32_t idle = 0;
-            while (ns < total || no < total || nd < 2 * total) {
-                bool progressed = false;
-                if (ns < total) {
-                    const int st0 = (int)((2 * ns) % L::kBStages), st1 = (int)((2 * ns + 1) % L::kBStages);
-                    if (mbar_test_wait(&bars[PB_UPD], ns & 1) && mbar_test_wait(&bars[PB_CONV], ns & 1) &&
-                        mbar_test_wait(&bars[PB_BF + st0], ((2 * ns) / L::kBStages) & 1) &&
-                        mbar_test_wait(&bars[PB_BF + st1], ((2 * ns + 1) / L::kBStages) & 1)) {
-                        tc_fence_after();
-                        // S[n][64 j + p] += sum_t B_t[n] X~_t[j][p]: A = fp16 B (MN-major, n-halves
-                        // 8 KB apart), B = X~ (MN-major, heads 16 KB apart)
-#pragma unroll 1
-                        for (int ks = 0; ks < 8; ++ks) {
-                            const int st = ks < 4 ? st0 : st1;
-                            umma_f16(tmem + kColH,
-                                     smem_desc_sw128(smem_u32(sm + L::kB0 + st * L::kBStage) + (ks & 3) * 2048, 8192, 1024),
-                                     smem_desc_sw128(aXt + ks * 2048, kBox, 1024), idS, 1u);
-                            if (ks == 3) umma_commit(&bars[PB_BE + st0]);
-                        }
-                        umma_commit(&bars[PB_BE + st1]);
-                        umma_commit(&bars[PB_SD]);
-                        ++ns;
-                        progressed = true;
-                    }
-                }
-                if (no < ns && mbar_test_wait(&bars[PB_CF], no & 1) &&
-                    (no == 0 || (mbar_test_wait(&bars[PB_EPI], (no - 1) & 1) &&
-                                 mbar_test_wait(&bars[PB_EPI + 1], (no - 1) & 1)))) {
-                    tc_fence_after();
-                    // Yo[t][64 j + p] = sum_n C_t[n] H_j[n][p]: A = C (K-major), B = the images
-                    // (MN-major, 64-byte swizzle, the four 32-column blocks 8 KB apart)
-#pragma unroll 1
-                    for (int ks = 0; ks < 8; ++ks)
-                        umma_f16(tmem + kColYo, smem_desc_sw128(aC + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
-                                 smem_desc_sw64(aImg + ks * 1024, 8192, 512), idO, ks > 0 ? 1u : 0u);
-                    umma_commit(&bars[PB_CE]);
-                    umma_commit(&bars[PB_YO]);
-                    ++no;
-                    progressed = true;
-                }
-                if (nd < 2 * total) {
-                    const long long sd = nd >> 1;
-                    const int j = (int)(nd & 1);
-                    if (mbar_test_wait(&bars[PB_PF + j], sd & 1) &&
-                        mbar_test_wait(&bars[PB_XF + (sd & 1)], (sd >> 1) & 1) &&
-                        (sd == 0 || mbar_test_wait(&bars[PB_EPI + j], (sd - 1) & 1))) {
-                        tc_fence_after();
-                        const uint32_t aX = smem_u32(xslot(sd) + j * kBox);
-#pragma unroll 1
-                        for (int ks = 0; ks < 8; ++ks)
-                            umma_f16_ts(tmem + kColYd + 64 * j, tmem + kColP + 64 * j + ks * 8,
-                                        smem_desc_sw128(aX + ks * 2048, kBox, 1024), idD, ks > 0 ? 1u : 0u);
-                        umma_commit(&bars[PB_YD + j]);
-                        if (j == 1) umma_commit(&bars[PB_XE + (sd & 1)]);
-                        ++nd;
-                        progressed = true;
-                    }
-                }
-                if (progressed) {
-                    idle = 0;
-                } else if (++idle >= (1u << 24) || ((idle & 1023u) == 0 && *abort_flag)) {
-                    if (idle >= (1u << 24)) {
-                        record_error(err, SSD_ERR_TIMEOUT);
-                        *abort_flag = 1;
-                    }
+            // ------------------------------------------------ S = B_k^T [X~_0 | X~_1] onto the states
+            // A = fp16 B (MN-major, n-halves 8 KB apart), B = X~ (MN-major, heads 16 KB apart)
+            constexpr uint32_t idS = idesc_f16_f32(128, 128, true, true);
+            const uint32_t aXt = smem_u32(sm + L::kXt);
+            int ns = 0;
+            for (; ns < total; ++ns) {
+                const int st0 = (int)((2 * ns) % L::kBStages), st1 = (int)((2 * ns + 1) % L::kBStages);
+                if (!chain_wait(&bars[PB_UPD], ns & 1, err, abort_flag) ||
+                    !chain_wait(&bars[PB_CONV], ns & 1, err, abort_flag) ||
+                    !chain_wait(&bars[PB_BF + st0], ((2 * ns) / L::kBStages) & 1, err, abort_flag) ||
+                    !chain_wait(&bars[PB_BF + st1], ((2 * ns + 1) / L::kBStages) & 1, err, abort_flag))
                     break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int ks = 0; ks < 8; ++ks) {
+                    const int st = ks < 4 ? st0 : st1;
+                    umma_f16(tmem + kColH,
+                             smem_desc_sw128(smem_u32(sm + L::kB0 + st * L::kBStage) + (ks & 3) * 2048, 8192, 1024),
+                             smem_desc_sw128(aXt + ks * 2048, kBox, 1024), idS, 1u);
+                    if (ks == 3) umma_commit(&bars[PB_BE + st0]);
                 }
+                umma_commit(&bars[PB_BE + st1]);
+                umma_commit(&bars[PB_SD]);
             }
-            // the CTA does not release TMEM with MMAs in flight: every commit covers all earlier MMAs
-            if (nd > 0) mbar_wait(&bars[PB_YD + ((nd - 1) & 1)], ((nd - 1) >> 1) & 1, err);
-            if (no > 0) mbar_wait(&bars[PB_YO], (no - 1) & 1, err);
+            // the CTA does not release TMEM with MMAs in flight
             if (ns > 0) mbar_wait(&bars[PB_SD], (ns - 1) & 1, err);
         }
-    } else if (warp < kWarpP0) {
-        // ---------------------------------------------------- X~ = w o X, then the previous step's epilogue
+    } else if (warp == kWarpMmaO) {
+        if (lane == 0) {
+            // ------------------------------------------------ Yo = C_k [H_0 | H_1]
+            // A = C (K-major), B = the images (MN-major, 64-byte swizzle, the four 32-column
+            // blocks 8 KB apart); waits for the image (UPD), C, and the epilogue's reads of Yo
+            constexpr uint32_t idO = idesc_bf16_f32(128, 128, false, true);
+            const uint32_t aC = smem_u32(sm + L::kC), aImg = smem_u32(sm + L::kImg);
+            int no = 0;
+            for (; no < total; ++no) {
+                if (!chain_wait(&bars[PB_UPD], no & 1, err, abort_flag) ||
+                    !chain_wait(&bars[PB_CF], no & 1, err, abort_flag) ||
+                    (no > 0 && (!chain_wait(&bars[PB_EPI], (no - 1) & 1, err, abort_flag) ||
+                                !chain_wait(&bars[PB_EPI + 1], (no - 1) & 1, err, abort_flag))))
+                    break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_f16(tmem + kColYo, smem_desc_sw128(aC + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024),
+                             smem_desc_sw64(aImg + ks * 1024, 8192, 512), idO, ks > 0 ? 1u : 0u);
+                umma_commit(&bars[PB_CE]);
+                umma_commit(&bars[PB_YO]);
+            }
+            if (no > 0) mbar_wait(&bars[PB_YO], (no - 1) & 1, err);
+        }
+    } else if (warp == kWarpMmaD) {
+        if (lane == 0) {
+            // ------------------------------------------------ Yd_j += P_j X_j (onto D x)
+            constexpr uint32_t idD = idesc_bf16_f32(128, 64, false, true);
+            int nd = 0;
+            for (; nd < 2 * total; ++nd) {
+                const int sd = nd >> 1;
+                const int j = (int)(nd & 1);
+                if (!chain_wait(&bars[PB_PF + j], sd & 1, err, abort_flag) ||
+                    !chain_wait(&bars[PB_DXR + j], sd & 1, err, abort_flag) ||
+                    !chain_wait(&bars[PB_XF + (sd & 1)], (sd >> 1) & 1, err, abort_flag))
+                    break;
+                tc_fence_after();
+                const uint32_t aX = smem_u32(xslot(sd) + j * kBox);
+#pragma unroll 1
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_f16_ts(tmem + kColYd + 64 * j, tmem + kColP + 64 * j + ks * 8,
+                                smem_desc_sw128(aX + ks * 2048, kBox, 1024), idD, 1u);
+                umma_commit(&bars[PB_YD + j]);
+                if (j == 1) umma_commit(&bars[PB_XE + (sd & 1)]);
+            }
+            if (nd > 0) mbar_wait(&bars[PB_YD + ((nd - 1) & 1)], ((nd - 1) >> 1) & 1, err);
+        }
+    } else if (warp >= kWarpE0 && warp < kWarpP0) {
+        // ---------------------------------------------------- X~, the previous step's epilogue, D x
+        // Per step s: X~_s = w o X_s (the state GEMM's operand); the epilogue of step s - 1
+        // (y = Yd + exp(Lam_t) Yo, D x being in Yd already); then D x_s written into the freed
+        // Yd accumulators, onto which the Yd MMA of step s adds P X.  After that the step's x
+        // slot is no longer read here, so its refill does not wait for the epilogue.
         const int q = warp & 3;
         const int t = q * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
         StepIter it;
-        it.start(seq);
-        long long s = 0;
+        it.start(seq, um);
+        int s = 0;
         int pb = 0, pk = 0, ph0 = 0;                     // the previous step: batch, block, first head
-        float pD0 = 0.f, pD1 = 0.f;
+        float pu0 = 0.f, pu1 = 0.f;                      // and its exp(Lam_t) of both heads
 
-        // y = Yd + exp(Lam_t) Yo + D x of step ps, row t, heads j = 0, 1, stored to global memory
-        auto epilogue = [&](long long ps) -> bool {
+        // y = Yd + exp(Lam_t) Yo of step ps, row t, heads j = 0, 1, stored to global memory
+        auto epilogue = [&](int ps) -> bool {
             if (!wait_warp(PB_YO, ps & 1)) return false;
-            const uint8_t* sl = xslot(ps);
             for (int j = 0; j < 2; ++j) {
                 if (!wait_warp(PB_YD + j, ps & 1)) return false;
                 tc_fence_after();
-                const float u = expf(facp(ps, j)[t]);
-                const float Dh = j ? pD1 : pD0;
-                const uint8_t* xrow = sl + j * kBox + t * 128;
+                const float u = j ? pu1 : pu0;
                 __nv_bfloat16* yhead = y + ((size_t)pb * seqlen * nheads + ph0 + j) * kP;
                 const int rbase = pk * kBlk + q * 32 + (lane & ~3);     // the quad's first row
 #pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
-                    uint4 ch[4];
-#pragma unroll
-                    for (int qq = 0; qq < 2; ++qq) {
-                        const int col = 32 * half + 16 * qq;
-                        uint32_t yd[16], yo[16];
-                        tmem_ld16(tl + kColYd + 64 * j + col, yd);
-                        tmem_ld16(tl + kColYo + 64 * j + col, yo);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int hq = 0; hq < 2; ++hq) {
-                            const int cx = 4 * half + 2 * qq + hq;          // 16-byte chunk of the row
-                            const uint4 xu = *reinterpret_cast<const uint4*>(xrow + ((cx ^ (t & 7)) << 4));
-                            const uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w};
-                            uint32_t o[4];
-#pragma unroll
-                            for (int k2 = 0; k2 < 4; ++k2) {
-                                const int e = hq * 8 + 2 * k2;
-                                const float a0 = fmaf(u, __uint_as_float(yo[e]), __uint_as_float(yd[e])) + Dh * bf16lo(xw[k2]);
-                                const float a1 = fmaf(u, __uint_as_float(yo[e + 1]), __uint_as_float(yd[e + 1])) + Dh * bf16hi(xw[k2]);
-                                o[k2] = pack_bf16x2(a0, a1);
-                            }
-                            ch[2 * qq + hq] = make_uint4(o[0], o[1], o[2], o[3]);
-                        }
-                    }
+                    uint32_t yd[32], yo[32];
+                    tmem_ld32(tl + kColYd + 64 * j + 32 * half, yd);
+                    tmem_ld32(tl + kColYo + 64 * j + 32 * half, yo);
+                    tmem_wait_ld();
                     if (half == 1) {
                         // Yd and Yo of head j have been read
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&bars[PB_EPI + j]);
+                    }
+                    uint4 ch[4];
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        uint32_t o[4];
+#pragma unroll
+                        for (int k2 = 0; k2 < 4; ++k2) {
+                            const int e = 8 * c4 + 2 * k2;
+                            o[k2] = pack_bf16x2(fmaf(u, __uint_as_float(yo[e]), __uint_as_float(yd[e])),
+                                                fmaf(u, __uint_as_float(yo[e + 1]), __uint_as_float(yd[e + 1])));
+                        }
+                        ch[c4] = make_uint4(o[0], o[1], o[2], o[3]);
                     }
                     // four lanes write one row's 64 bytes of this half per store
                     transpose_quad(ch, lane);
@@ -664,24 +709,26 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                     }
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[PB_XE + (ps & 1)]);
             return true;
         };
 
         bool live = true;
         for (; it.valid() && live; it.next(), ++s) {
-            int b, g, h0;
-            um.map(it.unit(), &b, &g, &h0);
+            const int b = it.b, g = it.g, h0 = it.h0;
             const int k = it.block();
-            // X~_s (the state GEMM's operand): waits for the slot and for S of the previous step
+            const float d0 = D[h0], d1 = D[h0 + 1];
+            // X~_s: waits for the slot and for S of the previous step
             live = wait_warp(PB_XF + (s & 1), (s >> 1) & 1) && (s == 0 || wait_warp(PB_SD, (s - 1) & 1));
             if (!live) break;
             const uint8_t* sl = xslot(s);
+            float u0 = 0.f, u1 = 0.f;
 #pragma unroll 1
             for (int j = 0; j < 2; ++j) {
                 const float* sLam = facp(s, j);
                 const float w = expf(sLam[kBlk - 1] - sLam[t]) * sLam[kBlk + t];
+                const float u = expf(sLam[t]);
+                if (j) u1 = u;
+                else u0 = u;
                 const uint4* src = reinterpret_cast<const uint4*>(sl + j * kBox + t * 128);
                 uint4* dst = reinterpret_cast<uint4*>(sm + L::kXt + j * kBox + t * 128);
                 uint4 u8[8];
@@ -695,16 +742,47 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[PB_CONV]);
-            const float d0 = D[h0], d1 = D[h0 + 1];
-            if (s > 0) live = epilogue(s - 1);
+            if (s > 0) {
+                live = epilogue(s - 1);
+                if (!live) break;
+            }
+            // D x_s into the Yd accumulators the epilogue has just read (free at the first step)
+#pragma unroll 1
+            for (int j = 0; j < 2; ++j) {
+                const float Dh = j ? d1 : d0;
+                const uint8_t* xrow = sl + j * kBox + t * 128;
+#pragma unroll 1
+                for (int q16 = 0; q16 < 4; ++q16) {
+                    uint32_t v[16];
+#pragma unroll
+                    for (int hc = 0; hc < 2; ++hc) {
+                        const int cx = 2 * q16 + hc;                    // 16-byte chunk of the row
+                        const uint4 xu = *reinterpret_cast<const uint4*>(xrow + ((cx ^ (t & 7)) << 4));
+                        const uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w};
+#pragma unroll
+                        for (int k2 = 0; k2 < 4; ++k2) {
+                            v[8 * hc + 2 * k2] = __float_as_uint(Dh * bf16lo(xw[k2]));
+                            v[8 * hc + 2 * k2 + 1] = __float_as_uint(Dh * bf16hi(xw[k2]));
+                        }
+                    }
+                    tmem_st16(tl + kColYd + 64 * j + 16 * q16, v);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars[PB_DXR + j]);
+            }
+            // this step's x slot is no longer read by these warps
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[PB_XE + (s & 1)]);
             pb = b;
             pk = k;
             ph0 = h0;
-            pD0 = d0;
-            pD1 = d1;
+            pu0 = u0;
+            pu1 = u1;
         }
         if (live && s > 0) epilogue(s - 1);
-    } else {
+    } else if (warp >= kWarpP0 && warp < kWarpP0 + 8) {
         // ---------------------------------------------------- state of head c, then P_j
         // Warp (quarter q, c): TMEM lanes 32 q .. 32 q + 31.  The state part treats the lane as
         // state row n and owns head c's 64 columns; the P part treats it as row r of P_j and
@@ -716,8 +794,7 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
         const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
         const int kc0 = c, kc1 = c + 2;
         auto load_g = [&](const StepIter& at, uint4 (&gv)[8]) {
-            int b, g, h0;
-            um.map(at.unit(), &b, &g, &h0);
+            const int b = at.b, g = at.g, h0 = at.h0;
             const uint4* gk = gram + ((size_t)(b * ngroups + g) * nblk + at.block()) * (kGramBytes / 16);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -727,18 +804,17 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
         };
         griddep_wait();                                  // G and the hand-off flags come from earlier kernels
         StepIter it;
-        it.start(seq);
+        it.start(seq, um);
         // G of the current step; the next step's G is loaded once this step's P is built, and
         // lands while the next step's state update runs
         uint4 gv[8];
         if (it.valid()) load_g(it, gv);
         const uint32_t hc = tl + kColH + 64 * c;         // this warp's head's state columns
         const int sw = (r >> 1) & 3;
-        long long s = 0;
+        int s = 0;
         bool live = true;
         for (; it.valid() && live; it.next(), ++s) {
-            int b, g, h0;
-            um.map(it.unit(), &b, &g, &h0);
+            const int b = it.b, g = it.g, h0 = it.h0;
             const int k = it.block();
             // ---- state
             if (it.first()) {
@@ -777,24 +853,23 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                 const float e = expf(facp(s, c)[kBlk - 1]);
                 uint8_t* img = sm + L::kImg + c * kHImage + r * 64;
 #pragma unroll 1
-                for (int q16 = 0; q16 < 4; ++q16) {       // columns 16 q16 .. 16 q16 + 15
-                    uint32_t v[16];
-                    tmem_ld16(hc + 16 * q16, v);
+                for (int half = 0; half < 2; ++half) {    // columns 32 half .. 32 half + 31
+                    uint32_t v[32];
+                    tmem_ld32(hc + 32 * half, v);
                     tmem_wait_ld();
-                    uint8_t* half_row = img + (q16 >> 1) * 8192;
 #pragma unroll
-                    for (int j2 = 0; j2 < 2; ++j2) {
-                        const int jj = (q16 & 1) * 2 + j2;
-                        const uint32_t* h8 = &v[8 * j2];
-                        *reinterpret_cast<uint4*>(half_row + ((jj ^ sw) << 4)) = make_uint4(
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const uint32_t* h8 = &v[8 * jj];
+                        *reinterpret_cast<uint4*>(img + half * 8192 + ((jj ^ sw) << 4)) = make_uint4(
                             pack_bf16x2(__uint_as_float(h8[0]), __uint_as_float(h8[1])),
                             pack_bf16x2(__uint_as_float(h8[2]), __uint_as_float(h8[3])),
                             pack_bf16x2(__uint_as_float(h8[4]), __uint_as_float(h8[5])),
                             pack_bf16x2(__uint_as_float(h8[6]), __uint_as_float(h8[7])));
                     }
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(e * __uint_as_float(v[i]));
-                    tmem_st16(hc + 16 * q16, v);
+                    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(e * __uint_as_float(v[i]));
+                    tmem_st16(hc + 32 * half, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+                    tmem_st16(hc + 32 * half + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
                 }
                 tmem_wait_st();
                 fence_proxy_async_smem();                // image -> visible to the tensor cores
