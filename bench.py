@@ -3,18 +3,22 @@
 and cached decode steps/s (fraction of HBM bandwidth).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload prefill_130m|prefill_2p7b_long|decode_2p7b] [--no-extras]
+                    [--workload prefill_2p7b_long|prefill_130m|decode_2p7b|...] [--no-extras]
 
 One process per GPU (torchrun for N > 1).  Every rank runs its own independent
 problem (weak scaling, no collective on the data path); rank 0 prints one JSON line
 with the whole-job value = units of all ranks / max-over-ranks device time.
 
 Workloads (synthetic, seeded; the shapes of Mamba-2 SSD layers):
-  prefill_130m       bf16 x/B/C, fp32 dt/A/D/state: batch 8, 2048 tokens, 24 heads,
-                     P 64, N 128, 1 group, chunk 256                     (headline)
-  prefill_2p7b_long  batch 4, 16384 tokens, 80 heads, P 64, N 128, chunk 256
+  prefill_2p7b_long  bf16 x/B/C, fp32 dt/A/D/state: batch 4, 16384 tokens, 80 heads,
+                     P 64, N 128, 1 group, chunk 256 (the largest single-GPU prefill: headline)
+  prefill_130m       batch 8, 2048 tokens, 24 heads, P 64, N 128, chunk 256
   decode_2p7b        batch 64, 80 heads, P 64, N 128 fp32 state seeded by a 512-token
                      prefill; 1024 decode steps with fresh inputs, one CUDA graph
+  deep_decode_2p7b   64 layers of that shape at batch 256 (42.9 GB of fp32 states), one token
+                     per layer per step
+The headline run also measures the other workloads and ends its JSON line with a short
+"summary" of every workload's number.
 """
 from __future__ import annotations
 
@@ -38,6 +42,7 @@ if ROOT not in sys.path:
 from state_space_model_05_b200 import inputs as gen  # noqa: E402
 
 L2_BYTES = 126 * 2 ** 20
+HEADLINE = "prefill_2p7b_long"
 WORKLOADS = {
     "prefill_130m": dict(kind="prefill", batch=8, seqlen=2048, nheads=24, headdim=64, ngroups=1,
                          dstate=128, chunk_len=256, dtype="bf16"),
@@ -65,7 +70,7 @@ def tc_path(w) -> bool:
 
 def prefill_flops(w, q=None) -> dict:
     """Algorithmic (causal-exact) FLOPs per call for chunk length q (default: the configured
-    chunk), total and per kernel."""
+    chunk), total and each kernel's share (the cumsum kernel does no tensor work)."""
     b, T, H, P, G, N = (w[k] for k in ("batch", "seqlen", "nheads", "headdim", "ngroups", "dstate"))
     Q = q or w["chunk_len"]
     tokens = b * T
@@ -74,7 +79,9 @@ def prefill_flops(w, q=None) -> dict:
     cstate = tokens * H * 2 * N * P           # chunk states
     cout = tokens * H * 2 * N * P             # carried state -> output
     return {"total": gemm1 + gemm2 + cstate + cout,
-            "chunk_output": gemm1 + gemm2 + cout, "chunk_state": cstate}
+            "chunk_output_tc": gemm1 + gemm2 + cout, "chunk_output_simt": gemm1 + gemm2 + cout,
+            "chunk_state_scan_tc": cstate, "chunk_state_simt": cstate,
+            "block_gram_tc": gemm1, "chain_prefill_tc": gemm2 + cstate + cout}
 
 
 def prefill_bytes(w) -> dict:
@@ -624,29 +631,47 @@ def run_deep_decode(w, steps, warmup, rank, world, one_launch=True):
 
 
 def roofline_prefill(w, res, peaks, src, workload):
-    """Roofline of the dominant kernel.  The tensor-core path's kernels sit far below the
-    ridge point (the output kernel does ~60 FLOP per byte it must move), so they are
-    measured against HBM bandwidth; the CUDA-core chunk-state kernel against the tensor
-    peak (the work it stands in for)."""
-    byts = prefill_bytes(w)
+    """Roofline of the dominant kernel against the bf16 tensor peak: its share of the
+    chunked method's algorithmic (causal-exact) FLOPs per launch over its average launch
+    duration.  Beside it: the whole path's algorithmic bytes (x, dt, B and C read once, y
+    and the final state written once), the kernel's own design traffic, and the DRAM bytes
+    ncu measured for that kernel (null unless taken on the current sources)."""
     kernels = res["kernels"]
     dom = max(kernels, key=lambda k: kernels[k][0])
     ms, n = kernels[dom]
     per_launch_ms = ms / n
-    if dom in byts:
-        work = byts[dom]
-        achieved = work / (per_launch_ms / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s"}
-    else:
-        work = prefill_flops(w)["chunk_output" if dom.startswith("chunk_output") else "chunk_state"]
-        achieved = work / (per_launch_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s"}
-    roof.update({"frac": achieved / peak, "traffic": recorded_traffic(dom, workload), "kernel": dom,
-                 "kernel_ms": per_launch_ms, "algorithmic_bytes": work if roof["bound"] == "hbm" else None,
-                 "peak_source": src})
-    return roof
+    flops = prefill_flops(w).get(dom, 0)
+    achieved = flops / (per_launch_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops"]
+    design = prefill_bytes(w).get(dom)
+    traffic = recorded_traffic(dom, workload)
+    algo = prefill_bytes(w)["total"]
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": traffic, "kernel": dom, "kernel_ms": per_launch_ms, "kernel_flops": flops,
+            "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", peak),
+            "algorithmic_bytes": algo, "design_bytes": design,
+            "traffic_over_algorithmic": (traffic / algo) if traffic else None,
+            "peak_source": src, "peak_note": "burst cuBLAS bf16 (the kernel runs in a short timed region)"}
+
+
+def prefill_entry(w, workload, res, peaks, src):
+    """The numbers of one prefill workload (headline or extra)."""
+    sec = res["ms_per_step"] / 1e3
+    flops = prefill_flops(w)["total"]
+    out = {"value": res["tokens_per_s"], "unit": "tokens/s", "ms_per_step": res["ms_per_step"],
+           "prefill_tflops": flops / sec / 1e12, "prefill_tensor_frac": flops / sec / 1e12 / peaks["bf16_tflops"],
+           "prefill_hbm_gbs": prefill_bytes(w)["total"] / sec / 1e9,
+           "prefill_hbm_frac": prefill_bytes(w)["total"] / sec / 1e9 / peaks["hbm_gbs"],
+           "roofline": roofline_prefill(w, res, peaks, src, workload),
+           "kernels_ms": {k: v[0] / v[1] for k, v in res["kernels"].items()}}
+    if tc_path(w):
+        out["prefill_tflops_executed"] = prefill_flops(w, TC_BLOCK)["total"] / sec / 1e12
+    return out
+
+
+def decode_roofline(gbs, kernel, peaks, src, traffic=None):
+    return {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+            "traffic": traffic, "kernel": kernel, "peak_source": src}
 
 
 def ours(args, rank, world):
@@ -666,32 +691,30 @@ def ours(args, rank, world):
     line = {"metric": "", "value": None, "unit": "", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "data": "synthetic (seeded generators, state_space_model_05_b200/inputs.py)"}
+    summary = {}
+    solo = rank == 0 and world == 1 and not args.no_cpu_baseline
     if w["kind"] == "prefill":
         res = run_prefill(w, args.steps, args.warmup, rank, world, args.workload)
-        flops = prefill_flops(w)["total"]
+        entry = prefill_entry(w, args.workload, res, peaks, src)
         line.update({"metric": "SSD prefill tokens/s", "value": res["tokens_per_s"], "unit": "tokens/s",
                      "ms_per_step": res["ms_per_step"], "dtype": w["dtype"]})
-        sec = res["ms_per_step"] / 1e3
-        # tensor-peak fraction of the whole call: FLOPs of the chunked algorithm at the
-        # configured chunk, and (tensor-core path) at the 128-token blocks it executes
-        line["prefill_tflops"] = flops / sec / 1e12
-        line["prefill_tensor_frac"] = line["prefill_tflops"] / peaks["bf16_tflops"]
-        if tc_path(w):
-            line["prefill_tflops_executed"] = prefill_flops(w, TC_BLOCK)["total"] / sec / 1e12
-        line["prefill_hbm_gbs"] = prefill_bytes(w)["total"] / sec / 1e9
-        line["roofline"] = roofline_prefill(w, res, peaks, src, args.workload)
+        line["roofline"] = entry.pop("roofline")
+        for k in ("prefill_tflops", "prefill_tensor_frac", "prefill_tflops_executed", "prefill_hbm_gbs",
+                  "prefill_hbm_frac", "kernels_ms"):
+            if k in entry:
+                line[k] = entry[k]
         line["e2e"] = res.get("e2e")
         line["gpu_launches"] = res["launches"]
-        line["kernels_ms"] = {k: v[0] / v[1] for k, v in res["kernels"].items()}
         cfg = {"workload": args.workload, **{k: w[k] for k in w if k != "kind"},
                "l2": f"inputs rotated over {res['replicas']} resident replicas (> 3x L2) between steps"}
+        summary[args.workload] = {"tok_s": round(res["tokens_per_s"]), "ms": round(res["ms_per_step"], 4),
+                                  "tensor_frac": round(line["prefill_tensor_frac"], 4),
+                                  "kernel_frac": round(line["roofline"]["frac"], 4)}
     elif w["kind"] == "gdn":
         res = run_gdn(w, max(1, args.steps // 100), max(1, args.warmup // 3), rank, world)
         line.update({"metric": "GDN decode steps/s", "value": res["steps_per_s"], "unit": "steps/s",
                      "ms_per_step": res["us_per_step"] / 1e3, "dtype": "f32"})
-        line["roofline"] = {"bound": "hbm", "achieved": res["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                            "frac": res["gbs"] / peaks["hbm_gbs"], "traffic": None,
-                            "kernel": "gdn_decode_step", "peak_source": src}
+        line["roofline"] = decode_roofline(res["gbs"], "gdn_decode_step", peaks, src)
         line["gpu_launches"] = res["launches"]
         line["e2e"] = None
         cfg = {"workload": args.workload, **{k: w[k] for k in w if k != "kind"}}
@@ -699,107 +722,118 @@ def ours(args, rank, world):
         res = run_deep_decode(w, args.steps, 3, rank, world)
         line.update({"metric": "SSD decode steps/s (64-layer stack)", "value": res["steps_per_s"],
                      "unit": "steps/s", "ms_per_step": res["ms_per_step"], "dtype": "f32"})
-        line["roofline"] = {"bound": "hbm", "achieved": res["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                            "frac": res["gbs"] / peaks["hbm_gbs"], "traffic": None,
-                            "kernel": "decode_layers (all layers, one launch per step)", "peak_source": src}
+        line["roofline"] = decode_roofline(res["gbs"], "decode_layers (all layers, one launch per step)", peaks, src)
         line["gpu_launches"] = res["launches"]
         line["e2e"] = None
         cfg = {"workload": args.workload, **{k: w[k] for k in w if k != "kind"}}
+        if solo:
+            line["cpu_baseline"] = cpu_baseline_decode(w, budget_s=8.0)
     else:
         res = run_decode(w, max(1, args.steps // 100), max(1, args.warmup // 3), rank, world)
         line.update({"metric": "SSD decode steps/s", "value": res["steps_per_s"], "unit": "steps/s",
                      "ms_per_step": res["ms_per_step"], "dtype": "f32"})
         kgbs = res["bytes_per_step"] / (res["ms_per_step"] / 1e3) / 1e9
-        line["roofline"] = {"bound": "hbm", "achieved": kgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                            "frac": kgbs / peaks["hbm_gbs"], "traffic": recorded_traffic("decode_step", args.workload),
-                            "kernel": "decode_step", "peak_source": src}
+        line["roofline"] = decode_roofline(kgbs, "decode_step", peaks, src,
+                                           recorded_traffic("decode_step", args.workload))
         line["gpu_launches"] = res["launches"]
         line["e2e"] = None
         cfg = {"workload": args.workload, **{k: w[k] for k in w if k != "kind"}}
+        if solo:
+            line["cpu_baseline"] = cpu_baseline_decode(w, budget_s=8.0)
     cfg["parallelism"] = f"independent problem per GPU x{world}"
     if args.prefill_path != "auto":
         cfg["prefill_path"] = args.prefill_path
     line["config"] = cfg
 
-    if not args.no_extras and args.workload == "prefill_130m":
+    if not args.no_extras and args.workload == HEADLINE:
+        extras = {}
+        # the 130M-shaped layer (the other prefill configuration), on the default path
+        pw = WORKLOADS["prefill_130m"]
+        r = run_prefill(pw, 100, 5, rank, world, "prefill_130m", e2e=False)
+        e = prefill_entry(pw, "prefill_130m", r, peaks, src)
+        e["config"] = {k: pw[k] for k in pw if k != "kind"}
+        extras["prefill_130m"] = e
+        summary["prefill_130m"] = {"tok_s": round(r["tokens_per_s"]), "ms": round(r["ms_per_step"], 4),
+                                   "tensor_frac": round(e["prefill_tensor_frac"], 4),
+                                   "kernel_frac": round(e["roofline"]["frac"], 4)}
+        # both prefill workloads on each tensor-core path, for comparison with the default
+        for path in ("fused", "two_pass"):
+            prev_path = _binding.ssd_set_prefill_path(path)
+            try:
+                for name in (args.workload, "prefill_130m"):
+                    pw2 = WORKLOADS[name]
+                    r = run_prefill(pw2, 20 if name == args.workload else 100, 3, rank, world, f"{name}_{path}", e2e=False)
+                    extras[f"{name}_{path}_path"] = {"value": r["tokens_per_s"], "unit": "tokens/s",
+                                                     "ms_per_step": r["ms_per_step"],
+                                                     "kernels_ms": {k: v[0] / v[1] for k, v in r["kernels"].items()}}
+                    summary[f"{name}_{path}"] = {"tok_s": round(r["tokens_per_s"]), "ms": round(r["ms_per_step"], 4)}
+            finally:
+                _binding.ssd_set_prefill_path(prev_path)
+        # cached decode: 1024 steps in one CUDA graph; every launch in the timed graph is a
+        # decode kernel, so the average launch duration is the timed region over the launches
         dw = WORKLOADS["decode_2p7b"]
         d = run_decode(dw, 3, 1, rank, world)
-        # every launch in the timed graph is a decode kernel: the average launch duration is
-        # the timed region over the launches (the per-launch event pairs of the instrumented
-        # replay add their own overhead and are reported beside it)
         kgbs = d["bytes_per_step"] / (d["ms_per_step"] / 1e3) / 1e9
-        line["decode_2p7b"] = {"value": d["steps_per_s"], "unit": "steps/s", "ms_per_step": d["ms_per_step"],
-                               "kernel_ms_event_pairs": d["kernel_ms"], "roofline": {
-                                   "bound": "hbm", "achieved": kgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                   "frac": kgbs / peaks["hbm_gbs"], "kernel": "decode_step",
-                                   "traffic": recorded_traffic("decode_step", "decode_2p7b"), "peak_source": src},
-                               "config": {k: dw[k] for k in dw if k != "kind"}}
+        extras["decode_2p7b"] = {"value": d["steps_per_s"], "unit": "steps/s", "ms_per_step": d["ms_per_step"],
+                                 "kernel_ms_event_pairs": d["kernel_ms"],
+                                 "roofline": decode_roofline(kgbs, "decode_step", peaks, src,
+                                                             recorded_traffic("decode_step", "decode_2p7b")),
+                                 "config": {k: dw[k] for k in dw if k != "kind"}}
+        summary["decode_2p7b"] = {"steps_s": round(d["steps_per_s"]), "us": round(d["ms_per_step"] * 1e3, 2),
+                                  "hbm_frac": round(kgbs / peaks["hbm_gbs"], 4)}
         ddw = WORKLOADS["deep_decode_2p7b"]
         dd = run_deep_decode(ddw, 64, 3, rank, world, one_launch=True)
-        dp = run_deep_decode(ddw, 64, 3, rank, world, one_launch=False)
-        line["deep_decode_2p7b"] = {"value": dd["steps_per_s"], "unit": "steps/s", "ms_per_step": dd["ms_per_step"],
-                                    "steps_timed": dd["steps"], "launches_per_step": 1, "roofline": {
-                                        "bound": "hbm", "achieved": dd["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                        "frac": dd["gbs"] / peaks["hbm_gbs"], "kernel": "decode_layers (64 layers, one launch)",
-                                        "peak_source": src},
-                                    "per_layer_launches": {"value": dp["steps_per_s"], "ms_per_step": dp["ms_per_step"],
-                                                           "gbs": dp["gbs"], "launches_per_step": ddw["layers"]},
-                                    "config": {k: ddw[k] for k in ddw if k != "kind"}}
-        # the same headline prefill with dt = softplus(dt_raw + dt_bias) formed in the kernels
-        r = run_prefill(w, 100, 5, rank, world, "prefill_130m_dtraw", e2e=False, dt_softplus=True)
-        line["prefill_130m_dt_softplus"] = {"value": r["tokens_per_s"], "unit": "tokens/s",
-                                            "ms_per_step": r["ms_per_step"],
-                                            "kernels_ms": {k: v[0] / v[1] for k, v in r["kernels"].items()}}
-        # the same headline prefill on the fused tensor-core path (opt-in; the default two-pass
-        # kernels are faster on this workload)
-        from state_space_model_05_b200 import binding as _binding
-        prev_path = _binding.ssd_set_prefill_path("fused")
-        try:
-            r = run_prefill(w, 100, 5, rank, world, "prefill_130m_fused", e2e=False)
-        finally:
-            _binding.ssd_set_prefill_path(prev_path)
-        line["prefill_130m_fused_path"] = {"value": r["tokens_per_s"], "unit": "tokens/s",
-                                           "ms_per_step": r["ms_per_step"],
-                                           "kernels_ms": {k: v[0] / v[1] for k, v in r["kernels"].items()}}
-        # the same tokens as one packed batch of mixed-length sequences (state reset per sequence)
-        vr = run_prefill_varlen(w, 100, 5, rank, world)
-        line["prefill_130m_varlen"] = {"value": vr["tokens_per_s"], "unit": "tokens/s",
-                                       "ms_per_step": vr["ms_per_step"], "sequences": vr["lengths"]}
+        dp = run_deep_decode(ddw, 16, 3, rank, world, one_launch=False)
+        extras["deep_decode_2p7b"] = {"value": dd["steps_per_s"], "unit": "steps/s", "ms_per_step": dd["ms_per_step"],
+                                      "steps_timed": dd["steps"], "launches_per_step": 1,
+                                      "roofline": decode_roofline(dd["gbs"], "decode_layers (64 layers, one launch)",
+                                                                  peaks, src),
+                                      "per_layer_launches": {"value": dp["steps_per_s"], "ms_per_step": dp["ms_per_step"],
+                                                             "gbs": dp["gbs"], "launches_per_step": ddw["layers"]},
+                                      "config": {k: ddw[k] for k in ddw if k != "kind"}}
+        summary["deep_decode_2p7b"] = {"steps_s": round(dd["steps_per_s"], 2), "ms": round(dd["ms_per_step"], 3),
+                                       "hbm_frac": round(dd["gbs"] / peaks["hbm_gbs"], 4)}
+        # the headline prefill with dt = softplus(dt_raw + dt_bias) formed in the kernels
+        r = run_prefill(pw, 100, 5, rank, world, "prefill_130m_dtraw", e2e=False, dt_softplus=True)
+        extras["prefill_130m_dt_softplus"] = {"value": r["tokens_per_s"], "unit": "tokens/s",
+                                              "ms_per_step": r["ms_per_step"]}
+        # the 130M workload's tokens as one packed batch of mixed-length sequences
+        vr = run_prefill_varlen(pw, 100, 5, rank, world)
+        extras["prefill_130m_varlen"] = {"value": vr["tokens_per_s"], "unit": "tokens/s",
+                                         "ms_per_step": vr["ms_per_step"], "sequences": vr["lengths"]}
         for name in ("gdn_decode_b1", "gdn_decode_b64"):
             gw = WORKLOADS[name]
             r = run_gdn(gw, 3, 1, rank, world)
-            line[name] = {"value": r["steps_per_s"], "unit": "steps/s", "us_per_step": r["us_per_step"],
-                          "roofline": {"bound": "hbm", "achieved": r["gbs"], "peak": peaks["hbm_gbs"],
-                                       "unit": "GB/s", "frac": r["gbs"] / peaks["hbm_gbs"],
-                                       "kernel": "gdn_decode_step", "peak_source": src,
-                                       "note": "state L2-resident" if gw["batch"] == 1 else "state in HBM"},
-                          "config": {k: gw[k] for k in gw if k != "kind"}}
-        lw = WORKLOADS["prefill_2p7b_long"]
-        l = run_prefill(lw, 5, 2, rank, world, "prefill_2p7b_long", e2e=False)
-        fl = prefill_flops(lw)["total"]
-        lsec = l["ms_per_step"] / 1e3
-        line["prefill_2p7b_long"] = {"value": l["tokens_per_s"], "unit": "tokens/s", "ms_per_step": l["ms_per_step"],
-                                     "prefill_tflops": fl / lsec / 1e12,
-                                     "prefill_tensor_frac": fl / lsec / 1e12 / peaks["bf16_tflops"],
-                                     "prefill_tflops_executed": prefill_flops(lw, TC_BLOCK)["total"] / lsec / 1e12,
-                                     "prefill_hbm_gbs": prefill_bytes(lw)["total"] / lsec / 1e9,
-                                     "roofline": roofline_prefill(lw, l, peaks, src, "prefill_2p7b_long"),
-                                     "kernels_ms": {k: v[0] / v[1] for k, v in l["kernels"].items()}}
+            extras[name] = {"value": r["steps_per_s"], "unit": "steps/s", "us_per_step": r["us_per_step"],
+                            "roofline": dict(decode_roofline(r["gbs"], "gdn_decode_step", peaks, src),
+                                             note="state L2-resident" if gw["batch"] == 1 else "state in HBM"),
+                            "config": {k: gw[k] for k in gw if k != "kind"}}
+            summary[name] = {"steps_s": round(r["steps_per_s"]), "us": round(r["us_per_step"], 2),
+                             "hbm_frac": round(r["gbs"] / peaks["hbm_gbs"], 4)}
+        if solo:
+            extras["prefill_130m"]["cpu_baseline"] = cpu_baseline(pw, budget_s=6.0)
+            extras["decode_2p7b"]["cpu_baseline"] = cpu_baseline_decode(dw, budget_s=6.0)
+            extras["deep_decode_2p7b"]["cpu_baseline"] = cpu_baseline_decode(ddw, budget_s=6.0)
+        line.update(extras)
     line["clocks"] = clocks.stop()
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and w["kind"] == "prefill":
+    if solo and w["kind"] == "prefill":
         line["cpu_baseline"] = cpu_baseline(w, budget_s=20.0)
+    # last, so that a reader of the end of the output sees every workload's number
+    line["summary"] = summary
     return line
 
 
 # ------------------------------------------------------------------ oracle timing
-def oracle_sample_step(w, inp, units):
+def oracle_sample_step(w, inp, units, nthreads=0):
     import oracle
     t = time.perf_counter()
-    oracle.prefill(inp.x, inp.dt, inp.A, inp.B, inp.C, inp.D, units=units)
+    oracle.prefill(inp.x, inp.dt, inp.A, inp.B, inp.C, inp.D, units=units, nthreads=nthreads)
     return time.perf_counter() - t
 
 
 def cpu_baseline(w, budget_s=20.0):
+    """The fp64 oracle on a bounded sample of the prefill workload's (batch, head) units, on
+    all host cores, and on one core for one unit."""
     import oracle
     oracle.build()
     inp = prefill_problem(w, seed=0)
@@ -811,10 +845,54 @@ def cpu_baseline(w, budget_s=20.0):
     n = int(min(n_all, max(len(probe), budget_s / max(per_unit, 1e-9))))
     units = list(range(n))
     t = oracle_sample_step(w, inp, units)
+    t_one = oracle_sample_step(w, inp, [0], nthreads=1)
     tokens = n / H * T
     return {"value": tokens / t, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "single_core": {"value": T / H / t_one, "unit": "tokens/s", "cores": 1},
             "sample": f"{n} of {n_all} (batch, head) units of the {w['batch']}x{T}-token workload, "
-                      f"fp64 sequential recurrence, {t:.2f} s"}
+                      f"fp64 sequential recurrence, {t:.2f} s; one unit on one core, {t_one:.2f} s"}
+
+
+def _decode_units(w):
+    """(units per step, batch, heads) of a decode workload (a unit is one (layer, b, h))."""
+    layers = w.get("layers", 1)
+    return layers * w["batch"] * w["nheads"], w["batch"], w["nheads"]
+
+
+def oracle_decode_rate(w, budget_s, nthreads=0, seed=0):
+    """Decode steps/s of the fp64 oracle: steps of a sample of units (one layer's batch and
+    heads), scaled to the workload's units per step."""
+    import oracle
+    oracle.build()
+    per_step, b, H = _decode_units(w)
+    P, G, N = w["headdim"], w["ngroups"], w["dstate"]
+    shape = gen.SSDShape(b, 1, H, P, G, N)
+    dec = gen.decode_inputs(shape, steps=4, seed=seed + 7)
+    hp = gen.prefill_inputs(gen.SSDShape(1, 1, H, P, G, N), seed=seed)
+    n_all = b * H
+    cores = oracle.threads(nthreads) if nthreads else oracle.threads()
+    units = list(range(min(n_all, max(64, 64 * cores))))
+    state = gen.state_inputs(1, len(units), P, N, seed=seed + 8)[0].astype(np.float64)
+    t0, steps = time.perf_counter(), 0
+    while True:
+        k = steps % 4
+        oracle.decode_step(state, dec.x[k], dec.dt[k], hp.A, dec.B[k], dec.C[k], hp.D, units=units, nthreads=nthreads)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or steps >= 4096:
+            break
+    unit_steps_per_s = len(units) * steps / el
+    return unit_steps_per_s / per_step, len(units), steps, el, cores
+
+
+def cpu_baseline_decode(w, budget_s=6.0):
+    rate, nu, st, el, cores = oracle_decode_rate(w, budget_s)
+    one, nu1, st1, el1, _ = oracle_decode_rate(w, max(1.0, budget_s / 4), nthreads=1)
+    per_step, _, _ = _decode_units(w)
+    return {"value": rate, "unit": "steps/s", "cores": cores, "kind": "oracle",
+            "single_core": {"value": one, "unit": "steps/s", "cores": 1},
+            "sample": f"{st} steps of {nu} of the {per_step} (layer, batch, head) units a step, fp64, "
+                      f"{el:.2f} s, scaled to whole steps; one core: {st1} steps of {nu1} units, {el1:.2f} s"}
 
 
 def reference(args, rank, world):
@@ -822,8 +900,26 @@ def reference(args, rank, world):
     import oracle
     oracle.build()
     w = WORKLOADS[args.workload]
+    cfg = {"workload": args.workload, **{k: w[k] for k in w if k != "kind"}}
+    base = {"impl": "reference", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "config": cfg}
+    if w["kind"] in ("decode", "deep_decode"):
+        budget = 150.0 / max(1, args.steps + args.warmup)
+        for _ in range(args.warmup):
+            oracle_decode_rate(w, budget / 4)
+        rates = [oracle_decode_rate(w, budget) for _ in range(args.steps)]
+        value = statistics.mean(r[0] for r in rates)
+        nu, st = rates[0][1], rates[0][2]
+        per_step, _, _ = _decode_units(w)
+        sample = f"each step: {st} decode steps of {nu} of the {per_step} units a step, scaled to whole steps"
+        metric = "SSD decode steps/s" if w["kind"] == "decode" else "SSD decode steps/s (64-layer stack)"
+        return dict(base, metric=metric, value=value, unit="steps/s", ms_per_step=1e3 / value,
+                    cpu_baseline={"value": value, "unit": "steps/s", "cores": oracle.threads(), "kind": "oracle",
+                                  "sample": sample},
+                    e2e={"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
     if w["kind"] != "prefill":
-        return {"impl": "reference", "unavailable": "the oracle reference arm times the prefill workloads"}
+        return {"impl": "reference", "unavailable": "the oracle reference arm times the SSD prefill and decode workloads"}
     inp = prefill_problem(w, seed=0)
     H, T = w["nheads"], w["seqlen"]
     n_all = w["batch"] * H
@@ -838,14 +934,11 @@ def reference(args, rank, world):
     tokens = n / H * T * args.steps
     value = tokens / total
     sample = f"{n} of {n_all} (batch, head) units per step of the {w['batch']}x{T}-token workload"
-    return {"impl": "reference", "metric": "SSD prefill tokens/s", "value": value, "unit": "tokens/s",
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": total / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-            "config": {"workload": args.workload, **{k: w[k] for k in w if k != "kind"}},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(),
-                             "kind": "oracle", "sample": sample},
-            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return dict(base, metric="SSD prefill tokens/s", value=value, unit="tokens/s",
+                ms_per_step=total / args.steps * 1e3,
+                cpu_baseline={"value": value, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+                              "sample": sample},
+                e2e={"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
 
 
 def main(argv=None):
@@ -854,7 +947,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill_130m")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=HEADLINE)
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-path", choices=["auto", "fused", "two_pass"], default="auto",

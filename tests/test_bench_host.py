@@ -68,11 +68,22 @@ def test_roofline_prefill_record():
                        "chunk_output_tc": (5.0, 100)}}
     peaks = {"hbm_gbs": 6545.3, "bf16_tflops": 1651.2}
     r = bench.roofline_prefill(w, res, peaks, "measured", "prefill_130m")
-    assert r["kernel"] == "chunk_output_tc" and r["bound"] == "hbm" and r["unit"] == "GB/s"
-    expect = bench.prefill_bytes(w)["chunk_output_tc"] / (0.05e-3) / 1e9
+    # the prefill is a dense contraction: measured against the tensor peak, with the dominant
+    # kernel's share of the causal-exact FLOPs per launch over its launch duration
+    assert r["kernel"] == "chunk_output_tc" and r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    b, T, H, P, N = 8, 2048, 24, 64, 128
+    flops = b * T * (257 * N + H * (257 * P + 2 * N * P))      # C B^T, masked X, state -> output
+    assert r["kernel_flops"] == flops
+    expect = flops / (0.05e-3) / 1e12
     assert abs(r["achieved"] - expect) < 1e-6 * expect
-    assert abs(r["frac"] - r["achieved"] / 6545.3) < 1e-12
+    assert abs(r["frac"] - r["achieved"] / 1651.2) < 1e-12
+    # the path's algorithmic bytes: x, dt, B, C read once, y and the final state written once
+    assert r["algorithmic_bytes"] == b * T * (2 * H * P * 2 + 2 * N * 2 + H * 4) + b * H * P * N * 4
     assert set(r) >= {"bound", "achieved", "peak", "unit", "frac", "traffic"}
+    # the fused path's dominant kernel carries every GEMM but C B^T
+    fused = bench.roofline_prefill(w, {"kernels": {"chain_prefill_tc": (3.0, 100), "block_gram_tc": (0.5, 100)}},
+                                   peaks, "measured", "prefill_130m")
+    assert fused["kernel_flops"] == b * T * H * (257 * P + 4 * N * P)
 
 
 def test_reference_arm_line(monkeypatch, capsys):
@@ -83,7 +94,7 @@ def test_reference_arm_line(monkeypatch, capsys):
     monkeypatch.setenv("WORLD_SIZE", "1")
     # the oracle's per-step sample is sized from this budget: keep the test to seconds
     monkeypatch.setattr(bench, "oracle_sample_step", _fast_sample(bench.oracle_sample_step))
-    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"]) == 0
+    assert bench.main(["--impl", "reference", "--workload", "prefill_130m", "--steps", "1", "--warmup", "3"]) == 0
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
                 "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
@@ -97,6 +108,21 @@ def test_reference_arm_line(monkeypatch, capsys):
                            "d2h_bytes_per_step": 0}
 
 
+def test_reference_arm_decode_line(monkeypatch, capsys):
+    """The decode workloads' reference arm: the oracle's decode steps on a sample of units,
+    scaled to whole steps."""
+    import json
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    real = bench.oracle_decode_rate
+    monkeypatch.setattr(bench, "oracle_decode_rate", lambda w, budget, nthreads=0, seed=0: real(w, 0.05, nthreads, seed))
+    assert bench.main(["--impl", "reference", "--workload", "decode_2p7b", "--steps", "1", "--warmup", "3"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == "SSD decode steps/s" and line["unit"] == "steps/s"
+    assert line["value"] > 0 and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["value"] == line["value"] and line["config"]["workload"] == "decode_2p7b"
+
+
 def test_reference_arm_other_ranks_do_nothing(monkeypatch, capsys):
     monkeypatch.setenv("RANK", "1")
     monkeypatch.setenv("WORLD_SIZE", "2")
@@ -107,6 +133,6 @@ def test_reference_arm_other_ranks_do_nothing(monkeypatch, capsys):
 
 def _fast_sample(step):
     """The real oracle step on at most two (batch, head) units."""
-    def run(w, inp, units):
-        return step(w, inp, list(units)[:2])
+    def run(w, inp, units, nthreads=0):
+        return step(w, inp, list(units)[:2], nthreads)
     return run
