@@ -339,38 +339,41 @@ def run_prefill(w, steps, warmup, rank, world, name, e2e=True, dt_softplus=False
            "kernels": kernels, "replicas": replicas, "launches": int(round(launches_per_step * steps))}
 
     if e2e:
-        # end to end through the public call with host buffers: H2D inputs, prefill, D2H outputs
+        # end to end through the library's host-buffer entry (HostPrefill): every step copies
+        # that step's inputs in from pinned host memory and y and the final state back out,
+        # with step i's outputs travelling while step i + 1's inputs arrive and are computed
+        from state_space_model_05_b200.host_pipeline import HostPrefill
         pin = lambda a, d: torch.from_numpy(np.ascontiguousarray(a)).to(d).pin_memory()
         hx, hdt, hB, hC = pin(inp.x, dt_), pin(inp.dt, torch.float32), pin(inp.B, dt_), pin(inp.C, dt_)
-        hy = torch.empty((b, T, H, P), dtype=dt_).pin_memory()
-        hst = torch.empty((b, H, P, N), dtype=torch.float32).pin_memory()
-        r = reps[0]
+        outs = [(torch.empty((b, T, H, P), dtype=dt_).pin_memory(),
+                 torch.empty((b, H, P, N), dtype=torch.float32).pin_memory()) for _ in range(2)]
+        del reps
+        torch.cuda.empty_cache()
+        pipe = HostPrefill(b, T, H, P, G, N, Q, dt_, _dev(inp.A, torch.float32), _dev(inp.D, torch.float32))
 
-        def e2e_step():
-            r["x"].copy_(hx, non_blocking=True)
-            r["dt"].copy_(hdt, non_blocking=True)
-            r["B"].copy_(hB, non_blocking=True)
-            r["C"].copy_(hC, non_blocking=True)
-            ssd.ssd_prefill(r["x"], r["dt"], r["A"], r["B"], r["C"], r["D"], Q, y=r["y"],
-                            final_state=r["st"], workspace=r["ws"])
-            hy.copy_(r["y"], non_blocking=True)
-            hst.copy_(r["st"], non_blocking=True)
+        def e2e_run(n):
+            for i in range(n):
+                hy, hst = outs[i % 2]
+                pipe.submit(hx, hdt, hB, hC, hy, hst)
 
-        for _ in range(max(1, warmup)):
-            e2e_step()
+        e2e_run(max(2, warmup))
+        pipe.synchronize()
         barrier(world)
         torch.cuda.synchronize()
-        s0.record()
-        for _ in range(steps):
-            e2e_step()
-        s1.record()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(pipe.copy_in)
+        e2e_run(steps)
+        t1.record(pipe.copy_out)
+        pipe.synchronize()
         torch.cuda.synchronize()
         barrier(world)
-        erate, _ = whole_job_rate(b * T * steps, s0.elapsed_time(s1), world)
+        erate, _ = whole_job_rate(b * T * steps, t0.elapsed_time(t1), world)
         h2d = sum(t.numel() * t.element_size() for t in (hx, hdt, hB, hC))
+        hy, hst = outs[0]
         d2h = hy.numel() * hy.element_size() + hst.numel() * hst.element_size()
         res["e2e"] = {"value": erate, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                      "d2h_bytes_per_step": d2h}
+                      "d2h_bytes_per_step": d2h,
+                      "path": "HostPrefill: copies in and out overlapped with compute (two device buffer sets)"}
     return res
 
 
@@ -824,10 +827,19 @@ def ours(args, rank, world):
 
 
 # ------------------------------------------------------------------ oracle timing
+def host_cores() -> int:
+    """The host cores this process may run on (the oracle's all-core runs use them all; the
+    thread count is passed on every call, since an OpenMP thread-count setting persists)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
 def oracle_sample_step(w, inp, units, nthreads=0):
     import oracle
     t = time.perf_counter()
-    oracle.prefill(inp.x, inp.dt, inp.A, inp.B, inp.C, inp.D, units=units, nthreads=nthreads)
+    oracle.prefill(inp.x, inp.dt, inp.A, inp.B, inp.C, inp.D, units=units, nthreads=nthreads or host_cores())
     return time.perf_counter() - t
 
 
@@ -839,7 +851,7 @@ def cpu_baseline(w, budget_s=20.0):
     inp = prefill_problem(w, seed=0)
     H, T = w["nheads"], w["seqlen"]
     n_all = w["batch"] * H
-    probe = list(range(min(n_all, max(1, oracle.threads()))))
+    probe = list(range(min(n_all, host_cores())))
     t1 = oracle_sample_step(w, inp, probe)
     per_unit = t1 / len(probe)
     n = int(min(n_all, max(len(probe), budget_s / max(per_unit, 1e-9))))
@@ -847,7 +859,7 @@ def cpu_baseline(w, budget_s=20.0):
     t = oracle_sample_step(w, inp, units)
     t_one = oracle_sample_step(w, inp, [0], nthreads=1)
     tokens = n / H * T
-    return {"value": tokens / t, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+    return {"value": tokens / t, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
             "single_core": {"value": T / H / t_one, "unit": "tokens/s", "cores": 1},
             "sample": f"{n} of {n_all} (batch, head) units of the {w['batch']}x{T}-token workload, "
                       f"fp64 sequential recurrence, {t:.2f} s; one unit on one core, {t_one:.2f} s"}
@@ -870,13 +882,13 @@ def oracle_decode_rate(w, budget_s, nthreads=0, seed=0):
     dec = gen.decode_inputs(shape, steps=4, seed=seed + 7)
     hp = gen.prefill_inputs(gen.SSDShape(1, 1, H, P, G, N), seed=seed)
     n_all = b * H
-    cores = oracle.threads(nthreads) if nthreads else oracle.threads()
+    cores = nthreads or host_cores()
     units = list(range(min(n_all, max(64, 64 * cores))))
     state = gen.state_inputs(1, len(units), P, N, seed=seed + 8)[0].astype(np.float64)
     t0, steps = time.perf_counter(), 0
     while True:
         k = steps % 4
-        oracle.decode_step(state, dec.x[k], dec.dt[k], hp.A, dec.B[k], dec.C[k], hp.D, units=units, nthreads=nthreads)
+        oracle.decode_step(state, dec.x[k], dec.dt[k], hp.A, dec.B[k], dec.C[k], hp.D, units=units, nthreads=cores)
         steps += 1
         el = time.perf_counter() - t0
         if el >= budget_s or steps >= 4096:
@@ -915,7 +927,7 @@ def reference(args, rank, world):
         sample = f"each step: {st} decode steps of {nu} of the {per_step} units a step, scaled to whole steps"
         metric = "SSD decode steps/s" if w["kind"] == "decode" else "SSD decode steps/s (64-layer stack)"
         return dict(base, metric=metric, value=value, unit="steps/s", ms_per_step=1e3 / value,
-                    cpu_baseline={"value": value, "unit": "steps/s", "cores": oracle.threads(), "kind": "oracle",
+                    cpu_baseline={"value": value, "unit": "steps/s", "cores": host_cores(), "kind": "oracle",
                                   "sample": sample},
                     e2e={"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
     if w["kind"] != "prefill":
@@ -923,7 +935,7 @@ def reference(args, rank, world):
     inp = prefill_problem(w, seed=0)
     H, T = w["nheads"], w["seqlen"]
     n_all = w["batch"] * H
-    probe = list(range(min(n_all, max(1, oracle.threads()))))
+    probe = list(range(min(n_all, host_cores())))
     per_unit = oracle_sample_step(w, inp, probe) / len(probe)
     budget = 150.0 / max(1, args.steps + args.warmup)
     n = int(min(n_all, max(len(probe), budget / max(per_unit, 1e-9))))
@@ -936,7 +948,7 @@ def reference(args, rank, world):
     sample = f"{n} of {n_all} (batch, head) units per step of the {w['batch']}x{T}-token workload"
     return dict(base, metric="SSD prefill tokens/s", value=value, unit="tokens/s",
                 ms_per_step=total / args.steps * 1e3,
-                cpu_baseline={"value": value, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+                cpu_baseline={"value": value, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
                               "sample": sample},
                 e2e={"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
 

@@ -136,3 +136,13 @@ def _fast_sample(step):
     def run(w, inp, units, nthreads=0):
         return step(w, inp, list(units)[:2], nthreads)
     return run
+
+
+def test_oracle_baselines_keep_all_cores_after_a_single_core_run():
+    """An OpenMP thread-count setting persists in the process: the all-core oracle timings
+    must still use every core after a single-core one."""
+    w = bench.WORKLOADS["decode_2p7b"]
+    one = bench.oracle_decode_rate(w, 0.02, nthreads=1)
+    assert one[4] == 1
+    rate, nu, steps, el, cores = bench.oracle_decode_rate(w, 0.02)
+    assert cores == bench.host_cores() and rate > 0 and nu >= 64
