@@ -56,6 +56,12 @@ WORKLOADS = {
     "gdn_decode_b64": dict(kind="gdn", batch=64, heads_qk=16, heads_v=32, dk=128, dv=128, steps=256),
     "deep_decode_2p7b": dict(kind="deep_decode", layers=64, batch=256, nheads=80, headdim=64, ngroups=1,
                              dstate=128, steps=256, dtype="f32"),
+    # ssd_decode_steps against one launch per step: the cached-decode shape, and batch 1
+    # (where a launch per token costs more than the step's work)
+    "decode_steps_2p7b": dict(kind="decode_steps", batch=64, nheads=80, headdim=64, ngroups=1, dstate=128,
+                              steps=1024, dtype="f32"),
+    "decode_steps_2p7b_b1": dict(kind="decode_steps", batch=1, nheads=80, headdim=64, ngroups=1, dstate=128,
+                                 steps=1024, dtype="f32"),
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -547,6 +553,60 @@ def run_decode(w, repeats, warmup, rank, world):
     return res
 
 
+def run_decode_steps(w, repeats, warmup, rank, world):
+    """The decode workload's steps run two ways on the same device-resident inputs: one
+    ssd_decode_step launch per token (captured in a CUDA graph), and one ssd_decode_steps
+    launch for all of them.  Both compute the same result bit for bit."""
+    import torch
+    import state_space_model_05_b200 as ssd
+    b, H, P, G, N, S = (w[k] for k in ("batch", "nheads", "headdim", "ngroups", "dstate", "steps"))
+    shape = gen.SSDShape(b, 1, H, P, G, N)
+    dec = gen.decode_inputs(shape, steps=S, seed=2000 + rank)
+    head = gen.prefill_inputs(shape, seed=2001 + rank)
+    f32 = torch.float32
+    X, DT, Bs, Cs = (_dev(a, f32) for a in (dec.x, dec.dt, dec.B, dec.C))
+    A, D = _dev(head.A, f32), _dev(head.D, f32)
+    state = _dev(gen.state_inputs(b, H, P, N, seed=2002 + rank), f32)
+    Y = torch.empty((S, b, H, P), device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for k in range(4):
+            ssd.ssd_decode_step(state, X[k], DT[k], A, Bs[k], Cs[k], D, y_t=Y[k])
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            for k in range(S):
+                ssd.ssd_decode_step(state, X[k], DT[k], A, Bs[k], Cs[k], D, y_t=Y[k])
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(repeats):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        return whole_job_rate(S * repeats, e0.elapsed_time(e1), world)
+
+    per_step, _ = timed(graph.replay)
+    one_launch, ms = timed(lambda: ssd.ssd_decode_steps(state, X, DT, A, Bs, Cs, D, y=Y))
+    if ssd.ssd_device_status() != 0:
+        raise RuntimeError("device status after decode steps")
+    del graph
+    # one launch: the state is read and written once per call, the per-step inputs and y once
+    io = S * (2 * b * H * P * 4 + 2 * b * G * N * 4 + b * H * 4) + 2 * b * H * P * N * 4
+    return {"steps_per_s_one_launch": one_launch, "steps_per_s_launch_per_step": per_step,
+            "us_per_step_one_launch": ms / (S * repeats) * 1e3, "bytes_per_call": io,
+            "gbs": io * repeats / (ms / 1e3) / 1e9}
+
+
 class DeepStack:
     """64 independent SSD layers of the 2.7B shape at batch 256: fp32 states (~43 GB) drawn
     i.i.d. N(0,1) on the device, and fresh per-layer inputs drawn on the device every step
@@ -721,6 +781,17 @@ def ours(args, rank, world):
         line["gpu_launches"] = res["launches"]
         line["e2e"] = None
         cfg = {"workload": args.workload, **{k: w[k] for k in w if k != "kind"}}
+    elif w["kind"] == "decode_steps":
+        res = run_decode_steps(w, max(1, args.steps // 4), max(1, args.warmup), rank, world)
+        line.update({"metric": "SSD decode steps/s (all steps in one launch)", "value": res["steps_per_s_one_launch"],
+                     "unit": "steps/s", "ms_per_step": res["us_per_step_one_launch"] / 1e3, "dtype": "f32"})
+        line["roofline"] = decode_roofline(res["gbs"], "decode_steps", peaks, src)
+        line["launch_per_step_steps_per_s"] = res["steps_per_s_launch_per_step"]
+        line["gpu_launches"] = max(1, args.steps // 4)
+        line["e2e"] = None
+        cfg = {"workload": args.workload, **{k: w[k] for k in w if k != "kind"}}
+        if solo:
+            line["cpu_baseline"] = cpu_baseline_decode(w, budget_s=8.0)
     elif w["kind"] == "deep_decode":
         res = run_deep_decode(w, args.steps, 3, rank, world)
         line.update({"metric": "SSD decode steps/s (64-layer stack)", "value": res["steps_per_s"],
@@ -804,6 +875,17 @@ def ours(args, rank, world):
         vr = run_prefill_varlen(pw, 100, 5, rank, world)
         extras["prefill_130m_varlen"] = {"value": vr["tokens_per_s"], "unit": "tokens/s",
                                          "ms_per_step": vr["ms_per_step"], "sequences": vr["lengths"]}
+        for name in ("decode_steps_2p7b", "decode_steps_2p7b_b1"):
+            sw = WORKLOADS[name]
+            r = run_decode_steps(sw, 5, 2, rank, world)
+            extras[name] = {"value": r["steps_per_s_one_launch"], "unit": "steps/s",
+                            "us_per_step": r["us_per_step_one_launch"],
+                            "launch_per_step_steps_per_s": r["steps_per_s_launch_per_step"],
+                            "roofline": decode_roofline(r["gbs"], "decode_steps (all steps, one launch; state "
+                                                        "read and written once per call)", peaks, src),
+                            "config": {k: sw[k] for k in sw if k != "kind"}}
+            summary[name] = {"steps_s": round(r["steps_per_s_one_launch"]),
+                             "launch_per_step_steps_s": round(r["steps_per_s_launch_per_step"])}
         for name in ("gdn_decode_b1", "gdn_decode_b64"):
             gw = WORKLOADS[name]
             r = run_gdn(gw, 3, 1, rank, world)
@@ -916,7 +998,7 @@ def reference(args, rank, world):
     base = {"impl": "reference", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded)", "config": cfg}
-    if w["kind"] in ("decode", "deep_decode"):
+    if w["kind"] in ("decode", "deep_decode", "decode_steps"):
         budget = 150.0 / max(1, args.steps + args.warmup)
         for _ in range(args.warmup):
             oracle_decode_rate(w, budget / 4)
@@ -925,7 +1007,8 @@ def reference(args, rank, world):
         nu, st = rates[0][1], rates[0][2]
         per_step, _, _ = _decode_units(w)
         sample = f"each step: {st} decode steps of {nu} of the {per_step} units a step, scaled to whole steps"
-        metric = "SSD decode steps/s" if w["kind"] == "decode" else "SSD decode steps/s (64-layer stack)"
+        metric = {"decode": "SSD decode steps/s", "deep_decode": "SSD decode steps/s (64-layer stack)",
+                  "decode_steps": "SSD decode steps/s (all steps in one launch)"}[w["kind"]]
         return dict(base, metric=metric, value=value, unit="steps/s", ms_per_step=1e3 / value,
                     cpu_baseline={"value": value, "unit": "steps/s", "cores": host_cores(), "kind": "oracle",
                                   "sample": sample},

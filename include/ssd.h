@@ -112,9 +112,11 @@ ssd_status_t ssd_prefill(const void* x, const float* dt, const float* A, const v
  *   SSD_PREFILL_TWO_PASS: a chunk-state walk writes each block's start state to the
  *     workspace, then a block-output kernel reads it back (one CTA per block and group
  *     of heads);
- *   SSD_PREFILL_FUSED: one kernel walks the 128-token blocks of each (batch, 1-3 heads) in
- *     order with the states in tensor memory and writes y and the final state, after a
- *     kernel forming G = C B^T per block (x read once, no state through HBM);
+ *   SSD_PREFILL_FUSED: after a kernel forming G = C B^T per block, one kernel walks the
+ *     128-token blocks of head pairs in order with the pairs' states in tensor memory and
+ *     writes y and the final state (x read once; a state goes through global memory only
+ *     where a pair's blocks are split between two CTAs).  It needs an even number of heads
+ *     per group; other shapes take the two-pass kernels;
  *   SSD_PREFILL_AUTO (the default): the two-pass kernels, the faster of the two on every
  *     workload measured so far.
  * Both compute the same chunked algorithm with bf16 operands and fp32 accumulation; the
@@ -138,6 +140,25 @@ ssd_status_t ssd_decode_step(float* state, const void* x_t, const float* dt_t, c
                              const void* B_t, const void* C_t, const float* D, int batch,
                              int nheads, int headdim, int ngroups, int dstate, ssd_dtype_t dtype,
                              void* y_t, void* stream);
+
+/*
+ * `steps` successive decode steps of one layer in one launch, for tokens whose inputs are
+ * already on the device: the O(1) cache advanced on the device by a loop with no host round
+ * trip per token ("Compiler-First State Space Duality and Portable O(1) Autoregressive
+ * Caching for Inference", section "2. Metodologia": the compiled generation loop).
+ *   x, y: [steps][batch][nheads][headdim] (`dtype`); dt: [steps][batch][nheads] fp32;
+ *   B, C: [steps][batch][ngroups][dstate] (`dtype`); A, D: [nheads] fp32; state in/out as
+ *   for ssd_decode_step.  Step k uses the k-th slice of each input and writes the k-th slice
+ *   of y.
+ * The result equals `steps` calls of ssd_decode_step on the slices, bit for bit.  With
+ * dstate <= 128 each (batch, head) state stays on chip for all the steps, so the state is
+ * read once and written once per call instead of once per step.  steps = 0 does nothing;
+ * steps < 0 is SSD_ERR_SHAPE; errors as for ssd_decode_step.
+ */
+ssd_status_t ssd_decode_steps(float* state, const void* x, const float* dt, const float* A,
+                              const void* B, const void* C, const float* D, int steps, int batch,
+                              int nheads, int headdim, int ngroups, int dstate, ssd_dtype_t dtype,
+                              void* y, void* stream);
 
 /*
  * ssd_prefill / ssd_decode_step with the dt pre-processing folded into the kernels: the dt

@@ -34,6 +34,7 @@ SIGNATURES = {
     "ssd_prefill_workspace_bytes": ([_I, _I, _I, _I, _I, _I, _I, _I], _Z),
     "ssd_prefill": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _Z, _P], _I),
     "ssd_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
+    "ssd_decode_steps": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ssd_decode_step_layers": ([_P, _I, _I, _I, _I, _I, _I, _I, _P], _I),
     "ssd_gdn_decode_step": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ssd_prefill_varlen_workspace_bytes": ([_I, _I, _I, _I, _I, _I, _I, _I], _Z),
@@ -262,6 +263,26 @@ def ssd_decode_step(state, x_t, dt_t, A, B_t, C_t, D, y_t=None, stream=None, dt_
                                _ptr(y_t), _stream(stream))
     _check(st, "ssd_decode_step")
     return y_t
+
+
+def ssd_decode_steps(state, x, dt, A, B, C, D, y=None, stream=None):
+    """``steps`` decode steps in one launch; ``state`` [b][H][P][N] fp32 is updated in place.
+    x [steps][b][H][P], dt [steps][b][H], B/C [steps][b][G][N].  Returns y [steps][b][H][P]."""
+    _rank(x, "x", "[steps][batch][nheads][headdim]")
+    _rank(B, "B", "[steps][batch][ngroups][dstate]")
+    steps, batch, nheads, headdim = x.shape
+    ngroups, dstate = B.shape[2], B.shape[3]
+    f32 = torch.float32
+    _check_args(x, ((state, "state", (batch, nheads, headdim, dstate), f32), (x, "x", x.shape, x.dtype),
+                    (dt, "dt", (steps, batch, nheads), f32), (A, "A", (nheads,), f32),
+                    (B, "B", B.shape, x.dtype), (C, "C", B.shape, x.dtype), (D, "D", (nheads,), f32),
+                    (y, "y", x.shape, x.dtype)))
+    if y is None:
+        y = torch.empty_like(x)
+    st = lib().ssd_decode_steps(_ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), steps,
+                                batch, nheads, headdim, ngroups, dstate, _dtype_code(x), _ptr(y), _stream(stream))
+    _check(st, "ssd_decode_steps")
+    return y
 
 
 # field order of ssd_decode_layer_t

@@ -68,11 +68,12 @@ ssd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_E
 
 // ---- opt-in kernel profiling: an event pair around each launch -------------------
 enum Stage { kCumsum, kStateTc, kStateSimt, kScan, kOutTc, kOutSimt, kDecode, kCopy, kDecodeLayers, kGdn,
-             kGram, kChain, kNumStages };
+             kGram, kChain, kDecodeSteps, kNumStages };
 const char* const kStageNames[kNumStages] = {"chunk_cumsum", "chunk_state_scan_tc", "chunk_state_simt",
                                               "state_scan", "chunk_output_tc", "chunk_output_simt",
                                               "decode_step", "copy_state", "decode_step_layers",
-                                              "gdn_decode_step", "block_gram_tc", "chain_prefill_tc"};
+                                              "gdn_decode_step", "block_gram_tc", "chain_prefill_tc",
+                                              "decode_steps"};
 
 // which tensor-core prefill batched calls take (ssd_set_prefill_path)
 std::atomic<int> g_prefill_path{SSD_PREFILL_AUTO};
@@ -457,6 +458,25 @@ ssd_status_t ssd_decode_step(float* state, const void* x_t, const float* dt_t, c
 {
     return decode_impl(state, x_t, dt_t, nullptr, 0, A, B_t, C_t, D, batch, nheads, headdim, ngroups,
                        dstate, dtype, y_t, stream);
+}
+
+ssd_status_t ssd_decode_steps(float* state, const void* x, const float* dt, const float* A, const void* B,
+                              const void* C, const float* D, int steps, int batch, int nheads, int headdim,
+                              int ngroups, int dstate, ssd_dtype_t dtype, void* y, void* stream)
+{
+    ssd_status_t st = check_common(batch, nheads, headdim, ngroups, dstate, dtype, 512);
+    if (st != SSD_OK) return st;
+    if (steps < 0) return SSD_ERR_SHAPE;
+    if (batch == 0 || steps == 0) return SSD_OK;
+    if (!state || !x || !dt || !A || !B || !C || !D || !y) return SSD_ERR_NULL;
+    if (!aligned16(state) || !aligned16(x) || !aligned16(dt) || !aligned16(A) || !aligned16(B) ||
+        !aligned16(C) || !aligned16(D) || !aligned16(y))
+        return SSD_ERR_ALIGN;
+    Dims d{batch, 1, nheads, headdim, ngroups, dstate, 1, 1};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return from_cuda(profiled(kDecodeSteps, s, [&] {
+        return launch_decode_steps(d, dtype, steps, state, x, dt, A, B, C, D, y, s);
+    }));
 }
 
 ssd_status_t ssd_decode_step_dtraw(float* state, const void* x_t, const float* dt_raw_t,

@@ -151,6 +151,132 @@ decode_layers_kernel(const ssd_decode_layer_t* __restrict__ layers, int nheads, 
                               static_cast<T*>(L.y_t), blockIdx.x, nheads, headdim, ngroups, dstate);
 }
 
+// ---------------------------------------------------------------- several steps, one launch
+// `steps` successive tokens of one layer in one launch (the device-side counterpart of a
+// generation loop that advances the cache with no host round trip per token, when the
+// tokens' inputs are on the device already).  One CTA per (b, h) keeps that unit's state in
+// registers for all the steps -- warp w holds rows w RPW .. w RPW + RPW - 1, lane j the
+// 16-byte quad j of a row -- so the state is read once and written once, and the next
+// step's inputs are loaded while this step is computed.  Each row's arithmetic is the
+// single step's, operation for operation, so the results equal `steps` launches of
+// decode_step_kernel bit for bit.  Inputs and outputs are [steps][...] arrays of the
+// single step's layouts.
+template <typename T, int RPW>
+__global__ void __launch_bounds__(kDecodeThreads, RPW <= 8 ? 2 : 1)
+decode_steps_kernel(float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
+                    const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
+                    const float* __restrict__ D, T* __restrict__ y, int steps, int batch, int nheads,
+                    int headdim, int ngroups, int dstate)
+{
+    const int unit = blockIdx.x;
+    const int b = unit / nheads;
+    const int h = unit - b * nheads;
+    const int g = h / (nheads / ngroups);
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const bool qon = lane < (dstate >> 2);             // this lane's quad exists (dstate <= 128)
+    const int p0 = warp * RPW;
+    const size_t units = (size_t)batch * nheads;
+    const float Ah = A[h], Dh = D[h];
+
+    float4 s[RPW];
+    float* S = state + (size_t)unit * headdim * dstate;
+#pragma unroll
+    for (int r = 0; r < RPW; ++r)
+        if (p0 + r < headdim && qon) s[r] = *reinterpret_cast<const float4*>(S + (size_t)(p0 + r) * dstate + 4 * lane);
+
+    // the inputs of step k: dt, B_t and C_t (this lane's quad), x of this warp's rows
+    auto load_step = [&](int k, float& dtv, float4& bq, float4& cq, float (&xv)[RPW]) {
+        dtv = dt[(size_t)k * units + unit];
+        const size_t bc = ((size_t)k * batch * ngroups + (size_t)b * ngroups + g) * dstate;
+        bq = qon ? load4<T>(Bm + bc + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+        cq = qon ? load4<T>(Cm + bc + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const T* xr = x + ((size_t)k * units + unit) * headdim;
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) xv[r] = p0 + r < headdim ? Elem<T>::load(xr + p0 + r) : 0.f;
+    };
+    float dtn = 0.f, xn[RPW];
+    float4 bn, cn;
+    if (steps > 0) load_step(0, dtn, bn, cn, xn);
+    for (int k = 0; k < steps; ++k) {
+        const float dtv = dtn;
+        const float4 bq = bn, cq = cn;
+        float xv[RPW];
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) xv[r] = xn[r];
+        if (k + 1 < steps) load_step(k + 1, dtn, bn, cn, xn);
+        const float a = expf(dtv * Ah);                // fp32 decay exponent
+        T* yr = y + ((size_t)k * units + unit) * headdim;
+#pragma unroll
+        for (int r = 0; r < RPW; ++r) {
+            const int p = p0 + r;
+            if (p >= headdim) break;                   // warp-uniform
+            const float dx = dtv * xv[r];
+            float acc = 0.f;
+            if (qon) {
+                float4 v = s[r];
+                v.x = fmaf(a, v.x, dx * bq.x);
+                v.y = fmaf(a, v.y, dx * bq.y);
+                v.z = fmaf(a, v.z, dx * bq.z);
+                v.w = fmaf(a, v.w, dx * bq.w);
+                acc = fmaf(cq.x, v.x, acc);
+                acc = fmaf(cq.y, v.y, acc);
+                acc = fmaf(cq.z, v.z, acc);
+                acc = fmaf(cq.w, v.w, acc);
+                s[r] = v;
+            }
+            acc = warp_sum(acc);
+            if (lane == 0) Elem<T>::store(yr + p, fmaf(Dh, xv[r], acc));
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < RPW; ++r)
+        if (p0 + r < headdim && qon) *reinterpret_cast<float4*>(S + (size_t)(p0 + r) * dstate + 4 * lane) = s[r];
+}
+
+// Shapes whose state does not fit in registers: the single step's body once per step, still
+// one launch (each CTA owns its unit's state, so the steps need no synchronisation).
+template <typename T, int QPL, int ROWS>
+__global__ void __launch_bounds__(kDecodeThreads, QPL == 1 ? 4 : 2)
+decode_steps_loop_kernel(float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
+                         const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
+                         const float* __restrict__ D, T* __restrict__ y, int steps, int batch, int nheads,
+                         int headdim, int ngroups, int dstate)
+{
+    const size_t units = (size_t)batch * nheads;
+    for (int k = 0; k < steps; ++k)
+        decode_unit<T, QPL, ROWS>(state, x + (size_t)k * units * headdim, dt + (size_t)k * units, A,
+                                  Bm + (size_t)k * batch * ngroups * dstate, Cm + (size_t)k * batch * ngroups * dstate,
+                                  D, y + (size_t)k * units * headdim, blockIdx.x, nheads, headdim, ngroups, dstate);
+}
+
+template <typename T>
+cudaError_t launch_steps_dtype(const Dims& d, int steps, float* state, const void* x, const float* dt,
+                               const float* A, const void* B, const void* C, const float* D, void* y,
+                               cudaStream_t s)
+{
+    const unsigned grid = (unsigned)(d.batch * d.nheads);
+    const T* xt = static_cast<const T*>(x);
+    const T* Bt = static_cast<const T*>(B);
+    const T* Ct = static_cast<const T*>(C);
+    T* yt = static_cast<T*>(y);
+    if (d.dstate <= 128 && d.headdim <= 64)
+        decode_steps_kernel<T, 8><<<grid, kDecodeThreads, 0, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch,
+                                                                  d.nheads, d.headdim, d.ngroups, d.dstate);
+    else if (d.dstate <= 128)
+        decode_steps_kernel<T, 16><<<grid, kDecodeThreads, 0, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch,
+                                                                   d.nheads, d.headdim, d.ngroups, d.dstate);
+    else if (d.dstate <= 256)
+        decode_steps_loop_kernel<T, 2, 4><<<grid, kDecodeThreads, 0, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps,
+                                                                          d.batch, d.nheads, d.headdim, d.ngroups,
+                                                                          d.dstate);
+    else
+        decode_steps_loop_kernel<T, 4, 2><<<grid, kDecodeThreads, 0, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps,
+                                                                          d.batch, d.nheads, d.headdim, d.ngroups,
+                                                                          d.dstate);
+    return cudaGetLastError();
+}
+
 template <typename T, int QPL, int ROWS>
 cudaError_t launch_decode_t(const Dims& d, float* state, const void* x, const float* dt,
                             const float* A, const void* B, const void* C, const float* D, void* y,
@@ -200,6 +326,15 @@ cudaError_t launch_decode_layers(const Dims& d, ssd_dtype_t dtype, const ssd_dec
     if (d.batch == 0 || n_layers == 0) return cudaSuccess;
     if (dtype == SSD_F32) return launch_layers_dtype<float>(d, layers, n_layers, s);
     return launch_layers_dtype<__nv_bfloat16>(d, layers, n_layers, s);
+}
+
+cudaError_t launch_decode_steps(const Dims& d, ssd_dtype_t dtype, int steps, float* state, const void* x,
+                                const float* dt, const float* A, const void* B, const void* C, const float* D,
+                                void* y, cudaStream_t s)
+{
+    if (d.batch == 0 || steps == 0) return cudaSuccess;
+    if (dtype == SSD_F32) return launch_steps_dtype<float>(d, steps, state, x, dt, A, B, C, D, y, s);
+    return launch_steps_dtype<__nv_bfloat16>(d, steps, state, x, dt, A, B, C, D, y, s);
 }
 
 cudaError_t launch_decode(const Dims& d, ssd_dtype_t dtype, float* state, const void* x,

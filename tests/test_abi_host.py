@@ -131,6 +131,21 @@ def test_decode_validation(lib):
     assert _decode(lib, batch=0) == 0
 
 
+def test_decode_steps_validation(lib):
+    """Sizes and pointers are checked on the host before any launch."""
+    f = lib.ssd_decode_steps
+    args = lambda steps=3, nh=8, ng=1, ds=128, st=FAKE, y=FAKE, B=FAKE, dtype=binding.SSD_F32: (
+        st, FAKE, FAKE, FAKE, B, FAKE, FAKE, steps, 2, nh, 64, ng, ds, dtype, y, None)
+    assert f(*args(steps=-1)) == 2                   # negative step count
+    assert f(*args(nh=6, ng=4)) == 2                 # nheads % ngroups
+    assert f(*args(ds=1024)) == 5                    # dstate > 512
+    assert f(*args(st=None)) == 1
+    assert f(*args(y=None)) == 1
+    assert f(*args(B=FAKE + 4)) == 4                 # misaligned
+    assert f(*args(dtype=9)) == 3
+    assert f(*args(steps=0, st=None)) == 0           # nothing to do
+
+
 def test_decode_layers_validation(lib):
     """Sizes are checked on the host before any launch; the table is read only by the kernel."""
     f = lib.ssd_decode_step_layers
