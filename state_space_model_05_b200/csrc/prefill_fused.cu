@@ -22,7 +22,7 @@
 // and output GEMMs are one MMA each with the heads side by side along N (N = 128):
 //   S      = B_k^T [X~_0 | X~_1]   onto the pair's states in TMEM (lane n, column 64 j + p)
 //   Yo     = C_k [H_0 | H_1]       (the states' bf16 image in shared memory)
-//   Yd_j   = D x_j + P_j X_j       (P_j in TMEM, one per head; D x stored first)
+//   Yd_j   = P_j X_j               (P_j in TMEM, one per head)
 // The steps of all units, unit-major, are cut into one contiguous range per CTA, so every
 // CTA does the same number of blocks however the units divide among the SMs.  A range
 // starts and ends inside a unit at most once each; the CTA runs the piece at its end first
@@ -36,8 +36,7 @@
 //               fetched into L2 four steps ahead); fp16 B_k in 64-token stages (three deep); C_k
 //   warps 1, 14, 15  tcgen05.mma issue, one stream each: S, Yo, Yd_j
 //   warps 2-5   X~ = w o X (fp16) for the state GEMM; the epilogue of the previous step,
-//               y = Yd + exp(Lam_t) Yo, written straight to global memory; then D x of this
-//               step into the Yd accumulators, onto which the Yd MMA adds P X
+//               y = Yd + exp(Lam_t) Yo + D x, written over that step's x and TMA-stored
 //   warps 6-13  per step, first the state of one head for the warp's 32 TMEM lanes (the
 //               bf16 image of H, the operand of Yo, then H <- exp(Lam_end) H, onto which S
 //               accumulates; start and end states at piece boundaries), then two of the
@@ -212,51 +211,56 @@ struct UnitMap {
     }
 };
 
-// Walks a CTA's steps in order.  The unit, block, batch, group and first head of the current
-// step are kept incrementally: the divisions that locate a step run only where an interval
-// starts or the unit changes, not on every step.
+// Walks a CTA's steps in order.  The current interval's bounds and the unit, block, batch,
+// group and first head of the current step are kept in registers and advanced
+// incrementally: the divisions that locate a step run only where an interval starts or the
+// unit changes, not on every step.
 struct StepIter {
     const StepSeq* q;
-    const UnitMap* um;
-    int r;
-    long long i;
+    UnitMap um;
+    int r, nb;
+    long long i, lo, hi;
     int u, k, b, g, h0;
     __device__ void start(const StepSeq& s, const UnitMap& m) {
         q = &s;
-        um = &m;
-        r = 0;
-        i = s.lo[0];
-        skip();
+        um = m;
+        nb = s.nb;
+        r = -1;
+        hi = 0;
+        i = 0;
+        advance();
     }
-    __device__ void locate() {
-        u = (int)(i / q->nb);
-        k = (int)(i - (long long)u * q->nb);
-        um->map(u, &b, &g, &h0);
-    }
-    __device__ void skip() {
-        while (r < 3 && i >= q->hi[r]) {
+    // moves to the next non-empty interval (or past the last)
+    __device__ void advance() {
+        for (;;) {
             ++r;
-            if (r < 3) i = q->lo[r];
+            if (r >= 3) return;
+            lo = r == 0 ? q->lo[0] : (r == 1 ? q->lo[1] : q->lo[2]);
+            hi = r == 0 ? q->hi[0] : (r == 1 ? q->hi[1] : q->hi[2]);
+            if (lo < hi) break;
         }
-        if (r < 3) locate();
+        i = lo;
+        u = (int)(i / nb);
+        k = (int)(i - (long long)u * nb);
+        um.map(u, &b, &g, &h0);
     }
     __device__ bool valid() const { return r < 3; }
     __device__ void next() {
         ++i;
-        if (i >= q->hi[r]) {
-            skip();
+        if (i >= hi) {
+            advance();
             return;
         }
-        if (++k == q->nb) {
+        if (++k == nb) {
             k = 0;
             ++u;
-            um->map(u, &b, &g, &h0);
+            um.map(u, &b, &g, &h0);
         }
     }
     __device__ int unit() const { return u; }
     __device__ int block() const { return k; }
-    __device__ bool first() const { return i == q->lo[r] || k == 0; }
-    __device__ bool last() const { return i == q->hi[r] - 1 || k == q->nb - 1; }
+    __device__ bool first() const { return i == lo || k == 0; }
+    __device__ bool last() const { return i == hi - 1 || k == nb - 1; }
 };
 
 // ================================================================ chain kernel
@@ -297,7 +301,7 @@ enum {
     PB_BF = PB_XE + PairSmem::kXSlots, PB_BE = PB_BF + PairSmem::kBStages,
     PB_CF = PB_BE + PairSmem::kBStages, PB_CE,
     PB_UPD, PB_CONV, PB_SD, PB_YO,
-    PB_PF, PB_YD = PB_PF + 2, PB_EPI = PB_YD + 2, PB_DXR = PB_EPI + 2, PB_COUNT = PB_DXR + 2
+    PB_PF, PB_YD = PB_PF + 2, PB_EPI = PB_YD + 2, PB_COUNT = PB_EPI + 2
 };
 static_assert(PB_COUNT <= PairSmem::kNumBars, "chain barriers");
 
@@ -361,9 +365,18 @@ __device__ __noinline__ bool wait_handoff(const int* flag, int value, int* err, 
     return false;
 }
 
+// Two bf16 products at once: (a.lo * b.lo, a.hi * b.hi), each rounded to bf16.
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 // One 32-column sub-block of row r of P = G o exp(Lam_t - Lam_s) o dt_s (s <= t), from 16
 // bf16 pairs of G, stored to TMEM at taddr (warp-collective; the sub-block is below, on or
-// above the diagonal for the warp's 32 rows alike).  Below-diagonal sub-blocks use
+// above the diagonal for the warp's 32 rows alike).  The decay-times-dt factor of each
+// element is formed in fp32, rounded to bf16 and multiplied into G two columns at a time
+// (a second bf16 rounding of P, well inside the tolerance: the parity tests bound it).  Below-diagonal sub-blocks use
 // exp(Lam_t - Lam_q) exp(Lam_q - Lam_s), q the sub-block's last column; sub-blocks on the
 // diagonal use the first column as reference when their own decay is below 40 (both factors
 // within e^+-40) and one exponential per element otherwise.
@@ -382,8 +395,8 @@ __device__ __forceinline__ void p_store_subblock(uint32_t taddr, uint4 g0, uint4
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
             const float4 f = v4[e4];
-            pk[2 * e4] = pack_bf16x2(bf16lo(gw[2 * e4]) * u * f.x, bf16hi(gw[2 * e4]) * u * f.y);
-            pk[2 * e4 + 1] = pack_bf16x2(bf16lo(gw[2 * e4 + 1]) * u * f.z, bf16hi(gw[2 * e4 + 1]) * u * f.w);
+            pk[2 * e4] = mul_bf16x2(gw[2 * e4], pack_bf16x2(u * f.x, u * f.y));
+            pk[2 * e4 + 1] = mul_bf16x2(gw[2 * e4 + 1], pack_bf16x2(u * f.z, u * f.w));
         }
     } else if (s0 >= r0 + 32) {
 #pragma unroll
@@ -395,10 +408,9 @@ __device__ __forceinline__ void p_store_subblock(uint32_t taddr, uint4 g0, uint4
         for (int e4 = 0; e4 < 8; ++e4) {
             const float4 f = w4[e4];
             const int sa = s0 + 4 * e4;
-            pk[2 * e4] = pack_bf16x2(sa <= r ? bf16lo(gw[2 * e4]) * u * f.x : 0.f,
-                                     sa + 1 <= r ? bf16hi(gw[2 * e4]) * u * f.y : 0.f);
-            pk[2 * e4 + 1] = pack_bf16x2(sa + 2 <= r ? bf16lo(gw[2 * e4 + 1]) * u * f.z : 0.f,
-                                         sa + 3 <= r ? bf16hi(gw[2 * e4 + 1]) * u * f.w : 0.f);
+            pk[2 * e4] = mul_bf16x2(gw[2 * e4], pack_bf16x2(sa <= r ? u * f.x : 0.f, sa + 1 <= r ? u * f.y : 0.f));
+            pk[2 * e4 + 1] = mul_bf16x2(gw[2 * e4 + 1],
+                                        pack_bf16x2(sa + 2 <= r ? u * f.z : 0.f, sa + 3 <= r ? u * f.w : 0.f));
         }
     } else {
         p_subblock_strong_decay(taddr, g0, g1, g2, g3, s0, r, sLam, sDt);
@@ -407,32 +419,10 @@ __device__ __forceinline__ void p_store_subblock(uint32_t taddr, uint4 g0, uint4
     tmem_st16(taddr, pk);
 }
 
-// Four 16-byte chunks per lane: lane i of each group of four lanes starts with four chunks
-// of its own row and ends with chunk i of the group's four rows (that of row m at d[m]).
-__device__ __forceinline__ void transpose_quad(uint4 (&d)[4], int lane)
-{
-#pragma unroll
-    for (int s = 2; s >= 1; s >>= 1) {
-        const bool hi = (lane & s) != 0;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            if (c & s) continue;
-            const uint4 keep = hi ? d[c | s] : d[c];
-            const uint4 send = hi ? d[c] : d[c | s];
-            uint4 got;
-            got.x = __shfl_xor_sync(0xffffffffu, send.x, s);
-            got.y = __shfl_xor_sync(0xffffffffu, send.y, s);
-            got.z = __shfl_xor_sync(0xffffffffu, send.z, s);
-            got.w = __shfl_xor_sync(0xffffffffu, send.w, s);
-            d[c] = hi ? got : keep;
-            d[c | s] = hi ? keep : got;
-        }
-    }
-}
-
 __global__ void __launch_bounds__(kPairThreads, 1)
 pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b16,
-                  const __grid_constant__ CUtensorMap tm_c, const float* __restrict__ fac,
+                  const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
+                  const float* __restrict__ fac,
                   const uint4* __restrict__ gram, const float* __restrict__ D,
                   const float* __restrict__ init_state, float* __restrict__ final_state,
                   __nv_bfloat16* __restrict__ y, float* __restrict__ handoff, int* __restrict__ handoff_flag,
@@ -455,7 +445,7 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
     if (tid == 0) {
         for (int i = 0; i < L::kXSlots; ++i) {
             mbar_init(&bars[PB_XF + i], 1);
-            mbar_init(&bars[PB_XE + i], 1 + 4);           // the last Yd MMA, the 4 X~ / epilogue warps
+            mbar_init(&bars[PB_XE + i], 1 + 4);           // the last Yd MMA, the 4 epilogue warps
         }
         for (int i = 0; i < L::kBStages; ++i) {
             mbar_init(&bars[PB_BF + i], 1);
@@ -471,7 +461,6 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
             mbar_init(&bars[PB_PF + j], kPThreads);
             mbar_init(&bars[PB_YD + j], 1);
             mbar_init(&bars[PB_EPI + j], 4);
-            mbar_init(&bars[PB_DXR + j], 4);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -630,14 +619,14 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
         }
     } else if (warp == kWarpMmaD) {
         if (lane == 0) {
-            // ------------------------------------------------ Yd_j += P_j X_j (onto D x)
+            // ------------------------------------------------ Yd_j = P_j X_j
             constexpr uint32_t idD = idesc_bf16_f32(128, 64, false, true);
             int nd = 0;
             for (; nd < 2 * total; ++nd) {
                 const int sd = nd >> 1;
                 const int j = (int)(nd & 1);
                 if (!chain_wait(&bars[PB_PF + j], sd & 1, err, abort_flag) ||
-                    !chain_wait(&bars[PB_DXR + j], sd & 1, err, abort_flag) ||
+                    (sd > 0 && !chain_wait(&bars[PB_EPI + j], (sd - 1) & 1, err, abort_flag)) ||
                     !chain_wait(&bars[PB_XF + (sd & 1)], (sd >> 1) & 1, err, abort_flag))
                     break;
                 tc_fence_after();
@@ -645,18 +634,18 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
 #pragma unroll 1
                 for (int ks = 0; ks < 8; ++ks)
                     umma_f16_ts(tmem + kColYd + 64 * j, tmem + kColP + 64 * j + ks * 8,
-                                smem_desc_sw128(aX + ks * 2048, kBox, 1024), idD, 1u);
+                                smem_desc_sw128(aX + ks * 2048, kBox, 1024), idD, ks > 0 ? 1u : 0u);
                 umma_commit(&bars[PB_YD + j]);
                 if (j == 1) umma_commit(&bars[PB_XE + (sd & 1)]);
             }
             if (nd > 0) mbar_wait(&bars[PB_YD + ((nd - 1) & 1)], ((nd - 1) >> 1) & 1, err);
         }
     } else if (warp >= kWarpE0 && warp < kWarpP0) {
-        // ---------------------------------------------------- X~, the previous step's epilogue, D x
-        // Per step s: X~_s = w o X_s (the state GEMM's operand); the epilogue of step s - 1
-        // (y = Yd + exp(Lam_t) Yo, D x being in Yd already); then D x_s written into the freed
-        // Yd accumulators, onto which the Yd MMA of step s adds P X.  After that the step's x
-        // slot is no longer read here, so its refill does not wait for the epilogue.
+        // ---------------------------------------------------- X~, then the previous step's epilogue
+        // Per step s: X~_s = w o X_s (the state GEMM's operand); then the epilogue of step
+        // s - 1, y = Yd + exp(Lam_t) Yo + D x written over that step's x rows (each thread its
+        // own row) and stored with one TMA store per warp and head; the slot is released once
+        // the stores have read it.
         const int q = warp & 3;
         const int t = q * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
@@ -664,17 +653,17 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
         it.start(seq, um);
         int s = 0;
         int pb = 0, pk = 0, ph0 = 0;                     // the previous step: batch, block, first head
-        float pu0 = 0.f, pu1 = 0.f;                      // and its exp(Lam_t) of both heads
+        float pD0 = 0.f, pD1 = 0.f;
 
-        // y = Yd + exp(Lam_t) Yo of step ps, row t, heads j = 0, 1, stored to global memory
         auto epilogue = [&](int ps) -> bool {
             if (!wait_warp(PB_YO, ps & 1)) return false;
+            uint8_t* sl = xslot(ps);
             for (int j = 0; j < 2; ++j) {
                 if (!wait_warp(PB_YD + j, ps & 1)) return false;
                 tc_fence_after();
-                const float u = j ? pu1 : pu0;
-                __nv_bfloat16* yhead = y + ((size_t)pb * seqlen * nheads + ph0 + j) * kP;
-                const int rbase = pk * kBlk + q * 32 + (lane & ~3);     // the quad's first row
+                const float u = expf(facp(ps, j)[t]);
+                const float Dh = j ? pD1 : pD0;
+                uint8_t* xrow = sl + j * kBox + t * 128;
 #pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     uint32_t yd[32], yo[32];
@@ -687,48 +676,51 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&bars[PB_EPI + j]);
                     }
-                    uint4 ch[4];
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
+                        const int cx = 4 * half + c4;                   // 16-byte chunk of the row
+                        uint4* xp = reinterpret_cast<uint4*>(xrow + ((cx ^ (t & 7)) << 4));
+                        const uint4 xu = *xp;
+                        const uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w};
                         uint32_t o[4];
 #pragma unroll
                         for (int k2 = 0; k2 < 4; ++k2) {
                             const int e = 8 * c4 + 2 * k2;
-                            o[k2] = pack_bf16x2(fmaf(u, __uint_as_float(yo[e]), __uint_as_float(yd[e])),
-                                                fmaf(u, __uint_as_float(yo[e + 1]), __uint_as_float(yd[e + 1])));
+                            o[k2] = pack_bf16x2(
+                                fmaf(u, __uint_as_float(yo[e]), __uint_as_float(yd[e])) + Dh * bf16lo(xw[k2]),
+                                fmaf(u, __uint_as_float(yo[e + 1]), __uint_as_float(yd[e + 1])) + Dh * bf16hi(xw[k2]));
                         }
-                        ch[c4] = make_uint4(o[0], o[1], o[2], o[3]);
-                    }
-                    // four lanes write one row's 64 bytes of this half per store
-                    transpose_quad(ch, lane);
-#pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        const int tr = rbase + m;
-                        if (tr < seqlen)
-                            *reinterpret_cast<uint4*>(yhead + (size_t)tr * nheads * kP + 32 * half + (lane & 3) * 8) = ch[m];
+                        *xp = make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 }
+                // this warp's 32 rows of y (rows past seqlen are not written)
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && pk * kBlk + 32 * q < seqlen)
+                    tma_store_3d(&tm_y, (ph0 + j) * kP, pk * kBlk + 32 * q, pb, sl + j * kBox + q * 32 * 128);
             }
+            if (lane == 0) {
+                bulk_commit_group();
+                bulk_wait_group_read0();                 // the stores have read the slot
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[PB_XE + (ps & 1)]);
             return true;
         };
 
         bool live = true;
         for (; it.valid() && live; it.next(), ++s) {
-            const int b = it.b, g = it.g, h0 = it.h0;
+            const int b = it.b, h0 = it.h0;
             const int k = it.block();
             const float d0 = D[h0], d1 = D[h0 + 1];
             // X~_s: waits for the slot and for S of the previous step
             live = wait_warp(PB_XF + (s & 1), (s >> 1) & 1) && (s == 0 || wait_warp(PB_SD, (s - 1) & 1));
             if (!live) break;
             const uint8_t* sl = xslot(s);
-            float u0 = 0.f, u1 = 0.f;
 #pragma unroll 1
             for (int j = 0; j < 2; ++j) {
                 const float* sLam = facp(s, j);
                 const float w = expf(sLam[kBlk - 1] - sLam[t]) * sLam[kBlk + t];
-                const float u = expf(sLam[t]);
-                if (j) u1 = u;
-                else u0 = u;
                 const uint4* src = reinterpret_cast<const uint4*>(sl + j * kBox + t * 128);
                 uint4* dst = reinterpret_cast<uint4*>(sm + L::kXt + j * kBox + t * 128);
                 uint4 u8[8];
@@ -746,42 +738,14 @@ pair_chain_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                 live = epilogue(s - 1);
                 if (!live) break;
             }
-            // D x_s into the Yd accumulators the epilogue has just read (free at the first step)
-#pragma unroll 1
-            for (int j = 0; j < 2; ++j) {
-                const float Dh = j ? d1 : d0;
-                const uint8_t* xrow = sl + j * kBox + t * 128;
-#pragma unroll 1
-                for (int q16 = 0; q16 < 4; ++q16) {
-                    uint32_t v[16];
-#pragma unroll
-                    for (int hc = 0; hc < 2; ++hc) {
-                        const int cx = 2 * q16 + hc;                    // 16-byte chunk of the row
-                        const uint4 xu = *reinterpret_cast<const uint4*>(xrow + ((cx ^ (t & 7)) << 4));
-                        const uint32_t xw[4] = {xu.x, xu.y, xu.z, xu.w};
-#pragma unroll
-                        for (int k2 = 0; k2 < 4; ++k2) {
-                            v[8 * hc + 2 * k2] = __float_as_uint(Dh * bf16lo(xw[k2]));
-                            v[8 * hc + 2 * k2 + 1] = __float_as_uint(Dh * bf16hi(xw[k2]));
-                        }
-                    }
-                    tmem_st16(tl + kColYd + 64 * j + 16 * q16, v);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars[PB_DXR + j]);
-            }
-            // this step's x slot is no longer read by these warps
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[PB_XE + (s & 1)]);
             pb = b;
             pk = k;
             ph0 = h0;
-            pu0 = u0;
-            pu1 = u1;
+            pD0 = d0;
+            pD1 = d1;
         }
         if (live && s > 0) epilogue(s - 1);
+        if (lane == 0) bulk_wait_group0();
     } else if (warp >= kWarpP0 && warp < kWarpP0 + 8) {
         // ---------------------------------------------------- state of head c, then P_j
         // Warp (quarter q, c): TMEM lanes 32 q .. 32 q + 31.  The state part treats the lane as
@@ -981,7 +945,7 @@ cudaError_t launch_chain_prefill(const Dims& d, const void* x, const void* C, co
 {
     if (d.nchunks == 0 || d.batch == 0) return cudaSuccess;
     if (d.chunk_len != kBlk || !fused_prefill_supported(d)) return cudaErrorInvalidValue;
-    CUtensorMap mx, mb, mc;
+    CUtensorMap mx, mb, mc, my;
     // fp16 B [b][T][G][N] seen as (n mod 64, t, 2 g + n / 64, b): a box is both n-halves of 64 rows
     const uint64_t T = d.seqlen, G = d.ngroups, Bt = d.batch;
     const uint64_t bdim[4] = {64, T, 2 * G, Bt};
@@ -989,13 +953,14 @@ cudaError_t launch_chain_prefill(const Dims& d, const void* x, const void* C, co
     const uint32_t bbox[4] = {64, 64, 2, 1};
     if (!tc_make_map(&mx, x, (uint64_t)d.nheads * kP, d.seqlen, d.batch) ||
         !tc_encode_map(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, w.b16, bdim, bstr, bbox, true) ||
-        !tc_make_map(&mc, C, (uint64_t)d.ngroups * kN, d.seqlen, d.batch))
+        !tc_make_map(&mc, C, (uint64_t)d.ngroups * kN, d.seqlen, d.batch) ||
+        !tc_make_map(&my, y, (uint64_t)d.nheads * kP, d.seqlen, d.batch, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 32))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(pair_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          PairSmem::kBytes);
     if (e != cudaSuccess) return e;
     const int ctas = pair_ctas(d);
-    return launch_dependent(pair_chain_kernel, dim3(ctas), dim3(kPairThreads), PairSmem::kBytes, s, mx, mb, mc,
+    return launch_dependent(pair_chain_kernel, dim3(ctas), dim3(kPairThreads), PairSmem::kBytes, s, mx, mb, mc, my,
                             static_cast<const float*>(w.fac), static_cast<const uint4*>(w.gram), D, init_state,
                             final_state, static_cast<__nv_bfloat16*>(y), w.handoff, w.handoff_flag, d.seqlen,
                             d.nheads, d.ngroups, d.nchunks, (int)fused_units(d), device_error_word());
