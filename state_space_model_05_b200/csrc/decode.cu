@@ -16,6 +16,7 @@
 // are read once per CTA into registers (lane j holds elements 4j..4j+3).  The y reduction along dstate is a
 // warp shuffle tree; the state is written back with 16-byte stores.
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace ssd {
 
@@ -155,83 +156,176 @@ decode_layers_kernel(const ssd_decode_layer_t* __restrict__ layers, int nheads, 
 // `steps` successive tokens of one layer in one launch (the device-side counterpart of a
 // generation loop that advances the cache with no host round trip per token, when the
 // tokens' inputs are on the device already).  One CTA per (b, h) keeps that unit's state in
-// registers for all the steps -- warp w holds rows w RPW .. w RPW + RPW - 1, lane j the
-// 16-byte quad j of a row -- so the state is read once and written once, and the next
-// step's inputs are loaded while this step is computed.  Each row's arithmetic is the
-// single step's, operation for operation, so the results equal `steps` launches of
-// decode_step_kernel bit for bit.  Inputs and outputs are [steps][...] arrays of the
-// single step's layouts.
-template <typename T, int RPW>
-__global__ void __launch_bounds__(kDecodeThreads, RPW <= 8 ? 2 : 1)
+// registers for all the steps, so the state is read once and written once.
+//
+// Lanes: the 4 lanes of a group share R rows of the state (group j of warp w holds rows
+// w 8R + j + 8i, i < R), and lane L of the group the quads q = L + 4m (m < 8) of each row.
+// A row's output is then summed in the single step's order without most of its shuffles:
+// the single step forms one partial per quad (4 FMAs in order) and folds the 32 partials by
+// the xor tree 16, 8, 4, 2, 1 over the quad index; here the levels 16, 8 and 4 pair quads of
+// the same lane (m ^ 4, m ^ 2, m ^ 1) and only the levels 2 and 1 cross lanes.  Every level
+// adds the same two partials, so the results equal `steps` launches of decode_step_kernel
+// bit for bit (absent quads, dstate < 128, add the same +0 partials there and here).
+//
+// Inputs: the steps' x, B_t and C_t rows stream through a ring of kStepStages shared-memory
+// stages filled kStepAhead steps ahead -- step j by lane 0 of warp j % 8, so the issuing is
+// spread over the warps and stage w is always filled by warp w -- the rows by bulk copies (headdim and
+// dstate are multiples of 8 and the pointers 16-byte aligned, so every row copy is 16-byte
+// aligned and sized) and dt by a 4-byte cp.async that the stage's barrier also waits for.  A
+// warp releases a stage after its step's arithmetic, so B_t and C_t are read from shared
+// memory where they are used.  Inputs and outputs are [steps][...] arrays of the single
+// step's layouts.  Every wait is bounded: expiry records SSD_ERR_TIMEOUT, the CTA stops
+// stepping, waits for its copies in flight and writes back the state it has.
+constexpr int kStepStages = 8;
+constexpr int kStepAhead = 6;                          // the refilled stage was used 2 steps ago
+static_assert(kStepStages == kDecodeWarps, "stage w is filled by warp w");
+
+template <typename T>
+__host__ __device__ constexpr int step_row_bytes(int n) { return (int)((n * sizeof(T) + 15) & ~size_t(15)); }
+
+template <typename T, int R>
+__global__ void __launch_bounds__(kDecodeThreads, R == 1 ? 3 : 1)
 decode_steps_kernel(float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
                     const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
                     const float* __restrict__ D, T* __restrict__ y, int steps, int batch, int nheads,
-                    int headdim, int ngroups, int dstate)
+                    int headdim, int ngroups, int dstate, int* err)
 {
+    static_assert(R == 1 || R == 2, "rows per lane group");
+    extern __shared__ __align__(16) uint8_t stage_mem[]; // per stage: x row | B_t row | C_t row | dt
+    __shared__ __align__(8) uint64_t full[kStepStages], empty[kStepStages];
+    __shared__ int abort_flag;
+    const int xbytes = step_row_bytes<T>(headdim);
+    const int nbytes = step_row_bytes<T>(dstate);
+    const int stage_bytes = xbytes + 2 * nbytes + 16;
+
     const int unit = blockIdx.x;
     const int b = unit / nheads;
     const int h = unit - b * nheads;
     const int g = h / (nheads / ngroups);
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const bool qon = lane < (dstate >> 2);             // this lane's quad exists (dstate <= 128)
-    const int p0 = warp * RPW;
+    const int grp = lane >> 2, L = lane & 3;
+    const int nq = dstate >> 2;                        // quads in a row (<= 32)
+    const int p0 = warp * 8 * R;                       // rows p0 + 8i + grp, i < R
     const size_t units = (size_t)batch * nheads;
     const float Ah = A[h], Dh = D[h];
+    volatile int* abort = &abort_flag;
 
-    float4 s[RPW];
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStepStages; ++i) {
+            ptx::mbar_init(&full[i], 1);
+            ptx::mbar_init(&empty[i], kDecodeWarps);
+        }
+        abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+
+    // lane 0 of warp k % kStepStages: the copies of step k into stage k % kStepStages, once
+    // every warp has finished the step that used the stage before
+    int last_issued = -1;
+    auto issue = [&](int k) -> bool {
+        const int st = k % kStepStages;
+        if (k >= kStepStages && !ptx::mbar_wait_or_abort(&empty[st], ((k / kStepStages) - 1) & 1, err, abort))
+            return false;
+        uint8_t* sp = stage_mem + (size_t)st * stage_bytes;
+        const size_t bc = ((size_t)k * batch * ngroups + (size_t)b * ngroups + g) * dstate;
+        ptx::cp_async_4(sp + xbytes + 2 * nbytes, dt + (size_t)k * units + unit);
+        ptx::cp_async_mbar_arrive(&full[st]);          // before the arrival below
+        ptx::mbar_expect_tx(&full[st], (uint32_t)((headdim + 2 * dstate) * sizeof(T)));
+        ptx::bulk_load(sp, x + ((size_t)k * units + unit) * headdim, headdim * sizeof(T), &full[st]);
+        ptx::bulk_load(sp + xbytes, Bm + bc, dstate * sizeof(T), &full[st]);
+        ptx::bulk_load(sp + xbytes + nbytes, Cm + bc, dstate * sizeof(T), &full[st]);
+        last_issued = k;
+        return true;
+    };
+    if (lane == 0 && warp < steps && warp < kStepAhead) issue(warp);
+
+    // rows of this lane that exist (headdim is a multiple of 8: all 8 groups of a warp agree)
+    bool row_on[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) row_on[i] = p0 + 8 * i < headdim;
+    float4 s[R][8];
     float* S = state + (size_t)unit * headdim * dstate;
 #pragma unroll
-    for (int r = 0; r < RPW; ++r)
-        if (p0 + r < headdim && qon) s[r] = *reinterpret_cast<const float4*>(S + (size_t)(p0 + r) * dstate + 4 * lane);
+    for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+            s[i][m] = row_on[i] && L + 4 * m < nq
+                          ? *reinterpret_cast<const float4*>(S + (size_t)(p0 + 8 * i + grp) * dstate + 4 * (L + 4 * m))
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
 
-    // the inputs of step k: dt, B_t and C_t (this lane's quad), x of this warp's rows
-    auto load_step = [&](int k, float& dtv, float4& bq, float4& cq, float (&xv)[RPW]) {
-        dtv = dt[(size_t)k * units + unit];
-        const size_t bc = ((size_t)k * batch * ngroups + (size_t)b * ngroups + g) * dstate;
-        bq = qon ? load4<T>(Bm + bc + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
-        cq = qon ? load4<T>(Cm + bc + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
-        const T* xr = x + ((size_t)k * units + unit) * headdim;
-#pragma unroll
-        for (int r = 0; r < RPW; ++r) xv[r] = p0 + r < headdim ? Elem<T>::load(xr + p0 + r) : 0.f;
-    };
-    float dtn = 0.f, xn[RPW];
-    float4 bn, cn;
-    if (steps > 0) load_step(0, dtn, bn, cn, xn);
     for (int k = 0; k < steps; ++k) {
-        const float dtv = dtn;
-        const float4 bq = bn, cq = cn;
-        float xv[RPW];
-#pragma unroll
-        for (int r = 0; r < RPW; ++r) xv[r] = xn[r];
-        if (k + 1 < steps) load_step(k + 1, dtn, bn, cn, xn);
+        if (lane == 0 && k + kStepAhead < steps && (k + kStepAhead) % kStepStages == warp && !issue(k + kStepAhead))
+            *abort = 1;
+        const int st = k % kStepStages;
+        if (!ptx::mbar_wait_or_abort(&full[st], (k / kStepStages) & 1, err, abort)) break;
+        const uint8_t* sp = stage_mem + (size_t)st * stage_bytes;
+        const T* sx = reinterpret_cast<const T*>(sp);
+        const T* sb = reinterpret_cast<const T*>(sp + xbytes);
+        const T* sc = reinterpret_cast<const T*>(sp + xbytes + nbytes);
+        const float dtv = *reinterpret_cast<const float*>(sp + xbytes + 2 * nbytes);
         const float a = expf(dtv * Ah);                // fp32 decay exponent
-        T* yr = y + ((size_t)k * units + unit) * headdim;
+        float xv[R], acc[R];
 #pragma unroll
-        for (int r = 0; r < RPW; ++r) {
-            const int p = p0 + r;
-            if (p >= headdim) break;                   // warp-uniform
-            const float dx = dtv * xv[r];
-            float acc = 0.f;
-            if (qon) {
-                float4 v = s[r];
-                v.x = fmaf(a, v.x, dx * bq.x);
-                v.y = fmaf(a, v.y, dx * bq.y);
-                v.z = fmaf(a, v.z, dx * bq.z);
-                v.w = fmaf(a, v.w, dx * bq.w);
-                acc = fmaf(cq.x, v.x, acc);
-                acc = fmaf(cq.y, v.y, acc);
-                acc = fmaf(cq.z, v.z, acc);
-                acc = fmaf(cq.w, v.w, acc);
-                s[r] = v;
+        for (int i = 0; i < R; ++i) xv[i] = row_on[i] ? Elem<T>::load(sx + p0 + 8 * i + grp) : 0.f;
+        float part[R][8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const bool qon = L + 4 * m < nq;
+            const float4 bq = qon ? load4<T>(sb + 4 * (L + 4 * m)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 cq = qon ? load4<T>(sc + 4 * (L + 4 * m)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                const float dx = dtv * xv[i];
+                float pa = 0.f;
+                if (qon) {
+                    float4 v = s[i][m];
+                    v.x = fmaf(a, v.x, dx * bq.x);
+                    v.y = fmaf(a, v.y, dx * bq.y);
+                    v.z = fmaf(a, v.z, dx * bq.z);
+                    v.w = fmaf(a, v.w, dx * bq.w);
+                    pa = fmaf(cq.x, v.x, pa);
+                    pa = fmaf(cq.y, v.y, pa);
+                    pa = fmaf(cq.z, v.z, pa);
+                    pa = fmaf(cq.w, v.w, pa);
+                    s[i][m] = v;
+                }
+                part[i][m] = pa;
             }
-            acc = warp_sum(acc);
-            if (lane == 0) Elem<T>::store(yr + p, fmaf(Dh, xv[r], acc));
         }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&empty[st]);   // the stage may be refilled
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            // quad levels 16, 8, 4 inside the lane, then 2 and 1 across the group
+            float t0 = part[i][0] + part[i][4], t1 = part[i][1] + part[i][5];
+            float t2 = part[i][2] + part[i][6], t3 = part[i][3] + part[i][7];
+            t0 = t0 + t2;
+            t1 = t1 + t3;
+            float v = t0 + t1;
+            v += __shfl_xor_sync(0xffffffffu, v, 2);
+            v += __shfl_xor_sync(0xffffffffu, v, 1);
+            acc[i] = v;
+        }
+        if (L == 0) {
+            T* yr = y + ((size_t)k * units + unit) * headdim + p0 + grp;
+#pragma unroll
+            for (int i = 0; i < R; ++i)
+                if (row_on[i]) Elem<T>::store(yr + 8 * i, fmaf(Dh, xv[i], acc[i]));
+        }
+        if (*abort) break;
     }
 #pragma unroll
-    for (int r = 0; r < RPW; ++r)
-        if (p0 + r < headdim && qon) *reinterpret_cast<float4*>(S + (size_t)(p0 + r) * dstate + 4 * lane) = s[r];
+    for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+            if (row_on[i] && L + 4 * m < nq)
+                *reinterpret_cast<float4*>(S + (size_t)(p0 + 8 * i + grp) * dstate + 4 * (L + 4 * m)) = s[i][m];
+    // the CTA does not exit with copies in flight: each warp waits for the last fill of its stage
+    __syncthreads();
+    if (lane == 0 && last_issued >= 0)
+        ptx::mbar_wait(&full[last_issued % kStepStages], (last_issued / kStepStages) & 1, err);
 }
 
 // Shapes whose state does not fit in registers: the single step's body once per step, still
@@ -260,12 +354,15 @@ cudaError_t launch_steps_dtype(const Dims& d, int steps, float* state, const voi
     const T* Bt = static_cast<const T*>(B);
     const T* Ct = static_cast<const T*>(C);
     T* yt = static_cast<T*>(y);
+    const size_t smem = (size_t)kStepStages * (step_row_bytes<T>(d.headdim) + 2 * step_row_bytes<T>(d.dstate) + 16);
     if (d.dstate <= 128 && d.headdim <= 64)
-        decode_steps_kernel<T, 8><<<grid, kDecodeThreads, 0, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch,
-                                                                  d.nheads, d.headdim, d.ngroups, d.dstate);
+        decode_steps_kernel<T, 1><<<grid, kDecodeThreads, smem, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch,
+                                                                     d.nheads, d.headdim, d.ngroups, d.dstate,
+                                                                     device_error_word());
     else if (d.dstate <= 128)
-        decode_steps_kernel<T, 16><<<grid, kDecodeThreads, 0, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch,
-                                                                   d.nheads, d.headdim, d.ngroups, d.dstate);
+        decode_steps_kernel<T, 2><<<grid, kDecodeThreads, smem, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch,
+                                                                      d.nheads, d.headdim, d.ngroups, d.dstate,
+                                                                      device_error_word());
     else if (d.dstate <= 256)
         decode_steps_loop_kernel<T, 2, 4><<<grid, kDecodeThreads, 0, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps,
                                                                           d.batch, d.nheads, d.headdim, d.ngroups,
