@@ -280,11 +280,12 @@ decode_steps_kernel(float* __restrict__ state, const T* __restrict__ x, const fl
                 const float dx = dtv * xv[i];
                 float pa = 0.f;
                 if (qon) {
+                    // a v + (dx b) per element, two elements per packed instruction
+                    const float2 dx2 = make_float2(dx, dx), a2 = make_float2(a, a);
                     float4 v = s[i][m];
-                    v.x = fmaf(a, v.x, dx * bq.x);
-                    v.y = fmaf(a, v.y, dx * bq.y);
-                    v.z = fmaf(a, v.z, dx * bq.z);
-                    v.w = fmaf(a, v.w, dx * bq.w);
+                    const float2 vxy = ptx::ffma2(a2, make_float2(v.x, v.y), ptx::fmul2(dx2, make_float2(bq.x, bq.y)));
+                    const float2 vzw = ptx::ffma2(a2, make_float2(v.z, v.w), ptx::fmul2(dx2, make_float2(bq.z, bq.w)));
+                    v = make_float4(vxy.x, vxy.y, vzw.x, vzw.y);
                     pa = fmaf(cq.x, v.x, pa);
                     pa = fmaf(cq.y, v.y, pa);
                     pa = fmaf(cq.z, v.z, pa);
