@@ -62,6 +62,10 @@ WORKLOADS = {
                               steps=1024, dtype="f32"),
     "decode_steps_2p7b_b1": dict(kind="decode_steps", batch=1, nheads=80, headdim=64, ngroups=1, dstate=128,
                                  steps=1024, dtype="f32"),
+    # ssd_decode_steps_layers: 64 layers of the 2.7B shape at batch 1 advanced by 64 tokens in
+    # one launch, against one ssd_decode_step_layers launch per token (a CUDA graph)
+    "decode_steps_stack_b1": dict(kind="decode_steps", layers=64, batch=1, nheads=80, headdim=64, ngroups=1,
+                                  dstate=128, steps=64, dtype="f32"),
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -553,10 +557,78 @@ def run_decode(w, repeats, warmup, rank, world):
     return res
 
 
+def _timed_rate(fn, steps, repeats, warmup, world):
+    """Steps/s of `fn` (one call = `steps` steps) over `repeats` calls, CUDA events, after
+    `warmup` calls; max over ranks."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(repeats):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return whole_job_rate(steps * repeats, e0.elapsed_time(e1), world)
+
+
+def run_decode_steps_stack(w, repeats, warmup, rank, world):
+    """A stack of layers advanced by the workload's tokens two ways on the same
+    device-resident per-layer inputs: one ssd_decode_step_layers launch per token (the whole
+    stack, captured in a CUDA graph), and one ssd_decode_steps_layers launch for all tokens.
+    Both compute the same result bit for bit."""
+    import torch
+    import state_space_model_05_b200 as ssd
+    L, b, H, P, G, N, S = (w[k] for k in ("layers", "batch", "nheads", "headdim", "ngroups", "dstate", "steps"))
+    shape = gen.SSDShape(b, 1, H, P, G, N)
+    f32 = torch.float32
+    layers = []
+    for l in range(L):
+        dec = gen.decode_inputs(shape, steps=S, seed=3000 + 10 * l + rank)
+        A, D = gen.deep_head_params(l, H)
+        X = _dev(dec.x, f32)
+        layers.append(dict(state=_dev(gen.state_inputs(b, H, P, N, seed=3001 + 10 * l + rank), f32), x_t=X,
+                           dt_t=_dev(dec.dt, f32), A=_dev(A, f32), B_t=_dev(dec.B, f32), C_t=_dev(dec.C, f32),
+                           D=_dev(D, f32), y_t=torch.empty_like(X)))
+    table = ssd.decode_layer_table(layers)
+    per_token = [ssd.decode_layer_table([dict(ly, x_t=ly["x_t"][k], dt_t=ly["dt_t"][k], B_t=ly["B_t"][k],
+                                              C_t=ly["C_t"][k], y_t=ly["y_t"][k]) for ly in layers])
+                 for k in range(S)]
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for k in range(2):
+            ssd.ssd_decode_step_layers(per_token[k], b, H, P, G, N, f32)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            for k in range(S):
+                ssd.ssd_decode_step_layers(per_token[k], b, H, P, G, N, f32)
+    per_step, _ = _timed_rate(graph.replay, S, repeats, warmup, world)
+    one_launch, ms = _timed_rate(lambda: ssd.ssd_decode_steps_layers(table, S, b, H, P, G, N, f32), S, repeats,
+                                 warmup, world)
+    if ssd.ssd_device_status() != 0:
+        raise RuntimeError("device status after stacked decode steps")
+    del graph
+    # one launch: every layer's state read and written once per call, its inputs and y once
+    io = L * (S * (2 * b * H * P * 4 + 2 * b * G * N * 4 + b * H * 4) + 2 * b * H * P * N * 4)
+    return {"steps_per_s_one_launch": one_launch, "steps_per_s_launch_per_step": per_step,
+            "us_per_step_one_launch": ms / (S * repeats) * 1e3, "bytes_per_call": io,
+            "gbs": io * repeats / (ms / 1e3) / 1e9}
+
+
 def run_decode_steps(w, repeats, warmup, rank, world):
     """The decode workload's steps run two ways on the same device-resident inputs: one
     ssd_decode_step launch per token (captured in a CUDA graph), and one ssd_decode_steps
-    launch for all of them.  Both compute the same result bit for bit."""
+    launch for all of them.  Both compute the same result bit for bit.  A workload with
+    several layers runs the stack version."""
+    if w.get("layers", 1) > 1:
+        return run_decode_steps_stack(w, repeats, warmup, rank, world)
     import torch
     import state_space_model_05_b200 as ssd
     b, H, P, G, N, S = (w[k] for k in ("batch", "nheads", "headdim", "ngroups", "dstate", "steps"))
@@ -875,7 +947,7 @@ def ours(args, rank, world):
         vr = run_prefill_varlen(pw, 100, 5, rank, world)
         extras["prefill_130m_varlen"] = {"value": vr["tokens_per_s"], "unit": "tokens/s",
                                          "ms_per_step": vr["ms_per_step"], "sequences": vr["lengths"]}
-        for name in ("decode_steps_2p7b", "decode_steps_2p7b_b1"):
+        for name in ("decode_steps_2p7b", "decode_steps_2p7b_b1", "decode_steps_stack_b1"):
             sw = WORKLOADS[name]
             r = run_decode_steps(sw, 5, 2, rank, world)
             extras[name] = {"value": r["steps_per_s_one_launch"], "unit": "steps/s",

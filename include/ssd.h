@@ -239,6 +239,25 @@ ssd_status_t ssd_decode_step_layers(const ssd_decode_layer_t* layers, int n_laye
                                     ssd_dtype_t dtype, void* stream);
 
 /*
+ * `steps` successive decode steps of every layer of a stack in one launch: the stack's O(1)
+ * caches advanced by a device-side loop with no host round trip per token ("Compiler-First
+ * State Space Duality and Portable O(1) Autoregressive Caching for Inference", section
+ * "2. Metodologia"), for tokens whose per-layer inputs are already on the device.  Each of
+ * the n_layers entries of `layers` (a DEVICE array, as for ssd_decode_step_layers) holds the
+ * arguments of ssd_decode_steps for its layer: x_t, dt_t, B_t, C_t and y_t point at that
+ * layer's [steps][...] arrays.  The result equals ssd_decode_steps on each layer (and so
+ * `steps` calls of ssd_decode_step per layer) bit for bit.  Sizes are checked on the host
+ * (SSD_ERR_SHAPE/DTYPE/UNSUPPORTED; steps < 0 or n_layers outside [0, 65535] is
+ * SSD_ERR_SHAPE; SSD_ERR_NULL for a NULL table); entries on the device as for
+ * ssd_decode_step_layers (a NULL or misaligned entry is skipped and recorded in the device
+ * error word).  steps = 0 or n_layers = 0 does nothing.  No state buffer may overlap another
+ * layer's buffers or any input.
+ */
+ssd_status_t ssd_decode_steps_layers(const ssd_decode_layer_t* layers, int n_layers, int steps, int batch,
+                                     int nheads, int headdim, int ngroups, int dstate, ssd_dtype_t dtype,
+                                     void* stream);
+
+/*
  * Gated DeltaNet decode step (a second recurrent workload, on its own state cache):
  * "Persistent-State Dataflow Accelerator for Memory-Bound Linear Attention Decode on
  * FPGA", section 2.B.  Per (b, value head h), with query/key head hk = h / (heads_v /

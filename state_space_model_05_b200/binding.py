@@ -36,6 +36,7 @@ SIGNATURES = {
     "ssd_decode_step": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ssd_decode_steps": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ssd_decode_step_layers": ([_P, _I, _I, _I, _I, _I, _I, _I, _P], _I),
+    "ssd_decode_steps_layers": ([_P, _I, _I, _I, _I, _I, _I, _I, _I, _P], _I),
     "ssd_gdn_decode_step": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ssd_prefill_varlen_workspace_bytes": ([_I, _I, _I, _I, _I, _I, _I, _I], _Z),
     "ssd_prefill_varlen": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _Z, _P], _I),
@@ -305,6 +306,17 @@ def ssd_decode_step_layers(table, batch, nheads, headdim, ngroups, dstate, dtype
     st = lib().ssd_decode_step_layers(_ptr(table), table.shape[0], batch, nheads, headdim, ngroups,
                                       dstate, code, _stream(stream))
     _check(st, "ssd_decode_step_layers")
+
+
+def ssd_decode_steps_layers(table, steps, batch, nheads, headdim, ngroups, dstate, dtype, stream=None):
+    """``steps`` decode steps of every layer in ``table`` (from decode_layer_table, whose
+    per-step entries point at each layer's [steps][...] arrays), one launch."""
+    if not table.is_cuda or table.dtype != torch.int64 or table.dim() != 2 or table.shape[1] != len(LAYER_FIELDS):
+        raise ValueError("table must be a CUDA int64 [n_layers][8] tensor")
+    code = SSD_BF16 if dtype in (torch.bfloat16, SSD_BF16) else SSD_F32
+    st = lib().ssd_decode_steps_layers(_ptr(table), table.shape[0], steps, batch, nheads, headdim, ngroups,
+                                       dstate, code, _stream(stream))
+    _check(st, "ssd_decode_steps_layers")
 
 
 def ssd_gdn_decode_step(state, q, k, v, gate, beta, out=None, stream=None):

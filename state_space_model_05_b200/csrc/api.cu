@@ -68,12 +68,12 @@ ssd_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_E
 
 // ---- opt-in kernel profiling: an event pair around each launch -------------------
 enum Stage { kCumsum, kStateTc, kStateSimt, kScan, kOutTc, kOutSimt, kDecode, kCopy, kDecodeLayers, kGdn,
-             kGram, kChain, kDecodeSteps, kNumStages };
+             kGram, kChain, kDecodeSteps, kDecodeStepsLayers, kNumStages };
 const char* const kStageNames[kNumStages] = {"chunk_cumsum", "chunk_state_scan_tc", "chunk_state_simt",
                                               "state_scan", "chunk_output_tc", "chunk_output_simt",
                                               "decode_step", "copy_state", "decode_step_layers",
                                               "gdn_decode_step", "block_gram_tc", "chain_prefill_tc",
-                                              "decode_steps"};
+                                              "decode_steps", "decode_steps_layers"};
 
 // which tensor-core prefill batched calls take (ssd_set_prefill_path)
 std::atomic<int> g_prefill_path{SSD_PREFILL_AUTO};
@@ -422,6 +422,23 @@ ssd_status_t ssd_decode_step_layers(const ssd_decode_layer_t* layers, int n_laye
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return from_cuda(profiled(kDecodeLayers, s, [&] {
         return launch_decode_layers(d, dtype, layers, n_layers, s);
+    }));
+}
+
+ssd_status_t ssd_decode_steps_layers(const ssd_decode_layer_t* layers, int n_layers, int steps, int batch,
+                                     int nheads, int headdim, int ngroups, int dstate, ssd_dtype_t dtype,
+                                     void* stream)
+{
+    ssd_status_t st = check_common(batch, nheads, headdim, ngroups, dstate, dtype, 512);
+    if (st != SSD_OK) return st;
+    if (n_layers < 0 || n_layers > 65535 || steps < 0) return SSD_ERR_SHAPE;
+    if (batch == 0 || n_layers == 0 || steps == 0) return SSD_OK;
+    if (!layers) return SSD_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(layers) % alignof(ssd_decode_layer_t)) return SSD_ERR_ALIGN;
+    Dims d{batch, 1, nheads, headdim, ngroups, dstate, 1, 1};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return from_cuda(profiled(kDecodeStepsLayers, s, [&] {
+        return launch_decode_steps_layers(d, dtype, layers, n_layers, steps, s);
     }));
 }
 

@@ -101,6 +101,10 @@ cudaError_t launch_gdn_decode(ssd_dtype_t dtype, float* state, const void* q, co
 cudaError_t launch_decode_layers(const Dims& d, ssd_dtype_t dtype, const ssd_decode_layer_t* layers,
                                  int n_layers, cudaStream_t s);
 
+// `steps` successive decode steps of every layer of a table, one launch.
+cudaError_t launch_decode_steps_layers(const Dims& d, ssd_dtype_t dtype, const ssd_decode_layer_t* layers,
+                                       int n_layers, int steps, cudaStream_t s);
+
 // `steps` successive decode steps in one launch (inputs and outputs [steps][...]).
 cudaError_t launch_decode_steps(const Dims& d, ssd_dtype_t dtype, int steps, float* state, const void* x,
                                 const float* dt, const float* A, const void* B, const void* C, const float* D,

@@ -129,24 +129,32 @@ decode_step_kernel(float* __restrict__ state, const T* __restrict__ x, const flo
 
 // Every layer of a stack in one launch: blockIdx.y is the layer, whose tensors come from
 // the table.  A layer entry with a null or misaligned pointer is skipped and recorded.
-template <typename T, int QPL, int ROWS>
-__global__ void __launch_bounds__(kDecodeThreads, QPL == 1 ? 4 : 2)
-decode_layers_kernel(const ssd_decode_layer_t* __restrict__ layers, int nheads, int headdim,
-                     int ngroups, int dstate, int* err)
+// A layer table entry is used when none of its pointers is null and all are 16-byte
+// aligned; otherwise the CTA skips it and thread 0 records SSD_ERR_NULL / SSD_ERR_ALIGN.
+__device__ __forceinline__ bool layer_entry_ok(const ssd_decode_layer_t& L, int* err)
 {
-    const ssd_decode_layer_t L = layers[blockIdx.y];
     const uintptr_t any = reinterpret_cast<uintptr_t>(L.state) | reinterpret_cast<uintptr_t>(L.x_t) |
                           reinterpret_cast<uintptr_t>(L.dt_t) | reinterpret_cast<uintptr_t>(L.A) |
                           reinterpret_cast<uintptr_t>(L.B_t) | reinterpret_cast<uintptr_t>(L.C_t) |
                           reinterpret_cast<uintptr_t>(L.D) | reinterpret_cast<uintptr_t>(L.y_t);
     if (!L.state || !L.x_t || !L.dt_t || !L.A || !L.B_t || !L.C_t || !L.D || !L.y_t) {
         if (threadIdx.x == 0) record_error(err, SSD_ERR_NULL);
-        return;
+        return false;
     }
     if (any & 15u) {
         if (threadIdx.x == 0) record_error(err, SSD_ERR_ALIGN);
-        return;
+        return false;
     }
+    return true;
+}
+
+template <typename T, int QPL, int ROWS>
+__global__ void __launch_bounds__(kDecodeThreads, QPL == 1 ? 4 : 2)
+decode_layers_kernel(const ssd_decode_layer_t* __restrict__ layers, int nheads, int headdim,
+                     int ngroups, int dstate, int* err)
+{
+    const ssd_decode_layer_t L = layers[blockIdx.y];
+    if (!layer_entry_ok(L, err)) return;
     decode_unit<T, QPL, ROWS>(L.state, static_cast<const T*>(L.x_t), L.dt_t, L.A,
                               static_cast<const T*>(L.B_t), static_cast<const T*>(L.C_t), L.D,
                               static_cast<T*>(L.y_t), blockIdx.x, nheads, headdim, ngroups, dstate);
@@ -183,12 +191,13 @@ static_assert(kStepStages == kDecodeWarps, "stage w is filled by warp w");
 template <typename T>
 __host__ __device__ constexpr int step_row_bytes(int n) { return (int)((n * sizeof(T) + 15) & ~size_t(15)); }
 
+// The steps of (b, h) unit `unit` of one layer (the CTA's whole work).
 template <typename T, int R>
-__global__ void __launch_bounds__(kDecodeThreads, R == 1 ? 3 : 1)
-decode_steps_kernel(float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
-                    const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
-                    const float* __restrict__ D, T* __restrict__ y, int steps, int batch, int nheads,
-                    int headdim, int ngroups, int dstate, int* err)
+__device__ __forceinline__ void steps_unit(float* __restrict__ state, const T* __restrict__ x,
+                                           const float* __restrict__ dt, const float* __restrict__ A,
+                                           const T* __restrict__ Bm, const T* __restrict__ Cm,
+                                           const float* __restrict__ D, T* __restrict__ y, int steps, int batch,
+                                           int nheads, int headdim, int ngroups, int dstate, int unit, int* err)
 {
     static_assert(R == 1 || R == 2, "rows per lane group");
     extern __shared__ __align__(16) uint8_t stage_mem[]; // per stage: x row | B_t row | C_t row | dt
@@ -198,7 +207,6 @@ decode_steps_kernel(float* __restrict__ state, const T* __restrict__ x, const fl
     const int nbytes = step_row_bytes<T>(dstate);
     const int stage_bytes = xbytes + 2 * nbytes + 16;
 
-    const int unit = blockIdx.x;
     const int b = unit / nheads;
     const int h = unit - b * nheads;
     const int g = h / (nheads / ngroups);
@@ -329,8 +337,46 @@ decode_steps_kernel(float* __restrict__ state, const T* __restrict__ x, const fl
         ptx::mbar_wait(&full[last_issued % kStepStages], (last_issued / kStepStages) & 1, err);
 }
 
+template <typename T, int R>
+__global__ void __launch_bounds__(kDecodeThreads, R == 1 ? 3 : 1)
+decode_steps_kernel(float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
+                    const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
+                    const float* __restrict__ D, T* __restrict__ y, int steps, int batch, int nheads,
+                    int headdim, int ngroups, int dstate, int* err)
+{
+    steps_unit<T, R>(state, x, dt, A, Bm, Cm, D, y, steps, batch, nheads, headdim, ngroups, dstate, blockIdx.x, err);
+}
+
+// The same for every layer of a table (blockIdx.y = layer): each entry's per-step pointers
+// address [steps][...] arrays, so one launch advances the whole stack by `steps` tokens.
+template <typename T, int R>
+__global__ void __launch_bounds__(kDecodeThreads, R == 1 ? 3 : 1)
+decode_steps_layers_kernel(const ssd_decode_layer_t* __restrict__ layers, int steps, int batch, int nheads,
+                           int headdim, int ngroups, int dstate, int* err)
+{
+    const ssd_decode_layer_t L = layers[blockIdx.y];
+    if (!layer_entry_ok(L, err)) return;
+    steps_unit<T, R>(L.state, static_cast<const T*>(L.x_t), L.dt_t, L.A, static_cast<const T*>(L.B_t),
+                     static_cast<const T*>(L.C_t), L.D, static_cast<T*>(L.y_t), steps, batch, nheads, headdim,
+                     ngroups, dstate, blockIdx.x, err);
+}
+
 // Shapes whose state does not fit in registers: the single step's body once per step, still
 // one launch (each CTA owns its unit's state, so the steps need no synchronisation).
+template <typename T, int QPL, int ROWS>
+__device__ __forceinline__ void steps_loop_unit(float* __restrict__ state, const T* __restrict__ x,
+                                                const float* __restrict__ dt, const float* __restrict__ A,
+                                                const T* __restrict__ Bm, const T* __restrict__ Cm,
+                                                const float* __restrict__ D, T* __restrict__ y, int steps,
+                                                int batch, int nheads, int headdim, int ngroups, int dstate)
+{
+    const size_t units = (size_t)batch * nheads;
+    for (int k = 0; k < steps; ++k)
+        decode_unit<T, QPL, ROWS>(state, x + (size_t)k * units * headdim, dt + (size_t)k * units, A,
+                                  Bm + (size_t)k * batch * ngroups * dstate, Cm + (size_t)k * batch * ngroups * dstate,
+                                  D, y + (size_t)k * units * headdim, blockIdx.x, nheads, headdim, ngroups, dstate);
+}
+
 template <typename T, int QPL, int ROWS>
 __global__ void __launch_bounds__(kDecodeThreads, QPL == 1 ? 4 : 2)
 decode_steps_loop_kernel(float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
@@ -338,11 +384,19 @@ decode_steps_loop_kernel(float* __restrict__ state, const T* __restrict__ x, con
                          const float* __restrict__ D, T* __restrict__ y, int steps, int batch, int nheads,
                          int headdim, int ngroups, int dstate)
 {
-    const size_t units = (size_t)batch * nheads;
-    for (int k = 0; k < steps; ++k)
-        decode_unit<T, QPL, ROWS>(state, x + (size_t)k * units * headdim, dt + (size_t)k * units, A,
-                                  Bm + (size_t)k * batch * ngroups * dstate, Cm + (size_t)k * batch * ngroups * dstate,
-                                  D, y + (size_t)k * units * headdim, blockIdx.x, nheads, headdim, ngroups, dstate);
+    steps_loop_unit<T, QPL, ROWS>(state, x, dt, A, Bm, Cm, D, y, steps, batch, nheads, headdim, ngroups, dstate);
+}
+
+template <typename T, int QPL, int ROWS>
+__global__ void __launch_bounds__(kDecodeThreads, QPL == 1 ? 4 : 2)
+decode_steps_layers_loop_kernel(const ssd_decode_layer_t* __restrict__ layers, int steps, int batch,
+                                int nheads, int headdim, int ngroups, int dstate, int* err)
+{
+    const ssd_decode_layer_t L = layers[blockIdx.y];
+    if (!layer_entry_ok(L, err)) return;
+    steps_loop_unit<T, QPL, ROWS>(L.state, static_cast<const T*>(L.x_t), L.dt_t, L.A,
+                                  static_cast<const T*>(L.B_t), static_cast<const T*>(L.C_t), L.D,
+                                  static_cast<T*>(L.y_t), steps, batch, nheads, headdim, ngroups, dstate);
 }
 
 template <typename T>
@@ -372,6 +426,28 @@ cudaError_t launch_steps_dtype(const Dims& d, int steps, float* state, const voi
         decode_steps_loop_kernel<T, 4, 2><<<grid, kDecodeThreads, 0, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps,
                                                                           d.batch, d.nheads, d.headdim, d.ngroups,
                                                                           d.dstate);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_steps_layers_dtype(const Dims& d, const ssd_decode_layer_t* layers, int n_layers, int steps,
+                                      cudaStream_t s)
+{
+    const dim3 grid((unsigned)(d.batch * d.nheads), (unsigned)n_layers);
+    const size_t smem = (size_t)kStepStages * (step_row_bytes<T>(d.headdim) + 2 * step_row_bytes<T>(d.dstate) + 16);
+    int* err = device_error_word();
+    if (d.dstate <= 128 && d.headdim <= 64)
+        decode_steps_layers_kernel<T, 1><<<grid, kDecodeThreads, smem, s>>>(layers, steps, d.batch, d.nheads,
+                                                                            d.headdim, d.ngroups, d.dstate, err);
+    else if (d.dstate <= 128)
+        decode_steps_layers_kernel<T, 2><<<grid, kDecodeThreads, smem, s>>>(layers, steps, d.batch, d.nheads,
+                                                                            d.headdim, d.ngroups, d.dstate, err);
+    else if (d.dstate <= 256)
+        decode_steps_layers_loop_kernel<T, 2, 4><<<grid, kDecodeThreads, 0, s>>>(layers, steps, d.batch, d.nheads,
+                                                                                 d.headdim, d.ngroups, d.dstate, err);
+    else
+        decode_steps_layers_loop_kernel<T, 4, 2><<<grid, kDecodeThreads, 0, s>>>(layers, steps, d.batch, d.nheads,
+                                                                                 d.headdim, d.ngroups, d.dstate, err);
     return cudaGetLastError();
 }
 
@@ -433,6 +509,14 @@ cudaError_t launch_decode_steps(const Dims& d, ssd_dtype_t dtype, int steps, flo
     if (d.batch == 0 || steps == 0) return cudaSuccess;
     if (dtype == SSD_F32) return launch_steps_dtype<float>(d, steps, state, x, dt, A, B, C, D, y, s);
     return launch_steps_dtype<__nv_bfloat16>(d, steps, state, x, dt, A, B, C, D, y, s);
+}
+
+cudaError_t launch_decode_steps_layers(const Dims& d, ssd_dtype_t dtype, const ssd_decode_layer_t* layers,
+                                       int n_layers, int steps, cudaStream_t s)
+{
+    if (d.batch == 0 || n_layers == 0 || steps == 0) return cudaSuccess;
+    if (dtype == SSD_F32) return launch_steps_layers_dtype<float>(d, layers, n_layers, steps, s);
+    return launch_steps_layers_dtype<__nv_bfloat16>(d, layers, n_layers, steps, s);
 }
 
 cudaError_t launch_decode(const Dims& d, ssd_dtype_t dtype, float* state, const void* x,

@@ -159,6 +159,24 @@ def test_decode_layers_validation(lib):
     assert f(None, 4, 0, 8, 64, 4, 128, binding.SSD_F32, None) == 0
 
 
+def test_decode_steps_layers_validation(lib):
+    """The multi-step stack call validates sizes on the host before any launch, like the
+    one-step stack call, and also rejects a negative step count."""
+    f = lib.ssd_decode_steps_layers
+    F32 = binding.SSD_F32
+    assert f(FAKE, 4, 3, 2, 6, 64, 4, 128, F32, None) == 2       # nheads % ngroups
+    assert f(FAKE, 4, 3, 2, 8, 64, 4, 1024, F32, None) == 5      # dstate > 512
+    assert f(FAKE, 4, 3, 2, 8, 64, 4, 128, 7, None) == 3         # dtype
+    assert f(FAKE, -1, 3, 2, 8, 64, 4, 128, F32, None) == 2      # n_layers < 0
+    assert f(FAKE, 65536, 3, 2, 8, 64, 4, 128, F32, None) == 2   # n_layers > 65535
+    assert f(FAKE, 4, -1, 2, 8, 64, 4, 128, F32, None) == 2      # steps < 0
+    assert f(None, 4, 3, 2, 8, 64, 4, 128, F32, None) == 1       # NULL table
+    assert f(FAKE + 4, 4, 3, 2, 8, 64, 4, 128, F32, None) == 4   # misaligned table
+    assert f(None, 0, 3, 2, 8, 64, 4, 128, F32, None) == 0       # nothing to do
+    assert f(None, 4, 0, 2, 8, 64, 4, 128, F32, None) == 0
+    assert f(None, 4, 3, 0, 8, 64, 4, 128, F32, None) == 0
+
+
 def test_dtraw_validation(lib):
     """The raw-dt variants validate like the plain calls, and reject a misaligned bias
     (every call here fails validation before any launch)."""

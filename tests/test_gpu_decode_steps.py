@@ -6,7 +6,9 @@ Inference", section "2. Metodologia").  For tokens whose inputs are on the devic
 launch runs the whole loop; it must give exactly what k launches of ssd_decode_step give
 (same arithmetic per row, so bitwise), and match the fp64 oracle stepped k times.
 Covered: the register-resident kernel (headdim <= 64 and <= 128, dstate <= 128), the
-looped kernel (dstate 256), bf16 inputs, odd small shapes, grouped B/C and steps = 0.
+looped kernel (dstate 256), bf16 inputs, odd small shapes, grouped B/C and steps = 0; and
+ssd_decode_steps_layers, the same loop over every layer of a table in one launch (bitwise
+equal to the per-layer call, oracle-checked, a bad entry skipped and reported).
 """
 import numpy as np
 import pytest
@@ -76,3 +78,62 @@ def test_zero_steps_leave_state_untouched():
     torch.cuda.synchronize()
     assert y.shape == (0, 2, 4, 64)
     assert np.array_equal(s.cpu().numpy(), st0)
+
+
+def _stack(nl, b, H, P, G, N, steps, dtype, seed):
+    """nl layers of one shape: per-layer tensors for the table, and what ssd_decode_steps
+    gives for each layer on its own (copies of the same start states)."""
+    from state_space_model_05_b200 import ssd_decode_steps
+    layers, refs = [], []
+    for l in range(nl):
+        dec, head, st0 = _case(b, H, P, G, N, steps, seed=seed + 10 * l, dtype=dtype)
+        X, DT, Bs, Cs = to_dev(dec.x, dtype), to_dev(dec.dt), to_dev(dec.B, dtype), to_dev(dec.C, dtype)
+        A, D = to_dev(head.A), to_dev(head.D)
+        layers.append(dict(state=to_dev(st0), x_t=X, dt_t=DT, A=A, B_t=Bs, C_t=Cs, D=D, y_t=torch.full_like(X, 7.0)))
+        s_ref = to_dev(st0)
+        refs.append((s_ref, ssd_decode_steps(s_ref, X, DT, A, Bs, Cs, D), dec, head, st0))
+    return layers, refs
+
+
+@pytest.mark.parametrize("P,N,dtype", [
+    (64, 128, torch.float32),      # register-resident, one row per lane group
+    (128, 128, torch.bfloat16),    # register-resident, two rows per lane group, bf16
+    (64, 256, torch.float32),      # looped kernel
+])
+def test_stack_steps_equal_per_layer_calls_bitwise(P, N, dtype):
+    """ssd_decode_steps_layers advances every layer of a table by k tokens in one launch:
+    bit for bit what ssd_decode_steps gives per layer (itself bitwise equal to k single
+    steps, above), and for fp32 within tolerance of the oracle stepped k times."""
+    from state_space_model_05_b200 import decode_layer_table, ssd_decode_steps_layers, ssd_device_status
+    b, H, G, steps, nl = 2, 4, 2, 13, 3
+    layers, refs = _stack(nl, b, H, P, G, N, steps, dtype, seed=300 + P + N)
+    ssd_decode_steps_layers(decode_layer_table(layers), steps, b, H, P, G, N, dtype)
+    assert ssd_device_status() == 0
+    for l, (layer, (s_ref, y_ref, dec, head, st0)) in enumerate(zip(layers, refs)):
+        assert torch.equal(layer["y_t"], y_ref), f"layer {l}: y differs from ssd_decode_steps"
+        assert torch.equal(layer["state"], s_ref), f"layer {l}: state differs from ssd_decode_steps"
+    if dtype == torch.float32:
+        layer, (_, _, dec, head, st0) = layers[1], refs[1]
+        ref = st0.reshape(b * H, P, N).astype(np.float64)
+        for k in range(steps):
+            yo = oracle.decode_step(ref, dec.x[k], dec.dt[k], head.A, dec.B[k], dec.C[k], head.D)
+            assert_fp32(layer["y_t"][k].cpu().numpy().reshape(b * H, P), yo, f"stack steps y, step {k}")
+        assert_fp32(layer["state"].cpu().numpy().reshape(b * H, P, N), ref, "stack steps final state")
+
+
+def test_stack_steps_bad_entry_skipped_and_reported():
+    """A table entry with a NULL pointer is skipped (its state and y untouched) and reported
+    through the device error word; the other layers are still advanced."""
+    from state_space_model_05_b200 import decode_layer_table, ssd_decode_steps_layers, ssd_device_status
+    b, H, P, G, N, steps = 2, 4, 64, 1, 128, 5
+    layers, refs = _stack(3, b, H, P, G, N, steps, torch.float32, seed=900)
+    table = decode_layer_table(layers)
+    table[1, 0] = 0                                   # layer 1: NULL state pointer
+    s1_before = layers[1]["state"].clone()
+    ssd_decode_steps_layers(table, steps, b, H, P, G, N, torch.float32)
+    assert ssd_device_status() == 1                   # SSD_ERR_NULL
+    assert torch.equal(layers[1]["state"], s1_before)
+    assert bool((layers[1]["y_t"] == 7.0).all())
+    for l in (0, 2):
+        assert torch.equal(layers[l]["y_t"], refs[l][1])
+        assert torch.equal(layers[l]["state"], refs[l][0])
