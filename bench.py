@@ -857,7 +857,8 @@ def ours(args, rank, world):
         res = run_decode_steps(w, max(1, args.steps // 4), max(1, args.warmup), rank, world)
         line.update({"metric": "SSD decode steps/s (all steps in one launch)", "value": res["steps_per_s_one_launch"],
                      "unit": "steps/s", "ms_per_step": res["us_per_step_one_launch"] / 1e3, "dtype": "f32"})
-        line["roofline"] = decode_roofline(res["gbs"], "decode_steps", peaks, src)
+        line["roofline"] = decode_roofline(res["gbs"], "decode_steps", peaks, src,
+                                           recorded_traffic("decode_steps", args.workload))
         line["launch_per_step_steps_per_s"] = res["steps_per_s_launch_per_step"]
         line["gpu_launches"] = max(1, args.steps // 4)
         line["e2e"] = None
@@ -954,7 +955,8 @@ def ours(args, rank, world):
                             "us_per_step": r["us_per_step_one_launch"],
                             "launch_per_step_steps_per_s": r["steps_per_s_launch_per_step"],
                             "roofline": decode_roofline(r["gbs"], "decode_steps (all steps, one launch; state "
-                                                        "read and written once per call)", peaks, src),
+                                                        "read and written once per call)", peaks, src,
+                                                        recorded_traffic("decode_steps", name)),
                             "config": {k: sw[k] for k in sw if k != "kind"}}
             summary[name] = {"steps_s": round(r["steps_per_s_one_launch"]),
                              "launch_per_step_steps_s": round(r["steps_per_s_launch_per_step"])}

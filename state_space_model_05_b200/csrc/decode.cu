@@ -191,8 +191,9 @@ static_assert(kStepStages == kDecodeWarps, "stage w is filled by warp w");
 template <typename T>
 __host__ __device__ constexpr int step_row_bytes(int n) { return (int)((n * sizeof(T) + 15) & ~size_t(15)); }
 
-// The steps of (b, h) unit `unit` of one layer (the CTA's whole work).
-template <typename T, int R>
+// The steps of (b, h) unit `unit` of one layer (the CTA's whole work).  FULL: dstate is 128,
+// so every lane holds all 8 of its quads (no per-quad presence tests).
+template <typename T, int R, bool FULL>
 __device__ __forceinline__ void steps_unit(float* __restrict__ state, const T* __restrict__ x,
                                            const float* __restrict__ dt, const float* __restrict__ A,
                                            const T* __restrict__ Bm, const T* __restrict__ Cm,
@@ -213,7 +214,7 @@ __device__ __forceinline__ void steps_unit(float* __restrict__ state, const T* _
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int grp = lane >> 2, L = lane & 3;
-    const int nq = dstate >> 2;                        // quads in a row (<= 32)
+    const int nq = FULL ? 32 : dstate >> 2;            // quads in a row (<= 32)
     const int p0 = warp * 8 * R;                       // rows p0 + 8i + grp, i < R
     const size_t units = (size_t)batch * nheads;
     const float Ah = A[h], Dh = D[h];
@@ -337,26 +338,26 @@ __device__ __forceinline__ void steps_unit(float* __restrict__ state, const T* _
         ptx::mbar_wait(&full[last_issued % kStepStages], (last_issued / kStepStages) & 1, err);
 }
 
-template <typename T, int R>
+template <typename T, int R, bool FULL>
 __global__ void __launch_bounds__(kDecodeThreads, R == 1 ? 3 : 1)
 decode_steps_kernel(float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
                     const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
                     const float* __restrict__ D, T* __restrict__ y, int steps, int batch, int nheads,
                     int headdim, int ngroups, int dstate, int* err)
 {
-    steps_unit<T, R>(state, x, dt, A, Bm, Cm, D, y, steps, batch, nheads, headdim, ngroups, dstate, blockIdx.x, err);
+    steps_unit<T, R, FULL>(state, x, dt, A, Bm, Cm, D, y, steps, batch, nheads, headdim, ngroups, dstate, blockIdx.x, err);
 }
 
 // The same for every layer of a table (blockIdx.y = layer): each entry's per-step pointers
 // address [steps][...] arrays, so one launch advances the whole stack by `steps` tokens.
-template <typename T, int R>
+template <typename T, int R, bool FULL>
 __global__ void __launch_bounds__(kDecodeThreads, R == 1 ? 3 : 1)
 decode_steps_layers_kernel(const ssd_decode_layer_t* __restrict__ layers, int steps, int batch, int nheads,
                            int headdim, int ngroups, int dstate, int* err)
 {
     const ssd_decode_layer_t L = layers[blockIdx.y];
     if (!layer_entry_ok(L, err)) return;
-    steps_unit<T, R>(L.state, static_cast<const T*>(L.x_t), L.dt_t, L.A, static_cast<const T*>(L.B_t),
+    steps_unit<T, R, FULL>(L.state, static_cast<const T*>(L.x_t), L.dt_t, L.A, static_cast<const T*>(L.B_t),
                      static_cast<const T*>(L.C_t), L.D, static_cast<T*>(L.y_t), steps, batch, nheads, headdim,
                      ngroups, dstate, blockIdx.x, err);
 }
@@ -410,22 +411,25 @@ cudaError_t launch_steps_dtype(const Dims& d, int steps, float* state, const voi
     const T* Ct = static_cast<const T*>(C);
     T* yt = static_cast<T*>(y);
     const size_t smem = (size_t)kStepStages * (step_row_bytes<T>(d.headdim) + 2 * step_row_bytes<T>(d.dstate) + 16);
-    if (d.dstate <= 128 && d.headdim <= 64)
-        decode_steps_kernel<T, 1><<<grid, kDecodeThreads, smem, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch,
-                                                                     d.nheads, d.headdim, d.ngroups, d.dstate,
-                                                                     device_error_word());
-    else if (d.dstate <= 128)
-        decode_steps_kernel<T, 2><<<grid, kDecodeThreads, smem, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch,
-                                                                      d.nheads, d.headdim, d.ngroups, d.dstate,
-                                                                      device_error_word());
-    else if (d.dstate <= 256)
+    int* err = device_error_word();
+    const bool full = d.dstate == 128;
+    if (d.dstate <= 128 && d.headdim <= 64) {
+        auto k = full ? decode_steps_kernel<T, 1, true> : decode_steps_kernel<T, 1, false>;
+        k<<<grid, kDecodeThreads, smem, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch, d.nheads, d.headdim,
+                                             d.ngroups, d.dstate, err);
+    } else if (d.dstate <= 128) {
+        auto k = full ? decode_steps_kernel<T, 2, true> : decode_steps_kernel<T, 2, false>;
+        k<<<grid, kDecodeThreads, smem, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch, d.nheads, d.headdim,
+                                             d.ngroups, d.dstate, err);
+    } else if (d.dstate <= 256) {
         decode_steps_loop_kernel<T, 2, 4><<<grid, kDecodeThreads, 0, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps,
                                                                           d.batch, d.nheads, d.headdim, d.ngroups,
                                                                           d.dstate);
-    else
+    } else {
         decode_steps_loop_kernel<T, 4, 2><<<grid, kDecodeThreads, 0, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps,
                                                                           d.batch, d.nheads, d.headdim, d.ngroups,
                                                                           d.dstate);
+    }
     return cudaGetLastError();
 }
 
@@ -436,18 +440,20 @@ cudaError_t launch_steps_layers_dtype(const Dims& d, const ssd_decode_layer_t* l
     const dim3 grid((unsigned)(d.batch * d.nheads), (unsigned)n_layers);
     const size_t smem = (size_t)kStepStages * (step_row_bytes<T>(d.headdim) + 2 * step_row_bytes<T>(d.dstate) + 16);
     int* err = device_error_word();
-    if (d.dstate <= 128 && d.headdim <= 64)
-        decode_steps_layers_kernel<T, 1><<<grid, kDecodeThreads, smem, s>>>(layers, steps, d.batch, d.nheads,
-                                                                            d.headdim, d.ngroups, d.dstate, err);
-    else if (d.dstate <= 128)
-        decode_steps_layers_kernel<T, 2><<<grid, kDecodeThreads, smem, s>>>(layers, steps, d.batch, d.nheads,
-                                                                            d.headdim, d.ngroups, d.dstate, err);
-    else if (d.dstate <= 256)
+    const bool full = d.dstate == 128;
+    if (d.dstate <= 128 && d.headdim <= 64) {
+        auto k = full ? decode_steps_layers_kernel<T, 1, true> : decode_steps_layers_kernel<T, 1, false>;
+        k<<<grid, kDecodeThreads, smem, s>>>(layers, steps, d.batch, d.nheads, d.headdim, d.ngroups, d.dstate, err);
+    } else if (d.dstate <= 128) {
+        auto k = full ? decode_steps_layers_kernel<T, 2, true> : decode_steps_layers_kernel<T, 2, false>;
+        k<<<grid, kDecodeThreads, smem, s>>>(layers, steps, d.batch, d.nheads, d.headdim, d.ngroups, d.dstate, err);
+    } else if (d.dstate <= 256) {
         decode_steps_layers_loop_kernel<T, 2, 4><<<grid, kDecodeThreads, 0, s>>>(layers, steps, d.batch, d.nheads,
                                                                                  d.headdim, d.ngroups, d.dstate, err);
-    else
+    } else {
         decode_steps_layers_loop_kernel<T, 4, 2><<<grid, kDecodeThreads, 0, s>>>(layers, steps, d.batch, d.nheads,
                                                                                  d.headdim, d.ngroups, d.dstate, err);
+    }
     return cudaGetLastError();
 }
 

@@ -44,6 +44,7 @@ def _case(b, H, P, G, N, steps, seed, dtype=torch.float32):
     (3, 4, 64, 1, 256, 9, torch.float32),       # looped kernel (state too large for registers)
     (2, 4, 8, 2, 16, 50, torch.float32),        # small odd shape, lanes without a quad
     (4, 8, 64, 1, 128, 24, torch.bfloat16),     # bf16 inputs and outputs
+    (2, 4, 128, 1, 64, 11, torch.bfloat16),     # 16 rows a warp with dstate < 128 (absent quads)
 ])
 def test_steps_equal_single_step_launches_bitwise(b, H, P, G, N, steps, dtype):
     from state_space_model_05_b200 import ssd_decode_step, ssd_decode_steps
@@ -99,6 +100,7 @@ def _stack(nl, b, H, P, G, N, steps, dtype, seed):
     (64, 128, torch.float32),      # register-resident, one row per lane group
     (128, 128, torch.bfloat16),    # register-resident, two rows per lane group, bf16
     (64, 256, torch.float32),      # looped kernel
+    (64, 32, torch.float32),       # dstate < 128: lanes with absent quads
 ])
 def test_stack_steps_equal_per_layer_calls_bitwise(P, N, dtype):
     """ssd_decode_steps_layers advances every layer of a table by k tokens in one launch:
