@@ -127,8 +127,6 @@ decode_step_kernel(float* __restrict__ state, const T* __restrict__ x, const flo
                               dt_bias, dt_softplus);
 }
 
-// Every layer of a stack in one launch: blockIdx.y is the layer, whose tensors come from
-// the table.  A layer entry with a null or misaligned pointer is skipped and recorded.
 // A layer table entry is used when none of its pointers is null and all are 16-byte
 // aligned; otherwise the CTA skips it and thread 0 records SSD_ERR_NULL / SSD_ERR_ALIGN.
 __device__ __forceinline__ bool layer_entry_ok(const ssd_decode_layer_t& L, int* err)
@@ -148,6 +146,8 @@ __device__ __forceinline__ bool layer_entry_ok(const ssd_decode_layer_t& L, int*
     return true;
 }
 
+// Every layer of a stack in one launch: blockIdx.y is the layer, whose tensors come from
+// the table.  A layer entry with a null or misaligned pointer is skipped and recorded.
 template <typename T, int QPL, int ROWS>
 __global__ void __launch_bounds__(kDecodeThreads, QPL == 1 ? 4 : 2)
 decode_layers_kernel(const ssd_decode_layer_t* __restrict__ layers, int nheads, int headdim,
