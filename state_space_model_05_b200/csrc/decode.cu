@@ -16,6 +16,7 @@
 // are read once per CTA into registers (lane j holds elements 4j..4j+3).  The y reduction along dstate is a
 // warp shuffle tree; the state is written back with 16-byte stores.
 #include "common.cuh"
+#include "prefill_tc.h"
 #include "ptx.cuh"
 
 namespace ssd {
@@ -191,33 +192,43 @@ static_assert(kStepStages == kDecodeWarps, "stage w is filled by warp w");
 template <typename T>
 __host__ __device__ constexpr int step_row_bytes(int n) { return (int)((n * sizeof(T) + 15) & ~size_t(15)); }
 
-// The steps of (b, h) unit `unit` of one layer (the CTA's whole work).  FULL: dstate is 128,
-// so every lane holds all 8 of its quads (no per-quad presence tests).
-template <typename T, int R, bool FULL>
+// The steps of U consecutive (b, h) units of one layer from `unit0` on (the CTA's whole
+// work).  U = 2 takes two heads of one batch row and one group (they share B_t and C_t): row
+// i of a lane group then belongs to unit i / R, so each warp carries two independent chains.
+// FULL: dstate is 128, so every lane holds all 8 of its quads (no per-quad presence tests).
+template <typename T, int R, int U, bool FULL>
 __device__ __forceinline__ void steps_unit(float* __restrict__ state, const T* __restrict__ x,
                                            const float* __restrict__ dt, const float* __restrict__ A,
                                            const T* __restrict__ Bm, const T* __restrict__ Cm,
                                            const float* __restrict__ D, T* __restrict__ y, int steps, int batch,
-                                           int nheads, int headdim, int ngroups, int dstate, int unit, int* err)
+                                           int nheads, int headdim, int ngroups, int dstate, int unit0, int* err)
 {
     static_assert(R == 1 || R == 2, "rows per lane group");
-    extern __shared__ __align__(16) uint8_t stage_mem[]; // per stage: x row | B_t row | C_t row | dt
+    static_assert(U == 1 || (U == 2 && R == 1), "units per CTA");
+    constexpr int NR = R * U;                          // rows per lane
+    // per stage: the units' x rows | B_t row | C_t row | the units' dt
+    extern __shared__ __align__(16) uint8_t stage_mem[];
     __shared__ __align__(8) uint64_t full[kStepStages], empty[kStepStages];
     __shared__ int abort_flag;
-    const int xbytes = step_row_bytes<T>(headdim);
+    const int xbytes = step_row_bytes<T>(U * headdim);
     const int nbytes = step_row_bytes<T>(dstate);
     const int stage_bytes = xbytes + 2 * nbytes + 16;
 
-    const int b = unit / nheads;
-    const int h = unit - b * nheads;
-    const int g = h / (nheads / ngroups);
+    const int b = unit0 / nheads;
+    const int h0 = unit0 - b * nheads;
+    const int g = h0 / (nheads / ngroups);
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int grp = lane >> 2, L = lane & 3;
     const int nq = FULL ? 32 : dstate >> 2;            // quads in a row (<= 32)
-    const int p0 = warp * 8 * R;                       // rows p0 + 8i + grp, i < R
+    const int p0 = warp * 8 * R;                       // row of lane row i: p0 + 8 (i % R) + grp
     const size_t units = (size_t)batch * nheads;
-    const float Ah = A[h], Dh = D[h];
+    float Ah[U], Dh[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        Ah[u] = A[h0 + u];
+        Dh[u] = D[h0 + u];
+    }
     volatile int* abort = &abort_flag;
 
     if (threadIdx.x == 0) {
@@ -239,10 +250,13 @@ __device__ __forceinline__ void steps_unit(float* __restrict__ state, const T* _
             return false;
         uint8_t* sp = stage_mem + (size_t)st * stage_bytes;
         const size_t bc = ((size_t)k * batch * ngroups + (size_t)b * ngroups + g) * dstate;
-        ptx::cp_async_4(sp + xbytes + 2 * nbytes, dt + (size_t)k * units + unit);
+        if (U == 1)
+            ptx::cp_async_4(sp + xbytes + 2 * nbytes, dt + (size_t)k * units + unit0);
+        else
+            ptx::cp_async_8(sp + xbytes + 2 * nbytes, dt + (size_t)k * units + unit0);
         ptx::cp_async_mbar_arrive(&full[st]);          // before the arrival below
-        ptx::mbar_expect_tx(&full[st], (uint32_t)((headdim + 2 * dstate) * sizeof(T)));
-        ptx::bulk_load(sp, x + ((size_t)k * units + unit) * headdim, headdim * sizeof(T), &full[st]);
+        ptx::mbar_expect_tx(&full[st], (uint32_t)((U * headdim + 2 * dstate) * sizeof(T)));
+        ptx::bulk_load(sp, x + ((size_t)k * units + unit0) * headdim, U * headdim * sizeof(T), &full[st]);
         ptx::bulk_load(sp + xbytes, Bm + bc, dstate * sizeof(T), &full[st]);
         ptx::bulk_load(sp + xbytes + nbytes, Cm + bc, dstate * sizeof(T), &full[st]);
         last_issued = k;
@@ -251,18 +265,21 @@ __device__ __forceinline__ void steps_unit(float* __restrict__ state, const T* _
     if (lane == 0 && warp < steps && warp < kStepAhead) issue(warp);
 
     // rows of this lane that exist (headdim is a multiple of 8: all 8 groups of a warp agree)
-    bool row_on[R];
+    bool row_on[NR];
+    float* S[NR];
 #pragma unroll
-    for (int i = 0; i < R; ++i) row_on[i] = p0 + 8 * i < headdim;
-    float4 s[R][8];
-    float* S = state + (size_t)unit * headdim * dstate;
+    for (int i = 0; i < NR; ++i) {
+        const int p = p0 + 8 * (i % R) + grp;
+        row_on[i] = p0 + 8 * (i % R) < headdim;
+        S[i] = state + ((size_t)(unit0 + i / R) * headdim + p) * dstate;
+    }
+    float4 s[NR][8];
 #pragma unroll
-    for (int i = 0; i < R; ++i)
+    for (int i = 0; i < NR; ++i)
 #pragma unroll
         for (int m = 0; m < 8; ++m)
-            s[i][m] = row_on[i] && L + 4 * m < nq
-                          ? *reinterpret_cast<const float4*>(S + (size_t)(p0 + 8 * i + grp) * dstate + 4 * (L + 4 * m))
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+            s[i][m] = row_on[i] && L + 4 * m < nq ? *reinterpret_cast<const float4*>(S[i] + 4 * (L + 4 * m))
+                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
 
     for (int k = 0; k < steps; ++k) {
         if (lane == 0 && k + kStepAhead < steps && (k + kStepAhead) % kStepStages == warp && !issue(k + kStepAhead))
@@ -273,24 +290,29 @@ __device__ __forceinline__ void steps_unit(float* __restrict__ state, const T* _
         const T* sx = reinterpret_cast<const T*>(sp);
         const T* sb = reinterpret_cast<const T*>(sp + xbytes);
         const T* sc = reinterpret_cast<const T*>(sp + xbytes + nbytes);
-        const float dtv = *reinterpret_cast<const float*>(sp + xbytes + 2 * nbytes);
-        const float a = expf(dtv * Ah);                // fp32 decay exponent
-        float xv[R], acc[R];
+        float dtv[U], a[U];
 #pragma unroll
-        for (int i = 0; i < R; ++i) xv[i] = row_on[i] ? Elem<T>::load(sx + p0 + 8 * i + grp) : 0.f;
-        float part[R][8];
+        for (int u = 0; u < U; ++u) {
+            dtv[u] = reinterpret_cast<const float*>(sp + xbytes + 2 * nbytes)[u];
+            a[u] = expf(dtv[u] * Ah[u]);               // fp32 decay exponent
+        }
+        float xv[NR], acc[NR];
+#pragma unroll
+        for (int i = 0; i < NR; ++i)
+            xv[i] = row_on[i] ? Elem<T>::load(sx + (i / R) * headdim + p0 + 8 * (i % R) + grp) : 0.f;
+        float part[NR][8];
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
             const bool qon = L + 4 * m < nq;
             const float4 bq = qon ? load4<T>(sb + 4 * (L + 4 * m)) : make_float4(0.f, 0.f, 0.f, 0.f);
             const float4 cq = qon ? load4<T>(sc + 4 * (L + 4 * m)) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int i = 0; i < R; ++i) {
-                const float dx = dtv * xv[i];
+            for (int i = 0; i < NR; ++i) {
+                const float dx = dtv[i / R] * xv[i];
                 float pa = 0.f;
                 if (qon) {
                     // a v + (dx b) per element, two elements per packed instruction
-                    const float2 dx2 = make_float2(dx, dx), a2 = make_float2(a, a);
+                    const float2 dx2 = make_float2(dx, dx), a2 = make_float2(a[i / R], a[i / R]);
                     float4 v = s[i][m];
                     const float2 vxy = ptx::ffma2(a2, make_float2(v.x, v.y), ptx::fmul2(dx2, make_float2(bq.x, bq.y)));
                     const float2 vzw = ptx::ffma2(a2, make_float2(v.z, v.w), ptx::fmul2(dx2, make_float2(bq.z, bq.w)));
@@ -307,7 +329,7 @@ __device__ __forceinline__ void steps_unit(float* __restrict__ state, const T* _
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&empty[st]);   // the stage may be refilled
 #pragma unroll
-        for (int i = 0; i < R; ++i) {
+        for (int i = 0; i < NR; ++i) {
             // quad levels 16, 8, 4 inside the lane, then 2 and 1 across the group
             float t0 = part[i][0] + part[i][4], t1 = part[i][1] + part[i][5];
             float t2 = part[i][2] + part[i][6], t3 = part[i][3] + part[i][7];
@@ -319,47 +341,53 @@ __device__ __forceinline__ void steps_unit(float* __restrict__ state, const T* _
             acc[i] = v;
         }
         if (L == 0) {
-            T* yr = y + ((size_t)k * units + unit) * headdim + p0 + grp;
 #pragma unroll
-            for (int i = 0; i < R; ++i)
-                if (row_on[i]) Elem<T>::store(yr + 8 * i, fmaf(Dh, xv[i], acc[i]));
+            for (int i = 0; i < NR; ++i)
+                if (row_on[i])
+                    Elem<T>::store(y + ((size_t)k * units + unit0 + i / R) * headdim + p0 + 8 * (i % R) + grp,
+                                   fmaf(Dh[i / R], xv[i], acc[i]));
         }
         if (*abort) break;
     }
 #pragma unroll
-    for (int i = 0; i < R; ++i)
+    for (int i = 0; i < NR; ++i)
 #pragma unroll
         for (int m = 0; m < 8; ++m)
-            if (row_on[i] && L + 4 * m < nq)
-                *reinterpret_cast<float4*>(S + (size_t)(p0 + 8 * i + grp) * dstate + 4 * (L + 4 * m)) = s[i][m];
+            if (row_on[i] && L + 4 * m < nq) *reinterpret_cast<float4*>(S[i] + 4 * (L + 4 * m)) = s[i][m];
     // the CTA does not exit with copies in flight: each warp waits for the last fill of its stage
     __syncthreads();
     if (lane == 0 && last_issued >= 0)
         ptx::mbar_wait(&full[last_issued % kStepStages], (last_issued / kStepStages) & 1, err);
 }
 
-template <typename T, int R, bool FULL>
-__global__ void __launch_bounds__(kDecodeThreads, R == 1 ? 3 : 1)
+// CTAs an SM holds: three with one row per lane, two with two rows of two units, one with
+// two rows of one unit (its register count is above 128)
+template <int R, int U>
+constexpr int steps_ctas_per_sm() { return R * U == 1 ? 3 : (R == 1 ? 2 : 1); }
+
+template <typename T, int R, int U, bool FULL>
+__global__ void __launch_bounds__(kDecodeThreads, steps_ctas_per_sm<R, U>())
 decode_steps_kernel(float* __restrict__ state, const T* __restrict__ x, const float* __restrict__ dt,
                     const float* __restrict__ A, const T* __restrict__ Bm, const T* __restrict__ Cm,
                     const float* __restrict__ D, T* __restrict__ y, int steps, int batch, int nheads,
                     int headdim, int ngroups, int dstate, int* err)
 {
-    steps_unit<T, R, FULL>(state, x, dt, A, Bm, Cm, D, y, steps, batch, nheads, headdim, ngroups, dstate, blockIdx.x, err);
+    steps_unit<T, R, U, FULL>(state, x, dt, A, Bm, Cm, D, y, steps, batch, nheads, headdim, ngroups, dstate,
+                              blockIdx.x * U, err);
 }
 
 // The same for every layer of a table (blockIdx.y = layer): each entry's per-step pointers
 // address [steps][...] arrays, so one launch advances the whole stack by `steps` tokens.
-template <typename T, int R, bool FULL>
-__global__ void __launch_bounds__(kDecodeThreads, R == 1 ? 3 : 1)
+template <typename T, int R, int U, bool FULL>
+__global__ void __launch_bounds__(kDecodeThreads, steps_ctas_per_sm<R, U>())
 decode_steps_layers_kernel(const ssd_decode_layer_t* __restrict__ layers, int steps, int batch, int nheads,
                            int headdim, int ngroups, int dstate, int* err)
 {
     const ssd_decode_layer_t L = layers[blockIdx.y];
     if (!layer_entry_ok(L, err)) return;
-    steps_unit<T, R, FULL>(L.state, static_cast<const T*>(L.x_t), L.dt_t, L.A, static_cast<const T*>(L.B_t),
-                     static_cast<const T*>(L.C_t), L.D, static_cast<T*>(L.y_t), steps, batch, nheads, headdim,
-                     ngroups, dstate, blockIdx.x, err);
+    steps_unit<T, R, U, FULL>(L.state, static_cast<const T*>(L.x_t), L.dt_t, L.A, static_cast<const T*>(L.B_t),
+                              static_cast<const T*>(L.C_t), L.D, static_cast<T*>(L.y_t), steps, batch, nheads,
+                              headdim, ngroups, dstate, blockIdx.x * U, err);
 }
 
 // Shapes whose state does not fit in registers: the single step's body once per step, still
@@ -400,6 +428,24 @@ decode_steps_layers_loop_kernel(const ssd_decode_layer_t* __restrict__ layers, i
                                   static_cast<T*>(L.y_t), steps, batch, nheads, headdim, ngroups, dstate);
 }
 
+// Two units per CTA where a pair of heads shares B_t and C_t, every quad is present, and the
+// units (of all layers) are more than one wave of one-unit CTAs: below that, one unit a CTA
+// keeps more SMs busy (a batch-1 layer has 80 units for 148 SMs).
+bool steps_pair(const Dims& d, int n_layers)
+{
+    const long long units = (long long)d.batch * d.nheads * n_layers;
+    return d.dstate == 128 && d.headdim <= 64 && (d.nheads / d.ngroups) % 2 == 0 &&
+           units > (long long)steps_ctas_per_sm<1, 1>() * tc_sm_count();
+}
+
+// Dynamic shared memory of the multi-step kernels: the ring of input stages.
+template <typename T>
+size_t steps_smem(const Dims& d, int units_per_cta)
+{
+    return (size_t)kStepStages *
+           (step_row_bytes<T>(units_per_cta * d.headdim) + 2 * step_row_bytes<T>(d.dstate) + 16);
+}
+
 template <typename T>
 cudaError_t launch_steps_dtype(const Dims& d, int steps, float* state, const void* x, const float* dt,
                                const float* A, const void* B, const void* C, const float* D, void* y,
@@ -410,17 +456,19 @@ cudaError_t launch_steps_dtype(const Dims& d, int steps, float* state, const voi
     const T* Bt = static_cast<const T*>(B);
     const T* Ct = static_cast<const T*>(C);
     T* yt = static_cast<T*>(y);
-    const size_t smem = (size_t)kStepStages * (step_row_bytes<T>(d.headdim) + 2 * step_row_bytes<T>(d.dstate) + 16);
     int* err = device_error_word();
     const bool full = d.dstate == 128;
-    if (d.dstate <= 128 && d.headdim <= 64) {
-        auto k = full ? decode_steps_kernel<T, 1, true> : decode_steps_kernel<T, 1, false>;
-        k<<<grid, kDecodeThreads, smem, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch, d.nheads, d.headdim,
-                                             d.ngroups, d.dstate, err);
+    if (steps_pair(d, 1)) {
+        decode_steps_kernel<T, 1, 2, true><<<grid / 2, kDecodeThreads, steps_smem<T>(d, 2), s>>>(
+            state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch, d.nheads, d.headdim, d.ngroups, d.dstate, err);
+    } else if (d.dstate <= 128 && d.headdim <= 64) {
+        auto k = full ? decode_steps_kernel<T, 1, 1, true> : decode_steps_kernel<T, 1, 1, false>;
+        k<<<grid, kDecodeThreads, steps_smem<T>(d, 1), s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch,
+                                                            d.nheads, d.headdim, d.ngroups, d.dstate, err);
     } else if (d.dstate <= 128) {
-        auto k = full ? decode_steps_kernel<T, 2, true> : decode_steps_kernel<T, 2, false>;
-        k<<<grid, kDecodeThreads, smem, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch, d.nheads, d.headdim,
-                                             d.ngroups, d.dstate, err);
+        auto k = full ? decode_steps_kernel<T, 2, 1, true> : decode_steps_kernel<T, 2, 1, false>;
+        k<<<grid, kDecodeThreads, steps_smem<T>(d, 1), s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps, d.batch,
+                                                            d.nheads, d.headdim, d.ngroups, d.dstate, err);
     } else if (d.dstate <= 256) {
         decode_steps_loop_kernel<T, 2, 4><<<grid, kDecodeThreads, 0, s>>>(state, xt, dt, A, Bt, Ct, D, yt, steps,
                                                                           d.batch, d.nheads, d.headdim, d.ngroups,
@@ -438,15 +486,19 @@ cudaError_t launch_steps_layers_dtype(const Dims& d, const ssd_decode_layer_t* l
                                       cudaStream_t s)
 {
     const dim3 grid((unsigned)(d.batch * d.nheads), (unsigned)n_layers);
-    const size_t smem = (size_t)kStepStages * (step_row_bytes<T>(d.headdim) + 2 * step_row_bytes<T>(d.dstate) + 16);
     int* err = device_error_word();
     const bool full = d.dstate == 128;
-    if (d.dstate <= 128 && d.headdim <= 64) {
-        auto k = full ? decode_steps_layers_kernel<T, 1, true> : decode_steps_layers_kernel<T, 1, false>;
-        k<<<grid, kDecodeThreads, smem, s>>>(layers, steps, d.batch, d.nheads, d.headdim, d.ngroups, d.dstate, err);
+    if (steps_pair(d, n_layers)) {
+        decode_steps_layers_kernel<T, 1, 2, true><<<dim3(grid.x / 2, grid.y), kDecodeThreads, steps_smem<T>(d, 2), s>>>(
+            layers, steps, d.batch, d.nheads, d.headdim, d.ngroups, d.dstate, err);
+    } else if (d.dstate <= 128 && d.headdim <= 64) {
+        auto k = full ? decode_steps_layers_kernel<T, 1, 1, true> : decode_steps_layers_kernel<T, 1, 1, false>;
+        k<<<grid, kDecodeThreads, steps_smem<T>(d, 1), s>>>(layers, steps, d.batch, d.nheads, d.headdim, d.ngroups,
+                                                            d.dstate, err);
     } else if (d.dstate <= 128) {
-        auto k = full ? decode_steps_layers_kernel<T, 2, true> : decode_steps_layers_kernel<T, 2, false>;
-        k<<<grid, kDecodeThreads, smem, s>>>(layers, steps, d.batch, d.nheads, d.headdim, d.ngroups, d.dstate, err);
+        auto k = full ? decode_steps_layers_kernel<T, 2, 1, true> : decode_steps_layers_kernel<T, 2, 1, false>;
+        k<<<grid, kDecodeThreads, steps_smem<T>(d, 1), s>>>(layers, steps, d.batch, d.nheads, d.headdim, d.ngroups,
+                                                            d.dstate, err);
     } else if (d.dstate <= 256) {
         decode_steps_layers_loop_kernel<T, 2, 4><<<grid, kDecodeThreads, 0, s>>>(layers, steps, d.batch, d.nheads,
                                                                                  d.headdim, d.ngroups, d.dstate, err);

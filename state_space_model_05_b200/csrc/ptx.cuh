@@ -193,6 +193,11 @@ __device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
+// 8-byte asynchronous copy global -> shared (both addresses 8-byte aligned).
+__device__ __forceinline__ void cp_async_8(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
 // Makes the phase of `bar` wait for this thread's earlier cp.async copies: the pending
 // count is raised by one now and lowered when those copies have landed.  Issue it before
 // the arrival that could otherwise complete the phase.

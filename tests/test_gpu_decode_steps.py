@@ -5,7 +5,8 @@ token ("Compiler-First State Space Duality and Portable O(1) Autoregressive Cach
 Inference", section "2. Metodologia").  For tokens whose inputs are on the device, one
 launch runs the whole loop; it must give exactly what k launches of ssd_decode_step give
 (same arithmetic per row, so bitwise), and match the fp64 oracle stepped k times.
-Covered: the register-resident kernel (headdim <= 64 and <= 128, dstate <= 128), the
+Covered: the register-resident kernel (headdim <= 64 and <= 128, dstate <= 128; one head a
+CTA, or two heads of a group when the units exceed a wave), the
 looped kernel (dstate 256), bf16 inputs, odd small shapes, grouped B/C and steps = 0; and
 ssd_decode_steps_layers, the same loop over every layer of a table in one launch (bitwise
 equal to the per-layer call, oracle-checked, a bad entry skipped and reported).
@@ -40,6 +41,9 @@ def _case(b, H, P, G, N, steps, seed, dtype=torch.float32):
 
 @pytest.mark.parametrize("b,H,P,G,N,steps,dtype", [
     (4, 8, 64, 1, 128, 37, torch.float32),      # register-resident, 2.7B head shape
+    (2, 6, 64, 2, 128, 15, torch.float32),      # three heads a group: one head a CTA
+    (8, 64, 64, 1, 128, 9, torch.float32),      # 512 units, more than a wave: two heads a CTA
+    (8, 64, 64, 4, 128, 7, torch.bfloat16),     # the same in bf16, four groups
     (2, 6, 128, 2, 128, 20, torch.float32),     # register-resident, 16 rows a warp
     (3, 4, 64, 1, 256, 9, torch.float32),       # looped kernel (state too large for registers)
     (2, 4, 8, 2, 16, 50, torch.float32),        # small odd shape, lanes without a quad
@@ -96,18 +100,19 @@ def _stack(nl, b, H, P, G, N, steps, dtype, seed):
     return layers, refs
 
 
-@pytest.mark.parametrize("P,N,dtype", [
-    (64, 128, torch.float32),      # register-resident, one row per lane group
-    (128, 128, torch.bfloat16),    # register-resident, two rows per lane group, bf16
-    (64, 256, torch.float32),      # looped kernel
-    (64, 32, torch.float32),       # dstate < 128: lanes with absent quads
+@pytest.mark.parametrize("P,N,dtype,H", [
+    (64, 128, torch.float32, 4),       # register-resident, one row per lane group
+    (64, 128, torch.float32, 96),      # 576 units over the layers: two heads a CTA
+    (128, 128, torch.bfloat16, 4),     # register-resident, two rows per lane group, bf16
+    (64, 256, torch.float32, 4),       # looped kernel
+    (64, 32, torch.float32, 4),        # dstate < 128: lanes with absent quads
 ])
-def test_stack_steps_equal_per_layer_calls_bitwise(P, N, dtype):
+def test_stack_steps_equal_per_layer_calls_bitwise(P, N, dtype, H):
     """ssd_decode_steps_layers advances every layer of a table by k tokens in one launch:
     bit for bit what ssd_decode_steps gives per layer (itself bitwise equal to k single
     steps, above), and for fp32 within tolerance of the oracle stepped k times."""
     from state_space_model_05_b200 import decode_layer_table, ssd_decode_steps_layers, ssd_device_status
-    b, H, G, steps, nl = 2, 4, 2, 13, 3
+    b, G, steps, nl = 2, 2, 13, 3
     layers, refs = _stack(nl, b, H, P, G, N, steps, dtype, seed=300 + P + N)
     ssd_decode_steps_layers(decode_layer_table(layers), steps, b, H, P, G, N, dtype)
     assert ssd_device_status() == 0
